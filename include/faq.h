@@ -1,0 +1,206 @@
+/*
+ * faq.h -- C ABI of the B200 (sm_100a) FA-quantization library (libfaq.so).
+ *
+ * FA quantization quantizes the Q/K/V activations that feed flash attention
+ * and then computes attention on the low-bit operands (msModelSlim wiki
+ * "FA 量化", section 概述 / overview; MindIE SD "量化", section FA量化).
+ * This header declares the whole boundary: calibration, quantization of
+ * Q/K/V in the pages' modes, the rotate -> block-quant step, and attention
+ * on the quantized operands (prefill, and split-KV decode for Sq = 1).
+ *
+ * Conventions shared by every entry point
+ *   - All data pointers are DEVICE pointers owned by the caller.  The
+ *     library never allocates, frees or synchronises on these paths; every
+ *     call is asynchronous on the caller's stream `s` (0 = legacy default).
+ *   - bf16 tensors use layout BNSD = [B, H, S, D] or BSND = [B, S, H, D]
+ *     (MindIE SD "量化", FA量化 / 注意事项: Q/K/V input layouts BNSD and
+ *     BSND), dense, D contiguous, 16-byte aligned base pointers.
+ *   - D must be 64 or 128.
+ *   - Arguments are validated on the host before any launch; a rejected call
+ *     launches nothing and returns a non-zero fa_status.
+ *   - Kernel-side failures (a bounded wait that ran out) are recorded in a
+ *     per-device status word and reported by fa_check_device_status().
+ *
+ * Quantized tensor (fa_qtensor) storage, per mode -- codes keep the data
+ * layout, scale arrays are canonical whatever the layout:
+ *   FA_MODE_INT8_PER_HEAD    codes int8 [..D];   scales fp32 [H]
+ *   FA_MODE_FP8_PER_TOKEN    codes e4m3 [..D];   scales fp32 [B, H, S]
+ *   FA_MODE_FP8_BLOCK        codes e4m3 [..D];   scales fp32 [B, H, ceil(S/block_tokens)]
+ *   FA_MODE_MXFP4_PER_BLOCK  codes packed e2m1 [..D/2] (element 2i in the
+ *                            low nibble, 2i+1 in the high nibble);
+ *                            scales uint8 E8M0 [B, H, S, D/32]
+ */
+#ifndef FAQ_H
+#define FAQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define FAQ_API __attribute__((visibility("default")))
+#else
+#define FAQ_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* fa_stream_t; /* a cudaStream_t */
+
+typedef enum {
+  FA_OK = 0,
+  FA_ERR_INVALID_ARG = 1,     /* bad pointer, shape, layout, alignment      */
+  FA_ERR_UNSUPPORTED = 2,     /* valid request this build does not run      */
+  FA_ERR_NO_CALIBRATION = 3,  /* static mode without calibration data       */
+  FA_ERR_CONFIG_CONFLICT = 4, /* qconfig and details both given             */
+  FA_ERR_CUDA = 5,            /* a CUDA runtime call or launch failed       */
+  FA_ERR_TIMEOUT = 6,         /* a kernel's bounded wait ran out            */
+  FA_ERR_WORKSPACE = 7        /* workspace missing or too small             */
+} fa_status;
+
+typedef enum { FA_LAYOUT_BNSD = 0, FA_LAYOUT_BSND = 1 } fa_layout;
+
+/* The pages' FA modes (msModelSlim wiki "FA 量化", 分支组合 / branch
+ * combinations 组合1-3; MindIE SD "量化", FA量化 / 块量化). */
+typedef enum {
+  FA_MODE_FLOAT = 0,           /* not quantized ("float": the branch stays bf16) */
+  FA_MODE_INT8_PER_HEAD = 1,   /* 组合1: INT8, per-head static minmax, s = amax/127 */
+  FA_MODE_FP8_PER_TOKEN = 2,   /* 组合2: E4M3, per-token dynamic, s = amax/448     */
+  FA_MODE_MXFP4_PER_BLOCK = 3, /* 组合3: E2M1 + E8M0 per 32 elements of head_dim   */
+  FA_MODE_FP8_BLOCK = 4        /* 块量化: E4M3, one scale per block of tokens      */
+} fa_mode;
+
+/* A bf16 activation tensor. */
+typedef struct {
+  const void* data; /* device, bf16 */
+  int B, H, S, D;
+  fa_layout layout;
+} fa_tensor;
+
+/* A quantized tensor: codes + scales + mode + layout.  Filled by the caller
+ * (pointers to caller-owned device buffers of the sizes listed above). */
+typedef struct {
+  void* codes;
+  void* scales;
+  fa_mode mode;
+  int B, H, S, D;
+  fa_layout layout;
+  int block_tokens; /* FA_MODE_FP8_BLOCK only: tokens per scale block */
+} fa_qtensor;
+
+/* Per-branch quantization settings (msModelSlim "fa3_quant 配置说明",
+ * §2.1 FA3QuantProcessorConfig and §2.3 FA3AttentionDetails). */
+typedef struct {
+  int set;      /* 0 = not given */
+  fa_mode mode; /* FA_MODE_FLOAT = the branch is not quantized */
+} fa_branch_cfg;
+
+/*
+ * fa_resolve_config -- turn a unified qconfig and/or per-branch details into
+ * the mode of each branch (q, k, v).
+ *   Source: "fa3_quant 配置说明" §2.1 配置约束 -- qconfig and details are
+ *   mutually exclusive; both given is an error; neither given means the
+ *   default int8 / per_head / symmetric / minmax.  §2.3 and the wiki's
+ *   分支组合 note: a branch that details leaves unset is not quantized.
+ *   qconfig: nullable; details: nullable array of 3 (q, k, v).
+ *   modes_out: host array of 3.
+ *   Returns FA_ERR_CONFIG_CONFLICT when both are set, FA_ERR_INVALID_ARG on
+ *   a NULL modes_out or an out-of-range mode.  Host only, no CUDA call.
+ */
+FAQ_API fa_status fa_resolve_config(const fa_branch_cfg* qconfig, const fa_branch_cfg* details, fa_mode modes_out[3]);
+
+/*
+ * fa_calibrate_per_head -- static per-head minmax calibration.
+ *   Source: wiki "FA 量化", 组合1 -- one scale per attention head, found
+ *   offline (minmax) and then frozen; calibration data is mandatory.
+ *   x: bf16 calibration batch.  amax_h: device fp32 [x->H], a RUNNING
+ *   maximum: on return amax_h[h] = max(amax_h[h], max |x| over head h).
+ *   The caller zero-fills it before the first batch.  Call once per batch.
+ */
+FAQ_API fa_status fa_calibrate_per_head(const fa_tensor* x, float* amax_h, fa_stream_t s);
+
+/*
+ * fa_quantize -- quantize Q, K and V with one unified mode, in one launch.
+ *   Sources: wiki "FA 量化" 组合1 (INT8 per-head static: s_h = amax_h/127,
+ *   code = int8 round-half-even(x / s_h), saturated to [-128, 127], the
+ *   range printed in MindIE SD "量化", Linear量化 / 通用原理), 组合2 (FP8
+ *   E4M3 per-token dynamic: s = amax_token/448, code = e4m3(x / s)),
+ *   组合3 (MXFP4: per 32 elements of head_dim, e = floor(log2 amax) - 2,
+ *   E8M0 byte e + 127, code = e2m1(x / 2^e)); MindIE SD FA量化 / 块量化
+ *   (E4M3 with one scale = amax/448 per block of block_tokens tokens).
+ *   Rounding is round-half-to-even, saturating; x / s is one IEEE fp32
+ *   division; a zero scale gives zero codes.
+ *   q, k, v: bf16 inputs; any of them may be NULL to skip that operand.
+ *   mode: one of the quantized modes.  amax_q/k/v: device fp32 [H] from
+ *   fa_calibrate_per_head, required for FA_MODE_INT8_PER_HEAD (NULL there
+ *   -> FA_ERR_NO_CALIBRATION), ignored otherwise.
+ *   q_out/k_out/v_out: caller-filled descriptors whose codes/scales point to
+ *   buffers of the sizes above; their dims/layout must equal the input's
+ *   and their mode must equal `mode`.  For FA_MODE_FP8_BLOCK,
+ *   block_tokens >= 1 (the pages use 128 for Q and 256 for K/V).
+ */
+FAQ_API fa_status fa_quantize(const fa_tensor* q, const fa_tensor* k, const fa_tensor* v, fa_mode mode,
+                      const float* amax_q, const float* amax_k, const float* amax_v, fa_qtensor* q_out,
+                      fa_qtensor* k_out, fa_qtensor* v_out, fa_stream_t s);
+
+/*
+ * fa_rotate_quantize -- rotate Q and K, then FP8 block-quantize Q, K, V.
+ *   Source: MindIE SD "量化", FA量化 / 技术特点: 旋转 (Q and K are
+ *   multiplied by trained rotation matrices q_rot / k_rot to spread
+ *   outliers; V is not rotated), then 块量化 (E4M3, block 128 for Q and
+ *   256 for K/V).  Q' = bf16(Q R_q) (fp32 accumulation, one rounding),
+ *   K' = bf16(K R_k), V' = V; then FA_MODE_FP8_BLOCK quantization.
+ *   rot_q, rot_k: device bf16 [D, D] row-major (x' = x * R).  q_block,
+ *   kv_block: tokens per scale block; must equal q_out->block_tokens and
+ *   k_out/v_out->block_tokens.  rot_q_dbg / rot_k_dbg: nullable device bf16
+ *   outputs (input layout) receiving Q', K' as rounded before quantization.
+ *   Outputs must have mode FA_MODE_FP8_BLOCK.
+ */
+FAQ_API fa_status fa_rotate_quantize(const fa_tensor* q, const fa_tensor* k, const fa_tensor* v, const void* rot_q,
+                             const void* rot_k, int q_block, int kv_block, fa_qtensor* q_out, fa_qtensor* k_out,
+                             fa_qtensor* v_out, void* rot_q_dbg, void* rot_k_dbg, fa_stream_t s);
+
+/*
+ * fa_attention_quant -- flash attention on quantized Q/K/V, bf16 output.
+ *   Sources: MindIE SD "量化", FA量化 / FP8 Attention (attention computed
+ *   on the low-bit operands, the output dequantized back to the original
+ *   precision); FlashAttention (Dao et al. 2022), cited by the wiki's
+ *   参考资料: O = softmax(Q K^T * scale) V with an online softmax.
+ *   q, k, v: quantized descriptors, all the same mode and layout and D;
+ *   q->B == k->B == v->B, k and v have equal dims, q->H % k->H == 0 (GQA:
+ *   query head h reads kv head h / (Hq / Hkv)).  causal: key j is visible
+ *   to query i iff j <= i + (Sk - Sq).  softmax_scale <= 0 means 1/sqrt(D).
+ *   out: device bf16, q's layout and dims.  lse: nullable device fp32
+ *   [B, Hq, Sq], natural-log sum-exp of the scaled scores (-inf for a row
+ *   with no visible key, whose output is 0).
+ *   Decode (q->S == 1) runs a split-KV kernel and an LSE combine; it needs
+ *   `workspace` of at least fa_attention_workspace_size() bytes
+ *   (FA_ERR_WORKSPACE otherwise).  num_splits: 0 = choose automatically.
+ *   Modes run here: INT8_PER_HEAD, FP8_PER_TOKEN, FP8_BLOCK and
+ *   MXFP4_PER_BLOCK for prefill; INT8_PER_HEAD for decode (others ->
+ *   FA_ERR_UNSUPPORTED).
+ */
+FAQ_API fa_status fa_attention_quant(const fa_qtensor* q, const fa_qtensor* k, const fa_qtensor* v, int causal,
+                             float softmax_scale, void* out, float* lse, int num_splits, void* workspace,
+                             size_t ws_bytes, fa_stream_t s);
+
+/* Workspace bytes fa_attention_quant needs for these operands and split
+ * count (0 for prefill).  Returns 0 on invalid arguments. */
+FAQ_API size_t fa_attention_workspace_size(const fa_qtensor* q, const fa_qtensor* k, int num_splits);
+
+/* Synchronise `s`, read and clear this device's status word.  Returns
+ * FA_ERR_TIMEOUT if a kernel's bounded wait ran out since the last check,
+ * FA_ERR_CUDA if the stream reports an error, FA_OK otherwise. */
+FAQ_API fa_status fa_check_device_status(fa_stream_t s);
+
+/* Static text for a status code. */
+FAQ_API const char* fa_status_str(fa_status st);
+
+/* Library version string. */
+FAQ_API const char* fa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* FAQ_H */

@@ -1,0 +1,71 @@
+// internal.cuh -- declarations shared by the library's translation units.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "faq.h"
+
+namespace faq {
+
+// One operand of a quantize launch: bf16 input rows -> codes + scales.
+struct QuantOperand {
+  const void* x;       // bf16 input
+  void* codes;         // output codes
+  void* scales;        // output scales (fp32 or E8M0 bytes)
+  const float* amax;   // INT8 per head: calibration maxima [H]
+  long long rows;      // B * H * S
+  int B, H, S, D;
+  int layout;
+  int blk;             // FP8 block: tokens per block
+};
+
+// Per-device status word (timeouts recorded by bounded waits).
+int* device_status_ptr();
+
+// Driver entry point for tensor-map encoding (resolved once).
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn encode_tiled_fn();
+
+// Number of SMs of the current device (cached).
+int sm_count();
+
+// Launchers (quant.cu).
+cudaError_t launch_calibrate(const QuantOperand& op, float* amax, cudaStream_t s);
+cudaError_t launch_quantize_rows(int mode, const QuantOperand* ops, int nops, cudaStream_t s);
+cudaError_t launch_quantize_fp8_block(const QuantOperand* ops, int nops, cudaStream_t s);
+
+// Launchers (rotate.cu).
+struct RotateOperand {
+  const void* x;       // bf16 input [.., D]
+  const void* R;       // bf16 [D, D] or nullptr (no rotation)
+  void* codes;         // e4m3
+  float* scales;       // [B, H, nblk]
+  void* dbg;           // nullable bf16 rotated output
+  int B, H, S, D, layout, blk;
+};
+cudaError_t launch_rotate_block_quant(const RotateOperand* ops, int nops, int* status, cudaStream_t s);
+
+// Launchers (attn.cu / decode.cu).
+struct AttnArgs {
+  const fa_qtensor* q;
+  const fa_qtensor* k;
+  const fa_qtensor* v;
+  int causal;
+  float softmax_scale;
+  void* out;
+  float* lse;
+  int* status;
+};
+cudaError_t launch_attention_prefill(const AttnArgs& a, cudaStream_t s);
+
+size_t decode_workspace_bytes(int B, int Hq, int D, int splits);
+int decode_auto_splits(int B, int Hkv, int Sk);
+cudaError_t launch_attention_decode(const AttnArgs& a, int splits, void* ws, cudaStream_t s);
+
+cudaError_t launch_fill_empty_rows(void* out, float* lse, long long rows, int D, cudaStream_t s);
+
+}  // namespace faq

@@ -1,0 +1,312 @@
+// quant.cu -- HBM-bound quantization kernels for FA quantization:
+//   calibrate_kernel          running per-head max |x|        (wiki "FA 量化", 组合1)
+//   quant_rows_kernel<MODE>   one pass over token rows:
+//       INT8 per head   code = sat8(rne(x / s_h)), s_h = amax_h / 127  (组合1)
+//       FP8 per token   s = amax_row / 448, code = e4m3(x / s)        (组合2)
+//       MXFP4           per 32 elements: e = floor(log2 amax) - 2,
+//                       code = e2m1(x * 2^-e), E8M0 byte e + 127      (组合3)
+//   fp8_block_kernel          one scale = amax / 448 per block of tokens
+//                             (MindIE SD "量化", FA量化 / 块量化)
+// Rows are D contiguous bf16 values in either layout; each row is handled by
+// D/8 lanes with one 16-byte load each.  Division is IEEE (div.rn.f32) so
+// the codes match a correctly rounded x / s exactly.
+#include <cuda_bf16.h>
+
+#include "internal.cuh"
+#include "sm100.cuh"
+
+namespace faq {
+namespace {
+
+__device__ __forceinline__ void unpack_bf16x8(const uint4& u, float (&f)[8]) {
+  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    f[2 * i] = __uint_as_float(w[i] << 16);
+    f[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+  }
+}
+
+// Four fp32 values -> four E4M3 bytes (a in the lowest byte), RNE, saturating.
+__device__ __forceinline__ uint32_t e4m3x4(float a, float b, float c, float d) {
+  uint16_t lo, hi;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(lo) : "f"(b), "f"(a));
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(hi) : "f"(d), "f"(c));
+  return (uint32_t)lo | ((uint32_t)hi << 16);
+}
+
+// Eight fp32 values -> eight E2M1 nibbles (v[0] in the lowest nibble).
+__device__ __forceinline__ uint32_t e2m1x8(const float (&v)[8]) {
+  uint32_t r;
+  asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b2, %6, %5;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n\t"
+      "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
+      : "=r"(r)
+      : "f"(v[0]), "f"(v[1]), "f"(v[2]), "f"(v[3]), "f"(v[4]), "f"(v[5]), "f"(v[6]), "f"(v[7]));
+  return r;
+}
+
+__device__ __forceinline__ uint32_t s8_of(float x) {
+  int i = __float2int_rn(x);  // round half to even; saturates to the int32 range
+  i = max(-128, min(127, i));
+  return (uint32_t)(i & 0xFF);
+}
+__device__ __forceinline__ uint32_t s8x4(float a, float b, float c, float d) {
+  return s8_of(a) | (s8_of(b) << 8) | (s8_of(c) << 16) | (s8_of(d) << 24);
+}
+
+// Canonical [B, H, S] index of token row r of the data layout.
+__device__ __forceinline__ long long scale_index(long long r, int layout, int H, int S) {
+  if (layout == FA_LAYOUT_BNSD) return r;
+  const long long h = r % H, bs = r / H;
+  return ((bs / S) * H + h) * S + (bs % S);
+}
+__device__ __forceinline__ int head_of(long long r, int layout, int H, int S) {
+  return layout == FA_LAYOUT_BNSD ? (int)((r / S) % H) : (int)(r % H);
+}
+
+// Exponent e of the MX shared scale: floor(log2 amax) - 2, clamped to
+// [-127, 127]; amax == 0 or an fp32-subnormal amax gives -127.
+__device__ __forceinline__ int mx_exponent(float amax) {
+  const int E = (int)((__float_as_uint(amax) >> 23) & 0xFF);
+  if (E == 0) return -127;
+  return max(-127, min(127, E - 127 - 2));
+}
+
+template <int MODE, int D>
+__global__ void __launch_bounds__(256) quant_rows_kernel(QuantOperand o0, QuantOperand o1, QuantOperand o2) {
+  constexpr int G = D / 8;     // lanes per row
+  constexpr int RPW = 32 / G;  // rows per warp per step
+  constexpr int UNROLL = 2;
+  const int lane = threadIdx.x & 31;
+  const int gl = lane % G;
+  const int sub = lane / G;
+
+  if (MODE == FA_MODE_INT8_PER_HEAD && blockIdx.x == 0) {
+    for (int t = threadIdx.x; t < o0.H && o0.rows > 0; t += blockDim.x)
+      static_cast<float*>(o0.scales)[t] = __fdiv_rn(o0.amax[t], 127.0f);
+    for (int t = threadIdx.x; t < o1.H && o1.rows > 0; t += blockDim.x)
+      static_cast<float*>(o1.scales)[t] = __fdiv_rn(o1.amax[t], 127.0f);
+    for (int t = threadIdx.x; t < o2.H && o2.rows > 0; t += blockDim.x)
+      static_cast<float*>(o2.scales)[t] = __fdiv_rn(o2.amax[t], 127.0f);
+  }
+
+  const long long total = o0.rows + o1.rows + o2.rows;
+  const long long nwarps = (long long)gridDim.x * (blockDim.x / 32);
+  const long long wid = ((long long)blockIdx.x * blockDim.x + threadIdx.x) / 32;
+  const long long step = nwarps * RPW;
+
+  for (long long base = wid * RPW * UNROLL; base < total; base += step * UNROLL) {
+    uint4 raw[UNROLL];
+    long long rr[UNROLL];
+    int which[UNROLL];
+#pragma unroll
+    for (int u = 0; u < UNROLL; ++u) {
+      const long long r = base + u * RPW + sub;
+      which[u] = r < o0.rows ? 0 : (r < o0.rows + o1.rows ? 1 : 2);
+      rr[u] = which[u] == 0 ? r : (which[u] == 1 ? r - o0.rows : r - o0.rows - o1.rows);
+      raw[u] = make_uint4(0, 0, 0, 0);
+      if (r < total) {
+        const void* x = which[u] == 0 ? o0.x : (which[u] == 1 ? o1.x : o2.x);
+        raw[u] = __ldg(reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(x) + rr[u] * D) + gl);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < UNROLL; ++u) {
+      const long long r = base + u * RPW + sub;
+      const bool valid = r < total;
+      const QuantOperand& op = which[u] == 0 ? o0 : (which[u] == 1 ? o1 : o2);
+      float f[8];
+      unpack_bf16x8(raw[u], f);
+      if (MODE == FA_MODE_FP8_PER_TOKEN) {
+        float m = 0.0f;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) m = fmaxf(m, fabsf(f[i]));
+#pragma unroll
+        for (int off = G / 2; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+        const float sc = __fdiv_rn(m, 448.0f);
+        float v[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) v[i] = sc > 0.0f ? __fdiv_rn(f[i], sc) : 0.0f;
+        if (valid) {
+          uint2 out = make_uint2(e4m3x4(v[0], v[1], v[2], v[3]), e4m3x4(v[4], v[5], v[6], v[7]));
+          reinterpret_cast<uint2*>(static_cast<uint8_t*>(op.codes) + rr[u] * D)[gl] = out;
+          if (gl == 0) static_cast<float*>(op.scales)[scale_index(rr[u], op.layout, op.H, op.S)] = sc;
+        }
+      } else if (MODE == FA_MODE_INT8_PER_HEAD) {
+        float sc = 0.0f;
+        if (valid) sc = __fdiv_rn(__ldg(op.amax + head_of(rr[u], op.layout, op.H, op.S)), 127.0f);
+        float v[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) v[i] = sc > 0.0f ? __fdiv_rn(f[i], sc) : 0.0f;
+        if (valid) {
+          uint2 out = make_uint2(s8x4(v[0], v[1], v[2], v[3]), s8x4(v[4], v[5], v[6], v[7]));
+          reinterpret_cast<uint2*>(static_cast<int8_t*>(op.codes) + rr[u] * D)[gl] = out;
+        }
+      } else {  // MXFP4: one 32-element block = 4 lanes
+        float m = 0.0f;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) m = fmaxf(m, fabsf(f[i]));
+        m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
+        m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 2));
+        const int e = mx_exponent(m);
+        const float inv = __uint_as_float((uint32_t)(127 - e) << 23);  // 2^-e, exact
+        float v[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) v[i] = f[i] * inv;
+        if (valid) {
+          reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(op.codes) + rr[u] * (D / 2))[gl] = e2m1x8(v);
+          if ((gl & 3) == 0)
+            static_cast<uint8_t*>(op.scales)[scale_index(rr[u], op.layout, op.H, op.S) * (D / 32) + gl / 4] =
+                (uint8_t)(e + 127);
+        }
+      }
+    }
+  }
+}
+
+// Per-head running max: grid (chunks, H); each CTA reduces a slice of one
+// head's rows and folds it into amax[h] with one atomic max on the float
+// bits (valid because every value is >= 0).
+__global__ void __launch_bounds__(256) calibrate_kernel(const __nv_bfloat16* __restrict__ x, int B, int H, int S,
+                                                        int D, int layout, float* amax) {
+  const int h = blockIdx.y;
+  const long long rows = (long long)B * S;  // rows of this head
+  const int vpr = D / 8;                    // uint4 per row
+  const long long nvec = rows * vpr;
+  float m = 0.0f;
+  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < nvec;
+       i += (long long)gridDim.x * blockDim.x) {
+    const long long rh = i / vpr;
+    const int c = (int)(i % vpr);
+    const long long b = rh / S, s = rh % S;
+    const long long row = layout == FA_LAYOUT_BNSD ? (b * H + h) * S + s : (b * S + s) * H + h;
+    const uint4 u = __ldg(reinterpret_cast<const uint4*>(x + row * D) + c);
+    float f[8];
+    unpack_bf16x8(u, f);
+#pragma unroll
+    for (int k = 0; k < 8; ++k) m = fmaxf(m, fabsf(f[k]));
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+  __shared__ float wm[8];
+  if ((threadIdx.x & 31) == 0) wm[threadIdx.x >> 5] = m;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float bm = 0.0f;
+    for (int w = 0; w < (int)(blockDim.x >> 5); ++w) bm = fmaxf(bm, wm[w]);
+    atomicMax(reinterpret_cast<int*>(amax + h), __float_as_int(bm));
+  }
+}
+
+// FP8 block quantization without rotation: one CTA per (b, h, block).
+// Pass 1 finds the block's amax, pass 2 quantizes (the re-read hits L2).
+__global__ void __launch_bounds__(256) fp8_block_kernel(QuantOperand op) {
+  const int g = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  const int s0 = g * op.blk;
+  const int s1 = min(op.S, s0 + op.blk);
+  const int vpr = op.D / 8;
+  const int nvec = (s1 - s0) * vpr;
+  const __nv_bfloat16* x = static_cast<const __nv_bfloat16*>(op.x);
+  auto row_of = [&](int s) -> long long {
+    return op.layout == FA_LAYOUT_BNSD ? ((long long)b * op.H + h) * op.S + s : ((long long)b * op.S + s) * op.H + h;
+  };
+  float m = 0.0f;
+  for (int i = threadIdx.x; i < nvec; i += blockDim.x) {
+    const uint4 u = __ldg(reinterpret_cast<const uint4*>(x + row_of(s0 + i / vpr) * op.D) + (i % vpr));
+    float f[8];
+    unpack_bf16x8(u, f);
+#pragma unroll
+    for (int k = 0; k < 8; ++k) m = fmaxf(m, fabsf(f[k]));
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+  __shared__ float wm[8];
+  __shared__ float s_sc;
+  if ((threadIdx.x & 31) == 0) wm[threadIdx.x >> 5] = m;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float bm = 0.0f;
+    for (int w = 0; w < (int)(blockDim.x >> 5); ++w) bm = fmaxf(bm, wm[w]);
+    s_sc = __fdiv_rn(bm, 448.0f);
+    const int nblk = (op.S + op.blk - 1) / op.blk;
+    static_cast<float*>(op.scales)[((long long)b * op.H + h) * nblk + g] = s_sc;
+  }
+  __syncthreads();
+  const float sc = s_sc;
+  for (int i = threadIdx.x; i < nvec; i += blockDim.x) {
+    const long long row = row_of(s0 + i / vpr);
+    const uint4 u = __ldg(reinterpret_cast<const uint4*>(x + row * op.D) + (i % vpr));
+    float f[8];
+    unpack_bf16x8(u, f);
+    float v[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) v[k] = sc > 0.0f ? __fdiv_rn(f[k], sc) : 0.0f;
+    reinterpret_cast<uint2*>(static_cast<uint8_t*>(op.codes) + row * op.D)[i % vpr] =
+        make_uint2(e4m3x4(v[0], v[1], v[2], v[3]), e4m3x4(v[4], v[5], v[6], v[7]));
+  }
+}
+
+template <int MODE>
+cudaError_t launch_rows_mode(const QuantOperand (&o)[3], int D, cudaStream_t s) {
+  const long long total = o[0].rows + o[1].rows + o[2].rows;
+  if (total == 0) {
+    if (MODE != FA_MODE_INT8_PER_HEAD) return cudaSuccess;
+  }
+  const int rows_per_block = (256 / 32) * (32 / (D / 8)) * 2;
+  long long want = (total + rows_per_block - 1) / rows_per_block;
+  const long long cap = (long long)sm_count() * 8 * 4;  // enough resident warps, grid-stride beyond
+  int grid = (int)(want < 1 ? 1 : (want > cap ? cap : want));
+  if (D == 128)
+    quant_rows_kernel<MODE, 128><<<grid, 256, 0, s>>>(o[0], o[1], o[2]);
+  else
+    quant_rows_kernel<MODE, 64><<<grid, 256, 0, s>>>(o[0], o[1], o[2]);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_calibrate(const QuantOperand& op, float* amax, cudaStream_t s) {
+  const long long nvec = (long long)op.B * op.S * (op.D / 8);
+  if (nvec == 0) return cudaSuccess;
+  long long chunks = (nvec + 256 * 8 - 1) / (256 * 8);
+  const long long cap = ((long long)sm_count() * 8 + op.H - 1) / op.H;
+  if (chunks > cap) chunks = cap;
+  if (chunks < 1) chunks = 1;
+  dim3 grid((unsigned)chunks, (unsigned)op.H);
+  calibrate_kernel<<<grid, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(op.x), op.B, op.H, op.S, op.D, op.layout,
+                                        amax);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_quantize_rows(int mode, const QuantOperand* ops, int nops, cudaStream_t s) {
+  QuantOperand o[3] = {};
+  int D = 128;
+  for (int i = 0; i < nops && i < 3; ++i) {
+    o[i] = ops[i];
+    D = ops[i].D;
+  }
+  switch (mode) {
+    case FA_MODE_FP8_PER_TOKEN: return launch_rows_mode<FA_MODE_FP8_PER_TOKEN>(o, D, s);
+    case FA_MODE_INT8_PER_HEAD: return launch_rows_mode<FA_MODE_INT8_PER_HEAD>(o, D, s);
+    case FA_MODE_MXFP4_PER_BLOCK: return launch_rows_mode<FA_MODE_MXFP4_PER_BLOCK>(o, D, s);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+cudaError_t launch_quantize_fp8_block(const QuantOperand* ops, int nops, cudaStream_t s) {
+  for (int i = 0; i < nops; ++i) {
+    const QuantOperand& op = ops[i];
+    if (op.rows == 0) continue;
+    dim3 grid((unsigned)((op.S + op.blk - 1) / op.blk), (unsigned)op.H, (unsigned)op.B);
+    fp8_block_kernel<<<grid, 256, 0, s>>>(op);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  return cudaSuccess;
+}
+
+}  // namespace faq

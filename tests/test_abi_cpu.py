@@ -1,0 +1,135 @@
+"""The C-ABI library loads, exports every symbol include/faq.h declares, and
+rejects bad arguments on the host before any CUDA call (no GPU needed)."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def N():
+    from quantized_attention_amax_b200 import build
+    build.build()
+    from quantized_attention_amax_b200 import _native
+    _native.lib()
+    return _native
+
+
+def declared_symbols():
+    hdr = open(os.path.join(ROOT, "include", "faq.h")).read()
+    return sorted(set(re.findall(r"FAQ_API\s+[\w\s\*]*?\b(fa_\w+)\s*\(", hdr)))
+
+
+def test_header_declares_the_boundary():
+    syms = declared_symbols()
+    for name in ("fa_calibrate_per_head", "fa_quantize", "fa_rotate_quantize", "fa_attention_quant"):
+        assert name in syms
+
+
+def test_library_exports_every_declared_symbol(N):
+    out = subprocess.run(["nm", "-D", "--defined-only", N.LIB_PATH], capture_output=True, text=True).stdout
+    exported = set(re.findall(r"\bT (fa_\w+)", out))
+    assert set(declared_symbols()) <= exported
+    assert set(N.EXPORTS) == set(declared_symbols())
+    L = N.lib()
+    for name in declared_symbols():
+        assert getattr(L, name) is not None
+
+
+def test_status_strings(N):
+    L = N.lib()
+    for code in range(8):
+        assert L.fa_status_str(code)
+    assert b"x" in L.fa_version() or L.fa_version()
+
+
+def test_resolve_config_rules():
+    import quantized_attention_amax_b200 as faq
+    # neither given: the default int8 / per_head
+    assert faq.resolve_config() == ("int8_per_head",) * 3
+    assert faq.resolve_config("fp8_per_token") == ("fp8_per_token",) * 3
+    # a branch details leaves unset stays float
+    assert faq.resolve_config(details=["mxfp4", None, None]) == ("mxfp4", "float", "float")
+    with pytest.raises(faq.FaqError) as e:
+        faq.resolve_config("int8_per_head", ["int8_per_head", None, None])
+    assert e.value.status == 4
+
+
+def _t(N, B=1, H=2, S=8, D=64, layout=0, ptr=0x10000):
+    return N.FaTensor(ptr, B, H, S, D, layout)
+
+
+def _q(N, mode, B=1, H=2, S=8, D=64, layout=0, blk=0, codes=0x20000, scales=0x30000):
+    return N.FaQTensor(codes, scales, mode, B, H, S, D, layout, blk)
+
+
+def test_quantize_validation_before_launch(N):
+    L = N.lib()
+    t = _t(N)
+    o = _q(N, 2)
+    by = ctypes.byref
+    assert L.fa_quantize(by(t), None, None, 0, None, None, None, by(o), None, None, None) == 1   # float mode
+    t96 = _t(N, D=96)
+    o96 = _q(N, 2, D=96)
+    assert L.fa_quantize(by(t96), None, None, 2, None, None, None, by(o96), None, None, None) == 2  # D
+    oi = _q(N, 1)
+    assert L.fa_quantize(by(t), None, None, 1, None, None, None, by(oi), None, None, None) == 3  # no calibration
+    bad = _q(N, 2, S=9)
+    assert L.fa_quantize(by(t), None, None, 2, None, None, None, by(bad), None, None, None) == 1  # shape mismatch
+    mis = _t(N, ptr=0x10008)
+    assert L.fa_quantize(by(mis), None, None, 2, None, None, None, by(o), None, None, None) == 1  # alignment
+    ob = _q(N, 4, blk=0)
+    assert L.fa_quantize(by(t), None, None, 4, None, None, None, by(ob), None, None, None) == 1  # block size
+    assert L.fa_quantize(None, None, None, 2, None, None, None, None, None, None, None) == 1     # nothing to do
+    assert L.fa_calibrate_per_head(by(t96), ctypes.c_void_p(0x40000), None) == 2
+    assert L.fa_calibrate_per_head(by(t), None, None) == 1
+
+
+def test_rotate_validation_before_launch(N):
+    L = N.lib()
+    by = ctypes.byref
+    t = _t(N)
+    oq, ok, ov = _q(N, 4, blk=128), _q(N, 4, blk=256), _q(N, 4, blk=256)
+    # missing rotation matrix
+    assert L.fa_rotate_quantize(by(t), by(t), by(t), None, None, 128, 256, by(oq), by(ok), by(ov),
+                                None, None, None) == 1
+    # block size disagreeing with the output descriptor
+    assert L.fa_rotate_quantize(by(t), by(t), by(t), 0x50000, 0x50000, 64, 256, by(oq), by(ok), by(ov),
+                                None, None, None) == 1
+    # wrong output mode
+    om = _q(N, 2)
+    assert L.fa_rotate_quantize(by(t), by(t), by(t), 0x50000, 0x50000, 128, 256, by(om), by(ok), by(ov),
+                                None, None, None) == 1
+
+
+def test_attention_validation_before_launch(N):
+    L = N.lib()
+    by = ctypes.byref
+    q = _q(N, 2, H=4)
+    k = _q(N, 2, H=2)
+    v = _q(N, 2, H=2)
+    km = _q(N, 1, H=2)
+    assert L.fa_attention_quant(by(q), by(km), by(v), 0, 0.0, 0x60000, None, 0, None, 0, None) == 2  # mixed
+    k3 = _q(N, 2, H=3)
+    assert L.fa_attention_quant(by(q), by(k3), by(k3), 0, 0.0, 0x60000, None, 0, None, 0, None) == 1  # GQA
+    kd = _q(N, 2, H=2, D=128)
+    assert L.fa_attention_quant(by(q), by(kd), by(kd), 0, 0.0, 0x60000, None, 0, None, 0, None) == 1  # D
+    assert L.fa_attention_quant(by(q), by(k), by(v), 0, 0.0, None, None, 0, None, 0, None) == 1      # out
+    qf = _q(N, 0, H=4)
+    assert L.fa_attention_quant(by(qf), by(k), by(v), 0, 0.0, 0x60000, None, 0, None, 0, None) == 2  # float
+    # decode without workspace
+    qd = _q(N, 1, B=2, H=4, S=1, D=128)
+    kd = _q(N, 1, B=2, H=2, S=1000, D=128)
+    need = L.fa_attention_workspace_size(by(qd), by(kd), 0)
+    assert need > 0
+    assert L.fa_attention_quant(by(qd), by(kd), by(kd), 0, 0.0, 0x60000, None, 0, None, 0, None) == 7
+    assert L.fa_attention_quant(by(qd), by(kd), by(kd), 0, 0.0, 0x60000, None, 0, 0x70000, need - 16,
+                                None) == 7
+    assert L.fa_attention_quant(by(qd), by(kd), by(kd), 0, 0.0, 0x60000, None, -1, None, 0, None) == 1
+    # prefill needs no workspace
+    qp = _q(N, 1, B=2, H=4, S=100, D=128)
+    assert L.fa_attention_workspace_size(by(qp), by(kd), 0) == 0
