@@ -229,7 +229,9 @@ fa_status fa_rotate_quantize(const fa_tensor* q, const fa_tensor* k, const fa_te
 }
 
 size_t fa_attention_workspace_size(const fa_qtensor* q, const fa_qtensor* k, int num_splits) {
-  if (!q || !k || q->S != 1) return 0;
+  if (!q || !k || q->S != 1 || q->mode != FA_MODE_INT8_PER_HEAD || q->D != 128 || k->H < 1 || q->H % k->H) return 0;
+  const int group = q->H / k->H;
+  if (!(group == 1 || group == 2 || group == 4 || group == 8 || group == 16)) return 0;
   const int splits = num_splits > 0 ? num_splits : decode_auto_splits(k->B, k->H, k->S);
   return decode_workspace_bytes(q->B, q->H, q->D, splits);
 }
@@ -253,7 +255,9 @@ fa_status fa_attention_quant(const fa_qtensor* q, const fa_qtensor* k, const fa_
   if (qrows == 0) return FA_OK;
   if (!out || !aligned16(out)) return FA_ERR_INVALID_ARG;
   if (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)) return FA_ERR_INVALID_ARG;
-  const bool decode = q->S == 1 && q->mode == FA_MODE_INT8_PER_HEAD;
+  const int group = q->H / k->H;
+  const bool decode = q->S == 1 && q->mode == FA_MODE_INT8_PER_HEAD && q->D == 128 &&
+                      (group == 1 || group == 2 || group == 4 || group == 8 || group == 16);
   const int splits = decode ? (num_splits > 0 ? num_splits : decode_auto_splits(k->B, k->H, k->S)) : 0;
   if (decode && k->S > 0) {
     const size_t need = decode_workspace_bytes(q->B, q->H, q->D, splits);
