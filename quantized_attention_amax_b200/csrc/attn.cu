@@ -10,10 +10,14 @@
 //   warp 0      TMA producer: Q once, then K and V code tiles into a 2-stage
 //               ring (128B- or 64B-swizzled, zero-filled past the sequence).
 //   warp 1      MMA issuer (one thread): S = Q K^T with tcgen05.mma
-//               kind::f8f6f4 (E4M3) or kind::i8 (INT8) into a double-buffered
-//               S in TMEM; then O += P' V' with kind::f16 into O in TMEM.
-//   warps 2-3   V converters: V code tile -> V' = fp16(code) (exact) in the
-//               MN-major 128B-swizzled layout the P.V MMA reads.
+//               kind::f8f6f4 (E4M3), kind::i8 (INT8) or block-scaled
+//               kind::mxf4 (E2M1 with the UE8M0 scales of every 32 elements
+//               along head_dim copied into TMEM) into a double-buffered S in
+//               TMEM; then O += P' V' with kind::f16 into O in TMEM.
+//   warps 2-3   V converters: V code tile -> V' = fp16(code) (exact; for
+//               MXFP4 fp16(e2m1 * 2^(e - e_ref)) with e_ref the largest
+//               exponent the CTA reads) in the MN-major 128B-swizzled layout
+//               the P.V MMA reads.
 //   warps 4-7   softmax, one thread per query row: load S from TMEM, apply
 //               the K scales, causal / ragged masks, online max and sum in
 //               the exp2 domain, P' = fp16(p * s_v / vref) into shared memory.
@@ -36,7 +40,7 @@ constexpr int BN = 128;  // keys per tile
 constexpr int NS = 2;    // K/V code stages
 constexpr int NTHREADS = 256;
 
-enum { KIND_E4M3 = 0, KIND_S8 = 1 };
+enum { KIND_E4M3 = 0, KIND_S8 = 1, KIND_MXF4 = 2 };
 
 struct AttnParams {
   int B, Hq, Hkv, Sq, Sk, group, causal, layout;
@@ -46,21 +50,26 @@ struct AttnParams {
   const float* vs;
   int q_blk, k_blk, v_blk;     // tokens per scale (1 = per token); 0 = one scale per head
   int q_nblk, k_nblk, v_nblk;  // scale blocks per (b, h)
+  const uint8_t* qe8;  // MXFP4: E8M0 [B, H, S, D/32]
+  const uint8_t* ke8;
+  const uint8_t* ve8;
   __nv_bfloat16* out;
   float* lse;
   int* status;
   int n_qtiles;
 };
 
-template <int D>
+template <int KIND, int D>
 struct Smem {
+  static constexpr uint32_t RB = KIND == KIND_MXF4 ? D / 2 : D;  // code bytes per token row
   static constexpr uint32_t Q = 0;
-  static constexpr uint32_t K = Q + BM * D;
-  static constexpr uint32_t V = K + NS * BN * D;
-  static constexpr uint32_t VH = V + NS * BN * D;  // 2 x fp16 V' tiles
-  static constexpr uint32_t P = VH + 2 * BN * D * 2;  // 2 x fp16 P' tiles
+  static constexpr uint32_t K = Q + BM * RB;
+  static constexpr uint32_t V = K + NS * BN * RB;
+  static constexpr uint32_t VH = V + NS * BN * RB;     // 2 x fp16 V' tiles
+  static constexpr uint32_t P = VH + 2 * BN * D * 2;   // 2 x fp16 P' tiles
   static constexpr uint32_t SC = P + 2 * BM * BN * 2;  // [2][BN] K scales, [2][BN] V factors
-  static constexpr uint32_t BAR = SC + 4 * BN * 4;
+  static constexpr uint32_t SF = SC + 4 * BN * 4;      // MXFP4: Q scale atom + NS K scale atoms (512 B each)
+  static constexpr uint32_t BAR = SF + (1 + NS) * 512;
   static constexpr uint32_t TOTAL = BAR + 512;
   static constexpr uint32_t ALLOC = TOTAL + 1024;  // slack for 1024-byte alignment
 };
@@ -80,7 +89,8 @@ enum {
   B_FINAL = 19,
   B_SC = 20,     // [2] softmax threads published this tile's per-column scales
   B_RED = 22,    // softmax threads published their V-scale maxima
-  B_COUNT = 23
+  B_ERED = 23,   // converter threads published their E8M0 maxima (MXFP4)
+  B_COUNT = 24
 };
 
 __device__ __forceinline__ float ex2(float x) {
@@ -106,6 +116,34 @@ __device__ __forceinline__ uint32_t e4m3x2_to_h2(uint16_t v) {
   asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(r) : "h"(v));
   return r;
 }
+// Two E2M1 codes (one byte, low nibble first) -> two fp16 (exact).
+__device__ __forceinline__ uint32_t e2m1x2_to_h2(uint32_t byte) {
+  uint32_t r;
+  asm("{ .reg .b8 b; cvt.u8.u32 b, %1; cvt.rn.f16x2.e2m1x2 %0, b; }" : "=r"(r) : "r"(byte));
+  return r;
+}
+
+// Copy a 128-row x 4-byte scale-factor atom (byte (m % 32) * 16 + (m / 32) * 4
+// + k) from shared memory into TMEM lanes m % 32 of every lane quarter,
+// column m / 32, byte k -- the layout block-scaled tcgen05.mma reads.
+__device__ __forceinline__ void sf_to_tmem(uint32_t taddr, uint32_t saddr) {
+  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr),
+               "l"(make_sdesc(saddr, 16, 128, kSwzNone))
+               : "memory");
+}
+
+// 32 lanes write the scale atom of 128 token rows from E8M0 [rows][4];
+// rows at or past `valid` get byte 0 (their codes are zero-filled).
+__device__ __forceinline__ void write_sf_atom(uint8_t* atom, const uint8_t* e8, long long row0, int valid, int lane) {
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const int m = lane * 4 + q;
+    uint32_t v = 0;
+    if (m < valid) v = __ldg(reinterpret_cast<const uint32_t*>(e8 + (row0 + m) * 4));
+    *reinterpret_cast<uint32_t*>(atom + (m & 31) * 16 + (m >> 5) * 4) = v;
+  }
+}
+
 // Two int8 codes -> two fp16 (exact): fp16(1024 + u) - 1152 with u = c + 128.
 __device__ __forceinline__ uint32_t s8x2_to_h2(uint32_t w_biased, int sel) {
   const uint32_t h = __byte_perm(w_biased, 0x6464u, sel);
@@ -117,7 +155,9 @@ template <int KIND, int D>
 __global__ void __launch_bounds__(NTHREADS, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
                     const __grid_constant__ CUtensorMap tmv, const AttnParams p) {
-  using L = Smem<D>;
+  using L = Smem<KIND, D>;
+  constexpr uint32_t RB = L::RB;
+  constexpr bool MX = KIND == KIND_MXF4;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bar = reinterpret_cast<uint64_t*>(smem + L::BAR);
@@ -160,6 +200,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     mbar_init(&bar[B_SC], 128);
     mbar_init(&bar[B_SC + 1], 128);
     mbar_init(&bar[B_RED], 128);
+    mbar_init(&bar[B_ERED], 64);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -172,61 +213,91 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   const uint32_t tbase = *tmem_slot;
   const uint32_t tS[2] = {tbase, tbase + 128};
   const uint32_t tO = tbase + 256;
+  const uint32_t tSFA = tbase + 384;                       // MXFP4: Q scale factors
+  const uint32_t tSFB[2] = {tbase + 392, tbase + 400};     // MXFP4: K scale factors
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
+    if (MX && n_tiles > 0) {
+      // Scale-factor atoms (all 32 lanes): Q once, then every K tile in the
+      // stage of its codes.  Published with the TMA's barrier arrival below.
+      write_sf_atom(smem + L::SF, p.qe8, (long long)(b * p.Hq + hq) * p.Sq + q0, p.Sq - q0, lane);
+      fence_async_smem();
+      __syncwarp();
+    }
     if (lane == 0 && n_tiles > 0) {
       tma_prefetch_desc(&tmq);
       tma_prefetch_desc(&tmk);
       tma_prefetch_desc(&tmv);
       const bool bnsd = p.layout == FA_LAYOUT_BNSD;
-      mbar_arrive_expect_tx(&bar[B_Q], BM * D);
+      mbar_arrive_expect_tx(&bar[B_Q], BM * RB);
       tma_load_4d(smem + L::Q, &tmq, &bar[B_Q], 0, bnsd ? q0 : hq, bnsd ? hq : q0, b);
-      int j = 0;
-      for (; j < n_tiles; ++j) {
-        const int s = j % NS;
-        const int k0 = j * BN;
-        if (j >= NS && !mbar_wait(&bar[B_KEMPTY + s], ((j / NS) - 1) & 1, abort_flag, p.status, 1)) break;
-        mbar_arrive_expect_tx(&bar[B_KFULL + s], BN * D);
-        tma_load_4d(smem + L::K + s * BN * D, &tmk, &bar[B_KFULL + s], 0, bnsd ? k0 : hk, bnsd ? hk : k0, b);
-        if (j >= NS && !mbar_wait(&bar[B_VEMPTY + s], ((j / NS) - 1) & 1, abort_flag, p.status, 2)) break;
-        mbar_arrive_expect_tx(&bar[B_VFULL + s], BN * D);
-        tma_load_4d(smem + L::V + s * BN * D, &tmv, &bar[B_VFULL + s], 0, bnsd ? k0 : hk, bnsd ? hk : k0, b);
+    }
+    int j = 0;
+    const bool bnsd = p.layout == FA_LAYOUT_BNSD;
+    for (; j < n_tiles; ++j) {
+      const int s = j % NS;
+      const int k0 = j * BN;
+      bool ok = true;
+      if (j >= NS) ok = mbar_wait(&bar[B_KEMPTY + s], ((j / NS) - 1) & 1, abort_flag, p.status, 1);
+      if (!__all_sync(0xffffffffu, ok)) break;
+      if (MX) {
+        write_sf_atom(smem + L::SF + (1 + s) * 512, p.ke8, (long long)bhk * p.Sk + k0, p.Sk - k0, lane);
+        fence_async_smem();
+        __syncwarp();
       }
-      if (*abort_flag) {
-        // Let loads already issued land before the CTA can exit.
-        for (int t = max(0, j - NS); t < j; ++t) {
-          mbar_wait(&bar[B_KFULL + t % NS], (t / NS) & 1, abort_flag, nullptr, 0);
-          mbar_wait(&bar[B_VFULL + t % NS], (t / NS) & 1, abort_flag, nullptr, 0);
+      if (lane == 0) {
+        mbar_arrive_expect_tx(&bar[B_KFULL + s], BN * RB);
+        tma_load_4d(smem + L::K + s * BN * RB, &tmk, &bar[B_KFULL + s], 0, bnsd ? k0 : hk, bnsd ? hk : k0, b);
+        if (j >= NS) ok = mbar_wait(&bar[B_VEMPTY + s], ((j / NS) - 1) & 1, abort_flag, p.status, 2);
+        if (ok) {
+          mbar_arrive_expect_tx(&bar[B_VFULL + s], BN * RB);
+          tma_load_4d(smem + L::V + s * BN * RB, &tmv, &bar[B_VFULL + s], 0, bnsd ? k0 : hk, bnsd ? hk : k0, b);
         }
+      }
+      if (!__all_sync(0xffffffffu, ok)) { ++j; break; }
+    }
+    if (lane == 0 && *abort_flag) {
+      // Let loads already issued land before the CTA can exit.
+      for (int t = max(0, j - NS); t < j; ++t) {
+        mbar_wait(&bar[B_KFULL + t % NS], (t / NS) & 1, abort_flag, nullptr, 0);
+        mbar_wait(&bar[B_VFULL + t % NS], (t / NS) & 1, abort_flag, nullptr, 0);
       }
     }
     __syncwarp();
   } else if (warp == 1) {
     // ---------------------------------------------------------- MMA issuer
     if (lane == 0 && n_tiles > 0) {
-      constexpr uint32_t SW = D == 128 ? kSwz128 : kSwz64;
-      constexpr uint32_t SBO8 = D == 128 ? 1024 : 512;
+      constexpr uint32_t SW = RB == 128 ? kSwz128 : kSwz64;
+      constexpr uint32_t SBO8 = RB == 128 ? 1024 : 512;
       constexpr uint32_t idesc_qk = KIND == KIND_E4M3 ? make_idesc(kAccF32, kFmtE4M3, kFmtE4M3, 0, 0, BN, BM)
                                                       : make_idesc(kAccS32, kFmtS8, kFmtS8, 0, 0, BN, BM);
       constexpr uint32_t idesc_pv = make_idesc(kAccF32, kFmtF16, kFmtF16, 0, 1, D, BM);
       const uint32_t sQ = smem_u32(smem + L::Q);
       bool ok = mbar_wait(&bar[B_Q], 0, abort_flag, p.status, 3);
+      if (MX && ok) {
+        tc_fence_after();
+        sf_to_tmem(tSFA, smem_u32(smem + L::SF));
+      }
       for (int j = 0; ok && j <= n_tiles; ++j) {
         if (j < n_tiles) {
           const int s = j % NS, bb = j & 1;
           if (!mbar_wait(&bar[B_KFULL + s], (j / NS) & 1, abort_flag, p.status, 4)) break;
           if (j >= 2 && !mbar_wait(&bar[B_SEMPTY + bb], ((j >> 1) - 1) & 1, abort_flag, p.status, 5)) break;
           tc_fence_after();
-          const uint32_t sK = smem_u32(smem + L::K + s * BN * D);
+          const uint32_t sK = smem_u32(smem + L::K + s * BN * RB);
+          if (MX) sf_to_tmem(tSFB[bb], smem_u32(smem + L::SF + (1 + s) * 512));
 #pragma unroll
-          for (int kk = 0; kk < D / 32; ++kk) {
+          for (int kk = 0; kk < (int)RB / 32; ++kk) {
             const uint64_t da = make_sdesc(sQ + kk * 32, 16, SBO8, SW);
             const uint64_t db = make_sdesc(sK + kk * 32, 16, SBO8, SW);
             if (KIND == KIND_E4M3)
               mma_f8f6f4(tS[bb], da, db, idesc_qk, kk > 0);
-            else
+            else if (KIND == KIND_S8)
               mma_i8(tS[bb], da, db, idesc_qk, kk > 0);
+            else  // 64 E2M1 per MMA: scale bytes 2kk, 2kk+1 of each row
+              mma_mxf4(tS[bb], da, db, make_idesc_bs(kFmtE2M1x, kFmtE2M1x, BN, BM, 2 * kk, 2 * kk), tSFA, tSFB[bb],
+                       kk > 0);
           }
           mma_commit(&bar[B_KEMPTY + s]);
           mma_commit(&bar[B_SFULL + bb]);
@@ -255,18 +326,67 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   } else if (warp < 4) {
     // --------------------------------------------------------- V converter
     const int ct = tid - 64;  // 0..63
+    int eref = 0;  // MXFP4: largest E8M0 byte of the V rows this CTA reads
+    if (MX) {
+      int m = 0;
+      for (int t = ct; t < kv_end; t += 64) {
+        const uint32_t w = __ldg(reinterpret_cast<const uint32_t*>(p.ve8 + ((long long)bhk * p.Sk + t) * 4));
+        m = max(m, (int)max(max(w & 0xFF, (w >> 8) & 0xFF), max((w >> 16) & 0xFF, w >> 24)));
+      }
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, off));
+      int* ered = reinterpret_cast<int*>(red) + 4;
+      if (lane == 0) ered[warp - 2] = m;
+      mbar_arrive(&bar[B_ERED]);
+      warp_wait(&bar[B_ERED], 0, abort_flag, p.status, 16);
+      eref = max(ered[0], ered[1]);
+    }
     for (int j = 0; j < n_tiles; ++j) {
       const int s = j % NS, bb = j & 1;
       if (!warp_wait(&bar[B_VFULL + s], (j / NS) & 1, abort_flag, p.status, 8)) break;
       if (j >= 2 && !warp_wait(&bar[B_PVDONE + bb], ((j >> 1) - 1) & 1, abort_flag, p.status, 9)) break;
-      const uint8_t* src = smem + L::V + s * BN * D;
+      const uint8_t* src = smem + L::V + s * BN * RB;
       uint8_t* dst = smem + L::VH + bb * BN * D * 2;
 #pragma unroll
       for (int rr = 0; rr < 2; ++rr) {
         const int r = ct + rr * 64;
+        if (MX) {
+          // 16 raw bytes = 32 E2M1 = one 32-element scale block of head_dim.
+          const int key = j * BN + r;
+          uint32_t e4 = 0;
+          if (key < p.Sk) e4 = __ldg(reinterpret_cast<const uint32_t*>(p.ve8 + ((long long)bhk * p.Sk + key) * 4));
+#pragma unroll
+          for (int c = 0; c < D / 32; ++c) {
+            const uint4 raw = *reinterpret_cast<const uint4*>(src + swz64_offset(r, c));  // D = 128: 64-byte rows
+            const int de = (int)((e4 >> (8 * c)) & 0xFF) - eref;  // <= 0
+            const __half fs = de >= -24 ? __float2half_rn(ldexpf(1.0f, de)) : __float2half_rn(0.0f);
+            const __half2 f2 = __halves2half2(fs, fs);
+            const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+            uint32_t h[16];
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+#pragma unroll
+              for (int y = 0; y < 2; ++y) {
+                uint32_t v2 = e2m1x2_to_h2((w[q] >> (16 * y)) & 0xFF);
+                uint32_t v3 = e2m1x2_to_h2((w[q] >> (16 * y + 8)) & 0xFF);
+                __half2 a = __hmul2(*reinterpret_cast<__half2*>(&v2), f2);
+                __half2 c2 = __hmul2(*reinterpret_cast<__half2*>(&v3), f2);
+                h[q * 4 + y * 2] = *reinterpret_cast<uint32_t*>(&a);
+                h[q * 4 + y * 2 + 1] = *reinterpret_cast<uint32_t*>(&c2);
+              }
+            const int d0 = c * 32;
+            const int nb = d0 >> 6, cc = (d0 & 63) >> 3;
+            uint8_t* base = dst + nb * (BN * 128);
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+              *reinterpret_cast<uint4*>(base + swz128_offset(r, cc + q)) =
+                  make_uint4(h[4 * q], h[4 * q + 1], h[4 * q + 2], h[4 * q + 3]);
+          }
+          continue;
+        }
 #pragma unroll
         for (int c = 0; c < D / 16; ++c) {
-          const uint32_t soff = D == 128 ? swz128_offset(r, c) : swz64_offset(r, c);
+          const uint32_t soff = RB == 128 ? swz128_offset(r, c) : swz64_offset(r, c);
           const uint4 raw = *reinterpret_cast<const uint4*>(src + soff);
           const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
           uint32_t h[8];
@@ -305,14 +425,30 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     const int kbh = bhk, qbh = b * p.Hq + hq;
 
     // Row constant: s_q * softmax_scale * log2(e) (per-head K scale folded in too).
-    const float sq = row_ok ? scale_at(p.qs, p.q_blk, p.q_nblk, qbh, hq, row) : 0.0f;
+    // MXFP4: the block scales are applied inside the MMA, so only the softmax scale.
+    const float sq = MX ? 1.0f : (row_ok ? scale_at(p.qs, p.q_blk, p.q_nblk, qbh, hq, row) : 0.0f);
     float crow = sq * p.scale_log2;
-    const bool k_head = p.k_blk == 0;
+    const bool k_head = MX || p.k_blk == 0;
     const bool k_tile_const = k_head || (p.k_blk % BN == 0);
-    if (k_head) crow *= __ldg(p.ks + hk);
-    // V reference: the largest V scale this CTA reads (per-head: the head's scale).
+    if (k_head && !MX) crow *= __ldg(p.ks + hk);
+    // V reference: the largest V scale this CTA reads (per-head: the head's
+    // scale; MXFP4: 2^(e_ref - 127), the factor the converters divided out).
     float vref;
-    if (p.v_blk == 0) {
+    if (MX) {
+      int m = 0;
+      for (int t = i; t < kv_end; t += BM) {
+        const uint32_t w = __ldg(reinterpret_cast<const uint32_t*>(p.ve8 + ((long long)bhk * p.Sk + t) * 4));
+        m = max(m, (int)max(max(w & 0xFF, (w >> 8) & 0xFF), max((w >> 16) & 0xFF, w >> 24)));
+      }
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, off));
+      if (lane == 0) red[wg] = __int_as_float(m);
+      mbar_arrive(&bar[B_RED]);
+      warp_wait(&bar[B_RED], 0, abort_flag, p.status, 14);
+      const int e = max(max(__float_as_int(red[0]), __float_as_int(red[1])),
+                        max(__float_as_int(red[2]), __float_as_int(red[3])));
+      vref = ldexpf(1.0f, e - 127);
+    } else if (p.v_blk == 0) {
       vref = __ldg(p.vs + hk);
     } else {
       float m = 0.0f;
@@ -336,12 +472,12 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       float ksc_tile = 1.0f, vf_tile = 1.0f;
       float my_k = 0.0f, my_v = 0.0f;
       const int tok = k0 + i;
-      if (!k_head) {
+      if (!k_head && !MX) {
         if (k_tile_const) ksc_tile = __ldg(p.ks + (long long)kbh * p.k_nblk + k0 / p.k_blk);
         else my_k = tok < p.Sk ? __ldg(p.ks + (long long)kbh * p.k_nblk + tok / p.k_blk) : 0.0f;
       }
-      const bool v_tile_const = p.v_blk == 0 || (p.v_blk % BN == 0);
-      if (p.v_blk != 0) {
+      const bool v_tile_const = MX || p.v_blk == 0 || (p.v_blk % BN == 0);
+      if (!MX && p.v_blk != 0) {
         if (v_tile_const) vf_tile = __ldg(p.vs + (long long)kbh * p.v_nblk + k0 / p.v_blk) * vinv;
         else my_v = tok < p.Sk ? __ldg(p.vs + (long long)kbh * p.v_nblk + tok / p.v_blk) * vinv : 0.0f;
       }
@@ -362,7 +498,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         tmem_ld_wait();
 #pragma unroll
         for (int k = 0; k < 32; ++k)
-          sv[c * 32 + k] = KIND == KIND_E4M3 ? __uint_as_float(r[k]) : (float)(int)r[k];
+          sv[c * 32 + k] = KIND == KIND_S8 ? (float)(int)r[k] : __uint_as_float(r[k]);  // s32 only for INT8
       }
       tc_fence_before();
       __syncwarp();
@@ -547,21 +683,23 @@ void scale_desc(const fa_qtensor* t, int& blk, int& nblk) {
 
 template <int KIND, int D>
 cudaError_t launch_kind(const AttnArgs& a, const AttnParams& prm, cudaStream_t s) {
+  using L = Smem<KIND, D>;
   CUtensorMap mq, mk, mv;
   cudaError_t e;
-  if ((e = make_code_map(&mq, a.q->codes, a.q->B, a.q->H, a.q->S, D, a.q->layout, BM)) != cudaSuccess) return e;
-  if ((e = make_code_map(&mk, a.k->codes, a.k->B, a.k->H, a.k->S, D, a.k->layout, BN)) != cudaSuccess) return e;
-  if ((e = make_code_map(&mv, a.v->codes, a.v->B, a.v->H, a.v->S, D, a.v->layout, BN)) != cudaSuccess) return e;
+  const int RB = (int)L::RB;
+  if ((e = make_code_map(&mq, a.q->codes, a.q->B, a.q->H, a.q->S, RB, a.q->layout, BM)) != cudaSuccess) return e;
+  if ((e = make_code_map(&mk, a.k->codes, a.k->B, a.k->H, a.k->S, RB, a.k->layout, BN)) != cudaSuccess) return e;
+  if ((e = make_code_map(&mv, a.v->codes, a.v->B, a.v->H, a.v->S, RB, a.v->layout, BN)) != cudaSuccess) return e;
   auto kern = attn_fwd_kernel<KIND, D>;
   static bool attr_set = false;  // one attribute call per instantiation (idempotent, benign race)
   if (!attr_set) {
-    if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Smem<D>::ALLOC)) != cudaSuccess)
+    if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::ALLOC)) != cudaSuccess)
       return e;
     attr_set = true;
   }
   const long long grid = (long long)prm.n_qtiles * prm.B * prm.Hq;
   if (grid > 0x7FFFFFFFLL) return cudaErrorInvalidValue;
-  kern<<<(unsigned)grid, NTHREADS, Smem<D>::ALLOC, s>>>(mq, mk, mv, prm);
+  kern<<<(unsigned)grid, NTHREADS, L::ALLOC, s>>>(mq, mk, mv, prm);
   return cudaGetLastError();
 }
 
@@ -591,6 +729,12 @@ cudaError_t launch_attention_prefill(const AttnArgs& a, cudaStream_t s) {
       return q->D == 128 ? launch_kind<KIND_E4M3, 128>(a, prm, s) : launch_kind<KIND_E4M3, 64>(a, prm, s);
     case FA_MODE_INT8_PER_HEAD:
       return q->D == 128 ? launch_kind<KIND_S8, 128>(a, prm, s) : launch_kind<KIND_S8, 64>(a, prm, s);
+    case FA_MODE_MXFP4_PER_BLOCK:
+      if (q->D != 128) return cudaErrorNotSupported;
+      prm.qe8 = static_cast<const uint8_t*>(q->scales);
+      prm.ke8 = static_cast<const uint8_t*>(k->scales);
+      prm.ve8 = static_cast<const uint8_t*>(a.v->scales);
+      return launch_kind<KIND_MXF4, 128>(a, prm, s);
     default:
       return cudaErrorNotSupported;
   }

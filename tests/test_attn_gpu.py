@@ -26,7 +26,9 @@ def to_bnsd(a, layout):
 
 
 def run_case(faq, orc, mode, layout, D, B, Hq, Hkv, Sq, Sk, causal, seed, q_blk=128, kv_blk=256, rows=None,
-             dist="normal", lse=True):
+             dist=None, lse=True):
+    if dist is None:
+        dist = "t4" if mode == "mxfp4" else "normal"
     gen = wl.student_t4 if dist == "t4" else wl.normal
     q = gen(shp(B, Hq, Sq, D, layout), seed)
     k = gen(shp(B, Hkv, Sk, D, layout), seed + 1)
@@ -72,6 +74,9 @@ CASES = [
     ("fp8_block", "BNSD", 64, 1, 2, 2, 200, 200, True),
     ("int8_per_head", "BNSD", 64, 1, 2, 2, 256, 256, False),
     ("int8_per_head", "BSND", 128, 2, 4, 2, 300, 300, True),
+    ("mxfp4", "BNSD", 128, 1, 2, 2, 300, 300, False),
+    ("mxfp4", "BSND", 128, 2, 4, 2, 257, 257, True),
+    ("mxfp4", "BNSD", 128, 1, 2, 1, 100, 300, True),
 ]
 
 
@@ -125,7 +130,7 @@ def test_constant_v(faq, orc):
     assert torch.allclose(o, torch.full_like(o, vq), rtol=0, atol=4e-3 * vq)
 
 
-@pytest.mark.parametrize("name", ["fp8_prefill", "int8_tiny"])
+@pytest.mark.parametrize("name", ["fp8_prefill", "int8_tiny", "mxfp4"])
 def test_full_size_workload(faq, orc, name):
     """Full-size workload in the benchmark's launch configuration, checked on
     sampled query rows (rows are independent, so a sample is exact)."""
