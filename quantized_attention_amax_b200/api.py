@@ -151,12 +151,15 @@ def quantize(q: Optional[torch.Tensor], k: Optional[torch.Tensor], v: Optional[t
 
 
 def rotate_quantize(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, rot_q: torch.Tensor, rot_k: torch.Tensor,
-                    layout: str = "BNSD", q_block: int = 128, kv_block: int = 256, debug: bool = False):
+                    layout: str = "BNSD", q_block: int = 128, kv_block: int = 256, debug: bool = False,
+                    out: Optional[Sequence[QTensor]] = None):
     """Rotate Q and K, then FP8 block-quantize Q, K, V (fa_rotate_quantize).
-    Returns (Qq, Kq, Vq) or, with debug=True, (Qq, Kq, Vq, Q_rot, K_rot)."""
+    Returns (Qq, Kq, Vq) or, with debug=True, (Qq, Kq, Vq, Q_rot, K_rot).
+    ``out`` reuses existing output QTensors (e.g. inside a CUDA graph)."""
     ts = [_tensor(x, layout) for x in (q, k, v)]
     blks = (q_block, kv_block, kv_block)
-    outs = [empty_qtensor(t.B, t.H, t.S, t.D, "fp8_block", layout, blks[i], q.device) for i, t in enumerate(ts)]
+    outs = list(out) if out is not None else [
+        empty_qtensor(t.B, t.H, t.S, t.D, "fp8_block", layout, blks[i], q.device) for i, t in enumerate(ts)]
     for R in (rot_q, rot_k):
         if R.dtype != torch.bfloat16 or not R.is_cuda or not R.is_contiguous() or R.shape != (ts[0].D, ts[0].D):
             raise ValueError("rotation must be a contiguous bf16 CUDA tensor [D, D]")
