@@ -185,6 +185,39 @@ FAQ_API fa_status fa_attention_quant(const fa_qtensor* q, const fa_qtensor* k, c
                              float softmax_scale, void* out, float* lse, int num_splits, void* workspace,
                              size_t ws_bytes, fa_stream_t s);
 
+/* Size of the fixed device buffer that fa_attention_decode_noalloc keeps its
+ * split-KV partials in (16 MiB per GPU that loads the library). */
+#define FA_DECODE_NOALLOC_SCRATCH_BYTES (16u << 20)
+
+/*
+ * fa_attention_decode_noalloc -- the INT8 split-KV decode of
+ * fa_attention_quant (q->S == 1) for callers that cannot allocate device
+ * memory where they run decode: a serving loop that must never synchronise
+ * the device (cudaMalloc / cudaFree can), or plain C/C++ host code linking
+ * libfaq.so without a device allocator of its own.  The pages have no
+ * counterpart to this call; it only changes where the per-split partial
+ * results live.
+ *   Instead of a caller workspace, the partials live in a buffer of
+ *   FA_DECODE_NOALLOC_SCRATCH_BYTES inside the library's own device memory
+ *   (one per GPU, held until the process exits).  Nothing is allocated and
+ *   no allocating routine is called.
+ *   The first call on a device looks the buffer's device address up (with
+ *   that device current) and caches it; make that first call before any
+ *   stream capture.
+ *   All calls on a device share the buffer: calls whose kernels overlap on
+ *   the GPU (for example on two streams) race; keep them on one stream or
+ *   serialise them.  Each call overwrites every partial it reads, so nothing
+ *   needs clearing between calls.
+ *   Arguments as for fa_attention_quant, restricted to FA_MODE_INT8_PER_HEAD,
+ *   q->S == 1, D == 128 and Hq / Hkv in {1, 2, 4, 8, 16} (FA_ERR_UNSUPPORTED
+ *   otherwise).  num_splits: 0 = automatic, reduced until the partials fit;
+ *   a split count whose partials, B * Hq * splits * (D + 2) * 4 bytes,
+ *   exceed the buffer returns FA_ERR_WORKSPACE before any launch.
+ */
+FAQ_API fa_status fa_attention_decode_noalloc(const fa_qtensor* q, const fa_qtensor* k, const fa_qtensor* v,
+                                              float softmax_scale, void* out, float* lse, int num_splits,
+                                              fa_stream_t s);
+
 /* Workspace bytes fa_attention_quant needs for these operands and split
  * count (0 for prefill).  Returns 0 on invalid arguments. */
 FAQ_API size_t fa_attention_workspace_size(const fa_qtensor* q, const fa_qtensor* k, int num_splits);

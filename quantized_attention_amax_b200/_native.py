@@ -18,6 +18,7 @@ EXPORTS = (
     "fa_rotate_quantize",
     "fa_attention_quant",
     "fa_attention_workspace_size",
+    "fa_attention_decode_noalloc",
     "fa_check_device_status",
     "fa_status_str",
     "fa_version",
@@ -62,6 +63,8 @@ def lib() -> ctypes.CDLL:
     L.fa_quantize.argtypes = [pT, pT, pT, I, P, P, P, pQ, pQ, pQ, P]
     L.fa_rotate_quantize.argtypes = [pT, pT, pT, P, P, I, I, pQ, pQ, pQ, P, P, P]
     L.fa_attention_quant.argtypes = [pQ, pQ, pQ, I, F, P, P, I, P, S, P]
+    L.fa_attention_decode_noalloc.argtypes = [pQ, pQ, pQ, F, P, P, I, P]
+    L.fa_attention_decode_noalloc.restype = I
     L.fa_attention_workspace_size.argtypes = [pQ, pQ, I]
     L.fa_attention_workspace_size.restype = S
     L.fa_check_device_status.argtypes = [P]
