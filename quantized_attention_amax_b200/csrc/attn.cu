@@ -29,11 +29,13 @@
 #include <cuda_fp16.h>
 #include <math.h>
 
+#include "attn_common.cuh"
 #include "internal.cuh"
 #include "sm100.cuh"
 
 namespace faq {
 namespace {
+using namespace attn;
 
 constexpr int BM = 128;  // query rows per tile
 constexpr int BN = 128;  // keys per tile
@@ -92,64 +94,6 @@ enum {
   B_ERED = 23,   // converter threads published their E8M0 maxima (MXFP4)
   B_COUNT = 24
 };
-
-__device__ __forceinline__ float ex2(float x) {
-  float y;
-  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-  return y;
-}
-
-// Every lane waits; the warp proceeds only if all lanes saw the phase complete.
-__device__ __forceinline__ bool warp_wait(uint64_t* b, uint32_t parity, volatile int* abort_flag, int* status,
-                                          int where) {
-  const bool ok = mbar_wait(b, parity, abort_flag, status, where);
-  return __all_sync(0xffffffffu, ok);
-}
-
-__device__ __forceinline__ float scale_at(const float* s, int blk, int nblk, int bh, int h, int tok) {
-  return blk == 0 ? __ldg(s + h) : __ldg(s + (long long)bh * nblk + tok / blk);
-}
-
-// Two E4M3 codes -> two fp16 (exact).  Low byte -> low half.
-__device__ __forceinline__ uint32_t e4m3x2_to_h2(uint16_t v) {
-  uint32_t r;
-  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(r) : "h"(v));
-  return r;
-}
-// Two E2M1 codes (one byte, low nibble first) -> two fp16 (exact).
-__device__ __forceinline__ uint32_t e2m1x2_to_h2(uint32_t byte) {
-  uint32_t r;
-  asm("{ .reg .b8 b; cvt.u8.u32 b, %1; cvt.rn.f16x2.e2m1x2 %0, b; }" : "=r"(r) : "r"(byte));
-  return r;
-}
-
-// Copy a 128-row x 4-byte scale-factor atom (byte (m % 32) * 16 + (m / 32) * 4
-// + k) from shared memory into TMEM lanes m % 32 of every lane quarter,
-// column m / 32, byte k -- the layout block-scaled tcgen05.mma reads.
-__device__ __forceinline__ void sf_to_tmem(uint32_t taddr, uint32_t saddr) {
-  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr),
-               "l"(make_sdesc(saddr, 16, 128, kSwzNone))
-               : "memory");
-}
-
-// 32 lanes write the scale atom of 128 token rows from E8M0 [rows][4];
-// rows at or past `valid` get byte 0 (their codes are zero-filled).
-__device__ __forceinline__ void write_sf_atom(uint8_t* atom, const uint8_t* e8, long long row0, int valid, int lane) {
-#pragma unroll
-  for (int q = 0; q < 4; ++q) {
-    const int m = lane * 4 + q;
-    uint32_t v = 0;
-    if (m < valid) v = __ldg(reinterpret_cast<const uint32_t*>(e8 + (row0 + m) * 4));
-    *reinterpret_cast<uint32_t*>(atom + (m & 31) * 16 + (m >> 5) * 4) = v;
-  }
-}
-
-// Two int8 codes -> two fp16 (exact): fp16(1024 + u) - 1152 with u = c + 128.
-__device__ __forceinline__ uint32_t s8x2_to_h2(uint32_t w_biased, int sel) {
-  const uint32_t h = __byte_perm(w_biased, 0x6464u, sel);
-  const __half2 v = __hsub2(*reinterpret_cast<const __half2*>(&h), __halves2half2(__ushort_as_half(0x6480), __ushort_as_half(0x6480)));
-  return *reinterpret_cast<const uint32_t*>(&v);
-}
 
 template <int KIND, int D>
 __global__ void __launch_bounds__(NTHREADS, 1)
@@ -645,31 +589,6 @@ __global__ void fill_empty_kernel(__nv_bfloat16* out, float* lse, long long rows
     for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < rows;
          i += (long long)gridDim.x * blockDim.x)
       lse[i] = -INFINITY;
-}
-
-// 4D tensor map over 8-bit codes: (D bytes, rows of the layout...).
-cudaError_t make_code_map(CUtensorMap* map, const void* base, int B, int H, int S, int D_bytes, int layout,
-                          int box_rows) {
-  EncodeTiledFn enc = encode_tiled_fn();
-  if (!enc) return cudaErrorNotSupported;
-  cuuint64_t dims[4], strides[3];
-  cuuint32_t box[4], es[4] = {1, 1, 1, 1};
-  if (layout == FA_LAYOUT_BNSD) {
-    dims[0] = D_bytes; dims[1] = S; dims[2] = H; dims[3] = B;
-    strides[0] = (cuuint64_t)D_bytes; strides[1] = (cuuint64_t)S * D_bytes; strides[2] = (cuuint64_t)H * S * D_bytes;
-    box[0] = D_bytes; box[1] = box_rows; box[2] = 1; box[3] = 1;
-  } else {
-    dims[0] = D_bytes; dims[1] = H; dims[2] = S; dims[3] = B;
-    strides[0] = (cuuint64_t)D_bytes; strides[1] = (cuuint64_t)H * D_bytes; strides[2] = (cuuint64_t)S * H * D_bytes;
-    box[0] = D_bytes; box[1] = 1; box[2] = box_rows; box[3] = 1;
-  }
-  const CUtensorMapSwizzle swz = D_bytes == 128 ? CU_TENSOR_MAP_SWIZZLE_128B
-                                 : D_bytes == 64 ? CU_TENSOR_MAP_SWIZZLE_64B
-                                                 : CU_TENSOR_MAP_SWIZZLE_32B;
-  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 4, const_cast<void*>(base), dims, strides, box, es,
-                   CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
 void scale_desc(const fa_qtensor* t, int& blk, int& nblk) {

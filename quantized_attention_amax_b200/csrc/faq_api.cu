@@ -268,7 +268,13 @@ fa_status fa_attention_quant(const fa_qtensor* q, const fa_qtensor* k, const fa_
   int* status = device_status_ptr();
   if (!status) return FA_ERR_CUDA;
   AttnArgs a = {q, k, v, causal ? 1 : 0, softmax_scale, out, lse, status};
-  cudaError_t e = decode ? launch_attention_decode(a, splits, workspace, cs) : launch_attention_prefill(a, cs);
+  cudaError_t e;
+  if (decode)
+    e = launch_attention_decode(a, splits, workspace, cs);
+  else if (q->mode == FA_MODE_MXFP4_PER_BLOCK)
+    e = launch_attention_prefill(a, cs);
+  else
+    e = launch_attention_prefill2(a, cs);
   if (e == cudaErrorNotSupported) return FA_ERR_UNSUPPORTED;
   return from_cuda(e);
 }

@@ -61,6 +61,7 @@ struct AttnArgs {
   int* status;
 };
 cudaError_t launch_attention_prefill(const AttnArgs& a, cudaStream_t s);
+cudaError_t launch_attention_prefill2(const AttnArgs& a, cudaStream_t s);
 
 size_t decode_workspace_bytes(int B, int Hq, int D, int splits);
 int decode_auto_splits(int B, int Hkv, int Sk);

@@ -117,7 +117,11 @@ def test_gqa_equals_repeated_kv(faq, orc):
     Q2, K2, V2 = faq.quantize(q, k.repeat_interleave(2, 1).contiguous(), v.repeat_interleave(2, 1).contiguous(),
                               "fp8_per_token")
     o2 = faq.attention(Q2, K2, V2, causal=True)
-    assert torch.equal(o1, o2)
+    # Same arithmetic up to the fp16 rounding of P' (the two launches pair
+    # query tiles differently, so the V-scale reference of a CTA can differ).
+    M = float(np_of(V.scales).max() * 448.0)
+    d = (o1.float() - o2.float()).abs()
+    assert d.max().item() <= 5e-3 * M and d.mean().item() <= 2e-4 * M
 
 
 def test_constant_v(faq, orc):
