@@ -5,22 +5,27 @@
 // A CTA owns two 128-row query "slots" that read the same kv head (two query
 // heads of one GQA group at the same rows, or two consecutive row tiles of one
 // head) and streams their visible 128-key K/V tiles once for both:
-//   warpgroup 0 (registers lowered with setmaxnreg):
-//     warp 0   producer: Q tiles once; per K/V tile the K codes (2-stage ring),
-//              the V codes (1 stage) by TMA, and the tile's K scales and V
-//              factors s_v / v_ref into a 2-stage shared ring.
-//     warp 1   MMA issuer (one thread), ping-pong over the two slots:
+//   warpgroup 0 (88 registers per thread after setmaxnreg):
+//     warp 0   producer: Q tiles once; per K/V tile the K codes (3-stage ring)
+//              and V codes (2-stage ring) by TMA, and the tile's K scales and
+//              V factors s_v / v_ref into a 2-stage shared ring.
+//     warp 1   MMA issuer (one thread), over the two slots:
 //              S_s = Q_s K^T (kind::f8f6f4 / kind::i8) into slot s's TMEM S,
-//              and O_s += P'_s V' (kind::f16).  PV_s(j) and QK_s(j+1) are issued
-//              as soon as slot s's softmax of tile j is done, so the two
-//              softmax warpgroups overlap.
+//              and O_s += P'_s V' (kind::f16 with the A operand P'_s in TMEM,
+//              where the softmax stored it over S_s).  PV_s(j) and then
+//              QK_s(j+1) are issued once slot s's softmax of tile j is done;
+//              the tensor pipe runs them in order, so P'_s is read before S_s
+//              is overwritten, and the other slot's softmax runs meanwhile.
 //     warps 2-3  V codes -> V' = fp16(code) (exact), MN-major, 128B-swizzled,
 //              double-buffered.
-//   warpgroups 1 and 2 (registers raised): softmax of slot 0 and slot 1, one
+//   warpgroups 1 and 2 (208 registers per thread): softmax of slot 0 and slot 1, one
 //     thread per query row: S from TMEM, K scale, mask, online max in the
 //     exp2 domain (O rescaled in TMEM only when the max grows by more than
-//     2^8), p = exp2(t * c - m), P' = fp16(p * s_v / v_ref) into shared memory.
-// TMEM: S_0, S_1, O_0, O_1 (4 x 128 columns).  Every wait is bounded.
+//     2^8), p = exp2(t * c - m), P' = fp16(p * s_v / v_ref) stored into the
+//     first 64 TMEM columns of S_s (tcgen05.st).
+// TMEM: S_0/P'_0, S_1/P'_1, O_0, O_1 (4 x 128 columns).  Keeping P' in TMEM
+// keeps it off the shared-memory port, which the shared-memory operands of
+// Q K^T and the V' operand of P.V already load heavily.  Every wait is bounded.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <math.h>
@@ -36,6 +41,8 @@ using namespace attn;
 constexpr int BM = 128;
 constexpr int BN = 128;
 constexpr int NT = 384;  // 12 warps
+constexpr int NKS = 3;   // K code stages
+constexpr int NVS = 2;   // V code stages
 
 enum { K_E4M3 = 0, K_S8 = 1 };
 enum { SC_HEAD = 0, SC_COL = 1, SC_TILE = 2 };  // one scale per head / per key / per 128-key tile
@@ -57,11 +64,10 @@ struct P2 {
 template <int D>
 struct L2 {
   static constexpr uint32_t Q = 0;                   // 2 x [128][D]
-  static constexpr uint32_t K = Q + 2 * BM * D;      // 2 stages
-  static constexpr uint32_t V = K + 2 * BN * D;      // 1 stage
-  static constexpr uint32_t VH = V + BN * D;         // 2 x fp16 V'
-  static constexpr uint32_t P = VH + 2 * BN * D * 2; // 2 slots x fp16 P'
-  static constexpr uint32_t SC = P + 2 * BM * BN * 2;  // 2 stages x ([128] k scale, [128] v factor)
+  static constexpr uint32_t K = Q + 2 * BM * D;        // NKS stages
+  static constexpr uint32_t V = K + NKS * BN * D;      // NVS stages
+  static constexpr uint32_t VH = V + NVS * BN * D;     // 2 x fp16 V'
+  static constexpr uint32_t SC = VH + 2 * BN * D * 2;  // 2 stages x ([128] k scale, [128] v factor)
   static constexpr uint32_t MISC = SC + 2 * 2 * BN * 4;
   static constexpr uint32_t BAR = MISC + 64;
   static constexpr uint32_t TOTAL = BAR + 512;
@@ -70,23 +76,23 @@ struct L2 {
 
 enum {
   X_Q = 0,
-  X_KF = 1,    // [2]
-  X_KE = 3,    // [2]
-  X_VF = 5,
-  X_VE = 6,
-  X_VHF = 7,   // [2]
-  X_VHE = 9,   // [2]
-  X_SF = 11,   // [2 slots]
-  X_PF = 13,   // [2 slots]
-  X_PVD = 15,  // [2 slots]
-  X_SCF = 17,  // [2]
-  X_SCE = 19,  // [2 slots][2 stages]
-  X_FIN = 23,
-  X_COUNT = 24
+  X_KF = 1,    // [NKS]
+  X_KE = 4,    // [NKS]
+  X_VF = 7,    // [NVS]
+  X_VE = 9,    // [NVS]
+  X_VHF = 11,  // [2]
+  X_VHE = 13,  // [2]
+  X_SF = 15,   // [2 slots]
+  X_PF = 17,   // [2 slots]
+  X_PVD = 19,  // [2 slots]
+  X_SCF = 21,  // [2]
+  X_SCE = 23,  // [2 slots][2 stages]
+  X_FIN = 27,
+  X_COUNT = 28
 };
 
-__device__ __forceinline__ void setmaxnreg_inc224() { asm volatile("setmaxnreg.inc.sync.aligned.u32 224;"); }
-__device__ __forceinline__ void setmaxnreg_dec56() { asm volatile("setmaxnreg.dec.sync.aligned.u32 56;"); }
+__device__ __forceinline__ void setmaxnreg_inc208() { asm volatile("setmaxnreg.inc.sync.aligned.u32 208;"); }
+__device__ __forceinline__ void setmaxnreg_dec88() { asm volatile("setmaxnreg.dec.sync.aligned.u32 88;"); }
 
 template <int KIND, int D, int SC>
 __global__ void __launch_bounds__(NT, 1)
@@ -143,9 +149,13 @@ __global__ void __launch_bounds__(NT, 1)
 
   if (tid == 0) {
     mbar_init(&bar[X_Q], 1);
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < NKS; ++i) {
       mbar_init(&bar[X_KF + i], 1);
       mbar_init(&bar[X_KE + i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&bar[X_VF + i], 1);
+      mbar_init(&bar[X_VE + i], 2);
       mbar_init(&bar[X_VHF + i], 2);
       mbar_init(&bar[X_VHE + i], 1);
       mbar_init(&bar[X_SF + i], 1);
@@ -155,8 +165,6 @@ __global__ void __launch_bounds__(NT, 1)
       mbar_init(&bar[X_SCE + i], 4);
       mbar_init(&bar[X_SCE + 2 + i], 4);
     }
-    mbar_init(&bar[X_VF], 1);
-    mbar_init(&bar[X_VE], 2);
     mbar_init(&bar[X_FIN], 1);
     *abort_flag = 0;
     fence_barrier_init();
@@ -170,7 +178,7 @@ __global__ void __launch_bounds__(NT, 1)
   const uint32_t tbase = *tmem_slot;
 
   if (warp < 4) {
-    setmaxnreg_dec56();
+    setmaxnreg_dec88();
     if (warp == 0) {
       // ------------------------------------------------------------ producer
       if (n_tiles > 0) {
@@ -223,22 +231,24 @@ __global__ void __launch_bounds__(NT, 1)
             if (lane == 0) mbar_arrive(&bar[X_SCF + st]);
           }
           if (lane == 0) {
-            if (j >= 2) ok = mbar_wait(&bar[X_KE + st], ((j >> 1) - 1) & 1, abort_flag, p.status, 61);
+            const int ks = j % NKS, vs = j % NVS;
+            if (j >= NKS) ok = mbar_wait(&bar[X_KE + ks], ((j / NKS) - 1) & 1, abort_flag, p.status, 61);
             if (ok) {
-              mbar_arrive_expect_tx(&bar[X_KF + st], BN * D);
-              tma_load_4d(smem + L::K + st * BN * D, &tmk, &bar[X_KF + st], 0, bnsd ? k0 : hk, bnsd ? hk : k0, b);
-              if (j >= 1) ok = mbar_wait(&bar[X_VE], (j - 1) & 1, abort_flag, p.status, 62);
+              mbar_arrive_expect_tx(&bar[X_KF + ks], BN * D);
+              tma_load_4d(smem + L::K + ks * BN * D, &tmk, &bar[X_KF + ks], 0, bnsd ? k0 : hk, bnsd ? hk : k0, b);
+              if (j >= NVS) ok = mbar_wait(&bar[X_VE + vs], ((j / NVS) - 1) & 1, abort_flag, p.status, 62);
               if (ok) {
-                mbar_arrive_expect_tx(&bar[X_VF], BN * D);
-                tma_load_4d(smem + L::V, &tmv, &bar[X_VF], 0, bnsd ? k0 : hk, bnsd ? hk : k0, b);
+                mbar_arrive_expect_tx(&bar[X_VF + vs], BN * D);
+                tma_load_4d(smem + L::V + vs * BN * D, &tmv, &bar[X_VF + vs], 0, bnsd ? k0 : hk, bnsd ? hk : k0, b);
               }
             }
           }
           if (!__all_sync(0xffffffffu, ok)) { ++j; break; }
         }
         if (lane == 0 && *abort_flag) {
-          for (int t = max(0, j - 2); t < j; ++t) mbar_wait(&bar[X_KF + (t & 1)], (t >> 1) & 1, abort_flag, nullptr, 0);
-          if (j > 0) mbar_wait(&bar[X_VF], (j - 1) & 1, abort_flag, nullptr, 0);
+          // let issued loads land before the CTA can exit
+          for (int t = max(0, j - NKS); t < j; ++t) mbar_wait(&bar[X_KF + t % NKS], (t / NKS) & 1, abort_flag, nullptr, 0);
+          for (int t = max(0, j - NVS); t < j; ++t) mbar_wait(&bar[X_VF + t % NVS], (t / NVS) & 1, abort_flag, nullptr, 0);
         }
       }
       __syncwarp();
@@ -252,7 +262,7 @@ __global__ void __launch_bounds__(NT, 1)
         constexpr uint32_t idesc_pv = make_idesc(kAccF32, kFmtF16, kFmtF16, 0, 1, D, BM);
         auto qk = [&](int s, int j) {
           const uint32_t sQ = smem_u32(smem + L::Q + s * BM * D);
-          const uint32_t sK = smem_u32(smem + L::K + (j & 1) * BN * D);
+          const uint32_t sK = smem_u32(smem + L::K + (j % NKS) * BN * D);
 #pragma unroll
           for (int kk = 0; kk < D / 32; ++kk) {
             const uint64_t da = make_sdesc(sQ + kk * 32, 16, SBO8, SW);
@@ -265,13 +275,12 @@ __global__ void __launch_bounds__(NT, 1)
           mma_commit(&bar[X_SF + s]);
         };
         auto pv = [&](int s, int j) {
-          const uint32_t sP = smem_u32(smem + L::P + s * BM * BN * 2);
+          // A = P'_s in TMEM: 16 fp16 of K per MMA = 8 columns
           const uint32_t sVh = smem_u32(smem + L::VH + (j & 1) * BN * D * 2);
 #pragma unroll
           for (int ks = 0; ks < BN / 16; ++ks) {
-            const uint64_t da = make_sdesc(sP + (ks >> 2) * (BM * 128) + (ks & 3) * 32, 16, 1024, kSwz128);
             const uint64_t db = make_sdesc(sVh + ks * 16 * 128, BN * 128, 1024, kSwz128);
-            mma_f16(tbase + 256 + s * 128, da, db, idesc_pv, (j > 0 || ks > 0) ? 1u : 0u);
+            mma_f16_ts(tbase + 256 + s * 128, tbase + s * 128 + ks * 8, db, idesc_pv, (j > 0 || ks > 0) ? 1u : 0u);
           }
           mma_commit(&bar[X_PVD + s]);
         };
@@ -284,21 +293,21 @@ __global__ void __launch_bounds__(NT, 1)
           mma_commit(&bar[X_KE]);
         }
         for (int j = 0; ok && j < n_tiles; ++j) {
+          // slot s: PV_s(j) (reads P'_s over S_s), then QK_s(j+1) (rewrites S_s)
           bool vh = false, k1 = false;
           for (int s = 0; s < 2 && ok; ++s) {
-            if (j < ns[s]) {
-              ok = mbar_wait(&bar[X_PF + s], j & 1, abort_flag, p.status, 65);
-              if (ok && !vh) {
-                ok = mbar_wait(&bar[X_VHF + (j & 1)], (j >> 1) & 1, abort_flag, p.status, 66);
-                vh = true;
-              }
-              if (!ok) break;
-              tc_fence_after();
-              pv(s, j);
+            if (j >= ns[s]) continue;
+            ok = mbar_wait(&bar[X_PF + s], j & 1, abort_flag, p.status, 65);
+            if (ok && !vh) {
+              ok = mbar_wait(&bar[X_VHF + (j & 1)], (j >> 1) & 1, abort_flag, p.status, 66);
+              vh = true;
             }
+            if (!ok) break;
+            tc_fence_after();
+            pv(s, j);
             if (j + 1 < ns[s]) {
               if (!k1) {
-                ok = mbar_wait(&bar[X_KF + ((j + 1) & 1)], ((j + 1) >> 1) & 1, abort_flag, p.status, 67);
+                ok = mbar_wait(&bar[X_KF + (j + 1) % NKS], ((j + 1) / NKS) & 1, abort_flag, p.status, 67);
                 k1 = true;
                 if (!ok) break;
                 tc_fence_after();
@@ -308,7 +317,7 @@ __global__ void __launch_bounds__(NT, 1)
           }
           if (!ok) break;
           mma_commit(&bar[X_VHE + (j & 1)]);
-          if (k1) mma_commit(&bar[X_KE + ((j + 1) & 1)]);
+          if (k1) mma_commit(&bar[X_KE + (j + 1) % NKS]);
         }
         mma_commit(&bar[X_FIN]);
         mbar_wait(&bar[X_FIN], 0, abort_flag, nullptr, 0);
@@ -319,9 +328,9 @@ __global__ void __launch_bounds__(NT, 1)
       const int ct = tid - 64;
       for (int j = 0; j < n_tiles; ++j) {
         const int vb = j & 1;
-        if (!warp_wait(&bar[X_VF], j & 1, abort_flag, p.status, 68)) break;
+        if (!warp_wait(&bar[X_VF + j % NVS], (j / NVS) & 1, abort_flag, p.status, 68)) break;
         if (j >= 2 && !warp_wait(&bar[X_VHE + vb], ((j >> 1) - 1) & 1, abort_flag, p.status, 69)) break;
-        const uint8_t* src = smem + L::V;
+        const uint8_t* src = smem + L::V + (j % NVS) * BN * D;
         uint8_t* dst = smem + L::VH + vb * BN * D * 2;
 #pragma unroll
         for (int rr = 0; rr < 2; ++rr) {
@@ -354,12 +363,12 @@ __global__ void __launch_bounds__(NT, 1)
         __syncwarp();
         if (lane == 0) {
           mbar_arrive(&bar[X_VHF + vb]);
-          mbar_arrive(&bar[X_VE]);
+          mbar_arrive(&bar[X_VE + j % NVS]);
         }
       }
     }
   } else {
-    setmaxnreg_inc224();
+    setmaxnreg_inc208();
     // ------------------------------------------------------------- softmax
     const int s = (warp - 4) >> 2;  // slot
     const int i = tid - 128 - s * 128;
@@ -378,7 +387,6 @@ __global__ void __launch_bounds__(NT, 1)
     float vref = SC == SC_HEAD ? __ldg(p.vs + hk) : 1.0f;
     float m_run = -INFINITY, l_run = 0.0f;
     bool ok = true;
-    uint8_t* sP = smem + L::P + s * BM * BN * 2;
     for (int j = 0; j < n && ok; ++j) {
       const int k0 = j * BN, st = j & 1;
       const float* ksc = reinterpret_cast<const float*>(smem + L::SC + st * 2 * BN * 4);
@@ -387,17 +395,16 @@ __global__ void __launch_bounds__(NT, 1)
       if (SC != SC_HEAD && j == 0) vref = misc[0];
       if (!warp_wait(&bar[X_SF + s], j & 1, abort_flag, p.status, 71)) { ok = false; break; }
       tc_fence_after();
+      // All four 32-column loads in flight before one wait; values used in place.
+      uint32_t tr[BN];
+      tmem_ld32(tS + loff + 0, *reinterpret_cast<uint32_t(*)[32]>(&tr[0]));
+      tmem_ld32(tS + loff + 32, *reinterpret_cast<uint32_t(*)[32]>(&tr[32]));
+      tmem_ld32(tS + loff + 64, *reinterpret_cast<uint32_t(*)[32]>(&tr[64]));
+      tmem_ld32(tS + loff + 96, *reinterpret_cast<uint32_t(*)[32]>(&tr[96]));
+      tmem_ld_wait();
       float t[BN];
 #pragma unroll
-      for (int c = 0; c < BN / 32; ++c) {
-        uint32_t r[32];
-        tmem_ld32(tS + loff + c * 32, r);
-        tmem_ld_wait();
-#pragma unroll
-        for (int k = 0; k < 32; ++k)
-          t[c * 32 + k] = KIND == K_S8 ? __uint_as_float(0x4B400000u + r[k]) : __uint_as_float(r[k]);
-      }
-      tc_fence_before();
+      for (int k = 0; k < BN; ++k) t[k] = KIND == K_S8 ? __uint_as_float(0x4B400000u + tr[k]) : __uint_as_float(tr[k]);
       // per-key K scale; tile-constant K scale folds into the row constant
       float cr = crow;
       if (SC == SC_COL) {
@@ -417,13 +424,12 @@ __global__ void __launch_bounds__(NT, 1)
         for (int k = 0; k < BN; ++k)
           if (k0 + k > lim) t[k] = -INFINITY;
       }
-      float mx0 = -INFINITY, mx1 = -INFINITY;
+      float mx[8];
 #pragma unroll
-      for (int k = 0; k < BN; k += 2) {
-        mx0 = fmaxf(mx0, t[k]);
-        mx1 = fmaxf(mx1, t[k + 1]);
-      }
-      const float mt = fmaxf(mx0, mx1);
+      for (int e = 0; e < 8; ++e) mx[e] = t[e];
+#pragma unroll
+      for (int k = 8; k < BN; ++k) mx[k & 7] = fmaxf(mx[k & 7], t[k]);
+      const float mt = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])), fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
       const float mts = mt == -INFINITY ? -INFINITY : (mt - kBias) * cr;  // tile max of the log2-domain score
       const float m_new = fmaxf(m_run, mts);
       const bool grow = m_new > m_run + 8.0f;
@@ -456,37 +462,36 @@ __global__ void __launch_bounds__(NT, 1)
         vt = vcf[0];
         nbv = vt > 0.0f ? nb + __log2f(vt) : -INFINITY;  // fold s_v / v_ref into the exponent
       }
-      float ls0 = 0.0f, ls1 = 0.0f;
+      // exp2 of all 128 scores first (independent, keeps the XU pipe fed), then
+      // the row sum, then V fold + fp16 packing + stores.
 #pragma unroll
-      for (int c = 0; c < BN / 8; ++c) {
-        uint32_t h[4];
+      for (int k = 0; k < BN; ++k) t[k] = ex2(fmaf(t[k], cr, SC == SC_COL ? nb : nbv));
+      float ls[8];
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int k = c * 8 + 2 * e;
-          float p0, p1;
+      for (int e = 0; e < 8; ++e) ls[e] = t[e];
+#pragma unroll
+      for (int k = 8; k < BN; ++k) ls[k & 7] += t[k];
+      // P' (fp16 pairs) into the first 64 TMEM columns of S_s: two 32-column stores.
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        uint32_t h[32];
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+          const int k = half * 64 + 2 * e;
+          float a = t[k], c2 = t[k + 1];
           if (SC == SC_COL) {
-            p0 = ex2(fmaf(t[k], cr, nb));
-            p1 = ex2(fmaf(t[k + 1], cr, nb));
-            ls0 += p0;
-            ls1 += p1;
-            p0 *= vcf[k];
-            p1 *= vcf[k + 1];
-          } else {
-            p0 = ex2(fmaf(t[k], cr, nbv));
-            p1 = ex2(fmaf(t[k + 1], cr, nbv));
-            ls0 += p0;
-            ls1 += p1;
+            a *= vcf[k];
+            c2 *= vcf[k + 1];
           }
-          const __half2 hv = __floats2half2_rn(p0, p1);
+          const __half2 hv = __floats2half2_rn(a, c2);
           h[e] = *reinterpret_cast<const uint32_t*>(&hv);
         }
-        *reinterpret_cast<uint4*>(sP + (c >> 3) * (BM * 128) + swz128_offset(i, c & 7)) =
-            make_uint4(h[0], h[1], h[2], h[3]);
+        tmem_st32(tS + loff + half * 32, h);
       }
-      float lsum = ls0 + ls1;
+      tmem_st_wait();
+      float lsum = ((ls[0] + ls[1]) + (ls[2] + ls[3])) + ((ls[4] + ls[5]) + (ls[6] + ls[7]));
       if (SC == SC_TILE) lsum = vt > 0.0f ? lsum / vt : 0.0f;
       l_run += lsum;
-      fence_async_smem();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) {
