@@ -174,9 +174,14 @@ FAQ_API fa_status fa_rotate_quantize(const fa_tensor* q, const fa_tensor* k, con
  *   out: device bf16, q's layout and dims.  lse: nullable device fp32
  *   [B, Hq, Sq], natural-log sum-exp of the scaled scores (-inf for a row
  *   with no visible key, whose output is 0).
- *   Decode (q->S == 1) runs a split-KV kernel and an LSE combine; it needs
- *   `workspace` of at least fa_attention_workspace_size() bytes
- *   (FA_ERR_WORKSPACE otherwise).  num_splits: 0 = choose automatically.
+ *   workspace: device memory of at least fa_attention_workspace_size()
+ *   bytes, 256-byte aligned, owned by the caller and only used during the
+ *   call's kernels (FA_ERR_WORKSPACE if missing, short or misaligned).
+ *   Decode (q->S == 1) keeps its split-KV partials there before an LSE
+ *   combine; FP8 / INT8 prefill keeps V' = fp16(code * s_v / r_t) there
+ *   (r_t the largest V scale of each 128-key tile, written beside it), made
+ *   once per call by a pre-pass and read by every query tile; MXFP4 needs
+ *   none.  num_splits (decode only): 0 = choose automatically.
  *   Modes run here: INT8_PER_HEAD, FP8_PER_TOKEN, FP8_BLOCK and
  *   MXFP4_PER_BLOCK for prefill; INT8_PER_HEAD for decode (others ->
  *   FA_ERR_UNSUPPORTED).
@@ -219,7 +224,9 @@ FAQ_API fa_status fa_attention_decode_noalloc(const fa_qtensor* q, const fa_qten
                                               fa_stream_t s);
 
 /* Workspace bytes fa_attention_quant needs for these operands and split
- * count (0 for prefill).  Returns 0 on invalid arguments. */
+ * count: decode B*Hq*splits*(D+2)*4; FP8 / INT8 prefill
+ * B*Hkv*Sk*D*2 + B*Hkv*ceil(Sk/128)*4 (each part rounded up to 256);
+ * MXFP4 prefill 0.  Returns 0 on invalid arguments. */
 FAQ_API size_t fa_attention_workspace_size(const fa_qtensor* q, const fa_qtensor* k, int num_splits);
 
 /* Synchronise `s`, read and clear this device's status word.  Returns

@@ -1,31 +1,33 @@
-// attn2.cu -- prefill attention on FP8 (E4M3) and INT8 operands, two query
-// tiles per CTA (FlashAttention's online softmax on the low-bit operands:
-// MindIE SD "量化", FA量化 / FP8 Attention; wiki "FA 量化" 参考资料).
+// attn2.cu -- prefill attention on FP8 (E4M3) and INT8 operands
+// (FlashAttention's online softmax on low-bit operands: MindIE SD "量化",
+// FA量化 / FP8 Attention; wiki "FA 量化" 参考资料).
 //
-// A CTA owns two 128-row query "slots" that read the same kv head (two query
-// heads of one GQA group at the same rows, or two consecutive row tiles of one
-// head) and streams their visible 128-key K/V tiles once for both:
+// Two kernels per call:
+//   vprep: V codes -> V' = fp16(code * s_v / r_t) once per call, r_t = the
+//     largest V scale of 128-key tile t (INT8: V' = fp16(code), exact), into
+//     a caller workspace, with r_t beside it.  Every query tile reads the same
+//     V tiles, so the conversion is done once instead of once per query tile.
+//   attn2: one CTA owns one 128-row query tile of one head and streams its
+//     visible 128-key tiles.  S is double-buffered in TMEM, so Q K^T of tile
+//     j+1 runs on the tensor pipe while the softmax of tile j runs on the SM
+//     cores:
 //   warpgroup 0 (88 registers per thread after setmaxnreg):
-//     warp 0   producer: Q tiles once; per K/V tile the K codes (3-stage ring)
-//              and V codes (2-stage ring) by TMA, and the tile's K scales and
-//              V factors s_v / v_ref into a 2-stage shared ring.
-//     warp 1   MMA issuer (one thread), over the two slots:
-//              S_s = Q_s K^T (kind::f8f6f4 / kind::i8) into slot s's TMEM S,
-//              and O_s += P'_s V' (kind::f16 with the A operand P'_s in TMEM,
-//              where the softmax stored it over S_s).  PV_s(j) and then
-//              QK_s(j+1) are issued once slot s's softmax of tile j is done;
-//              the tensor pipe runs them in order, so P'_s is read before S_s
-//              is overwritten, and the other slot's softmax runs meanwhile.
-//     warps 2-3  V codes -> V' = fp16(code) (exact), MN-major, 128B-swizzled,
-//              double-buffered.
-//   warpgroups 1 and 2 (208 registers per thread): softmax of slot 0 and slot 1, one
-//     thread per query row: S from TMEM, K scale, mask, online max in the
-//     exp2 domain (O rescaled in TMEM only when the max grows by more than
-//     2^8), p = exp2(t * c - m), P' = fp16(p * s_v / v_ref) stored into the
-//     first 64 TMEM columns of S_s (tcgen05.st).
-// TMEM: S_0/P'_0, S_1/P'_1, O_0, O_1 (4 x 128 columns).  Keeping P' in TMEM
-// keeps it off the shared-memory port, which the shared-memory operands of
-// Q K^T and the V' operand of P.V already load heavily.  Every wait is bounded.
+//     warp 0   producer: Q once; per tile the K codes (3-stage ring) and the
+//              V' tile (2-stage ring) by TMA, and the tile's per-key K scales
+//              and V' factor r_t / v_ref into a 4-stage shared ring.
+//     warp 1   MMA issuer (one thread): S_b = Q K^T (kind::f8f6f4 / kind::i8)
+//              into TMEM buffer b = j % 2, and O += P' V' (kind::f16, A = P'
+//              read from TMEM where the softmax stored it over S_b).  QK(j+2)
+//              is issued right after PV(j); the tensor pipe runs them in
+//              order, so P'_b is consumed before S_b is rewritten.
+//   warpgroups 1 and 2 (208 registers per thread): the softmax, one thread
+//     per (query row, half of the 128 keys): S from TMEM, per-key K scale,
+//     mask, the tile's row maximum combined across the two halves through
+//     shared memory, online max in the exp2 domain (O rescaled in TMEM only
+//     when the max grows by more than 2^8), p = exp2(t * c - m), and
+//     P' = fp16(p * r_t / v_ref) (the factor enters the exponent; the row sum
+//     takes p itself) stored over the half's own S columns (tcgen05.st).
+// TMEM: S_0/P'_0, S_1/P'_1, O (384 of 512 columns).  Every wait is bounded.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <math.h>
@@ -40,9 +42,11 @@ using namespace attn;
 
 constexpr int BM = 128;
 constexpr int BN = 128;
-constexpr int NT = 384;  // 12 warps
-constexpr int NKS = 3;   // K code stages
-constexpr int NVS = 2;   // V code stages
+constexpr int HN = BN / 2;  // keys per softmax half
+constexpr int NT = 384;     // 12 warps
+constexpr int NKS = 3;      // K code stages
+constexpr int NVS = 2;      // V' stages
+constexpr int NSC = 4;      // scale ring stages
 
 enum { K_E4M3 = 0, K_S8 = 1 };
 enum { SC_HEAD = 0, SC_COL = 1, SC_TILE = 2 };  // one scale per head / per key / per 128-key tile
@@ -53,22 +57,24 @@ struct P2 {
   const float* qs;
   const float* ks;
   const float* vs;
+  const float* fv;  // [B, Hkv, ntiles] V' tile factors r_t (FP8 operands)
   int q_blk, k_blk, v_blk, q_nblk, k_nblk, v_nblk;
+  int ntiles_k;
   __nv_bfloat16* out;
   float* lse;
   int* status;
   int n_qtiles;
-  int pair_heads;  // 1: the slots are query heads 2p, 2p+1 at one row tile; 0: row tiles 2t, 2t+1 of one head
 };
 
 template <int D>
 struct L2 {
-  static constexpr uint32_t Q = 0;                   // 2 x [128][D]
-  static constexpr uint32_t K = Q + 2 * BM * D;        // NKS stages
-  static constexpr uint32_t V = K + NKS * BN * D;      // NVS stages
-  static constexpr uint32_t VH = V + NVS * BN * D;     // 2 x fp16 V'
-  static constexpr uint32_t SC = VH + 2 * BN * D * 2;  // 2 stages x ([128] k scale, [128] v factor)
-  static constexpr uint32_t MISC = SC + 2 * 2 * BN * 4;
+  static constexpr uint32_t Q = 0;                   // [128][D]
+  static constexpr uint32_t K = Q + BM * D;            // NKS stages
+  static constexpr uint32_t VH = K + NKS * BN * D;     // NVS stages of fp16 V'
+  static constexpr uint32_t SC = VH + NVS * BN * D * 2;  // NSC stages x ([128] k scale, V' factor log2, its inverse)
+  static constexpr uint32_t XM = SC + NSC * 2 * BN * 4;  // 2 stages x 2 halves x [128] tile row max
+  static constexpr uint32_t XL = XM + 2 * 2 * BM * 4;  // 2 halves x [128] row sum
+  static constexpr uint32_t MISC = XL + 2 * BM * 4;
   static constexpr uint32_t BAR = MISC + 64;
   static constexpr uint32_t TOTAL = BAR + 512;
   static constexpr uint32_t ALLOC = TOTAL + 1024;
@@ -78,17 +84,17 @@ enum {
   X_Q = 0,
   X_KF = 1,    // [NKS]
   X_KE = 4,    // [NKS]
-  X_VF = 7,    // [NVS]
-  X_VE = 9,    // [NVS]
-  X_VHF = 11,  // [2]
-  X_VHE = 13,  // [2]
-  X_SF = 15,   // [2 slots]
-  X_PF = 17,   // [2 slots]
-  X_PVD = 19,  // [2 slots]
-  X_SCF = 21,  // [2]
-  X_SCE = 23,  // [2 slots][2 stages]
-  X_FIN = 27,
-  X_COUNT = 28
+  X_VF = 7,    // [NVS] V' stage full
+  X_VE = 9,    // [NVS] V' stage empty
+  X_SF = 15,   // [2] S buffer full
+  X_PF = 17,   // [2] P' buffer full
+  X_PVD = 19,  // P V done
+  X_SCF = 20,  // [NSC] scale ring stage full
+  X_SCE = 24,  // [NSC] scale ring stage empty
+  X_MX = 28,   // [2] row-max exchange
+  X_LX = 30,   // row-sum exchange
+  X_FIN = 31,
+  X_COUNT = 32
 };
 
 __device__ __forceinline__ void setmaxnreg_inc208() { asm volatile("setmaxnreg.inc.sync.aligned.u32 208;"); }
@@ -98,6 +104,7 @@ template <int KIND, int D, int SC>
 __global__ void __launch_bounds__(NT, 1)
     attn2_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
                  const __grid_constant__ CUtensorMap tmv, const P2 p) {
+  static_assert(KIND == K_E4M3 || SC == SC_HEAD, "INT8 operands carry one scale per head");
   using L = L2<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -108,43 +115,22 @@ __global__ void __launch_bounds__(NT, 1)
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
-  // ---- work item: (b, kv head) and two query slots
-  int hqs[2], q0s[2], ns[2], kv_ends[2];
-  int b, hk;
+  // ---- work item: (b, query head, query tile); causal runs the longest tiles first
+  int b, hq, q0;
   {
+    const int per_t = p.B * p.Hq;
     const int widx = blockIdx.x;
-    if (p.pair_heads) {
-      const int npair = p.Hq / 2;
-      const int per_t = p.B * npair;
-      const int qt = p.causal ? (p.n_qtiles - 1 - widx / per_t) : (widx / per_t);
-      const int r = widx % per_t;
-      b = r / npair;
-      const int pr = r % npair;
-      hqs[0] = 2 * pr;
-      hqs[1] = 2 * pr + 1;
-      q0s[0] = q0s[1] = qt * BM;
-    } else {
-      const int npairs_t = (p.n_qtiles + 1) / 2;
-      const int per_t = p.B * p.Hq;
-      const int tp = p.causal ? (npairs_t - 1 - widx / per_t) : (widx / per_t);
-      const int r = widx % per_t;
-      b = r / p.Hq;
-      hqs[0] = hqs[1] = r % p.Hq;
-      q0s[0] = 2 * tp * BM;
-      q0s[1] = (2 * tp + 1) * BM;
-    }
-    hk = hqs[0] / p.group;
-    const int diag = p.Sk - p.Sq;
-#pragma unroll
-    for (int s = 0; s < 2; ++s) {
-      int e = 0;
-      if (q0s[s] < p.Sq) e = p.causal ? min(p.Sk, max(0, min(q0s[s] + BM, p.Sq) - 1 + diag + 1)) : p.Sk;
-      kv_ends[s] = e;
-      ns[s] = (e + BN - 1) / BN;
-    }
+    const int qt = p.causal ? (p.n_qtiles - 1 - widx / per_t) : (widx / per_t);
+    const int r = widx % per_t;
+    b = r / p.Hq;
+    hq = r % p.Hq;
+    q0 = qt * BM;
   }
-  const int n_tiles = max(ns[0], ns[1]);
-  const int kv_end = max(kv_ends[0], kv_ends[1]);
+  const int hk = hq / p.group;
+  const int diag = p.Sk - p.Sq;
+  int kv_end = 0;
+  if (q0 < p.Sq) kv_end = p.causal ? min(p.Sk, max(0, min(q0 + BM, p.Sq) - 1 + diag + 1)) : p.Sk;
+  const int n = (kv_end + BN - 1) / BN;
   const int bhk = b * p.Hkv + hk;
 
   if (tid == 0) {
@@ -155,16 +141,17 @@ __global__ void __launch_bounds__(NT, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&bar[X_VF + i], 1);
-      mbar_init(&bar[X_VE + i], 2);
-      mbar_init(&bar[X_VHF + i], 2);
-      mbar_init(&bar[X_VHE + i], 1);
+      mbar_init(&bar[X_VE + i], 1);
       mbar_init(&bar[X_SF + i], 1);
-      mbar_init(&bar[X_PF + i], 4);
-      mbar_init(&bar[X_PVD + i], 1);
-      mbar_init(&bar[X_SCF + i], 1);
-      mbar_init(&bar[X_SCE + i], 4);
-      mbar_init(&bar[X_SCE + 2 + i], 4);
+      mbar_init(&bar[X_PF + i], 8);
+      mbar_init(&bar[X_MX + i], 8);
     }
+    for (int i = 0; i < NSC; ++i) {
+      mbar_init(&bar[X_SCF + i], 1);
+      mbar_init(&bar[X_SCE + i], 8);  // the softmax warps
+    }
+    mbar_init(&bar[X_PVD], 1);
+    mbar_init(&bar[X_LX], 8);
     mbar_init(&bar[X_FIN], 1);
     *abort_flag = 0;
     fence_barrier_init();
@@ -176,209 +163,159 @@ __global__ void __launch_bounds__(NT, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tbase = *tmem_slot;
+  const uint32_t tO = tbase + 256;
 
   if (warp < 4) {
     setmaxnreg_dec88();
+    const bool bnsd = p.layout == FA_LAYOUT_BNSD;
     if (warp == 0) {
-      // ------------------------------------------------------------ producer
-      if (n_tiles > 0) {
-        const bool bnsd = p.layout == FA_LAYOUT_BNSD;
-        float vref = 1.0f;
-        if (SC != SC_HEAD) {
-          float m = 0.0f;
-          const int nb_end = (kv_end + p.v_blk - 1) / p.v_blk;
-          for (int t = lane; t < nb_end; t += 32) m = fmaxf(m, __ldg(p.vs + (long long)bhk * p.v_nblk + t));
-#pragma unroll
-          for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
-          vref = m > 0.0f ? m : 1.0f;
-          if (lane == 0) misc[0] = vref;
-        }
-        const float vinv = 1.0f / vref;
-        if (lane == 0) {
-          tma_prefetch_desc(&tmq);
-          tma_prefetch_desc(&tmk);
-          tma_prefetch_desc(&tmv);
-          const int nq = (ns[0] > 0 ? 1 : 0) + (ns[1] > 0 ? 1 : 0);
-          mbar_arrive_expect_tx(&bar[X_Q], nq * BM * D);
-#pragma unroll
-          for (int s = 0; s < 2; ++s)
-            if (ns[s] > 0)
-              tma_load_4d(smem + L::Q + s * BM * D, &tmq, &bar[X_Q], 0, bnsd ? q0s[s] : hqs[s], bnsd ? hqs[s] : q0s[s], b);
-        }
+      // ------------------------------------------------------ Q and K loads
+      if (lane == 0 && n > 0) {
+        tma_prefetch_desc(&tmq);
+        tma_prefetch_desc(&tmk);
+        mbar_arrive_expect_tx(&bar[X_Q], BM * D);
+        tma_load_4d(smem + L::Q, &tmq, &bar[X_Q], 0, bnsd ? q0 : hq, bnsd ? hq : q0, b);
         int j = 0;
-        for (; j < n_tiles; ++j) {
-          const int k0 = j * BN, st = j & 1;
-          bool ok = true;
-          if (SC != SC_HEAD) {
-            // scale ring stage st is free once both slots finished tile j - 2
-            for (int s = 0; s < 2 && ok; ++s)
-              if (j >= 2 && j - 2 < ns[s]) ok = mbar_wait(&bar[X_SCE + 2 * s + st], ((j >> 1) - 1) & 1, abort_flag, p.status, 60);
-            if (!__all_sync(0xffffffffu, ok)) break;
-            float* ksc = reinterpret_cast<float*>(smem + L::SC + st * 2 * BN * 4);
-            float* vcf = ksc + BN;
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              const int c = lane * 4 + q, tok = k0 + c;
-              float kv = 0.0f, vv = 0.0f;
-              if (tok < p.Sk) {
-                kv = __ldg(p.ks + (long long)bhk * p.k_nblk + tok / p.k_blk);
-                vv = __ldg(p.vs + (long long)bhk * p.v_nblk + tok / p.v_blk) * vinv;
-              }
-              ksc[c] = kv;
-              vcf[c] = vv;
-            }
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&bar[X_SCF + st]);
-          }
-          if (lane == 0) {
-            const int ks = j % NKS, vs = j % NVS;
-            if (j >= NKS) ok = mbar_wait(&bar[X_KE + ks], ((j / NKS) - 1) & 1, abort_flag, p.status, 61);
-            if (ok) {
-              mbar_arrive_expect_tx(&bar[X_KF + ks], BN * D);
-              tma_load_4d(smem + L::K + ks * BN * D, &tmk, &bar[X_KF + ks], 0, bnsd ? k0 : hk, bnsd ? hk : k0, b);
-              if (j >= NVS) ok = mbar_wait(&bar[X_VE + vs], ((j / NVS) - 1) & 1, abort_flag, p.status, 62);
-              if (ok) {
-                mbar_arrive_expect_tx(&bar[X_VF + vs], BN * D);
-                tma_load_4d(smem + L::V + vs * BN * D, &tmv, &bar[X_VF + vs], 0, bnsd ? k0 : hk, bnsd ? hk : k0, b);
-              }
-            }
-          }
-          if (!__all_sync(0xffffffffu, ok)) { ++j; break; }
+        for (; j < n; ++j) {
+          const int k0 = j * BN, ks = j % NKS;
+          if (j >= NKS && !mbar_wait(&bar[X_KE + ks], ((j / NKS) - 1) & 1, abort_flag, p.status, 61)) break;
+          mbar_arrive_expect_tx(&bar[X_KF + ks], BN * D);
+          tma_load_4d(smem + L::K + ks * BN * D, &tmk, &bar[X_KF + ks], 0, bnsd ? k0 : hk, bnsd ? hk : k0, b);
         }
-        if (lane == 0 && *abort_flag) {
+        if (*abort_flag) {
           // let issued loads land before the CTA can exit
+          mbar_wait(&bar[X_Q], 0, abort_flag, nullptr, 0);
           for (int t = max(0, j - NKS); t < j; ++t) mbar_wait(&bar[X_KF + t % NKS], (t / NKS) & 1, abort_flag, nullptr, 0);
+        }
+      }
+      __syncwarp();
+    } else if (warp == 3) {
+      // --------------------------------------------------------- V' loads
+      if (lane == 0 && n > 0) {
+        tma_prefetch_desc(&tmv);
+        int j = 0;
+        for (; j < n; ++j) {
+          const int k0 = j * BN, vs = j % NVS;
+          if (j >= NVS && !mbar_wait(&bar[X_VE + vs], ((j / NVS) - 1) & 1, abort_flag, p.status, 62)) break;
+          // V' [b][hk][token][D] fp16: one 64-column box per 128-byte swizzle atom
+          mbar_arrive_expect_tx(&bar[X_VF + vs], BN * D * 2);
+#pragma unroll
+          for (int a2 = 0; a2 < D / 64; ++a2)
+            tma_load_4d(smem + L::VH + vs * BN * D * 2 + a2 * BN * 128, &tmv, &bar[X_VF + vs], 64 * a2, k0, hk, b);
+        }
+        if (*abort_flag)
           for (int t = max(0, j - NVS); t < j; ++t) mbar_wait(&bar[X_VF + t % NVS], (t / NVS) & 1, abort_flag, nullptr, 0);
+      }
+      __syncwarp();
+    } else if (warp == 2) {
+      // ------------------------------------------------------- scale ring
+      if (SC != SC_HEAD && n > 0) {
+        // v_ref = the largest V' factor over this CTA's visible tiles
+        const float* fvh = p.fv + (long long)bhk * p.ntiles_k;
+        float m = 0.0f;
+        for (int t = lane; t < n; t += 32) m = fmaxf(m, __ldg(fvh + t));
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+        const float vref = m > 0.0f ? m : 1.0f;
+        if (lane == 0) misc[0] = vref;
+        for (int j = 0; j < n; ++j) {
+          const int k0 = j * BN, st = j % NSC;
+          float kv[4];
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const int tok = k0 + lane * 4 + q;
+            kv[q] = tok < p.Sk ? __ldg(p.ks + (long long)bhk * p.k_nblk + tok / p.k_blk) : 0.0f;
+          }
+          const float fj = __ldg(fvh + j);
+          if (j >= NSC && !warp_wait(&bar[X_SCE + st], ((j / NSC) - 1) & 1, abort_flag, p.status, 60)) break;
+          float* ksc = reinterpret_cast<float*>(smem + L::SC + st * 2 * BN * 4);
+          *reinterpret_cast<float4*>(ksc + lane * 4) = make_float4(kv[0], kv[1], kv[2], kv[3]);
+          if (lane == 0) {
+            // V' factor r_t / v_ref enters the exponent as its log2, floored at -60
+            // (a tile that small adds nothing visible to O); the row sum divides it out.
+            const float fl = fmaxf(__log2f(fj / vref), -60.0f);
+            ksc[BN] = fl;
+            ksc[BN + 1] = exp2f(-fl);
+          }
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&bar[X_SCF + st]);
         }
       }
       __syncwarp();
     } else if (warp == 1) {
       // ---------------------------------------------------------- MMA issuer
-      if (lane == 0 && n_tiles > 0) {
+      if (lane == 0 && n > 0) {
         constexpr uint32_t SW = D == 128 ? kSwz128 : kSwz64;
         constexpr uint32_t SBO8 = D == 128 ? 1024 : 512;
         constexpr uint32_t idesc_qk = KIND == K_E4M3 ? make_idesc(kAccF32, kFmtE4M3, kFmtE4M3, 0, 0, BN, BM)
                                                      : make_idesc(kAccS32, kFmtS8, kFmtS8, 0, 0, BN, BM);
         constexpr uint32_t idesc_pv = make_idesc(kAccF32, kFmtF16, kFmtF16, 0, 1, D, BM);
-        auto qk = [&](int s, int j) {
-          const uint32_t sQ = smem_u32(smem + L::Q + s * BM * D);
+        const uint32_t sQ = smem_u32(smem + L::Q);
+        auto qk = [&](int j) {
           const uint32_t sK = smem_u32(smem + L::K + (j % NKS) * BN * D);
 #pragma unroll
           for (int kk = 0; kk < D / 32; ++kk) {
             const uint64_t da = make_sdesc(sQ + kk * 32, 16, SBO8, SW);
             const uint64_t db = make_sdesc(sK + kk * 32, 16, SBO8, SW);
             if (KIND == K_E4M3)
-              mma_f8f6f4(tbase + s * 128, da, db, idesc_qk, kk > 0);
+              mma_f8f6f4(tbase + (j & 1) * 128, da, db, idesc_qk, kk > 0);
             else
-              mma_i8(tbase + s * 128, da, db, idesc_qk, kk > 0);
+              mma_i8(tbase + (j & 1) * 128, da, db, idesc_qk, kk > 0);
           }
-          mma_commit(&bar[X_SF + s]);
+          mma_commit(&bar[X_SF + (j & 1)]);
+          mma_commit(&bar[X_KE + j % NKS]);
         };
-        auto pv = [&](int s, int j) {
-          // A = P'_s in TMEM: 16 fp16 of K per MMA = 8 columns
-          const uint32_t sVh = smem_u32(smem + L::VH + (j & 1) * BN * D * 2);
+        auto pv = [&](int j) {
+          // A = P' in TMEM: keys [0, 64) in columns 0..31 and keys [64, 128) in
+          // columns 64..95 of the S buffer; 16 keys (8 columns) per MMA.
+          const uint32_t sVh = smem_u32(smem + L::VH + (j % NVS) * BN * D * 2);
+          const uint32_t tP = tbase + (j & 1) * 128;
 #pragma unroll
           for (int ks = 0; ks < BN / 16; ++ks) {
             const uint64_t db = make_sdesc(sVh + ks * 16 * 128, BN * 128, 1024, kSwz128);
-            mma_f16_ts(tbase + 256 + s * 128, tbase + s * 128 + ks * 8, db, idesc_pv, (j > 0 || ks > 0) ? 1u : 0u);
+            mma_f16_ts(tO, tP + (ks >> 2) * 64 + (ks & 3) * 8, db, idesc_pv, (j > 0 || ks > 0) ? 1u : 0u);
           }
-          mma_commit(&bar[X_PVD + s]);
+          mma_commit(&bar[X_PVD]);
+          mma_commit(&bar[X_VE + j % NVS]);
         };
         bool ok = mbar_wait(&bar[X_Q], 0, abort_flag, p.status, 63);
-        if (ok) ok = mbar_wait(&bar[X_KF], 0, abort_flag, p.status, 64);
-        if (ok) {
-          tc_fence_after();
-          if (ns[0] > 0) qk(0, 0);
-          if (ns[1] > 0) qk(1, 0);
-          mma_commit(&bar[X_KE]);
+        for (int j = 0; ok && j < 2 && j < n; ++j) {
+          ok = mbar_wait(&bar[X_KF + j], 0, abort_flag, p.status, 64);
+          if (ok) {
+            tc_fence_after();
+            qk(j);
+          }
         }
-        for (int j = 0; ok && j < n_tiles; ++j) {
-          // slot s: PV_s(j) (reads P'_s over S_s), then QK_s(j+1) (rewrites S_s)
-          bool vh = false, k1 = false;
-          for (int s = 0; s < 2 && ok; ++s) {
-            if (j >= ns[s]) continue;
-            ok = mbar_wait(&bar[X_PF + s], j & 1, abort_flag, p.status, 65);
-            if (ok && !vh) {
-              ok = mbar_wait(&bar[X_VHF + (j & 1)], (j >> 1) & 1, abort_flag, p.status, 66);
-              vh = true;
-            }
+        for (int j = 0; ok && j < n; ++j) {
+          ok = mbar_wait(&bar[X_PF + (j & 1)], (j >> 1) & 1, abort_flag, p.status, 65);
+          if (ok) ok = mbar_wait(&bar[X_VF + j % NVS], (j / NVS) & 1, abort_flag, p.status, 66);
+          if (!ok) break;
+          tc_fence_after();
+          pv(j);
+          if (j + 2 < n) {
+            ok = mbar_wait(&bar[X_KF + (j + 2) % NKS], ((j + 2) / NKS) & 1, abort_flag, p.status, 67);
             if (!ok) break;
             tc_fence_after();
-            pv(s, j);
-            if (j + 1 < ns[s]) {
-              if (!k1) {
-                ok = mbar_wait(&bar[X_KF + (j + 1) % NKS], ((j + 1) / NKS) & 1, abort_flag, p.status, 67);
-                k1 = true;
-                if (!ok) break;
-                tc_fence_after();
-              }
-              qk(s, j + 1);
-            }
+            qk(j + 2);
           }
-          if (!ok) break;
-          mma_commit(&bar[X_VHE + (j & 1)]);
-          if (k1) mma_commit(&bar[X_KE + (j + 1) % NKS]);
         }
         mma_commit(&bar[X_FIN]);
         mbar_wait(&bar[X_FIN], 0, abort_flag, nullptr, 0);
       }
       __syncwarp();
-    } else {
-      // --------------------------------------------------------- V converter
-      const int ct = tid - 64;
-      for (int j = 0; j < n_tiles; ++j) {
-        const int vb = j & 1;
-        if (!warp_wait(&bar[X_VF + j % NVS], (j / NVS) & 1, abort_flag, p.status, 68)) break;
-        if (j >= 2 && !warp_wait(&bar[X_VHE + vb], ((j >> 1) - 1) & 1, abort_flag, p.status, 69)) break;
-        const uint8_t* src = smem + L::V + (j % NVS) * BN * D;
-        uint8_t* dst = smem + L::VH + vb * BN * D * 2;
-#pragma unroll
-        for (int rr = 0; rr < 2; ++rr) {
-          const int r = ct + rr * 64;
-#pragma unroll
-          for (int c = 0; c < D / 16; ++c) {
-            const uint32_t soff = D == 128 ? swz128_offset(r, c) : swz64_offset(r, c);
-            const uint4 raw = *reinterpret_cast<const uint4*>(src + soff);
-            const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
-            uint32_t h[8];
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              if (KIND == K_E4M3) {
-                h[2 * i] = e4m3x2_to_h2((uint16_t)(w[i] & 0xFFFF));
-                h[2 * i + 1] = e4m3x2_to_h2((uint16_t)(w[i] >> 16));
-              } else {
-                const uint32_t ub = w[i] ^ 0x80808080u;
-                h[2 * i] = s8x2_to_h2(ub, 0x4140);
-                h[2 * i + 1] = s8x2_to_h2(ub, 0x4342);
-              }
-            }
-            const int d0 = c * 16;
-            uint8_t* base = dst + (d0 >> 6) * (BN * 128);
-            const int cc = (d0 & 63) >> 3;
-            *reinterpret_cast<uint4*>(base + swz128_offset(r, cc)) = make_uint4(h[0], h[1], h[2], h[3]);
-            *reinterpret_cast<uint4*>(base + swz128_offset(r, cc + 1)) = make_uint4(h[4], h[5], h[6], h[7]);
-          }
-        }
-        fence_async_smem();
-        __syncwarp();
-        if (lane == 0) {
-          mbar_arrive(&bar[X_VHF + vb]);
-          mbar_arrive(&bar[X_VE + j % NVS]);
-        }
-      }
     }
   } else {
     setmaxnreg_inc208();
     // ------------------------------------------------------------- softmax
-    const int s = (warp - 4) >> 2;  // slot
-    const int i = tid - 128 - s * 128;
-    const uint32_t loff = (uint32_t)(((warp - 4) & 3) * 32) << 16;
-    const uint32_t tS = tbase + s * 128, tO = tbase + 256 + s * 128;
-    const int hq = hqs[s], q0 = q0s[s], n = ns[s];
+    const int h = (warp - 4) >> 2;  // key half: columns [h * 64, h * 64 + 64) of each S tile
+    const int i = tid - 128 - h * 128;
+    const uint32_t loff = (uint32_t)((warp & 3) * 32) << 16;
+    const int cb = h * HN;
     const int row = q0 + i;
     const bool row_ok = row < p.Sq;
     const int qbh = b * p.Hq + hq;
-    const int diag = p.Sk - p.Sq;
+    float* xm = reinterpret_cast<float*>(smem + L::XM);
+    float* xl = reinterpret_cast<float*>(smem + L::XL);
     const float sq = row_ok ? scale_at(p.qs, p.q_blk, p.q_nblk, qbh, hq, row) : 0.0f;
     float crow = sq * p.scale_log2;
     if (SC == SC_HEAD) crow *= __ldg(p.ks + hk);
@@ -389,134 +326,148 @@ __global__ void __launch_bounds__(NT, 1)
     bool ok = true;
     for (int j = 0; j < n && ok; ++j) {
       const int k0 = j * BN, st = j & 1;
-      const float* ksc = reinterpret_cast<const float*>(smem + L::SC + st * 2 * BN * 4);
-      const float* vcf = ksc + BN;
-      if (SC != SC_HEAD && !warp_wait(&bar[X_SCF + st], (j >> 1) & 1, abort_flag, p.status, 70)) { ok = false; break; }
+      const uint32_t tS = tbase + st * 128 + cb;
+      const int sst = j % NSC;
+      const float* ksc = reinterpret_cast<const float*>(smem + L::SC + sst * 2 * BN * 4);
+      if (SC != SC_HEAD && !warp_wait(&bar[X_SCF + sst], (j / NSC) & 1, abort_flag, p.status, 70)) { ok = false; break; }
       if (SC != SC_HEAD && j == 0) vref = misc[0];
-      if (!warp_wait(&bar[X_SF + s], j & 1, abort_flag, p.status, 71)) { ok = false; break; }
+      // this tile's K scales and V' factor, loaded while S is still being computed
+      float4 kk4[HN / 4];
+      if (SC == SC_COL) {
+#pragma unroll
+        for (int k = 0; k < HN; k += 4) kk4[k / 4] = *reinterpret_cast<const float4*>(ksc + cb + k);
+      }
+      float flog = 0.0f, finv = 1.0f, ktile = 1.0f;
+      if (SC != SC_HEAD) {
+        flog = ksc[BN];
+        finv = ksc[BN + 1];
+      }
+      if (SC == SC_TILE) ktile = ksc[0];
+      if (!warp_wait(&bar[X_SF + st], (j >> 1) & 1, abort_flag, p.status, 71)) { ok = false; break; }
       tc_fence_after();
-      // All four 32-column loads in flight before one wait; values used in place.
-      uint32_t tr[BN];
+      uint32_t tr[HN];
       tmem_ld32(tS + loff + 0, *reinterpret_cast<uint32_t(*)[32]>(&tr[0]));
       tmem_ld32(tS + loff + 32, *reinterpret_cast<uint32_t(*)[32]>(&tr[32]));
-      tmem_ld32(tS + loff + 64, *reinterpret_cast<uint32_t(*)[32]>(&tr[64]));
-      tmem_ld32(tS + loff + 96, *reinterpret_cast<uint32_t(*)[32]>(&tr[96]));
       tmem_ld_wait();
-      float t[BN];
+      float t[HN];
 #pragma unroll
-      for (int k = 0; k < BN; ++k) t[k] = KIND == K_S8 ? __uint_as_float(0x4B400000u + tr[k]) : __uint_as_float(tr[k]);
-      // per-key K scale; tile-constant K scale folds into the row constant
+      for (int k = 0; k < HN; ++k) t[k] = KIND == K_S8 ? __uint_as_float(0x4B400000u + tr[k]) : __uint_as_float(tr[k]);
+      // per-key K scale; a tile-constant K scale folds into the row constant
       float cr = crow;
       if (SC == SC_COL) {
 #pragma unroll
-        for (int k = 0; k < BN; k += 4) {
-          const float4 kk4 = *reinterpret_cast<const float4*>(ksc + k);
-          t[k] *= kk4.x; t[k + 1] *= kk4.y; t[k + 2] *= kk4.z; t[k + 3] *= kk4.w;
+        for (int k = 0; k < HN; k += 4) {
+          fmul2(t[k], t[k + 1], kk4[k / 4].x, kk4[k / 4].y);
+          fmul2(t[k + 2], t[k + 3], kk4[k / 4].z, kk4[k / 4].w);
         }
       } else if (SC == SC_TILE) {
-        cr *= ksc[0];
+        cr *= ktile;
       }
       // masks: keys past the sequence, and causal
-      const bool need_mask = (k0 + BN > p.Sk) || (p.causal && (k0 + BN - 1 > q0 + diag));
+      const int kc0 = k0 + cb;
+      const bool need_mask = (kc0 + HN > p.Sk) || (p.causal && (kc0 + HN - 1 > q0 + diag));
       if (need_mask) {
         const int lim = p.causal ? min(p.Sk - 1, row + diag) : p.Sk - 1;
 #pragma unroll
-        for (int k = 0; k < BN; ++k)
-          if (k0 + k > lim) t[k] = -INFINITY;
+        for (int k = 0; k < HN; ++k)
+          if (kc0 + k > lim) t[k] = -INFINITY;
       }
       float mx[8];
 #pragma unroll
       for (int e = 0; e < 8; ++e) mx[e] = t[e];
 #pragma unroll
-      for (int k = 8; k < BN; ++k) mx[k & 7] = fmaxf(mx[k & 7], t[k]);
+      for (int k = 8; k < HN; ++k) mx[k & 7] = fmaxf(mx[k & 7], t[k]);
       const float mt = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])), fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
-      const float mts = mt == -INFINITY ? -INFINITY : (mt - kBias) * cr;  // tile max of the log2-domain score
-      const float m_new = fmaxf(m_run, mts);
+      const float mts = mt == -INFINITY ? -INFINITY : (mt - kBias) * cr;  // half-tile max of the log2-domain score
+      // combine the two halves' maxima
+      xm[(st * 2 + h) * BM + i] = mts;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bar[X_MX + st]);
+      if (!warp_wait(&bar[X_MX + st], (j >> 1) & 1, abort_flag, p.status, 75)) { ok = false; break; }
+      const float m_tile = fmaxf(mts, xm[(st * 2 + (h ^ 1)) * BM + i]);
+      const float m_new = fmaxf(m_run, m_tile);
       const bool grow = m_new > m_run + 8.0f;
       const float m_use = grow ? m_new : m_run;
       const float alpha = grow ? ex2(m_run - m_use) : 1.0f;
       const bool any_grow = __any_sync(0xffffffffu, grow) && j > 0;
-      if (j > 0) {
-        // P'_s and O_s are free once P V of tile j-1 has completed.
-        if (!warp_wait(&bar[X_PVD + s], (j - 1) & 1, abort_flag, p.status, 72)) { ok = false; break; }
-        if (any_grow) {
-          tc_fence_after();
+      if (any_grow) {
+        // O is free once P V of tile j-1 has completed; each half rescales its own O columns.
+        if (!warp_wait(&bar[X_PVD], (j - 1) & 1, abort_flag, p.status, 72)) { ok = false; break; }
+        tc_fence_after();
 #pragma unroll
-          for (int c = 0; c < D / 16; ++c) {
-            uint32_t r[16];
-            tmem_ld16(tO + loff + c * 16, r);
-            tmem_ld_wait();
+        for (int c = 0; c < D / 64; ++c) {
+          uint32_t r[32];
+          tmem_ld32(tO + loff + h * (D / 2) + c * 32, r);
+          tmem_ld_wait();
 #pragma unroll
-            for (int k = 0; k < 16; ++k) r[k] = __float_as_uint(__uint_as_float(r[k]) * alpha);
-            tmem_st16(tO + loff + c * 16, r);
+          for (int k = 0; k < 32; k += 2) {
+            float a0 = __uint_as_float(r[k]), a1 = __uint_as_float(r[k + 1]);
+            fmul2(a0, a1, alpha, alpha);
+            r[k] = __float_as_uint(a0);
+            r[k + 1] = __float_as_uint(a1);
           }
-          tmem_st_wait();
+          tmem_st32(tO + loff + h * (D / 2) + c * 32, r);
         }
+        tmem_st_wait();
       }
       l_run *= alpha;
       m_run = m_use;
-      // exp2 argument: t * cr - (bias * cr + m)   (the bias term is 0 for E4M3)
-      const float nb = m_use == -INFINITY ? 0.0f : -(kBias * cr + m_use);
-      float vt = 1.0f, nbv = nb;
-      if (SC == SC_TILE) {
-        vt = vcf[0];
-        nbv = vt > 0.0f ? nb + __log2f(vt) : -INFINITY;  // fold s_v / v_ref into the exponent
-      }
-      // exp2 of all 128 scores first (independent, keeps the XU pipe fed), then
-      // the row sum, then V fold + fp16 packing + stores.
+      // exp2 argument: t * cr - (bias * cr + m) + log2(r_t / v_ref)   (bias 0 for E4M3; factor 1 for INT8)
+      const float nb = (m_use == -INFINITY ? 0.0f : -(kBias * cr + m_use)) + flog;
 #pragma unroll
-      for (int k = 0; k < BN; ++k) t[k] = ex2(fmaf(t[k], cr, SC == SC_COL ? nb : nbv));
+      for (int k = 0; k < HN; k += 2) {
+        ffma2(t[k], t[k + 1], cr, cr, nb, nb);
+        t[k] = ex2(t[k]);
+        t[k + 1] = ex2(t[k + 1]);
+      }
       float ls[8];
 #pragma unroll
       for (int e = 0; e < 8; ++e) ls[e] = t[e];
 #pragma unroll
-      for (int k = 8; k < BN; ++k) ls[k & 7] += t[k];
-      // P' (fp16 pairs) into the first 64 TMEM columns of S_s: two 32-column stores.
-#pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        uint32_t h[32];
+      for (int k = 8; k < HN; k += 2) fadd2(ls[k & 7], ls[(k & 7) + 1], t[k], t[k + 1]);
+      // P' = fp16(p) over this half's first 32 S columns
+      {
+        uint32_t hp[32];
 #pragma unroll
         for (int e = 0; e < 32; ++e) {
-          const int k = half * 64 + 2 * e;
-          float a = t[k], c2 = t[k + 1];
-          if (SC == SC_COL) {
-            a *= vcf[k];
-            c2 *= vcf[k + 1];
-          }
-          const __half2 hv = __floats2half2_rn(a, c2);
-          h[e] = *reinterpret_cast<const uint32_t*>(&hv);
+          const __half2 hv = __floats2half2_rn(t[2 * e], t[2 * e + 1]);
+          hp[e] = *reinterpret_cast<const uint32_t*>(&hv);
         }
-        tmem_st32(tS + loff + half * 32, h);
+        tmem_st32(tS + loff, hp);
       }
       tmem_st_wait();
-      float lsum = ((ls[0] + ls[1]) + (ls[2] + ls[3])) + ((ls[4] + ls[5]) + (ls[6] + ls[7]));
-      if (SC == SC_TILE) lsum = vt > 0.0f ? lsum / vt : 0.0f;
-      l_run += lsum;
+      l_run += (((ls[0] + ls[1]) + (ls[2] + ls[3])) + ((ls[4] + ls[5]) + (ls[6] + ls[7]))) * finv;
       tc_fence_before();
       __syncwarp();
       if (lane == 0) {
-        mbar_arrive(&bar[X_PF + s]);
-        if (SC != SC_HEAD) mbar_arrive(&bar[X_SCE + 2 * s + st]);
+        mbar_arrive(&bar[X_PF + st]);
+        if (SC != SC_HEAD) mbar_arrive(&bar[X_SCE + sst]);
       }
     }
     // ---------------------------------------------------------- epilogue
     if (ok && n > 0) {
-      ok = warp_wait(&bar[X_PVD + s], (n - 1) & 1, abort_flag, p.status, 73);
+      ok = warp_wait(&bar[X_PVD], (n - 1) & 1, abort_flag, p.status, 73);
       tc_fence_after();
     }
+    // row sum = the two halves' partial sums
+    xl[h * BM + i] = l_run;
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&bar[X_LX]);
+    const bool lx = warp_wait(&bar[X_LX], 0, abort_flag, p.status, 76);
+    const float l_tot = lx ? xl[i] + xl[BM + i] : 0.0f;
     if (q0 < p.Sq) {
-      const float ofac = l_run > 0.0f ? vref / l_run : 0.0f;
+      const float ofac = l_tot > 0.0f ? vref / l_tot : 0.0f;
       __nv_bfloat16* orow = nullptr;
       if (row_ok) {
         const long long ridx = p.layout == FA_LAYOUT_BNSD ? ((long long)qbh * p.Sq + row)
                                                           : (((long long)b * p.Sq + row) * p.Hq + hq);
-        orow = p.out + ridx * D;
+        orow = p.out + ridx * D + h * (D / 2);
       }
 #pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
+      for (int c = 0; c < D / 64; ++c) {
         uint32_t r[32];
         if (ok && n > 0) {
-          tmem_ld32(tO + loff + c * 32, r);
+          tmem_ld32(tO + loff + h * (D / 2) + c * 32, r);
           tmem_ld_wait();
         } else {
 #pragma unroll
@@ -536,9 +487,9 @@ __global__ void __launch_bounds__(NT, 1)
           }
         }
       }
-      if (row_ok && p.lse)
+      if (h == 0 && row_ok && p.lse)
         p.lse[(long long)qbh * p.Sq + row] =
-            l_run > 0.0f ? (m_run + __log2f(l_run)) * 0.69314718055994530942f : -INFINITY;
+            l_tot > 0.0f ? (m_run + __log2f(l_tot)) * 0.69314718055994530942f : -INFINITY;
     }
   }
 
@@ -550,14 +501,109 @@ __global__ void __launch_bounds__(NT, 1)
   }
 }
 
+// ---- V pre-pass: one CTA per (128-token tile, b * Hkv + h).
+// E4M3: r_t = max s_v over the tile's tokens (1 if all are 0), V' = fp16(code * (s_v / r_t)), |V'| <= 448.
+// INT8: V' = fp16(code) exactly (the per-head scale stays outside).
+template <int KIND, int D>
+__global__ void __launch_bounds__(256) vprep_kernel(const uint8_t* __restrict__ codes, const float* __restrict__ vs,
+                                                    int v_blk, int v_nblk, int H, int S, int layout,
+                                                    __half* __restrict__ vh, float* __restrict__ fv, int ntiles) {
+  constexpr int CPT = D / 32;  // 16-code chunks per thread: each thread owns half a token row
+  const int t = blockIdx.x, bh = blockIdx.y;
+  const int b = bh / H, h = bh % H;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int tok0 = t * BN;
+  const int tok = tok0 + warp * 16 + (lane >> 1);
+  const bool live = tok < S;  // rows past S stay unwritten: the attention's TMA box reads them as zero
+  const long long src_row = layout == FA_LAYOUT_BNSD ? ((long long)bh * S + tok) : (((long long)b * S + tok) * H + h);
+  const uint8_t* src = codes + src_row * D + (lane & 1) * (D / 2);
+  uint4 raw[CPT];
+#pragma unroll
+  for (int c = 0; c < CPT; ++c) raw[c] = live ? __ldg(reinterpret_cast<const uint4*>(src) + c) : make_uint4(0, 0, 0, 0);
+  float f = 1.0f;
+  if (KIND == K_E4M3) {
+    // every warp reduces the tile's 128 scales itself (no block barrier)
+    const float* vsh = vs + (long long)bh * v_nblk;
+    float m = 0.0f;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const int tt = tok0 + lane * 4 + q;
+      if (tt < S) m = fmaxf(m, __ldg(vsh + tt / v_blk));
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+    const float r = m > 0.0f ? m : 1.0f;
+    f = live ? __ldg(vsh + tok / v_blk) / r : 0.0f;
+    if (threadIdx.x == 0) fv[(long long)bh * ntiles + t] = r;
+  }
+  if (!live) return;
+  uint4* dst = reinterpret_cast<uint4*>(vh + ((long long)bh * S + tok) * D + (lane & 1) * (D / 2));
+#pragma unroll
+  for (int c = 0; c < CPT; ++c) {
+    const uint32_t w[4] = {raw[c].x, raw[c].y, raw[c].z, raw[c].w};
+    uint32_t o[8];
+    if (KIND == K_E4M3) {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const uint32_t h2 = e4m3x2_to_h2((uint16_t)(w[i >> 1] >> ((i & 1) * 16)));
+        const float2 x = __half22float2(*reinterpret_cast<const __half2*>(&h2));
+        const __half2 y = __floats2half2_rn(x.x * f, x.y * f);
+        o[i] = *reinterpret_cast<const uint32_t*>(&y);
+      }
+    } else {
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const uint32_t ub = w[i] ^ 0x80808080u;
+        o[2 * i] = s8x2_to_h2(ub, 0x4140);
+        o[2 * i + 1] = s8x2_to_h2(ub, 0x4342);
+      }
+    }
+    dst[2 * c] = make_uint4(o[0], o[1], o[2], o[3]);
+    dst[2 * c + 1] = make_uint4(o[4], o[5], o[6], o[7]);
+  }
+}
+
+// Tensor map over V' [B][H][S][D] fp16: 64-column x 128-token boxes, 128-byte swizzle.
+cudaError_t make_vh_map(CUtensorMap* map, const void* base, int B, int H, int S, int D) {
+  EncodeTiledFn enc = encode_tiled_fn();
+  if (!enc) return cudaErrorNotSupported;
+  const cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)S, (cuuint64_t)H, (cuuint64_t)B};
+  const cuuint64_t strides[3] = {(cuuint64_t)D * 2, (cuuint64_t)S * D * 2, (cuuint64_t)H * S * D * 2};
+  const cuuint32_t box[4] = {64, (cuuint32_t)BN, 1, 1};
+  const cuuint32_t es[4] = {1, 1, 1, 1};
+  const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 4, const_cast<void*>(base), dims, strides, box, es,
+                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+struct Prefill2Ws {
+  __half* vh;
+  float* fv;
+};
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+Prefill2Ws carve_ws(void* ws, int B, int Hkv, int Sk, int D) {
+  Prefill2Ws w;
+  w.vh = static_cast<__half*>(ws);
+  w.fv = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + align256((size_t)B * Hkv * Sk * D * 2));
+  return w;
+}
+
 template <int KIND, int D, int SC>
-cudaError_t launch2(const AttnArgs& a, const P2& prm, cudaStream_t s) {
+cudaError_t launch2(const AttnArgs& a, const P2& prm, const Prefill2Ws& w, cudaStream_t s) {
   using L = L2<D>;
   CUtensorMap mq, mk, mv;
   cudaError_t e;
   if ((e = make_code_map(&mq, a.q->codes, a.q->B, a.q->H, a.q->S, D, a.q->layout, BM)) != cudaSuccess) return e;
   if ((e = make_code_map(&mk, a.k->codes, a.k->B, a.k->H, a.k->S, D, a.k->layout, BN)) != cudaSuccess) return e;
-  if ((e = make_code_map(&mv, a.v->codes, a.v->B, a.v->H, a.v->S, D, a.v->layout, BN)) != cudaSuccess) return e;
+  if ((e = make_vh_map(&mv, w.vh, a.v->B, a.v->H, a.v->S, D)) != cudaSuccess) return e;
+  const dim3 pgrid((unsigned)prm.ntiles_k, (unsigned)(a.v->B * a.v->H));
+  if (pgrid.y > 65535u) return cudaErrorInvalidValue;
+  vprep_kernel<KIND, D><<<pgrid, 256, 0, s>>>(static_cast<const uint8_t*>(a.v->codes), prm.vs, prm.v_blk,
+                                               prm.v_nblk, a.v->H, a.v->S, a.v->layout, w.vh, w.fv, prm.ntiles_k);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
   auto kern = attn2_kernel<KIND, D, SC>;
   static bool attr_set = false;
   if (!attr_set) {
@@ -565,22 +611,18 @@ cudaError_t launch2(const AttnArgs& a, const P2& prm, cudaStream_t s) {
       return e;
     attr_set = true;
   }
-  long long grid;
-  if (prm.pair_heads)
-    grid = (long long)prm.n_qtiles * prm.B * (prm.Hq / 2);
-  else
-    grid = (long long)((prm.n_qtiles + 1) / 2) * prm.B * prm.Hq;
+  const long long grid = (long long)prm.n_qtiles * prm.B * prm.Hq;
   if (grid > 0x7FFFFFFFLL) return cudaErrorInvalidValue;
   kern<<<(unsigned)grid, NT, L::ALLOC, s>>>(mq, mk, mv, prm);
   return cudaGetLastError();
 }
 
 template <int KIND, int D>
-cudaError_t launch2_sc(const AttnArgs& a, const P2& prm, int sc, cudaStream_t s) {
+cudaError_t launch2_sc(const AttnArgs& a, const P2& prm, const Prefill2Ws& w, int sc, cudaStream_t s) {
   switch (sc) {
-    case SC_HEAD: return launch2<KIND, D, SC_HEAD>(a, prm, s);
-    case SC_COL: return launch2<KIND, D, SC_COL>(a, prm, s);
-    default: return launch2<KIND, D, SC_TILE>(a, prm, s);
+    case SC_HEAD: return launch2<KIND, D, SC_HEAD>(a, prm, w, s);
+    case SC_COL: return launch2<KIND, D, SC_COL>(a, prm, w, s);
+    default: return launch2<KIND, D, SC_TILE>(a, prm, w, s);
   }
 }
 
@@ -595,8 +637,13 @@ void scale_desc2(const fa_qtensor* t, int& blk, int& nblk) {
 
 }  // namespace
 
-// Prefill attention for E4M3 and INT8 operands (two query tiles per CTA).
-cudaError_t launch_attention_prefill2(const AttnArgs& a, cudaStream_t s) {
+// Prefill attention for E4M3 and INT8 operands.
+size_t prefill2_workspace_bytes(int B, int Hkv, int Sk, int D) {
+  const size_t ntiles = ((size_t)Sk + BN - 1) / BN;
+  return align256((size_t)B * Hkv * Sk * D * 2) + align256((size_t)B * Hkv * ntiles * 4);
+}
+
+cudaError_t launch_attention_prefill2(const AttnArgs& a, void* ws, cudaStream_t s) {
   const fa_qtensor* q = a.q;
   const fa_qtensor* k = a.k;
   P2 prm = {};
@@ -614,16 +661,18 @@ cudaError_t launch_attention_prefill2(const AttnArgs& a, cudaStream_t s) {
   prm.lse = a.lse;
   prm.status = a.status;
   prm.n_qtiles = (q->S + BM - 1) / BM;
-  prm.pair_heads = (prm.group % 2 == 0) ? 1 : 0;
+  prm.ntiles_k = (k->S + BN - 1) / BN;
+  const Prefill2Ws w = carve_ws(ws, k->B, k->H, k->S, q->D);
+  prm.fv = w.fv;
   int sc = SC_HEAD;
   if (q->mode == FA_MODE_FP8_PER_TOKEN) sc = SC_COL;
   if (q->mode == FA_MODE_FP8_BLOCK) sc = (k->block_tokens % BN == 0) ? SC_TILE : SC_COL;
   switch (q->mode) {
     case FA_MODE_FP8_PER_TOKEN:
     case FA_MODE_FP8_BLOCK:
-      return q->D == 128 ? launch2_sc<K_E4M3, 128>(a, prm, sc, s) : launch2_sc<K_E4M3, 64>(a, prm, sc, s);
+      return q->D == 128 ? launch2_sc<K_E4M3, 128>(a, prm, w, sc, s) : launch2_sc<K_E4M3, 64>(a, prm, w, sc, s);
     case FA_MODE_INT8_PER_HEAD:
-      return q->D == 128 ? launch2_sc<K_S8, 128>(a, prm, SC_HEAD, s) : launch2_sc<K_S8, 64>(a, prm, SC_HEAD, s);
+      return q->D == 128 ? launch2<K_S8, 128, SC_HEAD>(a, prm, w, s) : launch2<K_S8, 64, SC_HEAD>(a, prm, w, s);
     default:
       return cudaErrorNotSupported;
   }

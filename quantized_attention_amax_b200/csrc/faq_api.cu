@@ -228,12 +228,23 @@ fa_status fa_rotate_quantize(const fa_tensor* q, const fa_tensor* k, const fa_te
   return from_cuda(e);
 }
 
-size_t fa_attention_workspace_size(const fa_qtensor* q, const fa_qtensor* k, int num_splits) {
-  if (!q || !k || q->S != 1 || q->mode != FA_MODE_INT8_PER_HEAD || q->D != 128 || k->H < 1 || q->H % k->H) return 0;
+static bool is_decode(const fa_qtensor* q, const fa_qtensor* k) {
+  if (q->S != 1 || q->mode != FA_MODE_INT8_PER_HEAD || q->D != 128) return false;
   const int group = q->H / k->H;
-  if (!(group == 1 || group == 2 || group == 4 || group == 8 || group == 16)) return 0;
-  const int splits = num_splits > 0 ? num_splits : decode_auto_splits(k->B, k->H, k->S);
-  return decode_workspace_bytes(q->B, q->H, q->D, splits);
+  return group == 1 || group == 2 || group == 4 || group == 8 || group == 16;
+}
+
+size_t fa_attention_workspace_size(const fa_qtensor* q, const fa_qtensor* k, int num_splits) {
+  if (!q || !k || k->H < 1 || q->H % k->H || num_splits < 0) return 0;
+  if (is_decode(q, k)) {
+    const int splits = num_splits > 0 ? num_splits : decode_auto_splits(k->B, k->H, k->S);
+    return decode_workspace_bytes(q->B, q->H, q->D, splits);
+  }
+  if (q->mode == FA_MODE_INT8_PER_HEAD || q->mode == FA_MODE_FP8_PER_TOKEN || q->mode == FA_MODE_FP8_BLOCK) {
+    if (k->B < 0 || k->S < 0 || (q->D != 64 && q->D != 128)) return 0;
+    return prefill2_workspace_bytes(k->B, k->H, k->S, q->D);
+  }
+  return 0;
 }
 
 fa_status fa_attention_quant(const fa_qtensor* q, const fa_qtensor* k, const fa_qtensor* v, int causal,
@@ -255,13 +266,12 @@ fa_status fa_attention_quant(const fa_qtensor* q, const fa_qtensor* k, const fa_
   if (qrows == 0) return FA_OK;
   if (!out || !aligned16(out)) return FA_ERR_INVALID_ARG;
   if (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)) return FA_ERR_INVALID_ARG;
-  const int group = q->H / k->H;
-  const bool decode = q->S == 1 && q->mode == FA_MODE_INT8_PER_HEAD && q->D == 128 &&
-                      (group == 1 || group == 2 || group == 4 || group == 8 || group == 16);
+  const bool decode = is_decode(q, k);
   const int splits = decode ? (num_splits > 0 ? num_splits : decode_auto_splits(k->B, k->H, k->S)) : 0;
-  if (decode && k->S > 0) {
-    const size_t need = decode_workspace_bytes(q->B, q->H, q->D, splits);
-    if (!workspace || ws_bytes < need || !aligned16(workspace)) return FA_ERR_WORKSPACE;
+  if (k->S > 0 && q->mode != FA_MODE_MXFP4_PER_BLOCK) {
+    const size_t need = decode ? decode_workspace_bytes(q->B, q->H, q->D, splits)
+                               : prefill2_workspace_bytes(k->B, k->H, k->S, q->D);
+    if (!workspace || ws_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255u)) return FA_ERR_WORKSPACE;
   }
   cudaStream_t cs = reinterpret_cast<cudaStream_t>(s);
   if (k->S == 0) return from_cuda(launch_fill_empty_rows(out, lse, qrows, q->D, cs));
@@ -274,7 +284,7 @@ fa_status fa_attention_quant(const fa_qtensor* q, const fa_qtensor* k, const fa_
   else if (q->mode == FA_MODE_MXFP4_PER_BLOCK)
     e = launch_attention_prefill(a, cs);
   else
-    e = launch_attention_prefill2(a, cs);
+    e = launch_attention_prefill2(a, workspace, cs);
   if (e == cudaErrorNotSupported) return FA_ERR_UNSUPPORTED;
   return from_cuda(e);
 }

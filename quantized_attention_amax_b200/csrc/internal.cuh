@@ -61,7 +61,9 @@ struct AttnArgs {
   int* status;
 };
 cudaError_t launch_attention_prefill(const AttnArgs& a, cudaStream_t s);
-cudaError_t launch_attention_prefill2(const AttnArgs& a, cudaStream_t s);
+// FP8 / INT8 prefill: V' pre-pass + attention; `ws` holds prefill2_workspace_bytes().
+size_t prefill2_workspace_bytes(int B, int Hkv, int Sk, int D);
+cudaError_t launch_attention_prefill2(const AttnArgs& a, void* ws, cudaStream_t s);
 
 size_t decode_workspace_bytes(int B, int Hq, int D, int splits);
 int decode_auto_splits(int B, int Hkv, int Sk);

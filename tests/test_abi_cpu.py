@@ -130,6 +130,18 @@ def test_attention_validation_before_launch(N):
     assert L.fa_attention_quant(by(qd), by(kd), by(kd), 0, 0.0, 0x60000, None, 0, 0x70000, need - 16,
                                 None) == 7
     assert L.fa_attention_quant(by(qd), by(kd), by(kd), 0, 0.0, 0x60000, None, -1, None, 0, None) == 1
-    # prefill needs no workspace
+    # FP8 / INT8 prefill: fp16 V' plus one factor per 128-key tile, each 256-byte aligned
     qp = _q(N, 1, B=2, H=4, S=100, D=128)
-    assert L.fa_attention_workspace_size(by(qp), by(kd), 0) == 0
+    need_p = L.fa_attention_workspace_size(by(qp), by(kd), 0)
+    vh = 2 * 2 * 1000 * 128 * 2
+    fv = 2 * 2 * ((1000 + 127) // 128) * 4
+    assert need_p == ((vh + 255) // 256) * 256 + ((fv + 255) // 256) * 256
+    assert L.fa_attention_quant(by(qp), by(kd), by(kd), 0, 0.0, 0x60000, None, 0, None, 0, None) == 7
+    assert L.fa_attention_quant(by(qp), by(kd), by(kd), 0, 0.0, 0x60000, None, 0, 0x70000, need_p - 256,
+                                None) == 7
+    assert L.fa_attention_quant(by(qp), by(kd), by(kd), 0, 0.0, 0x60000, None, 0, 0x70010, need_p,
+                                None) == 7  # workspace not 256-byte aligned
+    # MXFP4 prefill needs none
+    qm = _q(N, 3, B=2, H=4, S=100, D=128)
+    km = _q(N, 3, B=2, H=2, S=1000, D=128)
+    assert L.fa_attention_workspace_size(by(qm), by(km), 0) == 0
