@@ -379,18 +379,47 @@ __global__ void __launch_bounds__(NT, 1)
       for (int k = 8; k < HN; ++k) mx[k & 7] = fmaxf(mx[k & 7], t[k]);
       const float mt = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])), fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
       const float mts = mt == -INFINITY ? -INFINITY : (mt - kBias) * cr;  // half-tile max of the log2-domain score
-      // combine the two halves' maxima
+      // publish this half's maximum; the partner's is read once it is needed
       xm[(st * 2 + h) * BM + i] = mts;
       __syncwarp();
       if (lane == 0) mbar_arrive(&bar[X_MX + st]);
-      if (!warp_wait(&bar[X_MX + st], (j >> 1) & 1, abort_flag, p.status, 75)) { ok = false; break; }
-      const float m_tile = fmaxf(mts, xm[(st * 2 + (h ^ 1)) * BM + i]);
-      const float m_new = fmaxf(m_run, m_tile);
-      const bool grow = m_new > m_run + 8.0f;
-      const float m_use = grow ? m_new : m_run;
-      const float alpha = grow ? ex2(m_run - m_use) : 1.0f;
-      const bool any_grow = __any_sync(0xffffffffu, grow) && j > 0;
-      if (any_grow) {
+      const float* xpart = xm + (st * 2 + (h ^ 1)) * BM + i;
+      // The running max moves only when a tile's max exceeds it by more than 2^8, so the
+      // exponentials normally use m_run before the partner's half is known.  A warp where
+      // this half alone forces a move (always on a row's first visible tile) takes both
+      // halves' maxima first.
+      float m_use = m_run;
+      bool have_part = false;
+      if (__any_sync(0xffffffffu, mts > m_run + 8.0f)) {
+        if (!warp_wait(&bar[X_MX + st], (j >> 1) & 1, abort_flag, p.status, 75)) { ok = false; break; }
+        have_part = true;
+        const float m_new = fmaxf(m_run, fmaxf(mts, *xpart));
+        if (m_new > m_run + 8.0f) m_use = m_new;
+      }
+      // exp2 argument: t * cr - (bias * cr + m) + log2(r_t / v_ref)   (bias 0 for E4M3; factor 1 for INT8)
+      const float nb = (m_use == -INFINITY ? 0.0f : -(kBias * cr + m_use)) + flog;
+#pragma unroll
+      for (int k = 0; k < HN; k += 2) {
+        ffma2(t[k], t[k + 1], cr, cr, nb, nb);
+        if (k & 2) {
+          ex2_poly2(t[k], t[k + 1]);  // every other pair on the FMA pipe
+        } else {
+          t[k] = ex2(t[k]);
+          t[k + 1] = ex2(t[k + 1]);
+        }
+      }
+      if (!have_part && !warp_wait(&bar[X_MX + st], (j >> 1) & 1, abort_flag, p.status, 75)) { ok = false; break; }
+      // the decision both halves take from the same three numbers
+      const float m_new = fmaxf(m_run, fmaxf(mts, *xpart));
+      const float m_fin = m_new > m_run + 8.0f ? m_new : m_run;
+      if (__any_sync(0xffffffffu, m_fin != m_use)) {
+        // the partner's half moved the max: rescale this half's p (each <= 2^8 here)
+        const float c = m_fin != m_use ? ex2(m_use - m_fin) : 1.0f;
+#pragma unroll
+        for (int k = 0; k < HN; k += 2) fmul2(t[k], t[k + 1], c, c);
+      }
+      const float alpha = m_fin != m_run ? ex2(m_run - m_fin) : 1.0f;
+      if (__any_sync(0xffffffffu, m_fin != m_run) && j > 0) {
         // O is free once P V of tile j-1 has completed; each half rescales its own O columns.
         if (!warp_wait(&bar[X_PVD], (j - 1) & 1, abort_flag, p.status, 72)) { ok = false; break; }
         tc_fence_after();
@@ -411,15 +440,7 @@ __global__ void __launch_bounds__(NT, 1)
         tmem_st_wait();
       }
       l_run *= alpha;
-      m_run = m_use;
-      // exp2 argument: t * cr - (bias * cr + m) + log2(r_t / v_ref)   (bias 0 for E4M3; factor 1 for INT8)
-      const float nb = (m_use == -INFINITY ? 0.0f : -(kBias * cr + m_use)) + flog;
-#pragma unroll
-      for (int k = 0; k < HN; k += 2) {
-        ffma2(t[k], t[k + 1], cr, cr, nb, nb);
-        t[k] = ex2(t[k]);
-        t[k + 1] = ex2(t[k + 1]);
-      }
+      m_run = m_fin;
       float ls[8];
 #pragma unroll
       for (int e = 0; e < 8; ++e) ls[e] = t[e];

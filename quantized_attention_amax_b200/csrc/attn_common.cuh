@@ -36,6 +36,31 @@ __device__ __forceinline__ void fadd2(float& a0, float& a1, float b0, float b1) 
       : "f"(b0), "f"(b1));
 }
 
+// 2^x for a pair on the FMA pipe (takes load off the MUFU unit, which runs ex2
+// at a quarter of the FMA rate): x = n + f with n = rint(x), f in [-0.5, 0.5];
+// 2^f from a cubic fitted here for least maximum relative error on that interval
+// (Lawson's reweighted least squares), 7.5e-5 relative error in fp32 -- below
+// half an fp16 ulp, the precision P' is stored in; 2^n enters through the
+// exponent field.  x is clamped at -126: p(f) >= 2^-0.5 has a biased exponent of
+// at least 126, so n >= -126 never borrows past the exponent field (the result
+// for x <= -126 is a denormal, read as 0 downstream).
+__device__ __forceinline__ void ex2_poly2(float& a, float& b) {
+  constexpr float kRound = 12582912.0f;  // 1.5 * 2^23: x + kRound holds rint(x) in its low mantissa bits
+  float x0 = fmaxf(a, -126.0f), x1 = fmaxf(b, -126.0f);
+  float j0 = x0, j1 = x1;
+  fadd2(j0, j1, kRound, kRound);
+  float n0 = j0, n1 = j1;
+  fadd2(n0, n1, -kRound, -kRound);
+  float f0 = x0, f1 = x1;
+  fadd2(f0, f1, -n0, -n1);
+  float p0 = 5.517132208e-02f, p1 = 5.517132208e-02f;
+  ffma2(p0, p1, f0, f1, 2.426105440e-01f, 2.426105440e-01f);
+  ffma2(p0, p1, f0, f1, 6.932609677e-01f, 6.932609677e-01f);
+  ffma2(p0, p1, f0, f1, 9.999281168e-01f, 9.999281168e-01f);
+  a = __int_as_float(__float_as_int(p0) + (__float_as_int(j0) << 23));
+  b = __int_as_float(__float_as_int(p1) + (__float_as_int(j1) << 23));
+}
+
 // Every lane waits; the warp proceeds only if all lanes saw the phase complete.
 __device__ __forceinline__ bool warp_wait(uint64_t* b, uint32_t parity, volatile int* abort_flag, int* status,
                                           int where) {
