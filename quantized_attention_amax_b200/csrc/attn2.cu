@@ -42,8 +42,18 @@ using namespace attn;
 
 constexpr int BM = 128;
 constexpr int BN = 128;
-constexpr int HN = BN / 2;  // keys per softmax half
-constexpr int NT = 384;     // 12 warps
+// NSW softmax warpgroups share each S tile, NSW * 128 + 128 threads.
+template <int NSW>
+struct Cfg {
+  static constexpr int NT = 128 * (NSW + 1);
+  static constexpr int HN = BN / NSW;  // keys per softmax thread and tile
+  // setmaxnreg split of the launch's registers (65536 / NT, rounded down to 8, per thread):
+  // warpgroup 0 shrinks to R0, the softmax warpgroups grow to RS; 128 * R0 + NSW * 128 * RS
+  // stays within NT * (launch registers).
+  static constexpr int R0 = NSW == 2 ? 88 : 56;
+  static constexpr int RS = NSW == 2 ? 208 : 104;
+  static_assert(128 * R0 + NSW * 128 * RS <= NT * ((65536 / NT) & ~7), "register split exceeds the launch");
+};
 constexpr int NKS = 3;      // K code stages
 constexpr int NVS = 2;      // V' stages
 constexpr int NSC = 4;      // scale ring stages
@@ -57,7 +67,8 @@ struct P2 {
   const float* qs;
   const float* ks;
   const float* vs;
-  const float* fv;  // [B, Hkv, ntiles] V' tile factors r_t (FP8 operands)
+  const float* ksp;   // [B, Hkv, ntiles * 128] per-key K scales, zero past Sk (FP8 operands)
+  const float4* fvr;  // [B, Hkv, ntiles] V' tile factor records {r_t, 0, 0, 0} (FP8 operands)
   int q_blk, k_blk, v_blk, q_nblk, k_nblk, v_nblk;
   int ntiles_k;
   __nv_bfloat16* out;
@@ -72,40 +83,48 @@ struct L2 {
   static constexpr uint32_t K = Q + BM * D;            // NKS stages
   static constexpr uint32_t VH = K + NKS * BN * D;     // NVS stages of fp16 V'
   static constexpr uint32_t SC = VH + NVS * BN * D * 2;  // NSC stages x ([128] k scale, V' factor log2, its inverse)
-  static constexpr uint32_t XM = SC + NSC * 2 * BN * 4;  // 2 stages x 2 halves x [128] tile row max
-  static constexpr uint32_t XL = XM + 2 * 2 * BM * 4;  // 2 halves x [128] row sum
-  static constexpr uint32_t MISC = XL + 2 * BM * 4;
+  static constexpr uint32_t XM = SC + NSC * 2 * BN * 4;  // 2 stages x 4 key groups x [128] tile row max
+  static constexpr uint32_t XL = XM + 2 * 4 * BM * 4;    // 4 key groups x [128] row sum
+  static constexpr uint32_t MISC = XL + 4 * BM * 4;
   static constexpr uint32_t BAR = MISC + 64;
   static constexpr uint32_t TOTAL = BAR + 512;
   static constexpr uint32_t ALLOC = TOTAL + 1024;
+  static_assert(ALLOC <= 227 * 1024, "shared memory per CTA");
 };
 
+// mbarrier slots, laid out from the ring depths
 enum {
   X_Q = 0,
-  X_KF = 1,    // [NKS]
-  X_KE = 4,    // [NKS]
-  X_VF = 7,    // [NVS] V' stage full
-  X_VE = 9,    // [NVS] V' stage empty
-  X_SF = 15,   // [2] S buffer full
-  X_PF = 17,   // [2] P' buffer full
-  X_PVD = 19,  // P V done
-  X_SCF = 20,  // [NSC] scale ring stage full
-  X_SCE = 24,  // [NSC] scale ring stage empty
-  X_MX = 28,   // [2] row-max exchange
-  X_LX = 30,   // row-sum exchange
-  X_FIN = 31,
-  X_COUNT = 32
+  X_KF = 1,              // [NKS] K stage full
+  X_KE = X_KF + NKS,     // [NKS] K stage empty
+  X_VF = X_KE + NKS,     // [NVS] V' stage full
+  X_VE = X_VF + NVS,     // [NVS] V' stage empty
+  X_SF = X_VE + NVS,     // [2] S buffer full
+  X_PF = X_SF + 2,       // [2] P' buffer full
+  X_PVD = X_PF + 2,      // P V done
+  X_SCF = X_PVD + 1,     // [NSC] scale ring stage full
+  X_SCE = X_SCF + NSC,   // [NSC] scale ring stage empty
+  X_MX = X_SCE + NSC,    // [2] row-max exchange
+  X_LX = X_MX + 2,       // row-sum exchange
+  X_FIN = X_LX + 1,
+  X_COUNT = X_FIN + 1
 };
+static_assert(X_COUNT * 8 + 8 <= 512, "barrier block overflows its region");
 
-__device__ __forceinline__ void setmaxnreg_inc208() { asm volatile("setmaxnreg.inc.sync.aligned.u32 208;"); }
-__device__ __forceinline__ void setmaxnreg_dec88() { asm volatile("setmaxnreg.dec.sync.aligned.u32 88;"); }
+template <int R>
+__device__ __forceinline__ void setmaxnreg_inc() { asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(R)); }
+template <int R>
+__device__ __forceinline__ void setmaxnreg_dec() { asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(R)); }
 
-template <int KIND, int D, int SC>
-__global__ void __launch_bounds__(NT, 1)
+template <int KIND, int D, int SC, int NSW>
+__global__ void __launch_bounds__(Cfg<NSW>::NT, 1)
     attn2_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
                  const __grid_constant__ CUtensorMap tmv, const P2 p) {
   static_assert(KIND == K_E4M3 || SC == SC_HEAD, "INT8 operands carry one scale per head");
   using L = L2<D>;
+  constexpr int HN = Cfg<NSW>::HN;
+  constexpr int NSWW = 4 * NSW;   // softmax warps
+  constexpr int DC = D / NSW;     // O columns per softmax thread
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bar = reinterpret_cast<uint64_t*>(smem + L::BAR);
@@ -139,19 +158,21 @@ __global__ void __launch_bounds__(NT, 1)
       mbar_init(&bar[X_KF + i], 1);
       mbar_init(&bar[X_KE + i], 1);
     }
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < NVS; ++i) {
       mbar_init(&bar[X_VF + i], 1);
       mbar_init(&bar[X_VE + i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
       mbar_init(&bar[X_SF + i], 1);
-      mbar_init(&bar[X_PF + i], 8);
-      mbar_init(&bar[X_MX + i], 8);
+      mbar_init(&bar[X_PF + i], NSWW);
+      mbar_init(&bar[X_MX + i], NSWW);
     }
     for (int i = 0; i < NSC; ++i) {
       mbar_init(&bar[X_SCF + i], 1);
-      mbar_init(&bar[X_SCE + i], 8);  // the softmax warps
+      mbar_init(&bar[X_SCE + i], NSWW);  // the softmax warps
     }
     mbar_init(&bar[X_PVD], 1);
-    mbar_init(&bar[X_LX], 8);
+    mbar_init(&bar[X_LX], NSWW);
     mbar_init(&bar[X_FIN], 1);
     *abort_flag = 0;
     fence_barrier_init();
@@ -166,7 +187,7 @@ __global__ void __launch_bounds__(NT, 1)
   const uint32_t tO = tbase + 256;
 
   if (warp < 4) {
-    setmaxnreg_dec88();
+    setmaxnreg_dec<Cfg<NSW>::R0>();
     const bool bnsd = p.layout == FA_LAYOUT_BNSD;
     if (warp == 0) {
       // ------------------------------------------------------ Q and K loads
@@ -209,36 +230,28 @@ __global__ void __launch_bounds__(NT, 1)
       __syncwarp();
     } else if (warp == 2) {
       // ------------------------------------------------------- scale ring
+      // Per tile, the pre-pass's 128 per-key K scales and the V' factor record land in a
+      // ring stage by two bulk copies (512 + 16 bytes) that complete on the stage's barrier.
       if (SC != SC_HEAD && n > 0) {
-        // v_ref = the largest V' factor over this CTA's visible tiles
-        const float* fvh = p.fv + (long long)bhk * p.ntiles_k;
+        const float4* fvh = p.fvr + (long long)bhk * p.ntiles_k;
         float m = 0.0f;
-        for (int t = lane; t < n; t += 32) m = fmaxf(m, __ldg(fvh + t));
+        for (int t = lane; t < n; t += 32) m = fmaxf(m, __ldg(&fvh[t].x));
 #pragma unroll
         for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
-        const float vref = m > 0.0f ? m : 1.0f;
-        if (lane == 0) misc[0] = vref;
-        for (int j = 0; j < n; ++j) {
-          const int k0 = j * BN, st = j % NSC;
-          float kv[4];
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            const int tok = k0 + lane * 4 + q;
-            kv[q] = tok < p.Sk ? __ldg(p.ks + (long long)bhk * p.k_nblk + tok / p.k_blk) : 0.0f;
+        if (lane == 0) {
+          misc[0] = m > 0.0f ? m : 1.0f;  // v_ref: the largest V' factor over this CTA's visible tiles
+          const float* kph = p.ksp + (long long)bhk * p.ntiles_k * BN;
+          int j = 0;
+          for (; j < n; ++j) {
+            const int st = j % NSC;
+            if (j >= NSC && !mbar_wait(&bar[X_SCE + st], ((j / NSC) - 1) & 1, abort_flag, p.status, 60)) break;
+            uint8_t* stage = smem + L::SC + st * 2 * BN * 4;
+            mbar_arrive_expect_tx(&bar[X_SCF + st], BN * 4 + 16);
+            bulk_load(stage, kph + (long long)j * BN, BN * 4, &bar[X_SCF + st]);
+            bulk_load(stage + BN * 4, fvh + j, 16, &bar[X_SCF + st]);
           }
-          const float fj = __ldg(fvh + j);
-          if (j >= NSC && !warp_wait(&bar[X_SCE + st], ((j / NSC) - 1) & 1, abort_flag, p.status, 60)) break;
-          float* ksc = reinterpret_cast<float*>(smem + L::SC + st * 2 * BN * 4);
-          *reinterpret_cast<float4*>(ksc + lane * 4) = make_float4(kv[0], kv[1], kv[2], kv[3]);
-          if (lane == 0) {
-            // V' factor r_t / v_ref enters the exponent as its log2, floored at -60
-            // (a tile that small adds nothing visible to O); the row sum divides it out.
-            const float fl = fmaxf(__log2f(fj / vref), -60.0f);
-            ksc[BN] = fl;
-            ksc[BN + 1] = exp2f(-fl);
-          }
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&bar[X_SCF + st]);
+          if (*abort_flag)
+            for (int t = max(0, j - NSC); t < j; ++t) mbar_wait(&bar[X_SCF + t % NSC], (t / NSC) & 1, abort_flag, nullptr, 0);
         }
       }
       __syncwarp();
@@ -266,14 +279,15 @@ __global__ void __launch_bounds__(NT, 1)
           mma_commit(&bar[X_KE + j % NKS]);
         };
         auto pv = [&](int j) {
-          // A = P' in TMEM: keys [0, 64) in columns 0..31 and keys [64, 128) in
-          // columns 64..95 of the S buffer; 16 keys (8 columns) per MMA.
+          // A = P' in TMEM: key group g's HN keys sit (as fp16 pairs) in columns
+          // [g * HN, g * HN + HN / 2) of the S buffer; 16 keys (8 columns) per MMA.
           const uint32_t sVh = smem_u32(smem + L::VH + (j % NVS) * BN * D * 2);
           const uint32_t tP = tbase + (j & 1) * 128;
 #pragma unroll
           for (int ks = 0; ks < BN / 16; ++ks) {
             const uint64_t db = make_sdesc(sVh + ks * 16 * 128, BN * 128, 1024, kSwz128);
-            mma_f16_ts(tO, tP + (ks >> 2) * 64 + (ks & 3) * 8, db, idesc_pv, (j > 0 || ks > 0) ? 1u : 0u);
+            const int g = ks * 16 / HN;
+            mma_f16_ts(tO, tP + g * HN + ((ks * 16 - g * HN) >> 1), db, idesc_pv, (j > 0 || ks > 0) ? 1u : 0u);
           }
           mma_commit(&bar[X_PVD]);
           mma_commit(&bar[X_VE + j % NVS]);
@@ -305,9 +319,9 @@ __global__ void __launch_bounds__(NT, 1)
       __syncwarp();
     }
   } else {
-    setmaxnreg_inc208();
+    setmaxnreg_inc<Cfg<NSW>::RS>();
     // ------------------------------------------------------------- softmax
-    const int h = (warp - 4) >> 2;  // key half: columns [h * 64, h * 64 + 64) of each S tile
+    const int h = (warp - 4) >> 2;  // key group: columns [h * HN, h * HN + HN) of each S tile
     const int i = tid - 128 - h * 128;
     const uint32_t loff = (uint32_t)((warp & 3) * 32) << 16;
     const int cb = h * HN;
@@ -339,15 +353,17 @@ __global__ void __launch_bounds__(NT, 1)
       }
       float flog = 0.0f, finv = 1.0f, ktile = 1.0f;
       if (SC != SC_HEAD) {
-        flog = ksc[BN];
-        finv = ksc[BN + 1];
+        // V' factor r_t / v_ref enters the exponent as its log2, floored at -60 (a tile that
+        // small adds nothing visible to O); the row sum divides it back out.
+        flog = fmaxf(__log2f(ksc[BN] / vref), -60.0f);
+        finv = ex2(-flog);
       }
       if (SC == SC_TILE) ktile = ksc[0];
       if (!warp_wait(&bar[X_SF + st], (j >> 1) & 1, abort_flag, p.status, 71)) { ok = false; break; }
       tc_fence_after();
       uint32_t tr[HN];
-      tmem_ld32(tS + loff + 0, *reinterpret_cast<uint32_t(*)[32]>(&tr[0]));
-      tmem_ld32(tS + loff + 32, *reinterpret_cast<uint32_t(*)[32]>(&tr[32]));
+#pragma unroll
+      for (int c = 0; c < HN / 32; ++c) tmem_ld32(tS + loff + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(&tr[32 * c]));
       tmem_ld_wait();
       float t[HN];
 #pragma unroll
@@ -372,18 +388,28 @@ __global__ void __launch_bounds__(NT, 1)
         for (int k = 0; k < HN; ++k)
           if (kc0 + k > lim) t[k] = -INFINITY;
       }
+      // eight max chains over HN / 8 keys each, three-input max
+      constexpr int PER = HN / 8;
       float mx[8];
 #pragma unroll
-      for (int e = 0; e < 8; ++e) mx[e] = t[e];
+      for (int e = 0; e < 8; ++e) {
+        mx[e] = t[e];
 #pragma unroll
-      for (int k = 8; k < HN; ++k) mx[k & 7] = fmaxf(mx[k & 7], t[k]);
-      const float mt = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])), fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
-      const float mts = mt == -INFINITY ? -INFINITY : (mt - kBias) * cr;  // half-tile max of the log2-domain score
-      // publish this half's maximum; the partner's is read once it is needed
-      xm[(st * 2 + h) * BM + i] = mts;
+        for (int q = 1; q < PER; q += 2) mx[e] = q + 1 < PER ? fmax3(mx[e], t[e + 8 * q], t[e + 8 * q + 8]) : fmaxf(mx[e], t[e + 8 * q]);
+      }
+      const float mt = fmax3(fmax3(mx[0], mx[1], mx[2]), fmax3(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7]));
+      const float mts = mt == -INFINITY ? -INFINITY : (mt - kBias) * cr;  // this group's tile max, log2 domain
+      // publish this group's maximum; the others' are read once they are needed
+      xm[(st * 4 + h) * BM + i] = mts;
       __syncwarp();
       if (lane == 0) mbar_arrive(&bar[X_MX + st]);
-      const float* xpart = xm + (st * 2 + (h ^ 1)) * BM + i;
+      auto others_max = [&]() {
+        float m = -INFINITY;
+#pragma unroll
+        for (int g = 0; g < NSW; ++g)
+          if (g != h) m = fmaxf(m, xm[(st * 4 + g) * BM + i]);
+        return m;
+      };
       // The running max moves only when a tile's max exceeds it by more than 2^8, so the
       // exponentials normally use m_run before the partner's half is known.  A warp where
       // this half alone forces a move (always on a row's first visible tile) takes both
@@ -393,7 +419,7 @@ __global__ void __launch_bounds__(NT, 1)
       if (__any_sync(0xffffffffu, mts > m_run + 8.0f)) {
         if (!warp_wait(&bar[X_MX + st], (j >> 1) & 1, abort_flag, p.status, 75)) { ok = false; break; }
         have_part = true;
-        const float m_new = fmaxf(m_run, fmaxf(mts, *xpart));
+        const float m_new = fmaxf(m_run, fmaxf(mts, others_max()));
         if (m_new > m_run + 8.0f) m_use = m_new;
       }
       // exp2 argument: t * cr - (bias * cr + m) + log2(r_t / v_ref)   (bias 0 for E4M3; factor 1 for INT8)
@@ -409,33 +435,47 @@ __global__ void __launch_bounds__(NT, 1)
         }
       }
       if (!have_part && !warp_wait(&bar[X_MX + st], (j >> 1) & 1, abort_flag, p.status, 75)) { ok = false; break; }
-      // the decision both halves take from the same three numbers
-      const float m_new = fmaxf(m_run, fmaxf(mts, *xpart));
+      // the decision every group takes from the same numbers
+      const float m_new = fmaxf(m_run, fmaxf(mts, others_max()));
       const float m_fin = m_new > m_run + 8.0f ? m_new : m_run;
       if (__any_sync(0xffffffffu, m_fin != m_use)) {
-        // the partner's half moved the max: rescale this half's p (each <= 2^8 here)
+        // another group moved the max: rescale this group's p (each <= 2^8 here)
         const float c = m_fin != m_use ? ex2(m_use - m_fin) : 1.0f;
 #pragma unroll
         for (int k = 0; k < HN; k += 2) fmul2(t[k], t[k + 1], c, c);
       }
       const float alpha = m_fin != m_run ? ex2(m_run - m_fin) : 1.0f;
       if (__any_sync(0xffffffffu, m_fin != m_run) && j > 0) {
-        // O is free once P V of tile j-1 has completed; each half rescales its own O columns.
+        // O is free once P V of tile j-1 has completed; each group rescales its own DC O columns.
         if (!warp_wait(&bar[X_PVD], (j - 1) & 1, abort_flag, p.status, 72)) { ok = false; break; }
         tc_fence_after();
+        if (DC >= 32) {
 #pragma unroll
-        for (int c = 0; c < D / 64; ++c) {
-          uint32_t r[32];
-          tmem_ld32(tO + loff + h * (D / 2) + c * 32, r);
+          for (int c = 0; c < DC / 32; ++c) {
+            uint32_t r[32];
+            tmem_ld32(tO + loff + h * DC + c * 32, r);
+            tmem_ld_wait();
+#pragma unroll
+            for (int k = 0; k < 32; k += 2) {
+              float a0 = __uint_as_float(r[k]), a1 = __uint_as_float(r[k + 1]);
+              fmul2(a0, a1, alpha, alpha);
+              r[k] = __float_as_uint(a0);
+              r[k + 1] = __float_as_uint(a1);
+            }
+            tmem_st32(tO + loff + h * DC + c * 32, r);
+          }
+        } else {
+          uint32_t r[16];
+          tmem_ld16(tO + loff + h * DC, r);
           tmem_ld_wait();
 #pragma unroll
-          for (int k = 0; k < 32; k += 2) {
+          for (int k = 0; k < 16; k += 2) {
             float a0 = __uint_as_float(r[k]), a1 = __uint_as_float(r[k + 1]);
             fmul2(a0, a1, alpha, alpha);
             r[k] = __float_as_uint(a0);
             r[k + 1] = __float_as_uint(a1);
           }
-          tmem_st32(tO + loff + h * (D / 2) + c * 32, r);
+          tmem_st16(tO + loff + h * DC, r);
         }
         tmem_st_wait();
       }
@@ -446,15 +486,18 @@ __global__ void __launch_bounds__(NT, 1)
       for (int e = 0; e < 8; ++e) ls[e] = t[e];
 #pragma unroll
       for (int k = 8; k < HN; k += 2) fadd2(ls[k & 7], ls[(k & 7) + 1], t[k], t[k + 1]);
-      // P' = fp16(p) over this half's first 32 S columns
+      // P' = fp16(p) over this group's first HN / 2 S columns
       {
-        uint32_t hp[32];
+        uint32_t hp[HN / 2];
 #pragma unroll
-        for (int e = 0; e < 32; ++e) {
+        for (int e = 0; e < HN / 2; ++e) {
           const __half2 hv = __floats2half2_rn(t[2 * e], t[2 * e + 1]);
           hp[e] = *reinterpret_cast<const uint32_t*>(&hv);
         }
-        tmem_st32(tS + loff, hp);
+        if constexpr (HN == 64)
+          tmem_st32(tS + loff, *reinterpret_cast<uint32_t(*)[32]>(&hp[0]));
+        else
+          tmem_st16(tS + loff, *reinterpret_cast<uint32_t(*)[16]>(&hp[0]));
       }
       tmem_st_wait();
       l_run += (((ls[0] + ls[1]) + (ls[2] + ls[3])) + ((ls[4] + ls[5]) + (ls[6] + ls[7]))) * finv;
@@ -470,33 +513,41 @@ __global__ void __launch_bounds__(NT, 1)
       ok = warp_wait(&bar[X_PVD], (n - 1) & 1, abort_flag, p.status, 73);
       tc_fence_after();
     }
-    // row sum = the two halves' partial sums
+    // row sum = the groups' partial sums (added in one order by every group)
     xl[h * BM + i] = l_run;
     __syncwarp();
     if (lane == 0) mbar_arrive(&bar[X_LX]);
     const bool lx = warp_wait(&bar[X_LX], 0, abort_flag, p.status, 76);
-    const float l_tot = lx ? xl[i] + xl[BM + i] : 0.0f;
+    float l_tot = 0.0f;
+    if (lx) {
+#pragma unroll
+      for (int g = 0; g < NSW; ++g) l_tot += xl[g * BM + i];
+    }
     if (q0 < p.Sq) {
       const float ofac = l_tot > 0.0f ? vref / l_tot : 0.0f;
       __nv_bfloat16* orow = nullptr;
       if (row_ok) {
         const long long ridx = p.layout == FA_LAYOUT_BNSD ? ((long long)qbh * p.Sq + row)
                                                           : (((long long)b * p.Sq + row) * p.Hq + hq);
-        orow = p.out + ridx * D + h * (D / 2);
+        orow = p.out + ridx * D + h * DC;
       }
+      constexpr int OW = DC >= 32 ? 32 : 16;  // O columns per TMEM load
 #pragma unroll
-      for (int c = 0; c < D / 64; ++c) {
-        uint32_t r[32];
+      for (int c = 0; c < DC / OW; ++c) {
+        uint32_t r[OW];
         if (ok && n > 0) {
-          tmem_ld32(tO + loff + h * (D / 2) + c * 32, r);
+          if constexpr (OW == 32)
+            tmem_ld32(tO + loff + h * DC + c * 32, r);
+          else
+            tmem_ld16(tO + loff + h * DC, r);
           tmem_ld_wait();
         } else {
 #pragma unroll
-          for (int k = 0; k < 32; ++k) r[k] = 0u;
+          for (int k = 0; k < OW; ++k) r[k] = 0u;
         }
         if (row_ok) {
 #pragma unroll
-          for (int k = 0; k < 32; k += 8) {
+          for (int k = 0; k < OW; k += 8) {
             uint32_t o[4];
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
@@ -504,7 +555,7 @@ __global__ void __launch_bounds__(NT, 1)
                                                               __uint_as_float(r[k + 2 * e + 1]) * ofac);
               o[e] = *reinterpret_cast<const uint32_t*>(&v2);
             }
-            *reinterpret_cast<uint4*>(orow + c * 32 + k) = make_uint4(o[0], o[1], o[2], o[3]);
+            *reinterpret_cast<uint4*>(orow + c * OW + k) = make_uint4(o[0], o[1], o[2], o[3]);
           }
         }
       }
@@ -528,7 +579,9 @@ __global__ void __launch_bounds__(NT, 1)
 template <int KIND, int D>
 __global__ void __launch_bounds__(256) vprep_kernel(const uint8_t* __restrict__ codes, const float* __restrict__ vs,
                                                     int v_blk, int v_nblk, int H, int S, int layout,
-                                                    __half* __restrict__ vh, float* __restrict__ fv, int ntiles) {
+                                                    __half* __restrict__ vh, float4* __restrict__ fvr, int ntiles,
+                                                    const float* __restrict__ ks, int k_blk, int k_nblk,
+                                                    float* __restrict__ ksp) {
   constexpr int CPT = D / 32;  // 16-code chunks per thread: each thread owns half a token row
   const int t = blockIdx.x, bh = blockIdx.y;
   const int b = bh / H, h = bh % H;
@@ -555,7 +608,12 @@ __global__ void __launch_bounds__(256) vprep_kernel(const uint8_t* __restrict__ 
     for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
     const float r = m > 0.0f ? m : 1.0f;
     f = live ? __ldg(vsh + tok / v_blk) / r : 0.0f;
-    if (threadIdx.x == 0) fv[(long long)bh * ntiles + t] = r;
+    if (threadIdx.x == 0) fvr[(long long)bh * ntiles + t] = make_float4(r, 0.0f, 0.0f, 0.0f);
+    // the tile's per-key K scales, zero past S, at a 16-byte aligned per-tile slot
+    if (threadIdx.x < BN) {
+      const int key = tok0 + threadIdx.x;
+      ksp[((long long)bh * ntiles + t) * BN + threadIdx.x] = key < S ? __ldg(ks + (long long)bh * k_nblk + key / k_blk) : 0.0f;
+    }
   }
   if (!live) return;
   uint4* dst = reinterpret_cast<uint4*>(vh + ((long long)bh * S + tok) * D + (lane & 1) * (D / 2));
@@ -600,20 +658,32 @@ cudaError_t make_vh_map(CUtensorMap* map, const void* base, int B, int H, int S,
 
 struct Prefill2Ws {
   __half* vh;
-  float* fv;
+  float4* fvr;
+  float* ksp;
 };
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
+// Workspace: V' fp16 [B, Hkv, Sk, D] | V' factor records [B, Hkv, ntiles] | K scales [B, Hkv, ntiles * 128].
 Prefill2Ws carve_ws(void* ws, int B, int Hkv, int Sk, int D) {
+  const size_t ntiles = ((size_t)Sk + BN - 1) / BN;
+  uint8_t* base = static_cast<uint8_t*>(ws);
   Prefill2Ws w;
-  w.vh = static_cast<__half*>(ws);
-  w.fv = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + align256((size_t)B * Hkv * Sk * D * 2));
+  w.vh = reinterpret_cast<__half*>(base);
+  base += align256((size_t)B * Hkv * Sk * D * 2);
+  w.fvr = reinterpret_cast<float4*>(base);
+  base += align256((size_t)B * Hkv * ntiles * 16);
+  w.ksp = reinterpret_cast<float*>(base);
   return w;
 }
 
+#ifndef FAQ_ATTN_NSW
+#define FAQ_ATTN_NSW 4
+#endif
+
 template <int KIND, int D, int SC>
 cudaError_t launch2(const AttnArgs& a, const P2& prm, const Prefill2Ws& w, cudaStream_t s) {
+  constexpr int NSW = FAQ_ATTN_NSW;
   using L = L2<D>;
   CUtensorMap mq, mk, mv;
   cudaError_t e;
@@ -623,9 +693,10 @@ cudaError_t launch2(const AttnArgs& a, const P2& prm, const Prefill2Ws& w, cudaS
   const dim3 pgrid((unsigned)prm.ntiles_k, (unsigned)(a.v->B * a.v->H));
   if (pgrid.y > 65535u) return cudaErrorInvalidValue;
   vprep_kernel<KIND, D><<<pgrid, 256, 0, s>>>(static_cast<const uint8_t*>(a.v->codes), prm.vs, prm.v_blk,
-                                               prm.v_nblk, a.v->H, a.v->S, a.v->layout, w.vh, w.fv, prm.ntiles_k);
+                                               prm.v_nblk, a.v->H, a.v->S, a.v->layout, w.vh, w.fvr, prm.ntiles_k,
+                                               prm.ks, prm.k_blk, prm.k_nblk, w.ksp);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  auto kern = attn2_kernel<KIND, D, SC>;
+  auto kern = attn2_kernel<KIND, D, SC, NSW>;
   static bool attr_set = false;
   if (!attr_set) {
     if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::ALLOC)) != cudaSuccess)
@@ -634,7 +705,7 @@ cudaError_t launch2(const AttnArgs& a, const P2& prm, const Prefill2Ws& w, cudaS
   }
   const long long grid = (long long)prm.n_qtiles * prm.B * prm.Hq;
   if (grid > 0x7FFFFFFFLL) return cudaErrorInvalidValue;
-  kern<<<(unsigned)grid, NT, L::ALLOC, s>>>(mq, mk, mv, prm);
+  kern<<<(unsigned)grid, Cfg<NSW>::NT, L::ALLOC, s>>>(mq, mk, mv, prm);
   return cudaGetLastError();
 }
 
@@ -661,7 +732,8 @@ void scale_desc2(const fa_qtensor* t, int& blk, int& nblk) {
 // Prefill attention for E4M3 and INT8 operands.
 size_t prefill2_workspace_bytes(int B, int Hkv, int Sk, int D) {
   const size_t ntiles = ((size_t)Sk + BN - 1) / BN;
-  return align256((size_t)B * Hkv * Sk * D * 2) + align256((size_t)B * Hkv * ntiles * 4);
+  return align256((size_t)B * Hkv * Sk * D * 2) + align256((size_t)B * Hkv * ntiles * 16) +
+         align256((size_t)B * Hkv * ntiles * BN * 4);
 }
 
 cudaError_t launch_attention_prefill2(const AttnArgs& a, void* ws, cudaStream_t s) {
@@ -684,7 +756,8 @@ cudaError_t launch_attention_prefill2(const AttnArgs& a, void* ws, cudaStream_t 
   prm.n_qtiles = (q->S + BM - 1) / BM;
   prm.ntiles_k = (k->S + BN - 1) / BN;
   const Prefill2Ws w = carve_ws(ws, k->B, k->H, k->S, q->D);
-  prm.fv = w.fv;
+  prm.fvr = w.fvr;
+  prm.ksp = w.ksp;
   int sc = SC_HEAD;
   if (q->mode == FA_MODE_FP8_PER_TOKEN) sc = SC_COL;
   if (q->mode == FA_MODE_FP8_BLOCK) sc = (k->block_tokens % BN == 0) ? SC_TILE : SC_COL;

@@ -61,6 +61,13 @@ __device__ __forceinline__ void ex2_poly2(float& a, float& b) {
   b = __int_as_float(__float_as_int(p1) + (__float_as_int(j1) << 23));
 }
 
+// max(a, b, c) in one instruction (sm_100 three-input form).
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
 // Every lane waits; the warp proceeds only if all lanes saw the phase complete.
 __device__ __forceinline__ bool warp_wait(uint64_t* b, uint32_t parity, volatile int* abort_flag, int* status,
                                           int where) {

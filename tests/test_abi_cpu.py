@@ -130,12 +130,13 @@ def test_attention_validation_before_launch(N):
     assert L.fa_attention_quant(by(qd), by(kd), by(kd), 0, 0.0, 0x60000, None, 0, 0x70000, need - 16,
                                 None) == 7
     assert L.fa_attention_quant(by(qd), by(kd), by(kd), 0, 0.0, 0x60000, None, -1, None, 0, None) == 1
-    # FP8 / INT8 prefill: fp16 V' plus one factor per 128-key tile, each 256-byte aligned
+    # FP8 / INT8 prefill: fp16 V', a 16-byte factor record and 128 K scales per 128-key tile,
+    # each part 256-byte aligned
     qp = _q(N, 1, B=2, H=4, S=100, D=128)
     need_p = L.fa_attention_workspace_size(by(qp), by(kd), 0)
-    vh = 2 * 2 * 1000 * 128 * 2
-    fv = 2 * 2 * ((1000 + 127) // 128) * 4
-    assert need_p == ((vh + 255) // 256) * 256 + ((fv + 255) // 256) * 256
+    ntiles = (1000 + 127) // 128
+    parts = (2 * 2 * 1000 * 128 * 2, 2 * 2 * ntiles * 16, 2 * 2 * ntiles * 128 * 4)
+    assert need_p == sum(((x + 255) // 256) * 256 for x in parts)
     assert L.fa_attention_quant(by(qp), by(kd), by(kd), 0, 0.0, 0x60000, None, 0, None, 0, None) == 7
     assert L.fa_attention_quant(by(qp), by(kd), by(kd), 0, 0.0, 0x60000, None, 0, 0x70000, need_p - 256,
                                 None) == 7
