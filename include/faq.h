@@ -79,7 +79,8 @@ typedef struct {
 } fa_tensor;
 
 /* A quantized tensor: codes + scales + mode + layout.  Filled by the caller
- * (pointers to caller-owned device buffers of the sizes listed above). */
+ * (pointers to caller-owned device buffers of the sizes listed above; codes
+ * 16-byte aligned, scales 4-byte aligned, else FA_ERR_INVALID_ARG). */
 typedef struct {
   void* codes;
   void* scales;

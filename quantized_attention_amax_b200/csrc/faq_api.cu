@@ -75,7 +75,8 @@ fa_status check_out(const fa_tensor* t, const fa_qtensor* o, fa_mode mode) {
   if (o->mode != mode || o->B != t->B || o->H != t->H || o->S != t->S || o->D != t->D || o->layout != t->layout)
     return FA_ERR_INVALID_ARG;
   if ((long long)t->B * t->S == 0) return FA_OK;
-  if (!o->codes || !o->scales || !aligned16(o->codes)) return FA_ERR_INVALID_ARG;
+  if (!o->codes || !o->scales || !aligned16(o->codes) || (reinterpret_cast<uintptr_t>(o->scales) & 3u))
+    return FA_ERR_INVALID_ARG;
   if (mode == FA_MODE_FP8_BLOCK && o->block_tokens < 1) return FA_ERR_INVALID_ARG;
   if (mode == FA_MODE_MXFP4_PER_BLOCK && o->D % 32 != 0) return FA_ERR_INVALID_ARG;
   return FA_OK;
