@@ -10,10 +10,12 @@
 //   warp 1     tcgen05.mma kind::f16 (bf16 x bf16 -> fp32): X R into TMEM,
 //              R read as the MN-major B operand exactly as stored ([D, D]
 //              row-major, x' = x R).
-//   warps 4-7  epilogue, one thread per token row: TMEM (or, for V, the
-//              shared-memory tile) -> bf16 row -> row amax -> block amax ->
-//              scale -> E4M3 codes (IEEE division), optional bf16 copy of
-//              the rotated row.
+//   all 8 warps, then, the epilogue: warp w takes TMEM lane quarter w % 4
+//              and column half w / 4 of each 128-token tile; its bf16 half
+//              rows (rotated in TMEM, or V from the shared tile) stay in
+//              registers for half-row maxima -> block maxima (one warp per
+//              block, through shared memory) -> scale -> E4M3 codes (IEEE
+//              division), with an optional bf16 copy of the rotated rows.
 // blk must divide 256.
 #include <cuda_bf16.h>
 #include <string.h>
@@ -45,8 +47,9 @@ struct RotParams {
 struct RSmem {
   static constexpr uint32_t X = 0;           // [2 tiles][2 K atoms][128 rows][128 B]
   static constexpr uint32_t R = 65536;       // [2 N atoms][128 d rows][128 B]
-  static constexpr uint32_t RMAX = R + 32768;  // [256] row maxima
-  static constexpr uint32_t BAR = RMAX + 1024;
+  static constexpr uint32_t RMAX = R + 32768;    // [2 tiles][2 halves][128] half-row maxima
+  static constexpr uint32_t BMAX = RMAX + 2048;  // [256] per-block scale (up to 256 blocks per chunk)
+  static constexpr uint32_t BAR = BMAX + 1024;
   static constexpr uint32_t TOTAL = BAR + 256;
   static constexpr uint32_t ALLOC = TOTAL + 1024;
 };
@@ -69,10 +72,11 @@ __global__ void __launch_bounds__(RTHREADS, 2)
                               const __grid_constant__ CUtensorMap mrk, const RotParams prm) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* bar = reinterpret_cast<uint64_t*>(smem + RSmem::BAR);  // 0: loads, 1: mma, 2: row maxima
+  uint64_t* bar = reinterpret_cast<uint64_t*>(smem + RSmem::BAR);  // 0: loads, 1: mma, 2: row maxima, 3: block scales
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar + 4);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(bar + 5);
   float* rmax = reinterpret_cast<float*>(smem + RSmem::RMAX);
+  float* bsc = reinterpret_cast<float*>(smem + RSmem::BMAX);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const long long cta = blockIdx.x;
@@ -93,7 +97,8 @@ __global__ void __launch_bounds__(RTHREADS, 2)
   if (tid == 0) {
     mbar_init(&bar[0], 1);
     mbar_init(&bar[1], 1);
-    mbar_init(&bar[2], 128);
+    mbar_init(&bar[2], RTHREADS);
+    mbar_init(&bar[3], RTHREADS);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -138,94 +143,94 @@ __global__ void __launch_bounds__(RTHREADS, 2)
       mbar_wait(&bar[1], 0, abort_flag, nullptr, 0);
     }
     __syncwarp();
-  } else if (warp >= 4) {
-    const int i = tid - 128;
-    const uint32_t loff = (uint32_t)((warp - 4) * 32) << 16;
-    bool ok = true;
-    if (op.rotate) {
-      ok = mbar_wait(&bar[1], 0, abort_flag, prm.status, 41);
-      tc_fence_after();
-    } else {
-      ok = mbar_wait(&bar[0], 0, abort_flag, prm.status, 42);
-    }
-    ok = __all_sync(0xffffffffu, ok);
-    // 32 elements of row i of tile u, chunk c (0..3), as 16 packed bf16x2.
-    auto load32 = [&](int u, int c, uint32_t (&v)[16]) {
-      if (op.rotate) {
-        uint32_t r[32];
-        tmem_ld32(tbase + u * 128 + loff + c * 32, r);
-        tmem_ld_wait();
+  }
+
+  // ---------------------------------------------------------------- epilogue
+  const int half = warp >> 2;                 // columns [64 * half, 64 * half + 64)
+  const int i = (warp & 3) * 32 + lane;       // row within a 128-token tile
+  const uint32_t loff = (uint32_t)((warp & 3) * 32) << 16;
+  bool ok = mbar_wait(&bar[op.rotate ? 1 : 0], 0, abort_flag, prm.status, op.rotate ? 41 : 42);
+  ok = __all_sync(0xffffffffu, ok);
+  if (op.rotate) tc_fence_after();
+  // 64 elements (half a row) of each tile as 32 packed bf16x2
+  uint32_t v[2][32];
 #pragma unroll
-        for (int k = 0; k < 16; ++k) v[k] = bf16x2_rn(__uint_as_float(r[2 * k]), __uint_as_float(r[2 * k + 1]));
+  for (int u = 0; u < 2; ++u) {
+    const int t = t0 + u * 128 + i;
+    const bool live = u < ntile && t < op.S;
+    float am = 0.0f;
+    if (u < ntile && ok) {  // warp-uniform: TMEM loads are warp-collective
+      if (op.rotate) {
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          uint32_t r[32];
+          tmem_ld32(tbase + u * 128 + loff + half * 64 + c * 32, r);
+          tmem_ld_wait();
+#pragma unroll
+          for (int k = 0; k < 16; ++k) v[u][c * 16 + k] = bf16x2_rn(__uint_as_float(r[2 * k]), __uint_as_float(r[2 * k + 1]));
+        }
       } else {
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const int cc = c * 4 + q;  // 16-byte chunk 0..15 of the 256-byte row
-          const uint4 x = *reinterpret_cast<const uint4*>(smem + RSmem::X + (u * 2 + (cc >> 3)) * 16384 +
-                                                          swz128_offset(i, cc & 7));
-          v[4 * q] = x.x; v[4 * q + 1] = x.y; v[4 * q + 2] = x.z; v[4 * q + 3] = x.w;
+        for (int q = 0; q < 8; ++q) {
+          const uint4 x = *reinterpret_cast<const uint4*>(smem + RSmem::X + (u * 2 + half) * 16384 + swz128_offset(i, q));
+          v[u][4 * q] = x.x; v[u][4 * q + 1] = x.y; v[u][4 * q + 2] = x.z; v[u][4 * q + 3] = x.w;
         }
       }
-    };
-    // Pass 1: row maxima of the bf16 rows (and the optional bf16 copy).
-#pragma unroll 1
-    for (int u = 0; u < 2; ++u) {
-      const int t = t0 + u * 128 + i;
-      float am = 0.0f;
-      if (u < ntile && ok) {
+#pragma unroll
+      for (int k = 0; k < 32; ++k)
+        am = fmaxf(am, fmaxf(fabsf(__uint_as_float(v[u][k] << 16)), fabsf(__uint_as_float(v[u][k] & 0xFFFF0000u))));
+      if (op.dbg && live) {
         const long long ridx = bnsd ? (((long long)b * op.H + h) * op.S + t) : (((long long)b * op.S + t) * op.H + h);
-#pragma unroll 1
-        for (int c = 0; c < 4; ++c) {
-          uint32_t v[16];
-          load32(u, c, v);
+        uint4* d = reinterpret_cast<uint4*>(op.dbg + ridx * 128 + half * 64);
 #pragma unroll
-          for (int k = 0; k < 16; ++k)
-            am = fmaxf(am, fmaxf(fabsf(__uint_as_float(v[k] << 16)), fabsf(__uint_as_float(v[k] & 0xFFFF0000u))));
-          if (op.dbg && t < op.S) {
-            uint4* d = reinterpret_cast<uint4*>(op.dbg + ridx * 128 + c * 32);
-#pragma unroll
-            for (int q = 0; q < 4; ++q) d[q] = make_uint4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
-          }
-        }
+        for (int q = 0; q < 8; ++q) d[q] = make_uint4(v[u][4 * q], v[u][4 * q + 1], v[u][4 * q + 2], v[u][4 * q + 3]);
       }
-      rmax[u * 128 + i] = (u < ntile && t < op.S) ? am : 0.0f;
     }
-    mbar_arrive(&bar[2]);
-    ok = __all_sync(0xffffffffu, mbar_wait(&bar[2], 0, abort_flag, prm.status, 43)) && ok;
+    rmax[(u * 2 + half) * 128 + i] = live ? am : 0.0f;
+  }
+  mbar_arrive(&bar[2]);
+  ok = __all_sync(0xffffffffu, mbar_wait(&bar[2], 0, abort_flag, prm.status, 43)) && ok;
 
-    // Pass 2: block scale and codes.
-    const int nblk = (op.S + op.blk - 1) / op.blk;
-#pragma unroll 1
-    for (int u = 0; u < 2; ++u) {
-      const int r_in = u * 128 + i;  // row within the chunk
-      const int t = t0 + r_in;
-      const bool live = u < ntile && t < op.S;
-      const int g0 = (r_in / op.blk) * op.blk;  // block start within the chunk
-      float bm = 0.0f;
-      for (int q = g0; q < g0 + op.blk && q < CH; ++q) bm = fmaxf(bm, rmax[q]);
-      const float sc = __fdiv_rn(bm, 448.0f);
-      const long long ridx = bnsd ? (((long long)b * op.H + h) * op.S + t) : (((long long)b * op.S + t) * op.H + h);
-      if (live && r_in == g0) op.scales[((long long)b * op.H + h) * nblk + t / op.blk] = ok ? sc : 0.0f;
-#pragma unroll 1
-      for (int c = 0; c < 4; ++c) {
-        uint32_t v[16];
-        if (u < ntile && ok) load32(u, c, v);  // warp-uniform: TMEM loads are warp-collective
-        if (!live) continue;
-        uint32_t w[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          const uint32_t p0 = v[2 * e], p1 = v[2 * e + 1];
-          const float x0 = __uint_as_float(p0 << 16), x1 = __uint_as_float(p0 & 0xFFFF0000u);
-          const float x2 = __uint_as_float(p1 << 16), x3 = __uint_as_float(p1 & 0xFFFF0000u);
-          w[e] = (sc > 0.0f && ok) ? e4m3x4(__fdiv_rn(x0, sc), __fdiv_rn(x1, sc), __fdiv_rn(x2, sc), __fdiv_rn(x3, sc))
-                                   : 0u;
-        }
-        uint4* crow = reinterpret_cast<uint4*>(static_cast<uint8_t*>(op.codes) + ridx * 128 + c * 32);
-        crow[0] = make_uint4(w[0], w[1], w[2], w[3]);
-        crow[1] = make_uint4(w[4], w[5], w[6], w[7]);
-      }
+  // block scales: warp w reduces blocks w, w + 8, ... of the chunk (2 * blk half-row maxima each)
+  const int nb_chunk = CH / op.blk;
+  const int nblk = (op.S + op.blk - 1) / op.blk;
+  for (int bb = warp; bb < nb_chunk; bb += RTHREADS / 32) {
+    float m = 0.0f;
+    for (int k = lane; k < 2 * op.blk; k += 32) {
+      const int row = bb * op.blk + (k >> 1);
+      m = fmaxf(m, rmax[((row >> 7) * 2 + (k & 1)) * 128 + (row & 127)]);
     }
-    if (op.rotate) tc_fence_before();
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+    const float sc = __fdiv_rn(m, 448.0f);
+    if (lane == 0) {
+      bsc[bb] = sc;
+      const int t = t0 + bb * op.blk;
+      if (t < op.S) op.scales[((long long)b * op.H + h) * nblk + t / op.blk] = ok ? sc : 0.0f;
+    }
+  }
+  mbar_arrive(&bar[3]);
+  ok = __all_sync(0xffffffffu, mbar_wait(&bar[3], 0, abort_flag, prm.status, 44)) && ok;
+
+  // codes: this thread's 64 values of each tile row
+#pragma unroll
+  for (int u = 0; u < 2; ++u) {
+    const int r_in = u * 128 + i;
+    const int t = t0 + r_in;
+    if (!(u < ntile && t < op.S)) continue;
+    const float sc = bsc[r_in / op.blk];
+    const long long ridx = bnsd ? (((long long)b * op.H + h) * op.S + t) : (((long long)b * op.S + t) * op.H + h);
+    uint32_t w[16];
+#pragma unroll
+    for (int e = 0; e < 16; ++e) {
+      const uint32_t p0 = v[u][2 * e], p1 = v[u][2 * e + 1];
+      const float x0 = __uint_as_float(p0 << 16), x1 = __uint_as_float(p0 & 0xFFFF0000u);
+      const float x2 = __uint_as_float(p1 << 16), x3 = __uint_as_float(p1 & 0xFFFF0000u);
+      w[e] = (sc > 0.0f && ok) ? e4m3x4(__fdiv_rn(x0, sc), __fdiv_rn(x1, sc), __fdiv_rn(x2, sc), __fdiv_rn(x3, sc)) : 0u;
+    }
+    uint4* crow = reinterpret_cast<uint4*>(static_cast<uint8_t*>(op.codes) + ridx * 128 + half * 64);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) crow[q] = make_uint4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
   }
 
   tc_fence_before();
