@@ -222,7 +222,21 @@ def make_step(faq, wl, w, device, seed_offset=0):
 
 
 def launches_per_step(w):
-    return 1 + (2 if w.name == "int8_decode" else 1)
+    """This library's kernels per step: the quantize (or rotate + quantize) launch, then
+    the attention call: decode + LSE combine; MXFP4 one kernel; FP8 / INT8 prefill the
+    V' pre-pass and the attention kernel."""
+    if w.name == "int8_decode":
+        return 1 + 2
+    return 1 + (1 if w.mode == "mxfp4" else 2)
+
+
+def attention_kernels(w):
+    """(label, source file) of the attention call's kernels for this workload."""
+    if w.name == "int8_decode":
+        return "decode_kernel + attn_combine_kernel", "decode.cu"
+    if w.mode == "mxfp4":
+        return "attn_fwd_kernel", "attn.cu"
+    return "vprep_kernel + attn2_kernel (one fa_attention_quant call)", "attn2.cu"
 
 
 def gpu_run(args, w, rank, world, device):
@@ -543,13 +557,13 @@ def main():
     if unit == "GB/s":
         ach = work / (r["attn_ms"] * 1e-3) / 1e9
         roof = {"bound": "hbm", "achieved": ach, "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": ach / pk["hbm_gbs"],
-                "traffic": None, "kernel": "decode_kernel + attn_combine_kernel",
+                "traffic": None, "kernel": attention_kernels(w)[0],
                 "peak_source": f"{pk['src']} HBM copy bandwidth"}
     else:
         tp = tensor_peak(w, pk)
         ach = work / (r["attn_ms"] * 1e-3) / 1e12
         roof = {"bound": "tensor", "achieved": ach, "peak": tp, "unit": "TFLOP/s", "frac": ach / tp,
-                "traffic": None, "kernel": "attn_fwd_kernel",
+                "traffic": None, "kernel": attention_kernels(w)[0],
                 "peak_source": f"{pk['src']} bf16 burst x {4 if w.mode == 'mxfp4' else 2} (dense "
                                f"{'FP4' if w.mode == 'mxfp4' else 'FP8/INT8'} : bf16 nominal ratio)"}
     prof = os.path.join(ROOT, "profiles", f"traffic_{w.name}.json")
@@ -559,7 +573,8 @@ def main():
         try:
             import hashlib
             tr = json.load(open(prof))
-            src = os.path.join(ROOT, "quantized_attention_amax_b200", "csrc", tr.get("kernel_source", "attn.cu"))
+            src = os.path.join(ROOT, "quantized_attention_amax_b200", "csrc",
+                               tr.get("kernel_source", attention_kernels(w)[1]))
             sha = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
             if sha == tr.get("attn_cu_sha256_16"):
                 roof["traffic"] = tr.get("dram_bytes_per_launch")
