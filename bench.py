@@ -223,19 +223,15 @@ def make_step(faq, wl, w, device, seed_offset=0):
 
 def launches_per_step(w):
     """This library's kernels per step: the quantize (or rotate + quantize) launch, then
-    the attention call: decode + LSE combine; MXFP4 one kernel; FP8 / INT8 prefill the
-    V' pre-pass and the attention kernel."""
-    if w.name == "int8_decode":
-        return 1 + 2
-    return 1 + (1 if w.mode == "mxfp4" else 2)
+    the attention call: decode + LSE combine, or for prefill the V' pre-pass and the
+    attention kernel."""
+    return 1 + 2
 
 
 def attention_kernels(w):
     """(label, source file) of the attention call's kernels for this workload."""
     if w.name == "int8_decode":
         return "decode_kernel + attn_combine_kernel", "decode.cu"
-    if w.mode == "mxfp4":
-        return "attn_fwd_kernel", "attn.cu"
     return "vprep_kernel + attn2_kernel (one fa_attention_quant call)", "attn2.cu"
 
 

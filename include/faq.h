@@ -179,10 +179,12 @@ FAQ_API fa_status fa_rotate_quantize(const fa_tensor* q, const fa_tensor* k, con
  *   bytes, 256-byte aligned, owned by the caller and only used during the
  *   call's kernels (FA_ERR_WORKSPACE if missing, short or misaligned).
  *   Decode (q->S == 1) keeps its split-KV partials there before an LSE
- *   combine; FP8 / INT8 prefill keeps V' = fp16(code * s_v / r_t) there
- *   (r_t the largest V scale of each 128-key tile, written beside it), made
- *   once per call by a pre-pass and read by every query tile; MXFP4 needs
- *   none.  num_splits (decode only): 0 = choose automatically.
+ *   combine.  Prefill keeps there, made once per call by a pre-pass and
+ *   read by every query tile: V' = fp16(code * s_v / r_t) (r_t the largest
+ *   V scale of each 128-key tile; MXFP4: V' = fp16(e2m1 * 2^(e - E_t)), E_t
+ *   the tile's largest UE8M0 exponent), a 16-byte record per tile holding
+ *   r_t (E_t), and 512 bytes of K scales per tile (128 per-key floats, or
+ *   MXFP4's scale-factor atom).  num_splits (decode only): 0 = automatic.
  *   Modes run here: INT8_PER_HEAD, FP8_PER_TOKEN, FP8_BLOCK and
  *   MXFP4_PER_BLOCK for prefill; INT8_PER_HEAD for decode (others ->
  *   FA_ERR_UNSUPPORTED).
@@ -225,9 +227,10 @@ FAQ_API fa_status fa_attention_decode_noalloc(const fa_qtensor* q, const fa_qten
                                               fa_stream_t s);
 
 /* Workspace bytes fa_attention_quant needs for these operands and split
- * count: decode B*Hq*splits*(D+2)*4; FP8 / INT8 prefill
- * B*Hkv*Sk*D*2 + B*Hkv*ceil(Sk/128)*4 (each part rounded up to 256);
- * MXFP4 prefill 0.  Returns 0 on invalid arguments. */
+ * count: decode B*Hq*splits*(D+2)*4; prefill (every mode, MXFP4 with
+ * D == 128 only) B*Hkv*Sk*D*2 + B*Hkv*ceil(Sk/128)*16 +
+ * B*Hkv*ceil(Sk/128)*512, each part rounded up to 256.  Returns 0 on
+ * invalid arguments. */
 FAQ_API size_t fa_attention_workspace_size(const fa_qtensor* q, const fa_qtensor* k, int num_splits);
 
 /* Synchronise `s`, read and clear this device's status word.  Returns

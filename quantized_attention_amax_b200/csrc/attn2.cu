@@ -1,33 +1,40 @@
-// attn2.cu -- prefill attention on FP8 (E4M3) and INT8 operands
+// attn2.cu -- prefill attention on FP8 (E4M3), INT8 and MXFP4 operands
 // (FlashAttention's online softmax on low-bit operands: MindIE SD "量化",
-// FA量化 / FP8 Attention; wiki "FA 量化" 参考资料).
+// FA量化 / FP8 Attention and MXFP4 Attention; wiki "FA 量化" 参考资料).
 //
 // Two kernels per call:
 //   vprep: V codes -> V' = fp16(code * s_v / r_t) once per call, r_t = the
-//     largest V scale of 128-key tile t (INT8: V' = fp16(code), exact), into
-//     a caller workspace, with r_t beside it.  Every query tile reads the same
-//     V tiles, so the conversion is done once instead of once per query tile.
+//     largest V scale of 128-key tile t (INT8: V' = fp16(code), exact; MXFP4:
+//     V' = fp16(e2m1 * 2^(e - E_t)) with E_t the tile's largest block exponent),
+//     into a caller workspace, with r_t beside it.  Every query tile reads the
+//     same V tiles, so the conversion is done once instead of once per query
+//     tile.  The same pass lays out each K tile's scales for the attention:
+//     128 per-key floats (E4M3) or the tile's UE8M0 scale-factor atom (MXFP4).
 //   attn2: one CTA owns one 128-row query tile of one head and streams its
 //     visible 128-key tiles.  S is double-buffered in TMEM, so Q K^T of tile
 //     j+1 runs on the tensor pipe while the softmax of tile j runs on the SM
 //     cores:
-//   warpgroup 0 (88 registers per thread after setmaxnreg):
-//     warp 0   producer: Q once; per tile the K codes (3-stage ring) and the
-//              V' tile (2-stage ring) by TMA, and the tile's per-key K scales
-//              and V' factor r_t / v_ref into a 4-stage shared ring.
-//     warp 1   MMA issuer (one thread): S_b = Q K^T (kind::f8f6f4 / kind::i8)
-//              into TMEM buffer b = j % 2, and O += P' V' (kind::f16, A = P'
-//              read from TMEM where the softmax stored it over S_b).  QK(j+2)
-//              is issued right after PV(j); the tensor pipe runs them in
-//              order, so P'_b is consumed before S_b is rewritten.
-//   warpgroups 1 and 2 (208 registers per thread): the softmax, one thread
-//     per (query row, half of the 128 keys): S from TMEM, per-key K scale,
-//     mask, the tile's row maximum combined across the two halves through
-//     shared memory, online max in the exp2 domain (O rescaled in TMEM only
-//     when the max grows by more than 2^8), p = exp2(t * c - m), and
-//     P' = fp16(p * r_t / v_ref) (the factor enters the exponent; the row sum
-//     takes p itself) stored over the half's own S columns (tcgen05.st).
-// TMEM: S_0/P'_0, S_1/P'_1, O (384 of 512 columns).  Every wait is bounded.
+//   warpgroup 0 (setmaxnreg shrinks it):
+//     warp 0   Q once, then per tile the K codes (3-stage ring), by TMA.
+//     warp 3   per tile the V' tile (2-stage ring), by TMA.
+//     warp 2   per tile the K scales (or atom) and the V' factor record into a
+//              4-stage shared ring by bulk copies; MXFP4: Q's scale atom.
+//     warp 1   MMA issuer (one thread): S_b = Q K^T (kind::f8f6f4 / kind::i8 /
+//              kind::mxf4 with the 32-element block scales copied into TMEM
+//              beside the accumulators) into TMEM buffer b = j % 2, and
+//              O += P' V' (kind::f16, A = P' read from TMEM where the softmax
+//              stored it over S_b).  QK(j+2) is issued right after PV(j); the
+//              tensor pipe runs them in order, so P'_b is consumed before S_b
+//              is rewritten.
+//   NSW softmax warpgroups (setmaxnreg grows them): one thread per (query row,
+//     128 / NSW keys of the tile): S from TMEM, per-key K scale, mask, the
+//     tile's row maximum combined across the groups through shared memory,
+//     online max in the exp2 domain (O rescaled in TMEM only when the max grows
+//     by more than 2^8), p = exp2(t * c - m), and P' = fp16(p * r_t / v_ref)
+//     (the factor enters the exponent; the row sum takes p itself) stored over
+//     the group's own S columns (tcgen05.st).
+// TMEM: S_0/P'_0, S_1/P'_1, O, and for MXFP4 the Q and K scale factors.
+// Every wait is bounded.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <math.h>
@@ -58,7 +65,7 @@ constexpr int NKS = 3;      // K code stages
 constexpr int NVS = 2;      // V' stages
 constexpr int NSC = 4;      // scale ring stages
 
-enum { K_E4M3 = 0, K_S8 = 1 };
+enum { K_E4M3 = 0, K_S8 = 1, K_MXF4 = 2 };
 enum { SC_HEAD = 0, SC_COL = 1, SC_TILE = 2 };  // one scale per head / per key / per 128-key tile
 
 struct P2 {
@@ -67,8 +74,11 @@ struct P2 {
   const float* qs;
   const float* ks;
   const float* vs;
-  const float* ksp;   // [B, Hkv, ntiles * 128] per-key K scales, zero past Sk (FP8 operands)
-  const float4* fvr;  // [B, Hkv, ntiles] V' tile factor records {r_t, 0, 0, 0} (FP8 operands)
+  const float* ksp;   // [B, Hkv, ntiles] x 512 B: per-key K scales, zero past Sk (E4M3) / UE8M0 atom (MXFP4)
+  const float4* fvr;  // [B, Hkv, ntiles] V' tile factor records {r_t, 0, 0, 0} (E4M3) / {E_t, 0, 0, 0} (MXFP4)
+  const uint8_t* qe8; // MXFP4 UE8M0 scales [B, H, S, D / 32]
+  const uint8_t* ke8;
+  const uint8_t* ve8;
   int q_blk, k_blk, v_blk, q_nblk, k_nblk, v_nblk;
   int ntiles_k;
   __nv_bfloat16* out;
@@ -77,16 +87,18 @@ struct P2 {
   int n_qtiles;
 };
 
-template <int D>
+template <int KIND, int D>
 struct L2 {
-  static constexpr uint32_t Q = 0;                   // [128][D]
-  static constexpr uint32_t K = Q + BM * D;            // NKS stages
-  static constexpr uint32_t VH = K + NKS * BN * D;     // NVS stages of fp16 V'
+  static constexpr uint32_t RB = KIND == K_MXF4 ? D / 2 : D;  // code bytes per token row
+  static constexpr uint32_t Q = 0;                     // [128][RB]
+  static constexpr uint32_t K = Q + BM * RB;           // NKS stages
+  static constexpr uint32_t VH = K + NKS * BN * RB;    // NVS stages of fp16 V'
   static constexpr uint32_t SC = VH + NVS * BN * D * 2;  // NSC stages x ([128] k scale, V' factor log2, its inverse)
   static constexpr uint32_t XM = SC + NSC * 2 * BN * 4;  // 2 stages x 4 key groups x [128] tile row max
   static constexpr uint32_t XL = XM + 2 * 4 * BM * 4;    // 4 key groups x [128] row sum
   static constexpr uint32_t MISC = XL + 4 * BM * 4;
-  static constexpr uint32_t BAR = MISC + 64;
+  static constexpr uint32_t SFA = MISC + 64;           // MXFP4: Q scale-factor atom (512 B)
+  static constexpr uint32_t BAR = SFA + 512;
   static constexpr uint32_t TOTAL = BAR + 512;
   static constexpr uint32_t ALLOC = TOTAL + 1024;
   static_assert(ALLOC <= 227 * 1024, "shared memory per CTA");
@@ -120,8 +132,11 @@ template <int KIND, int D, int SC, int NSW>
 __global__ void __launch_bounds__(Cfg<NSW>::NT, 1)
     attn2_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
                  const __grid_constant__ CUtensorMap tmv, const P2 p) {
-  static_assert(KIND == K_E4M3 || SC == SC_HEAD, "INT8 operands carry one scale per head");
-  using L = L2<D>;
+  static_assert(KIND == K_E4M3 || SC == SC_HEAD, "INT8 and MXFP4 operands take no per-key scale path");
+  constexpr bool MX = KIND == K_MXF4;
+  constexpr bool RING = MX || SC != SC_HEAD;  // per-tile records (and K scales / atoms) through the scale ring
+  using L = L2<KIND, D>;
+  constexpr uint32_t RB = L::RB;
   constexpr int HN = Cfg<NSW>::HN;
   constexpr int NSWW = 4 * NSW;   // softmax warps
   constexpr int DC = D / NSW;     // O columns per softmax thread
@@ -130,7 +145,7 @@ __global__ void __launch_bounds__(Cfg<NSW>::NT, 1)
   uint64_t* bar = reinterpret_cast<uint64_t*>(smem + L::BAR);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar + X_COUNT);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(bar + X_COUNT + 1);
-  float* misc = reinterpret_cast<float*>(smem + L::MISC);  // [0] = v_ref
+  float* misc = reinterpret_cast<float*>(smem + L::MISC);  // [0] = v_ref (MXFP4: E_ref)
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
@@ -153,7 +168,7 @@ __global__ void __launch_bounds__(Cfg<NSW>::NT, 1)
   const int bhk = b * p.Hkv + hk;
 
   if (tid == 0) {
-    mbar_init(&bar[X_Q], 1);
+    mbar_init(&bar[X_Q], MX ? 2 : 1);  // MXFP4: the Q codes and the Q scale-factor atom
     for (int i = 0; i < NKS; ++i) {
       mbar_init(&bar[X_KF + i], 1);
       mbar_init(&bar[X_KE + i], 1);
@@ -185,6 +200,8 @@ __global__ void __launch_bounds__(Cfg<NSW>::NT, 1)
   tc_fence_after();
   const uint32_t tbase = *tmem_slot;
   const uint32_t tO = tbase + 256;
+  const uint32_t tSFA = tbase + 384;  // MXFP4 scale factors: Q, then K for S buffers 0 and 1
+  const uint32_t tSFB[2] = {tbase + 392, tbase + 400};
 
   if (warp < 4) {
     setmaxnreg_dec<Cfg<NSW>::R0>();
@@ -194,14 +211,14 @@ __global__ void __launch_bounds__(Cfg<NSW>::NT, 1)
       if (lane == 0 && n > 0) {
         tma_prefetch_desc(&tmq);
         tma_prefetch_desc(&tmk);
-        mbar_arrive_expect_tx(&bar[X_Q], BM * D);
+        mbar_arrive_expect_tx(&bar[X_Q], BM * RB);
         tma_load_4d(smem + L::Q, &tmq, &bar[X_Q], 0, bnsd ? q0 : hq, bnsd ? hq : q0, b);
         int j = 0;
         for (; j < n; ++j) {
           const int k0 = j * BN, ks = j % NKS;
           if (j >= NKS && !mbar_wait(&bar[X_KE + ks], ((j / NKS) - 1) & 1, abort_flag, p.status, 61)) break;
-          mbar_arrive_expect_tx(&bar[X_KF + ks], BN * D);
-          tma_load_4d(smem + L::K + ks * BN * D, &tmk, &bar[X_KF + ks], 0, bnsd ? k0 : hk, bnsd ? hk : k0, b);
+          mbar_arrive_expect_tx(&bar[X_KF + ks], BN * RB);
+          tma_load_4d(smem + L::K + ks * BN * RB, &tmk, &bar[X_KF + ks], 0, bnsd ? k0 : hk, bnsd ? hk : k0, b);
         }
         if (*abort_flag) {
           // let issued loads land before the CTA can exit
@@ -230,16 +247,25 @@ __global__ void __launch_bounds__(Cfg<NSW>::NT, 1)
       __syncwarp();
     } else if (warp == 2) {
       // ------------------------------------------------------- scale ring
-      // Per tile, the pre-pass's 128 per-key K scales and the V' factor record land in a
-      // ring stage by two bulk copies (512 + 16 bytes) that complete on the stage's barrier.
-      if (SC != SC_HEAD && n > 0) {
+      // Per tile, the pre-pass's 128 per-key K scales (MXFP4: the K scale-factor atom) and
+      // the V' factor record land in a ring stage by two bulk copies (512 + 16 bytes) that
+      // complete on the stage's barrier.
+      if (MX && n > 0) {
+        // Q's scale-factor atom, published with the Q codes' barrier
+        write_sf_atom(smem + L::SFA, p.qe8, (long long)(b * p.Hq + hq) * p.Sq + q0, p.Sq - q0, lane);
+        fence_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bar[X_Q]);
+      }
+      if (RING && n > 0) {
         const float4* fvh = p.fvr + (long long)bhk * p.ntiles_k;
         float m = 0.0f;
         for (int t = lane; t < n; t += 32) m = fmaxf(m, __ldg(&fvh[t].x));
 #pragma unroll
         for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
         if (lane == 0) {
-          misc[0] = m > 0.0f ? m : 1.0f;  // v_ref: the largest V' factor over this CTA's visible tiles
+          // v_ref: the largest V' factor over this CTA's visible tiles (MXFP4: the largest E_t)
+          misc[0] = MX ? m : (m > 0.0f ? m : 1.0f);
           const float* kph = p.ksp + (long long)bhk * p.ntiles_k * BN;
           int j = 0;
           for (; j < n; ++j) {
@@ -258,22 +284,28 @@ __global__ void __launch_bounds__(Cfg<NSW>::NT, 1)
     } else if (warp == 1) {
       // ---------------------------------------------------------- MMA issuer
       if (lane == 0 && n > 0) {
-        constexpr uint32_t SW = D == 128 ? kSwz128 : kSwz64;
-        constexpr uint32_t SBO8 = D == 128 ? 1024 : 512;
+        constexpr uint32_t SW = RB == 128 ? kSwz128 : kSwz64;
+        constexpr uint32_t SBO8 = RB == 128 ? 1024 : 512;
         constexpr uint32_t idesc_qk = KIND == K_E4M3 ? make_idesc(kAccF32, kFmtE4M3, kFmtE4M3, 0, 0, BN, BM)
                                                      : make_idesc(kAccS32, kFmtS8, kFmtS8, 0, 0, BN, BM);
+        static_assert(!MX || RB == 64, "MXFP4 path: head_dim 128");
         constexpr uint32_t idesc_pv = make_idesc(kAccF32, kFmtF16, kFmtF16, 0, 1, D, BM);
         const uint32_t sQ = smem_u32(smem + L::Q);
         auto qk = [&](int j) {
-          const uint32_t sK = smem_u32(smem + L::K + (j % NKS) * BN * D);
+          const uint32_t sK = smem_u32(smem + L::K + (j % NKS) * BN * RB);
+          // MXFP4: the tile's K scale factors into TMEM, ordered before the MMAs that read them
+          if (MX) sf_to_tmem(tSFB[j & 1], smem_u32(smem + L::SC + (j % NSC) * 2 * BN * 4));
 #pragma unroll
-          for (int kk = 0; kk < D / 32; ++kk) {
+          for (int kk = 0; kk < (int)RB / 32; ++kk) {
             const uint64_t da = make_sdesc(sQ + kk * 32, 16, SBO8, SW);
             const uint64_t db = make_sdesc(sK + kk * 32, 16, SBO8, SW);
             if (KIND == K_E4M3)
               mma_f8f6f4(tbase + (j & 1) * 128, da, db, idesc_qk, kk > 0);
-            else
+            else if (KIND == K_S8)
               mma_i8(tbase + (j & 1) * 128, da, db, idesc_qk, kk > 0);
+            else  // 64 E2M1 per MMA: scale bytes 2kk and 2kk + 1 of each row
+              mma_mxf4(tbase + (j & 1) * 128, da, db, make_idesc_bs(kFmtE2M1x, kFmtE2M1x, BN, BM, 2 * kk, 2 * kk),
+                       tSFA, tSFB[j & 1], kk > 0);
           }
           mma_commit(&bar[X_SF + (j & 1)]);
           mma_commit(&bar[X_KE + j % NKS]);
@@ -292,9 +324,17 @@ __global__ void __launch_bounds__(Cfg<NSW>::NT, 1)
           mma_commit(&bar[X_PVD]);
           mma_commit(&bar[X_VE + j % NVS]);
         };
+        // MXFP4: QK(j) also needs the tile's scale-factor atom in its scale ring stage
+        auto sf_ready = [&](int j) {
+          return !MX || mbar_wait(&bar[X_SCF + j % NSC], (j / NSC) & 1, abort_flag, p.status, 68);
+        };
         bool ok = mbar_wait(&bar[X_Q], 0, abort_flag, p.status, 63);
+        if (MX && ok) {
+          tc_fence_after();
+          sf_to_tmem(tSFA, smem_u32(smem + L::SFA));
+        }
         for (int j = 0; ok && j < 2 && j < n; ++j) {
-          ok = mbar_wait(&bar[X_KF + j], 0, abort_flag, p.status, 64);
+          ok = mbar_wait(&bar[X_KF + j], 0, abort_flag, p.status, 64) && sf_ready(j);
           if (ok) {
             tc_fence_after();
             qk(j);
@@ -307,7 +347,7 @@ __global__ void __launch_bounds__(Cfg<NSW>::NT, 1)
           tc_fence_after();
           pv(j);
           if (j + 2 < n) {
-            ok = mbar_wait(&bar[X_KF + (j + 2) % NKS], ((j + 2) / NKS) & 1, abort_flag, p.status, 67);
+            ok = mbar_wait(&bar[X_KF + (j + 2) % NKS], ((j + 2) / NKS) & 1, abort_flag, p.status, 67) && sf_ready(j + 2);
             if (!ok) break;
             tc_fence_after();
             qk(j + 2);
@@ -330,12 +370,13 @@ __global__ void __launch_bounds__(Cfg<NSW>::NT, 1)
     const int qbh = b * p.Hq + hq;
     float* xm = reinterpret_cast<float*>(smem + L::XM);
     float* xl = reinterpret_cast<float*>(smem + L::XL);
-    const float sq = row_ok ? scale_at(p.qs, p.q_blk, p.q_nblk, qbh, hq, row) : 0.0f;
+    // MXFP4: the block scales are applied inside the MMA, so only the softmax scale
+    const float sq = MX ? 1.0f : (row_ok ? scale_at(p.qs, p.q_blk, p.q_nblk, qbh, hq, row) : 0.0f);
     float crow = sq * p.scale_log2;
-    if (SC == SC_HEAD) crow *= __ldg(p.ks + hk);
+    if (!RING) crow *= __ldg(p.ks + hk);
     // S8 accumulators arrive biased: t = float(0x4B400000 + acc) = 1.5 * 2^23 + acc (exact, |acc| < 2^22)
     constexpr float kBias = KIND == K_S8 ? 12582912.0f : 0.0f;
-    float vref = SC == SC_HEAD ? __ldg(p.vs + hk) : 1.0f;
+    float vref = RING ? 1.0f : __ldg(p.vs + hk);
     float m_run = -INFINITY, l_run = 0.0f;
     bool ok = true;
     for (int j = 0; j < n && ok; ++j) {
@@ -343,8 +384,8 @@ __global__ void __launch_bounds__(Cfg<NSW>::NT, 1)
       const uint32_t tS = tbase + st * 128 + cb;
       const int sst = j % NSC;
       const float* ksc = reinterpret_cast<const float*>(smem + L::SC + sst * 2 * BN * 4);
-      if (SC != SC_HEAD && !warp_wait(&bar[X_SCF + sst], (j / NSC) & 1, abort_flag, p.status, 70)) { ok = false; break; }
-      if (SC != SC_HEAD && j == 0) vref = misc[0];
+      if (RING && !warp_wait(&bar[X_SCF + sst], (j / NSC) & 1, abort_flag, p.status, 70)) { ok = false; break; }
+      if (RING && j == 0) vref = misc[0];
       // this tile's K scales and V' factor, loaded while S is still being computed
       float4 kk4[HN / 4];
       if (SC == SC_COL) {
@@ -352,10 +393,11 @@ __global__ void __launch_bounds__(Cfg<NSW>::NT, 1)
         for (int k = 0; k < HN; k += 4) kk4[k / 4] = *reinterpret_cast<const float4*>(ksc + cb + k);
       }
       float flog = 0.0f, finv = 1.0f, ktile = 1.0f;
-      if (SC != SC_HEAD) {
+      if (RING) {
         // V' factor r_t / v_ref enters the exponent as its log2, floored at -60 (a tile that
-        // small adds nothing visible to O); the row sum divides it back out.
-        flog = fmaxf(__log2f(ksc[BN] / vref), -60.0f);
+        // small adds nothing visible to O); the row sum divides it back out.  MXFP4: the
+        // factor is 2^(E_t - E_ref), its log2 an exact integer.
+        flog = fmaxf(MX ? ksc[BN] - vref : __log2f(ksc[BN] / vref), -60.0f);
         finv = ex2(-flog);
       }
       if (SC == SC_TILE) ktile = ksc[0];
@@ -505,7 +547,7 @@ __global__ void __launch_bounds__(Cfg<NSW>::NT, 1)
       __syncwarp();
       if (lane == 0) {
         mbar_arrive(&bar[X_PF + st]);
-        if (SC != SC_HEAD) mbar_arrive(&bar[X_SCE + sst]);
+        if (RING) mbar_arrive(&bar[X_SCE + sst]);
       }
     }
     // ---------------------------------------------------------- epilogue
@@ -524,7 +566,9 @@ __global__ void __launch_bounds__(Cfg<NSW>::NT, 1)
       for (int g = 0; g < NSW; ++g) l_tot += xl[g * BM + i];
     }
     if (q0 < p.Sq) {
-      const float ofac = l_tot > 0.0f ? vref / l_tot : 0.0f;
+      // MXFP4: V' was divided by 2^(E_ref - 127)
+      const float vmul = MX ? exp2f(vref - 127.0f) : vref;
+      const float ofac = l_tot > 0.0f ? vmul / l_tot : 0.0f;
       __nv_bfloat16* orow = nullptr;
       if (row_ok) {
         const long long ridx = p.layout == FA_LAYOUT_BNSD ? ((long long)qbh * p.Sq + row)
@@ -576,13 +620,14 @@ __global__ void __launch_bounds__(Cfg<NSW>::NT, 1)
 // ---- V pre-pass: one CTA per (128-token tile, b * Hkv + h).
 // E4M3: r_t = max s_v over the tile's tokens (1 if all are 0), V' = fp16(code * (s_v / r_t)), |V'| <= 448.
 // INT8: V' = fp16(code) exactly (the per-head scale stays outside).
+// MXFP4: E_t = the largest UE8M0 byte of the tile's tokens, V' = fp16(e2m1 * 2^(e - E_t)), |V'| <= 6.
 template <int KIND, int D>
 __global__ void __launch_bounds__(256) vprep_kernel(const uint8_t* __restrict__ codes, const float* __restrict__ vs,
                                                     int v_blk, int v_nblk, int H, int S, int layout,
                                                     __half* __restrict__ vh, float4* __restrict__ fvr, int ntiles,
                                                     const float* __restrict__ ks, int k_blk, int k_nblk,
-                                                    float* __restrict__ ksp) {
-  constexpr int CPT = D / 32;  // 16-code chunks per thread: each thread owns half a token row
+                                                    float* __restrict__ ksp, const uint8_t* __restrict__ ve8,
+                                                    const uint8_t* __restrict__ ke8) {
   const int t = blockIdx.x, bh = blockIdx.y;
   const int b = bh / H, h = bh % H;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -590,6 +635,54 @@ __global__ void __launch_bounds__(256) vprep_kernel(const uint8_t* __restrict__ 
   const int tok = tok0 + warp * 16 + (lane >> 1);
   const bool live = tok < S;  // rows past S stay unwritten: the attention's TMA box reads them as zero
   const long long src_row = layout == FA_LAYOUT_BNSD ? ((long long)bh * S + tok) : (((long long)b * S + tok) * H + h);
+  if constexpr (KIND == K_MXF4) {
+    static_assert(D == 128, "MXFP4 path: head_dim 128");
+    // each thread owns half a 64-byte code row: two 32-element scale blocks of 16 bytes
+    const uint8_t* src = codes + src_row * (D / 2) + (lane & 1) * (D / 4);
+    uint4 raw[2];
+#pragma unroll
+    for (int c = 0; c < 2; ++c) raw[c] = live ? __ldg(reinterpret_cast<const uint4*>(src) + c) : make_uint4(0, 0, 0, 0);
+    const uint32_t* ve4 = reinterpret_cast<const uint32_t*>(ve8) + (long long)bh * S;
+    int m = 0;  // E_t, reduced by every warp itself
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const int tt = tok0 + lane * 4 + q;
+      if (tt < S) {
+        const uint32_t w = __ldg(ve4 + tt);
+        m = max(m, (int)max(max(w & 0xFFu, (w >> 8) & 0xFFu), max((w >> 16) & 0xFFu, w >> 24)));
+      }
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, off));
+    if (threadIdx.x == 0) fvr[(long long)bh * ntiles + t] = make_float4((float)m, 0.0f, 0.0f, 0.0f);
+    // the K tile's scale-factor atom: token row r at byte (r % 32) * 16 + (r / 32) * 4, zero past S
+    if (threadIdx.x < BN) {
+      const int key = tok0 + threadIdx.x;
+      const uint32_t w = key < S ? __ldg(reinterpret_cast<const uint32_t*>(ke8) + (long long)bh * S + key) : 0u;
+      reinterpret_cast<uint32_t*>(ksp + ((long long)bh * ntiles + t) * BN)[(threadIdx.x & 31) * 4 + (threadIdx.x >> 5)] = w;
+    }
+    if (!live) return;
+    const uint32_t e4 = __ldg(ve4 + tok);
+    uint4* dst = reinterpret_cast<uint4*>(vh + ((long long)bh * S + tok) * D + (lane & 1) * (D / 2));
+#pragma unroll
+    for (int c = 0; c < 2; ++c) {
+      const int de = (int)((e4 >> (8 * ((lane & 1) * 2 + c))) & 0xFFu) - m;  // <= 0
+      const __half fs = de >= -24 ? __float2half_rn(ldexpf(1.0f, de)) : __float2half_rn(0.0f);
+      const __half2 f2 = __halves2half2(fs, fs);
+      const uint32_t w[4] = {raw[c].x, raw[c].y, raw[c].z, raw[c].w};
+      uint32_t o[16];  // byte i holds elements 2i (low nibble) and 2i + 1
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        const uint32_t v2 = e2m1x2_to_h2((w[i >> 2] >> (8 * (i & 3))) & 0xFFu);
+        const __half2 y = __hmul2(*reinterpret_cast<const __half2*>(&v2), f2);
+        o[i] = *reinterpret_cast<const uint32_t*>(&y);
+      }
+#pragma unroll
+      for (int q = 0; q < 4; ++q) dst[4 * c + q] = make_uint4(o[4 * q], o[4 * q + 1], o[4 * q + 2], o[4 * q + 3]);
+    }
+    return;
+  }
+  constexpr int CPT = D / 32;  // 16-code chunks per thread: each thread owns half a token row
   const uint8_t* src = codes + src_row * D + (lane & 1) * (D / 2);
   uint4 raw[CPT];
 #pragma unroll
@@ -684,17 +777,18 @@ Prefill2Ws carve_ws(void* ws, int B, int Hkv, int Sk, int D) {
 template <int KIND, int D, int SC>
 cudaError_t launch2(const AttnArgs& a, const P2& prm, const Prefill2Ws& w, cudaStream_t s) {
   constexpr int NSW = FAQ_ATTN_NSW;
-  using L = L2<D>;
+  using L = L2<KIND, D>;
   CUtensorMap mq, mk, mv;
   cudaError_t e;
-  if ((e = make_code_map(&mq, a.q->codes, a.q->B, a.q->H, a.q->S, D, a.q->layout, BM)) != cudaSuccess) return e;
-  if ((e = make_code_map(&mk, a.k->codes, a.k->B, a.k->H, a.k->S, D, a.k->layout, BN)) != cudaSuccess) return e;
+  const int RB = (int)L::RB;
+  if ((e = make_code_map(&mq, a.q->codes, a.q->B, a.q->H, a.q->S, RB, a.q->layout, BM)) != cudaSuccess) return e;
+  if ((e = make_code_map(&mk, a.k->codes, a.k->B, a.k->H, a.k->S, RB, a.k->layout, BN)) != cudaSuccess) return e;
   if ((e = make_vh_map(&mv, w.vh, a.v->B, a.v->H, a.v->S, D)) != cudaSuccess) return e;
   const dim3 pgrid((unsigned)prm.ntiles_k, (unsigned)(a.v->B * a.v->H));
   if (pgrid.y > 65535u) return cudaErrorInvalidValue;
   vprep_kernel<KIND, D><<<pgrid, 256, 0, s>>>(static_cast<const uint8_t*>(a.v->codes), prm.vs, prm.v_blk,
                                                prm.v_nblk, a.v->H, a.v->S, a.v->layout, w.vh, w.fvr, prm.ntiles_k,
-                                               prm.ks, prm.k_blk, prm.k_nblk, w.ksp);
+                                               prm.ks, prm.k_blk, prm.k_nblk, w.ksp, prm.ve8, prm.ke8);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   auto kern = attn2_kernel<KIND, D, SC, NSW>;
   static bool attr_set = false;
@@ -729,7 +823,7 @@ void scale_desc2(const fa_qtensor* t, int& blk, int& nblk) {
 
 }  // namespace
 
-// Prefill attention for E4M3 and INT8 operands.
+// Prefill attention for E4M3, INT8 and MXFP4 operands.
 size_t prefill2_workspace_bytes(int B, int Hkv, int Sk, int D) {
   const size_t ntiles = ((size_t)Sk + BN - 1) / BN;
   return align256((size_t)B * Hkv * Sk * D * 2) + align256((size_t)B * Hkv * ntiles * 16) +
@@ -767,6 +861,12 @@ cudaError_t launch_attention_prefill2(const AttnArgs& a, void* ws, cudaStream_t 
       return q->D == 128 ? launch2_sc<K_E4M3, 128>(a, prm, w, sc, s) : launch2_sc<K_E4M3, 64>(a, prm, w, sc, s);
     case FA_MODE_INT8_PER_HEAD:
       return q->D == 128 ? launch2<K_S8, 128, SC_HEAD>(a, prm, w, s) : launch2<K_S8, 64, SC_HEAD>(a, prm, w, s);
+    case FA_MODE_MXFP4_PER_BLOCK:
+      if (q->D != 128) return cudaErrorNotSupported;
+      prm.qe8 = static_cast<const uint8_t*>(q->scales);
+      prm.ke8 = static_cast<const uint8_t*>(k->scales);
+      prm.ve8 = static_cast<const uint8_t*>(a.v->scales);
+      return launch2<K_MXF4, 128, SC_HEAD>(a, prm, w, s);
     default:
       return cudaErrorNotSupported;
   }

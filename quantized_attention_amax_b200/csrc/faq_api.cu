@@ -245,6 +245,10 @@ size_t fa_attention_workspace_size(const fa_qtensor* q, const fa_qtensor* k, int
     if (k->B < 0 || k->S < 0 || (q->D != 64 && q->D != 128)) return 0;
     return prefill2_workspace_bytes(k->B, k->H, k->S, q->D);
   }
+  if (q->mode == FA_MODE_MXFP4_PER_BLOCK) {
+    if (k->B < 0 || k->S < 0 || q->D != 128) return 0;
+    return prefill2_workspace_bytes(k->B, k->H, k->S, q->D);
+  }
   return 0;
 }
 
@@ -268,8 +272,9 @@ fa_status fa_attention_quant(const fa_qtensor* q, const fa_qtensor* k, const fa_
   if (!out || !aligned16(out)) return FA_ERR_INVALID_ARG;
   if (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)) return FA_ERR_INVALID_ARG;
   const bool decode = is_decode(q, k);
+  if (q->mode == FA_MODE_MXFP4_PER_BLOCK && q->D != 128) return FA_ERR_UNSUPPORTED;
   const int splits = decode ? (num_splits > 0 ? num_splits : decode_auto_splits(k->B, k->H, k->S)) : 0;
-  if (k->S > 0 && q->mode != FA_MODE_MXFP4_PER_BLOCK) {
+  if (k->S > 0) {
     const size_t need = decode ? decode_workspace_bytes(q->B, q->H, q->D, splits)
                                : prefill2_workspace_bytes(k->B, k->H, k->S, q->D);
     if (!workspace || ws_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255u)) return FA_ERR_WORKSPACE;
@@ -282,8 +287,6 @@ fa_status fa_attention_quant(const fa_qtensor* q, const fa_qtensor* k, const fa_
   cudaError_t e;
   if (decode)
     e = launch_attention_decode(a, splits, workspace, cs);
-  else if (q->mode == FA_MODE_MXFP4_PER_BLOCK)
-    e = launch_attention_prefill(a, cs);
   else
     e = launch_attention_prefill2(a, workspace, cs);
   if (e == cudaErrorNotSupported) return FA_ERR_UNSUPPORTED;

@@ -130,7 +130,7 @@ def test_attention_validation_before_launch(N):
     assert L.fa_attention_quant(by(qd), by(kd), by(kd), 0, 0.0, 0x60000, None, 0, 0x70000, need - 16,
                                 None) == 7
     assert L.fa_attention_quant(by(qd), by(kd), by(kd), 0, 0.0, 0x60000, None, -1, None, 0, None) == 1
-    # FP8 / INT8 prefill: fp16 V', a 16-byte factor record and 128 K scales per 128-key tile,
+    # prefill: fp16 V', a 16-byte factor record and 512 bytes of K scales per 128-key tile,
     # each part 256-byte aligned
     qp = _q(N, 1, B=2, H=4, S=100, D=128)
     need_p = L.fa_attention_workspace_size(by(qp), by(kd), 0)
@@ -142,7 +142,11 @@ def test_attention_validation_before_launch(N):
                                 None) == 7
     assert L.fa_attention_quant(by(qp), by(kd), by(kd), 0, 0.0, 0x60000, None, 0, 0x70010, need_p,
                                 None) == 7  # workspace not 256-byte aligned
-    # MXFP4 prefill needs none
+    # MXFP4 prefill: the same parts (its K scales are the tile's scale-factor atom); head_dim 128 only
     qm = _q(N, 3, B=2, H=4, S=100, D=128)
     km = _q(N, 3, B=2, H=2, S=1000, D=128)
-    assert L.fa_attention_workspace_size(by(qm), by(km), 0) == 0
+    assert L.fa_attention_workspace_size(by(qm), by(km), 0) == need_p
+    assert L.fa_attention_quant(by(qm), by(km), by(km), 0, 0.0, 0x60000, None, 0, None, 0, None) == 7
+    qm64, km64 = _q(N, 3, B=2, H=4, S=100, D=64), _q(N, 3, B=2, H=2, S=1000, D=64)
+    assert L.fa_attention_workspace_size(by(qm64), by(km64), 0) == 0
+    assert L.fa_attention_quant(by(qm64), by(km64), by(km64), 0, 0.0, 0x60000, None, 0, None, 0, None) == 2
