@@ -812,6 +812,15 @@ cudaError_t launch2_sc(const AttnArgs& a, const P2& prm, const Prefill2Ws& w, in
   }
 }
 
+// Rows with no key (Sk == 0): output 0, LSE -inf.
+__global__ void fill_empty_kernel(__nv_bfloat16* out, float* lse, long long rows, int D) {
+  const long long n = rows * D;
+  const long long stride = (long long)gridDim.x * blockDim.x;
+  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += stride) out[i] = __float2bfloat16(0.0f);
+  if (lse)
+    for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < rows; i += stride) lse[i] = -INFINITY;
+}
+
 void scale_desc2(const fa_qtensor* t, int& blk, int& nblk) {
   switch (t->mode) {
     case FA_MODE_INT8_PER_HEAD: blk = 0; nblk = 1; break;
@@ -870,6 +879,15 @@ cudaError_t launch_attention_prefill2(const AttnArgs& a, void* ws, cudaStream_t 
     default:
       return cudaErrorNotSupported;
   }
+}
+
+cudaError_t launch_fill_empty_rows(void* out, float* lse, long long rows, int D, cudaStream_t s) {
+  const long long n = rows * D;
+  int grid = (int)((n + 255) / 256);
+  if (grid > 4096) grid = 4096;
+  if (grid < 1) grid = 1;
+  fill_empty_kernel<<<grid, 256, 0, s>>>(static_cast<__nv_bfloat16*>(out), lse, rows, D);
+  return cudaGetLastError();
 }
 
 }  // namespace faq

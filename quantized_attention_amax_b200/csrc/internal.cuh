@@ -49,7 +49,7 @@ struct RotateOperand {
 };
 cudaError_t launch_rotate_block_quant(const RotateOperand* ops, int nops, int* status, cudaStream_t s);
 
-// Launchers (attn.cu / decode.cu).
+// Launchers (attn2.cu / decode.cu).
 struct AttnArgs {
   const fa_qtensor* q;
   const fa_qtensor* k;
@@ -60,8 +60,7 @@ struct AttnArgs {
   float* lse;
   int* status;
 };
-cudaError_t launch_attention_prefill(const AttnArgs& a, cudaStream_t s);
-// FP8 / INT8 prefill: V' pre-pass + attention; `ws` holds prefill2_workspace_bytes().
+// Prefill (E4M3, INT8, MXFP4): V' pre-pass + attention; `ws` holds prefill2_workspace_bytes().
 size_t prefill2_workspace_bytes(int B, int Hkv, int Sk, int D);
 cudaError_t launch_attention_prefill2(const AttnArgs& a, void* ws, cudaStream_t s);
 
