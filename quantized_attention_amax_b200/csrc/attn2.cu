@@ -85,6 +85,7 @@ struct P2 {
   float* lse;
   int* status;
   int n_qtiles;
+  int pair_heads;  // two-tile kernel: 1 = the two tiles are query heads 2h, 2h+1 at one row block, 0 = row blocks 2t, 2t+1 of one head
 };
 
 template <int KIND, int D>
@@ -617,6 +618,453 @@ __global__ void __launch_bounds__(Cfg<NSW>::NT, 1)
   }
 }
 
+
+// ---- two query tiles per CTA (E4M3 / INT8) ------------------------------
+// One CTA owns two 128-row query tiles A and B that read the same K / V' tiles
+// (query heads 2h, 2h+1 of one kv head, or row blocks 2t, 2t+1 of one head),
+// with one S and one O accumulator each in TMEM (S_A, S_B, O_A, O_B = 512
+// columns for D = 128).  Each tile has its own softmax warpgroup, one thread
+// per query row holding the row's 128 scores, so the row maximum needs no
+// exchange between threads.  The MMA thread alternates the tiles:
+//   QK_A(0) QK_B(0) | PV_A(0) QK_A(1) PV_B(0) QK_B(1) | PV_A(1) QK_A(2) ...
+// so while one warpgroup runs the softmax of tile j, the tensor pipe runs the
+// other tile's P V and next Q K^T.
+constexpr int PNT = 384;  // warpgroup 0 (loads, MMA, scale ring) + two softmax warpgroups
+constexpr int PR0 = 56;
+constexpr int PRS = 224;
+static_assert(128 * PR0 + 256 * PRS <= PNT * ((65536 / PNT) & ~7), "register split exceeds the launch");
+
+template <int D>
+struct LP {
+  static constexpr uint32_t Q = 0;                       // 2 x [128][D]
+  static constexpr uint32_t K = Q + 2 * BM * D;          // NKS stages
+  static constexpr uint32_t VH = K + NKS * BN * D;       // NVS stages of fp16 V'
+  static constexpr uint32_t SC = VH + NVS * BN * D * 2;  // NSC stages x ([128] K scales, V' factor record)
+  static constexpr uint32_t MISC = SC + NSC * 2 * BN * 4;
+  static constexpr uint32_t BAR = MISC + 64;
+  static constexpr uint32_t TOTAL = BAR + 512;
+  static constexpr uint32_t ALLOC = TOTAL + 1024;
+  static_assert(ALLOC <= 227 * 1024, "shared memory per CTA");
+  static_assert(VH % 1024 == 0, "V' stages need 1024-byte alignment for the 128-byte swizzle");
+};
+
+enum {
+  Y_Q = 0,
+  Y_KF = 1,              // [NKS]
+  Y_KE = Y_KF + NKS,     // [NKS]
+  Y_VF = Y_KE + NKS,     // [NVS]
+  Y_VE = Y_VF + NVS,     // [NVS]
+  Y_SF = Y_VE + NVS,     // [2] S_A / S_B full
+  Y_PF = Y_SF + 2,       // [2] P'_A / P'_B stored
+  Y_PVD = Y_PF + 2,      // [2] P V of tile A / B done
+  Y_SCF = Y_PVD + 2,     // [NSC]
+  Y_SCE = Y_SCF + NSC,   // [NSC]
+  Y_FIN = Y_SCE + NSC,
+  Y_COUNT = Y_FIN + 1
+};
+static_assert(Y_COUNT * 8 + 8 <= 512, "barrier block overflows its region");
+
+template <int KIND, int D, int SC>
+__global__ void __launch_bounds__(PNT, 1)
+    attn_pair_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
+                     const __grid_constant__ CUtensorMap tmv, const P2 p) {
+  static_assert(KIND == K_E4M3 || (KIND == K_S8 && SC == SC_HEAD), "E4M3 or INT8 operands");
+  constexpr bool RING = SC != SC_HEAD;
+  using L = LP<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bar = reinterpret_cast<uint64_t*>(smem + L::BAR);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar + Y_COUNT);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(bar + Y_COUNT + 1);
+  float* misc = reinterpret_cast<float*>(smem + L::MISC);  // [0] = v_ref
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+
+  // ---- work item: batch b, the two tiles' query heads and first rows; heaviest first when causal
+  int b, hqt[2], q0t[2];
+  if (p.pair_heads) {
+    const int hp = p.Hq / 2, per_t = p.B * hp;
+    const int qt = p.causal ? (p.n_qtiles - 1 - (int)blockIdx.x / per_t) : ((int)blockIdx.x / per_t);
+    const int r = blockIdx.x % per_t;
+    b = r / hp;
+    hqt[0] = 2 * (r % hp);
+    hqt[1] = hqt[0] + 1;
+    q0t[0] = q0t[1] = qt * BM;
+  } else {
+    const int np = (p.n_qtiles + 1) / 2, per_t = p.B * p.Hq;
+    const int pt = p.causal ? (np - 1 - (int)blockIdx.x / per_t) : ((int)blockIdx.x / per_t);
+    const int r = blockIdx.x % per_t;
+    b = r / p.Hq;
+    hqt[0] = hqt[1] = r % p.Hq;
+    q0t[0] = 2 * pt * BM;
+    q0t[1] = q0t[0] + BM;
+  }
+  const int hk = hqt[0] / p.group;
+  const int diag = p.Sk - p.Sq;
+  int nt[2];
+#pragma unroll
+  for (int x = 0; x < 2; ++x) {
+    int kv_end = 0;
+    if (q0t[x] < p.Sq) kv_end = p.causal ? min(p.Sk, max(0, min(q0t[x] + BM, p.Sq) - 1 + diag + 1)) : p.Sk;
+    nt[x] = (kv_end + BN - 1) / BN;
+  }
+  const int n = max(nt[0], nt[1]);
+  const int bhk = b * p.Hkv + hk;
+
+  if (tid == 0) {
+    mbar_init(&bar[Y_Q], 1);
+    for (int i = 0; i < NKS; ++i) {
+      mbar_init(&bar[Y_KF + i], 1);
+      mbar_init(&bar[Y_KE + i], 1);
+    }
+    for (int i = 0; i < NVS; ++i) {
+      mbar_init(&bar[Y_VF + i], 1);
+      mbar_init(&bar[Y_VE + i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&bar[Y_SF + i], 1);
+      mbar_init(&bar[Y_PF + i], 4);
+      mbar_init(&bar[Y_PVD + i], 1);
+    }
+    for (int i = 0; i < NSC; ++i) {
+      mbar_init(&bar[Y_SCF + i], 1);
+      mbar_init(&bar[Y_SCE + i], 8);  // both softmax warpgroups
+    }
+    mbar_init(&bar[Y_FIN], 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tbase = *tmem_slot;  // S_A, S_B at columns 0, 128; O_A, O_B at 256, 256 + D
+
+  if (warp < 4) {
+    setmaxnreg_dec<PR0>();
+    const bool bnsd = p.layout == FA_LAYOUT_BNSD;
+    if (warp == 0) {
+      // ------------------------------------------------------ Q and K loads
+      if (lane == 0 && n > 0) {
+        tma_prefetch_desc(&tmq);
+        tma_prefetch_desc(&tmk);
+        mbar_arrive_expect_tx(&bar[Y_Q], ((nt[0] > 0) + (nt[1] > 0)) * BM * D);
+#pragma unroll
+        for (int x = 0; x < 2; ++x)
+          if (nt[x] > 0)
+            tma_load_4d(smem + L::Q + x * BM * D, &tmq, &bar[Y_Q], 0, bnsd ? q0t[x] : hqt[x], bnsd ? hqt[x] : q0t[x], b);
+        int j = 0;
+        for (; j < n; ++j) {
+          const int k0 = j * BN, ks = j % NKS;
+          if (j >= NKS && !mbar_wait(&bar[Y_KE + ks], ((j / NKS) - 1) & 1, abort_flag, p.status, 81)) break;
+          mbar_arrive_expect_tx(&bar[Y_KF + ks], BN * D);
+          tma_load_4d(smem + L::K + ks * BN * D, &tmk, &bar[Y_KF + ks], 0, bnsd ? k0 : hk, bnsd ? hk : k0, b);
+        }
+        if (*abort_flag) {
+          mbar_wait(&bar[Y_Q], 0, abort_flag, nullptr, 0);
+          for (int t = max(0, j - NKS); t < j; ++t) mbar_wait(&bar[Y_KF + t % NKS], (t / NKS) & 1, abort_flag, nullptr, 0);
+        }
+      }
+      __syncwarp();
+    } else if (warp == 3) {
+      // --------------------------------------------------------- V' loads
+      if (lane == 0 && n > 0) {
+        tma_prefetch_desc(&tmv);
+        int j = 0;
+        for (; j < n; ++j) {
+          const int k0 = j * BN, vs = j % NVS;
+          if (j >= NVS && !mbar_wait(&bar[Y_VE + vs], ((j / NVS) - 1) & 1, abort_flag, p.status, 82)) break;
+          mbar_arrive_expect_tx(&bar[Y_VF + vs], BN * D * 2);
+#pragma unroll
+          for (int a2 = 0; a2 < D / 64; ++a2)
+            tma_load_4d(smem + L::VH + vs * BN * D * 2 + a2 * BN * 128, &tmv, &bar[Y_VF + vs], 64 * a2, k0, hk, b);
+        }
+        if (*abort_flag)
+          for (int t = max(0, j - NVS); t < j; ++t) mbar_wait(&bar[Y_VF + t % NVS], (t / NVS) & 1, abort_flag, nullptr, 0);
+      }
+      __syncwarp();
+    } else if (warp == 2) {
+      // ------------------------------------------------------- scale ring
+      if (RING && n > 0) {
+        const float4* fvh = p.fvr + (long long)bhk * p.ntiles_k;
+        float m = 0.0f;
+        for (int t = lane; t < n; t += 32) m = fmaxf(m, __ldg(&fvh[t].x));
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+        if (lane == 0) {
+          misc[0] = m > 0.0f ? m : 1.0f;  // v_ref: the largest V' factor over this CTA's tiles
+          const float* kph = p.ksp + (long long)bhk * p.ntiles_k * BN;
+          int j = 0;
+          for (; j < n; ++j) {
+            const int st = j % NSC;
+            if (j >= NSC && !mbar_wait(&bar[Y_SCE + st], ((j / NSC) - 1) & 1, abort_flag, p.status, 80)) break;
+            uint8_t* stage = smem + L::SC + st * 2 * BN * 4;
+            mbar_arrive_expect_tx(&bar[Y_SCF + st], BN * 4 + 16);
+            bulk_load(stage, kph + (long long)j * BN, BN * 4, &bar[Y_SCF + st]);
+            bulk_load(stage + BN * 4, fvh + j, 16, &bar[Y_SCF + st]);
+          }
+          if (*abort_flag)
+            for (int t = max(0, j - NSC); t < j; ++t) mbar_wait(&bar[Y_SCF + t % NSC], (t / NSC) & 1, abort_flag, nullptr, 0);
+        }
+      }
+      __syncwarp();
+    } else {
+      // ---------------------------------------------------------- MMA issuer
+      if (lane == 0 && n > 0) {
+        constexpr uint32_t SW = D == 128 ? kSwz128 : kSwz64;
+        constexpr uint32_t SBO8 = D == 128 ? 1024 : 512;
+        constexpr uint32_t idesc_qk = KIND == K_E4M3 ? make_idesc(kAccF32, kFmtE4M3, kFmtE4M3, 0, 0, BN, BM)
+                                                     : make_idesc(kAccS32, kFmtS8, kFmtS8, 0, 0, BN, BM);
+        constexpr uint32_t idesc_pv = make_idesc(kAccF32, kFmtF16, kFmtF16, 0, 1, D, BM);
+        auto qk = [&](int x, int j) {
+          const uint32_t sQ = smem_u32(smem + L::Q + x * BM * D);
+          const uint32_t sK = smem_u32(smem + L::K + (j % NKS) * BN * D);
+#pragma unroll
+          for (int kk = 0; kk < D / 32; ++kk) {
+            const uint64_t da = make_sdesc(sQ + kk * 32, 16, SBO8, SW);
+            const uint64_t db = make_sdesc(sK + kk * 32, 16, SBO8, SW);
+            if (KIND == K_E4M3)
+              mma_f8f6f4(tbase + x * 128, da, db, idesc_qk, kk > 0);
+            else
+              mma_i8(tbase + x * 128, da, db, idesc_qk, kk > 0);
+          }
+          mma_commit(&bar[Y_SF + x]);
+        };
+        auto pv = [&](int x, int j) {
+          // A = P' in TMEM: key k of the tile sits in column k / 2 of S_x (fp16 pairs)
+          const uint32_t sVh = smem_u32(smem + L::VH + (j % NVS) * BN * D * 2);
+#pragma unroll
+          for (int ks = 0; ks < BN / 16; ++ks) {
+            const uint64_t db = make_sdesc(sVh + ks * 16 * 128, BN * 128, 1024, kSwz128);
+            mma_f16_ts(tbase + 256 + x * D, tbase + x * 128 + ks * 8, db, idesc_pv, (j > 0 || ks > 0) ? 1u : 0u);
+          }
+          mma_commit(&bar[Y_PVD + x]);
+        };
+        bool ok = mbar_wait(&bar[Y_Q], 0, abort_flag, p.status, 83);
+        if (ok) ok = mbar_wait(&bar[Y_KF], 0, abort_flag, p.status, 84);
+        if (ok) {
+          tc_fence_after();
+          if (nt[0] > 0) qk(0, 0);
+          if (nt[1] > 0) qk(1, 0);
+          mma_commit(&bar[Y_KE]);
+        }
+        for (int j = 0; ok && j < n; ++j) {
+          bool v_ready = false, k_ready = false;
+#pragma unroll
+          for (int x = 0; x < 2 && ok; ++x) {
+            if (j >= nt[x]) continue;
+            ok = mbar_wait(&bar[Y_PF + x], j & 1, abort_flag, p.status, 85);
+            if (ok && !v_ready) ok = v_ready = mbar_wait(&bar[Y_VF + j % NVS], (j / NVS) & 1, abort_flag, p.status, 86);
+            if (!ok) break;
+            tc_fence_after();
+            pv(x, j);
+            if (j + 1 < nt[x]) {
+              if (!k_ready) ok = k_ready = mbar_wait(&bar[Y_KF + (j + 1) % NKS], ((j + 1) / NKS) & 1, abort_flag, p.status, 87);
+              if (!ok) break;
+              tc_fence_after();
+              qk(x, j + 1);
+            }
+          }
+          if (!ok) break;
+          mma_commit(&bar[Y_VE + j % NVS]);
+          if (j + 1 < n) mma_commit(&bar[Y_KE + (j + 1) % NKS]);
+        }
+        mma_commit(&bar[Y_FIN]);
+        mbar_wait(&bar[Y_FIN], 0, abort_flag, nullptr, 0);
+      }
+      __syncwarp();
+    }
+  } else {
+    setmaxnreg_inc<PRS>();
+    // ------------------------------------------------------------- softmax
+    const int x = (warp - 4) >> 2;  // query tile of this warpgroup
+    const int i = tid - 128 - x * 128;
+    const uint32_t loff = (uint32_t)((warp & 3) * 32) << 16;
+    const int hq = x ? hqt[1] : hqt[0], q0 = x ? q0t[1] : q0t[0], nx = x ? nt[1] : nt[0];
+    const int row = q0 + i;
+    const bool row_ok = row < p.Sq;
+    const int qbh = b * p.Hq + hq;
+    const uint32_t tS = tbase + x * 128;
+    const uint32_t tO = tbase + 256 + x * D;
+    const float sq = row_ok ? scale_at(p.qs, p.q_blk, p.q_nblk, qbh, hq, row) : 0.0f;
+    float crow = sq * p.scale_log2;
+    if (!RING) crow *= __ldg(p.ks + hk);
+    constexpr float kBias = KIND == K_S8 ? 12582912.0f : 0.0f;
+    float vref = RING ? 1.0f : __ldg(p.vs + hk);
+    float m_run = -INFINITY, l_run = 0.0f;
+    bool ok = true;
+    for (int j = 0; j < n && ok; ++j) {
+      const int k0 = j * BN;
+      const int sst = j % NSC;
+      const float* ksc = reinterpret_cast<const float*>(smem + L::SC + sst * 2 * BN * 4);
+      if (RING && !warp_wait(&bar[Y_SCF + sst], (j / NSC) & 1, abort_flag, p.status, 90)) { ok = false; break; }
+      if (RING && j == 0) vref = misc[0];
+      if (j >= nx) {
+        // the other tile's key range is longer: release the ring stage and move on
+        if (RING) {
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&bar[Y_SCE + sst]);
+        }
+        continue;
+      }
+      float flog = 0.0f, finv = 1.0f, cr = crow;
+      if (RING) {
+        flog = fmaxf(__log2f(ksc[BN] / vref), -60.0f);
+        finv = ex2(-flog);
+      }
+      if (SC == SC_TILE) cr *= ksc[0];
+      // the tile's per-key K scales into registers while S is still being computed
+      float ksr[SC == SC_COL ? BN : 1];
+      if (SC == SC_COL) {
+#pragma unroll
+        for (int k = 0; k < BN; k += 4) *reinterpret_cast<float4*>(&ksr[k]) = *reinterpret_cast<const float4*>(ksc + k);
+      }
+      if (!warp_wait(&bar[Y_SF + x], j & 1, abort_flag, p.status, 91)) { ok = false; break; }
+      tc_fence_after();
+      uint32_t tr[BN];
+      float t[BN];
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+#pragma unroll
+        for (int c = 0; c < BN / 64; ++c)
+          tmem_ld32(tS + loff + 64 * hh + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(&tr[64 * hh + 32 * c]));
+        tmem_ld_wait();
+#pragma unroll
+        for (int k = 64 * hh; k < 64 * hh + 64; ++k)
+          t[k] = KIND == K_S8 ? __uint_as_float(0x4B400000u + tr[k]) : __uint_as_float(tr[k]);
+        if (SC == SC_COL) {
+#pragma unroll
+          for (int k = 64 * hh; k < 64 * hh + 64; k += 2) fmul2(t[k], t[k + 1], ksr[k], ksr[k + 1]);
+        }
+      }
+      const bool need_mask = (k0 + BN > p.Sk) || (p.causal && (k0 + BN - 1 > q0 + diag));
+      if (need_mask) {
+        const int lim = p.causal ? min(p.Sk - 1, row + diag) : p.Sk - 1;
+#pragma unroll
+        for (int k = 0; k < BN; ++k)
+          if (k0 + k > lim) t[k] = -INFINITY;
+      }
+      // row maximum: eight chains of three-input maxima
+      float mx[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        mx[e] = t[e];
+#pragma unroll
+        for (int q = 1; q < BN / 8; q += 2)
+          mx[e] = q + 1 < BN / 8 ? fmax3(mx[e], t[e + 8 * q], t[e + 8 * q + 8]) : fmaxf(mx[e], t[e + 8 * q]);
+      }
+      const float mt = fmax3(fmax3(mx[0], mx[1], mx[2]), fmax3(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7]));
+      const float mts = mt == -INFINITY ? -INFINITY : (mt - kBias) * cr;  // log2 domain
+      // the running max moves only when the tile's max exceeds it by more than 2^8
+      const float m_fin = mts > m_run + 8.0f ? mts : m_run;
+      const float alpha = m_fin != m_run ? ex2(m_run - m_fin) : 1.0f;
+      if (__any_sync(0xffffffffu, m_fin != m_run) && j > 0) {
+        // O is free once P V of tile j-1 has completed
+        if (!warp_wait(&bar[Y_PVD + x], (j - 1) & 1, abort_flag, p.status, 92)) { ok = false; break; }
+        tc_fence_after();
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t r[32];
+          tmem_ld32(tO + loff + c * 32, r);
+          tmem_ld_wait();
+#pragma unroll
+          for (int k = 0; k < 32; k += 2) {
+            float a0 = __uint_as_float(r[k]), a1 = __uint_as_float(r[k + 1]);
+            fmul2(a0, a1, alpha, alpha);
+            r[k] = __float_as_uint(a0);
+            r[k + 1] = __float_as_uint(a1);
+          }
+          tmem_st32(tO + loff + c * 32, r);
+        }
+        tmem_st_wait();
+      }
+      l_run *= alpha;
+      m_run = m_fin;
+      // p = 2^(t * cr - (bias * cr + m) + log2(r_t / v_ref))
+      const float nb = (m_run == -INFINITY ? 0.0f : -(kBias * cr + m_run)) + flog;
+#pragma unroll
+      for (int k = 0; k < BN; k += 2) {
+        ffma2(t[k], t[k + 1], cr, cr, nb, nb);
+        t[k] = ex2(t[k]);
+        t[k + 1] = ex2(t[k + 1]);
+      }
+      float ls[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) ls[e] = t[e];
+#pragma unroll
+      for (int k = 8; k < BN; k += 2) fadd2(ls[k & 7], ls[(k & 7) + 1], t[k], t[k + 1]);
+      {
+        uint32_t hp[BN / 2];
+#pragma unroll
+        for (int e = 0; e < BN / 2; ++e) {
+          const __half2 hv = __floats2half2_rn(t[2 * e], t[2 * e + 1]);
+          hp[e] = *reinterpret_cast<const uint32_t*>(&hv);
+        }
+        tmem_st32(tS + loff, *reinterpret_cast<uint32_t(*)[32]>(&hp[0]));
+        tmem_st32(tS + loff + 32, *reinterpret_cast<uint32_t(*)[32]>(&hp[32]));
+      }
+      tmem_st_wait();
+      l_run += (((ls[0] + ls[1]) + (ls[2] + ls[3])) + ((ls[4] + ls[5]) + (ls[6] + ls[7]))) * finv;
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(&bar[Y_PF + x]);
+        if (RING) mbar_arrive(&bar[Y_SCE + sst]);
+      }
+    }
+    // ---------------------------------------------------------- epilogue
+    if (ok && nx > 0) {
+      ok = warp_wait(&bar[Y_PVD + x], (nx - 1) & 1, abort_flag, p.status, 93);
+      tc_fence_after();
+    }
+    if (q0 < p.Sq) {
+      const float ofac = l_run > 0.0f ? vref / l_run : 0.0f;
+      __nv_bfloat16* orow = nullptr;
+      if (row_ok) {
+        const long long ridx = p.layout == FA_LAYOUT_BNSD ? ((long long)qbh * p.Sq + row)
+                                                          : (((long long)b * p.Sq + row) * p.Hq + hq);
+        orow = p.out + ridx * D;
+      }
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t r[32];
+        if (ok && nx > 0) {
+          tmem_ld32(tO + loff + c * 32, r);
+          tmem_ld_wait();
+        } else {
+#pragma unroll
+          for (int k = 0; k < 32; ++k) r[k] = 0u;
+        }
+        if (row_ok) {
+#pragma unroll
+          for (int k = 0; k < 32; k += 8) {
+            uint32_t o[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const __nv_bfloat162 v2 = __floats2bfloat162_rn(__uint_as_float(r[k + 2 * e]) * ofac,
+                                                              __uint_as_float(r[k + 2 * e + 1]) * ofac);
+              o[e] = *reinterpret_cast<const uint32_t*>(&v2);
+            }
+            *reinterpret_cast<uint4*>(orow + c * 32 + k) = make_uint4(o[0], o[1], o[2], o[3]);
+          }
+        }
+      }
+      if (row_ok && p.lse)
+        p.lse[(long long)qbh * p.Sq + row] =
+            l_run > 0.0f ? (m_run + __log2f(l_run)) * 0.69314718055994530942f : -INFINITY;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tbase, 512);
+  }
+}
+
 // ---- V pre-pass: one CTA per (128-token tile, b * Hkv + h).
 // E4M3: r_t = max s_v over the tile's tokens (1 if all are 0), V' = fp16(code * (s_v / r_t)), |V'| <= 448.
 // INT8: V' = fp16(code) exactly (the per-head scale stays outside).
@@ -774,22 +1222,29 @@ Prefill2Ws carve_ws(void* ws, int B, int Hkv, int Sk, int D) {
 #define FAQ_ATTN_NSW 4
 #endif
 
+// Tensor maps over the Q and K codes and V', then the V pre-pass.
+template <int KIND, int D>
+cudaError_t prepare2(const AttnArgs& a, const P2& prm, const Prefill2Ws& w, int RB, CUtensorMap* mq, CUtensorMap* mk,
+                     CUtensorMap* mv, cudaStream_t s) {
+  cudaError_t e;
+  if ((e = make_code_map(mq, a.q->codes, a.q->B, a.q->H, a.q->S, RB, a.q->layout, BM)) != cudaSuccess) return e;
+  if ((e = make_code_map(mk, a.k->codes, a.k->B, a.k->H, a.k->S, RB, a.k->layout, BN)) != cudaSuccess) return e;
+  if ((e = make_vh_map(mv, w.vh, a.v->B, a.v->H, a.v->S, D)) != cudaSuccess) return e;
+  const dim3 pgrid((unsigned)prm.ntiles_k, (unsigned)(a.v->B * a.v->H));
+  if (pgrid.y > 65535u) return cudaErrorInvalidValue;
+  vprep_kernel<KIND, D><<<pgrid, 256, 0, s>>>(static_cast<const uint8_t*>(a.v->codes), prm.vs, prm.v_blk,
+                                               prm.v_nblk, a.v->H, a.v->S, a.v->layout, w.vh, w.fvr, prm.ntiles_k,
+                                               prm.ks, prm.k_blk, prm.k_nblk, w.ksp, prm.ve8, prm.ke8);
+  return cudaGetLastError();
+}
+
 template <int KIND, int D, int SC>
 cudaError_t launch2(const AttnArgs& a, const P2& prm, const Prefill2Ws& w, cudaStream_t s) {
   constexpr int NSW = FAQ_ATTN_NSW;
   using L = L2<KIND, D>;
   CUtensorMap mq, mk, mv;
   cudaError_t e;
-  const int RB = (int)L::RB;
-  if ((e = make_code_map(&mq, a.q->codes, a.q->B, a.q->H, a.q->S, RB, a.q->layout, BM)) != cudaSuccess) return e;
-  if ((e = make_code_map(&mk, a.k->codes, a.k->B, a.k->H, a.k->S, RB, a.k->layout, BN)) != cudaSuccess) return e;
-  if ((e = make_vh_map(&mv, w.vh, a.v->B, a.v->H, a.v->S, D)) != cudaSuccess) return e;
-  const dim3 pgrid((unsigned)prm.ntiles_k, (unsigned)(a.v->B * a.v->H));
-  if (pgrid.y > 65535u) return cudaErrorInvalidValue;
-  vprep_kernel<KIND, D><<<pgrid, 256, 0, s>>>(static_cast<const uint8_t*>(a.v->codes), prm.vs, prm.v_blk,
-                                               prm.v_nblk, a.v->H, a.v->S, a.v->layout, w.vh, w.fvr, prm.ntiles_k,
-                                               prm.ks, prm.k_blk, prm.k_nblk, w.ksp, prm.ve8, prm.ke8);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  if ((e = prepare2<KIND, D>(a, prm, w, (int)L::RB, &mq, &mk, &mv, s)) != cudaSuccess) return e;
   auto kern = attn2_kernel<KIND, D, SC, NSW>;
   static bool attr_set = false;
   if (!attr_set) {
@@ -803,12 +1258,45 @@ cudaError_t launch2(const AttnArgs& a, const P2& prm, const Prefill2Ws& w, cudaS
   return cudaGetLastError();
 }
 
+template <int KIND, int D, int SC>
+cudaError_t launch_pair(const AttnArgs& a, P2 prm, const Prefill2Ws& w, cudaStream_t s) {
+  using L = LP<D>;
+  CUtensorMap mq, mk, mv;
+  cudaError_t e;
+  if ((e = prepare2<KIND, D>(a, prm, w, D, &mq, &mk, &mv, s)) != cudaSuccess) return e;
+  auto kern = attn_pair_kernel<KIND, D, SC>;
+  static bool attr_set = false;
+  if (!attr_set) {
+    if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::ALLOC)) != cudaSuccess)
+      return e;
+    attr_set = true;
+  }
+  // GQA groups of even size pair two query heads at one row block (equal key ranges); otherwise
+  // a head's row blocks pair up.
+  prm.pair_heads = prm.group % 2 == 0;
+  const long long grid = prm.pair_heads ? (long long)prm.n_qtiles * prm.B * (prm.Hq / 2)
+                                        : (long long)((prm.n_qtiles + 1) / 2) * prm.B * prm.Hq;
+  if (grid > 0x7FFFFFFFLL) return cudaErrorInvalidValue;
+  kern<<<(unsigned)grid, PNT, L::ALLOC, s>>>(mq, mk, mv, prm);
+  return cudaGetLastError();
+}
+
+#ifndef FAQ_PAIR
+#define FAQ_PAIR 1
+#endif
+
+template <int KIND, int D, int SC>
+cudaError_t launch_prefill(const AttnArgs& a, const P2& prm, const Prefill2Ws& w, cudaStream_t s) {
+  if (FAQ_PAIR) return launch_pair<KIND, D, SC>(a, prm, w, s);
+  return launch2<KIND, D, SC>(a, prm, w, s);
+}
+
 template <int KIND, int D>
 cudaError_t launch2_sc(const AttnArgs& a, const P2& prm, const Prefill2Ws& w, int sc, cudaStream_t s) {
   switch (sc) {
-    case SC_HEAD: return launch2<KIND, D, SC_HEAD>(a, prm, w, s);
-    case SC_COL: return launch2<KIND, D, SC_COL>(a, prm, w, s);
-    default: return launch2<KIND, D, SC_TILE>(a, prm, w, s);
+    case SC_HEAD: return launch_prefill<KIND, D, SC_HEAD>(a, prm, w, s);
+    case SC_COL: return launch_prefill<KIND, D, SC_COL>(a, prm, w, s);
+    default: return launch_prefill<KIND, D, SC_TILE>(a, prm, w, s);
   }
 }
 
@@ -869,7 +1357,7 @@ cudaError_t launch_attention_prefill2(const AttnArgs& a, void* ws, cudaStream_t 
     case FA_MODE_FP8_BLOCK:
       return q->D == 128 ? launch2_sc<K_E4M3, 128>(a, prm, w, sc, s) : launch2_sc<K_E4M3, 64>(a, prm, w, sc, s);
     case FA_MODE_INT8_PER_HEAD:
-      return q->D == 128 ? launch2<K_S8, 128, SC_HEAD>(a, prm, w, s) : launch2<K_S8, 64, SC_HEAD>(a, prm, w, s);
+      return q->D == 128 ? launch_prefill<K_S8, 128, SC_HEAD>(a, prm, w, s) : launch_prefill<K_S8, 64, SC_HEAD>(a, prm, w, s);
     case FA_MODE_MXFP4_PER_BLOCK:
       if (q->D != 128) return cudaErrorNotSupported;
       prm.qe8 = static_cast<const uint8_t*>(q->scales);
