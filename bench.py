@@ -232,7 +232,9 @@ def attention_kernels(w):
     """(label, source file) of the attention call's kernels for this workload."""
     if w.name == "int8_decode":
         return "decode_kernel + attn_combine_kernel", "decode.cu"
-    return "vprep_kernel + attn2_kernel (one fa_attention_quant call)", "attn2.cu"
+    if w.mode == "mxfp4":
+        return "vprep_kernel + attn2_kernel (one fa_attention_quant call)", "attn2.cu"
+    return "vprep_kernel + attn_pair_kernel (one fa_attention_quant call)", "attn2.cu"
 
 
 def gpu_run(args, w, rank, world, device):
