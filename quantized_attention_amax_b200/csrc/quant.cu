@@ -8,11 +8,14 @@
 //   fp8_block_kernel          one scale = amax / 448 per block of tokens
 //                             (MindIE SD "量化", FA量化 / 块量化)
 // Rows are D contiguous bf16 values in either layout; each row is handled by
-// D/8 lanes with one 16-byte load each.  Division is IEEE (div.rn.f32) so
-// the codes match a correctly rounded x / s exactly.
+// D/8 lanes with one 16-byte load each.  x / s is rounded as IEEE division
+// (div.rn.f32) rounds it, so the codes match a correctly rounded x / s exactly:
+// FP8 scales use the FMA-corrected reciprocal product of quant_common.cuh,
+// INT8 (whose static scale can be exceeded) uses IEEE division itself.
 #include <cuda_bf16.h>
 
 #include "internal.cuh"
+#include "quant_common.cuh"
 #include "sm100.cuh"
 
 namespace faq {
@@ -129,8 +132,14 @@ __global__ void __launch_bounds__(256) quant_rows_kernel(QuantOperand o0, QuantO
         for (int off = G / 2; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
         const float sc = __fdiv_rn(m, 448.0f);
         float v[8];
+        if (sc >= kFastDivMin) {
+          const float r = __frcp_rn(sc);
 #pragma unroll
-        for (int i = 0; i < 8; ++i) v[i] = sc > 0.0f ? __fdiv_rn(f[i], sc) : 0.0f;
+          for (int i = 0; i < 8; ++i) v[i] = fp8_div(f[i], sc, r);
+        } else {
+#pragma unroll
+          for (int i = 0; i < 8; ++i) v[i] = sc > 0.0f ? __fdiv_rn(f[i], sc) : 0.0f;
+        }
         if (valid) {
           uint2 out = make_uint2(e4m3x4(v[0], v[1], v[2], v[3]), e4m3x4(v[4], v[5], v[6], v[7]));
           reinterpret_cast<uint2*>(static_cast<uint8_t*>(op.codes) + rr[u] * D)[gl] = out;
@@ -168,27 +177,29 @@ __global__ void __launch_bounds__(256) quant_rows_kernel(QuantOperand o0, QuantO
   }
 }
 
-// Per-head running max: grid (chunks, H); each CTA reduces a slice of one
-// head's rows and folds it into amax[h] with one atomic max on the float
-// bits (valid because every value is >= 0).
+// Per-head running max: grid (chunks, H, batches); each CTA reduces a slice of one head's rows of
+// one batch and folds it into amax[h] with one atomic max on the float bits (valid because every
+// value is >= 0).  Row and chunk indices come from shifts (D / 8 is a power of two).
+template <int D>
 __global__ void __launch_bounds__(256) calibrate_kernel(const __nv_bfloat16* __restrict__ x, int B, int H, int S,
-                                                        int D, int layout, float* amax) {
+                                                        int layout, float* amax) {
+  constexpr int VPR = D / 8;  // uint4 per row
+  constexpr int VSH = D == 128 ? 4 : 3;
   const int h = blockIdx.y;
-  const long long rows = (long long)B * S;  // rows of this head
-  const int vpr = D / 8;                    // uint4 per row
-  const long long nvec = rows * vpr;
+  const long long nvec = (long long)S * VPR;
+  const long long rstride = layout == FA_LAYOUT_BNSD ? D : (long long)H * D;  // elements from token s to s + 1
   float m = 0.0f;
-  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < nvec;
-       i += (long long)gridDim.x * blockDim.x) {
-    const long long rh = i / vpr;
-    const int c = (int)(i % vpr);
-    const long long b = rh / S, s = rh % S;
-    const long long row = layout == FA_LAYOUT_BNSD ? (b * H + h) * S + s : (b * S + s) * H + h;
-    const uint4 u = __ldg(reinterpret_cast<const uint4*>(x + row * D) + c);
-    float f[8];
-    unpack_bf16x8(u, f);
+  for (int b = blockIdx.z; b < B; b += gridDim.z) {
+    const __nv_bfloat16* xb = layout == FA_LAYOUT_BNSD ? x + ((long long)b * H + h) * S * D
+                                                       : x + (long long)b * S * H * D + (long long)h * D;
+    for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < nvec;
+         i += (long long)gridDim.x * blockDim.x) {
+      const uint4 u = __ldg(reinterpret_cast<const uint4*>(xb + (i >> VSH) * rstride) + (i & (VPR - 1)));
+      float f[8];
+      unpack_bf16x8(u, f);
 #pragma unroll
-    for (int k = 0; k < 8; ++k) m = fmaxf(m, fabsf(f[k]));
+      for (int k = 0; k < 8; ++k) m = fmaxf(m, fabsf(f[k]));
+    }
   }
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
@@ -237,14 +248,20 @@ __global__ void __launch_bounds__(256) fp8_block_kernel(QuantOperand op) {
   }
   __syncthreads();
   const float sc = s_sc;
+  const float rc = sc >= kFastDivMin ? __frcp_rn(sc) : 0.0f;
   for (int i = threadIdx.x; i < nvec; i += blockDim.x) {
     const long long row = row_of(s0 + i / vpr);
     const uint4 u = __ldg(reinterpret_cast<const uint4*>(x + row * op.D) + (i % vpr));
     float f[8];
     unpack_bf16x8(u, f);
     float v[8];
+    if (sc >= kFastDivMin) {
 #pragma unroll
-    for (int k = 0; k < 8; ++k) v[k] = sc > 0.0f ? __fdiv_rn(f[k], sc) : 0.0f;
+      for (int k = 0; k < 8; ++k) v[k] = fp8_div(f[k], sc, rc);
+    } else {
+#pragma unroll
+      for (int k = 0; k < 8; ++k) v[k] = sc > 0.0f ? __fdiv_rn(f[k], sc) : 0.0f;
+    }
     reinterpret_cast<uint2*>(static_cast<uint8_t*>(op.codes) + row * op.D)[i % vpr] =
         make_uint2(e4m3x4(v[0], v[1], v[2], v[3]), e4m3x4(v[4], v[5], v[6], v[7]));
   }
@@ -272,13 +289,20 @@ cudaError_t launch_rows_mode(const QuantOperand (&o)[3], int D, cudaStream_t s) 
 cudaError_t launch_calibrate(const QuantOperand& op, float* amax, cudaStream_t s) {
   const long long nvec = (long long)op.B * op.S * (op.D / 8);
   if (nvec == 0) return cudaSuccess;
-  long long chunks = (nvec + 256 * 8 - 1) / (256 * 8);
-  const long long cap = ((long long)sm_count() * 8 + op.H - 1) / op.H;
-  if (chunks > cap) chunks = cap;
+  if (op.H > 65535) return cudaErrorInvalidValue;
+  // about eight resident CTAs per SM in total, spread over heads and batches
+  const long long per_b = (long long)op.S * (op.D / 8);
+  const int bz = op.B < 65535 ? op.B : 65535;
+  long long chunks = ((long long)sm_count() * 8 + (long long)op.H * bz - 1) / ((long long)op.H * bz);
+  const long long most = (per_b + 255) / 256;
+  if (chunks > most) chunks = most;
   if (chunks < 1) chunks = 1;
-  dim3 grid((unsigned)chunks, (unsigned)op.H);
-  calibrate_kernel<<<grid, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(op.x), op.B, op.H, op.S, op.D, op.layout,
-                                        amax);
+  dim3 grid((unsigned)chunks, (unsigned)op.H, (unsigned)bz);
+  const __nv_bfloat16* x = static_cast<const __nv_bfloat16*>(op.x);
+  if (op.D == 128)
+    calibrate_kernel<128><<<grid, 256, 0, s>>>(x, op.B, op.H, op.S, op.layout, amax);
+  else
+    calibrate_kernel<64><<<grid, 256, 0, s>>>(x, op.B, op.H, op.S, op.layout, amax);
   return cudaGetLastError();
 }
 

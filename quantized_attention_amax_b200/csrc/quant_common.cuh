@@ -1,0 +1,20 @@
+// quant_common.cuh -- arithmetic shared by the FP8 quantizers (per token, per block, rotate + block).
+#pragma once
+
+#include <cuda_runtime.h>
+
+namespace faq {
+
+// x / s rounded to fp32 as IEEE division does, for an FP8 scale s = fl(amax / 448) with
+// s >= kFastDivMin and a bf16 |x| <= amax: q0 = x * r with r the correctly rounded 1 / s, then one
+// FMA residual x - q0 * s (exact) and one FMA correction; copysign keeps the sign of a zero x.
+// Its E4M3 codes equal those of IEEE division for every bf16 amax whose scale reaches kFastDivMin
+// and every bf16 |x| <= amax (an exhaustive check on the GPU); scales below it use IEEE division.
+constexpr float kFastDivMin = 0x1p-90f;
+
+__device__ __forceinline__ float fp8_div(float x, float s, float r) {
+  const float q0 = x * r;
+  return copysignf(fmaf(fmaf(-q0, s, x), r, q0), x);
+}
+
+}  // namespace faq

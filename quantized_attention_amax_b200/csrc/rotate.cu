@@ -21,6 +21,7 @@
 #include <string.h>
 
 #include "internal.cuh"
+#include "quant_common.cuh"
 #include "sm100.cuh"
 
 namespace faq {
@@ -219,6 +220,8 @@ __global__ void __launch_bounds__(RTHREADS, 2)
     const int t = t0 + r_in;
     if (!(u < ntile && t < op.S)) continue;
     const float sc = bsc[r_in / op.blk];
+    const bool fast = sc >= kFastDivMin;
+    const float rc = fast ? __frcp_rn(sc) : 0.0f;
     const long long ridx = bnsd ? (((long long)b * op.H + h) * op.S + t) : (((long long)b * op.S + t) * op.H + h);
     uint32_t w[16];
 #pragma unroll
@@ -226,7 +229,10 @@ __global__ void __launch_bounds__(RTHREADS, 2)
       const uint32_t p0 = v[u][2 * e], p1 = v[u][2 * e + 1];
       const float x0 = __uint_as_float(p0 << 16), x1 = __uint_as_float(p0 & 0xFFFF0000u);
       const float x2 = __uint_as_float(p1 << 16), x3 = __uint_as_float(p1 & 0xFFFF0000u);
-      w[e] = (sc > 0.0f && ok) ? e4m3x4(__fdiv_rn(x0, sc), __fdiv_rn(x1, sc), __fdiv_rn(x2, sc), __fdiv_rn(x3, sc)) : 0u;
+      if (fast)
+        w[e] = ok ? e4m3x4(fp8_div(x0, sc, rc), fp8_div(x1, sc, rc), fp8_div(x2, sc, rc), fp8_div(x3, sc, rc)) : 0u;
+      else
+        w[e] = (sc > 0.0f && ok) ? e4m3x4(__fdiv_rn(x0, sc), __fdiv_rn(x1, sc), __fdiv_rn(x2, sc), __fdiv_rn(x3, sc)) : 0u;
     }
     uint4* crow = reinterpret_cast<uint4*>(static_cast<uint8_t*>(op.codes) + ridx * 128 + half * 64);
 #pragma unroll

@@ -105,8 +105,11 @@ def exhaustive_rows(group, maxima, seed):
 
 
 def test_fp8_per_token_exhaustive(faq, orc):
-    # power-of-two scales make the e4m3 midpoints land exactly (ties); others are generic
-    maxima = [448.0, 56.0, 3.5, 1.0, 0.0546875, 3.0e38, 1e-30, 2.0 ** -126, 7.1, 0.3]
+    # power-of-two scales make the e4m3 midpoints land exactly (ties); others are generic.  The
+    # kernel divides by one FMA-corrected reciprocal product when s = amax / 448 >= 2^-90 and by
+    # IEEE division below: maxima on both sides of amax = 448 * 2^-90 ~ 2^-81.2 cover the switch.
+    maxima = [448.0, 56.0, 3.5, 1.0, 0.0546875, 3.0e38, 1e-30, 2.0 ** -126, 7.1, 0.3,
+              2.0 ** -81, 2.0 ** -82, 3.6e-25, 1.7e-20]
     rows = exhaustive_rows(128, maxima, 1)
     x = rows.reshape(1, 1, -1, 128)
     o, = faq.quantize(bf16_from_bits(x), None, None, "fp8_per_token")[:1]
