@@ -22,7 +22,8 @@ import numpy as np
 from . import build as _build
 
 LAYOUTS = {"BNSD": 0, "BSND": 1}
-MODES = {"float": 0, "int8_per_head": 1, "fp8_per_token": 2, "mxfp4": 3, "fp8_block": 4}
+MODES = {"float": 0, "int8_per_head": 1, "fp8_per_token": 2, "mxfp4": 3, "fp8_block": 4, "fp8_per_head": 5,
+         "int8_per_token": 6}
 
 _lib = None
 
@@ -58,6 +59,8 @@ def lib() -> ctypes.CDLL:
         L.orc_calibrate_per_head.argtypes = [P, I, I, I, I, I, P]
         L.orc_quantize_int8_per_head.argtypes = [P, I, I, I, I, I, P, P, P]
         L.orc_quantize_fp8_per_token.argtypes = [P, I, I, I, I, I, P, P]
+        L.orc_quantize_fp8_per_head.argtypes = [P, I, I, I, I, I, P, P, P]
+        L.orc_quantize_int8_per_token.argtypes = [P, I, I, I, I, I, P, P]
         L.orc_quantize_mxfp4.argtypes = [P, I, I, I, I, I, P, P]
         L.orc_rotate_f64.argtypes = [P, I, I, I, I, I, P, P]
         L.orc_rotate.argtypes = [P, I, I, I, I, I, P, P]
@@ -176,6 +179,25 @@ def quantize_fp8_per_token(x: np.ndarray, layout: str = "BNSD"):
     codes = np.empty(x.shape, np.uint8)
     scales = np.empty((B, H, S), np.float32)
     lib().orc_quantize_fp8_per_token(_ptr(x), B, H, S, D, LAYOUTS[layout], _ptr(codes), _ptr(scales))
+    return codes, scales
+
+
+def quantize_fp8_per_head(x: np.ndarray, amax: np.ndarray, layout: str = "BNSD"):
+    x = np.ascontiguousarray(x, dtype=np.uint16)
+    B, H, S, D = dims(x.shape, layout)
+    amax = np.ascontiguousarray(amax, dtype=np.float32)
+    codes = np.empty(x.shape, np.uint8)
+    scales = np.empty(H, np.float32)
+    lib().orc_quantize_fp8_per_head(_ptr(x), B, H, S, D, LAYOUTS[layout], _ptr(amax), _ptr(codes), _ptr(scales))
+    return codes, scales
+
+
+def quantize_int8_per_token(x: np.ndarray, layout: str = "BNSD"):
+    x = np.ascontiguousarray(x, dtype=np.uint16)
+    B, H, S, D = dims(x.shape, layout)
+    codes = np.empty(x.shape, np.int8)
+    scales = np.empty((B, H, S), np.float32)
+    lib().orc_quantize_int8_per_token(_ptr(x), B, H, S, D, LAYOUTS[layout], _ptr(codes), _ptr(scales))
     return codes, scales
 
 

@@ -239,6 +239,50 @@ void orc_quantize_fp8_per_token(const uint16_t* x, int B, int H, int S, int D,
       }
 }
 
+/* [FA] 模式清单, FA PerHead with FP8: 组合1's static per-head calibration with
+ * the E4M3 range, s_h = amax_h / 448, code = e4m3(x / s_h) (values beyond the
+ * calibrated range saturate to +-448).  A zero scale gives code 0x00. */
+void orc_quantize_fp8_per_head(const uint16_t* x, int B, int H, int S, int D,
+                               int layout, const float* amax, uint8_t* codes,
+                               float* scales) {
+  for (int h = 0; h < H; ++h) {
+    const float sh = amax[h] / 448.0f;
+    scales[h] = sh;
+#pragma omp parallel for collapse(2) schedule(static)
+    for (int b = 0; b < B; ++b)
+      for (int s = 0; s < S; ++s)
+        for (int d = 0; d < D; ++d) {
+          const size_t i = elem_index(layout, H, S, D, b, h, s, d);
+          const float xf = orc_bf16_to_f32(x[i]);
+          codes[i] = (sh > 0.0f) ? orc_e4m3_encode(xf / sh) : (uint8_t)0;
+        }
+  }
+}
+
+/* [FA] 模式清单, FA PerToken with INT8: 组合2's dynamic per-token amax with the
+ * INT8 range, s = amax / 127 per (b, h, token), code = int8(x / s).  A zero
+ * scale gives code 0. */
+void orc_quantize_int8_per_token(const uint16_t* x, int B, int H, int S, int D,
+                                 int layout, int8_t* codes, float* scales) {
+#pragma omp parallel for collapse(3) schedule(static)
+  for (int b = 0; b < B; ++b)
+    for (int h = 0; h < H; ++h)
+      for (int s = 0; s < S; ++s) {
+        float amax = 0.0f;
+        for (int d = 0; d < D; ++d) {
+          const float a = fabsf(orc_bf16_to_f32(x[elem_index(layout, H, S, D, b, h, s, d)]));
+          if (a > amax) amax = a;
+        }
+        const float sc = amax / 127.0f;
+        scales[((size_t)b * H + h) * S + s] = sc;
+        for (int d = 0; d < D; ++d) {
+          const size_t i = elem_index(layout, H, S, D, b, h, s, d);
+          const float xf = orc_bf16_to_f32(x[i]);
+          codes[i] = (sc > 0.0f) ? orc_int8_encode(xf / sc) : (int8_t)0;
+        }
+      }
+}
+
 /* [FA] 组合3: blocks of 32 consecutive elements along head_dim share one
  * E8M0 exponent X = 2^e, e = floor(log2 amax) - 2; values are E2M1 of x / X. */
 void orc_quantize_mxfp4(const uint16_t* x, int B, int H, int S, int D,
@@ -341,6 +385,11 @@ double orc_dequant_elem(const orc_qt* t, int b, int h, int s, int d) {
       return (double)((const int8_t*)t->codes)[i] * (double)((const float*)t->scales)[h];
     case ORC_MODE_FP8_PER_TOKEN:
       return orc_e4m3_decode(((const uint8_t*)t->codes)[i]) *
+             (double)((const float*)t->scales)[((size_t)b * t->H + h) * t->S + s];
+    case ORC_MODE_FP8_PER_HEAD:
+      return orc_e4m3_decode(((const uint8_t*)t->codes)[i]) * (double)((const float*)t->scales)[h];
+    case ORC_MODE_INT8_PER_TOKEN:
+      return (double)((const int8_t*)t->codes)[i] *
              (double)((const float*)t->scales)[((size_t)b * t->H + h) * t->S + s];
     case ORC_MODE_FP8_BLOCK: {
       const int nblk = (t->S + t->blk - 1) / t->blk;

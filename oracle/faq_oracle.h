@@ -11,7 +11,9 @@
  * Sources (web pages on FA quantization):
  *   [FA]   msModelSlim wiki "FA 量化" -- sections 概述 (overview),
  *          分支组合 (branch combinations: 组合1 INT8 per-head static,
- *          组合2 FP8 E4M3 per-token dynamic, 组合3 MXFP4 per-block dynamic).
+ *          组合2 FP8 E4M3 per-token dynamic, 组合3 MXFP4 per-block dynamic),
+ *          该类下的模式清单 (mode list: FA PerHead INT8/FP8 static, FA PerToken
+ *          INT8/FP8 dynamic, FA PerBlock MXFP8/MXFP4).
  *   [MODE] msModelSlim wiki "量化模式" -- 模式索引 (mode index): FakeQuant
  *          means quantize and immediately dequantize.
  *   [SD]   MindIE SD "量化" -- Linear 量化 / 通用原理 (INT8 range figure
@@ -27,7 +29,9 @@
  * Layouts: BNSD = [B, H, S, D], BSND = [B, S, H, D]; D is contiguous in both.
  * Scale arrays are canonical whatever the data layout:
  *   INT8 per head  : fp32 [H]
+ *   FP8 per head   : fp32 [H]
  *   FP8 per token  : fp32 [B, H, S]
+ *   INT8 per token : fp32 [B, H, S]
  *   FP8 block      : fp32 [B, H, ceil(S / blk)]
  *   MXFP4          : uint8 E8M0 [B, H, S, D / 32]
  * MXFP4 codes are packed [.., D/2] in the data layout, element 2i in the low
@@ -49,7 +53,9 @@ enum {
   ORC_MODE_INT8_PER_HEAD = 1,  /* [FA] 组合1                                  */
   ORC_MODE_FP8_PER_TOKEN = 2,  /* [FA] 组合2                                  */
   ORC_MODE_MXFP4 = 3,          /* [FA] 组合3                                  */
-  ORC_MODE_FP8_BLOCK = 4       /* [SD] FA量化 块量化                           */
+  ORC_MODE_FP8_BLOCK = 4,      /* [SD] FA量化 块量化                           */
+  ORC_MODE_FP8_PER_HEAD = 5,   /* [FA] 模式清单: FA PerHead, FP8               */
+  ORC_MODE_INT8_PER_TOKEN = 6  /* [FA] 模式清单: FA PerToken, INT8             */
 };
 
 /* A quantized (or bf16) operand as the oracle sees it. */
@@ -81,6 +87,12 @@ void orc_quantize_int8_per_head(const uint16_t* x, int B, int H, int S, int D,
 void orc_quantize_fp8_per_token(const uint16_t* x, int B, int H, int S, int D,
                                 int layout, uint8_t* codes,
                                 float* scales /* [B,H,S] */);
+void orc_quantize_fp8_per_head(const uint16_t* x, int B, int H, int S, int D,
+                               int layout, const float* amax,
+                               uint8_t* codes, float* scales /* [H] */);
+void orc_quantize_int8_per_token(const uint16_t* x, int B, int H, int S, int D,
+                                 int layout, int8_t* codes,
+                                 float* scales /* [B,H,S] */);
 void orc_quantize_mxfp4(const uint16_t* x, int B, int H, int S, int D,
                         int layout, uint8_t* codes /* packed */,
                         uint8_t* e8m0 /* [B,H,S,D/32] */);
