@@ -42,6 +42,9 @@ DESCR = {
                      "non-causal, BSND",
     "mxfp4": "MXFP4 per-32-block (E2M1 + E8M0), image-edit B=1 H=24 S=4096 D=128, non-causal, BNSD, Student-t",
     "int8_decode": "INT8 per-head static split-KV decode, B=16 Hq=32 Hkv=8 Sq=1 Sk=32768 D=128, BNSD",
+    "int8_prefill": "INT8 per-head static, the fp8_prefill shape (B=2 Hq=32 Hkv=8 S=4096 D=128, causal, BNSD)",
+    "fp8_head_prefill": "FP8 E4M3 per-head static, the fp8_prefill shape (B=2 Hq=32 Hkv=8 S=4096 D=128, causal, BNSD)",
+    "int8_token_prefill": "INT8 per-token dynamic, the fp8_prefill shape (B=2 Hq=32 Hkv=8 S=4096 D=128, causal, BNSD)",
 }
 DATA = {
     "int8_tiny": "synthetic: seeded bf16 N(0,1); per-head scales from a seeded calibration batch",
@@ -49,6 +52,9 @@ DATA = {
     "rot_fp8_block": "synthetic: seeded bf16 N(0,1); R = bf16(Hadamard * seeded signs / sqrt(128))",
     "mxfp4": "synthetic: seeded bf16 Student-t (df=4)",
     "int8_decode": "synthetic: seeded bf16 N(0,1) cache and query; per-head scales from seeded calibration batches",
+    "int8_prefill": "synthetic: as fp8_prefill; per-head scales from seeded calibration batches",
+    "fp8_head_prefill": "synthetic: as fp8_prefill; per-head scales from seeded calibration batches",
+    "int8_token_prefill": "synthetic: as fp8_prefill",
 }
 DTYPE = {
     "int8_tiny": "s8 (QK^T, s32 acc) + f16 (PV)",
@@ -56,8 +62,14 @@ DTYPE = {
     "rot_fp8_block": "bf16 (rotation) + e4m3 (QK^T) + f16 (PV)",
     "mxfp4": "e2m1 block-scaled (QK^T) + f16 (PV)",
     "int8_decode": "s8 (QK^T) + u8/s8 (PV), s32 accumulate",
+    "int8_prefill": "s8 (QK^T, s32 acc) + f16 (PV)",
+    "fp8_head_prefill": "e4m3 (QK^T) + f16 (PV), fp32 accumulate",
+    "int8_token_prefill": "s8 (QK^T, s32 acc) + f16 (PV)",
 }
 
+
+# modes whose scales come from a calibration batch (per-head static)
+STATIC_MODES = ("int8_per_head", "fp8_per_head")
 
 def attn_flops(w) -> float:
     """Algorithmic attention FLOPs: 4 * D per unmasked (query, key) pair."""
@@ -76,7 +88,7 @@ def quant_bytes(w) -> float:
     if w.mode == "int8_decode" or w.name == "int8_decode":
         return nq * 2 + nq + w.Hq * 4  # only Q is quantized per step
     code = 0.5 if w.mode == "mxfp4" else 1.0
-    if w.mode == "fp8_per_token":
+    if w.mode in ("fp8_per_token", "int8_per_token"):
         sc = (w.B * w.Hq * w.Sq + 2 * w.B * w.Hkv * w.Sk) * 4
     elif w.mode == "fp8_block":
         sc = (w.B * w.Hq * -(-w.Sq // w.q_block) + 2 * w.B * w.Hkv * -(-w.Sk // w.kv_block)) * 4
@@ -171,10 +183,10 @@ def make_step(faq, wl, w, device, seed_offset=0):
     """Allocate inputs on the device and return (step_fn, attn_fn, quant_fn, state)."""
     import torch
     w2 = w.scaled(seed=w.seed + seed_offset)
-    inp = wl.make_inputs(w2, device=device, calib=(w.mode == "int8_per_head"))
+    inp = wl.make_inputs(w2, device=device, calib=(w.mode in STATIC_MODES))
     q, k, v = inp["q"], inp["k"], inp["v"]
     st = {"inp": inp}
-    if w.mode == "int8_per_head":
+    if w.mode in STATIC_MODES:
         amax = [faq.calibrate_per_head(inp[n + "_cal"], w.layout) for n in "qkv"]
         st["amax"] = amax
         if w.name == "int8_decode":
@@ -323,12 +335,12 @@ def e2e_run(args, w, device, steps):
     import quantized_attention_amax_b200 as faq
     import workloads as wl
 
-    inp = wl.make_inputs(w, device="cpu", calib=(w.mode == "int8_per_head"))
+    inp = wl.make_inputs(w, device="cpu", calib=(w.mode in STATIC_MODES))
     host = {n: inp[n].pin_memory() for n in ("q", "k", "v")}
     dev = [{n: torch.empty_like(host[n], device=device) for n in host} for _ in range(2)]
     R = inp["R"].to(device) if inp.get("R") is not None else None
     amax = None
-    if w.mode == "int8_per_head":
+    if w.mode in STATIC_MODES:
         amax = [faq.calibrate_per_head(inp[n + "_cal"].to(device), w.layout) for n in "qkv"]
     out_h = [torch.empty_like(host["q"]).pin_memory() for _ in range(2)]
     out_d = [torch.empty_like(host["q"], device=device) for _ in range(2)]
@@ -409,13 +421,13 @@ def oracle_sample(w, reps_seconds=None):
     G = w.Hq // w.Hkv
     rows = list(range(max(0, w.Sq - 64), w.Sq))
     sub = w.scaled(B=1, Hq=G, Hkv=1)
-    inp = wl.make_inputs(sub, calib=(w.mode == "int8_per_head"))
+    inp = wl.make_inputs(sub, calib=(w.mode in STATIC_MODES))
     qb = wl.bf16_bits(inp["q"])
     kb = wl.bf16_bits(inp["k"])
     vb = wl.bf16_bits(inp["v"])
     L = w.layout
     amax = None
-    if w.mode == "int8_per_head":
+    if w.mode in STATIC_MODES:
         amax = {n: orc.calibrate_per_head(wl.bf16_bits(inp[n + "_cal"]), L) for n in "qkv"}
     Rb = wl.bf16_bits(inp["R"]) if inp.get("R") is not None else None
 
@@ -425,6 +437,12 @@ def oracle_sample(w, reps_seconds=None):
             cq, sq = orc.quantize_int8_per_head(qb, amax["q"], L)
             ck, sk = orc.quantize_int8_per_head(kb, amax["k"], L)
             cv, sv = orc.quantize_int8_per_head(vb, amax["v"], L)
+            blks = (0, 0, 0)
+        elif w.mode == "fp8_per_head":
+            (cq, sq), (ck, sk), (cv, sv) = (orc.quantize_fp8_per_head(x, amax[n], L) for x, n in zip((qb, kb, vb), "qkv"))
+            blks = (0, 0, 0)
+        elif w.mode == "int8_per_token":
+            (cq, sq), (ck, sk), (cv, sv) = (orc.quantize_int8_per_token(x, L) for x in (qb, kb, vb))
             blks = (0, 0, 0)
         elif w.mode == "fp8_per_token":
             (cq, sq), (ck, sk), (cv, sv) = (orc.quantize_fp8_per_token(x, L) for x in (qb, kb, vb))
@@ -498,7 +516,8 @@ def supplemental(args, device):
     import workloads as wl
     out = {}
     pk = peaks()
-    for name in ("int8_tiny", "rot_fp8_block", "mxfp4", "int8_decode"):
+    for name in ("int8_tiny", "rot_fp8_block", "mxfp4", "int8_decode", "int8_prefill", "fp8_head_prefill",
+                 "int8_token_prefill"):
         w = wl.WORKLOADS[name]
         a = argparse.Namespace(steps=10 if name != "rot_fp8_block" else 4, warmup=3)
         r = gpu_run(a, w, 0, 1, device)

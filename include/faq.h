@@ -29,6 +29,8 @@
  *   FA_MODE_MXFP4_PER_BLOCK  codes packed e2m1 [..D/2] (element 2i in the
  *                            low nibble, 2i+1 in the high nibble);
  *                            scales uint8 E8M0 [B, H, S, D/32]
+ *   FA_MODE_FP8_PER_HEAD     codes e4m3 [..D];   scales fp32 [H]
+ *   FA_MODE_INT8_PER_TOKEN   codes int8 [..D];   scales fp32 [B, H, S]
  */
 #ifndef FAQ_H
 #define FAQ_H
@@ -62,13 +64,16 @@ typedef enum {
 typedef enum { FA_LAYOUT_BNSD = 0, FA_LAYOUT_BSND = 1 } fa_layout;
 
 /* The pages' FA modes (msModelSlim wiki "FA 量化", 分支组合 / branch
- * combinations 组合1-3; MindIE SD "量化", FA量化 / 块量化). */
+ * combinations 组合1-3 and 该类下的模式清单 / mode list: FA PerHead INT8/FP8
+ * static, FA PerToken INT8/FP8 dynamic; MindIE SD "量化", FA量化 / 块量化). */
 typedef enum {
   FA_MODE_FLOAT = 0,           /* not quantized ("float": the branch stays bf16) */
   FA_MODE_INT8_PER_HEAD = 1,   /* 组合1: INT8, per-head static minmax, s = amax/127 */
   FA_MODE_FP8_PER_TOKEN = 2,   /* 组合2: E4M3, per-token dynamic, s = amax/448     */
   FA_MODE_MXFP4_PER_BLOCK = 3, /* 组合3: E2M1 + E8M0 per 32 elements of head_dim   */
-  FA_MODE_FP8_BLOCK = 4        /* 块量化: E4M3, one scale per block of tokens      */
+  FA_MODE_FP8_BLOCK = 4,       /* 块量化: E4M3, one scale per block of tokens      */
+  FA_MODE_FP8_PER_HEAD = 5,    /* FA PerHead, FP8: per-head static, s = amax/448   */
+  FA_MODE_INT8_PER_TOKEN = 6   /* FA PerToken, INT8: per-token dynamic, s = amax/127 */
 } fa_mode;
 
 /* A bf16 activation tensor. */
@@ -129,13 +134,17 @@ FAQ_API fa_status fa_calibrate_per_head(const fa_tensor* x, float* amax_h, fa_st
  *   E4M3 per-token dynamic: s = amax_token/448, code = e4m3(x / s)),
  *   组合3 (MXFP4: per 32 elements of head_dim, e = floor(log2 amax) - 2,
  *   E8M0 byte e + 127, code = e2m1(x / 2^e)); MindIE SD FA量化 / 块量化
- *   (E4M3 with one scale = amax/448 per block of block_tokens tokens).
- *   Rounding is round-half-to-even, saturating; x / s is one IEEE fp32
- *   division; a zero scale gives zero codes.
+ *   (E4M3 with one scale = amax/448 per block of block_tokens tokens);
+ *   "FA 量化", 该类下的模式清单: FA PerHead with FP8 (组合1's calibration,
+ *   s_h = amax_h/448, values past the calibrated range saturate to +-448) and
+ *   FA PerToken with INT8 (组合2's per-token amax, s = amax_token/127).
+ *   Rounding is round-half-to-even, saturating; x / s is rounded as one IEEE
+ *   fp32 division; a zero scale gives zero codes.
  *   q, k, v: bf16 inputs; any of them may be NULL to skip that operand.
  *   mode: one of the quantized modes.  amax_q/k/v: device fp32 [H] from
- *   fa_calibrate_per_head, required for FA_MODE_INT8_PER_HEAD (NULL there
- *   -> FA_ERR_NO_CALIBRATION), ignored otherwise.
+ *   fa_calibrate_per_head, required for FA_MODE_INT8_PER_HEAD and
+ *   FA_MODE_FP8_PER_HEAD (NULL there -> FA_ERR_NO_CALIBRATION), ignored
+ *   otherwise.
  *   q_out/k_out/v_out: caller-filled descriptors whose codes/scales point to
  *   buffers of the sizes above; their dims/layout must equal the input's
  *   and their mode must equal `mode`.  For FA_MODE_FP8_BLOCK,
@@ -185,9 +194,9 @@ FAQ_API fa_status fa_rotate_quantize(const fa_tensor* q, const fa_tensor* k, con
  *   the tile's largest UE8M0 exponent), a 16-byte record per tile holding
  *   r_t (E_t), and 512 bytes of K scales per tile (128 per-key floats, or
  *   MXFP4's scale-factor atom).  num_splits (decode only): 0 = automatic.
- *   Modes run here: INT8_PER_HEAD, FP8_PER_TOKEN, FP8_BLOCK and
- *   MXFP4_PER_BLOCK for prefill; INT8_PER_HEAD for decode (others ->
- *   FA_ERR_UNSUPPORTED).
+ *   Modes run here: INT8_PER_HEAD, FP8_PER_TOKEN, FP8_BLOCK, MXFP4_PER_BLOCK,
+ *   FP8_PER_HEAD and INT8_PER_TOKEN for prefill; INT8_PER_HEAD for decode
+ *   (others -> FA_ERR_UNSUPPORTED).
  */
 FAQ_API fa_status fa_attention_quant(const fa_qtensor* q, const fa_qtensor* k, const fa_qtensor* v, int causal,
                              float softmax_scale, void* out, float* lse, int num_splits, void* workspace,

@@ -16,7 +16,8 @@ import torch
 from . import _native as N
 
 LAYOUTS = {"BNSD": 0, "BSND": 1}
-MODES = {"float": 0, "int8_per_head": 1, "fp8_per_token": 2, "mxfp4": 3, "fp8_block": 4}
+MODES = {"float": 0, "int8_per_head": 1, "fp8_per_token": 2, "mxfp4": 3, "fp8_block": 4, "fp8_per_head": 5,
+         "int8_per_token": 6}
 MODE_NAMES = {v: k for k, v in MODES.items()}
 
 
@@ -74,6 +75,12 @@ def empty_qtensor(B: int, H: int, S: int, D: int, mode: str, layout: str = "BNSD
     if mode == "int8_per_head":
         codes = torch.empty(shp, dtype=torch.int8, device=device)
         scales = torch.empty((H,), dtype=torch.float32, device=device)
+    elif mode == "fp8_per_head":
+        codes = torch.empty(shp, dtype=torch.uint8, device=device)
+        scales = torch.empty((H,), dtype=torch.float32, device=device)
+    elif mode == "int8_per_token":
+        codes = torch.empty(shp, dtype=torch.int8, device=device)
+        scales = torch.empty((B, H, S), dtype=torch.float32, device=device)
     elif mode == "fp8_per_token":
         codes = torch.empty(shp, dtype=torch.uint8, device=device)
         scales = torch.empty((B, H, S), dtype=torch.float32, device=device)

@@ -668,7 +668,7 @@ template <int KIND, int D, int SC>
 __global__ void __launch_bounds__(PNT, 1)
     attn_pair_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
                      const __grid_constant__ CUtensorMap tmv, const P2 p) {
-  static_assert(KIND == K_E4M3 || (KIND == K_S8 && SC == SC_HEAD), "E4M3 or INT8 operands");
+  static_assert(KIND == K_E4M3 || (KIND == K_S8 && SC != SC_TILE), "E4M3 or INT8 operands");
   constexpr bool RING = SC != SC_HEAD;
   using L = LP<D>;
   extern __shared__ uint8_t smem_raw[];
@@ -891,7 +891,10 @@ __global__ void __launch_bounds__(PNT, 1)
     const float sq = row_ok ? scale_at(p.qs, p.q_blk, p.q_nblk, qbh, hq, row) : 0.0f;
     float crow = sq * p.scale_log2;
     if (!RING) crow *= __ldg(p.ks + hk);
-    constexpr float kBias = KIND == K_S8 ? 12582912.0f : 0.0f;
+    // S8 accumulators with one K scale per head arrive biased (t = 1.5 * 2^23 + acc, exact for
+    // |acc| < 2^22); with per-key K scales they are converted exactly instead
+    constexpr bool BIASED = KIND == K_S8 && SC == SC_HEAD;
+    constexpr float kBias = BIASED ? 12582912.0f : 0.0f;
     float vref = RING ? 1.0f : __ldg(p.vs + hk);
     float m_run = -INFINITY, l_run = 0.0f;
     bool ok = true;
@@ -933,7 +936,8 @@ __global__ void __launch_bounds__(PNT, 1)
         tmem_ld_wait();
 #pragma unroll
         for (int k = 64 * hh; k < 64 * hh + 64; ++k)
-          t[k] = KIND == K_S8 ? __uint_as_float(0x4B400000u + tr[k]) : __uint_as_float(tr[k]);
+          t[k] = BIASED ? __uint_as_float(0x4B400000u + tr[k])
+                        : (KIND == K_S8 ? (float)(int)tr[k] : __uint_as_float(tr[k]));
         if (SC == SC_COL) {
 #pragma unroll
           for (int k = 64 * hh; k < 64 * hh + 64; k += 2) fmul2(t[k], t[k + 1], ksr[k], ksr[k + 1]);
@@ -1066,10 +1070,12 @@ __global__ void __launch_bounds__(PNT, 1)
 }
 
 // ---- V pre-pass: one CTA per (128-token tile, b * Hkv + h).
-// E4M3: r_t = max s_v over the tile's tokens (1 if all are 0), V' = fp16(code * (s_v / r_t)), |V'| <= 448.
-// INT8: V' = fp16(code) exactly (the per-head scale stays outside).
+// V scales per token or per block (VSC): r_t = max s_v over the tile's tokens (1 if all are 0),
+//   V' = fp16(code * (s_v / r_t)) (|V'| <= 448 for E4M3, 127 for INT8), r_t in the tile's record and
+//   the tile's per-key K scales beside it.
+// V scale per head: V' = fp16(code) exactly (the per-head scale stays outside).
 // MXFP4: E_t = the largest UE8M0 byte of the tile's tokens, V' = fp16(e2m1 * 2^(e - E_t)), |V'| <= 6.
-template <int KIND, int D>
+template <int KIND, int D, bool VSC>
 __global__ void __launch_bounds__(256) vprep_kernel(const uint8_t* __restrict__ codes, const float* __restrict__ vs,
                                                     int v_blk, int v_nblk, int H, int S, int layout,
                                                     __half* __restrict__ vh, float4* __restrict__ fvr, int ntiles,
@@ -1136,7 +1142,7 @@ __global__ void __launch_bounds__(256) vprep_kernel(const uint8_t* __restrict__ 
 #pragma unroll
   for (int c = 0; c < CPT; ++c) raw[c] = live ? __ldg(reinterpret_cast<const uint4*>(src) + c) : make_uint4(0, 0, 0, 0);
   float f = 1.0f;
-  if (KIND == K_E4M3) {
+  if (VSC) {
     // every warp reduces the tile's 128 scales itself (no block barrier)
     const float* vsh = vs + (long long)bh * v_nblk;
     float m = 0.0f;
@@ -1166,8 +1172,19 @@ __global__ void __launch_bounds__(256) vprep_kernel(const uint8_t* __restrict__ 
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
         const uint32_t h2 = e4m3x2_to_h2((uint16_t)(w[i >> 1] >> ((i & 1) * 16)));
-        const float2 x = __half22float2(*reinterpret_cast<const __half2*>(&h2));
-        const __half2 y = __floats2half2_rn(x.x * f, x.y * f);
+        if (VSC) {
+          const float2 x = __half22float2(*reinterpret_cast<const __half2*>(&h2));
+          const __half2 y = __floats2half2_rn(x.x * f, x.y * f);
+          o[i] = *reinterpret_cast<const uint32_t*>(&y);
+        } else {
+          o[i] = h2;  // exact
+        }
+      }
+    } else if (VSC) {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const uint32_t pr = w[i >> 1] >> ((i & 1) * 16);
+        const __half2 y = __floats2half2_rn((float)(int8_t)(pr & 0xFFu) * f, (float)(int8_t)((pr >> 8) & 0xFFu) * f);
         o[i] = *reinterpret_cast<const uint32_t*>(&y);
       }
     } else {
@@ -1223,7 +1240,7 @@ Prefill2Ws carve_ws(void* ws, int B, int Hkv, int Sk, int D) {
 #endif
 
 // Tensor maps over the Q and K codes and V', then the V pre-pass.
-template <int KIND, int D>
+template <int KIND, int D, bool VSC>
 cudaError_t prepare2(const AttnArgs& a, const P2& prm, const Prefill2Ws& w, int RB, CUtensorMap* mq, CUtensorMap* mk,
                      CUtensorMap* mv, cudaStream_t s) {
   cudaError_t e;
@@ -1232,7 +1249,7 @@ cudaError_t prepare2(const AttnArgs& a, const P2& prm, const Prefill2Ws& w, int 
   if ((e = make_vh_map(mv, w.vh, a.v->B, a.v->H, a.v->S, D)) != cudaSuccess) return e;
   const dim3 pgrid((unsigned)prm.ntiles_k, (unsigned)(a.v->B * a.v->H));
   if (pgrid.y > 65535u) return cudaErrorInvalidValue;
-  vprep_kernel<KIND, D><<<pgrid, 256, 0, s>>>(static_cast<const uint8_t*>(a.v->codes), prm.vs, prm.v_blk,
+  vprep_kernel<KIND, D, VSC><<<pgrid, 256, 0, s>>>(static_cast<const uint8_t*>(a.v->codes), prm.vs, prm.v_blk,
                                                prm.v_nblk, a.v->H, a.v->S, a.v->layout, w.vh, w.fvr, prm.ntiles_k,
                                                prm.ks, prm.k_blk, prm.k_nblk, w.ksp, prm.ve8, prm.ke8);
   return cudaGetLastError();
@@ -1244,7 +1261,7 @@ cudaError_t launch2(const AttnArgs& a, const P2& prm, const Prefill2Ws& w, cudaS
   using L = L2<KIND, D>;
   CUtensorMap mq, mk, mv;
   cudaError_t e;
-  if ((e = prepare2<KIND, D>(a, prm, w, (int)L::RB, &mq, &mk, &mv, s)) != cudaSuccess) return e;
+  if ((e = prepare2<KIND, D, true>(a, prm, w, (int)L::RB, &mq, &mk, &mv, s)) != cudaSuccess) return e;
   auto kern = attn2_kernel<KIND, D, SC, NSW>;
   static bool attr_set = false;
   if (!attr_set) {
@@ -1263,7 +1280,7 @@ cudaError_t launch_pair(const AttnArgs& a, P2 prm, const Prefill2Ws& w, cudaStre
   using L = LP<D>;
   CUtensorMap mq, mk, mv;
   cudaError_t e;
-  if ((e = prepare2<KIND, D>(a, prm, w, D, &mq, &mk, &mv, s)) != cudaSuccess) return e;
+  if ((e = prepare2<KIND, D, SC != SC_HEAD>(a, prm, w, D, &mq, &mk, &mv, s)) != cudaSuccess) return e;
   auto kern = attn_pair_kernel<KIND, D, SC>;
   static bool attr_set = false;
   if (!attr_set) {
@@ -1281,14 +1298,9 @@ cudaError_t launch_pair(const AttnArgs& a, P2 prm, const Prefill2Ws& w, cudaStre
   return cudaGetLastError();
 }
 
-#ifndef FAQ_PAIR
-#define FAQ_PAIR 1
-#endif
-
 template <int KIND, int D, int SC>
 cudaError_t launch_prefill(const AttnArgs& a, const P2& prm, const Prefill2Ws& w, cudaStream_t s) {
-  if (FAQ_PAIR) return launch_pair<KIND, D, SC>(a, prm, w, s);
-  return launch2<KIND, D, SC>(a, prm, w, s);
+  return launch_pair<KIND, D, SC>(a, prm, w, s);
 }
 
 template <int KIND, int D>
@@ -1312,7 +1324,8 @@ __global__ void fill_empty_kernel(__nv_bfloat16* out, float* lse, long long rows
 void scale_desc2(const fa_qtensor* t, int& blk, int& nblk) {
   switch (t->mode) {
     case FA_MODE_INT8_PER_HEAD: blk = 0; nblk = 1; break;
-    case FA_MODE_FP8_PER_TOKEN: blk = 1; nblk = t->S; break;
+    case FA_MODE_FP8_PER_TOKEN:
+    case FA_MODE_INT8_PER_TOKEN: blk = 1; nblk = t->S; break;
     case FA_MODE_FP8_BLOCK: blk = t->block_tokens; nblk = (t->S + t->block_tokens - 1) / t->block_tokens; break;
     default: blk = 0; nblk = 1; break;
   }
@@ -1358,6 +1371,11 @@ cudaError_t launch_attention_prefill2(const AttnArgs& a, void* ws, cudaStream_t 
       return q->D == 128 ? launch2_sc<K_E4M3, 128>(a, prm, w, sc, s) : launch2_sc<K_E4M3, 64>(a, prm, w, sc, s);
     case FA_MODE_INT8_PER_HEAD:
       return q->D == 128 ? launch_prefill<K_S8, 128, SC_HEAD>(a, prm, w, s) : launch_prefill<K_S8, 64, SC_HEAD>(a, prm, w, s);
+    case FA_MODE_FP8_PER_HEAD:
+      return q->D == 128 ? launch_prefill<K_E4M3, 128, SC_HEAD>(a, prm, w, s)
+                         : launch_prefill<K_E4M3, 64, SC_HEAD>(a, prm, w, s);
+    case FA_MODE_INT8_PER_TOKEN:
+      return q->D == 128 ? launch_prefill<K_S8, 128, SC_COL>(a, prm, w, s) : launch_prefill<K_S8, 64, SC_COL>(a, prm, w, s);
     case FA_MODE_MXFP4_PER_BLOCK:
       if (q->D != 128) return cudaErrorNotSupported;
       prm.qe8 = static_cast<const uint8_t*>(q->scales);

@@ -59,7 +59,7 @@ bool valid_layout(int l) { return l == FA_LAYOUT_BNSD || l == FA_LAYOUT_BSND; }
 
 bool quantized_mode(int m) {
   return m == FA_MODE_INT8_PER_HEAD || m == FA_MODE_FP8_PER_TOKEN || m == FA_MODE_MXFP4_PER_BLOCK ||
-         m == FA_MODE_FP8_BLOCK;
+         m == FA_MODE_FP8_BLOCK || m == FA_MODE_FP8_PER_HEAD || m == FA_MODE_INT8_PER_TOKEN;
 }
 
 fa_status check_tensor(const fa_tensor* t) {
@@ -139,13 +139,13 @@ fa_status fa_resolve_config(const fa_branch_cfg* qconfig, const fa_branch_cfg* d
   const bool has_d = details && (details[0].set || details[1].set || details[2].set);
   if (has_q && has_d) return FA_ERR_CONFIG_CONFLICT;
   if (has_q) {
-    if (qconfig->mode < FA_MODE_FLOAT || qconfig->mode > FA_MODE_FP8_BLOCK) return FA_ERR_INVALID_ARG;
+    if (qconfig->mode < FA_MODE_FLOAT || qconfig->mode > FA_MODE_INT8_PER_TOKEN) return FA_ERR_INVALID_ARG;
     modes_out[0] = modes_out[1] = modes_out[2] = qconfig->mode;
     return FA_OK;
   }
   if (has_d) {
     for (int i = 0; i < 3; ++i) {
-      if (details[i].set && (details[i].mode < FA_MODE_FLOAT || details[i].mode > FA_MODE_FP8_BLOCK))
+      if (details[i].set && (details[i].mode < FA_MODE_FLOAT || details[i].mode > FA_MODE_INT8_PER_TOKEN))
         return FA_ERR_INVALID_ARG;
       modes_out[i] = details[i].set ? details[i].mode : FA_MODE_FLOAT;
     }
@@ -180,7 +180,7 @@ fa_status fa_quantize(const fa_tensor* q, const fa_tensor* k, const fa_tensor* v
     if (st != FA_OK) return st;
     st = check_out(in[i], out[i], mode);
     if (st != FA_OK) return st;
-    if (mode == FA_MODE_INT8_PER_HEAD && !am[i]) return FA_ERR_NO_CALIBRATION;
+    if ((mode == FA_MODE_INT8_PER_HEAD || mode == FA_MODE_FP8_PER_HEAD) && !am[i]) return FA_ERR_NO_CALIBRATION;
     ops[n++] = make_op(in[i], out[i], am[i]);
   }
   if (n == 0) return FA_ERR_INVALID_ARG;
@@ -241,7 +241,8 @@ size_t fa_attention_workspace_size(const fa_qtensor* q, const fa_qtensor* k, int
     const int splits = num_splits > 0 ? num_splits : decode_auto_splits(k->B, k->H, k->S);
     return decode_workspace_bytes(q->B, q->H, q->D, splits);
   }
-  if (q->mode == FA_MODE_INT8_PER_HEAD || q->mode == FA_MODE_FP8_PER_TOKEN || q->mode == FA_MODE_FP8_BLOCK) {
+  if (q->mode == FA_MODE_INT8_PER_HEAD || q->mode == FA_MODE_FP8_PER_TOKEN || q->mode == FA_MODE_FP8_BLOCK ||
+      q->mode == FA_MODE_FP8_PER_HEAD || q->mode == FA_MODE_INT8_PER_TOKEN) {
     if (k->B < 0 || k->S < 0 || (q->D != 64 && q->D != 128)) return 0;
     return prefill2_workspace_bytes(k->B, k->H, k->S, q->D);
   }

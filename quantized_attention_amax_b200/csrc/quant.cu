@@ -88,13 +88,16 @@ __global__ void __launch_bounds__(256) quant_rows_kernel(QuantOperand o0, QuantO
   const int gl = lane % G;
   const int sub = lane / G;
 
-  if (MODE == FA_MODE_INT8_PER_HEAD && blockIdx.x == 0) {
+  // per-head static modes: one scale per head from the calibration maxima
+  constexpr bool PER_HEAD = MODE == FA_MODE_INT8_PER_HEAD || MODE == FA_MODE_FP8_PER_HEAD;
+  constexpr float QMAX = (MODE == FA_MODE_INT8_PER_HEAD || MODE == FA_MODE_INT8_PER_TOKEN) ? 127.0f : 448.0f;
+  if (PER_HEAD && blockIdx.x == 0) {
     for (int t = threadIdx.x; t < o0.H && o0.rows > 0; t += blockDim.x)
-      static_cast<float*>(o0.scales)[t] = __fdiv_rn(o0.amax[t], 127.0f);
+      static_cast<float*>(o0.scales)[t] = __fdiv_rn(o0.amax[t], QMAX);
     for (int t = threadIdx.x; t < o1.H && o1.rows > 0; t += blockDim.x)
-      static_cast<float*>(o1.scales)[t] = __fdiv_rn(o1.amax[t], 127.0f);
+      static_cast<float*>(o1.scales)[t] = __fdiv_rn(o1.amax[t], QMAX);
     for (int t = threadIdx.x; t < o2.H && o2.rows > 0; t += blockDim.x)
-      static_cast<float*>(o2.scales)[t] = __fdiv_rn(o2.amax[t], 127.0f);
+      static_cast<float*>(o2.scales)[t] = __fdiv_rn(o2.amax[t], QMAX);
   }
 
   const long long total = o0.rows + o1.rows + o2.rows;
@@ -145,15 +148,33 @@ __global__ void __launch_bounds__(256) quant_rows_kernel(QuantOperand o0, QuantO
           reinterpret_cast<uint2*>(static_cast<uint8_t*>(op.codes) + rr[u] * D)[gl] = out;
           if (gl == 0) static_cast<float*>(op.scales)[scale_index(rr[u], op.layout, op.H, op.S)] = sc;
         }
-      } else if (MODE == FA_MODE_INT8_PER_HEAD) {
+      } else if (PER_HEAD) {
+        // static scale: x can exceed the calibrated range, so IEEE division (codes saturate)
         float sc = 0.0f;
-        if (valid) sc = __fdiv_rn(__ldg(op.amax + head_of(rr[u], op.layout, op.H, op.S)), 127.0f);
+        if (valid) sc = __fdiv_rn(__ldg(op.amax + head_of(rr[u], op.layout, op.H, op.S)), QMAX);
+        float v[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) v[i] = sc > 0.0f ? __fdiv_rn(f[i], sc) : 0.0f;
+        if (valid) {
+          const uint2 out = MODE == FA_MODE_INT8_PER_HEAD
+                                ? make_uint2(s8x4(v[0], v[1], v[2], v[3]), s8x4(v[4], v[5], v[6], v[7]))
+                                : make_uint2(e4m3x4(v[0], v[1], v[2], v[3]), e4m3x4(v[4], v[5], v[6], v[7]));
+          reinterpret_cast<uint2*>(static_cast<uint8_t*>(op.codes) + rr[u] * D)[gl] = out;
+        }
+      } else if (MODE == FA_MODE_INT8_PER_TOKEN) {
+        float m = 0.0f;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) m = fmaxf(m, fabsf(f[i]));
+#pragma unroll
+        for (int off = G / 2; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+        const float sc = __fdiv_rn(m, 127.0f);
         float v[8];
 #pragma unroll
         for (int i = 0; i < 8; ++i) v[i] = sc > 0.0f ? __fdiv_rn(f[i], sc) : 0.0f;
         if (valid) {
           uint2 out = make_uint2(s8x4(v[0], v[1], v[2], v[3]), s8x4(v[4], v[5], v[6], v[7]));
           reinterpret_cast<uint2*>(static_cast<int8_t*>(op.codes) + rr[u] * D)[gl] = out;
+          if (gl == 0) static_cast<float*>(op.scales)[scale_index(rr[u], op.layout, op.H, op.S)] = sc;
         }
       } else {  // MXFP4: one 32-element block = 4 lanes
         float m = 0.0f;
@@ -271,7 +292,7 @@ template <int MODE>
 cudaError_t launch_rows_mode(const QuantOperand (&o)[3], int D, cudaStream_t s) {
   const long long total = o[0].rows + o[1].rows + o[2].rows;
   if (total == 0) {
-    if (MODE != FA_MODE_INT8_PER_HEAD) return cudaSuccess;
+    if (MODE != FA_MODE_INT8_PER_HEAD && MODE != FA_MODE_FP8_PER_HEAD) return cudaSuccess;
   }
   const int rows_per_block = (256 / 32) * (32 / (D / 8)) * 2;
   long long want = (total + rows_per_block - 1) / rows_per_block;
@@ -317,6 +338,8 @@ cudaError_t launch_quantize_rows(int mode, const QuantOperand* ops, int nops, cu
     case FA_MODE_FP8_PER_TOKEN: return launch_rows_mode<FA_MODE_FP8_PER_TOKEN>(o, D, s);
     case FA_MODE_INT8_PER_HEAD: return launch_rows_mode<FA_MODE_INT8_PER_HEAD>(o, D, s);
     case FA_MODE_MXFP4_PER_BLOCK: return launch_rows_mode<FA_MODE_MXFP4_PER_BLOCK>(o, D, s);
+    case FA_MODE_FP8_PER_HEAD: return launch_rows_mode<FA_MODE_FP8_PER_HEAD>(o, D, s);
+    case FA_MODE_INT8_PER_TOKEN: return launch_rows_mode<FA_MODE_INT8_PER_TOKEN>(o, D, s);
     default: return cudaErrorInvalidValue;
   }
 }

@@ -35,7 +35,7 @@ def run_case(faq, orc, mode, layout, D, B, Hq, Hkv, Sq, Sk, causal, seed, q_blk=
     v = gen(shp(B, Hkv, Sk, D, layout), seed + 2)
     bits = {n: wl.bf16_bits(t) for n, t in zip("qkv", (q, k, v))}
     amax = {}
-    if mode == "int8_per_head":
+    if mode in ("int8_per_head", "fp8_per_head"):
         for n, t in zip("qkv", (q, k, v)):
             cal = gen(t.shape, seed + 50 + "qkv".index(n))
             amax[n] = orc.calibrate_per_head(wl.bf16_bits(cal), layout)
@@ -45,7 +45,7 @@ def run_case(faq, orc, mode, layout, D, B, Hq, Hkv, Sq, Sk, causal, seed, q_blk=
     ref, ref_lse = orc.attention(oq["q"], oq["k"], oq["v"], causal, 0.0, rows)
     # GPU path
     dq, dk, dv = q.cuda(), k.cuda(), v.cuda()
-    if mode == "int8_per_head":
+    if mode in ("int8_per_head", "fp8_per_head"):
         am = [torch.from_numpy(amax[n]).cuda() for n in "qkv"]
         Q, K, V = faq.quantize(dq, dk, dv, mode, layout, amax=am)
     else:
@@ -77,6 +77,12 @@ CASES = [
     ("mxfp4", "BNSD", 128, 1, 2, 2, 300, 300, False),
     ("mxfp4", "BSND", 128, 2, 4, 2, 257, 257, True),
     ("mxfp4", "BNSD", 128, 1, 2, 1, 100, 300, True),
+    # FA PerHead FP8 and FA PerToken INT8 ("FA 量化", 该类下的模式清单)
+    ("fp8_per_head", "BNSD", 128, 2, 4, 2, 300, 300, True),
+    ("fp8_per_head", "BSND", 64, 1, 3, 3, 257, 257, False),
+    ("int8_per_token", "BNSD", 128, 2, 4, 2, 300, 300, True),
+    ("int8_per_token", "BSND", 64, 1, 2, 1, 100, 300, True),
+    ("int8_per_token", "BNSD", 128, 1, 3, 3, 384, 384, False),
 ]
 
 

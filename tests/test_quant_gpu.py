@@ -72,6 +72,51 @@ def test_int8_calibrate_and_quantize_bit_exact(faq, orc, layout, D, S):
         assert np.array_equal(np_of(o.codes), codes)
 
 
+@pytest.mark.parametrize("layout,D,S", CASES)
+def test_fp8_per_head_bit_exact(faq, orc, layout, D, S):
+    """FA PerHead with FP8: static scale amax_h / 448 from calibration; data past the
+    calibrated range saturates to +-448."""
+    cal = [rand_bf16(shp(2, 3, S, D, layout), 130 + i) for i in range(3)]
+    xs = [rand_bf16(shp(2, 3, S, D, layout), 140 + i, scale=1.5) for i in range(3)]
+    amax = [faq.calibrate_per_head(c.cuda(), layout) for c in cal]
+    out = faq.quantize(*[x.cuda() for x in xs], "fp8_per_head", layout, amax=amax)
+    torch.cuda.synchronize()
+    for c, x, o in zip(cal, xs, out):
+        ra = orc.calibrate_per_head(wl.bf16_bits(c), layout)
+        codes, scales = orc.quantize_fp8_per_head(wl.bf16_bits(x), ra, layout)
+        assert np.array_equal(np_of(o.scales), scales)
+        assert np.array_equal(np_of(o.codes), codes)
+
+
+@pytest.mark.parametrize("layout,D,S", CASES)
+def test_int8_per_token_bit_exact(faq, orc, layout, D, S):
+    """FA PerToken with INT8: dynamic scale amax_token / 127."""
+    xs = [rand_bf16(shp(2, 3, S, D, layout), 150 + i, scale=[1.0, 30.0, 1e-3][i]) for i in range(3)]
+    out = faq.quantize(*[x.cuda() for x in xs], "int8_per_token", layout)
+    torch.cuda.synchronize()
+    for x, o in zip(xs, out):
+        codes, scales = orc.quantize_int8_per_token(wl.bf16_bits(x), layout)
+        assert np.array_equal(np_of(o.scales), scales)
+        assert np.array_equal(np_of(o.codes), codes)
+
+
+def test_new_modes_exhaustive(faq, orc):
+    """Every finite bf16 value through both new modes (rows of 128)."""
+    bits = np.arange(65536, dtype=np.uint32)
+    f = (bits << 16).view(np.float32)
+    fin = bits[np.isfinite(f)].astype(np.uint16)
+    x = np.resize(fin, 4 * 128 * 130).reshape(1, 4, 130, 128)
+    am = np.array([448.0, 3.3e-3, 1.0, 7.5e4], np.float32)
+    o, = faq.quantize(bf16_from_bits(x), None, None, "fp8_per_head", amax=[torch.from_numpy(am).cuda(), None, None])[:1]
+    torch.cuda.synchronize()
+    codes, scales = orc.quantize_fp8_per_head(x, am)
+    assert np.array_equal(np_of(o.scales), scales) and np.array_equal(np_of(o.codes), codes)
+    o, = faq.quantize(bf16_from_bits(x), None, None, "int8_per_token")[:1]
+    torch.cuda.synchronize()
+    codes, scales = orc.quantize_int8_per_token(x)
+    assert np.array_equal(np_of(o.scales), scales) and np.array_equal(np_of(o.codes), codes)
+
+
 @pytest.mark.parametrize("layout,D,S,blk", [("BSND", 128, 300, 128), ("BSND", 128, 300, 256),
                                              ("BNSD", 64, 300, 100), ("BNSD", 128, 1, 128)])
 def test_fp8_block_bit_exact(faq, orc, layout, D, S, blk):

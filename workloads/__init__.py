@@ -31,7 +31,7 @@ import torch
 @dataclass(frozen=True)
 class Workload:
     name: str
-    mode: str          # int8_per_head | fp8_per_token | fp8_block | mxfp4
+    mode: str          # int8_per_head | fp8_per_token | fp8_block | mxfp4 | fp8_per_head | int8_per_token
     B: int
     Hq: int
     Hkv: int
@@ -58,6 +58,13 @@ WORKLOADS: Dict[str, Workload] = {
                               "normal", 2, rotate=True),
     "mxfp4": Workload("mxfp4", "mxfp4", 1, 24, 24, 4096, 4096, 128, "BNSD", False, "student_t4", 3),
     "int8_decode": Workload("int8_decode", "int8_per_head", 16, 32, 8, 1, 32768, 128, "BNSD", False, "normal", 4),
+    # the FP8 prefill shape in the other static / dynamic modes (supplemental measurements)
+    "int8_prefill": Workload("int8_prefill", "int8_per_head", 2, 32, 8, 4096, 4096, 128, "BNSD", True,
+                             "normal_k_outliers", 5),
+    "fp8_head_prefill": Workload("fp8_head_prefill", "fp8_per_head", 2, 32, 8, 4096, 4096, 128, "BNSD", True,
+                                 "normal_k_outliers", 6),
+    "int8_token_prefill": Workload("int8_token_prefill", "int8_per_token", 2, 32, 8, 4096, 4096, 128, "BNSD", True,
+                                   "normal_k_outliers", 7),
 }
 
 CALIB_SEED_OFFSET = 1000
@@ -146,7 +153,7 @@ def make_inputs(w: Workload, device="cpu", calib: bool = True) -> Dict[str, Opti
         "v": _draw(w, "v", ks, 3 * w.seed + 2 + 100, device),
         "R": rotation(w.D, w.seed, device) if w.rotate else None,
     }
-    if calib and w.mode == "int8_per_head":
+    if calib and w.mode in ("int8_per_head", "fp8_per_head"):
         c = CALIB_SEED_OFFSET
         out["q_cal"] = _draw(w, "q", qs, 3 * w.seed + 0 + 100 + c, device)
         out["k_cal"] = _draw(w, "k", ks, 3 * w.seed + 1 + 100 + c, device)
