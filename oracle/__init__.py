@@ -23,7 +23,7 @@ from . import build as _build
 
 LAYOUTS = {"BNSD": 0, "BSND": 1}
 MODES = {"float": 0, "int8_per_head": 1, "fp8_per_token": 2, "mxfp4": 3, "fp8_block": 4, "fp8_per_head": 5,
-         "int8_per_token": 6}
+         "int8_per_token": 6, "mxfp8": 7}
 
 _lib = None
 
@@ -53,7 +53,7 @@ def lib() -> ctypes.CDLL:
         L.orc_mx_exponent.restype = ctypes.c_int
         L.orc_mx_exponent.argtypes = [ctypes.c_float]
         for name in ("orc_e4m3_encode_n", "orc_e2m1_encode_n", "orc_int8_encode_n",
-                     "orc_mx_exponent_n", "orc_f64_to_bf16_n"):
+                     "orc_mx_exponent_n", "orc_mx_exponent_e4m3_n", "orc_f64_to_bf16_n"):
             getattr(L, name).restype = None
             getattr(L, name).argtypes = [P, P, Z]
         L.orc_calibrate_per_head.argtypes = [P, I, I, I, I, I, P]
@@ -62,6 +62,7 @@ def lib() -> ctypes.CDLL:
         L.orc_quantize_fp8_per_head.argtypes = [P, I, I, I, I, I, P, P, P]
         L.orc_quantize_int8_per_token.argtypes = [P, I, I, I, I, I, P, P]
         L.orc_quantize_mxfp4.argtypes = [P, I, I, I, I, I, P, P]
+        L.orc_quantize_mxfp8.argtypes = [P, I, I, I, I, I, P, P]
         L.orc_rotate_f64.argtypes = [P, I, I, I, I, I, P, P]
         L.orc_rotate.argtypes = [P, I, I, I, I, I, P, P]
         L.orc_quantize_fp8_block.argtypes = [P, I, I, I, I, I, I, P, P]
@@ -143,6 +144,13 @@ def mx_exponent(amax: np.ndarray) -> np.ndarray:
     return out
 
 
+def mx_exponent_e4m3(amax: np.ndarray) -> np.ndarray:
+    amax = np.ascontiguousarray(amax, dtype=np.float32)
+    out = np.empty(amax.shape, np.int32)
+    lib().orc_mx_exponent_e4m3_n(_ptr(amax), _ptr(out), amax.size)
+    return out
+
+
 def f64_to_bf16(v: np.ndarray) -> np.ndarray:
     v = np.ascontiguousarray(v, dtype=np.float64)
     out = np.empty(v.shape, np.uint16)
@@ -207,6 +215,15 @@ def quantize_mxfp4(x: np.ndarray, layout: str = "BNSD"):
     codes = np.empty(x.shape[:-1] + (D // 2,), np.uint8)
     e8m0 = np.empty((B, H, S, D // 32), np.uint8)
     lib().orc_quantize_mxfp4(_ptr(x), B, H, S, D, LAYOUTS[layout], _ptr(codes), _ptr(e8m0))
+    return codes, e8m0
+
+
+def quantize_mxfp8(x: np.ndarray, layout: str = "BNSD"):
+    x = np.ascontiguousarray(x, dtype=np.uint16)
+    B, H, S, D = dims(x.shape, layout)
+    codes = np.empty(x.shape, np.uint8)
+    e8m0 = np.empty((B, H, S, D // 32), np.uint8)
+    lib().orc_quantize_mxfp8(_ptr(x), B, H, S, D, LAYOUTS[layout], _ptr(codes), _ptr(e8m0))
     return codes, e8m0
 
 

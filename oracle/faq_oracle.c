@@ -177,6 +177,18 @@ int orc_mx_exponent(float amax) {
   return x;
 }
 
+/* The same rule for E4M3 elements ([FA] 模式清单, FA PerBlock with MXFP8):
+ * floor(log2 amax) - 8, E4M3's largest exponent (max 448 = 1.75 * 2^8). */
+int orc_mx_exponent_e4m3(float amax) {
+  if (!(amax > 0.0f)) return -127;
+  int e;
+  frexp((double)amax, &e);
+  int x = (e - 1) - 8;
+  if (x < -127) x = -127;
+  if (x > 127) x = 127;
+  return x;
+}
+
 /* ------------------------------------------------------------------------ */
 /* Quantizers                                                                */
 /* ------------------------------------------------------------------------ */
@@ -372,6 +384,32 @@ void orc_quantize_fp8_block(const uint16_t* x, int B, int H, int S, int D,
       }
 }
 
+/* [FA] 模式清单, FA PerBlock with MXFP8: as 组合3, 32 consecutive elements of
+ * head_dim share X = 2^e, e = floor(log2 amax) - 8, with E4M3 elements
+ * e4m3(x / X) (x / X < 512; values above 448 saturate). */
+void orc_quantize_mxfp8(const uint16_t* x, int B, int H, int S, int D,
+                        int layout, uint8_t* codes, uint8_t* e8m0) {
+  const int G = D / 32;
+#pragma omp parallel for collapse(3) schedule(static)
+  for (int b = 0; b < B; ++b)
+    for (int h = 0; h < H; ++h)
+      for (int s = 0; s < S; ++s)
+        for (int g = 0; g < G; ++g) {
+          float amax = 0.0f;
+          for (int j = 0; j < 32; ++j) {
+            const float a = fabsf(orc_bf16_to_f32(x[elem_index(layout, H, S, D, b, h, s, g * 32 + j)]));
+            if (a > amax) amax = a;
+          }
+          const int e = orc_mx_exponent_e4m3(amax);
+          e8m0[(((size_t)b * H + h) * S + s) * G + g] = (uint8_t)(e + 127);
+          const float X = ldexpf(1.0f, e);
+          for (int j = 0; j < 32; ++j) {
+            const size_t i = elem_index(layout, H, S, D, b, h, s, g * 32 + j);
+            codes[i] = orc_e4m3_encode(orc_bf16_to_f32(x[i]) / X);
+          }
+        }
+}
+
 /* ------------------------------------------------------------------------ */
 /* FakeQuant dequantization ([MODE] 模式索引: quantize, then dequantize)      */
 /* ------------------------------------------------------------------------ */
@@ -386,6 +424,11 @@ double orc_dequant_elem(const orc_qt* t, int b, int h, int s, int d) {
     case ORC_MODE_FP8_PER_TOKEN:
       return orc_e4m3_decode(((const uint8_t*)t->codes)[i]) *
              (double)((const float*)t->scales)[((size_t)b * t->H + h) * t->S + s];
+    case ORC_MODE_MXFP8: {
+      const int G = t->D / 32;
+      const int e = (int)((const uint8_t*)t->scales)[(((size_t)b * t->H + h) * t->S + s) * G + d / 32] - 127;
+      return ldexp(orc_e4m3_decode(((const uint8_t*)t->codes)[i]), e);
+    }
     case ORC_MODE_FP8_PER_HEAD:
       return orc_e4m3_decode(((const uint8_t*)t->codes)[i]) * (double)((const float*)t->scales)[h];
     case ORC_MODE_INT8_PER_TOKEN:
@@ -497,6 +540,9 @@ void orc_e2m1_encode_n(const float* v, uint8_t* out, size_t n) {
 }
 void orc_int8_encode_n(const float* v, int8_t* out, size_t n) {
   for (size_t i = 0; i < n; ++i) out[i] = orc_int8_encode(v[i]);
+}
+void orc_mx_exponent_e4m3_n(const float* v, int* out, size_t n) {
+  for (size_t i = 0; i < n; ++i) out[i] = orc_mx_exponent_e4m3(v[i]);
 }
 void orc_mx_exponent_n(const float* v, int* out, size_t n) {
   for (size_t i = 0; i < n; ++i) out[i] = orc_mx_exponent(v[i]);

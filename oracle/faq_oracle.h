@@ -33,7 +33,7 @@
  *   FP8 per token  : fp32 [B, H, S]
  *   INT8 per token : fp32 [B, H, S]
  *   FP8 block      : fp32 [B, H, ceil(S / blk)]
- *   MXFP4          : uint8 E8M0 [B, H, S, D / 32]
+ *   MXFP4, MXFP8   : uint8 E8M0 [B, H, S, D / 32]
  * MXFP4 codes are packed [.., D/2] in the data layout, element 2i in the low
  * nibble, 2i+1 in the high nibble.
  */
@@ -55,7 +55,8 @@ enum {
   ORC_MODE_MXFP4 = 3,          /* [FA] 组合3                                  */
   ORC_MODE_FP8_BLOCK = 4,      /* [SD] FA量化 块量化                           */
   ORC_MODE_FP8_PER_HEAD = 5,   /* [FA] 模式清单: FA PerHead, FP8               */
-  ORC_MODE_INT8_PER_TOKEN = 6  /* [FA] 模式清单: FA PerToken, INT8             */
+  ORC_MODE_INT8_PER_TOKEN = 6, /* [FA] 模式清单: FA PerToken, INT8             */
+  ORC_MODE_MXFP8 = 7           /* [FA] 模式清单: FA PerBlock, MXFP8            */
 };
 
 /* A quantized (or bf16) operand as the oracle sees it. */
@@ -77,6 +78,7 @@ uint8_t  orc_e2m1_encode(float v);      /* 4-bit E2M1, RNE, sat +-6         */
 double   orc_e2m1_decode(uint8_t c);
 int8_t   orc_int8_encode(float v);      /* RNE to integer, clamp [-128,127] */
 int      orc_mx_exponent(float amax);   /* floor(log2 amax) - 2, [-127,127] */
+int      orc_mx_exponent_e4m3(float amax); /* floor(log2 amax) - 8, [-127,127] */
 
 /* ---- quantizers ---------------------------------------------------------*/
 void orc_calibrate_per_head(const uint16_t* x, int B, int H, int S, int D,
@@ -95,6 +97,9 @@ void orc_quantize_int8_per_token(const uint16_t* x, int B, int H, int S, int D,
                                  float* scales /* [B,H,S] */);
 void orc_quantize_mxfp4(const uint16_t* x, int B, int H, int S, int D,
                         int layout, uint8_t* codes /* packed */,
+                        uint8_t* e8m0 /* [B,H,S,D/32] */);
+void orc_quantize_mxfp8(const uint16_t* x, int B, int H, int S, int D,
+                        int layout, uint8_t* codes /* e4m3 [..D] */,
                         uint8_t* e8m0 /* [B,H,S,D/32] */);
 void orc_rotate_f64(const uint16_t* x, int B, int H, int S, int D, int layout,
                     const uint16_t* R /* [D,D] row-major, x*R */,

@@ -119,3 +119,75 @@ def test_dequantize_new_modes_by_hand(orc):
     qt = orc.QT("int8_per_token", ct, st, 1, 2, 64, 64)
     assert np.array_equal(orc.dequant(qh), orc.e4m3_decode(ch) * sh[None, :, None, None].astype(np.float64))
     assert np.array_equal(orc.dequant(qt), ct.astype(np.float64) * st[..., None])
+
+
+# --------------------------------------------------------------- MXFP8 --
+# FA PerBlock with E4M3 elements: the 组合3 rule with E4M3's largest exponent, 8
+# (448 = 1.75 * 2^8), in place of E2M1's 2.
+
+def test_mx_exponent_e4m3_brute_force(orc):
+    bits = np.arange(1, 0x7F80, dtype=np.uint32)  # every positive finite bf16
+    x = (bits << 16).view(np.float32)
+    got = orc.mx_exponent_e4m3(x)
+    # e is the integer with 2^(e+8) <= amax < 2^(e+9), clamped to [-127, 127]
+    lo = np.floor(np.log2(x.astype(np.float64))).astype(np.int64) - 8
+    exp = np.clip(lo, -127, 127)
+    assert np.array_equal(got, exp)
+    for a, e in zip(x[::997].astype(np.float64), got[::997]):  # the bracket, checked in exact arithmetic
+        if -127 < e < 127:
+            assert np.ldexp(1.0, int(e) + 8) <= a < np.ldexp(1.0, int(e) + 9)
+    assert orc.mx_exponent_e4m3(np.array([0.0], np.float32))[0] == -127
+    # the E4M3 exponent is the E2M1 exponent shifted by the two formats' emax difference
+    big = (got > -127) & (got < 121)
+    assert np.array_equal(got[big], orc.mx_exponent(x[big]) - 6)
+
+
+def test_mxfp8_invariants(orc):
+    x = bits_of(wl.student_t4((1, 3, 50, 128), 41))
+    codes, e8 = orc.quantize_mxfp8(x)
+    assert codes.shape == (1, 3, 50, 128) and e8.shape == (1, 3, 50, 4)
+    xf = f32(orc, x).astype(np.float64)
+    blocks = xf.reshape(1, 3, 50, 4, 32)
+    amax = np.abs(blocks).max(-1)
+    e = e8.astype(np.int64) - 127
+    X = np.ldexp(1.0, np.repeat(e, 32, axis=-1))
+    ratio = amax / np.ldexp(1.0, e)
+    assert ((ratio >= 256) & (ratio < 512)).all()
+    deq = orc.e4m3_decode(codes) * X
+    # the block maximum codes to an E4M3 magnitude in [256, 448]
+    top = np.take_along_axis(codes.reshape(1, 3, 50, 4, 32), np.argmax(np.abs(blocks), -1)[..., None], -1)[..., 0]
+    assert np.isin(top & 0x7F, np.arange(0x78, 0x7F)).all()
+    # error: half an E4M3 step (relative 2^-4 in the normal range) or saturation beyond 448
+    v = np.abs(xf) / X
+    bound = np.where(v <= 448, np.where(v >= 2.0 ** -6, v * 2.0 ** -4, 2.0 ** -10), v - 448) * X
+    assert (np.abs(deq - xf) <= bound * (1 + 1e-9) + 1e-300).all()
+    cb, eb = orc.quantize_mxfp8(to_bsnd(x), "BSND")
+    assert np.array_equal(cb, to_bsnd(codes)) and np.array_equal(eb, e8)
+
+
+def test_mxfp8_grid_round_trip_and_zero_block(orc):
+    rng = np.random.default_rng(42)
+    fin = np.array([c for c in range(256) if (c & 0x7F) != 0x7F], np.uint8)
+    big = fin[(orc.e4m3_decode(fin) >= 256)]  # magnitudes 256..448
+    ok = fin[np.abs(orc.e4m3_decode(fin)) >= 2.0 ** -3]
+    rows, es = [], []
+    for t in range(16):
+        blk = []
+        for g in range(4):
+            c = rng.choice(ok, 32)
+            c[rng.integers(32)] = rng.choice(big)  # the block max in [256, 448]: the exponent is k exactly
+            blk.append(c)
+            es.append(int(rng.integers(-20, 20)))
+        rows.append(np.concatenate(blk))
+    codes = np.array(rows, np.uint8).reshape(1, 1, 16, 128)
+    X = np.ldexp(1.0, np.repeat(np.array(es).reshape(1, 1, 16, 4), 32, axis=-1))
+    x = bf16_from_f32((orc.e4m3_decode(codes) * X).astype(np.float32))
+    c2, e8 = orc.quantize_mxfp8(x)
+    assert np.array_equal(e8.astype(np.int64) - 127, np.array(es).reshape(1, 1, 16, 4))
+    assert np.array_equal(c2, codes)
+    z = np.zeros((1, 1, 2, 64), np.uint16)
+    z[0, 0, 0, 3] = 0x8000
+    cz, ez = orc.quantize_mxfp8(z)
+    assert not ez.any() and np.array_equal(cz[0, 0, 0, 3], np.uint8(0x80)) and (cz & 0x7F == 0).all()
+    q = orc.QT("mxfp8", codes, e8, 1, 1, 16, 128)
+    assert np.array_equal(orc.dequant(q), orc.e4m3_decode(codes) * X)
