@@ -45,6 +45,7 @@ DESCR = {
     "int8_prefill": "INT8 per-head static, the fp8_prefill shape (B=2 Hq=32 Hkv=8 S=4096 D=128, causal, BNSD)",
     "fp8_head_prefill": "FP8 E4M3 per-head static, the fp8_prefill shape (B=2 Hq=32 Hkv=8 S=4096 D=128, causal, BNSD)",
     "int8_token_prefill": "INT8 per-token dynamic, the fp8_prefill shape (B=2 Hq=32 Hkv=8 S=4096 D=128, causal, BNSD)",
+    "mxfp8": "MXFP8 per-32-block (E4M3 + E8M0), the mxfp4 shape (B=1 H=24 S=4096 D=128, non-causal, BNSD, Student-t)",
 }
 DATA = {
     "int8_tiny": "synthetic: seeded bf16 N(0,1); per-head scales from a seeded calibration batch",
@@ -55,6 +56,7 @@ DATA = {
     "int8_prefill": "synthetic: as fp8_prefill; per-head scales from seeded calibration batches",
     "fp8_head_prefill": "synthetic: as fp8_prefill; per-head scales from seeded calibration batches",
     "int8_token_prefill": "synthetic: as fp8_prefill",
+    "mxfp8": "synthetic: seeded bf16 Student-t (df=4)",
 }
 DTYPE = {
     "int8_tiny": "s8 (QK^T, s32 acc) + f16 (PV)",
@@ -65,6 +67,7 @@ DTYPE = {
     "int8_prefill": "s8 (QK^T, s32 acc) + f16 (PV)",
     "fp8_head_prefill": "e4m3 (QK^T) + f16 (PV), fp32 accumulate",
     "int8_token_prefill": "s8 (QK^T, s32 acc) + f16 (PV)",
+    "mxfp8": "e4m3 block-scaled (QK^T) + f16 (PV)",
 }
 
 
@@ -92,7 +95,7 @@ def quant_bytes(w) -> float:
         sc = (w.B * w.Hq * w.Sq + 2 * w.B * w.Hkv * w.Sk) * 4
     elif w.mode == "fp8_block":
         sc = (w.B * w.Hq * -(-w.Sq // w.q_block) + 2 * w.B * w.Hkv * -(-w.Sk // w.kv_block)) * 4
-    elif w.mode == "mxfp4":
+    elif w.mode in ("mxfp4", "mxfp8"):
         sc = (nq + 2 * nk) // 32
     else:
         sc = (w.Hq + 2 * w.Hkv) * 4
@@ -244,7 +247,7 @@ def attention_kernels(w):
     """(label, source file) of the attention call's kernels for this workload."""
     if w.name == "int8_decode":
         return "decode_kernel + attn_combine_kernel", "decode.cu"
-    if w.mode == "mxfp4":
+    if w.mode in ("mxfp4", "mxfp8"):
         return "vprep_kernel + attn2_kernel (one fa_attention_quant call)", "attn2.cu"
     return "vprep_kernel + attn_pair_kernel (one fa_attention_quant call)", "attn2.cu"
 
@@ -450,6 +453,9 @@ def oracle_sample(w, reps_seconds=None):
         elif w.mode == "mxfp4":
             (cq, sq), (ck, sk), (cv, sv) = (orc.quantize_mxfp4(x, L) for x in (qb, kb, vb))
             blks = (0, 0, 0)
+        elif w.mode == "mxfp8":
+            (cq, sq), (ck, sk), (cv, sv) = (orc.quantize_mxfp8(x, L) for x in (qb, kb, vb))
+            blks = (0, 0, 0)
         else:
             qr = orc.rotate(qb, Rb, L) if Rb is not None else qb
             kr = orc.rotate(kb, Rb, L) if Rb is not None else kb
@@ -517,7 +523,7 @@ def supplemental(args, device):
     out = {}
     pk = peaks()
     for name in ("int8_tiny", "rot_fp8_block", "mxfp4", "int8_decode", "int8_prefill", "fp8_head_prefill",
-                 "int8_token_prefill"):
+                 "int8_token_prefill", "mxfp8"):
         w = wl.WORKLOADS[name]
         a = argparse.Namespace(steps=10 if name != "rot_fp8_block" else 4, warmup=3)
         r = gpu_run(a, w, 0, 1, device)

@@ -31,6 +31,7 @@
  *                            scales uint8 E8M0 [B, H, S, D/32]
  *   FA_MODE_FP8_PER_HEAD     codes e4m3 [..D];   scales fp32 [H]
  *   FA_MODE_INT8_PER_TOKEN   codes int8 [..D];   scales fp32 [B, H, S]
+ *   FA_MODE_MXFP8_PER_BLOCK  codes e4m3 [..D];   scales uint8 E8M0 [B, H, S, D/32]
  */
 #ifndef FAQ_H
 #define FAQ_H
@@ -73,7 +74,8 @@ typedef enum {
   FA_MODE_MXFP4_PER_BLOCK = 3, /* 组合3: E2M1 + E8M0 per 32 elements of head_dim   */
   FA_MODE_FP8_BLOCK = 4,       /* 块量化: E4M3, one scale per block of tokens      */
   FA_MODE_FP8_PER_HEAD = 5,    /* FA PerHead, FP8: per-head static, s = amax/448   */
-  FA_MODE_INT8_PER_TOKEN = 6   /* FA PerToken, INT8: per-token dynamic, s = amax/127 */
+  FA_MODE_INT8_PER_TOKEN = 6,  /* FA PerToken, INT8: per-token dynamic, s = amax/127 */
+  FA_MODE_MXFP8_PER_BLOCK = 7  /* FA PerBlock, MXFP8: E4M3 + E8M0 per 32 elements  */
 } fa_mode;
 
 /* A bf16 activation tensor. */
@@ -137,7 +139,9 @@ FAQ_API fa_status fa_calibrate_per_head(const fa_tensor* x, float* amax_h, fa_st
  *   (E4M3 with one scale = amax/448 per block of block_tokens tokens);
  *   "FA 量化", 该类下的模式清单: FA PerHead with FP8 (组合1's calibration,
  *   s_h = amax_h/448, values past the calibrated range saturate to +-448) and
- *   FA PerToken with INT8 (组合2's per-token amax, s = amax_token/127).
+ *   FA PerToken with INT8 (组合2's per-token amax, s = amax_token/127) and
+ *   FA PerBlock with MXFP8 (组合3's rule with E4M3 elements: per 32 elements
+ *   of head_dim, e = floor(log2 amax) - 8, code = e4m3(x / 2^e), saturating).
  *   Rounding is round-half-to-even, saturating; x / s is rounded as one IEEE
  *   fp32 division; a zero scale gives zero codes.
  *   q, k, v: bf16 inputs; any of them may be NULL to skip that operand.
@@ -195,8 +199,8 @@ FAQ_API fa_status fa_rotate_quantize(const fa_tensor* q, const fa_tensor* k, con
  *   r_t (E_t), and 512 bytes of K scales per tile (128 per-key floats, or
  *   MXFP4's scale-factor atom).  num_splits (decode only): 0 = automatic.
  *   Modes run here: INT8_PER_HEAD, FP8_PER_TOKEN, FP8_BLOCK, MXFP4_PER_BLOCK,
- *   FP8_PER_HEAD and INT8_PER_TOKEN for prefill; INT8_PER_HEAD for decode
- *   (others -> FA_ERR_UNSUPPORTED).
+ *   FP8_PER_HEAD, INT8_PER_TOKEN and MXFP8_PER_BLOCK for prefill (the MX modes
+ *   with D == 128); INT8_PER_HEAD for decode (others -> FA_ERR_UNSUPPORTED).
  */
 FAQ_API fa_status fa_attention_quant(const fa_qtensor* q, const fa_qtensor* k, const fa_qtensor* v, int causal,
                              float softmax_scale, void* out, float* lse, int num_splits, void* workspace,
@@ -236,7 +240,7 @@ FAQ_API fa_status fa_attention_decode_noalloc(const fa_qtensor* q, const fa_qten
                                               fa_stream_t s);
 
 /* Workspace bytes fa_attention_quant needs for these operands and split
- * count: decode B*Hq*splits*(D+2)*4; prefill (every mode, MXFP4 with
+ * count: decode B*Hq*splits*(D+2)*4; prefill (every mode, the MX modes with
  * D == 128 only) B*Hkv*Sk*D*2 + B*Hkv*ceil(Sk/128)*16 +
  * B*Hkv*ceil(Sk/128)*512, each part rounded up to 256.  Returns 0 on
  * invalid arguments. */

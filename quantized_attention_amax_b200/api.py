@@ -17,7 +17,7 @@ from . import _native as N
 
 LAYOUTS = {"BNSD": 0, "BSND": 1}
 MODES = {"float": 0, "int8_per_head": 1, "fp8_per_token": 2, "mxfp4": 3, "fp8_block": 4, "fp8_per_head": 5,
-         "int8_per_token": 6}
+         "int8_per_token": 6, "mxfp8": 7}
 MODE_NAMES = {v: k for k, v in MODES.items()}
 
 
@@ -91,6 +91,9 @@ def empty_qtensor(B: int, H: int, S: int, D: int, mode: str, layout: str = "BNSD
         scales = torch.empty((B, H, (S + block_tokens - 1) // block_tokens), dtype=torch.float32, device=device)
     elif mode == "mxfp4":
         codes = torch.empty(shp[:-1] + (D // 2,), dtype=torch.uint8, device=device)
+        scales = torch.empty((B, H, S, D // 32), dtype=torch.uint8, device=device)
+    elif mode == "mxfp8":
+        codes = torch.empty(shp, dtype=torch.uint8, device=device)
         scales = torch.empty((B, H, S, D // 32), dtype=torch.uint8, device=device)
     else:
         raise ValueError(f"unknown mode {mode!r}")

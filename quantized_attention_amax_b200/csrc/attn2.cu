@@ -65,7 +65,7 @@ constexpr int NKS = 3;      // K code stages
 constexpr int NVS = 2;      // V' stages
 constexpr int NSC = 4;      // scale ring stages
 
-enum { K_E4M3 = 0, K_S8 = 1, K_MXF4 = 2 };
+enum { K_E4M3 = 0, K_S8 = 1, K_MXF4 = 2, K_MXF8 = 3 };
 enum { SC_HEAD = 0, SC_COL = 1, SC_TILE = 2 };  // one scale per head / per key / per 128-key tile
 
 struct P2 {
@@ -90,7 +90,7 @@ struct P2 {
 
 template <int KIND, int D>
 struct L2 {
-  static constexpr uint32_t RB = KIND == K_MXF4 ? D / 2 : D;  // code bytes per token row
+  static constexpr uint32_t RB = KIND == K_MXF4 ? D / 2 : D;  // code bytes per token row (E2M1: two per byte)
   static constexpr uint32_t Q = 0;                     // [128][RB]
   static constexpr uint32_t K = Q + BM * RB;           // NKS stages
   static constexpr uint32_t VH = K + NKS * BN * RB;    // NVS stages of fp16 V'
@@ -134,7 +134,7 @@ __global__ void __launch_bounds__(Cfg<NSW>::NT, 1)
     attn2_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
                  const __grid_constant__ CUtensorMap tmv, const P2 p) {
   static_assert(KIND == K_E4M3 || SC == SC_HEAD, "INT8 and MXFP4 operands take no per-key scale path");
-  constexpr bool MX = KIND == K_MXF4;
+  constexpr bool MX = KIND == K_MXF4 || KIND == K_MXF8;  // block-scaled QK^T (UE8M0 factors in TMEM)
   constexpr bool RING = MX || SC != SC_HEAD;  // per-tile records (and K scales / atoms) through the scale ring
   using L = L2<KIND, D>;
   constexpr uint32_t RB = L::RB;
@@ -289,7 +289,7 @@ __global__ void __launch_bounds__(Cfg<NSW>::NT, 1)
         constexpr uint32_t SBO8 = RB == 128 ? 1024 : 512;
         constexpr uint32_t idesc_qk = KIND == K_E4M3 ? make_idesc(kAccF32, kFmtE4M3, kFmtE4M3, 0, 0, BN, BM)
                                                      : make_idesc(kAccS32, kFmtS8, kFmtS8, 0, 0, BN, BM);
-        static_assert(!MX || RB == 64, "MXFP4 path: head_dim 128");
+        static_assert(!MX || D == 128, "MX paths: head_dim 128");
         constexpr uint32_t idesc_pv = make_idesc(kAccF32, kFmtF16, kFmtF16, 0, 1, D, BM);
         const uint32_t sQ = smem_u32(smem + L::Q);
         auto qk = [&](int j) {
@@ -304,9 +304,12 @@ __global__ void __launch_bounds__(Cfg<NSW>::NT, 1)
               mma_f8f6f4(tbase + (j & 1) * 128, da, db, idesc_qk, kk > 0);
             else if (KIND == K_S8)
               mma_i8(tbase + (j & 1) * 128, da, db, idesc_qk, kk > 0);
-            else  // 64 E2M1 per MMA: scale bytes 2kk and 2kk + 1 of each row
+            else if (KIND == K_MXF4)  // 64 E2M1 per MMA: scale bytes 2kk and 2kk + 1 of each row
               mma_mxf4(tbase + (j & 1) * 128, da, db, make_idesc_bs(kFmtE2M1x, kFmtE2M1x, BN, BM, 2 * kk, 2 * kk),
                        tSFA, tSFB[j & 1], kk > 0);
+            else  // 32 E4M3 per MMA: scale byte kk of each row
+              mma_mxf8(tbase + (j & 1) * 128, da, db, make_idesc_bs(kFmtE4M3, kFmtE4M3, BN, BM, kk, kk), tSFA,
+                       tSFB[j & 1], kk > 0);
           }
           mma_commit(&bar[X_SF + (j & 1)]);
           mma_commit(&bar[X_KE + j % NKS]);
@@ -1089,13 +1092,15 @@ __global__ void __launch_bounds__(256) vprep_kernel(const uint8_t* __restrict__ 
   const int tok = tok0 + warp * 16 + (lane >> 1);
   const bool live = tok < S;  // rows past S stay unwritten: the attention's TMA box reads them as zero
   const long long src_row = layout == FA_LAYOUT_BNSD ? ((long long)bh * S + tok) : (((long long)b * S + tok) * H + h);
-  if constexpr (KIND == K_MXF4) {
-    static_assert(D == 128, "MXFP4 path: head_dim 128");
-    // each thread owns half a 64-byte code row: two 32-element scale blocks of 16 bytes
-    const uint8_t* src = codes + src_row * (D / 2) + (lane & 1) * (D / 4);
-    uint4 raw[2];
+  if constexpr (KIND == K_MXF4 || KIND == K_MXF8) {
+    static_assert(D == 128, "MX paths: head_dim 128");
+    constexpr bool F8 = KIND == K_MXF8;
+    // each thread owns half a code row: two 32-element scale blocks of 16 (E2M1) or 32 (E4M3) bytes
+    constexpr int NC = F8 ? 4 : 2;  // 16-byte chunks per thread
+    const uint8_t* src = codes + src_row * (F8 ? D : D / 2) + (lane & 1) * (F8 ? D / 2 : D / 4);
+    uint4 raw[NC];
 #pragma unroll
-    for (int c = 0; c < 2; ++c) raw[c] = live ? __ldg(reinterpret_cast<const uint4*>(src) + c) : make_uint4(0, 0, 0, 0);
+    for (int c = 0; c < NC; ++c) raw[c] = live ? __ldg(reinterpret_cast<const uint4*>(src) + c) : make_uint4(0, 0, 0, 0);
     const uint32_t* ve4 = reinterpret_cast<const uint32_t*>(ve8) + (long long)bh * S;
     int m = 0;  // E_t, reduced by every warp itself
 #pragma unroll
@@ -1119,20 +1124,33 @@ __global__ void __launch_bounds__(256) vprep_kernel(const uint8_t* __restrict__ 
     const uint32_t e4 = __ldg(ve4 + tok);
     uint4* dst = reinterpret_cast<uint4*>(vh + ((long long)bh * S + tok) * D + (lane & 1) * (D / 2));
 #pragma unroll
-    for (int c = 0; c < 2; ++c) {
-      const int de = (int)((e4 >> (8 * ((lane & 1) * 2 + c))) & 0xFFu) - m;  // <= 0
+    for (int c = 0; c < NC; ++c) {
+      const int blk = (lane & 1) * 2 + (F8 ? c / 2 : c);             // 32-element block of the row
+      const int de = (int)((e4 >> (8 * blk)) & 0xFFu) - m;  // <= 0
       const __half fs = de >= -24 ? __float2half_rn(ldexpf(1.0f, de)) : __float2half_rn(0.0f);
       const __half2 f2 = __halves2half2(fs, fs);
       const uint32_t w[4] = {raw[c].x, raw[c].y, raw[c].z, raw[c].w};
-      uint32_t o[16];  // byte i holds elements 2i (low nibble) and 2i + 1
+      if (F8) {  // 16 E4M3 bytes -> 16 fp16
+        uint32_t o[8];
 #pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        const uint32_t v2 = e2m1x2_to_h2((w[i >> 2] >> (8 * (i & 3))) & 0xFFu);
-        const __half2 y = __hmul2(*reinterpret_cast<const __half2*>(&v2), f2);
-        o[i] = *reinterpret_cast<const uint32_t*>(&y);
+        for (int i = 0; i < 8; ++i) {
+          const uint32_t v2 = e4m3x2_to_h2((uint16_t)(w[i >> 1] >> ((i & 1) * 16)));
+          const __half2 y = __hmul2(*reinterpret_cast<const __half2*>(&v2), f2);
+          o[i] = *reinterpret_cast<const uint32_t*>(&y);
+        }
+        dst[2 * c] = make_uint4(o[0], o[1], o[2], o[3]);
+        dst[2 * c + 1] = make_uint4(o[4], o[5], o[6], o[7]);
+      } else {
+        uint32_t o[16];  // byte i holds elements 2i (low nibble) and 2i + 1
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const uint32_t v2 = e2m1x2_to_h2((w[i >> 2] >> (8 * (i & 3))) & 0xFFu);
+          const __half2 y = __hmul2(*reinterpret_cast<const __half2*>(&v2), f2);
+          o[i] = *reinterpret_cast<const uint32_t*>(&y);
+        }
+#pragma unroll
+        for (int q = 0; q < 4; ++q) dst[4 * c + q] = make_uint4(o[4 * q], o[4 * q + 1], o[4 * q + 2], o[4 * q + 3]);
       }
-#pragma unroll
-      for (int q = 0; q < 4; ++q) dst[4 * c + q] = make_uint4(o[4 * q], o[4 * q + 1], o[4 * q + 2], o[4 * q + 3]);
     }
     return;
   }
@@ -1377,11 +1395,13 @@ cudaError_t launch_attention_prefill2(const AttnArgs& a, void* ws, cudaStream_t 
     case FA_MODE_INT8_PER_TOKEN:
       return q->D == 128 ? launch_prefill<K_S8, 128, SC_COL>(a, prm, w, s) : launch_prefill<K_S8, 64, SC_COL>(a, prm, w, s);
     case FA_MODE_MXFP4_PER_BLOCK:
+    case FA_MODE_MXFP8_PER_BLOCK:
       if (q->D != 128) return cudaErrorNotSupported;
       prm.qe8 = static_cast<const uint8_t*>(q->scales);
       prm.ke8 = static_cast<const uint8_t*>(k->scales);
       prm.ve8 = static_cast<const uint8_t*>(a.v->scales);
-      return launch2<K_MXF4, 128, SC_HEAD>(a, prm, w, s);
+      return q->mode == FA_MODE_MXFP4_PER_BLOCK ? launch2<K_MXF4, 128, SC_HEAD>(a, prm, w, s)
+                                                 : launch2<K_MXF8, 128, SC_HEAD>(a, prm, w, s);
     default:
       return cudaErrorNotSupported;
   }

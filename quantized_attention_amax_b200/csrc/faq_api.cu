@@ -59,7 +59,8 @@ bool valid_layout(int l) { return l == FA_LAYOUT_BNSD || l == FA_LAYOUT_BSND; }
 
 bool quantized_mode(int m) {
   return m == FA_MODE_INT8_PER_HEAD || m == FA_MODE_FP8_PER_TOKEN || m == FA_MODE_MXFP4_PER_BLOCK ||
-         m == FA_MODE_FP8_BLOCK || m == FA_MODE_FP8_PER_HEAD || m == FA_MODE_INT8_PER_TOKEN;
+         m == FA_MODE_FP8_BLOCK || m == FA_MODE_FP8_PER_HEAD || m == FA_MODE_INT8_PER_TOKEN ||
+         m == FA_MODE_MXFP8_PER_BLOCK;
 }
 
 fa_status check_tensor(const fa_tensor* t) {
@@ -78,7 +79,7 @@ fa_status check_out(const fa_tensor* t, const fa_qtensor* o, fa_mode mode) {
   if (!o->codes || !o->scales || !aligned16(o->codes) || (reinterpret_cast<uintptr_t>(o->scales) & 3u))
     return FA_ERR_INVALID_ARG;
   if (mode == FA_MODE_FP8_BLOCK && o->block_tokens < 1) return FA_ERR_INVALID_ARG;
-  if (mode == FA_MODE_MXFP4_PER_BLOCK && o->D % 32 != 0) return FA_ERR_INVALID_ARG;
+  if ((mode == FA_MODE_MXFP4_PER_BLOCK || mode == FA_MODE_MXFP8_PER_BLOCK) && o->D % 32 != 0) return FA_ERR_INVALID_ARG;
   return FA_OK;
 }
 
@@ -139,13 +140,13 @@ fa_status fa_resolve_config(const fa_branch_cfg* qconfig, const fa_branch_cfg* d
   const bool has_d = details && (details[0].set || details[1].set || details[2].set);
   if (has_q && has_d) return FA_ERR_CONFIG_CONFLICT;
   if (has_q) {
-    if (qconfig->mode < FA_MODE_FLOAT || qconfig->mode > FA_MODE_INT8_PER_TOKEN) return FA_ERR_INVALID_ARG;
+    if (qconfig->mode < FA_MODE_FLOAT || qconfig->mode > FA_MODE_MXFP8_PER_BLOCK) return FA_ERR_INVALID_ARG;
     modes_out[0] = modes_out[1] = modes_out[2] = qconfig->mode;
     return FA_OK;
   }
   if (has_d) {
     for (int i = 0; i < 3; ++i) {
-      if (details[i].set && (details[i].mode < FA_MODE_FLOAT || details[i].mode > FA_MODE_INT8_PER_TOKEN))
+      if (details[i].set && (details[i].mode < FA_MODE_FLOAT || details[i].mode > FA_MODE_MXFP8_PER_BLOCK))
         return FA_ERR_INVALID_ARG;
       modes_out[i] = details[i].set ? details[i].mode : FA_MODE_FLOAT;
     }
@@ -246,7 +247,7 @@ size_t fa_attention_workspace_size(const fa_qtensor* q, const fa_qtensor* k, int
     if (k->B < 0 || k->S < 0 || (q->D != 64 && q->D != 128)) return 0;
     return prefill2_workspace_bytes(k->B, k->H, k->S, q->D);
   }
-  if (q->mode == FA_MODE_MXFP4_PER_BLOCK) {
+  if (q->mode == FA_MODE_MXFP4_PER_BLOCK || q->mode == FA_MODE_MXFP8_PER_BLOCK) {
     if (k->B < 0 || k->S < 0 || q->D != 128) return 0;
     return prefill2_workspace_bytes(k->B, k->H, k->S, q->D);
   }
@@ -273,7 +274,7 @@ fa_status fa_attention_quant(const fa_qtensor* q, const fa_qtensor* k, const fa_
   if (!out || !aligned16(out)) return FA_ERR_INVALID_ARG;
   if (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)) return FA_ERR_INVALID_ARG;
   const bool decode = is_decode(q, k);
-  if (q->mode == FA_MODE_MXFP4_PER_BLOCK && q->D != 128) return FA_ERR_UNSUPPORTED;
+  if ((q->mode == FA_MODE_MXFP4_PER_BLOCK || q->mode == FA_MODE_MXFP8_PER_BLOCK) && q->D != 128) return FA_ERR_UNSUPPORTED;
   const int splits = decode ? (num_splits > 0 ? num_splits : decode_auto_splits(k->B, k->H, k->S)) : 0;
   if (k->S > 0) {
     const size_t need = decode ? decode_workspace_bytes(q->B, q->H, q->D, splits)

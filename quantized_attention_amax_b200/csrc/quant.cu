@@ -5,6 +5,10 @@
 //       FP8 per token   s = amax_row / 448, code = e4m3(x / s)        (组合2)
 //       MXFP4           per 32 elements: e = floor(log2 amax) - 2,
 //                       code = e2m1(x * 2^-e), E8M0 byte e + 127      (组合3)
+//       FP8 per head    s_h = amax_h / 448 (static, calibrated)       (模式清单: FA PerHead)
+//       INT8 per token  s = amax_row / 127                            (模式清单: FA PerToken)
+//       MXFP8           as MXFP4 with e = floor(log2 amax) - 8 and E4M3 elements
+//                                                                     (模式清单: FA PerBlock)
 //   fp8_block_kernel          one scale = amax / 448 per block of tokens
 //                             (MindIE SD "量化", FA量化 / 块量化)
 // Rows are D contiguous bf16 values in either layout; each row is handled by
@@ -71,12 +75,13 @@ __device__ __forceinline__ int head_of(long long r, int layout, int H, int S) {
   return layout == FA_LAYOUT_BNSD ? (int)((r / S) % H) : (int)(r % H);
 }
 
-// Exponent e of the MX shared scale: floor(log2 amax) - 2, clamped to
-// [-127, 127]; amax == 0 or an fp32-subnormal amax gives -127.
+// Exponent e of the MX shared scale: floor(log2 amax) - EMAX (2 for E2M1, 8 for E4M3 elements),
+// clamped to [-127, 127]; amax == 0 or an fp32-subnormal amax gives -127.
+template <int EMAX>
 __device__ __forceinline__ int mx_exponent(float amax) {
   const int E = (int)((__float_as_uint(amax) >> 23) & 0xFF);
   if (E == 0) return -127;
-  return max(-127, min(127, E - 127 - 2));
+  return max(-127, min(127, E - 127 - EMAX));
 }
 
 template <int MODE, int D>
@@ -176,19 +181,23 @@ __global__ void __launch_bounds__(256) quant_rows_kernel(QuantOperand o0, QuantO
           reinterpret_cast<uint2*>(static_cast<int8_t*>(op.codes) + rr[u] * D)[gl] = out;
           if (gl == 0) static_cast<float*>(op.scales)[scale_index(rr[u], op.layout, op.H, op.S)] = sc;
         }
-      } else {  // MXFP4: one 32-element block = 4 lanes
+      } else {  // MXFP4 / MXFP8: one 32-element block = 4 lanes
         float m = 0.0f;
 #pragma unroll
         for (int i = 0; i < 8; ++i) m = fmaxf(m, fabsf(f[i]));
         m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
         m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 2));
-        const int e = mx_exponent(m);
+        const int e = mx_exponent<MODE == FA_MODE_MXFP8_PER_BLOCK ? 8 : 2>(m);
         const float inv = __uint_as_float((uint32_t)(127 - e) << 23);  // 2^-e, exact
         float v[8];
 #pragma unroll
         for (int i = 0; i < 8; ++i) v[i] = f[i] * inv;
         if (valid) {
-          reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(op.codes) + rr[u] * (D / 2))[gl] = e2m1x8(v);
+          if (MODE == FA_MODE_MXFP8_PER_BLOCK)
+            reinterpret_cast<uint2*>(static_cast<uint8_t*>(op.codes) + rr[u] * D)[gl] =
+                make_uint2(e4m3x4(v[0], v[1], v[2], v[3]), e4m3x4(v[4], v[5], v[6], v[7]));
+          else
+            reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(op.codes) + rr[u] * (D / 2))[gl] = e2m1x8(v);
           if ((gl & 3) == 0)
             static_cast<uint8_t*>(op.scales)[scale_index(rr[u], op.layout, op.H, op.S) * (D / 32) + gl / 4] =
                 (uint8_t)(e + 127);
@@ -340,6 +349,7 @@ cudaError_t launch_quantize_rows(int mode, const QuantOperand* ops, int nops, cu
     case FA_MODE_MXFP4_PER_BLOCK: return launch_rows_mode<FA_MODE_MXFP4_PER_BLOCK>(o, D, s);
     case FA_MODE_FP8_PER_HEAD: return launch_rows_mode<FA_MODE_FP8_PER_HEAD>(o, D, s);
     case FA_MODE_INT8_PER_TOKEN: return launch_rows_mode<FA_MODE_INT8_PER_TOKEN>(o, D, s);
+    case FA_MODE_MXFP8_PER_BLOCK: return launch_rows_mode<FA_MODE_MXFP8_PER_BLOCK>(o, D, s);
     default: return cudaErrorInvalidValue;
   }
 }

@@ -57,6 +57,8 @@ def oracle_quantize(orc, mode, x_bits, layout, blk=0, amax=None):
         c, s = orc.quantize_fp8_per_head(x_bits, amax, layout)
     elif mode == "int8_per_token":
         c, s = orc.quantize_int8_per_token(x_bits, layout)
+    elif mode == "mxfp8":
+        c, s = orc.quantize_mxfp8(x_bits, layout)
     else:
         raise ValueError(mode)
     return orc.QT(mode, c, s, B, H, S, D, layout, blk)

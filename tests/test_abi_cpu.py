@@ -83,7 +83,7 @@ def test_quantize_validation_before_launch(N):
     oh = _q(N, 5)  # FA PerHead FP8 is static too
     assert L.fa_quantize(by(t), None, None, 5, None, None, None, by(oh), None, None, None) == 3
     assert L.fa_quantize(by(t), None, None, 6, None, None, None, by(oh), None, None, None) == 1  # mode mismatch
-    assert L.fa_quantize(by(t), None, None, 7, None, None, None, by(oh), None, None, None) == 2  # unknown mode
+    assert L.fa_quantize(by(t), None, None, 8, None, None, None, by(oh), None, None, None) == 2  # unknown mode
     bad = _q(N, 2, S=9)
     assert L.fa_quantize(by(t), None, None, 2, None, None, None, by(bad), None, None, None) == 1  # shape mismatch
     mis = _t(N, ptr=0x10008)
@@ -148,8 +148,8 @@ def test_attention_validation_before_launch(N):
                                 None) == 7
     assert L.fa_attention_quant(by(qp), by(kd), by(kd), 0, 0.0, 0x60000, None, 0, 0x70010, need_p,
                                 None) == 7  # workspace not 256-byte aligned
-    # the FA PerHead FP8 / PerToken INT8 modes use the same prefill workspace
-    for m in (5, 6):
+    # the FA PerHead FP8 / PerToken INT8 / PerBlock MXFP8 modes use the same prefill workspace
+    for m in (5, 6, 7):
         assert L.fa_attention_workspace_size(by(_q(N, m, B=2, H=4, S=100, D=128)), by(_q(N, m, B=2, H=2, S=1000, D=128)),
                                              0) == need_p
     # MXFP4 prefill: the same parts (its K scales are the tile's scale-factor atom); head_dim 128 only

@@ -28,7 +28,7 @@ def to_bnsd(a, layout):
 def run_case(faq, orc, mode, layout, D, B, Hq, Hkv, Sq, Sk, causal, seed, q_blk=128, kv_blk=256, rows=None,
              dist=None, lse=True):
     if dist is None:
-        dist = "t4" if mode == "mxfp4" else "normal"
+        dist = "t4" if mode in ("mxfp4", "mxfp8") else "normal"
     gen = wl.student_t4 if dist == "t4" else wl.normal
     q = gen(shp(B, Hq, Sq, D, layout), seed)
     k = gen(shp(B, Hkv, Sk, D, layout), seed + 1)
@@ -83,6 +83,10 @@ CASES = [
     ("int8_per_token", "BNSD", 128, 2, 4, 2, 300, 300, True),
     ("int8_per_token", "BSND", 64, 1, 2, 1, 100, 300, True),
     ("int8_per_token", "BNSD", 128, 1, 3, 3, 384, 384, False),
+    # FA PerBlock MXFP8
+    ("mxfp8", "BNSD", 128, 1, 2, 2, 300, 300, False),
+    ("mxfp8", "BSND", 128, 2, 4, 2, 257, 257, True),
+    ("mxfp8", "BNSD", 128, 1, 2, 1, 100, 300, True),
 ]
 
 

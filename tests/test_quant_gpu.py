@@ -100,6 +100,30 @@ def test_int8_per_token_bit_exact(faq, orc, layout, D, S):
         assert np.array_equal(np_of(o.codes), codes)
 
 
+@pytest.mark.parametrize("layout,D,S", CASES)
+def test_mxfp8_bit_exact(faq, orc, layout, D, S):
+    """FA PerBlock with MXFP8: E4M3 elements, shared exponent floor(log2 amax) - 8 per 32."""
+    xs = [rand_bf16(shp(2, 3, S, D, layout), 160 + i, "t4", scale=[1.0, 1e4, 1e-5][i]) for i in range(3)]
+    out = faq.quantize(*[x.cuda() for x in xs], "mxfp8", layout)
+    torch.cuda.synchronize()
+    for x, o in zip(xs, out):
+        codes, e8 = orc.quantize_mxfp8(wl.bf16_bits(x), layout)
+        assert np.array_equal(np_of(o.scales), e8)
+        assert np.array_equal(np_of(o.codes), codes)
+
+
+def test_mxfp8_exhaustive(faq, orc):
+    maxima = [448.0, 256.0, 511.0, 3.0e38, 1e-38, 2.0 ** -130, 0.7, 100.0]
+    blocks = exhaustive_rows(32, maxima, 2)
+    blocks = blocks[: (len(blocks) // 4) * 4]
+    x = blocks.reshape(1, 1, -1, 128)
+    o, = faq.quantize(bf16_from_bits(x), None, None, "mxfp8")[:1]
+    torch.cuda.synchronize()
+    codes, e8 = orc.quantize_mxfp8(x)
+    assert np.array_equal(np_of(o.scales), e8)
+    assert np.array_equal(np_of(o.codes), codes)
+
+
 def test_new_modes_exhaustive(faq, orc):
     """Every finite bf16 value through both new modes (rows of 128)."""
     bits = np.arange(65536, dtype=np.uint32)

@@ -31,7 +31,7 @@ import torch
 @dataclass(frozen=True)
 class Workload:
     name: str
-    mode: str          # int8_per_head | fp8_per_token | fp8_block | mxfp4 | fp8_per_head | int8_per_token
+    mode: str          # int8_per_head | fp8_per_token | fp8_block | mxfp4 | fp8_per_head | int8_per_token | mxfp8
     B: int
     Hq: int
     Hkv: int
@@ -65,6 +65,7 @@ WORKLOADS: Dict[str, Workload] = {
                                  "normal_k_outliers", 6),
     "int8_token_prefill": Workload("int8_token_prefill", "int8_per_token", 2, 32, 8, 4096, 4096, 128, "BNSD", True,
                                    "normal_k_outliers", 7),
+    "mxfp8": Workload("mxfp8", "mxfp8", 1, 24, 24, 4096, 4096, 128, "BNSD", False, "student_t4", 8),
 }
 
 CALIB_SEED_OFFSET = 1000
