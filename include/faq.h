@@ -239,6 +239,40 @@ FAQ_API fa_status fa_attention_decode_noalloc(const fa_qtensor* q, const fa_qten
                                               float softmax_scale, void* out, float* lse, int num_splits,
                                               fa_stream_t s);
 
+/*
+ * fa_decode_append -- one decode step on an INT8 per-head KV cache: the new
+ * token's query is quantized, its key and value are quantized into the cache
+ * at position `pos`, and split-KV attention runs over the cache's first
+ * pos + 1 tokens, all in the decode kernel (then the LSE combine).
+ *   Sources: msModelSlim wiki "FA 量化", 概述 (K/V quantization compresses
+ *   the cache for long-context decode; 组合1 INT8 per-head static scales),
+ *   "量化模式", 模式索引 (decode); the split-KV decode and combine of
+ *   fa_attention_quant.
+ *   q: bf16 [B, Hq, 1, D]; k_new, v_new: bf16 [B, Hkv, 1, D]; D == 128,
+ *   Hq / Hkv in {1, 2, 4, 8, 16}; one layout for every operand.
+ *   amax_q/k/v: device fp32 [Hq] / [Hkv] / [Hkv] calibration maxima
+ *   (s = amax / 127 as in fa_quantize; NULL -> FA_ERR_NO_CALIBRATION).
+ *   k_cache, v_cache: FA_MODE_INT8_PER_HEAD descriptors whose S is the
+ *   cache capacity; codes at positions < pos must already hold the earlier
+ *   tokens (quantized with the same amax); position pos is written by this
+ *   call, and the scale arrays [Hkv] are (re)written with amax / 127.
+ *   0 <= pos < capacity.  out: bf16 [B, Hq, 1, D] in the layout; lse:
+ *   nullable [B, Hq].  workspace: fa_decode_append_workspace_size() bytes,
+ *   256-byte aligned.  num_splits: 0 = automatic (from pos + 1 keys).
+ *   Calls on one cache are ordered by the stream; the cache is read and
+ *   written by this call's kernels only.
+ */
+FAQ_API fa_status fa_decode_append(const fa_tensor* q, const fa_tensor* k_new, const fa_tensor* v_new,
+                                   const float* amax_q, const float* amax_k, const float* amax_v,
+                                   fa_qtensor* k_cache, fa_qtensor* v_cache, int pos, float softmax_scale,
+                                   void* out, float* lse, int num_splits, void* workspace, size_t ws_bytes,
+                                   fa_stream_t s);
+
+/* Workspace bytes fa_decode_append needs (its split-KV partials,
+ * B*Hq*splits*(D+2)*4).  Returns 0 on invalid arguments. */
+FAQ_API size_t fa_decode_append_workspace_size(const fa_tensor* q, const fa_qtensor* k_cache, int pos,
+                                               int num_splits);
+
 /* Workspace bytes fa_attention_quant needs for these operands and split
  * count: decode B*Hq*splits*(D+2)*4; prefill (every mode, the MX modes with
  * D == 128 only) B*Hkv*Sk*D*2 + B*Hkv*ceil(Sk/128)*16 +

@@ -19,6 +19,8 @@ EXPORTS = (
     "fa_attention_quant",
     "fa_attention_workspace_size",
     "fa_attention_decode_noalloc",
+    "fa_decode_append",
+    "fa_decode_append_workspace_size",
     "fa_check_device_status",
     "fa_status_str",
     "fa_version",
@@ -67,6 +69,10 @@ def lib() -> ctypes.CDLL:
     L.fa_attention_decode_noalloc.restype = I
     L.fa_attention_workspace_size.argtypes = [pQ, pQ, I]
     L.fa_attention_workspace_size.restype = S
+    L.fa_decode_append.argtypes = [pT, pT, pT, P, P, P, pQ, pQ, I, F, P, P, I, P, S, P]
+    L.fa_decode_append.restype = I
+    L.fa_decode_append_workspace_size.argtypes = [pT, pQ, I, I]
+    L.fa_decode_append_workspace_size.restype = S
     L.fa_check_device_status.argtypes = [P]
     L.fa_status_str.argtypes = [I]
     L.fa_status_str.restype = ctypes.c_char_p

@@ -212,6 +212,33 @@ def attention(q: QTensor, k: QTensor, v: QTensor, causal: bool = False, softmax_
     return (out, lse) if return_lse else out
 
 
+def decode_append(q: torch.Tensor, k_new: torch.Tensor, v_new: torch.Tensor, amax: Sequence[torch.Tensor],
+                  k_cache: QTensor, v_cache: QTensor, pos: int, softmax_scale: float = 0.0,
+                  out: Optional[torch.Tensor] = None, return_lse: bool = False, num_splits: int = 0,
+                  workspace: Optional[torch.Tensor] = None):
+    """One decode step on an INT8 per-head cache (fa_decode_append): q, k_new, v_new are the new
+    token's bf16 rows ([B, H, 1, D] in the cache's layout); k_new / v_new are quantized into the
+    caches at ``pos``, then attention runs over the first pos + 1 cached tokens.  ``amax`` holds
+    the per-head calibration maxima for q, k, v.  Returns out, or (out, lse)."""
+    layout = k_cache.layout
+    tq, tk, tv = _tensor(q, layout), _tensor(k_new, layout), _tensor(v_new, layout)
+    dev = q.device
+    if out is None:
+        out = torch.empty(_shape(tq.B, tq.H, 1, tq.D, layout), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((tq.B, tq.H, 1), dtype=torch.float32, device=dev) if return_lse else None
+    ck, cv = k_cache.c(), v_cache.c()
+    need = int(N.lib().fa_decode_append_workspace_size(ctypes.byref(tq), ctypes.byref(ck), int(pos), num_splits))
+    if workspace is None or workspace.numel() * workspace.element_size() < need:
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=dev)
+    _check(N.lib().fa_decode_append(ctypes.byref(tq), ctypes.byref(tk), ctypes.byref(tv), amax[0].data_ptr(),
+                                    amax[1].data_ptr(), amax[2].data_ptr(), ctypes.byref(ck), ctypes.byref(cv),
+                                    int(pos), float(softmax_scale), out.data_ptr(),
+                                    lse.data_ptr() if lse is not None else None, int(num_splits),
+                                    workspace.data_ptr(), workspace.numel() * workspace.element_size(), _stream()),
+           "fa_decode_append")
+    return (out, lse) if return_lse else out
+
+
 def check_device_status():
     """Synchronise the current stream and raise if a kernel's bounded wait ran out."""
     _check(N.lib().fa_check_device_status(_stream()), "fa_check_device_status")

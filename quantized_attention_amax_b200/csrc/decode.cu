@@ -40,6 +40,20 @@ struct DecParams {
   float* opart;  // [B*Hq][splits][D]
   float* ml;     // [B*Hq][splits][2]  (m in log2 units, L)
   int* status;
+  // Fused cache append: Q quantized from bf16 in every CTA, and the new token's K / V rows quantized
+  // into the cache at position pos by the CTA whose chunk holds it (before its TMA reads).
+  int append;
+  const __nv_bfloat16* qf;    // [B, Hq, D] bf16 (S = 1 in either layout)
+  const __nv_bfloat16* knew;  // [B, Hkv, D] bf16
+  const __nv_bfloat16* vnew;
+  const float* amax_q;        // per-head calibration maxima: s = amax / 127
+  const float* amax_k;
+  const float* amax_v;
+  int8_t* kc;                 // cache codes, capacity cap tokens
+  int8_t* vc;
+  float* ks_out;              // cache scales [Hkv]
+  float* vs_out;
+  int cap, pos;
 };
 
 template <int D>
@@ -76,6 +90,18 @@ __device__ __forceinline__ float ex2f(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+// x / s rounded as IEEE division, then round-half-to-even to an integer, saturated to int8.
+__device__ __forceinline__ uint32_t s8_code(float x, float s) {
+  if (!(s > 0.0f)) return 0u;
+  const int i = max(-128, min(127, __float2int_rn(__fdiv_rn(x, s))));
+  return (uint32_t)(i & 0xFF);
+}
+__device__ __forceinline__ uint32_t s8_codes4(uint2 bf4, float s) {
+  const float x0 = __uint_as_float(bf4.x << 16), x1 = __uint_as_float(bf4.x & 0xFFFF0000u);
+  const float x2 = __uint_as_float(bf4.y << 16), x3 = __uint_as_float(bf4.y & 0xFFFF0000u);
+  return s8_code(x0, s) | (s8_code(x1, s) << 8) | (s8_code(x2, s) << 16) | (s8_code(x3, s) << 24);
 }
 
 __device__ __forceinline__ bool wwait(uint64_t* b, uint32_t parity, volatile int* abort_flag, int* status, int where) {
@@ -134,6 +160,23 @@ __global__ void __launch_bounds__(DTHREADS, 2)
   const uint32_t tOT[2] = {tbase + 32, tbase + 48};
 
   if (warp == 0) {
+    if (p.append && key0 <= p.pos && p.pos < key1) {
+      // the new token's K / V rows into the cache (lane l: elements 4l .. 4l + 3), visible to the
+      // TMA reads below through the async-proxy fence
+      static_assert(D == 128, "decode: head_dim 128");
+      const float sk = __fdiv_rn(__ldg(p.amax_k + hk), 127.0f), sv = __fdiv_rn(__ldg(p.amax_v + hk), 127.0f);
+      const long long src = ((long long)b * p.Hkv + hk) * D;
+      const long long dst = p.layout == FA_LAYOUT_BNSD ? (((long long)b * p.Hkv + hk) * p.cap + p.pos) * D
+                                                       : (((long long)b * p.cap + p.pos) * p.Hkv + hk) * D;
+      reinterpret_cast<uint32_t*>(p.kc + dst)[lane] = s8_codes4(__ldg(reinterpret_cast<const uint2*>(p.knew + src) + lane), sk);
+      reinterpret_cast<uint32_t*>(p.vc + dst)[lane] = s8_codes4(__ldg(reinterpret_cast<const uint2*>(p.vnew + src) + lane), sv);
+      asm volatile("fence.proxy.async.global;" ::: "memory");
+    }
+    if (p.append && split == 0 && b == 0 && lane == 0) {
+      p.ks_out[hk] = __fdiv_rn(__ldg(p.amax_k + hk), 127.0f);
+      p.vs_out[hk] = __fdiv_rn(__ldg(p.amax_v + hk), 127.0f);
+    }
+    __syncwarp();
     if (lane == 0 && n_tiles > 0) {
       tma_prefetch_desc(&tmk);
       tma_prefetch_desc(&tmv);
@@ -212,9 +255,16 @@ __global__ void __launch_bounds__(DTHREADS, 2)
       if (c < D / 16) {
         uint4 v = make_uint4(0, 0, 0, 0);
         if (r < G) {
-          const long long qrow = p.layout == FA_LAYOUT_BNSD ? ((long long)b * p.Hq + hq0 + r)
-                                                            : ((long long)b * p.Hq + hq0 + r);
-          v = __ldg(reinterpret_cast<const uint4*>(p.q + qrow * D) + c);
+          const long long qrow = (long long)b * p.Hq + hq0 + r;  // S = 1: the same row in either layout
+          if (p.append) {
+            // quantize the new query row here: 16 codes from 16 bf16 values
+            const float sq = __fdiv_rn(__ldg(p.amax_q + hq0 + r), 127.0f);
+            const uint2* src = reinterpret_cast<const uint2*>(p.qf + qrow * D + c * 16);
+            v = make_uint4(s8_codes4(__ldg(src), sq), s8_codes4(__ldg(src + 1), sq), s8_codes4(__ldg(src + 2), sq),
+                           s8_codes4(__ldg(src + 3), sq));
+          } else {
+            v = __ldg(reinterpret_cast<const uint4*>(p.q + qrow * D) + c);
+          }
         }
         const uint32_t off = D == 128 ? swz128_offset(r, c) : swz64_offset(r, c);
         *reinterpret_cast<uint4*>(smem + L::Q + off) = v;
@@ -232,10 +282,11 @@ __global__ void __launch_bounds__(DTHREADS, 2)
     }
 
     float ch[G], m_run[G], alpha_prev[G], Lp[G], Oacc[G];
-    const float skv = __ldg(p.ks + hk);
+    const float skv = p.append ? __fdiv_rn(__ldg(p.amax_k + hk), 127.0f) : __ldg(p.ks + hk);
 #pragma unroll
     for (int h = 0; h < G; ++h) {
-      ch[h] = __ldg(p.qs + hq0 + h) * skv * p.scale_log2;
+      const float sqh = p.append ? __fdiv_rn(__ldg(p.amax_q + hq0 + h), 127.0f) : __ldg(p.qs + hq0 + h);
+      ch[h] = sqh * skv * p.scale_log2;
       m_run[h] = -INFINITY;
       alpha_prev[h] = 1.0f;
       Lp[h] = 0.0f;
@@ -382,18 +433,19 @@ __global__ void attn_combine_kernel(const float* __restrict__ opart, const float
   if (lse && lane == 0) lse[w] = Lsum > 0.0f ? (m + __log2f(Lsum / 255.0f)) * 0.69314718055994530942f : -INFINITY;
 }
 
-cudaError_t make_map(CUtensorMap* map, const void* base, int B, int H, int S, int D, int layout) {
+// Tensor map over int8 codes of S visible tokens stored in a buffer of cap >= S tokens.
+cudaError_t make_map(CUtensorMap* map, const void* base, int B, int H, int S, int D, int layout, int cap) {
   EncodeTiledFn enc = encode_tiled_fn();
   if (!enc) return cudaErrorNotSupported;
   cuuint64_t dims[4], strides[3];
   cuuint32_t box[4], es[4] = {1, 1, 1, 1};
   if (layout == FA_LAYOUT_BNSD) {
     dims[0] = D; dims[1] = S; dims[2] = H; dims[3] = B;
-    strides[0] = (cuuint64_t)D; strides[1] = (cuuint64_t)S * D; strides[2] = (cuuint64_t)H * S * D;
+    strides[0] = (cuuint64_t)D; strides[1] = (cuuint64_t)cap * D; strides[2] = (cuuint64_t)H * cap * D;
     box[0] = D; box[1] = DBN; box[2] = 1; box[3] = 1;
   } else {
     dims[0] = D; dims[1] = H; dims[2] = S; dims[3] = B;
-    strides[0] = (cuuint64_t)D; strides[1] = (cuuint64_t)H * D; strides[2] = (cuuint64_t)S * H * D;
+    strides[0] = (cuuint64_t)D; strides[1] = (cuuint64_t)H * D; strides[2] = (cuuint64_t)cap * H * D;
     box[0] = D; box[1] = 1; box[2] = DBN; box[3] = 1;
   }
   CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 4, const_cast<void*>(base), dims, strides, box, es,
@@ -448,28 +500,20 @@ size_t decode_workspace_bytes(int B, int Hq, int D, int splits) {
   return (size_t)B * Hq * splits * ((size_t)D + 2) * sizeof(float);
 }
 
-cudaError_t launch_attention_decode(const AttnArgs& a, int splits, void* ws, cudaStream_t s) {
-  const fa_qtensor* q = a.q;
-  const fa_qtensor* k = a.k;
-  const int G = q->H / k->H;
-  DecParams prm = {};
-  prm.B = q->B; prm.Hq = q->H; prm.Hkv = k->H; prm.Sk = k->S; prm.group = G; prm.layout = q->layout;
-  prm.splits = splits;
-  prm.chunk = chunk_of(k->S, splits);
-  const float scale = a.softmax_scale > 0.0f ? a.softmax_scale : 1.0f / sqrtf((float)q->D);
-  prm.scale_log2 = scale * 1.4426950408889634f;
-  prm.q = static_cast<const int8_t*>(q->codes);
-  prm.qs = static_cast<const float*>(q->scales);
-  prm.ks = static_cast<const float*>(k->scales);
-  prm.vs = static_cast<const float*>(a.v->scales);
-  prm.opart = static_cast<float*>(ws);
-  prm.ml = prm.opart + (size_t)q->B * q->H * splits * q->D;
-  prm.status = a.status;
+namespace {
+
+// Decode kernel (one CTA per split and (b, kv head)) then the combine; kv_len visible tokens in
+// K / V buffers of cap tokens.
+cudaError_t run_decode(DecParams prm, const void* kcodes, const void* vcodes, int D, int kv_len, int cap, int out_layout,
+                       void* out, float* lse, cudaStream_t s) {
+  const int G = prm.group;
+  prm.Sk = kv_len;
+  prm.chunk = chunk_of(kv_len, prm.splits);
   CUtensorMap mk, mv;
   cudaError_t e;
-  if ((e = make_map(&mk, k->codes, k->B, k->H, k->S, k->D, k->layout)) != cudaSuccess) return e;
-  if ((e = make_map(&mv, a.v->codes, a.v->B, a.v->H, a.v->S, a.v->D, a.v->layout)) != cudaSuccess) return e;
-  if (q->D == 128) {
+  if ((e = make_map(&mk, kcodes, prm.B, prm.Hkv, kv_len, D, prm.layout, cap)) != cudaSuccess) return e;
+  if ((e = make_map(&mv, vcodes, prm.B, prm.Hkv, kv_len, D, prm.layout, cap)) != cudaSuccess) return e;
+  if (D == 128) {
     switch (G) {
       case 1: e = launch_dec<128, 1>(mk, mv, prm, s); break;
       case 2: e = launch_dec<128, 2>(mk, mv, prm, s); break;
@@ -482,10 +526,55 @@ cudaError_t launch_attention_decode(const AttnArgs& a, int splits, void* ws, cud
     return cudaErrorNotSupported;
   }
   if (e != cudaSuccess) return e;
-  const int BH = q->B * q->H;
-  attn_combine_kernel<<<(BH * 32 + 255) / 256, 256, 0, s>>>(prm.opart, prm.ml, BH, q->H, k->H, splits, q->D, prm.vs,
-                                                            static_cast<__nv_bfloat16*>(a.out), a.lse, q->layout);
+  const int BH = prm.B * prm.Hq;
+  attn_combine_kernel<<<(BH * 32 + 255) / 256, 256, 0, s>>>(prm.opart, prm.ml, BH, prm.Hq, prm.Hkv, prm.splits, D,
+                                                            prm.vs, static_cast<__nv_bfloat16*>(out), lse, out_layout);
   return cudaGetLastError();
+}
+
+DecParams base_params(int B, int Hq, int Hkv, int D, int layout, int splits, float softmax_scale, void* ws,
+                      int* status) {
+  DecParams prm = {};
+  prm.B = B; prm.Hq = Hq; prm.Hkv = Hkv; prm.group = Hq / Hkv; prm.layout = layout;
+  prm.splits = splits;
+  const float scale = softmax_scale > 0.0f ? softmax_scale : 1.0f / sqrtf((float)D);
+  prm.scale_log2 = scale * 1.4426950408889634f;
+  prm.opart = static_cast<float*>(ws);
+  prm.ml = prm.opart + (size_t)B * Hq * splits * D;
+  prm.status = status;
+  return prm;
+}
+
+}  // namespace
+
+cudaError_t launch_attention_decode(const AttnArgs& a, int splits, void* ws, cudaStream_t s) {
+  const fa_qtensor* q = a.q;
+  const fa_qtensor* k = a.k;
+  DecParams prm = base_params(q->B, q->H, k->H, q->D, q->layout, splits, a.softmax_scale, ws, a.status);
+  prm.q = static_cast<const int8_t*>(q->codes);
+  prm.qs = static_cast<const float*>(q->scales);
+  prm.ks = static_cast<const float*>(k->scales);
+  prm.vs = static_cast<const float*>(a.v->scales);
+  return run_decode(prm, k->codes, a.v->codes, q->D, k->S, k->S, q->layout, a.out, a.lse, s);
+}
+
+cudaError_t launch_decode_append(const DecodeAppendArgs& a, int splits, void* ws, cudaStream_t s) {
+  DecParams prm = base_params(a.q->B, a.q->H, a.k_cache->H, a.q->D, a.q->layout, splits, a.softmax_scale, ws,
+                              a.status);
+  prm.append = 1;
+  prm.qf = static_cast<const __nv_bfloat16*>(a.q->data);
+  prm.knew = static_cast<const __nv_bfloat16*>(a.k_new->data);
+  prm.vnew = static_cast<const __nv_bfloat16*>(a.v_new->data);
+  prm.amax_q = a.amax_q; prm.amax_k = a.amax_k; prm.amax_v = a.amax_v;
+  prm.kc = static_cast<int8_t*>(a.k_cache->codes);
+  prm.vc = static_cast<int8_t*>(a.v_cache->codes);
+  prm.ks_out = static_cast<float*>(a.k_cache->scales);
+  prm.vs_out = static_cast<float*>(a.v_cache->scales);
+  prm.vs = prm.vs_out;  // the combine reads the V scales the decode kernel has written
+  prm.cap = a.k_cache->S;
+  prm.pos = a.pos;
+  return run_decode(prm, a.k_cache->codes, a.v_cache->codes, a.q->D, a.pos + 1, a.k_cache->S, a.q->layout, a.out,
+                    a.lse, s);
 }
 
 }  // namespace faq

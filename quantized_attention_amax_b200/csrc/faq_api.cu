@@ -295,6 +295,59 @@ fa_status fa_attention_quant(const fa_qtensor* q, const fa_qtensor* k, const fa_
   return from_cuda(e);
 }
 
+// Shared checks of fa_decode_append's operands; returns the split count through *splits.
+static fa_status check_decode_append(const fa_tensor* q, const fa_tensor* k_new, const fa_tensor* v_new,
+                                     const fa_qtensor* kc, const fa_qtensor* vc, int pos, int num_splits,
+                                     int* splits) {
+  if (!q || !k_new || !v_new || !kc || !vc) return FA_ERR_INVALID_ARG;
+  if (kc->mode != FA_MODE_INT8_PER_HEAD || vc->mode != FA_MODE_INT8_PER_HEAD) return FA_ERR_UNSUPPORTED;
+  if (q->D != 128 || k_new->D != 128 || v_new->D != 128 || kc->D != 128 || vc->D != 128) return FA_ERR_UNSUPPORTED;
+  if (!valid_layout(q->layout) || q->layout != k_new->layout || q->layout != v_new->layout ||
+      q->layout != kc->layout || q->layout != vc->layout)
+    return FA_ERR_INVALID_ARG;
+  if (q->S != 1 || k_new->S != 1 || v_new->S != 1) return FA_ERR_INVALID_ARG;
+  if (q->B < 1 || kc->H < 1 || q->H % kc->H != 0) return FA_ERR_INVALID_ARG;
+  if (k_new->B != q->B || v_new->B != q->B || kc->B != q->B || vc->B != q->B) return FA_ERR_INVALID_ARG;
+  if (k_new->H != kc->H || v_new->H != kc->H || vc->H != kc->H || vc->S != kc->S) return FA_ERR_INVALID_ARG;
+  const int group = q->H / kc->H;
+  if (!(group == 1 || group == 2 || group == 4 || group == 8 || group == 16)) return FA_ERR_UNSUPPORTED;
+  if (pos < 0 || pos >= kc->S || num_splits < 0) return FA_ERR_INVALID_ARG;
+  if (!q->data || !k_new->data || !v_new->data || !aligned16(q->data) || !aligned16(k_new->data) ||
+      !aligned16(v_new->data))
+    return FA_ERR_INVALID_ARG;
+  if (!kc->codes || !vc->codes || !kc->scales || !vc->scales || !aligned16(kc->codes) || !aligned16(vc->codes) ||
+      (reinterpret_cast<uintptr_t>(kc->scales) & 3u) || (reinterpret_cast<uintptr_t>(vc->scales) & 3u))
+    return FA_ERR_INVALID_ARG;
+  *splits = num_splits > 0 ? num_splits : decode_auto_splits(q->B, kc->H, pos + 1);
+  return FA_OK;
+}
+
+size_t fa_decode_append_workspace_size(const fa_tensor* q, const fa_qtensor* k_cache, int pos, int num_splits) {
+  if (!q || !k_cache || k_cache->H < 1 || q->H % k_cache->H || pos < 0 || num_splits < 0) return 0;
+  const int splits = num_splits > 0 ? num_splits : decode_auto_splits(q->B, k_cache->H, pos + 1);
+  return decode_workspace_bytes(q->B, q->H, q->D, splits);
+}
+
+fa_status fa_decode_append(const fa_tensor* q, const fa_tensor* k_new, const fa_tensor* v_new, const float* amax_q,
+                           const float* amax_k, const float* amax_v, fa_qtensor* k_cache, fa_qtensor* v_cache,
+                           int pos, float softmax_scale, void* out, float* lse, int num_splits, void* workspace,
+                           size_t ws_bytes, fa_stream_t s) {
+  int splits = 0;
+  fa_status st = check_decode_append(q, k_new, v_new, k_cache, v_cache, pos, num_splits, &splits);
+  if (st != FA_OK) return st;
+  if (!amax_q || !amax_k || !amax_v) return FA_ERR_NO_CALIBRATION;
+  if (!out || !aligned16(out)) return FA_ERR_INVALID_ARG;
+  if (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)) return FA_ERR_INVALID_ARG;
+  const size_t need = decode_workspace_bytes(q->B, q->H, q->D, splits);
+  if (!workspace || ws_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255u)) return FA_ERR_WORKSPACE;
+  int* status = device_status_ptr();
+  if (!status) return FA_ERR_CUDA;
+  DecodeAppendArgs a = {q, k_new, v_new, amax_q, amax_k, amax_v, k_cache, v_cache, pos, softmax_scale, out, lse, status};
+  const cudaError_t e = launch_decode_append(a, splits, workspace, reinterpret_cast<cudaStream_t>(s));
+  if (e == cudaErrorNotSupported) return FA_ERR_UNSUPPORTED;
+  return from_cuda(e);
+}
+
 fa_status fa_check_device_status(fa_stream_t s) {
   cudaStream_t cs = reinterpret_cast<cudaStream_t>(s);
   if (cudaStreamSynchronize(cs) != cudaSuccess) return FA_ERR_CUDA;

@@ -68,6 +68,24 @@ size_t decode_workspace_bytes(int B, int Hq, int D, int splits);
 int decode_auto_splits(int B, int Hkv, int Sk);
 cudaError_t launch_attention_decode(const AttnArgs& a, int splits, void* ws, cudaStream_t s);
 
+// Decode with the new token appended to an INT8 per-head cache in the same kernel.
+struct DecodeAppendArgs {
+  const fa_tensor* q;      // bf16 [B, Hq, 1, D]
+  const fa_tensor* k_new;  // bf16 [B, Hkv, 1, D]
+  const fa_tensor* v_new;
+  const float* amax_q;
+  const float* amax_k;
+  const float* amax_v;
+  const fa_qtensor* k_cache;  // S = capacity
+  const fa_qtensor* v_cache;
+  int pos;
+  float softmax_scale;
+  void* out;
+  float* lse;
+  int* status;
+};
+cudaError_t launch_decode_append(const DecodeAppendArgs& a, int splits, void* ws, cudaStream_t s);
+
 cudaError_t launch_fill_empty_rows(void* out, float* lse, long long rows, int D, cudaStream_t s);
 
 }  // namespace faq
