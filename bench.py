@@ -516,6 +516,48 @@ def reference_arm(args, w):
 
 # ------------------------------------------------------------------ main ---
 
+def decode_append_run(w, device, steps):
+    """fa_decode_append on the decode workload's cache: each step quantizes the query, appends the
+    last token's K / V into the cache and attends over all Sk tokens (one call, two launches)."""
+    import torch
+    import quantized_attention_amax_b200 as faq
+    import workloads as wl
+    inp = wl.make_inputs(w, device=device, calib=True)
+    am = [faq.calibrate_per_head(inp[n + "_cal"], w.layout) for n in "qkv"]
+    _, Kc, Vc = faq.quantize(None, inp["k"], inp["v"], w.mode, w.layout, amax=[None, am[1], am[2]])
+    pos = w.Sk - 1
+    k_new = inp["k"][:, :, pos:pos + 1].contiguous()
+    v_new = inp["v"][:, :, pos:pos + 1].contiguous()
+    out = faq.decode_append(inp["q"], k_new, v_new, am, Kc, Vc, pos)
+    ws = torch.empty(1 << 24, dtype=torch.uint8, device=device)
+    fn = lambda: faq.decode_append(inp["q"], k_new, v_new, am, Kc, Vc, pos, out=out, workspace=ws)
+    for _ in range(3):
+        fn()
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        fn()
+    torch.cuda.current_stream().wait_stream(s)
+    with torch.cuda.graph(g):
+        fn()
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
+    stream = torch.cuda.current_stream()
+    ms = []
+    for i in range(steps + 3):
+        flush.zero_()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        g.replay()
+        b.record(stream)
+        b.synchronize()
+        if i >= 3:
+            ms.append(a.elapsed_time(b))
+    faq.check_device_status()
+    return sum(ms) / len(ms)
+
+
 def supplemental(args, device):
     """Every other workload, briefly (graph replays, L2 flushed): kernel-level
     numbers against their rooflines.  Context for the headline line."""
@@ -545,6 +587,15 @@ def supplemental(args, device):
                               "frac_of_peak": fl / (r["attn_ms"] * 1e-3) / 1e12 / tp, "peak": tp, "flops": fl}
         out[name] = d
         del r
+    w = wl.WORKLOADS["int8_decode"]
+    ams = decode_append_run(w, device, 10)
+    db = decode_bytes(w)
+    out["int8_decode_append"] = {
+        "ms_per_step": ams, "unit": "GB/s (KV codes)", "value": db / (ams * 1e-3) / 1e9,
+        "attention": {"GB/s": db / (ams * 1e-3) / 1e9, "frac_of_hbm": db / (ams * 1e-3) / 1e9 / pk["hbm_gbs"],
+                      "bytes": db},
+        "note": "fa_decode_append: query quantize + K/V append at position Sk-1 + split-KV decode + combine, "
+                "two launches per step"}
     return out
 
 
