@@ -12,7 +12,7 @@
 //   fp8_block_kernel          one scale = amax / 448 per block of tokens
 //                             (MindIE SD "量化", FA量化 / 块量化)
 // Rows are D contiguous bf16 values in either layout; each row is handled by
-// D/8 lanes with one 16-byte load each.  x / s is rounded as IEEE division
+// D/32 lanes with four 16-byte loads each.  x / s is rounded as IEEE division
 // (div.rn.f32) rounds it, so the codes match a correctly rounded x / s exactly:
 // FP8 scales use the FMA-corrected reciprocal product of quant_common.cuh,
 // INT8 (whose static scale can be exceeded) uses IEEE division itself.
@@ -24,6 +24,13 @@
 
 namespace faq {
 namespace {
+
+// max(a, b, c) in one instruction (sm_100 three-input form).
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
 
 __device__ __forceinline__ void unpack_bf16x8(const uint4& u, float (&f)[8]) {
   const uint32_t w[4] = {u.x, u.y, u.z, u.w};
@@ -84,18 +91,22 @@ __device__ __forceinline__ int mx_exponent(float amax) {
   return max(-127, min(127, E - 127 - EMAX));
 }
 
+// One row = D / 32 lanes; each lane owns 32 consecutive elements (one MX block): four 16-byte
+// loads, so the per-row work (the scale, its reciprocal, the lane shuffles, the addresses) is
+// shared by 32 elements per lane.
 template <int MODE, int D>
 __global__ void __launch_bounds__(256) quant_rows_kernel(QuantOperand o0, QuantOperand o1, QuantOperand o2) {
-  constexpr int G = D / 8;     // lanes per row
-  constexpr int RPW = 32 / G;  // rows per warp per step
-  constexpr int UNROLL = 2;
+  constexpr int LPR = D / 32;  // lanes per row
+  constexpr int RPW = 32 / LPR;  // rows per warp
   const int lane = threadIdx.x & 31;
-  const int gl = lane % G;
-  const int sub = lane / G;
+  const int gl = lane % LPR;   // 32-element chunk of the row
+  const int sub = lane / LPR;
 
   // per-head static modes: one scale per head from the calibration maxima
   constexpr bool PER_HEAD = MODE == FA_MODE_INT8_PER_HEAD || MODE == FA_MODE_FP8_PER_HEAD;
-  constexpr float QMAX = (MODE == FA_MODE_INT8_PER_HEAD || MODE == FA_MODE_INT8_PER_TOKEN) ? 127.0f : 448.0f;
+  constexpr bool INT8 = MODE == FA_MODE_INT8_PER_HEAD || MODE == FA_MODE_INT8_PER_TOKEN;
+  constexpr bool MX = MODE == FA_MODE_MXFP4_PER_BLOCK || MODE == FA_MODE_MXFP8_PER_BLOCK;
+  constexpr float QMAX = INT8 ? 127.0f : 448.0f;
   if (PER_HEAD && blockIdx.x == 0) {
     for (int t = threadIdx.x; t < o0.H && o0.rows > 0; t += blockDim.x)
       static_cast<float*>(o0.scales)[t] = __fdiv_rn(o0.amax[t], QMAX);
@@ -105,103 +116,110 @@ __global__ void __launch_bounds__(256) quant_rows_kernel(QuantOperand o0, QuantO
       static_cast<float*>(o2.scales)[t] = __fdiv_rn(o2.amax[t], QMAX);
   }
 
-  const long long total = o0.rows + o1.rows + o2.rows;
+  const long long rows0 = o0.rows, rows01 = o0.rows + o1.rows;
+  const long long total = rows01 + o2.rows;
   const long long nwarps = (long long)gridDim.x * (blockDim.x / 32);
   const long long wid = ((long long)blockIdx.x * blockDim.x + threadIdx.x) / 32;
-  const long long step = nwarps * RPW;
 
-  for (long long base = wid * RPW * UNROLL; base < total; base += step * UNROLL) {
-    uint4 raw[UNROLL];
-    long long rr[UNROLL];
-    int which[UNROLL];
+  for (long long r = wid * RPW + sub; r - sub < total; r += nwarps * RPW) {
+    const bool valid = r < total;  // the same for every lane of the row
+    const int which = r < rows0 ? 0 : (r < rows01 ? 1 : 2);
+    const long long rr = which == 0 ? r : (which == 1 ? r - rows0 : r - rows01);
+    // the row's operand, field by field (no address of a kernel parameter is taken)
+    const void* const op_x = which == 0 ? o0.x : (which == 1 ? o1.x : o2.x);
+    void* const op_codes = which == 0 ? o0.codes : (which == 1 ? o1.codes : o2.codes);
+    void* const op_scales = which == 0 ? o0.scales : (which == 1 ? o1.scales : o2.scales);
+    uint4 raw[4];
+    const uint4* src = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(op_x) + rr * D) + gl * 4;
 #pragma unroll
-    for (int u = 0; u < UNROLL; ++u) {
-      const long long r = base + u * RPW + sub;
-      which[u] = r < o0.rows ? 0 : (r < o0.rows + o1.rows ? 1 : 2);
-      rr[u] = which[u] == 0 ? r : (which[u] == 1 ? r - o0.rows : r - o0.rows - o1.rows);
-      raw[u] = make_uint4(0, 0, 0, 0);
-      if (r < total) {
-        const void* x = which[u] == 0 ? o0.x : (which[u] == 1 ? o1.x : o2.x);
-        raw[u] = __ldg(reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(x) + rr[u] * D) + gl);
+    for (int c = 0; c < 4; ++c) raw[c] = valid ? __ldg(src + c) : make_uint4(0, 0, 0, 0);
+    float f[32];
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      float t8[8];
+      unpack_bf16x8(raw[c], t8);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) f[8 * c + i] = t8[i];
+    }
+    float m = 0.0f;
+    if (!PER_HEAD) {
+#pragma unroll
+      for (int i = 0; i < 32; i += 2) m = fmax3(m, fabsf(f[i]), fabsf(f[i + 1]));
+      if (!MX) {
+#pragma unroll
+        for (int off = LPR / 2; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
       }
     }
+    uint4 out[2];
+    if (MX) {
+      // one 32-element block per lane: e = floor(log2 amax) - emax, x * 2^-e exact
+      const int e = mx_exponent<MODE == FA_MODE_MXFP8_PER_BLOCK ? 8 : 2>(m);
+      const float inv = __uint_as_float((uint32_t)(127 - e) << 23);
+      if (valid) {
+        if (MODE == FA_MODE_MXFP8_PER_BLOCK) {
+          uint32_t w[8];
 #pragma unroll
-    for (int u = 0; u < UNROLL; ++u) {
-      const long long r = base + u * RPW + sub;
-      const bool valid = r < total;
-      const QuantOperand& op = which[u] == 0 ? o0 : (which[u] == 1 ? o1 : o2);
-      float f[8];
-      unpack_bf16x8(raw[u], f);
-      if (MODE == FA_MODE_FP8_PER_TOKEN) {
-        float m = 0.0f;
-#pragma unroll
-        for (int i = 0; i < 8; ++i) m = fmaxf(m, fabsf(f[i]));
-#pragma unroll
-        for (int off = G / 2; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
-        const float sc = __fdiv_rn(m, 448.0f);
-        float v[8];
-        if (sc >= kFastDivMin) {
-          const float r = __frcp_rn(sc);
-#pragma unroll
-          for (int i = 0; i < 8; ++i) v[i] = fp8_div(f[i], sc, r);
+          for (int i = 0; i < 8; ++i)
+            w[i] = e4m3x4(f[4 * i] * inv, f[4 * i + 1] * inv, f[4 * i + 2] * inv, f[4 * i + 3] * inv);
+          uint4* dst = reinterpret_cast<uint4*>(static_cast<uint8_t*>(op_codes) + rr * D + gl * 32);
+          dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
+          dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
         } else {
+          uint32_t w[4];
 #pragma unroll
-          for (int i = 0; i < 8; ++i) v[i] = sc > 0.0f ? __fdiv_rn(f[i], sc) : 0.0f;
+          for (int i = 0; i < 4; ++i) {
+            float v8[8];
+#pragma unroll
+            for (int k = 0; k < 8; ++k) v8[k] = f[8 * i + k] * inv;
+            w[i] = e2m1x8(v8);
+          }
+          *reinterpret_cast<uint4*>(static_cast<uint8_t*>(op_codes) + rr * (D / 2) + gl * 16) =
+              make_uint4(w[0], w[1], w[2], w[3]);
         }
-        if (valid) {
-          uint2 out = make_uint2(e4m3x4(v[0], v[1], v[2], v[3]), e4m3x4(v[4], v[5], v[6], v[7]));
-          reinterpret_cast<uint2*>(static_cast<uint8_t*>(op.codes) + rr[u] * D)[gl] = out;
-          if (gl == 0) static_cast<float*>(op.scales)[scale_index(rr[u], op.layout, op.H, op.S)] = sc;
-        }
-      } else if (PER_HEAD) {
-        // static scale: x can exceed the calibrated range, so IEEE division (codes saturate)
-        float sc = 0.0f;
-        if (valid) sc = __fdiv_rn(__ldg(op.amax + head_of(rr[u], op.layout, op.H, op.S)), QMAX);
-        float v[8];
+        const int op_layout = which == 0 ? o0.layout : (which == 1 ? o1.layout : o2.layout);
+        const int op_H = which == 0 ? o0.H : (which == 1 ? o1.H : o2.H);
+        const int op_S = which == 0 ? o0.S : (which == 1 ? o1.S : o2.S);
+        static_cast<uint8_t*>(op_scales)[scale_index(rr, op_layout, op_H, op_S) * (D / 32) + gl] = (uint8_t)(e + 127);
+      }
+      continue;
+    }
+    // one scale per row (dynamic modes) or per head (static modes)
+    float sc;
+    if (PER_HEAD) {
+      const int op_layout = which == 0 ? o0.layout : (which == 1 ? o1.layout : o2.layout);
+      const int op_H = which == 0 ? o0.H : (which == 1 ? o1.H : o2.H);
+      const int op_S = which == 0 ? o0.S : (which == 1 ? o1.S : o2.S);
+      const float* op_amax = which == 0 ? o0.amax : (which == 1 ? o1.amax : o2.amax);
+      sc = valid ? __fdiv_rn(__ldg(op_amax + head_of(rr, op_layout, op_H, op_S)), QMAX) : 0.0f;
+    } else {
+      sc = __fdiv_rn(m, QMAX);
+    }
+    float v[32];
+    if (MODE == FA_MODE_FP8_PER_TOKEN && sc >= kFastDivMin) {
+      const float rc = __frcp_rn(sc);
 #pragma unroll
-        for (int i = 0; i < 8; ++i) v[i] = sc > 0.0f ? __fdiv_rn(f[i], sc) : 0.0f;
-        if (valid) {
-          const uint2 out = MODE == FA_MODE_INT8_PER_HEAD
-                                ? make_uint2(s8x4(v[0], v[1], v[2], v[3]), s8x4(v[4], v[5], v[6], v[7]))
-                                : make_uint2(e4m3x4(v[0], v[1], v[2], v[3]), e4m3x4(v[4], v[5], v[6], v[7]));
-          reinterpret_cast<uint2*>(static_cast<uint8_t*>(op.codes) + rr[u] * D)[gl] = out;
-        }
-      } else if (MODE == FA_MODE_INT8_PER_TOKEN) {
-        float m = 0.0f;
+      for (int i = 0; i < 32; ++i) v[i] = fp8_div(f[i], sc, rc);
+    } else {
+      // static scales can be exceeded by x (codes saturate), and INT8: IEEE division
 #pragma unroll
-        for (int i = 0; i < 8; ++i) m = fmaxf(m, fabsf(f[i]));
+      for (int i = 0; i < 32; ++i) v[i] = sc > 0.0f ? __fdiv_rn(f[i], sc) : 0.0f;
+    }
+    if (valid) {
+      uint32_t w[8];
 #pragma unroll
-        for (int off = G / 2; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
-        const float sc = __fdiv_rn(m, 127.0f);
-        float v[8];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) v[i] = sc > 0.0f ? __fdiv_rn(f[i], sc) : 0.0f;
-        if (valid) {
-          uint2 out = make_uint2(s8x4(v[0], v[1], v[2], v[3]), s8x4(v[4], v[5], v[6], v[7]));
-          reinterpret_cast<uint2*>(static_cast<int8_t*>(op.codes) + rr[u] * D)[gl] = out;
-          if (gl == 0) static_cast<float*>(op.scales)[scale_index(rr[u], op.layout, op.H, op.S)] = sc;
-        }
-      } else {  // MXFP4 / MXFP8: one 32-element block = 4 lanes
-        float m = 0.0f;
-#pragma unroll
-        for (int i = 0; i < 8; ++i) m = fmaxf(m, fabsf(f[i]));
-        m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
-        m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 2));
-        const int e = mx_exponent<MODE == FA_MODE_MXFP8_PER_BLOCK ? 8 : 2>(m);
-        const float inv = __uint_as_float((uint32_t)(127 - e) << 23);  // 2^-e, exact
-        float v[8];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) v[i] = f[i] * inv;
-        if (valid) {
-          if (MODE == FA_MODE_MXFP8_PER_BLOCK)
-            reinterpret_cast<uint2*>(static_cast<uint8_t*>(op.codes) + rr[u] * D)[gl] =
-                make_uint2(e4m3x4(v[0], v[1], v[2], v[3]), e4m3x4(v[4], v[5], v[6], v[7]));
-          else
-            reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(op.codes) + rr[u] * (D / 2))[gl] = e2m1x8(v);
-          if ((gl & 3) == 0)
-            static_cast<uint8_t*>(op.scales)[scale_index(rr[u], op.layout, op.H, op.S) * (D / 32) + gl / 4] =
-                (uint8_t)(e + 127);
-        }
+      for (int i = 0; i < 8; ++i)
+        w[i] = INT8 ? s8x4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3])
+                    : e4m3x4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+      out[0] = make_uint4(w[0], w[1], w[2], w[3]);
+      out[1] = make_uint4(w[4], w[5], w[6], w[7]);
+      uint4* dst = reinterpret_cast<uint4*>(static_cast<uint8_t*>(op_codes) + rr * D + gl * 32);
+      dst[0] = out[0];
+      dst[1] = out[1];
+      if (!PER_HEAD && gl == 0) {
+        const int op_layout = which == 0 ? o0.layout : (which == 1 ? o1.layout : o2.layout);
+        const int op_H = which == 0 ? o0.H : (which == 1 ? o1.H : o2.H);
+        const int op_S = which == 0 ? o0.S : (which == 1 ? o1.S : o2.S);
+        static_cast<float*>(op_scales)[scale_index(rr, op_layout, op_H, op_S)] = sc;
       }
     }
   }
@@ -303,7 +321,7 @@ cudaError_t launch_rows_mode(const QuantOperand (&o)[3], int D, cudaStream_t s) 
   if (total == 0) {
     if (MODE != FA_MODE_INT8_PER_HEAD && MODE != FA_MODE_FP8_PER_HEAD) return cudaSuccess;
   }
-  const int rows_per_block = (256 / 32) * (32 / (D / 8)) * 2;
+  const int rows_per_block = (256 / 32) * (32 / (D / 32));
   long long want = (total + rows_per_block - 1) / rows_per_block;
   const long long cap = (long long)sm_count() * 8 * 4;  // enough resident warps, grid-stride beyond
   int grid = (int)(want < 1 ? 1 : (want > cap ? cap : want));
