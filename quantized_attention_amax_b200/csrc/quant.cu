@@ -14,8 +14,8 @@
 // Rows are D contiguous bf16 values in either layout; each row is handled by
 // D/32 lanes with four 16-byte loads each.  x / s is rounded as IEEE division
 // (div.rn.f32) rounds it, so the codes match a correctly rounded x / s exactly:
-// FP8 scales use the FMA-corrected reciprocal product of quant_common.cuh,
-// INT8 (whose static scale can be exceeded) uses IEEE division itself.
+// the FMA-corrected reciprocal products of quant_common.cuh (checked against
+// IEEE division exhaustively), IEEE division itself for scales below 2^-90.
 #include <cuda_bf16.h>
 
 #include "internal.cuh"
@@ -195,12 +195,13 @@ __global__ void __launch_bounds__(256) quant_rows_kernel(QuantOperand o0, QuantO
       sc = __fdiv_rn(m, QMAX);
     }
     float v[32];
-    if (MODE == FA_MODE_FP8_PER_TOKEN && sc >= kFastDivMin) {
+    if (sc >= kFastDivMin) {
+      // x / s as IEEE division rounds it where that decides the code (quant_common.cuh)
       const float rc = __frcp_rn(sc);
 #pragma unroll
-      for (int i = 0; i < 32; ++i) v[i] = fp8_div(f[i], sc, rc);
+      for (int i = 0; i < 32; ++i)
+        v[i] = INT8 ? int8_div(f[i], sc, rc) : (PER_HEAD ? fp8_div_sat(f[i], sc, rc) : fp8_div(f[i], sc, rc));
     } else {
-      // static scales can be exceeded by x (codes saturate), and INT8: IEEE division
 #pragma unroll
       for (int i = 0; i < 32; ++i) v[i] = sc > 0.0f ? __fdiv_rn(f[i], sc) : 0.0f;
     }

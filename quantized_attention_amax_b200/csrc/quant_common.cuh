@@ -17,4 +17,20 @@ __device__ __forceinline__ float fp8_div(float x, float s, float r) {
   return copysignf(fmaf(fmaf(-q0, s, x), r, q0), x);
 }
 
+// The same for a static scale that x can exceed (FP8 per head): quotients of 2^20 or more keep the
+// plain product (they saturate to +-448 either way; the correction would overflow).  Same E4M3
+// codes as IEEE division for every bf16 amax with s >= kFastDivMin and every finite bf16 x.
+__device__ __forceinline__ float fp8_div_sat(float x, float s, float r) {
+  const float q0 = x * r;
+  return fabsf(q0) < 0x1p20f ? copysignf(fmaf(fmaf(-q0, s, x), r, q0), x) : q0;
+}
+
+// INT8 (s = fl(amax / 127)): x / s before round-to-integer and saturation, as IEEE division
+// rounds it where that decides the code, for every bf16 amax with s >= kFastDivMin and every
+// finite bf16 x (the exhaustive check covers this too).
+__device__ __forceinline__ float int8_div(float x, float s, float r) {
+  const float q0 = x * r;
+  return fabsf(q0) < 0x1p20f ? fmaf(fmaf(-q0, s, x), r, q0) : q0;
+}
+
 }  // namespace faq

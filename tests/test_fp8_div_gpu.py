@@ -1,6 +1,7 @@
-"""The FP8 quantizers divide by the scale as x * r plus one FMA correction (quant_common.cuh)
-instead of IEEE division.  This compiles a sweep over every bf16 amax and every bf16 |x| <= amax
-against the product header and requires the same E4M3 code as IEEE division everywhere."""
+"""The quantizers divide by the scale as x * r plus one FMA correction (quant_common.cuh) instead of
+IEEE division.  This compiles a sweep against the product header -- every bf16 amax, and every bf16
+x with |x| <= amax (dynamic FP8) or every finite bf16 x (static FP8, INT8) -- and requires the same
+E4M3 / INT8 code as IEEE division everywhere."""
 import os
 import re
 import subprocess
@@ -21,7 +22,8 @@ def test_fp8_div_matches_ieee_division_exhaustively(tmp_path):
                     exe], check=True, capture_output=True, text=True)
     r = subprocess.run([exe], capture_output=True, text=True, timeout=300)
     assert r.returncode == 0, r.stderr
-    m = re.search(r"fast rows (\d+) mismatches (\d+)", r.stdout)
-    assert m, r.stdout
-    assert int(m.group(1)) > 26000  # nearly every scale takes the fast path
-    assert int(m.group(2)) == 0
+    found = re.findall(r"mode (\d) fast rows (\d+) mismatches (\d+)", r.stdout)
+    assert [int(m) for m, _, _ in found] == [0, 1, 2], r.stdout
+    for _, fast, bad in found:
+        assert int(fast) > 26000  # nearly every scale takes the fast path
+        assert int(bad) == 0
