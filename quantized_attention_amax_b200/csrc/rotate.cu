@@ -3,19 +3,23 @@
 //
 // Q' = bf16(Q R_q), K' = bf16(K R_k) (fp32 accumulation, one rounding), V' = V;
 // then one E4M3 scale = amax / 448 per (b, h, block of `blk` tokens) and
-// codes e4m3(x' / scale).  One CTA handles a 256-token chunk of one
-// (operand, batch, head):
-//   warp 0     TMA: the chunk as two 128-token bf16 tiles (128B-swizzled,
-//              64-element K atoms) and, for Q and K, the rotation R.
-//   warp 1     tcgen05.mma kind::f16 (bf16 x bf16 -> fp32): X R into TMEM,
-//              R read as the MN-major B operand exactly as stored ([D, D]
-//              row-major, x' = x R).
-//   all 8 warps, then, the epilogue: warp w takes TMEM lane quarter w % 4
-//              and column half w / 4 of each 128-token tile; its bf16 half
-//              rows (rotated in TMEM, or V from the shared tile) stay in
-//              registers for half-row maxima -> block maxima (one warp per
-//              block, through shared memory) -> scale -> E4M3 codes (IEEE
-//              division), with an optional bf16 copy of the rotated rows.
+// codes e4m3(x' / scale).  A work item is a 256-token chunk of one
+// (operand, batch, head); one persistent CTA per SM walks the items
+// blockIdx.x, blockIdx.x + gridDim.x, ... in a three-role pipeline:
+//   warp 8     TMA: both rotations once (resident), then each item as two
+//              128-token bf16 tiles (128B-swizzled, 64-element K atoms)
+//              into one of two 64 KB input stages.
+//   warp 9     tcgen05.mma kind::f16 (bf16 x bf16 -> fp32): X R into one of
+//              two 256-column TMEM buffers, R read as the MN-major B operand
+//              exactly as stored ([D, D] row-major, x' = x R).  V items skip it.
+//   warps 0-7  the epilogue of the previous item: warp w takes TMEM lane
+//              quarter w % 4 and column half w / 4 of each 128-token tile; its
+//              bf16 half rows (rotated in TMEM, or V from the shared tile) stay
+//              in registers for half-row maxima -> block maxima (lane
+//              butterflies, then one exchange through shared memory) -> scale
+//              -> E4M3 codes (division rounded as IEEE), with an optional bf16
+//              copy of the rotated rows.
+// So the loads and MMAs of item k + 1 overlap the epilogue of item k.
 // blk must divide 256.
 #include <cuda_bf16.h>
 #include <string.h>
@@ -27,32 +31,46 @@
 namespace faq {
 namespace {
 
-constexpr int CH = 256;  // tokens per CTA
-constexpr int RTHREADS = 256;
+constexpr int CH = 256;          // tokens per work item
+constexpr int REPI = 512;           // epilogue threads (warps 0-15)
+constexpr int RTHREADS = REPI + 64;  // + the TMA producer (warp 16) and the MMA issuer (warp 17)
+constexpr int WPROD = REPI / 32, WMMA = WPROD + 1;
 
 struct RotOp {
   void* codes;
   float* scales;
   __nv_bfloat16* dbg;
   int B, H, S, layout, blk, rotate;
-  long long first_cta;  // first CTA index of this operand
-  int chunks;           // 256-token chunks per (b, h)
+  long long first_item;  // first work item of this operand
+  int chunks;            // 256-token chunks per (b, h)
 };
 
 struct RotParams {
   RotOp op[3];
   int nops;
+  long long items;
   int* status;
 };
 
 struct RSmem {
-  static constexpr uint32_t X = 0;           // [2 tiles][2 K atoms][128 rows][128 B]
-  static constexpr uint32_t R = 65536;       // [2 N atoms][128 d rows][128 B]
-  static constexpr uint32_t RMAX = R + 32768;    // [2 tiles][2 halves][128] half-row maxima
-  static constexpr uint32_t BMAX = RMAX + 2048;  // [256] per-block scale (up to 256 blocks per chunk)
-  static constexpr uint32_t BAR = BMAX + 1024;
+  static constexpr uint32_t X = 0;                 // 2 stages x [2 tiles][2 K atoms][128 rows][128 B]
+  static constexpr uint32_t R = 2 * 65536;         // 2 rotations x [2 N atoms][128 d rows][128 B]
+  static constexpr uint32_t RED = R + 2 * 32768;  // [2 items][2 tiles][8 warps][32 lanes] group maxima
+  static constexpr uint32_t BAR = RED + 4096;
   static constexpr uint32_t TOTAL = BAR + 256;
   static constexpr uint32_t ALLOC = TOTAL + 1024;
+  static_assert(ALLOC <= 227 * 1024, "shared memory per CTA");
+};
+
+enum {
+  RB_XF = 0,    // [2] input stage full (TMA)
+  RB_XE = 2,    // [2] input stage free (the 8 epilogue warps)
+  RB_TF = 4,    // [2] TMEM buffer full (MMA commit)
+  RB_TE = 6,    // [2] TMEM buffer free (the 8 epilogue warps)
+  RB_RF = 8,    // rotations loaded
+  RB_RM = 9,    // group maxima written (256 epilogue threads)
+  RB_FIN = 10,  // every MMA complete
+  RB_COUNT = 11
 };
 
 __device__ __forceinline__ uint32_t e4m3x4(float a, float b, float c, float d) {
@@ -62,188 +80,299 @@ __device__ __forceinline__ uint32_t e4m3x4(float a, float b, float c, float d) {
   return (uint32_t)lo | ((uint32_t)hi << 16);
 }
 
+__device__ __forceinline__ uint32_t bf16x2_max(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("max.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+
 __device__ __forceinline__ uint32_t bf16x2_rn(float lo, float hi) {
   const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<const uint32_t*>(&v);
 }
 
-__global__ void __launch_bounds__(RTHREADS, 2)
+// E4M3 codes of 16 bf16 values (packed pairs in a, b) divided by sc with IEEE division;
+// zero codes when sc == 0.
+__device__ __noinline__ uint4 codes_ieee(uint4 a, uint4 b, float sc) {
+  const uint32_t p[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+  uint32_t w[4];
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    const uint32_t p0 = p[2 * e], p1 = p[2 * e + 1];
+    w[e] = sc > 0.0f ? e4m3x4(__fdiv_rn(__uint_as_float(p0 << 16), sc), __fdiv_rn(__uint_as_float(p0 & 0xFFFF0000u), sc),
+                              __fdiv_rn(__uint_as_float(p1 << 16), sc), __fdiv_rn(__uint_as_float(p1 & 0xFFFF0000u), sc))
+                     : 0u;
+  }
+  return make_uint4(w[0], w[1], w[2], w[3]);
+}
+
+struct RItem {
+  int oi, b, h, t0, ntile;
+};
+
+__device__ __forceinline__ RItem decode_item(const RotParams& prm, long long g) {
+  RItem it;
+  it.oi = 0;
+  if (prm.nops > 1 && g >= prm.op[1].first_item) it.oi = 1;
+  if (prm.nops > 2 && g >= prm.op[2].first_item) it.oi = 2;
+  const RotOp& op = prm.op[it.oi];
+  const long long local = g - op.first_item;
+  int chunk;
+  if (op.layout == FA_LAYOUT_BNSD) {
+    // (b, h, chunk): a chunk is one contiguous 64 KB stretch
+    chunk = (int)(local % op.chunks);
+    const long long bh = local / op.chunks;
+    it.h = (int)(bh % op.H);
+    it.b = (int)(bh / op.H);
+  } else {
+    // (b, chunk, h): a token's heads are adjacent in memory, so neighbouring CTAs, taking
+    // neighbouring heads of one token range, read and write whole DRAM pages between them
+    it.h = (int)(local % op.H);
+    const long long bc = local / op.H;
+    chunk = (int)(bc % op.chunks);
+    it.b = (int)(bc / op.chunks);
+  }
+  it.t0 = chunk * CH;
+  it.ntile = min(2, (op.S - it.t0 + 127) / 128);
+  return it;
+}
+
+// Persistent: one CTA per SM walks work items g = blockIdx.x, blockIdx.x + gridDim.x, ...
+// (operand, batch, head, 256-token chunk).  The producer loads item k + 1's tiles into the other
+// input stage and the MMA thread rotates it into the other TMEM buffer while the epilogue warps
+// quantize item k.
+__global__ void __launch_bounds__(RTHREADS, 1)
     rotate_block_quant_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtensorMap mk,
                               const __grid_constant__ CUtensorMap mv, const __grid_constant__ CUtensorMap mrq,
                               const __grid_constant__ CUtensorMap mrk, const RotParams prm) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* bar = reinterpret_cast<uint64_t*>(smem + RSmem::BAR);  // 0: loads, 1: mma, 2: row maxima, 3: block scales
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar + 4);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(bar + 5);
-  float* rmax = reinterpret_cast<float*>(smem + RSmem::RMAX);
-  float* bsc = reinterpret_cast<float*>(smem + RSmem::BMAX);
+  uint64_t* bar = reinterpret_cast<uint64_t*>(smem + RSmem::BAR);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar + RB_COUNT);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(bar + RB_COUNT + 1);
+  float* red = reinterpret_cast<float*>(smem + RSmem::RED);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const long long cta = blockIdx.x;
-  int oi = 0;
-  if (prm.nops > 1 && cta >= prm.op[1].first_cta) oi = 1;
-  if (prm.nops > 2 && cta >= prm.op[2].first_cta) oi = 2;
-  const RotOp& op = prm.op[oi];
-  const CUtensorMap* mx = oi == 0 ? &mq : (oi == 1 ? &mk : &mv);
-  const CUtensorMap* mr = oi == 0 ? &mrq : &mrk;
-  const long long local = cta - op.first_cta;
-  const int chunk = (int)(local % op.chunks);
-  const long long bh = local / op.chunks;
-  const int h = (int)(bh % op.H), b = (int)(bh / op.H);
-  const int t0 = chunk * CH;
-  const int ntile = min(2, (op.S - t0 + 127) / 128);
-  const bool bnsd = op.layout == FA_LAYOUT_BNSD;
+  const long long G = gridDim.x;
+  int nrot = 0;  // operands with a rotation (they come first: Q, then K)
+  for (int i = 0; i < prm.nops; ++i) nrot += prm.op[i].rotate;
 
   if (tid == 0) {
-    mbar_init(&bar[0], 1);
-    mbar_init(&bar[1], 1);
-    mbar_init(&bar[2], RTHREADS);
-    mbar_init(&bar[3], RTHREADS);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&bar[RB_XF + i], 1);
+      mbar_init(&bar[RB_XE + i], REPI / 32);
+      mbar_init(&bar[RB_TF + i], 1);
+      mbar_init(&bar[RB_TE + i], REPI / 32);
+    }
+    mbar_init(&bar[RB_RF], 1);
+    mbar_init(&bar[RB_RM], REPI);
+    mbar_init(&bar[RB_FIN], 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
-  if (warp == 1) {
-    tmem_alloc(tmem_slot, 256);
+  if (warp == WMMA) {
+    tmem_alloc(tmem_slot, 512);
     tmem_relinquish();
   }
   __syncthreads();
   tc_fence_after();
-  const uint32_t tbase = *tmem_slot;
+  const uint32_t tbase = *tmem_slot;  // TMEM buffer t at columns 256 t: [2 tiles][128]
 
-  if (warp == 0) {
+  if (warp == WPROD) {
+    // ------------------------------------------------------------- producer
     if (lane == 0) {
-      const uint32_t bytes = ntile * 2 * 16384 + (op.rotate ? 32768 : 0);
-      mbar_arrive_expect_tx(&bar[0], bytes);
-      for (int u = 0; u < ntile; ++u)
-        for (int kb = 0; kb < 2; ++kb) {
-          const int t = t0 + u * 128;
-          tma_load_4d(smem + RSmem::X + (u * 2 + kb) * 16384, mx, &bar[0], kb * 64, bnsd ? t : h, bnsd ? h : t, b);
-        }
-      if (op.rotate)
-        for (int nb = 0; nb < 2; ++nb) tma_load_4d(smem + RSmem::R + nb * 16384, mr, &bar[0], nb * 64, 0, 0, 0);
+      if (nrot > 0) {
+        mbar_arrive_expect_tx(&bar[RB_RF], nrot * 32768);
+        for (int r = 0; r < nrot; ++r)
+          for (int nb = 0; nb < 2; ++nb)
+            tma_load_4d(smem + RSmem::R + r * 32768 + nb * 16384, r == 0 ? &mrq : &mrk, &bar[RB_RF], nb * 64, 0, 0, 0);
+      }
+      long long k = 0;
+      for (long long g = blockIdx.x; g < prm.items; g += G, ++k) {
+        const int st = (int)(k & 1);
+        if (k >= 2 && !mbar_wait(&bar[RB_XE + st], (uint32_t)(((k >> 1) - 1) & 1), abort_flag, prm.status, 45)) break;
+        const RItem it = decode_item(prm, g);
+        const RotOp& op = prm.op[it.oi];
+        const CUtensorMap* mx = it.oi == 0 ? &mq : (it.oi == 1 ? &mk : &mv);
+        const bool bnsd = op.layout == FA_LAYOUT_BNSD;
+        mbar_arrive_expect_tx(&bar[RB_XF + st], it.ntile * 2 * 16384);
+        for (int u = 0; u < it.ntile; ++u)
+          for (int kb = 0; kb < 2; ++kb) {
+            const int t = it.t0 + u * 128;
+            tma_load_4d(smem + RSmem::X + st * 65536 + (u * 2 + kb) * 16384, mx, &bar[RB_XF + st], kb * 64,
+                        bnsd ? t : it.h, bnsd ? it.h : t, it.b);
+          }
+      }
+      if (*abort_flag) {
+        // let loads already issued land before the CTA can exit
+        if (nrot > 0) mbar_wait(&bar[RB_RF], 0, abort_flag, nullptr, 0);
+        for (long long t = (k >= 2 ? k - 2 : 0); t < k; ++t)
+          mbar_wait(&bar[RB_XF + (t & 1)], (uint32_t)((t >> 1) & 1), abort_flag, nullptr, 0);
+      }
     }
     __syncwarp();
-  } else if (warp == 1) {
-    if (lane == 0 && op.rotate) {
+  } else if (warp == WMMA) {
+    // ----------------------------------------------------------- MMA issuer
+    if (lane == 0) {
       constexpr uint32_t idesc = make_idesc(kAccF32, kFmtBF16, kFmtBF16, 0, 1, 128, 128);
-      if (mbar_wait(&bar[0], 0, abort_flag, prm.status, 40)) {
+      bool ok = nrot == 0 || mbar_wait(&bar[RB_RF], 0, abort_flag, prm.status, 46);
+      long long k = 0;
+      int tuse0 = 0, tuse1 = 0;  // rotate items so far per TMEM buffer
+      for (long long g = blockIdx.x; ok && g < prm.items; g += G, ++k) {
+        const RItem it = decode_item(prm, g);
+        const RotOp& op = prm.op[it.oi];
+        if (!op.rotate) continue;
+        const int st = (int)(k & 1), tb = (int)(k & 1);
+        if (!mbar_wait(&bar[RB_XF + st], (uint32_t)((k >> 1) & 1), abort_flag, prm.status, 47)) break;
+        const int tu = tb ? tuse1 : tuse0;
+        if (tu > 0 && !mbar_wait(&bar[RB_TE + tb], (uint32_t)((tu - 1) & 1), abort_flag, prm.status, 48)) break;
         tc_fence_after();
-        const uint32_t sR = smem_u32(smem + RSmem::R);
-        for (int u = 0; u < ntile; ++u) {
-          const uint32_t sX = smem_u32(smem + RSmem::X + u * 2 * 16384);
+        const uint32_t sR = smem_u32(smem + RSmem::R + it.oi * 32768);
+        for (int u = 0; u < it.ntile; ++u) {
+          const uint32_t sX = smem_u32(smem + RSmem::X + st * 65536 + u * 2 * 16384);
 #pragma unroll
           for (int ks = 0; ks < 8; ++ks) {
             const uint64_t da = make_sdesc(sX + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024, kSwz128);
             const uint64_t db = make_sdesc(sR + ks * 16 * 128, 16384, 1024, kSwz128);
-            mma_f16(tbase + u * 128, da, db, idesc, ks > 0);
+            mma_f16(tbase + tb * 256 + u * 128, da, db, idesc, ks > 0);
           }
         }
+        mma_commit(&bar[RB_TF + tb]);
+        if (tb) ++tuse1; else ++tuse0;
       }
-      mma_commit(&bar[1]);
-      mbar_wait(&bar[1], 0, abort_flag, nullptr, 0);
+      mma_commit(&bar[RB_FIN]);
+      mbar_wait(&bar[RB_FIN], 0, abort_flag, nullptr, 0);
     }
     __syncwarp();
-  }
-
-  // ---------------------------------------------------------------- epilogue
-  const int half = warp >> 2;                 // columns [64 * half, 64 * half + 64)
-  const int i = (warp & 3) * 32 + lane;       // row within a 128-token tile
-  const uint32_t loff = (uint32_t)((warp & 3) * 32) << 16;
-  bool ok = mbar_wait(&bar[op.rotate ? 1 : 0], 0, abort_flag, prm.status, op.rotate ? 41 : 42);
-  ok = __all_sync(0xffffffffu, ok);
-  if (op.rotate) tc_fence_after();
-  // 64 elements (half a row) of each tile as 32 packed bf16x2
-  uint32_t v[2][32];
-#pragma unroll
-  for (int u = 0; u < 2; ++u) {
-    const int t = t0 + u * 128 + i;
-    const bool live = u < ntile && t < op.S;
-    float am = 0.0f;
-    if (u < ntile && ok) {  // warp-uniform: TMEM loads are warp-collective
+  } else {
+    // -------------------------------------------------------------- epilogue
+    // warp e: tile u = e / 8, column half (e / 4) % 2, TMEM lane quarter e % 4
+    const int u = warp >> 3, half = (warp >> 2) & 1, quarter = warp & 3;
+    const int i = quarter * 32 + lane;  // row within the 128-token tile
+    const uint32_t loff = (uint32_t)(quarter * 32) << 16;
+    bool ok = true;
+    long long k = 0;
+    int tuse0 = 0, tuse1 = 0;  // rotate items so far per TMEM buffer
+    for (long long g = blockIdx.x; ok && g < prm.items; g += G, ++k) {
+      const RItem it = decode_item(prm, g);
+      const RotOp& op = prm.op[it.oi];
+      const int st = (int)(k & 1);
+      const bool bnsd = op.layout == FA_LAYOUT_BNSD;
+      const bool tile_live = u < it.ntile;  // warp-uniform
+      // 64 elements (half a row) as 32 packed bf16x2
+      uint32_t v[32];
       if (op.rotate) {
+        const int tb = (int)(k & 1);
+        const int tu = tb ? tuse1 : tuse0;
+        ok = __all_sync(0xffffffffu, mbar_wait(&bar[RB_TF + tb], (uint32_t)(tu & 1), abort_flag, prm.status, 41));
+        if (tb) ++tuse1; else ++tuse0;
+        if (!ok) break;
+        tc_fence_after();
+        if (tile_live) {  // TMEM loads are warp-collective
 #pragma unroll
-        for (int c = 0; c < 2; ++c) {
-          uint32_t r[32];
-          tmem_ld32(tbase + u * 128 + loff + half * 64 + c * 32, r);
-          tmem_ld_wait();
+          for (int c = 0; c < 2; ++c) {
+            uint32_t r[32];
+            tmem_ld32(tbase + tb * 256 + u * 128 + loff + half * 64 + c * 32, r);
+            tmem_ld_wait();
 #pragma unroll
-          for (int k = 0; k < 16; ++k) v[u][c * 16 + k] = bf16x2_rn(__uint_as_float(r[2 * k]), __uint_as_float(r[2 * k + 1]));
+            for (int q = 0; q < 16; ++q) v[c * 16 + q] = bf16x2_rn(__uint_as_float(r[2 * q]), __uint_as_float(r[2 * q + 1]));
+          }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive(&bar[RB_TE + tb]);
+          mbar_arrive(&bar[RB_XE + st]);  // the MMA that read the stage has completed
         }
       } else {
+        ok = __all_sync(0xffffffffu, mbar_wait(&bar[RB_XF + st], (uint32_t)((k >> 1) & 1), abort_flag, prm.status, 42));
+        if (!ok) break;
+        if (tile_live) {
 #pragma unroll
-        for (int q = 0; q < 8; ++q) {
-          const uint4 x = *reinterpret_cast<const uint4*>(smem + RSmem::X + (u * 2 + half) * 16384 + swz128_offset(i, q));
-          v[u][4 * q] = x.x; v[u][4 * q + 1] = x.y; v[u][4 * q + 2] = x.z; v[u][4 * q + 3] = x.w;
+          for (int q = 0; q < 8; ++q) {
+            const uint4 x = *reinterpret_cast<const uint4*>(smem + RSmem::X + st * 65536 + (u * 2 + half) * 16384 +
+                                                             swz128_offset(i, q));
+            v[4 * q] = x.x; v[4 * q + 1] = x.y; v[4 * q + 2] = x.z; v[4 * q + 3] = x.w;
+          }
         }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bar[RB_XE + st]);
       }
+      // Block maxima.  blk divides 256, so it is a power of two: a block is either a group of
+      // blk <= 32 adjacent lanes of one warp (its two column halves in warps e and e ^ 4) or
+      // blk / 32 whole row quarters, both halves.  Butterflies over the group's lanes leave
+      // every lane with its group's maximum; one shared exchange, double-buffered by item
+      // parity so a single barrier per item suffices, combines the rest.
+      const int t = it.t0 + u * 128 + i;
+      const bool live = tile_live && t < op.S;
+      float am = 0.0f;
+      if (live) {
+        uint32_t m2 = 0;  // running max of |x| as packed bf16x2 (bf16 max is exact)
 #pragma unroll
-      for (int k = 0; k < 32; ++k)
-        am = fmaxf(am, fmaxf(fabsf(__uint_as_float(v[u][k] << 16)), fabsf(__uint_as_float(v[u][k] & 0xFFFF0000u))));
-      if (op.dbg && live) {
-        const long long ridx = bnsd ? (((long long)b * op.H + h) * op.S + t) : (((long long)b * op.S + t) * op.H + h);
+        for (int q = 0; q < 32; ++q) m2 = bf16x2_max(m2, v[q] & 0x7FFF7FFFu);
+        am = fmaxf(__uint_as_float(m2 << 16), __uint_as_float(m2 & 0xFFFF0000u));
+      }
+      const long long ridx = bnsd ? (((long long)it.b * op.H + it.h) * op.S + t) : (((long long)it.b * op.S + t) * op.H + it.h);
+      if (live && op.dbg) {
         uint4* d = reinterpret_cast<uint4*>(op.dbg + ridx * 128 + half * 64);
 #pragma unroll
-        for (int q = 0; q < 8; ++q) d[q] = make_uint4(v[u][4 * q], v[u][4 * q + 1], v[u][4 * q + 2], v[u][4 * q + 3]);
+        for (int q = 0; q < 8; ++q) d[q] = make_uint4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+      }
+      const int gl = op.blk < 32 ? op.blk : 32;
+      for (int off = 1; off < gl; off <<= 1) am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, off));
+      float* rd = red + (k & 1) * 512;  // [16 warps][32 lanes]
+      rd[warp * 32 + lane] = am;
+      mbar_arrive(&bar[RB_RM]);
+      ok = __all_sync(0xffffffffu, mbar_wait(&bar[RB_RM], (uint32_t)(k & 1), abort_flag, prm.status, 43));
+      if (!ok) break;
+      if (!live) continue;
+      const int r_in = u * 128 + i;  // row within the chunk
+      float m;
+      if (op.blk <= 32) {
+        m = fmaxf(rd[(u * 8 + quarter) * 32 + lane], rd[(u * 8 + quarter + 4) * 32 + lane]);
+      } else {
+        m = 0.0f;
+        const int g0 = (r_in & ~(op.blk - 1)) >> 5;  // first 32-row group of the block
+        for (int gq = g0; gq < g0 + (op.blk >> 5); ++gq) {
+          const int uu = gq >> 2, qq = gq & 3;
+          m = fmaxf(m, fmaxf(rd[(uu * 8 + qq) * 32], rd[(uu * 8 + qq + 4) * 32]));
+        }
+      }
+      const float sc = __fdiv_rn(m, 448.0f);
+      if (half == 0 && (r_in & (op.blk - 1)) == 0) {
+        const int nblk = (op.S + op.blk - 1) / op.blk;
+        op.scales[((long long)it.b * op.H + it.h) * nblk + t / op.blk] = sc;
+      }
+      // codes: this thread's 64 values
+      uint4* crow = reinterpret_cast<uint4*>(static_cast<uint8_t*>(op.codes) + ridx * 128 + half * 64);
+      if (sc >= kFastDivMin) {
+        const float rc = __frcp_rn(sc);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          uint32_t w[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const uint32_t p0 = v[8 * q + 2 * e], p1 = v[8 * q + 2 * e + 1];
+            w[e] = e4m3x4(fp8_div(__uint_as_float(p0 << 16), sc, rc), fp8_div(__uint_as_float(p0 & 0xFFFF0000u), sc, rc),
+                          fp8_div(__uint_as_float(p1 << 16), sc, rc), fp8_div(__uint_as_float(p1 & 0xFFFF0000u), sc, rc));
+          }
+          crow[q] = make_uint4(w[0], w[1], w[2], w[3]);
+        }
+      } else {
+        // tiny or zero scale: IEEE division, out of line (rare)
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+          crow[q] = codes_ieee(make_uint4(v[8 * q], v[8 * q + 1], v[8 * q + 2], v[8 * q + 3]),
+                               make_uint4(v[8 * q + 4], v[8 * q + 5], v[8 * q + 6], v[8 * q + 7]), sc);
       }
     }
-    rmax[(u * 2 + half) * 128 + i] = live ? am : 0.0f;
-  }
-  mbar_arrive(&bar[2]);
-  ok = __all_sync(0xffffffffu, mbar_wait(&bar[2], 0, abort_flag, prm.status, 43)) && ok;
-
-  // block scales: warp w reduces blocks w, w + 8, ... of the chunk (2 * blk half-row maxima each)
-  const int nb_chunk = CH / op.blk;
-  const int nblk = (op.S + op.blk - 1) / op.blk;
-  for (int bb = warp; bb < nb_chunk; bb += RTHREADS / 32) {
-    float m = 0.0f;
-    for (int k = lane; k < 2 * op.blk; k += 32) {
-      const int row = bb * op.blk + (k >> 1);
-      m = fmaxf(m, rmax[((row >> 7) * 2 + (k & 1)) * 128 + (row & 127)]);
-    }
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
-    const float sc = __fdiv_rn(m, 448.0f);
-    if (lane == 0) {
-      bsc[bb] = sc;
-      const int t = t0 + bb * op.blk;
-      if (t < op.S) op.scales[((long long)b * op.H + h) * nblk + t / op.blk] = ok ? sc : 0.0f;
-    }
-  }
-  mbar_arrive(&bar[3]);
-  ok = __all_sync(0xffffffffu, mbar_wait(&bar[3], 0, abort_flag, prm.status, 44)) && ok;
-
-  // codes: this thread's 64 values of each tile row
-#pragma unroll
-  for (int u = 0; u < 2; ++u) {
-    const int r_in = u * 128 + i;
-    const int t = t0 + r_in;
-    if (!(u < ntile && t < op.S)) continue;
-    const float sc = bsc[r_in / op.blk];
-    const bool fast = sc >= kFastDivMin;
-    const float rc = fast ? __frcp_rn(sc) : 0.0f;
-    const long long ridx = bnsd ? (((long long)b * op.H + h) * op.S + t) : (((long long)b * op.S + t) * op.H + h);
-    uint32_t w[16];
-#pragma unroll
-    for (int e = 0; e < 16; ++e) {
-      const uint32_t p0 = v[u][2 * e], p1 = v[u][2 * e + 1];
-      const float x0 = __uint_as_float(p0 << 16), x1 = __uint_as_float(p0 & 0xFFFF0000u);
-      const float x2 = __uint_as_float(p1 << 16), x3 = __uint_as_float(p1 & 0xFFFF0000u);
-      if (fast)
-        w[e] = ok ? e4m3x4(fp8_div(x0, sc, rc), fp8_div(x1, sc, rc), fp8_div(x2, sc, rc), fp8_div(x3, sc, rc)) : 0u;
-      else
-        w[e] = (sc > 0.0f && ok) ? e4m3x4(__fdiv_rn(x0, sc), __fdiv_rn(x1, sc), __fdiv_rn(x2, sc), __fdiv_rn(x3, sc)) : 0u;
-    }
-    uint4* crow = reinterpret_cast<uint4*>(static_cast<uint8_t*>(op.codes) + ridx * 128 + half * 64);
-#pragma unroll
-    for (int q = 0; q < 4; ++q) crow[q] = make_uint4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
   }
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 1) {
+  if (warp == WMMA) {
     tc_fence_after();
-    tmem_dealloc(tbase, 256);
+    tmem_dealloc(tbase, 512);
   }
 }
 
@@ -302,7 +431,7 @@ cudaError_t launch_rotate_block_quant(const RotateOperand* ops, int nops, int* s
     r.B = o.B; r.H = o.H; r.S = o.S; r.layout = o.layout; r.blk = o.blk;
     r.rotate = o.R != nullptr;
     r.chunks = (o.S + CH - 1) / CH;
-    r.first_cta = total;
+    r.first_item = total;
     total += (long long)o.B * o.H * r.chunks;
     cudaError_t e = make_bf16_map(&maps[n], o.x, o.B, o.H, o.S, o.layout);
     if (e != cudaSuccess) return e;
@@ -314,8 +443,11 @@ cudaError_t launch_rotate_block_quant(const RotateOperand* ops, int nops, int* s
     ++n;
   }
   prm.nops = n;
+  prm.items = total;
   if (n == 0) return cudaSuccess;
-  if (total > 0x7FFFFFFFLL) return cudaErrorInvalidValue;
+  // the operands with a rotation come first (their rotations occupy shared-memory slots 0, 1)
+  for (int i = 1; i < n; ++i)
+    if (prm.op[i].rotate && !prm.op[i - 1].rotate) return cudaErrorNotSupported;
   static bool attr = false;
   if (!attr) {
     cudaError_t e = cudaFuncSetAttribute(rotate_block_quant_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -323,8 +455,9 @@ cudaError_t launch_rotate_block_quant(const RotateOperand* ops, int nops, int* s
     if (e != cudaSuccess) return e;
     attr = true;
   }
-  rotate_block_quant_kernel<<<(unsigned)total, RTHREADS, RSmem::ALLOC, s>>>(maps[0], maps[1], maps[2], rmaps[0],
-                                                                            rmaps[1], prm);
+  const long long grid = total < sm_count() ? total : sm_count();
+  rotate_block_quant_kernel<<<(unsigned)grid, RTHREADS, RSmem::ALLOC, s>>>(maps[0], maps[1], maps[2], rmaps[0],
+                                                                           rmaps[1], prm);
   return cudaGetLastError();
 }
 
