@@ -7,14 +7,16 @@ namespace faq {
 
 // x / s rounded to fp32 as IEEE division does, for an FP8 scale s = fl(amax / 448) with
 // s >= kFastDivMin and a bf16 |x| <= amax: q0 = x * r with r the correctly rounded 1 / s, then one
-// FMA residual x - q0 * s (exact) and one FMA correction; copysign keeps the sign of a zero x.
+// FMA for the negated residual q0 * s - x (exact) and one FMA correction q0 - that * r.  Taking the
+// residual negated keeps the sign of a zero x (-0 gives -0 where x - q0 * s would give +0); for a
+// nonzero result the two forms round identically, the sign flips being exact.
 // Its E4M3 codes equal those of IEEE division for every bf16 amax whose scale reaches kFastDivMin
 // and every bf16 |x| <= amax (an exhaustive check on the GPU); scales below it use IEEE division.
 constexpr float kFastDivMin = 0x1p-90f;
 
 __device__ __forceinline__ float fp8_div(float x, float s, float r) {
   const float q0 = x * r;
-  return copysignf(fmaf(fmaf(-q0, s, x), r, q0), x);
+  return fmaf(-fmaf(q0, s, -x), r, q0);
 }
 
 // The same for a static scale that x can exceed (FP8 per head): quotients of 2^20 or more keep the
@@ -22,7 +24,7 @@ __device__ __forceinline__ float fp8_div(float x, float s, float r) {
 // codes as IEEE division for every bf16 amax with s >= kFastDivMin and every finite bf16 x.
 __device__ __forceinline__ float fp8_div_sat(float x, float s, float r) {
   const float q0 = x * r;
-  return fabsf(q0) < 0x1p20f ? copysignf(fmaf(fmaf(-q0, s, x), r, q0), x) : q0;
+  return fabsf(q0) < 0x1p20f ? fmaf(-fmaf(q0, s, -x), r, q0) : q0;
 }
 
 // INT8 (s = fl(amax / 127)): x / s before round-to-integer and saturation, as IEEE division

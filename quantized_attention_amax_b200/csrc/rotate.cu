@@ -36,13 +36,36 @@ constexpr int REPI = 512;           // epilogue threads (warps 0-15)
 constexpr int RTHREADS = REPI + 64;  // + the TMA producer (warp 16) and the MMA issuer (warp 17)
 constexpr int WPROD = REPI / 32, WMMA = WPROD + 1;
 
+// n / d for 0 <= n < 2^31 as one widening multiply and a shift: l = ceil(log2 d),
+// m = floor(2^(31 + l) / d) + 1 < 2^32; then n m / 2^(31 + l) = n / d + n (m - 2^(31 + l) / d) / 2^(31 + l)
+// and the error term is below 2^-l <= 1 / d, so the floor is exact.
+struct FastDiv {
+  uint32_t d, m;
+  int l;
+};
+
+inline FastDiv make_fastdiv(uint32_t d) {
+  FastDiv f;
+  f.d = d;
+  f.l = 0;
+  while ((1u << f.l) < d) ++f.l;
+  f.m = (uint32_t)((1ull << (31 + f.l)) / d + 1);
+  return f;
+}
+
+__device__ __forceinline__ uint32_t fdiv(uint32_t n, const FastDiv& f) {
+  return (uint32_t)(((unsigned long long)n * f.m) >> (31 + f.l));
+}
+
 struct RotOp {
   void* codes;
   float* scales;
   __nv_bfloat16* dbg;
   int B, H, S, layout, blk, rotate;
+  int lblk;              // log2(blk) (blk divides 256, so it is a power of two)
   long long first_item;  // first work item of this operand
   int chunks;            // 256-token chunks per (b, h)
+  FastDiv fd_chunks, fd_h;
 };
 
 struct RotParams {
@@ -80,9 +103,10 @@ __device__ __forceinline__ uint32_t e4m3x4(float a, float b, float c, float d) {
   return (uint32_t)lo | ((uint32_t)hi << 16);
 }
 
-__device__ __forceinline__ uint32_t bf16x2_max(uint32_t a, uint32_t b) {
+// per half: max(|a|, |b|), its sign the XOR of the inputs' signs (exact; only magnitudes are used)
+__device__ __forceinline__ uint32_t bf16x2_absmax(uint32_t a, uint32_t b) {
   uint32_t d;
-  asm("max.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  asm("max.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
   return d;
 }
 
@@ -116,23 +140,25 @@ __device__ __forceinline__ RItem decode_item(const RotParams& prm, long long g) 
   if (prm.nops > 1 && g >= prm.op[1].first_item) it.oi = 1;
   if (prm.nops > 2 && g >= prm.op[2].first_item) it.oi = 2;
   const RotOp& op = prm.op[it.oi];
-  const long long local = g - op.first_item;
-  int chunk;
+  const uint32_t local = (uint32_t)(g - op.first_item);  // < 2^31 (checked at launch)
+  uint32_t chunk;
   if (op.layout == FA_LAYOUT_BNSD) {
     // (b, h, chunk): a chunk is one contiguous 64 KB stretch
-    chunk = (int)(local % op.chunks);
-    const long long bh = local / op.chunks;
-    it.h = (int)(bh % op.H);
-    it.b = (int)(bh / op.H);
+    const uint32_t bh = fdiv(local, op.fd_chunks);
+    chunk = local - bh * op.chunks;
+    const uint32_t b = fdiv(bh, op.fd_h);
+    it.h = (int)(bh - b * op.H);
+    it.b = (int)b;
   } else {
     // (b, chunk, h): a token's heads are adjacent in memory, so neighbouring CTAs, taking
     // neighbouring heads of one token range, read and write whole DRAM pages between them
-    it.h = (int)(local % op.H);
-    const long long bc = local / op.H;
-    chunk = (int)(bc % op.chunks);
-    it.b = (int)(bc / op.chunks);
+    const uint32_t bc = fdiv(local, op.fd_h);
+    it.h = (int)(local - bc * op.H);
+    const uint32_t b = fdiv(bc, op.fd_chunks);
+    chunk = bc - b * op.chunks;
+    it.b = (int)b;
   }
-  it.t0 = chunk * CH;
+  it.t0 = (int)chunk * CH;
   it.ntile = min(2, (op.S - it.t0 + 127) / 128);
   return it;
 }
@@ -307,9 +333,10 @@ __global__ void __launch_bounds__(RTHREADS, 1)
       const bool live = tile_live && t < op.S;
       float am = 0.0f;
       if (live) {
-        uint32_t m2 = 0;  // running max of |x| as packed bf16x2 (bf16 max is exact)
+        uint32_t m2 = 0;  // running max of |x| as packed bf16x2 (signs garbage until masked)
 #pragma unroll
-        for (int q = 0; q < 32; ++q) m2 = bf16x2_max(m2, v[q] & 0x7FFF7FFFu);
+        for (int q = 0; q < 32; ++q) m2 = bf16x2_absmax(m2, v[q]);
+        m2 &= 0x7FFF7FFFu;
         am = fmaxf(__uint_as_float(m2 << 16), __uint_as_float(m2 & 0xFFFF0000u));
       }
       const long long ridx = bnsd ? (((long long)it.b * op.H + it.h) * op.S + t) : (((long long)it.b * op.S + t) * op.H + it.h);
@@ -340,8 +367,8 @@ __global__ void __launch_bounds__(RTHREADS, 1)
       }
       const float sc = __fdiv_rn(m, 448.0f);
       if (half == 0 && (r_in & (op.blk - 1)) == 0) {
-        const int nblk = (op.S + op.blk - 1) / op.blk;
-        op.scales[((long long)it.b * op.H + it.h) * nblk + t / op.blk] = sc;
+        const int nblk = (op.S + op.blk - 1) >> op.lblk;
+        op.scales[((long long)it.b * op.H + it.h) * nblk + (t >> op.lblk)] = sc;
       }
       // codes: this thread's 64 values
       uint4* crow = reinterpret_cast<uint4*>(static_cast<uint8_t*>(op.codes) + ridx * 128 + half * 64);
@@ -423,7 +450,7 @@ cudaError_t launch_rotate_block_quant(const RotateOperand* ops, int nops, int* s
     const RotateOperand& o = ops[i];
     if (o.D != 128) return cudaErrorNotSupported;
     if (CH % o.blk != 0) return cudaErrorNotSupported;
-    if ((long long)o.B * o.S == 0) continue;
+    if ((long long)o.B * o.H * o.S == 0) continue;
     RotOp& r = prm.op[n];
     r.codes = o.codes;
     r.scales = o.scales;
@@ -431,6 +458,10 @@ cudaError_t launch_rotate_block_quant(const RotateOperand* ops, int nops, int* s
     r.B = o.B; r.H = o.H; r.S = o.S; r.layout = o.layout; r.blk = o.blk;
     r.rotate = o.R != nullptr;
     r.chunks = (o.S + CH - 1) / CH;
+    r.lblk = 0;
+    while ((1 << r.lblk) < o.blk) ++r.lblk;
+    r.fd_chunks = make_fastdiv((uint32_t)r.chunks);
+    r.fd_h = make_fastdiv((uint32_t)o.H);
     r.first_item = total;
     total += (long long)o.B * o.H * r.chunks;
     cudaError_t e = make_bf16_map(&maps[n], o.x, o.B, o.H, o.S, o.layout);
@@ -445,6 +476,7 @@ cudaError_t launch_rotate_block_quant(const RotateOperand* ops, int nops, int* s
   prm.nops = n;
   prm.items = total;
   if (n == 0) return cudaSuccess;
+  if (total > 0x7FFFFFFFLL) return cudaErrorInvalidValue;  // item indices stay below 2^31
   // the operands with a rotation come first (their rotations occupy shared-memory slots 0, 1)
   for (int i = 1; i < n; ++i)
     if (prm.op[i].rotate && !prm.op[i - 1].rotate) return cudaErrorNotSupported;
