@@ -6,19 +6,23 @@
 // codes e4m3(x' / scale).  A work item is a 256-token chunk of one
 // (operand, batch, head); one persistent CTA per SM walks the items
 // blockIdx.x, blockIdx.x + gridDim.x, ... in a three-role pipeline:
-//   warp 8     TMA: both rotations once (resident), then each item as two
-//              128-token bf16 tiles (128B-swizzled, 64-element K atoms)
-//              into one of two 64 KB input stages.
-//   warp 9     tcgen05.mma kind::f16 (bf16 x bf16 -> fp32): X R into one of
-//              two 256-column TMEM buffers, R read as the MN-major B operand
-//              exactly as stored ([D, D] row-major, x' = x R).  V items skip it.
-//   warps 0-7  the epilogue of the previous item: warp w takes TMEM lane
-//              quarter w % 4 and column half w / 4 of each 128-token tile; its
-//              bf16 half rows (rotated in TMEM, or V from the shared tile) stay
-//              in registers for half-row maxima -> block maxima (lane
-//              butterflies, then one exchange through shared memory) -> scale
-//              -> E4M3 codes (division rounded as IEEE), with an optional bf16
-//              copy of the rotated rows.
+//   warp 16     TMA: each item as two 128-token bf16 tiles (128B-swizzled,
+//               64-element K atoms) into one of two 64 KB input stages; the
+//               items come in operand order (Q, K, V), so the one resident
+//               rotation is loaded when the operand changes, after the MMAs
+//               that read the previous one.
+//   warp 17     tcgen05.mma kind::f16 (bf16 x bf16 -> fp32): X R into one of
+//               two 256-column TMEM buffers, R read as the MN-major B operand
+//               exactly as stored ([D, D] row-major, x' = x R).  V items skip it.
+//   warps 0-15  the epilogue of the previous item: warp e takes tile e / 8,
+//               column half (e / 4) % 2 and TMEM lane quarter e % 4; its bf16
+//               half row (rotated in TMEM, or V from the shared tile) stays in
+//               registers for half-row maxima -> block maxima (lane
+//               butterflies, then one exchange through shared memory) -> scale
+//               -> E4M3 codes (division rounded as IEEE), staged in a swizzled
+//               shared tile that one TMA store per 128-token tile writes out as
+//               whole 128-byte rows (an optional bf16 copy of the rotated rows
+//               goes out with plain stores).
 // So the loads and MMAs of item k + 1 overlap the epilogue of item k.
 // blk must divide 256.
 #include <cuda_bf16.h>
@@ -32,8 +36,10 @@ namespace faq {
 namespace {
 
 constexpr int CH = 256;          // tokens per work item
-constexpr int REPI = 512;           // epilogue threads (warps 0-15)
-constexpr int RTHREADS = REPI + 64;  // + the TMA producer (warp 16) and the MMA issuer (warp 17)
+constexpr int NCP = 2;                // column parts per row: a thread holds 128 / NCP values of a row
+constexpr int CW = 128 / NCP;         // columns per thread
+constexpr int REPI = 32 * 8 * NCP;    // epilogue threads: 2 tiles x 4 lane quarters x NCP parts
+constexpr int RTHREADS = REPI + 64;   // + the TMA producer and the MMA issuer warps
 constexpr int WPROD = REPI / 32, WMMA = WPROD + 1;
 
 // n / d for 0 <= n < 2^31 as one widening multiply and a shift: l = ceil(log2 d),
@@ -76,10 +82,11 @@ struct RotParams {
 };
 
 struct RSmem {
-  static constexpr uint32_t X = 0;                 // 2 stages x [2 tiles][2 K atoms][128 rows][128 B]
-  static constexpr uint32_t R = 2 * 65536;         // 2 rotations x [2 N atoms][128 d rows][128 B]
-  static constexpr uint32_t RED = R + 2 * 32768;  // [2 items][2 tiles][8 warps][32 lanes] group maxima
-  static constexpr uint32_t BAR = RED + 4096;
+  static constexpr uint32_t X = 0;               // 2 stages x [2 tiles][2 K atoms][128 rows][128 B]
+  static constexpr uint32_t R = 2 * 65536;       // the current rotation: [2 N atoms][128 d rows][128 B]
+  static constexpr uint32_t C = R + 32768;       // E4M3 codes: [2 tiles][128 rows][128 B], 128B-swizzled
+  static constexpr uint32_t RED = C + 32768;     // [2 items][epilogue warps][32 lanes] group maxima
+  static constexpr uint32_t BAR = RED + 2 * REPI * 4;
   static constexpr uint32_t TOTAL = BAR + 256;
   static constexpr uint32_t ALLOC = TOTAL + 1024;
   static_assert(ALLOC <= 227 * 1024, "shared memory per CTA");
@@ -87,13 +94,15 @@ struct RSmem {
 
 enum {
   RB_XF = 0,    // [2] input stage full (TMA)
-  RB_XE = 2,    // [2] input stage free (the 8 epilogue warps)
+  RB_XE = 2,    // [2] input stage free (every epilogue warp)
   RB_TF = 4,    // [2] TMEM buffer full (MMA commit)
-  RB_TE = 6,    // [2] TMEM buffer free (the 8 epilogue warps)
-  RB_RF = 8,    // rotations loaded
-  RB_RM = 9,    // group maxima written (256 epilogue threads)
-  RB_FIN = 10,  // every MMA complete
-  RB_COUNT = 11
+  RB_TE = 6,    // [2] TMEM buffer free (every epilogue warp)
+  RB_RF = 8,    // rotation loaded (TMA)
+  RB_RE = 9,    // rotation free (MMA commit after its last use)
+  RB_RM = 10,   // group maxima written (every epilogue thread)
+  RB_CW = 11,   // [2] a tile's codes staged (the tile's 8 epilogue warps)
+  RB_FIN = 13,  // every MMA complete
+  RB_COUNT = 14
 };
 
 __device__ __forceinline__ uint32_t e4m3x4(float a, float b, float c, float d) {
@@ -130,6 +139,16 @@ __device__ __noinline__ uint4 codes_ieee(uint4 a, uint4 b, float sc) {
   return make_uint4(w[0], w[1], w[2], w[3]);
 }
 
+__device__ __forceinline__ void tma_store_4d(const CUtensorMap* map, const void* src, int c0, int c1, int c2, int c3) {
+  asm volatile("cp.async.bulk.tensor.4d.global.shared::cta.bulk_group [%0, {%2, %3, %4, %5}], [%1];" ::"l"(map),
+               "r"(smem_u32(src)), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// this thread's bulk stores have finished reading shared memory / have completed
+__device__ __forceinline__ void bulk_wait_read_all() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
 struct RItem {
   int oi, b, h, t0, ntile;
 };
@@ -163,6 +182,53 @@ __device__ __forceinline__ RItem decode_item(const RotParams& prm, long long g) 
   return it;
 }
 
+// One row's part: its block's scale from the exchanged group maxima (rd), the scale itself
+// (written by the block's first row), and the row part's E4M3 codes into the staging tile
+// (128B-swizzled rows, as the TMA store reads them).
+__device__ __forceinline__ void stage_codes(const RotOp& op, const RItem& it, const float* rd, int u, int part,
+                                            int quarter, int lane, int i, int t, const uint32_t (&v)[CW / 2],
+                                            uint8_t* ctile) {
+  const int r_in = u * 128 + i;  // row within the chunk
+  float m = 0.0f;
+  if (op.blk <= 32) {
+#pragma unroll
+    for (int p = 0; p < NCP; ++p) m = fmaxf(m, rd[((u * NCP + p) * 4 + quarter) * 32 + lane]);
+  } else {
+    const int g0 = (r_in & ~(op.blk - 1)) >> 5;  // first 32-row group of the block
+    for (int gq = g0; gq < g0 + (op.blk >> 5); ++gq) {
+      const int uu = gq >> 2, qq = gq & 3;
+#pragma unroll
+      for (int p = 0; p < NCP; ++p) m = fmaxf(m, rd[((uu * NCP + p) * 4 + qq) * 32]);
+    }
+  }
+  const float sc = __fdiv_rn(m, 448.0f);
+  if (part == 0 && (r_in & (op.blk - 1)) == 0) {
+    const int nblk = (op.S + op.blk - 1) >> op.lblk;
+    op.scales[((long long)it.b * op.H + it.h) * nblk + (t >> op.lblk)] = sc;
+  }
+  if (sc >= kFastDivMin) {
+    const float rc = __frcp_rn(sc);
+#pragma unroll
+    for (int q = 0; q < CW / 16; ++q) {
+      uint32_t w[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const uint32_t p0 = v[8 * q + 2 * e], p1 = v[8 * q + 2 * e + 1];
+        w[e] = e4m3x4(fp8_div(__uint_as_float(p0 << 16), sc, rc), fp8_div(__uint_as_float(p0 & 0xFFFF0000u), sc, rc),
+                      fp8_div(__uint_as_float(p1 << 16), sc, rc), fp8_div(__uint_as_float(p1 & 0xFFFF0000u), sc, rc));
+      }
+      *reinterpret_cast<uint4*>(ctile + swz128_offset(i, part * (CW / 16) + q)) = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+  } else {
+    // tiny or zero scale: IEEE division, out of line (rare)
+#pragma unroll
+    for (int q = 0; q < CW / 16; ++q)
+      *reinterpret_cast<uint4*>(ctile + swz128_offset(i, part * (CW / 16) + q)) =
+          codes_ieee(make_uint4(v[8 * q], v[8 * q + 1], v[8 * q + 2], v[8 * q + 3]),
+                     make_uint4(v[8 * q + 4], v[8 * q + 5], v[8 * q + 6], v[8 * q + 7]), sc);
+  }
+}
+
 // Persistent: one CTA per SM walks work items g = blockIdx.x, blockIdx.x + gridDim.x, ...
 // (operand, batch, head, 256-token chunk).  The producer loads item k + 1's tiles into the other
 // input stage and the MMA thread rotates it into the other TMEM buffer while the epilogue warps
@@ -170,7 +236,9 @@ __device__ __forceinline__ RItem decode_item(const RotParams& prm, long long g) 
 __global__ void __launch_bounds__(RTHREADS, 1)
     rotate_block_quant_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtensorMap mk,
                               const __grid_constant__ CUtensorMap mv, const __grid_constant__ CUtensorMap mrq,
-                              const __grid_constant__ CUtensorMap mrk, const RotParams prm) {
+                              const __grid_constant__ CUtensorMap mrk, const __grid_constant__ CUtensorMap mcq,
+                              const __grid_constant__ CUtensorMap mck, const __grid_constant__ CUtensorMap mcv,
+                              const RotParams prm) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bar = reinterpret_cast<uint64_t*>(smem + RSmem::BAR);
@@ -180,8 +248,6 @@ __global__ void __launch_bounds__(RTHREADS, 1)
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const long long G = gridDim.x;
-  int nrot = 0;  // operands with a rotation (they come first: Q, then K)
-  for (int i = 0; i < prm.nops; ++i) nrot += prm.op[i].rotate;
 
   if (tid == 0) {
     for (int i = 0; i < 2; ++i) {
@@ -191,7 +257,10 @@ __global__ void __launch_bounds__(RTHREADS, 1)
       mbar_init(&bar[RB_TE + i], REPI / 32);
     }
     mbar_init(&bar[RB_RF], 1);
+    mbar_init(&bar[RB_RE], 1);
     mbar_init(&bar[RB_RM], REPI);
+    mbar_init(&bar[RB_CW], REPI / 64);
+    mbar_init(&bar[RB_CW + 1], REPI / 64);
     mbar_init(&bar[RB_FIN], 1);
     *abort_flag = 0;
     fence_barrier_init();
@@ -207,18 +276,23 @@ __global__ void __launch_bounds__(RTHREADS, 1)
   if (warp == WPROD) {
     // ------------------------------------------------------------- producer
     if (lane == 0) {
-      if (nrot > 0) {
-        mbar_arrive_expect_tx(&bar[RB_RF], nrot * 32768);
-        for (int r = 0; r < nrot; ++r)
-          for (int nb = 0; nb < 2; ++nb)
-            tma_load_4d(smem + RSmem::R + r * 32768 + nb * 16384, r == 0 ? &mrq : &mrk, &bar[RB_RF], nb * 64, 0, 0, 0);
-      }
       long long k = 0;
+      int rload = 0, rop = -1;  // rotations loaded so far; the operand whose rotation is resident
       for (long long g = blockIdx.x; g < prm.items; g += G, ++k) {
         const int st = (int)(k & 1);
         if (k >= 2 && !mbar_wait(&bar[RB_XE + st], (uint32_t)(((k >> 1) - 1) & 1), abort_flag, prm.status, 45)) break;
         const RItem it = decode_item(prm, g);
         const RotOp& op = prm.op[it.oi];
+        if (op.rotate && it.oi != rop) {
+          // a CTA meets its items in operand order, so each rotation is loaded once; the next
+          // one waits until the MMAs that read the previous one have completed
+          if (rload > 0 && !mbar_wait(&bar[RB_RE], (uint32_t)((rload - 1) & 1), abort_flag, prm.status, 49)) break;
+          mbar_arrive_expect_tx(&bar[RB_RF], 32768);
+          for (int nb = 0; nb < 2; ++nb)
+            tma_load_4d(smem + RSmem::R + nb * 16384, it.oi == 0 ? &mrq : &mrk, &bar[RB_RF], nb * 64, 0, 0, 0);
+          ++rload;
+          rop = it.oi;
+        }
         const CUtensorMap* mx = it.oi == 0 ? &mq : (it.oi == 1 ? &mk : &mv);
         const bool bnsd = op.layout == FA_LAYOUT_BNSD;
         mbar_arrive_expect_tx(&bar[RB_XF + st], it.ntile * 2 * 16384);
@@ -231,7 +305,7 @@ __global__ void __launch_bounds__(RTHREADS, 1)
       }
       if (*abort_flag) {
         // let loads already issued land before the CTA can exit
-        if (nrot > 0) mbar_wait(&bar[RB_RF], 0, abort_flag, nullptr, 0);
+        if (rload > 0) mbar_wait(&bar[RB_RF], (uint32_t)((rload - 1) & 1), abort_flag, nullptr, 0);
         for (long long t = (k >= 2 ? k - 2 : 0); t < k; ++t)
           mbar_wait(&bar[RB_XF + (t & 1)], (uint32_t)((t >> 1) & 1), abort_flag, nullptr, 0);
       }
@@ -241,19 +315,25 @@ __global__ void __launch_bounds__(RTHREADS, 1)
     // ----------------------------------------------------------- MMA issuer
     if (lane == 0) {
       constexpr uint32_t idesc = make_idesc(kAccF32, kFmtBF16, kFmtBF16, 0, 1, 128, 128);
-      bool ok = nrot == 0 || mbar_wait(&bar[RB_RF], 0, abort_flag, prm.status, 46);
       long long k = 0;
       int tuse0 = 0, tuse1 = 0;  // rotate items so far per TMEM buffer
-      for (long long g = blockIdx.x; ok && g < prm.items; g += G, ++k) {
+      int rwait = 0, rop = -1;   // rotations waited for; the operand whose rotation is resident
+      for (long long g = blockIdx.x; g < prm.items; g += G, ++k) {
         const RItem it = decode_item(prm, g);
         const RotOp& op = prm.op[it.oi];
         if (!op.rotate) continue;
+        if (it.oi != rop) {
+          if (rop >= 0) mma_commit(&bar[RB_RE]);  // fires once the previous rotation's MMAs complete
+          if (!mbar_wait(&bar[RB_RF], (uint32_t)(rwait & 1), abort_flag, prm.status, 46)) break;
+          ++rwait;
+          rop = it.oi;
+        }
         const int st = (int)(k & 1), tb = (int)(k & 1);
         if (!mbar_wait(&bar[RB_XF + st], (uint32_t)((k >> 1) & 1), abort_flag, prm.status, 47)) break;
         const int tu = tb ? tuse1 : tuse0;
         if (tu > 0 && !mbar_wait(&bar[RB_TE + tb], (uint32_t)((tu - 1) & 1), abort_flag, prm.status, 48)) break;
         tc_fence_after();
-        const uint32_t sR = smem_u32(smem + RSmem::R + it.oi * 32768);
+        const uint32_t sR = smem_u32(smem + RSmem::R);
         for (int u = 0; u < it.ntile; ++u) {
           const uint32_t sX = smem_u32(smem + RSmem::X + st * 65536 + u * 2 * 16384);
 #pragma unroll
@@ -272,21 +352,24 @@ __global__ void __launch_bounds__(RTHREADS, 1)
     __syncwarp();
   } else {
     // -------------------------------------------------------------- epilogue
-    // warp e: tile u = e / 8, column half (e / 4) % 2, TMEM lane quarter e % 4
-    const int u = warp >> 3, half = (warp >> 2) & 1, quarter = warp & 3;
+    // warp e: tile u = e / (4 NCP), column part p = (e / 4) % NCP, TMEM lane quarter e % 4
+    const int u = warp / (4 * NCP), part = (warp >> 2) % NCP, quarter = warp & 3;
     const int i = quarter * 32 + lane;  // row within the 128-token tile
     const uint32_t loff = (uint32_t)(quarter * 32) << 16;
+    // lane 0 of each tile's first warp stores the tile's staged codes with TMA
+    const bool issuer = part == 0 && quarter == 0 && lane == 0;
     bool ok = true;
     long long k = 0;
     int tuse0 = 0, tuse1 = 0;  // rotate items so far per TMEM buffer
+    int cw = 0;                // this tile's staged-code phases so far
     for (long long g = blockIdx.x; ok && g < prm.items; g += G, ++k) {
       const RItem it = decode_item(prm, g);
       const RotOp& op = prm.op[it.oi];
       const int st = (int)(k & 1);
       const bool bnsd = op.layout == FA_LAYOUT_BNSD;
       const bool tile_live = u < it.ntile;  // warp-uniform
-      // 64 elements (half a row) as 32 packed bf16x2
-      uint32_t v[32];
+      // CW elements of the row as packed bf16x2
+      uint32_t v[CW / 2];
       if (op.rotate) {
         const int tb = (int)(k & 1);
         const int tu = tb ? tuse1 : tuse0;
@@ -296,12 +379,12 @@ __global__ void __launch_bounds__(RTHREADS, 1)
         tc_fence_after();
         if (tile_live) {  // TMEM loads are warp-collective
 #pragma unroll
-          for (int c = 0; c < 2; ++c) {
-            uint32_t r[32];
-            tmem_ld32(tbase + tb * 256 + u * 128 + loff + half * 64 + c * 32, r);
+          for (int c = 0; c < CW / 16; ++c) {
+            uint32_t r[16];
+            tmem_ld16(tbase + tb * 256 + u * 128 + loff + part * CW + c * 16, r);
             tmem_ld_wait();
 #pragma unroll
-            for (int q = 0; q < 16; ++q) v[c * 16 + q] = bf16x2_rn(__uint_as_float(r[2 * q]), __uint_as_float(r[2 * q + 1]));
+            for (int q = 0; q < 8; ++q) v[c * 8 + q] = bf16x2_rn(__uint_as_float(r[2 * q]), __uint_as_float(r[2 * q + 1]));
           }
         }
         tc_fence_before();
@@ -314,10 +397,13 @@ __global__ void __launch_bounds__(RTHREADS, 1)
         ok = __all_sync(0xffffffffu, mbar_wait(&bar[RB_XF + st], (uint32_t)((k >> 1) & 1), abort_flag, prm.status, 42));
         if (!ok) break;
         if (tile_live) {
+          // column c of the row sits in K atom c / 64, 16-byte chunk (c % 64) / 8
+          const int c0 = part * CW;
 #pragma unroll
-          for (int q = 0; q < 8; ++q) {
-            const uint4 x = *reinterpret_cast<const uint4*>(smem + RSmem::X + st * 65536 + (u * 2 + half) * 16384 +
-                                                             swz128_offset(i, q));
+          for (int q = 0; q < CW / 8; ++q) {
+            const int c = c0 + q * 8;
+            const uint4 x = *reinterpret_cast<const uint4*>(smem + RSmem::X + st * 65536 + (u * 2 + (c >> 6)) * 16384 +
+                                                             swz128_offset(i, (c & 63) >> 3));
             v[4 * q] = x.x; v[4 * q + 1] = x.y; v[4 * q + 2] = x.z; v[4 * q + 3] = x.w;
           }
         }
@@ -325,9 +411,9 @@ __global__ void __launch_bounds__(RTHREADS, 1)
         if (lane == 0) mbar_arrive(&bar[RB_XE + st]);
       }
       // Block maxima.  blk divides 256, so it is a power of two: a block is either a group of
-      // blk <= 32 adjacent lanes of one warp (its two column halves in warps e and e ^ 4) or
-      // blk / 32 whole row quarters, both halves.  Butterflies over the group's lanes leave
-      // every lane with its group's maximum; one shared exchange, double-buffered by item
+      // blk <= 32 adjacent lanes of one warp (its NCP column parts in warps of the same tile and
+      // quarter) or blk / 32 whole row quarters, every part.  Butterflies over the group's lanes
+      // leave every lane with its group's maximum; one shared exchange, double-buffered by item
       // parity so a single barrier per item suffices, combines the rest.
       const int t = it.t0 + u * 128 + i;
       const bool live = tile_live && t < op.S;
@@ -335,64 +421,44 @@ __global__ void __launch_bounds__(RTHREADS, 1)
       if (live) {
         uint32_t m2 = 0;  // running max of |x| as packed bf16x2 (signs garbage until masked)
 #pragma unroll
-        for (int q = 0; q < 32; ++q) m2 = bf16x2_absmax(m2, v[q]);
+        for (int q = 0; q < CW / 2; ++q) m2 = bf16x2_absmax(m2, v[q]);
         m2 &= 0x7FFF7FFFu;
         am = fmaxf(__uint_as_float(m2 << 16), __uint_as_float(m2 & 0xFFFF0000u));
       }
       const long long ridx = bnsd ? (((long long)it.b * op.H + it.h) * op.S + t) : (((long long)it.b * op.S + t) * op.H + it.h);
       if (live && op.dbg) {
-        uint4* d = reinterpret_cast<uint4*>(op.dbg + ridx * 128 + half * 64);
+        uint4* d = reinterpret_cast<uint4*>(op.dbg + ridx * 128 + part * CW);
 #pragma unroll
-        for (int q = 0; q < 8; ++q) d[q] = make_uint4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+        for (int q = 0; q < CW / 8; ++q) d[q] = make_uint4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
       }
       const int gl = op.blk < 32 ? op.blk : 32;
       for (int off = 1; off < gl; off <<= 1) am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, off));
-      float* rd = red + (k & 1) * 512;  // [16 warps][32 lanes]
+      float* rd = red + (k & 1) * REPI;  // [epilogue warps][32 lanes]
       rd[warp * 32 + lane] = am;
+      // the previous item's code stores must have read the staging tile before it is rewritten;
+      // the barrier below passes that on to every epilogue thread
+      if (issuer) bulk_wait_read_all();
       mbar_arrive(&bar[RB_RM]);
       ok = __all_sync(0xffffffffu, mbar_wait(&bar[RB_RM], (uint32_t)(k & 1), abort_flag, prm.status, 43));
       if (!ok) break;
-      if (!live) continue;
-      const int r_in = u * 128 + i;  // row within the chunk
-      float m;
-      if (op.blk <= 32) {
-        m = fmaxf(rd[(u * 8 + quarter) * 32 + lane], rd[(u * 8 + quarter + 4) * 32 + lane]);
-      } else {
-        m = 0.0f;
-        const int g0 = (r_in & ~(op.blk - 1)) >> 5;  // first 32-row group of the block
-        for (int gq = g0; gq < g0 + (op.blk >> 5); ++gq) {
-          const int uu = gq >> 2, qq = gq & 3;
-          m = fmaxf(m, fmaxf(rd[(uu * 8 + qq) * 32], rd[(uu * 8 + qq + 4) * 32]));
+      if (!tile_live) continue;
+      if (live) stage_codes(op, it, rd, u, part, quarter, lane, i, t, v, smem + RSmem::C + u * 16384);
+      fence_async_smem();  // this thread's staged codes -> visible to the TMA store
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bar[RB_CW + u]);
+      if (issuer) {
+        ok = mbar_wait(&bar[RB_CW + u], (uint32_t)(cw & 1), abort_flag, prm.status, 44);
+        if (ok) {
+          const int tt = it.t0 + u * 128;
+          tma_store_4d(it.oi == 0 ? &mcq : (it.oi == 1 ? &mck : &mcv), smem + RSmem::C + u * 16384, 0,
+                       bnsd ? tt : it.h, bnsd ? it.h : tt, it.b);
+          bulk_commit();
         }
       }
-      const float sc = __fdiv_rn(m, 448.0f);
-      if (half == 0 && (r_in & (op.blk - 1)) == 0) {
-        const int nblk = (op.S + op.blk - 1) >> op.lblk;
-        op.scales[((long long)it.b * op.H + it.h) * nblk + (t >> op.lblk)] = sc;
-      }
-      // codes: this thread's 64 values
-      uint4* crow = reinterpret_cast<uint4*>(static_cast<uint8_t*>(op.codes) + ridx * 128 + half * 64);
-      if (sc >= kFastDivMin) {
-        const float rc = __frcp_rn(sc);
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          uint32_t w[4];
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const uint32_t p0 = v[8 * q + 2 * e], p1 = v[8 * q + 2 * e + 1];
-            w[e] = e4m3x4(fp8_div(__uint_as_float(p0 << 16), sc, rc), fp8_div(__uint_as_float(p0 & 0xFFFF0000u), sc, rc),
-                          fp8_div(__uint_as_float(p1 << 16), sc, rc), fp8_div(__uint_as_float(p1 & 0xFFFF0000u), sc, rc));
-          }
-          crow[q] = make_uint4(w[0], w[1], w[2], w[3]);
-        }
-      } else {
-        // tiny or zero scale: IEEE division, out of line (rare)
-#pragma unroll
-        for (int q = 0; q < 4; ++q)
-          crow[q] = codes_ieee(make_uint4(v[8 * q], v[8 * q + 1], v[8 * q + 2], v[8 * q + 3]),
-                               make_uint4(v[8 * q + 4], v[8 * q + 5], v[8 * q + 6], v[8 * q + 7]), sc);
-      }
+      ++cw;
+      ok = __all_sync(0xffffffffu, ok);
     }
+    if (issuer) bulk_wait_all();
   }
 
   tc_fence_before();
@@ -401,6 +467,27 @@ __global__ void __launch_bounds__(RTHREADS, 1)
     tc_fence_after();
     tmem_dealloc(tbase, 512);
   }
+}
+
+// E4M3 codes [.., D = 128] as a 4D u8 map in the operand's layout, one 128-token box (128B-swizzled).
+cudaError_t make_code_map(CUtensorMap* map, void* base, int B, int H, int S, int layout) {
+  EncodeTiledFn enc = encode_tiled_fn();
+  if (!enc) return cudaErrorNotSupported;
+  const int D = 128;
+  cuuint64_t dims[4], strides[3];
+  cuuint32_t box[4], es[4] = {1, 1, 1, 1};
+  if (layout == FA_LAYOUT_BNSD) {
+    dims[0] = D; dims[1] = S; dims[2] = H; dims[3] = B;
+    strides[0] = (cuuint64_t)D; strides[1] = (cuuint64_t)S * D; strides[2] = (cuuint64_t)H * S * D;
+    box[0] = 128; box[1] = 128; box[2] = 1; box[3] = 1;
+  } else {
+    dims[0] = D; dims[1] = H; dims[2] = S; dims[3] = B;
+    strides[0] = (cuuint64_t)D; strides[1] = (cuuint64_t)H * D; strides[2] = (cuuint64_t)S * H * D;
+    box[0] = 128; box[1] = 1; box[2] = 128; box[3] = 1;
+  }
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 4, base, dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                   CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
 cudaError_t make_bf16_map(CUtensorMap* map, const void* base, int B, int H, int S, int layout) {
@@ -441,9 +528,10 @@ cudaError_t make_rot_map(CUtensorMap* map, const void* R) {
 cudaError_t launch_rotate_block_quant(const RotateOperand* ops, int nops, int* status, cudaStream_t s) {
   RotParams prm = {};
   prm.status = status;
-  CUtensorMap maps[3], rmaps[2];
+  CUtensorMap maps[3], rmaps[2], cmaps[3];
   memset(maps, 0, sizeof maps);
   memset(rmaps, 0, sizeof rmaps);
+  memset(cmaps, 0, sizeof cmaps);
   long long total = 0;
   int n = 0;
   for (int i = 0; i < nops; ++i) {
@@ -466,6 +554,8 @@ cudaError_t launch_rotate_block_quant(const RotateOperand* ops, int nops, int* s
     total += (long long)o.B * o.H * r.chunks;
     cudaError_t e = make_bf16_map(&maps[n], o.x, o.B, o.H, o.S, o.layout);
     if (e != cudaSuccess) return e;
+    e = make_code_map(&cmaps[n], o.codes, o.B, o.H, o.S, o.layout);
+    if (e != cudaSuccess) return e;
     if (r.rotate) {
       // Q and K each bring their own rotation; slot by operand position.
       e = make_rot_map(&rmaps[n < 2 ? n : 1], o.R);
@@ -477,9 +567,6 @@ cudaError_t launch_rotate_block_quant(const RotateOperand* ops, int nops, int* s
   prm.items = total;
   if (n == 0) return cudaSuccess;
   if (total > 0x7FFFFFFFLL) return cudaErrorInvalidValue;  // item indices stay below 2^31
-  // the operands with a rotation come first (their rotations occupy shared-memory slots 0, 1)
-  for (int i = 1; i < n; ++i)
-    if (prm.op[i].rotate && !prm.op[i - 1].rotate) return cudaErrorNotSupported;
   static bool attr = false;
   if (!attr) {
     cudaError_t e = cudaFuncSetAttribute(rotate_block_quant_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -488,8 +575,8 @@ cudaError_t launch_rotate_block_quant(const RotateOperand* ops, int nops, int* s
     attr = true;
   }
   const long long grid = total < sm_count() ? total : sm_count();
-  rotate_block_quant_kernel<<<(unsigned)grid, RTHREADS, RSmem::ALLOC, s>>>(maps[0], maps[1], maps[2], rmaps[0],
-                                                                           rmaps[1], prm);
+  rotate_block_quant_kernel<<<(unsigned)grid, RTHREADS, RSmem::ALLOC, s>>>(
+      maps[0], maps[1], maps[2], rmaps[0], rmaps[1], cmaps[0], cmaps[1], cmaps[2], prm);
   return cudaGetLastError();
 }
 
