@@ -85,8 +85,9 @@ struct RSmem {
   static constexpr uint32_t X = 0;               // 2 stages x [2 tiles][2 K atoms][128 rows][128 B]
   static constexpr uint32_t R = 2 * 65536;       // the current rotation: [2 N atoms][128 d rows][128 B]
   static constexpr uint32_t C = R + 32768;       // E4M3 codes: [2 tiles][128 rows][128 B], 128B-swizzled
-  static constexpr uint32_t RED = C + 32768;     // [2 items][epilogue warps][32 lanes] group maxima
-  static constexpr uint32_t BAR = RED + 2 * REPI * 4;
+  static constexpr uint32_t RED = C + 32768;     // [2 items][epilogue warps][32 lanes] lane-group maxima
+  static constexpr uint32_t GM = RED + 2 * REPI * 4;  // [2 items][8 row groups of 32][NCP parts] group maxima
+  static constexpr uint32_t BAR = GM + 2 * 8 * NCP * 4;
   static constexpr uint32_t TOTAL = BAR + 256;
   static constexpr uint32_t ALLOC = TOTAL + 1024;
   static_assert(ALLOC <= 227 * 1024, "shared memory per CTA");
@@ -99,10 +100,17 @@ enum {
   RB_TE = 6,    // [2] TMEM buffer free (every epilogue warp)
   RB_RF = 8,    // rotation loaded (TMA)
   RB_RE = 9,    // rotation free (MMA commit after its last use)
-  RB_RM = 10,   // group maxima written (every epilogue thread)
-  RB_CW = 11,   // [2] a tile's codes staged (the tile's 8 epilogue warps)
-  RB_FIN = 13,  // every MMA complete
-  RB_COUNT = 14
+  RB_FIN = 10,  // every MMA complete
+  RB_COUNT = 11
+};
+
+// Hardware named barriers among the epilogue warps (0 is __syncthreads).  Every epilogue warp
+// reaches each of them once per item, whatever happened before (their mbarrier waits are bounded
+// and a failed one only marks the warp), and the decision to stop is the barrier's own OR
+// reduction, identical in every warp; so no warp can be left waiting at one.
+enum {
+  NB_MAX = 1,   // group maxima written (every epilogue thread)
+  NB_CODE = 2   // [2] a tile's codes staged (its 8 warps)
 };
 
 __device__ __forceinline__ uint32_t e4m3x4(float a, float b, float c, float d) {
@@ -149,6 +157,25 @@ __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.comm
 __device__ __forceinline__ void bulk_wait_read_all() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
 __device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
+// bar.red.or over `count` threads at named barrier `id`: true in every thread when any
+// participant passed true.
+__device__ __forceinline__ bool named_barrier_or(int id, int count, bool pred) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.or.pred q, %2, %3, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)pred), "r"(id), "r"(count)
+      : "memory");
+  return r != 0;
+}
+
+__device__ __forceinline__ void named_barrier_sync(int id, int count) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
 struct RItem {
   int oi, b, h, t0, ntile;
 };
@@ -185,21 +212,24 @@ __device__ __forceinline__ RItem decode_item(const RotParams& prm, long long g) 
 // One row's part: its block's scale from the exchanged group maxima (rd), the scale itself
 // (written by the block's first row), and the row part's E4M3 codes into the staging tile
 // (128B-swizzled rows, as the TMA store reads them).
-__device__ __forceinline__ void stage_codes(const RotOp& op, const RItem& it, const float* rd, int u, int part,
-                                            int quarter, int lane, int i, int t, const uint32_t (&v)[CW / 2],
-                                            uint8_t* ctile) {
+__device__ __forceinline__ float max4(float4 a) { return fmaxf(fmaxf(a.x, a.y), fmaxf(a.z, a.w)); }
+
+__device__ __forceinline__ void stage_codes(const RotOp& op, const RItem& it, const float* rd, const float* gm, int u,
+                                            int part, int quarter, int lane, int i, int t,
+                                            const uint32_t (&v)[CW / 2], uint8_t* ctile) {
+  static_assert(NCP == 2, "the group-max gather below reads 2 parts per 32-row group");
   const int r_in = u * 128 + i;  // row within the chunk
-  float m = 0.0f;
-  if (op.blk <= 32) {
-#pragma unroll
-    for (int p = 0; p < NCP; ++p) m = fmaxf(m, rd[((u * NCP + p) * 4 + quarter) * 32 + lane]);
+  float m;
+  if (op.blk < 32) {
+    m = fmaxf(rd[((u * NCP + 0) * 4 + quarter) * 32 + lane], rd[((u * NCP + 1) * 4 + quarter) * 32 + lane]);
   } else {
-    const int g0 = (r_in & ~(op.blk - 1)) >> 5;  // first 32-row group of the block
-    for (int gq = g0; gq < g0 + (op.blk >> 5); ++gq) {
-      const int uu = gq >> 2, qq = gq & 3;
-#pragma unroll
-      for (int p = 0; p < NCP; ++p) m = fmaxf(m, rd[((uu * NCP + p) * 4 + qq) * 32]);
-    }
+    // the block's 32-row groups are contiguous in gm: blk / 16 values from group (r_in / blk) * (blk / 32)
+    const float* gp = gm + ((r_in & ~(op.blk - 1)) >> 5) * NCP;
+    const float4* g4 = reinterpret_cast<const float4*>(gp);
+    if (op.lblk == 5) m = fmaxf(gp[0], gp[1]);
+    else if (op.lblk == 6) m = max4(g4[0]);
+    else if (op.lblk == 7) m = fmaxf(max4(g4[0]), max4(g4[1]));
+    else m = fmaxf(fmaxf(max4(g4[0]), max4(g4[1])), fmaxf(max4(g4[2]), max4(g4[3])));
   }
   const float sc = __fdiv_rn(m, 448.0f);
   if (part == 0 && (r_in & (op.blk - 1)) == 0) {
@@ -245,6 +275,7 @@ __global__ void __launch_bounds__(RTHREADS, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar + RB_COUNT);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(bar + RB_COUNT + 1);
   float* red = reinterpret_cast<float*>(smem + RSmem::RED);
+  float* gmax = reinterpret_cast<float*>(smem + RSmem::GM);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const long long G = gridDim.x;
@@ -258,9 +289,6 @@ __global__ void __launch_bounds__(RTHREADS, 1)
     }
     mbar_init(&bar[RB_RF], 1);
     mbar_init(&bar[RB_RE], 1);
-    mbar_init(&bar[RB_RM], REPI);
-    mbar_init(&bar[RB_CW], REPI / 64);
-    mbar_init(&bar[RB_CW + 1], REPI / 64);
     mbar_init(&bar[RB_FIN], 1);
     *abort_flag = 0;
     fence_barrier_init();
@@ -358,11 +386,9 @@ __global__ void __launch_bounds__(RTHREADS, 1)
     const uint32_t loff = (uint32_t)(quarter * 32) << 16;
     // lane 0 of each tile's first warp stores the tile's staged codes with TMA
     const bool issuer = part == 0 && quarter == 0 && lane == 0;
-    bool ok = true;
     long long k = 0;
     int tuse0 = 0, tuse1 = 0;  // rotate items so far per TMEM buffer
-    int cw = 0;                // this tile's staged-code phases so far
-    for (long long g = blockIdx.x; ok && g < prm.items; g += G, ++k) {
+    for (long long g = blockIdx.x; g < prm.items; g += G, ++k) {
       const RItem it = decode_item(prm, g);
       const RotOp& op = prm.op[it.oi];
       const int st = (int)(k & 1);
@@ -370,53 +396,57 @@ __global__ void __launch_bounds__(RTHREADS, 1)
       const bool tile_live = u < it.ntile;  // warp-uniform
       // CW elements of the row as packed bf16x2
       uint32_t v[CW / 2];
+      bool wok;  // this warp's wait succeeded (else the item is abandoned at the next barrier)
       if (op.rotate) {
         const int tb = (int)(k & 1);
         const int tu = tb ? tuse1 : tuse0;
-        ok = __all_sync(0xffffffffu, mbar_wait(&bar[RB_TF + tb], (uint32_t)(tu & 1), abort_flag, prm.status, 41));
+        wok = __all_sync(0xffffffffu, mbar_wait(&bar[RB_TF + tb], (uint32_t)(tu & 1), abort_flag, prm.status, 41));
         if (tb) ++tuse1; else ++tuse0;
-        if (!ok) break;
-        tc_fence_after();
-        if (tile_live) {  // TMEM loads are warp-collective
+        if (wok) {
+          tc_fence_after();
+          if (tile_live) {  // TMEM loads are warp-collective
 #pragma unroll
-          for (int c = 0; c < CW / 16; ++c) {
-            uint32_t r[16];
-            tmem_ld16(tbase + tb * 256 + u * 128 + loff + part * CW + c * 16, r);
-            tmem_ld_wait();
+            for (int c = 0; c < CW / 16; ++c) {
+              uint32_t r[16];
+              tmem_ld16(tbase + tb * 256 + u * 128 + loff + part * CW + c * 16, r);
+              tmem_ld_wait();
 #pragma unroll
-            for (int q = 0; q < 8; ++q) v[c * 8 + q] = bf16x2_rn(__uint_as_float(r[2 * q]), __uint_as_float(r[2 * q + 1]));
+              for (int q = 0; q < 8; ++q) v[c * 8 + q] = bf16x2_rn(__uint_as_float(r[2 * q]), __uint_as_float(r[2 * q + 1]));
+            }
           }
-        }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) {
-          mbar_arrive(&bar[RB_TE + tb]);
-          mbar_arrive(&bar[RB_XE + st]);  // the MMA that read the stage has completed
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) {
+            mbar_arrive(&bar[RB_TE + tb]);
+            mbar_arrive(&bar[RB_XE + st]);  // the MMA that read the stage has completed
+          }
         }
       } else {
-        ok = __all_sync(0xffffffffu, mbar_wait(&bar[RB_XF + st], (uint32_t)((k >> 1) & 1), abort_flag, prm.status, 42));
-        if (!ok) break;
-        if (tile_live) {
-          // column c of the row sits in K atom c / 64, 16-byte chunk (c % 64) / 8
-          const int c0 = part * CW;
+        wok = __all_sync(0xffffffffu, mbar_wait(&bar[RB_XF + st], (uint32_t)((k >> 1) & 1), abort_flag, prm.status, 42));
+        if (wok) {
+          if (tile_live) {
+            // column c of the row sits in K atom c / 64, 16-byte chunk (c % 64) / 8
+            const int c0 = part * CW;
 #pragma unroll
-          for (int q = 0; q < CW / 8; ++q) {
-            const int c = c0 + q * 8;
-            const uint4 x = *reinterpret_cast<const uint4*>(smem + RSmem::X + st * 65536 + (u * 2 + (c >> 6)) * 16384 +
-                                                             swz128_offset(i, (c & 63) >> 3));
-            v[4 * q] = x.x; v[4 * q + 1] = x.y; v[4 * q + 2] = x.z; v[4 * q + 3] = x.w;
+            for (int q = 0; q < CW / 8; ++q) {
+              const int c = c0 + q * 8;
+              const uint4 x = *reinterpret_cast<const uint4*>(smem + RSmem::X + st * 65536 + (u * 2 + (c >> 6)) * 16384 +
+                                                               swz128_offset(i, (c & 63) >> 3));
+              v[4 * q] = x.x; v[4 * q + 1] = x.y; v[4 * q + 2] = x.z; v[4 * q + 3] = x.w;
+            }
           }
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&bar[RB_XE + st]);
         }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&bar[RB_XE + st]);
       }
       // Block maxima.  blk divides 256, so it is a power of two: a block is either a group of
-      // blk <= 32 adjacent lanes of one warp (its NCP column parts in warps of the same tile and
-      // quarter) or blk / 32 whole row quarters, every part.  Butterflies over the group's lanes
-      // leave every lane with its group's maximum; one shared exchange, double-buffered by item
-      // parity so a single barrier per item suffices, combines the rest.
+      // blk < 32 adjacent lanes of one warp (its NCP column parts in warps of the same tile and
+      // quarter) or blk / 32 whole 32-row groups, every part.  Butterflies over the group's lanes
+      // leave every lane with its group's maximum; one shared exchange (per lane, or per warp
+      // into the group array), double-buffered by item parity so a single barrier per item
+      // suffices, combines the rest.
       const int t = it.t0 + u * 128 + i;
-      const bool live = tile_live && t < op.S;
+      const bool live = wok && tile_live && t < op.S;
       float am = 0.0f;
       if (live) {
         uint32_t m2 = 0;  // running max of |x| as packed bf16x2 (signs garbage until masked)
@@ -433,30 +463,24 @@ __global__ void __launch_bounds__(RTHREADS, 1)
       }
       const int gl = op.blk < 32 ? op.blk : 32;
       for (int off = 1; off < gl; off <<= 1) am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, off));
-      float* rd = red + (k & 1) * REPI;  // [epilogue warps][32 lanes]
-      rd[warp * 32 + lane] = am;
+      float* rd = red + (k & 1) * REPI;         // [epilogue warps][32 lanes]
+      float* gmx = gmax + (k & 1) * 8 * NCP;    // [32-row group][part]
+      if (op.blk < 32) rd[warp * 32 + lane] = am;
+      else if (lane == 0) gmx[(u * 4 + quarter) * NCP + part] = am;
       // the previous item's code stores must have read the staging tile before it is rewritten;
       // the barrier below passes that on to every epilogue thread
       if (issuer) bulk_wait_read_all();
-      mbar_arrive(&bar[RB_RM]);
-      ok = __all_sync(0xffffffffu, mbar_wait(&bar[RB_RM], (uint32_t)(k & 1), abort_flag, prm.status, 43));
-      if (!ok) break;
+      if (named_barrier_or(NB_MAX, REPI, !wok)) break;
       if (!tile_live) continue;
-      if (live) stage_codes(op, it, rd, u, part, quarter, lane, i, t, v, smem + RSmem::C + u * 16384);
+      if (live) stage_codes(op, it, rd, gmx, u, part, quarter, lane, i, t, v, smem + RSmem::C + u * 16384);
       fence_async_smem();  // this thread's staged codes -> visible to the TMA store
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bar[RB_CW + u]);
+      named_barrier_sync(NB_CODE + u, REPI / 2);
       if (issuer) {
-        ok = mbar_wait(&bar[RB_CW + u], (uint32_t)(cw & 1), abort_flag, prm.status, 44);
-        if (ok) {
-          const int tt = it.t0 + u * 128;
-          tma_store_4d(it.oi == 0 ? &mcq : (it.oi == 1 ? &mck : &mcv), smem + RSmem::C + u * 16384, 0,
-                       bnsd ? tt : it.h, bnsd ? it.h : tt, it.b);
-          bulk_commit();
-        }
+        const int tt = it.t0 + u * 128;
+        tma_store_4d(it.oi == 0 ? &mcq : (it.oi == 1 ? &mck : &mcv), smem + RSmem::C + u * 16384, 0,
+                     bnsd ? tt : it.h, bnsd ? it.h : tt, it.b);
+        bulk_commit();
       }
-      ++cw;
-      ok = __all_sync(0xffffffffu, ok);
     }
     if (issuer) bulk_wait_all();
   }

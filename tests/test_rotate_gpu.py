@@ -35,26 +35,32 @@ def shp(B, H, S, layout, D=128):
     return (B, H, S, D) if layout == "BNSD" else (B, S, H, D)
 
 
+def check_rotated(orc, name, x, R, got, layout, exact=False):
+    """The GPU's rotated bf16 tensor (bit patterns) against the oracle's fp64 rotation: within
+    half a bf16 ulp plus the fp32 summation bound; returns the fraction differing from the
+    oracle's own bf16 rounding (0 required when exact)."""
+    xb, Rb = wl.bf16_bits(x), wl.bf16_bits(R)
+    exact_f64 = orc.rotate_f64(xb, Rb, layout)
+    dist = ulp_diff(got, orc.f64_to_bf16(exact_f64))
+    if exact:
+        assert dist.max() == 0, name
+    absx = np.abs(orc.bf16_bits_to_f32(xb).astype(np.float64))
+    absR = np.abs(orc.bf16_bits_to_f32(Rb).astype(np.float64))
+    bound = 2.0 ** -17 * (absx @ absR)
+    half_ulp = np.ldexp(1.0, np.frexp(np.abs(exact_f64))[1] - 9)
+    err = np.abs(orc.bf16_bits_to_f32(got).astype(np.float64) - exact_f64)
+    assert (err <= bound + half_ulp + 1e-300).all(), f"{name}: rotation outside the fp32 summation bound"
+    return float((dist > 0).mean())
+
+
 def check_rotate(faq, orc, q, k, v, Rq, Rk, layout, q_blk, kv_blk, exact=False):
     Q, K, V, dq, dk = faq.rotate_quantize(q.cuda(), k.cuda(), v.cuda(), Rq.cuda(), Rk.cuda(), layout,
                                           q_blk, kv_blk, debug=True)
     faq.check_device_status()
     stats = {}
     for name, x, R, d, out, blk in (("q", q, Rq, dq, Q, q_blk), ("k", k, Rk, dk, K, kv_blk)):
-        xb, Rb = wl.bf16_bits(x), wl.bf16_bits(R)
-        exact_f64 = orc.rotate_f64(xb, Rb, layout)
-        ref = orc.f64_to_bf16(exact_f64)
         got = np_of(d)
-        dist = ulp_diff(got, ref)
-        if exact:
-            assert dist.max() == 0, name
-        absx = np.abs(orc.bf16_bits_to_f32(xb).astype(np.float64))
-        absR = np.abs(orc.bf16_bits_to_f32(Rb).astype(np.float64))
-        bound = 2.0 ** -17 * (absx @ absR)
-        half_ulp = np.ldexp(1.0, np.frexp(np.abs(exact_f64))[1] - 9)
-        err = np.abs(orc.bf16_bits_to_f32(got).astype(np.float64) - exact_f64)
-        assert (err <= bound + half_ulp + 1e-300).all(), f"{name}: rotation outside the fp32 summation bound"
-        stats[name] = float((dist > 0).mean())
+        stats[name] = check_rotated(orc, name, x, R, got, layout, exact)
         codes, scales = orc.quantize_fp8_block(got, blk, layout)
         assert np.array_equal(np_of(out.scales), scales), name
         assert np.array_equal(np_of(out.codes), codes), name
@@ -73,6 +79,40 @@ def test_rotate_block_quant(faq, orc, layout, S, q_blk, kv_blk):
     R = wl.rotation(128, 5)
     stats, _ = check_rotate(faq, orc, q, k, v, R, R, layout, q_blk, kv_blk)
     assert stats["q"] < 1e-2 and stats["k"] < 1e-2
+
+
+def test_rotate_many_items_per_cta(faq, orc):
+    """More 256-token chunks than SMs: each persistent CTA walks items of several operands
+    (Q, then K, then V), so the resident rotation is swapped mid-stream; distinct R_q and R_k
+    make a stale rotation show."""
+    B, H, S = 2, 8, 5000  # 20 chunks per (b, h): 960 items
+    q = wl.normal(shp(B, H, S, "BSND"), 31)
+    k = wl.normal(shp(B, H, S, "BSND"), 32)
+    v = wl.normal(shp(B, H, S, "BSND"), 33)
+    Rq = wl.rotation(128, 34)
+    Rk = (wl.normal((128, 128), 35).float() * 0.1).to(torch.bfloat16)
+    stats, _ = check_rotate(faq, orc, q, k, v, Rq, Rk, "BSND", 128, 256)
+    assert stats["q"] < 1e-2
+
+
+def test_rotate_key_only_through_abi(faq, orc):
+    """Only K passed through the C ABI (Q and V null): K's rotation is the first one resident."""
+    import ctypes
+    from quantized_attention_amax_b200 import _native as N, api
+    k = wl.normal((1, 700, 3, 128), 41).cuda()
+    Rk = (wl.normal((128, 128), 42).float() * 0.1).to(torch.bfloat16).cuda()
+    K = api.empty_qtensor(1, 3, 700, 128, "fp8_block", "BSND", 256, k.device)
+    tk, ck = api._tensor(k, "BSND"), K.c()
+    dk = torch.empty_like(k)
+    st = N.lib().fa_rotate_quantize(None, ctypes.byref(tk), None, None, Rk.data_ptr(), 128, 256, None,
+                                    ctypes.byref(ck), None, None, dk.data_ptr(), api._stream())
+    assert st == 0
+    faq.check_device_status()
+    got = np_of(dk)
+    check_rotated(orc, "k", k.cpu(), Rk.cpu(), got, "BSND")
+    codes, scales = orc.quantize_fp8_block(got, 256, "BSND")
+    assert np.array_equal(np_of(K.scales), scales)
+    assert np.array_equal(np_of(K.codes), codes)
 
 
 def test_rotate_general_matrix_catches_transpose(faq, orc):
