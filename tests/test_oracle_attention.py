@@ -157,3 +157,42 @@ def test_quantized_operands_dequantize_per_mode(orc):
     }
     for key, t in zip("ifmb", (qi, qf, qm, qb)):
         assert np.array_equal(orc.dequant(t), by_hand[key])
+
+
+def test_mixed_branches_are_attention_on_each_branch_dequantized(orc):
+    """fa3_quant details (FA3AttentionDetails): Q, K and V each in its own mode, an unset branch
+    left as bf16.  The oracle's attention must equal torch's fp64 SDPA (bottom-right causal mask,
+    kv heads repeated for GQA) on each branch dequantized by hand from the format tables."""
+    B, Hq, Hkv, S, D = 1, 4, 2, 48, 64
+    xq = wl.bf16_bits(wl.normal((B, Hq, S, D), 31))
+    xk = wl.bf16_bits(wl.normal((B, Hkv, S, D), 32))
+    xv = wl.bf16_bits(wl.normal((B, Hkv, S, D), 33))
+    cq, sq = orc.quantize_fp8_per_token(xq)
+    ck, sk = orc.quantize_int8_per_head(xk, orc.calibrate_per_head(xk))
+    cv, ev = orc.quantize_mxfp4(xv)
+    deq = {
+        "q": orc.e4m3_decode(cq) * sq[..., None],
+        "k": ck.astype(np.float64) * sk[None, :, None, None],
+        "v": orc.e2m1_decode(np.stack([cv & 15, cv >> 4], -1).reshape(B, Hkv, S, D))
+        * np.ldexp(1.0, np.repeat(ev.astype(np.int64) - 127, 32, -1)),
+        "vf": orc.bf16_bits_to_f32(xv).astype(np.float64),
+    }
+    Q = orc.QT("fp8_per_token", cq, sq, B, Hq, S, D)
+    K = orc.QT("int8_per_head", ck, sk, B, Hkv, S, D)
+    V = orc.QT("mxfp4", cv, ev, B, Hkv, S, D)
+    Vf = orc.qt_float(xv, "BNSD")
+
+    def sdpa(q, k, v, causal):
+        k = np.repeat(k, Hq // Hkv, 1)
+        v = np.repeat(v, Hq // Hkv, 1)
+        mask = None
+        if causal:
+            mask = torch.ones(S, S, dtype=torch.bool).tril()
+        return torch.nn.functional.scaled_dot_product_attention(
+            torch.from_numpy(q), torch.from_numpy(k), torch.from_numpy(v), attn_mask=mask).numpy()
+
+    for causal in (False, True):
+        out, _ = orc.attention(Q, K, V, causal, 0.0)
+        assert np.allclose(out, sdpa(deq["q"], deq["k"], deq["v"], causal), rtol=1e-12, atol=1e-12)
+        out, _ = orc.attention(Q, K, Vf, causal, 0.0)
+        assert np.allclose(out, sdpa(deq["q"], deq["k"], deq["vf"], causal), rtol=1e-12, atol=1e-12)
