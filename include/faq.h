@@ -181,14 +181,24 @@ FAQ_API fa_status fa_rotate_quantize(const fa_tensor* q, const fa_tensor* k, con
  *   on the low-bit operands, the output dequantized back to the original
  *   precision); FlashAttention (Dao et al. 2022), cited by the wiki's
  *   参考资料: O = softmax(Q K^T * scale) V with an online softmax.
- *   q, k, v: quantized descriptors, all the same mode and layout and D;
+ *   q, k, v: quantized descriptors of one layout and D.  Each branch has its
+ *   own mode (msModelSlim "fa3_quant 配置说明" §2.3 FA3AttentionDetails:
+ *   fa_q / fa_k / fa_v each take a QConfig; the wiki's 分支组合 note: a branch
+ *   left unset is not quantized): FA_MODE_FLOAT marks an unquantized branch,
+ *   whose `codes` is the bf16 tensor itself (scales unused).  When the three
+ *   modes differ, or any is FA_MODE_FLOAT, the call computes attention on
+ *   the dequantized operands (x = code * scale, MX: code * 2^(e - 127)):
+ *   Q and K are dequantized to bf16 in the workspace (a float branch is read
+ *   in place), V' is made from V's own mode, and QK^T runs on bf16 tensor
+ *   cores; all three FLOAT is plain bf16 attention.  A V in an MX mode needs
+ *   D == 128 there.
  *   q->B == k->B == v->B, k and v have equal dims, q->H % k->H == 0 (GQA:
  *   query head h reads kv head h / (Hq / Hkv)).  causal: key j is visible
  *   to query i iff j <= i + (Sk - Sq).  softmax_scale <= 0 means 1/sqrt(D).
  *   out: device bf16, q's layout and dims.  lse: nullable device fp32
  *   [B, Hq, Sq], natural-log sum-exp of the scaled scores (-inf for a row
  *   with no visible key, whose output is 0).
- *   workspace: device memory of at least fa_attention_workspace_size()
+ *   workspace: device memory of at least fa_attention_workspace_size_qkv()
  *   bytes, 256-byte aligned, owned by the caller and only used during the
  *   call's kernels (FA_ERR_WORKSPACE if missing, short or misaligned).
  *   Decode (q->S == 1) keeps its split-KV partials there before an LSE
@@ -279,6 +289,17 @@ FAQ_API size_t fa_decode_append_workspace_size(const fa_tensor* q, const fa_qten
  * B*Hkv*ceil(Sk/128)*512, each part rounded up to 256.  Returns 0 on
  * invalid arguments. */
 FAQ_API size_t fa_attention_workspace_size(const fa_qtensor* q, const fa_qtensor* k, int num_splits);
+
+/* The same for any three branches: equal to fa_attention_workspace_size when
+ * q, k and v share one quantized mode; with mixed branches (modes differ, or
+ * one is FA_MODE_FLOAT) the prefill parts above plus the bf16 dequantized
+ * copies of Q (B*Hq*Sq*D*2) and K (B*Hkv*Sk*D*2) that are not FA_MODE_FLOAT,
+ * each rounded up to 256.  fa_attention_workspace_size(q, k) already returns
+ * this when q and k differ in mode or one is FA_MODE_FLOAT; when only v
+ * differs it cannot know, so size mixed calls with this function.  Returns 0
+ * on invalid arguments (v NULL included). */
+FAQ_API size_t fa_attention_workspace_size_qkv(const fa_qtensor* q, const fa_qtensor* k, const fa_qtensor* v,
+                                               int num_splits);
 
 /* Synchronise `s`, read and clear this device's status word.  Returns
  * FA_ERR_TIMEOUT if a kernel's bounded wait ran out since the last check,

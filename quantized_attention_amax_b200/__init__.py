@@ -7,9 +7,10 @@ operands (prefill, split-KV decode, decode with the cache append fused), all in 
 include/faq.h (libfaq.so).  This package is the thin ctypes binding.
 """
 from .api import (LAYOUTS, MODES, FaqError, QTensor, attention, attention_workspace_size, calibrate_per_head,
-                  check_device_status, decode_append, dims, empty_qtensor, quantize, resolve_config, rotate_quantize,
-                  version)
+                  check_device_status, decode_append, dims, empty_qtensor, float_branch, quantize, resolve_config,
+                  rotate_quantize, version)
 
 __all__ = ["LAYOUTS", "MODES", "FaqError", "QTensor", "attention", "attention_workspace_size",
-           "calibrate_per_head", "check_device_status", "decode_append", "dims", "empty_qtensor", "quantize",
+           "calibrate_per_head", "check_device_status", "decode_append", "dims", "empty_qtensor", "float_branch",
+           "quantize",
            "resolve_config", "rotate_quantize", "version"]

@@ -18,6 +18,7 @@ EXPORTS = (
     "fa_rotate_quantize",
     "fa_attention_quant",
     "fa_attention_workspace_size",
+    "fa_attention_workspace_size_qkv",
     "fa_attention_decode_noalloc",
     "fa_decode_append",
     "fa_decode_append_workspace_size",
@@ -69,6 +70,8 @@ def lib() -> ctypes.CDLL:
     L.fa_attention_decode_noalloc.restype = I
     L.fa_attention_workspace_size.argtypes = [pQ, pQ, I]
     L.fa_attention_workspace_size.restype = S
+    L.fa_attention_workspace_size_qkv.argtypes = [pQ, pQ, pQ, I]
+    L.fa_attention_workspace_size_qkv.restype = S
     L.fa_decode_append.argtypes = [pT, pT, pT, P, P, P, pQ, pQ, I, F, P, P, I, P, S, P]
     L.fa_decode_append.restype = I
     L.fa_decode_append_workspace_size.argtypes = [pT, pQ, I, I]

@@ -64,8 +64,17 @@ class QTensor:
     block_tokens: int = 0
 
     def c(self) -> N.FaQTensor:
-        return N.FaQTensor(self.codes.data_ptr(), self.scales.data_ptr(), MODES[self.mode], self.B, self.H,
-                           self.S, self.D, LAYOUTS[self.layout], self.block_tokens)
+        return N.FaQTensor(self.codes.data_ptr(), self.scales.data_ptr() if self.scales is not None else None,
+                           MODES[self.mode], self.B, self.H, self.S, self.D, LAYOUTS[self.layout],
+                           self.block_tokens)
+
+
+def float_branch(x: torch.Tensor, layout: str = "BNSD") -> QTensor:
+    """An unquantized branch for attention (FA_MODE_FLOAT): the bf16 tensor itself."""
+    if x.dtype != torch.bfloat16 or not x.is_cuda or not x.is_contiguous():
+        raise ValueError("expected a contiguous bf16 CUDA tensor")
+    B, H, S, D = dims(x.shape, layout)
+    return QTensor(x, None, "float", B, H, S, D, layout)
 
 
 def empty_qtensor(B: int, H: int, S: int, D: int, mode: str, layout: str = "BNSD", block_tokens: int = 0,
@@ -185,8 +194,12 @@ def rotate_quantize(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, rot_q: to
     return tuple(outs) + ((dq, dk) if debug else ())
 
 
-def attention_workspace_size(q: QTensor, k: QTensor, num_splits: int = 0) -> int:
+def attention_workspace_size(q: QTensor, k: QTensor, num_splits: int = 0, v: Optional[QTensor] = None) -> int:
     cq, ck = q.c(), k.c()
+    if v is not None:
+        cv = v.c()
+        return int(N.lib().fa_attention_workspace_size_qkv(ctypes.byref(cq), ctypes.byref(ck), ctypes.byref(cv),
+                                                           num_splits))
     return int(N.lib().fa_attention_workspace_size(ctypes.byref(cq), ctypes.byref(ck), num_splits))
 
 
@@ -194,13 +207,15 @@ def attention(q: QTensor, k: QTensor, v: QTensor, causal: bool = False, softmax_
               out: Optional[torch.Tensor] = None, return_lse: bool = False, num_splits: int = 0,
               workspace: Optional[torch.Tensor] = None):
     """Attention on quantized operands, bf16 output in q's layout
-    (fa_attention_quant).  Returns out, or (out, lse) with return_lse."""
+    (fa_attention_quant).  Each branch may have its own mode; ``float_branch``
+    wraps an unquantized one.  Returns out, or (out, lse) with return_lse."""
     dev = q.codes.device
     if out is None:
         out = torch.empty(_shape(q.B, q.H, q.S, q.D, q.layout), dtype=torch.bfloat16, device=dev)
     lse = torch.empty((q.B, q.H, q.S), dtype=torch.float32, device=dev) if return_lse else None
     cq, ck, cv = q.c(), k.c(), v.c()
-    need = int(N.lib().fa_attention_workspace_size(ctypes.byref(cq), ctypes.byref(ck), num_splits))
+    need = int(N.lib().fa_attention_workspace_size_qkv(ctypes.byref(cq), ctypes.byref(ck), ctypes.byref(cv),
+                                                       num_splits))
     if need and (workspace is None or workspace.numel() * workspace.element_size() < need):
         workspace = torch.empty(need, dtype=torch.uint8, device=dev)
     ws_ptr = workspace.data_ptr() if workspace is not None else None

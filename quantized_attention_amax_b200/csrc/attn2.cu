@@ -65,7 +65,15 @@ constexpr int NKS = 3;      // K code stages
 constexpr int NVS = 2;      // V' stages
 constexpr int NSC = 4;      // scale ring stages
 
-enum { K_E4M3 = 0, K_S8 = 1, K_MXF4 = 2, K_MXF8 = 3 };
+// per half: max(|a|, |b|), its sign the XOR of the inputs' signs (only magnitudes are used)
+__device__ __forceinline__ uint32_t bf16x2_absmax(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("max.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+
+// K_BF16: bf16 Q and K (dequantized operands of mixed branches, or unquantized ones)
+enum { K_E4M3 = 0, K_S8 = 1, K_MXF4 = 2, K_MXF8 = 3, K_BF16 = 4 };
 enum { SC_HEAD = 0, SC_COL = 1, SC_TILE = 2 };  // one scale per head / per key / per 128-key tile
 
 struct P2 {
@@ -637,11 +645,15 @@ constexpr int PR0 = 56;
 constexpr int PRS = 224;
 static_assert(128 * PR0 + 256 * PRS <= PNT * ((65536 / PNT) & ~7), "register split exceeds the launch");
 
-template <int D>
+template <int KIND, int D>
 struct LP {
-  static constexpr uint32_t Q = 0;                       // 2 x [128][D]
-  static constexpr uint32_t K = Q + 2 * BM * D;          // NKS stages
-  static constexpr uint32_t VH = K + NKS * BN * D;       // NVS stages of fp16 V'
+  static constexpr int RB = KIND == K_BF16 ? 2 * D : D;  // Q / K bytes per token row
+  static constexpr int NA = RB > 128 ? RB / 128 : 1;     // 128-byte swizzle atoms per row (bf16 at D = 128: 2)
+  static constexpr int AB = RB > 128 ? 128 : RB;         // bytes per atom row
+  static constexpr int NK = KIND == K_BF16 ? 2 : NKS;    // K stages (bf16 tiles are twice as large)
+  static constexpr uint32_t Q = 0;                       // 2 x NA x [128][AB]
+  static constexpr uint32_t K = Q + 2 * BM * RB;         // NK stages
+  static constexpr uint32_t VH = K + NK * BN * RB;       // NVS stages of fp16 V'
   static constexpr uint32_t SC = VH + NVS * BN * D * 2;  // NSC stages x ([128] K scales, V' factor record)
   static constexpr uint32_t MISC = SC + NSC * 2 * BN * 4;
   static constexpr uint32_t BAR = MISC + 64;
@@ -671,9 +683,10 @@ template <int KIND, int D, int SC>
 __global__ void __launch_bounds__(PNT, 1)
     attn_pair_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
                      const __grid_constant__ CUtensorMap tmv, const P2 p) {
-  static_assert(KIND == K_E4M3 || (KIND == K_S8 && SC != SC_TILE), "E4M3 or INT8 operands");
+  static_assert(KIND == K_E4M3 || KIND == K_BF16 || (KIND == K_S8 && SC != SC_TILE), "E4M3, INT8 or bf16 operands");
   constexpr bool RING = SC != SC_HEAD;
-  using L = LP<D>;
+  using L = LP<KIND, D>;
+  constexpr int NKS = L::NK;  // K stages of this kind
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bar = reinterpret_cast<uint64_t*>(smem + L::BAR);
@@ -753,17 +766,23 @@ __global__ void __launch_bounds__(PNT, 1)
       if (lane == 0 && n > 0) {
         tma_prefetch_desc(&tmq);
         tma_prefetch_desc(&tmk);
-        mbar_arrive_expect_tx(&bar[Y_Q], ((nt[0] > 0) + (nt[1] > 0)) * BM * D);
+        mbar_arrive_expect_tx(&bar[Y_Q], ((nt[0] > 0) + (nt[1] > 0)) * BM * L::RB);
 #pragma unroll
         for (int x = 0; x < 2; ++x)
           if (nt[x] > 0)
-            tma_load_4d(smem + L::Q + x * BM * D, &tmq, &bar[Y_Q], 0, bnsd ? q0t[x] : hqt[x], bnsd ? hqt[x] : q0t[x], b);
+#pragma unroll
+            for (int a = 0; a < L::NA; ++a)
+              tma_load_4d(smem + L::Q + x * BM * L::RB + a * BM * L::AB, &tmq, &bar[Y_Q], a * L::AB,
+                          bnsd ? q0t[x] : hqt[x], bnsd ? hqt[x] : q0t[x], b);
         int j = 0;
         for (; j < n; ++j) {
           const int k0 = j * BN, ks = j % NKS;
           if (j >= NKS && !mbar_wait(&bar[Y_KE + ks], ((j / NKS) - 1) & 1, abort_flag, p.status, 81)) break;
-          mbar_arrive_expect_tx(&bar[Y_KF + ks], BN * D);
-          tma_load_4d(smem + L::K + ks * BN * D, &tmk, &bar[Y_KF + ks], 0, bnsd ? k0 : hk, bnsd ? hk : k0, b);
+          mbar_arrive_expect_tx(&bar[Y_KF + ks], BN * L::RB);
+#pragma unroll
+          for (int a = 0; a < L::NA; ++a)
+            tma_load_4d(smem + L::K + ks * BN * L::RB + a * BN * L::AB, &tmk, &bar[Y_KF + ks], a * L::AB,
+                        bnsd ? k0 : hk, bnsd ? hk : k0, b);
         }
         if (*abort_flag) {
           mbar_wait(&bar[Y_Q], 0, abort_flag, nullptr, 0);
@@ -816,20 +835,25 @@ __global__ void __launch_bounds__(PNT, 1)
     } else {
       // ---------------------------------------------------------- MMA issuer
       if (lane == 0 && n > 0) {
-        constexpr uint32_t SW = D == 128 ? kSwz128 : kSwz64;
-        constexpr uint32_t SBO8 = D == 128 ? 1024 : 512;
-        constexpr uint32_t idesc_qk = KIND == K_E4M3 ? make_idesc(kAccF32, kFmtE4M3, kFmtE4M3, 0, 0, BN, BM)
-                                                     : make_idesc(kAccS32, kFmtS8, kFmtS8, 0, 0, BN, BM);
+        constexpr uint32_t SW = L::AB == 128 ? kSwz128 : kSwz64;
+        constexpr uint32_t SBO8 = L::AB == 128 ? 1024 : 512;
+        constexpr uint32_t idesc_qk = KIND == K_E4M3   ? make_idesc(kAccF32, kFmtE4M3, kFmtE4M3, 0, 0, BN, BM)
+                                      : KIND == K_BF16 ? make_idesc(kAccF32, kFmtBF16, kFmtBF16, 0, 0, BN, BM)
+                                                       : make_idesc(kAccS32, kFmtS8, kFmtS8, 0, 0, BN, BM);
         constexpr uint32_t idesc_pv = make_idesc(kAccF32, kFmtF16, kFmtF16, 0, 1, D, BM);
         auto qk = [&](int x, int j) {
-          const uint32_t sQ = smem_u32(smem + L::Q + x * BM * D);
-          const uint32_t sK = smem_u32(smem + L::K + (j % NKS) * BN * D);
+          const uint32_t sQ = smem_u32(smem + L::Q + x * BM * L::RB);
+          const uint32_t sK = smem_u32(smem + L::K + (j % NKS) * BN * L::RB);
+          // one MMA per 32 bytes of the row (K = 32 codes, or K = 16 bf16): atom a = kk * 32 / AB
 #pragma unroll
-          for (int kk = 0; kk < D / 32; ++kk) {
-            const uint64_t da = make_sdesc(sQ + kk * 32, 16, SBO8, SW);
-            const uint64_t db = make_sdesc(sK + kk * 32, 16, SBO8, SW);
+          for (int kk = 0; kk < L::RB / 32; ++kk) {
+            const uint32_t off = (kk * 32 / L::AB) * BM * L::AB + (kk * 32) % L::AB;
+            const uint64_t da = make_sdesc(sQ + off, 16, SBO8, SW);
+            const uint64_t db = make_sdesc(sK + off, 16, SBO8, SW);
             if (KIND == K_E4M3)
               mma_f8f6f4(tbase + x * 128, da, db, idesc_qk, kk > 0);
+            else if (KIND == K_BF16)
+              mma_f16(tbase + x * 128, da, db, idesc_qk, kk > 0);
             else
               mma_i8(tbase + x * 128, da, db, idesc_qk, kk > 0);
           }
@@ -1078,7 +1102,10 @@ __global__ void __launch_bounds__(PNT, 1)
 //   the tile's per-key K scales beside it.
 // V scale per head: V' = fp16(code) exactly (the per-head scale stays outside).
 // MXFP4: E_t = the largest UE8M0 byte of the tile's tokens, V' = fp16(e2m1 * 2^(e - E_t)), |V'| <= 6.
-template <int KIND, int D, bool VSC>
+// V pre-pass: V' fp16 tiles + per-tile factor records (+ the K tile's per-key scales).  MIXED:
+// records are linear factors for every kind (the bf16 pair kernel's scale ring) and the per-key K
+// scales are 1 (Q and K arrive dequantized).
+template <int KIND, int D, bool VSC, bool MIXED = false>
 __global__ void __launch_bounds__(256) vprep_kernel(const uint8_t* __restrict__ codes, const float* __restrict__ vs,
                                                     int v_blk, int v_nblk, int H, int S, int layout,
                                                     __half* __restrict__ vh, float4* __restrict__ fvr, int ntiles,
@@ -1113,9 +1140,12 @@ __global__ void __launch_bounds__(256) vprep_kernel(const uint8_t* __restrict__ 
     }
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, off));
-    if (threadIdx.x == 0) fvr[(long long)bh * ntiles + t] = make_float4((float)m, 0.0f, 0.0f, 0.0f);
-    // the K tile's scale-factor atom: token row r at byte (r % 32) * 16 + (r / 32) * 4, zero past S
-    if (threadIdx.x < BN) {
+    if (threadIdx.x == 0)
+      fvr[(long long)bh * ntiles + t] = make_float4(MIXED ? ldexpf(1.0f, m - 127) : (float)m, 0.0f, 0.0f, 0.0f);
+    if (MIXED) {
+      if (threadIdx.x < BN) ksp[((long long)bh * ntiles + t) * BN + threadIdx.x] = tok0 + (int)threadIdx.x < S ? 1.0f : 0.0f;
+    } else if (threadIdx.x < BN) {
+      // the K tile's scale-factor atom: token row r at byte (r % 32) * 16 + (r / 32) * 4, zero past S
       const int key = tok0 + threadIdx.x;
       const uint32_t w = key < S ? __ldg(reinterpret_cast<const uint32_t*>(ke8) + (long long)bh * S + key) : 0u;
       reinterpret_cast<uint32_t*>(ksp + ((long long)bh * ntiles + t) * BN)[(threadIdx.x & 31) * 4 + (threadIdx.x >> 5)] = w;
@@ -1153,6 +1183,47 @@ __global__ void __launch_bounds__(256) vprep_kernel(const uint8_t* __restrict__ 
       }
     }
     return;
+  } else if constexpr (KIND == K_BF16) {
+    // unquantized V: V' = fp16(v / r_t), r_t the power of two that puts the tile's max |v| in
+    // [2^14, 2^15) (exact scaling; fp16 keeps 11 bits), records r_t
+    __shared__ float red[8];
+    constexpr int NC = D / 16;  // 16-byte chunks (8 bf16) per thread: half a row
+    const uint4* src = reinterpret_cast<const uint4*>(codes + (src_row * D + (lane & 1) * (D / 2)) * 2);
+    uint4 raw[NC];
+    uint32_t m2 = 0;
+#pragma unroll
+    for (int c = 0; c < NC; ++c) {
+      raw[c] = live ? __ldg(src + c) : make_uint4(0, 0, 0, 0);
+      m2 = bf16x2_absmax(bf16x2_absmax(m2, raw[c].x), bf16x2_absmax(raw[c].y, raw[c].z));
+      m2 = bf16x2_absmax(m2, raw[c].w);
+    }
+    m2 &= 0x7FFF7FFFu;
+    float am = fmaxf(__uint_as_float(m2 << 16), __uint_as_float(m2 & 0xFFFF0000u));
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, off));
+    if (lane == 0) red[warp] = am;
+    __syncthreads();
+    am = fmaxf(fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3])), fmaxf(fmaxf(red[4], red[5]), fmaxf(red[6], red[7])));
+    int E = (int)((__float_as_uint(am) >> 23) & 0xFFu) - 127;  // floor(log2 am) for a normal am
+    E = max(E, -112);
+    const float r = am > 0.0f ? __uint_as_float((uint32_t)(E - 14 + 127) << 23) : 1.0f;
+    const float inv = am > 0.0f ? __uint_as_float((uint32_t)(14 - E + 127) << 23) : 1.0f;
+    if (threadIdx.x == 0) fvr[(long long)bh * ntiles + t] = make_float4(r, 0.0f, 0.0f, 0.0f);
+    if (threadIdx.x < BN) ksp[((long long)bh * ntiles + t) * BN + threadIdx.x] = tok0 + (int)threadIdx.x < S ? 1.0f : 0.0f;
+    if (!live) return;
+    uint4* dst = reinterpret_cast<uint4*>(vh + ((long long)bh * S + tok) * D + (lane & 1) * (D / 2));
+#pragma unroll
+    for (int c = 0; c < NC; ++c) {
+      const uint32_t w[4] = {raw[c].x, raw[c].y, raw[c].z, raw[c].w};
+      uint32_t o[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const __half2 y = __floats2half2_rn(__uint_as_float(w[i] << 16) * inv, __uint_as_float(w[i] & 0xFFFF0000u) * inv);
+        o[i] = *reinterpret_cast<const uint32_t*>(&y);
+      }
+      dst[c] = make_uint4(o[0], o[1], o[2], o[3]);
+    }
+    return;
   }
   constexpr int CPT = D / 32;  // 16-code chunks per thread: each thread owns half a token row
   const uint8_t* src = codes + src_row * D + (lane & 1) * (D / 2);
@@ -1161,23 +1232,28 @@ __global__ void __launch_bounds__(256) vprep_kernel(const uint8_t* __restrict__ 
   for (int c = 0; c < CPT; ++c) raw[c] = live ? __ldg(reinterpret_cast<const uint4*>(src) + c) : make_uint4(0, 0, 0, 0);
   float f = 1.0f;
   if (VSC) {
-    // every warp reduces the tile's 128 scales itself (no block barrier)
+    // every warp reduces the tile's 128 scales itself (no block barrier); v_blk 0: one per head
     const float* vsh = vs + (long long)bh * v_nblk;
     float m = 0.0f;
+    if (v_blk == 0) {
+      m = __ldg(vs + h);
+    } else {
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const int tt = tok0 + lane * 4 + q;
-      if (tt < S) m = fmaxf(m, __ldg(vsh + tt / v_blk));
+      for (int q = 0; q < 4; ++q) {
+        const int tt = tok0 + lane * 4 + q;
+        if (tt < S) m = fmaxf(m, __ldg(vsh + tt / v_blk));
+      }
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
     }
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
     const float r = m > 0.0f ? m : 1.0f;
-    f = live ? __ldg(vsh + tok / v_blk) / r : 0.0f;
+    f = live ? (v_blk == 0 ? m : __ldg(vsh + tok / v_blk)) / r : 0.0f;
     if (threadIdx.x == 0) fvr[(long long)bh * ntiles + t] = make_float4(r, 0.0f, 0.0f, 0.0f);
     // the tile's per-key K scales, zero past S, at a 16-byte aligned per-tile slot
     if (threadIdx.x < BN) {
       const int key = tok0 + threadIdx.x;
-      ksp[((long long)bh * ntiles + t) * BN + threadIdx.x] = key < S ? __ldg(ks + (long long)bh * k_nblk + key / k_blk) : 0.0f;
+      ksp[((long long)bh * ntiles + t) * BN + threadIdx.x] =
+          key < S ? (MIXED ? 1.0f : __ldg(ks + (long long)bh * k_nblk + key / k_blk)) : 0.0f;
     }
   }
   if (!live) return;
@@ -1294,11 +1370,9 @@ cudaError_t launch2(const AttnArgs& a, const P2& prm, const Prefill2Ws& w, cudaS
 }
 
 template <int KIND, int D, int SC>
-cudaError_t launch_pair(const AttnArgs& a, P2 prm, const Prefill2Ws& w, cudaStream_t s) {
-  using L = LP<D>;
-  CUtensorMap mq, mk, mv;
+cudaError_t run_pair(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, P2 prm, cudaStream_t s) {
+  using L = LP<KIND, D>;
   cudaError_t e;
-  if ((e = prepare2<KIND, D, SC != SC_HEAD>(a, prm, w, D, &mq, &mk, &mv, s)) != cudaSuccess) return e;
   auto kern = attn_pair_kernel<KIND, D, SC>;
   static bool attr_set = false;
   if (!attr_set) {
@@ -1313,6 +1387,137 @@ cudaError_t launch_pair(const AttnArgs& a, P2 prm, const Prefill2Ws& w, cudaStre
                                         : (long long)((prm.n_qtiles + 1) / 2) * prm.B * prm.Hq;
   if (grid > 0x7FFFFFFFLL) return cudaErrorInvalidValue;
   kern<<<(unsigned)grid, PNT, L::ALLOC, s>>>(mq, mk, mv, prm);
+  return cudaGetLastError();
+}
+
+template <int KIND, int D, int SC>
+cudaError_t launch_pair(const AttnArgs& a, P2 prm, const Prefill2Ws& w, cudaStream_t s) {
+  CUtensorMap mq, mk, mv;
+  cudaError_t e;
+  if ((e = prepare2<KIND, D, SC != SC_HEAD>(a, prm, w, D, &mq, &mk, &mv, s)) != cudaSuccess) return e;
+  return run_pair<KIND, D, SC>(mq, mk, mv, prm, s);
+}
+
+// ------------------------------------------------------------ mixed branches
+
+// Dequantized bf16 copy of a quantized operand, in its own layout: x = code * s (E4M3 / INT8
+// codes, per-head, per-token or per-block scales) or code * 2^(e - 127) (MX, E8M0 e per 32
+// elements); the product in fp32, then rounded to bf16.  One thread per 8 elements.
+__global__ void __launch_bounds__(256) deq_bf16_kernel(const uint8_t* __restrict__ codes, const void* __restrict__ scales,
+                                                       int mode, int B, int H, int S, int D, int layout, int blk,
+                                                       __nv_bfloat16* __restrict__ out) {
+  const int cpr = D / 8;  // 8-element chunks per row
+  const long long n = (long long)B * H * S * cpr;
+  const long long stride = (long long)gridDim.x * blockDim.x;
+  for (long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x; idx < n; idx += stride) {
+    const long long r = idx / cpr;  // token row in memory order
+    const int c0 = (int)(idx - r * cpr) * 8;
+    int b, h, t;
+    if (layout == FA_LAYOUT_BNSD) {
+      t = (int)(r % S);
+      const long long bh = r / S;
+      h = (int)(bh % H);
+      b = (int)(bh / H);
+    } else {
+      h = (int)(r % H);
+      const long long bs = r / H;
+      t = (int)(bs % S);
+      b = (int)(bs / S);
+    }
+    const long long bht = ((long long)b * H + h) * S + t;  // scales are [B, H, S, ...] in every layout
+    float x[8];
+    if (mode == FA_MODE_MXFP4_PER_BLOCK || mode == FA_MODE_MXFP8_PER_BLOCK) {
+      const int e = (int)static_cast<const uint8_t*>(scales)[bht * (D / 32) + c0 / 32];
+      const float sc = ldexpf(1.0f, e - 127);
+      if (mode == FA_MODE_MXFP4_PER_BLOCK) {
+        const uint32_t w = *reinterpret_cast<const uint32_t*>(codes + r * (D / 2) + c0 / 2);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const uint32_t h2 = e2m1x2_to_h2((w >> (8 * i)) & 0xFFu);
+          const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&h2));
+          x[2 * i] = f.x * sc;
+          x[2 * i + 1] = f.y * sc;
+        }
+      } else {
+        const uint2 w = *reinterpret_cast<const uint2*>(codes + r * D + c0);
+        const uint32_t ww[2] = {w.x, w.y};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const uint32_t h2 = e4m3x2_to_h2((uint16_t)(ww[i >> 1] >> ((i & 1) * 16)));
+          const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&h2));
+          x[2 * i] = f.x * sc;
+          x[2 * i + 1] = f.y * sc;
+        }
+      }
+    } else {
+      const float* sf = static_cast<const float*>(scales);
+      float sc;
+      if (mode == FA_MODE_INT8_PER_HEAD || mode == FA_MODE_FP8_PER_HEAD) sc = __ldg(sf + h);
+      else if (mode == FA_MODE_FP8_BLOCK) sc = __ldg(sf + ((long long)b * H + h) * ((S + blk - 1) / blk) + t / blk);
+      else sc = __ldg(sf + bht);  // per token
+      const uint2 w = *reinterpret_cast<const uint2*>(codes + r * D + c0);
+      const uint32_t ww[2] = {w.x, w.y};
+      const bool s8 = mode == FA_MODE_INT8_PER_HEAD || mode == FA_MODE_INT8_PER_TOKEN;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const uint32_t pr = ww[i >> 1] >> ((i & 1) * 16);
+        if (s8) {
+          x[2 * i] = (float)(int8_t)(pr & 0xFFu) * sc;
+          x[2 * i + 1] = (float)(int8_t)((pr >> 8) & 0xFFu) * sc;
+        } else {
+          const uint32_t h2 = e4m3x2_to_h2((uint16_t)pr);
+          const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&h2));
+          x[2 * i] = f.x * sc;
+          x[2 * i + 1] = f.y * sc;
+        }
+      }
+    }
+    uint32_t o[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const __nv_bfloat162 y = __floats2bfloat162_rn(x[2 * i], x[2 * i + 1]);
+      o[i] = *reinterpret_cast<const uint32_t*>(&y);
+    }
+    *reinterpret_cast<uint4*>(out + r * D + c0) = make_uint4(o[0], o[1], o[2], o[3]);
+  }
+}
+
+cudaError_t launch_deq_bf16(const fa_qtensor* t, __nv_bfloat16* out, cudaStream_t s) {
+  const long long n = (long long)t->B * t->H * t->S * (t->D / 8);
+  if (n == 0) return cudaSuccess;
+  long long grid = (n + 255) / 256;
+  const long long cap = 8LL * sm_count();
+  if (grid > cap) grid = cap;
+  deq_bf16_kernel<<<(unsigned)grid, 256, 0, s>>>(static_cast<const uint8_t*>(t->codes), t->scales, (int)t->mode, t->B,
+                                                 t->H, t->S, t->D, (int)t->layout, t->block_tokens, out);
+  return cudaGetLastError();
+}
+
+template <int D>
+cudaError_t vprep_mixed(const AttnArgs& a, const P2& prm, const Prefill2Ws& w, cudaStream_t s) {
+  const dim3 pgrid((unsigned)prm.ntiles_k, (unsigned)(a.v->B * a.v->H));
+  if (pgrid.y > 65535u) return cudaErrorInvalidValue;
+  const uint8_t* vc = static_cast<const uint8_t*>(a.v->codes);
+#define FAQ_VPREP_MIXED(KIND_, D_)                                                                                   \
+  vprep_kernel<KIND_, D_, true, true><<<pgrid, 256, 0, s>>>(vc, prm.vs, prm.v_blk, prm.v_nblk, a.v->H, a.v->S,        \
+                                                         a.v->layout, w.vh, w.fvr, prm.ntiles_k, nullptr, 0, 1, w.ksp, \
+                                                         prm.ve8, nullptr)
+  switch (a.v->mode) {
+    case FA_MODE_FLOAT: FAQ_VPREP_MIXED(K_BF16, D); break;
+    case FA_MODE_FP8_PER_TOKEN:
+    case FA_MODE_FP8_BLOCK:
+    case FA_MODE_FP8_PER_HEAD: FAQ_VPREP_MIXED(K_E4M3, D); break;
+    case FA_MODE_INT8_PER_HEAD:
+    case FA_MODE_INT8_PER_TOKEN: FAQ_VPREP_MIXED(K_S8, D); break;
+    case FA_MODE_MXFP4_PER_BLOCK:
+      if constexpr (D == 128) { FAQ_VPREP_MIXED(K_MXF4, 128); break; }
+      return cudaErrorNotSupported;
+    case FA_MODE_MXFP8_PER_BLOCK:
+      if constexpr (D == 128) { FAQ_VPREP_MIXED(K_MXF8, 128); break; }
+      return cudaErrorNotSupported;
+    default: return cudaErrorNotSupported;
+  }
+#undef FAQ_VPREP_MIXED
   return cudaGetLastError();
 }
 
@@ -1405,6 +1610,66 @@ cudaError_t launch_attention_prefill2(const AttnArgs& a, void* ws, cudaStream_t 
     default:
       return cudaErrorNotSupported;
   }
+}
+
+// Mixed branches: Q and K as bf16 (dequantized into the workspace, or used as they are when not
+// quantized), V' from V's own mode, then the bf16 pair kernel with every scale already applied.
+size_t mixed_workspace_bytes(const fa_qtensor* q, const fa_qtensor* k) {
+  size_t n = prefill2_workspace_bytes(k->B, k->H, k->S, q->D);
+  if (q->mode != FA_MODE_FLOAT) n += align256((size_t)q->B * q->H * q->S * q->D * 2);
+  if (k->mode != FA_MODE_FLOAT) n += align256((size_t)k->B * k->H * k->S * k->D * 2);
+  return n;
+}
+
+cudaError_t launch_attention_mixed(const AttnArgs& a, void* ws, cudaStream_t s) {
+  const fa_qtensor* q = a.q;
+  const fa_qtensor* k = a.k;
+  const int D = q->D;
+  if ((a.v->mode == FA_MODE_MXFP4_PER_BLOCK || a.v->mode == FA_MODE_MXFP8_PER_BLOCK) && D != 128)
+    return cudaErrorNotSupported;
+  P2 prm = {};
+  prm.B = q->B; prm.Hq = q->H; prm.Hkv = k->H; prm.Sq = q->S; prm.Sk = k->S; prm.group = q->H / k->H;
+  prm.causal = a.causal; prm.layout = q->layout;
+  const float scale = a.softmax_scale > 0.0f ? a.softmax_scale : 1.0f / sqrtf((float)D);
+  prm.scale_log2 = scale * 1.4426950408889634f;
+  prm.q_blk = -1;  // Q arrives with its scales applied
+  prm.q_nblk = 1;
+  prm.vs = static_cast<const float*>(a.v->scales);
+  scale_desc2(a.v, prm.v_blk, prm.v_nblk);
+  if (a.v->mode == FA_MODE_MXFP4_PER_BLOCK || a.v->mode == FA_MODE_MXFP8_PER_BLOCK)
+    prm.ve8 = static_cast<const uint8_t*>(a.v->scales);
+  prm.out = static_cast<__nv_bfloat16*>(a.out);
+  prm.lse = a.lse;
+  prm.status = a.status;
+  prm.n_qtiles = (q->S + BM - 1) / BM;
+  prm.ntiles_k = (k->S + BN - 1) / BN;
+  const Prefill2Ws w = carve_ws(ws, k->B, k->H, k->S, D);
+  prm.fvr = w.fvr;
+  prm.ksp = w.ksp;
+  uint8_t* extra = static_cast<uint8_t*>(ws) + prefill2_workspace_bytes(k->B, k->H, k->S, D);
+  const void* qb = q->codes;
+  const void* kb = k->codes;
+  cudaError_t e;
+  if (q->mode != FA_MODE_FLOAT) {
+    if ((e = launch_deq_bf16(q, reinterpret_cast<__nv_bfloat16*>(extra), s)) != cudaSuccess) return e;
+    qb = extra;
+    extra += align256((size_t)q->B * q->H * q->S * D * 2);
+  }
+  if (k->mode != FA_MODE_FLOAT) {
+    if ((e = launch_deq_bf16(k, reinterpret_cast<__nv_bfloat16*>(extra), s)) != cudaSuccess) return e;
+    kb = extra;
+  }
+  CUtensorMap mq, mk, mv;
+  const int rb = 2 * D, ab = rb > 128 ? 128 : rb;
+  if ((e = make_code_map(&mq, qb, q->B, q->H, q->S, rb, q->layout, BM, ab)) != cudaSuccess) return e;
+  if ((e = make_code_map(&mk, kb, k->B, k->H, k->S, rb, k->layout, BN, ab)) != cudaSuccess) return e;
+  if ((e = make_vh_map(&mv, w.vh, a.v->B, a.v->H, a.v->S, D)) != cudaSuccess) return e;
+  if (D == 128) {
+    if ((e = vprep_mixed<128>(a, prm, w, s)) != cudaSuccess) return e;
+    return run_pair<K_BF16, 128, SC_TILE>(mq, mk, mv, prm, s);
+  }
+  if ((e = vprep_mixed<64>(a, prm, w, s)) != cudaSuccess) return e;
+  return run_pair<K_BF16, 64, SC_TILE>(mq, mk, mv, prm, s);
 }
 
 cudaError_t launch_fill_empty_rows(void* out, float* lse, long long rows, int D, cudaStream_t s) {

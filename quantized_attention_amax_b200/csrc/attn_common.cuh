@@ -75,8 +75,9 @@ __device__ __forceinline__ bool warp_wait(uint64_t* b, uint32_t parity, volatile
   return __all_sync(0xffffffffu, ok);
 }
 
+// blk < 0: no scale (operands whose scales are already applied)
 __device__ __forceinline__ float scale_at(const float* s, int blk, int nblk, int bh, int h, int tok) {
-  return blk == 0 ? __ldg(s + h) : __ldg(s + (long long)bh * nblk + tok / blk);
+  return blk < 0 ? 1.0f : blk == 0 ? __ldg(s + h) : __ldg(s + (long long)bh * nblk + tok / blk);
 }
 
 // Two E4M3 codes -> two fp16 (exact).  Low byte -> low half.
@@ -121,9 +122,11 @@ __device__ __forceinline__ uint32_t s8x2_to_h2(uint32_t w_biased, int sel) {
 }
 
 
-// 4D tensor map over 8-bit codes: (D bytes, rows of the layout...).
+// 4D tensor map over token rows of D_bytes bytes (8-bit codes, or bf16 rows read as bytes):
+// (row bytes, rows of the layout...), boxes of box_bytes (default: the whole row) x box_rows.
 inline cudaError_t make_code_map(CUtensorMap* map, const void* base, int B, int H, int S, int D_bytes, int layout,
-                          int box_rows) {
+                          int box_rows, int box_bytes = 0) {
+  const int bb = box_bytes > 0 ? box_bytes : D_bytes;
   EncodeTiledFn enc = encode_tiled_fn();
   if (!enc) return cudaErrorNotSupported;
   cuuint64_t dims[4], strides[3];
@@ -131,15 +134,15 @@ inline cudaError_t make_code_map(CUtensorMap* map, const void* base, int B, int 
   if (layout == FA_LAYOUT_BNSD) {
     dims[0] = D_bytes; dims[1] = S; dims[2] = H; dims[3] = B;
     strides[0] = (cuuint64_t)D_bytes; strides[1] = (cuuint64_t)S * D_bytes; strides[2] = (cuuint64_t)H * S * D_bytes;
-    box[0] = D_bytes; box[1] = box_rows; box[2] = 1; box[3] = 1;
+    box[0] = bb; box[1] = box_rows; box[2] = 1; box[3] = 1;
   } else {
     dims[0] = D_bytes; dims[1] = H; dims[2] = S; dims[3] = B;
     strides[0] = (cuuint64_t)D_bytes; strides[1] = (cuuint64_t)H * D_bytes; strides[2] = (cuuint64_t)S * H * D_bytes;
-    box[0] = D_bytes; box[1] = 1; box[2] = box_rows; box[3] = 1;
+    box[0] = bb; box[1] = 1; box[2] = box_rows; box[3] = 1;
   }
-  const CUtensorMapSwizzle swz = D_bytes == 128 ? CU_TENSOR_MAP_SWIZZLE_128B
-                                 : D_bytes == 64 ? CU_TENSOR_MAP_SWIZZLE_64B
-                                                 : CU_TENSOR_MAP_SWIZZLE_32B;
+  const CUtensorMapSwizzle swz = bb == 128 ? CU_TENSOR_MAP_SWIZZLE_128B
+                                 : bb == 64 ? CU_TENSOR_MAP_SWIZZLE_64B
+                                            : CU_TENSOR_MAP_SWIZZLE_32B;
   CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 4, const_cast<void*>(base), dims, strides, box, es,
                    CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);

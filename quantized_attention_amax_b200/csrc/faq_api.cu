@@ -111,6 +111,17 @@ fa_status check_qtensor(const fa_qtensor* t) {
   return FA_OK;
 }
 
+// An attention operand: a quantized descriptor, or FA_MODE_FLOAT whose codes are the bf16 tensor
+// itself (scales unused).
+fa_status check_operand(const fa_qtensor* t) {
+  if (!t) return FA_ERR_INVALID_ARG;
+  if (t->mode != FA_MODE_FLOAT) return check_qtensor(t);
+  if (t->B < 0 || t->H < 1 || t->S < 0 || !valid_layout(t->layout)) return FA_ERR_INVALID_ARG;
+  if (t->D != 64 && t->D != 128) return FA_ERR_UNSUPPORTED;
+  if ((long long)t->B * t->S > 0 && (!t->codes || !aligned16(t->codes))) return FA_ERR_INVALID_ARG;
+  return FA_OK;
+}
+
 }  // namespace
 }  // namespace faq
 
@@ -230,14 +241,24 @@ fa_status fa_rotate_quantize(const fa_tensor* q, const fa_tensor* k, const fa_te
   return from_cuda(e);
 }
 
+// Branches in different modes, or any branch not quantized: the bf16 mixed path.
+static bool is_mixed(const fa_qtensor* q, const fa_qtensor* k, const fa_qtensor* v) {
+  return q->mode != k->mode || (v && q->mode != v->mode) || q->mode == FA_MODE_FLOAT || k->mode == FA_MODE_FLOAT ||
+         (v && v->mode == FA_MODE_FLOAT);
+}
+
 static bool is_decode(const fa_qtensor* q, const fa_qtensor* k) {
   if (q->S != 1 || q->mode != FA_MODE_INT8_PER_HEAD || q->D != 128) return false;
   const int group = q->H / k->H;
   return group == 1 || group == 2 || group == 4 || group == 8 || group == 16;
 }
 
-size_t fa_attention_workspace_size(const fa_qtensor* q, const fa_qtensor* k, int num_splits) {
+static size_t attention_ws(const fa_qtensor* q, const fa_qtensor* k, const fa_qtensor* v, int num_splits) {
   if (!q || !k || k->H < 1 || q->H % k->H || num_splits < 0) return 0;
+  if (is_mixed(q, k, v)) {
+    if (k->B < 0 || k->S < 0 || q->B < 0 || q->S < 0 || (q->D != 64 && q->D != 128)) return 0;
+    return mixed_workspace_bytes(q, k);
+  }
   if (is_decode(q, k)) {
     const int splits = num_splits > 0 ? num_splits : decode_auto_splits(k->B, k->H, k->S);
     return decode_workspace_bytes(q->B, q->H, q->D, splits);
@@ -254,31 +275,45 @@ size_t fa_attention_workspace_size(const fa_qtensor* q, const fa_qtensor* k, int
   return 0;
 }
 
+size_t fa_attention_workspace_size(const fa_qtensor* q, const fa_qtensor* k, int num_splits) {
+  return attention_ws(q, k, nullptr, num_splits);
+}
+
+size_t fa_attention_workspace_size_qkv(const fa_qtensor* q, const fa_qtensor* k, const fa_qtensor* v,
+                                       int num_splits) {
+  if (!v) return 0;
+  return attention_ws(q, k, v, num_splits);
+}
+
 fa_status fa_attention_quant(const fa_qtensor* q, const fa_qtensor* k, const fa_qtensor* v, int causal,
                              float softmax_scale, void* out, float* lse, int num_splits, void* workspace,
                              size_t ws_bytes, fa_stream_t s) {
   fa_status st;
-  if ((st = check_qtensor(q)) != FA_OK) return st;
-  if ((st = check_qtensor(k)) != FA_OK) return st;
-  if ((st = check_qtensor(v)) != FA_OK) return st;
-  if (q->mode != k->mode || q->mode != v->mode) return FA_ERR_UNSUPPORTED;  // mixed branches
+  if ((st = check_operand(q)) != FA_OK) return st;
+  if ((st = check_operand(k)) != FA_OK) return st;
+  if ((st = check_operand(v)) != FA_OK) return st;
+  const bool mixed = is_mixed(q, k, v);
   if (q->layout != k->layout || q->layout != v->layout) return FA_ERR_INVALID_ARG;
   if (q->D != k->D || q->D != v->D) return FA_ERR_INVALID_ARG;
   if (q->B != k->B || q->B != v->B) return FA_ERR_INVALID_ARG;
   if (k->H != v->H || k->S != v->S) return FA_ERR_INVALID_ARG;
   if (q->H % k->H != 0) return FA_ERR_INVALID_ARG;
-  if (q->mode == FA_MODE_FP8_BLOCK && k->block_tokens != v->block_tokens) return FA_ERR_INVALID_ARG;
+  if (!mixed && q->mode == FA_MODE_FP8_BLOCK && k->block_tokens != v->block_tokens) return FA_ERR_INVALID_ARG;
   if (num_splits < 0) return FA_ERR_INVALID_ARG;
   const long long qrows = (long long)q->B * q->H * q->S;
   if (qrows == 0) return FA_OK;
   if (!out || !aligned16(out)) return FA_ERR_INVALID_ARG;
   if (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)) return FA_ERR_INVALID_ARG;
-  const bool decode = is_decode(q, k);
-  if ((q->mode == FA_MODE_MXFP4_PER_BLOCK || q->mode == FA_MODE_MXFP8_PER_BLOCK) && q->D != 128) return FA_ERR_UNSUPPORTED;
+  const bool decode = !mixed && is_decode(q, k);
+  if (!mixed && (q->mode == FA_MODE_MXFP4_PER_BLOCK || q->mode == FA_MODE_MXFP8_PER_BLOCK) && q->D != 128)
+    return FA_ERR_UNSUPPORTED;
+  if (mixed && (v->mode == FA_MODE_MXFP4_PER_BLOCK || v->mode == FA_MODE_MXFP8_PER_BLOCK) && v->D != 128)
+    return FA_ERR_UNSUPPORTED;
   const int splits = decode ? (num_splits > 0 ? num_splits : decode_auto_splits(k->B, k->H, k->S)) : 0;
   if (k->S > 0) {
-    const size_t need = decode ? decode_workspace_bytes(q->B, q->H, q->D, splits)
-                               : prefill2_workspace_bytes(k->B, k->H, k->S, q->D);
+    const size_t need = mixed    ? mixed_workspace_bytes(q, k)
+                        : decode ? decode_workspace_bytes(q->B, q->H, q->D, splits)
+                                 : prefill2_workspace_bytes(k->B, k->H, k->S, q->D);
     if (!workspace || ws_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255u)) return FA_ERR_WORKSPACE;
   }
   cudaStream_t cs = reinterpret_cast<cudaStream_t>(s);
@@ -287,7 +322,9 @@ fa_status fa_attention_quant(const fa_qtensor* q, const fa_qtensor* k, const fa_
   if (!status) return FA_ERR_CUDA;
   AttnArgs a = {q, k, v, causal ? 1 : 0, softmax_scale, out, lse, status};
   cudaError_t e;
-  if (decode)
+  if (mixed)
+    e = launch_attention_mixed(a, workspace, cs);
+  else if (decode)
     e = launch_attention_decode(a, splits, workspace, cs);
   else
     e = launch_attention_prefill2(a, workspace, cs);

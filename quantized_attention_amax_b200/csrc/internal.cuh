@@ -63,6 +63,10 @@ struct AttnArgs {
 // Prefill (E4M3, INT8, MXFP4): V' pre-pass + attention; `ws` holds prefill2_workspace_bytes().
 size_t prefill2_workspace_bytes(int B, int Hkv, int Sk, int D);
 cudaError_t launch_attention_prefill2(const AttnArgs& a, void* ws, cudaStream_t s);
+// Mixed branches (modes differ, or a branch is not quantized): bf16 Q / K pair kernel;
+// `ws` holds mixed_workspace_bytes(q, k).
+size_t mixed_workspace_bytes(const fa_qtensor* q, const fa_qtensor* k);
+cudaError_t launch_attention_mixed(const AttnArgs& a, void* ws, cudaStream_t s);
 
 size_t decode_workspace_bytes(int B, int Hq, int D, int splits);
 int decode_auto_splits(int B, int Hkv, int Sk);

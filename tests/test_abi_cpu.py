@@ -119,14 +119,15 @@ def test_attention_validation_before_launch(N):
     k = _q(N, 2, H=2)
     v = _q(N, 2, H=2)
     km = _q(N, 1, H=2)
-    assert L.fa_attention_quant(by(q), by(km), by(v), 0, 0.0, 0x60000, None, 0, None, 0, None) == 2  # mixed
+    # mixed branches run (the bf16 path): without a workspace they stop at the workspace check
+    assert L.fa_attention_quant(by(q), by(km), by(v), 0, 0.0, 0x60000, None, 0, None, 0, None) == 7  # mixed
     k3 = _q(N, 2, H=3)
     assert L.fa_attention_quant(by(q), by(k3), by(k3), 0, 0.0, 0x60000, None, 0, None, 0, None) == 1  # GQA
     kd = _q(N, 2, H=2, D=128)
     assert L.fa_attention_quant(by(q), by(kd), by(kd), 0, 0.0, 0x60000, None, 0, None, 0, None) == 1  # D
     assert L.fa_attention_quant(by(q), by(k), by(v), 0, 0.0, None, None, 0, None, 0, None) == 1      # out
     qf = _q(N, 0, H=4)
-    assert L.fa_attention_quant(by(qf), by(k), by(v), 0, 0.0, 0x60000, None, 0, None, 0, None) == 2  # float
+    assert L.fa_attention_quant(by(qf), by(k), by(v), 0, 0.0, 0x60000, None, 0, None, 0, None) == 7  # float
     # decode without workspace
     qd = _q(N, 1, B=2, H=4, S=1, D=128)
     kd = _q(N, 1, B=2, H=2, S=1000, D=128)
@@ -160,3 +161,42 @@ def test_attention_validation_before_launch(N):
     qm64, km64 = _q(N, 3, B=2, H=4, S=100, D=64), _q(N, 3, B=2, H=2, S=1000, D=64)
     assert L.fa_attention_workspace_size(by(qm64), by(km64), 0) == 0
     assert L.fa_attention_quant(by(qm64), by(km64), by(km64), 0, 0.0, 0x60000, None, 0, None, 0, None) == 2
+
+
+def test_mixed_branch_validation_and_workspace(N):
+    """Per-branch modes (fa3_quant details): a float branch is the bf16 tensor itself; mixed
+    calls need V' parts plus bf16 copies of the Q / K branches that are quantized."""
+    L = N.lib()
+    by = ctypes.byref
+    B, Hq, Hkv, Sq, Sk, D = 2, 4, 2, 100, 1000, 128
+    ntiles = (Sk + 127) // 128
+    r256 = lambda x: ((x + 255) // 256) * 256
+    base = sum(r256(x) for x in (B * Hkv * Sk * D * 2, B * Hkv * ntiles * 16, B * Hkv * ntiles * 128 * 4))
+    qcopy, kcopy = r256(B * Hq * Sq * D * 2), r256(B * Hkv * Sk * D * 2)
+    q8, k8 = _q(N, 2, B=B, H=Hq, S=Sq, D=D), _q(N, 2, B=B, H=Hkv, S=Sk, D=D)
+    qf, kf, vf = _q(N, 0, B=B, H=Hq, S=Sq, D=D), _q(N, 0, B=B, H=Hkv, S=Sk, D=D), _q(N, 0, B=B, H=Hkv, S=Sk, D=D)
+    ki = _q(N, 1, B=B, H=Hkv, S=Sk, D=D)
+    # all three float: plain bf16 attention, nothing to dequantize
+    assert L.fa_attention_workspace_size_qkv(by(qf), by(kf), by(vf), 0) == base
+    # Q quantized, K float: Q's bf16 copy only
+    assert L.fa_attention_workspace_size_qkv(by(q8), by(kf), by(vf), 0) == base + qcopy
+    # Q and K in different modes: both copies; fa_attention_workspace_size sees that without v
+    assert L.fa_attention_workspace_size_qkv(by(q8), by(ki), by(k8), 0) == base + qcopy + kcopy
+    assert L.fa_attention_workspace_size(by(q8), by(ki), 0) == base + qcopy + kcopy
+    # Q and K alike, only V differs: only the three-branch query knows
+    assert L.fa_attention_workspace_size(by(q8), by(k8), 0) == base
+    assert L.fa_attention_workspace_size_qkv(by(q8), by(k8), by(vf), 0) == base + qcopy + kcopy
+    assert L.fa_attention_workspace_size_qkv(by(q8), by(k8), by(k8), 0) == base
+    assert L.fa_attention_workspace_size_qkv(by(q8), by(k8), None, 0) == 0
+    # a workspace sized for the uniform call is too small once V differs
+    assert L.fa_attention_quant(by(q8), by(k8), by(vf), 0, 0.0, 0x60000, None, 0, 0x70000, base, None) == 7
+    # a float branch without data, or with an unsupported head_dim
+    qnull = _q(N, 0, B=B, H=Hq, S=Sq, D=D)
+    qnull.codes = None
+    assert L.fa_attention_quant(by(qnull), by(k8), by(k8), 0, 0.0, 0x60000, None, 0, None, 0, None) == 1
+    q96 = _q(N, 0, B=B, H=Hq, S=Sq, D=96)
+    assert L.fa_attention_quant(by(q96), by(kf), by(vf), 0, 0.0, 0x60000, None, 0, None, 0, None) == 2
+    # an MX V in a mixed call needs head_dim 128
+    q64, k64 = _q(N, 2, B=B, H=Hq, S=Sq, D=64), _q(N, 2, B=B, H=Hkv, S=Sk, D=64)
+    vm64 = _q(N, 3, B=B, H=Hkv, S=Sk, D=64)
+    assert L.fa_attention_quant(by(q64), by(k64), by(vm64), 0, 0.0, 0x60000, None, 0, None, 0, None) == 2
