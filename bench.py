@@ -46,6 +46,8 @@ DESCR = {
     "fp8_head_prefill": "FP8 E4M3 per-head static, the fp8_prefill shape (B=2 Hq=32 Hkv=8 S=4096 D=128, causal, BNSD)",
     "int8_token_prefill": "INT8 per-token dynamic, the fp8_prefill shape (B=2 Hq=32 Hkv=8 S=4096 D=128, causal, BNSD)",
     "mxfp8": "MXFP8 per-32-block (E4M3 + E8M0), the mxfp4 shape (B=1 H=24 S=4096 D=128, non-causal, BNSD, Student-t)",
+    "mixed_prefill": "per-branch modes: Q, K FP8 per-token, V unquantized bf16, the fp8_prefill shape "
+                     "(B=2 Hq=32 Hkv=8 S=4096 D=128, causal, BNSD)",
 }
 DATA = {
     "int8_tiny": "synthetic: seeded bf16 N(0,1); per-head scales from a seeded calibration batch",
@@ -57,6 +59,7 @@ DATA = {
     "fp8_head_prefill": "synthetic: as fp8_prefill; per-head scales from seeded calibration batches",
     "int8_token_prefill": "synthetic: as fp8_prefill",
     "mxfp8": "synthetic: seeded bf16 Student-t (df=4)",
+    "mixed_prefill": "synthetic: as fp8_prefill",
 }
 DTYPE = {
     "int8_tiny": "s8 (QK^T, s32 acc) + f16 (PV)",
@@ -68,6 +71,7 @@ DTYPE = {
     "fp8_head_prefill": "e4m3 (QK^T) + f16 (PV), fp32 accumulate",
     "int8_token_prefill": "s8 (QK^T, s32 acc) + f16 (PV)",
     "mxfp8": "e4m3 block-scaled (QK^T) + f16 (PV)",
+    "mixed_prefill": "bf16 (dequantized QK^T) + f16 (PV), fp32 accumulate",
 }
 
 
@@ -88,6 +92,10 @@ def quant_bytes(w) -> float:
     """Algorithmic bytes of the quantize step: bf16 in once, codes + scales out once."""
     nq = w.B * w.Hq * w.Sq * w.D
     nk = w.B * w.Hkv * w.Sk * w.D
+    if w.branch_modes is not None:
+        # this bench's mixed workload: Q and K FP8 per token, V not quantized
+        assert w.branch_modes == ("fp8_per_token", "fp8_per_token", "float")
+        return (nq + nk) * 3 + (w.B * w.Hq * w.Sq + w.B * w.Hkv * w.Sk) * 4
     if w.mode == "int8_decode" or w.name == "int8_decode":
         return nq * 2 + nq + w.Hq * 4  # only Q is quantized per step
     code = 0.5 if w.mode == "mxfp4" else 1.0
@@ -123,8 +131,10 @@ def peaks():
 
 def tensor_peak(w, pk):
     """Dense peak for the QK^T operand type: measured bf16 x the nominal ratio
-    (FP8/INT8 2x, FP4 4x the bf16 rate)."""
+    (FP8/INT8 2x, FP4 4x the bf16 rate; bf16 itself for mixed branches)."""
     ratio = 4.0 if w.mode == "mxfp4" else 2.0
+    if w.branch_modes is not None:
+        ratio = 1.0  # mixed branches: QK^T on bf16
     return pk["bf16"] * ratio
 
 
@@ -207,6 +217,15 @@ def make_step(faq, wl, w, device, seed_offset=0):
 
             def quant():
                 faq.quantize(q, k, v, w.mode, w.layout, amax=amax, out=QKV)
+    elif w.branch_modes is not None:
+        # Q and K quantized in one mode, V left as bf16 (the only mix this bench runs)
+        mq, mk, mv = w.branch_modes
+        assert mq == mk and mv == "float"
+        QK = list(faq.quantize(q, k, None, mq, w.layout))
+        st["QKV"] = [QK[0], QK[1], faq.float_branch(v, w.layout)]
+
+        def quant():
+            faq.quantize(q, k, None, mq, w.layout, out=QK)
     elif w.rotate:
         QKV = list(faq.rotate_quantize(q, k, v, inp["R"], inp["R"], w.layout, w.q_block, w.kv_block))
         st["QKV"] = QKV
@@ -222,7 +241,7 @@ def make_step(faq, wl, w, device, seed_offset=0):
 
     Qq, Kq, Vq = st["QKV"]
     out = torch.empty_like(q)
-    ws_bytes = faq.attention_workspace_size(Qq, Kq)
+    ws_bytes = faq.attention_workspace_size(Qq, Kq, v=Vq)
     ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=device)
     st["out"] = out
 
@@ -239,7 +258,9 @@ def make_step(faq, wl, w, device, seed_offset=0):
 def launches_per_step(w):
     """This library's kernels per step: the quantize (or rotate + quantize) launch, then
     the attention call: decode + LSE combine, or for prefill the V' pre-pass and the
-    attention kernel."""
+    attention kernel (mixed branches: one bf16 dequantize launch per quantized Q / K first)."""
+    if w.branch_modes is not None:
+        return 1 + sum(m != "float" for m in w.branch_modes[:2]) + 2
     return 1 + 2
 
 
@@ -247,6 +268,8 @@ def attention_kernels(w):
     """(label, source file) of the attention call's kernels for this workload."""
     if w.name == "int8_decode":
         return "decode_kernel + attn_combine_kernel", "decode.cu"
+    if w.branch_modes is not None:
+        return "deq_bf16_kernel x2 + vprep_kernel + attn_pair_kernel<bf16> (one fa_attention_quant call)", "attn2.cu"
     if w.mode in ("mxfp4", "mxfp8"):
         return "vprep_kernel + attn2_kernel (one fa_attention_quant call)", "attn2.cu"
     return "vprep_kernel + attn_pair_kernel (one fa_attention_quant call)", "attn2.cu"
@@ -565,7 +588,7 @@ def supplemental(args, device):
     out = {}
     pk = peaks()
     for name in ("int8_tiny", "rot_fp8_block", "mxfp4", "int8_decode", "int8_prefill", "fp8_head_prefill",
-                 "int8_token_prefill", "mxfp8"):
+                 "int8_token_prefill", "mxfp8", "mixed_prefill"):
         w = wl.WORKLOADS[name]
         a = argparse.Namespace(steps=10 if name != "rot_fp8_block" else 4, warmup=3)
         r = gpu_run(a, w, 0, 1, device)
@@ -661,8 +684,9 @@ def main():
         ach = work / (r["attn_ms"] * 1e-3) / 1e12
         roof = {"bound": "tensor", "achieved": ach, "peak": tp, "unit": "TFLOP/s", "frac": ach / tp,
                 "traffic": None, "kernel": attention_kernels(w)[0],
-                "peak_source": f"{pk['src']} bf16 burst x {4 if w.mode == 'mxfp4' else 2} (dense "
-                               f"{'FP4' if w.mode == 'mxfp4' else 'FP8/INT8'} : bf16 nominal ratio)"}
+                "peak_source": (f"{pk['src']} bf16 burst (mixed branches: QK^T on bf16)" if w.branch_modes is not None
+                                else f"{pk['src']} bf16 burst x {4 if w.mode == 'mxfp4' else 2} (dense "
+                                     f"{'FP4' if w.mode == 'mxfp4' else 'FP8/INT8'} : bf16 nominal ratio)")}
     prof = os.path.join(ROOT, "profiles", f"traffic_{w.name}.json")
     if os.path.exists(prof):
         # DRAM bytes per launch from one ncu capture, valid only while the

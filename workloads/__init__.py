@@ -45,6 +45,7 @@ class Workload:
     rotate: bool = False
     q_block: int = 128
     kv_block: int = 256
+    branch_modes: Optional[tuple] = None  # per-branch (q, k, v) modes; "float" = left unquantized
 
     def scaled(self, **kw) -> "Workload":
         return replace(self, **kw)
@@ -66,6 +67,9 @@ WORKLOADS: Dict[str, Workload] = {
     "int8_token_prefill": Workload("int8_token_prefill", "int8_per_token", 2, 32, 8, 4096, 4096, 128, "BNSD", True,
                                    "normal_k_outliers", 7),
     "mxfp8": Workload("mxfp8", "mxfp8", 1, 24, 24, 4096, 4096, 128, "BNSD", False, "student_t4", 8),
+    # per-branch details: Q and K FP8 per token, V left unquantized (bf16), the fp8_prefill shape
+    "mixed_prefill": Workload("mixed_prefill", "fp8_per_token", 2, 32, 8, 4096, 4096, 128, "BNSD", True,
+                              "normal_k_outliers", 9, branch_modes=("fp8_per_token", "fp8_per_token", "float")),
 }
 
 CALIB_SEED_OFFSET = 1000
