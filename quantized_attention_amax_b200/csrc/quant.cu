@@ -32,6 +32,13 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
   return r;
 }
 
+// per half: max(|a|, |b|), its sign the XOR of the inputs' signs (exact; only magnitudes are used)
+__device__ __forceinline__ uint32_t bf16x2_absmax(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("max.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+
 __device__ __forceinline__ void unpack_bf16x8(const uint4& u, float (&f)[8]) {
   const uint32_t w[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
@@ -133,18 +140,15 @@ __global__ void __launch_bounds__(256) quant_rows_kernel(QuantOperand o0, QuantO
     const uint4* src = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(op_x) + rr * D) + gl * 4;
 #pragma unroll
     for (int c = 0; c < 4; ++c) raw[c] = valid ? __ldg(src + c) : make_uint4(0, 0, 0, 0);
-    float f[32];
-#pragma unroll
-    for (int c = 0; c < 4; ++c) {
-      float t8[8];
-      unpack_bf16x8(raw[c], t8);
-#pragma unroll
-      for (int i = 0; i < 8; ++i) f[8 * c + i] = t8[i];
-    }
+    // max |x| over the lane's 32 elements on the packed bf16 pairs (exact, no unpacking)
     float m = 0.0f;
     if (!PER_HEAD) {
+      uint32_t m2 = 0;
 #pragma unroll
-      for (int i = 0; i < 32; i += 2) m = fmax3(m, fabsf(f[i]), fabsf(f[i + 1]));
+      for (int c = 0; c < 4; ++c)
+        m2 = bf16x2_absmax(bf16x2_absmax(m2, bf16x2_absmax(raw[c].x, raw[c].y)), bf16x2_absmax(raw[c].z, raw[c].w));
+      m2 &= 0x7FFF7FFFu;
+      m = fmaxf(__uint_as_float(m2 << 16), __uint_as_float(m2 & 0xFFFF0000u));
       if (!MX) {
 #pragma unroll
         for (int off = LPR / 2; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
@@ -159,8 +163,12 @@ __global__ void __launch_bounds__(256) quant_rows_kernel(QuantOperand o0, QuantO
         if (MODE == FA_MODE_MXFP8_PER_BLOCK) {
           uint32_t w[8];
 #pragma unroll
-          for (int i = 0; i < 8; ++i)
-            w[i] = e4m3x4(f[4 * i] * inv, f[4 * i + 1] * inv, f[4 * i + 2] * inv, f[4 * i + 3] * inv);
+          for (int c = 0; c < 4; ++c) {
+            float f[8];
+            unpack_bf16x8(raw[c], f);
+            w[2 * c] = e4m3x4(f[0] * inv, f[1] * inv, f[2] * inv, f[3] * inv);
+            w[2 * c + 1] = e4m3x4(f[4] * inv, f[5] * inv, f[6] * inv, f[7] * inv);
+          }
           uint4* dst = reinterpret_cast<uint4*>(static_cast<uint8_t*>(op_codes) + rr * D + gl * 32);
           dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
           dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
@@ -169,8 +177,9 @@ __global__ void __launch_bounds__(256) quant_rows_kernel(QuantOperand o0, QuantO
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
             float v8[8];
+            unpack_bf16x8(raw[i], v8);
 #pragma unroll
-            for (int k = 0; k < 8; ++k) v8[k] = f[8 * i + k] * inv;
+            for (int k = 0; k < 8; ++k) v8[k] *= inv;
             w[i] = e2m1x8(v8);
           }
           *reinterpret_cast<uint4*>(static_cast<uint8_t*>(op_codes) + rr * (D / 2) + gl * 16) =
@@ -194,23 +203,27 @@ __global__ void __launch_bounds__(256) quant_rows_kernel(QuantOperand o0, QuantO
     } else {
       sc = __fdiv_rn(m, QMAX);
     }
-    float v[32];
-    if (sc >= kFastDivMin) {
-      // x / s as IEEE division rounds it where that decides the code (quant_common.cuh)
-      const float rc = __frcp_rn(sc);
+    // codes, 8 elements at a time straight from the packed row
+    uint32_t w[8];
+    const bool fast = sc >= kFastDivMin;
+    const float rc = fast ? __frcp_rn(sc) : 0.0f;
 #pragma unroll
-      for (int i = 0; i < 32; ++i)
-        v[i] = INT8 ? int8_div(f[i], sc, rc) : (PER_HEAD ? fp8_div_sat(f[i], sc, rc) : fp8_div(f[i], sc, rc));
-    } else {
+    for (int c = 0; c < 4; ++c) {
+      float v[8];
+      unpack_bf16x8(raw[c], v);
+      if (fast) {
+        // x / s as IEEE division rounds it where that decides the code (quant_common.cuh)
 #pragma unroll
-      for (int i = 0; i < 32; ++i) v[i] = sc > 0.0f ? __fdiv_rn(f[i], sc) : 0.0f;
+        for (int i = 0; i < 8; ++i)
+          v[i] = INT8 ? int8_div(v[i], sc, rc) : (PER_HEAD ? fp8_div_sat(v[i], sc, rc) : fp8_div(v[i], sc, rc));
+      } else {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) v[i] = sc > 0.0f ? __fdiv_rn(v[i], sc) : 0.0f;
+      }
+      w[2 * c] = INT8 ? s8x4(v[0], v[1], v[2], v[3]) : e4m3x4(v[0], v[1], v[2], v[3]);
+      w[2 * c + 1] = INT8 ? s8x4(v[4], v[5], v[6], v[7]) : e4m3x4(v[4], v[5], v[6], v[7]);
     }
     if (valid) {
-      uint32_t w[8];
-#pragma unroll
-      for (int i = 0; i < 8; ++i)
-        w[i] = INT8 ? s8x4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3])
-                    : e4m3x4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
       out[0] = make_uint4(w[0], w[1], w[2], w[3]);
       out[1] = make_uint4(w[4], w[5], w[6], w[7]);
       uint4* dst = reinterpret_cast<uint4*>(static_cast<uint8_t*>(op_codes) + rr * D + gl * 32);
