@@ -25,13 +25,6 @@
 namespace faq {
 namespace {
 
-// max(a, b, c) in one instruction (sm_100 three-input form).
-__device__ __forceinline__ float fmax3(float a, float b, float c) {
-  float r;
-  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
-  return r;
-}
-
 // per half: max(|a|, |b|), its sign the XOR of the inputs' signs (exact; only magnitudes are used)
 __device__ __forceinline__ uint32_t bf16x2_absmax(uint32_t a, uint32_t b) {
   uint32_t d;
