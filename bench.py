@@ -275,6 +275,24 @@ def attention_kernels(w):
     return "vprep_kernel + attn_pair_kernel (one fa_attention_quant call)", "attn2.cu"
 
 
+def max_over_ranks(vals, world, device):
+    """Each rank's timed sums -> their maxima over ranks (the slowest rank sets the job's
+    time).  One all-reduce on the process group; identity for one rank."""
+    if world == 1:
+        return [float(x) for x in vals]
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(x) for x in vals], device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
+
+
+def job_value(work_per_rank, ms_per_step, world, unit):
+    """Whole-job throughput: every rank processes work_per_rank units per step (weak scaling),
+    the step takes ms_per_step on the slowest rank."""
+    return world * work_per_rank / (ms_per_step * 1e-3) / (1e9 if unit == "GB/s" else 1e12)
+
+
 def gpu_run(args, w, rank, world, device):
     import torch
     import quantized_attention_amax_b200 as faq
@@ -339,13 +357,7 @@ def gpu_run(args, w, rank, world, device):
     faq.check_device_status()
     q_ms = [ev[i][0].elapsed_time(ev[i][1]) for i in range(K)]
     a_ms = [ev[i][1].elapsed_time(ev[i][2]) for i in range(K)]
-    total_ms = sum(q_ms) + sum(a_ms)
-    if world > 1:
-        t = torch.tensor([total_ms, sum(a_ms), sum(q_ms)], device=device, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms, a_sum, q_sum = t.tolist()
-    else:
-        a_sum, q_sum = sum(a_ms), sum(q_ms)
+    total_ms, a_sum, q_sum = max_over_ranks([sum(q_ms) + sum(a_ms), sum(a_ms), sum(q_ms)], world, device)
     res = {"total_ms": total_ms, "attn_ms": a_sum / K, "quant_ms": q_sum / K, "wall_s": wall, "clocks": clk,
            "st": st, "step": step}
     return res
@@ -671,7 +683,7 @@ def main():
     else:
         unit = "TFLOP/s"
         work = attn_flops(w)
-    value = world * work / (ms_per_step * 1e-3) / (1e9 if unit == "GB/s" else 1e12)
+    value = job_value(work, ms_per_step, world, unit)
 
     # dominant kernel: attention
     if unit == "GB/s":
