@@ -231,8 +231,8 @@ __global__ void __launch_bounds__(Cfg<NSW>::NT, 1)
         }
         if (*abort_flag) {
           // let issued loads land before the CTA can exit
-          mbar_wait(&bar[X_Q], 0, abort_flag, nullptr, 0);
-          for (int t = max(0, j - NKS); t < j; ++t) mbar_wait(&bar[X_KF + t % NKS], (t / NKS) & 1, abort_flag, nullptr, 0);
+          mbar_drain(&bar[X_Q], 0);
+          for (int t = max(0, j - NKS); t < j; ++t) mbar_drain(&bar[X_KF + t % NKS], (t / NKS) & 1);
         }
       }
       __syncwarp();
@@ -251,7 +251,7 @@ __global__ void __launch_bounds__(Cfg<NSW>::NT, 1)
             tma_load_4d(smem + L::VH + vs * BN * D * 2 + a2 * BN * 128, &tmv, &bar[X_VF + vs], 64 * a2, k0, hk, b);
         }
         if (*abort_flag)
-          for (int t = max(0, j - NVS); t < j; ++t) mbar_wait(&bar[X_VF + t % NVS], (t / NVS) & 1, abort_flag, nullptr, 0);
+          for (int t = max(0, j - NVS); t < j; ++t) mbar_drain(&bar[X_VF + t % NVS], (t / NVS) & 1);
       }
       __syncwarp();
     } else if (warp == 2) {
@@ -286,7 +286,7 @@ __global__ void __launch_bounds__(Cfg<NSW>::NT, 1)
             bulk_load(stage + BN * 4, fvh + j, 16, &bar[X_SCF + st]);
           }
           if (*abort_flag)
-            for (int t = max(0, j - NSC); t < j; ++t) mbar_wait(&bar[X_SCF + t % NSC], (t / NSC) & 1, abort_flag, nullptr, 0);
+            for (int t = max(0, j - NSC); t < j; ++t) mbar_drain(&bar[X_SCF + t % NSC], (t / NSC) & 1);
         }
       }
       __syncwarp();
@@ -366,7 +366,7 @@ __global__ void __launch_bounds__(Cfg<NSW>::NT, 1)
           }
         }
         mma_commit(&bar[X_FIN]);
-        mbar_wait(&bar[X_FIN], 0, abort_flag, nullptr, 0);
+        mbar_drain(&bar[X_FIN], 0);
       }
       __syncwarp();
     }
@@ -785,8 +785,8 @@ __global__ void __launch_bounds__(PNT, 1)
                         bnsd ? k0 : hk, bnsd ? hk : k0, b);
         }
         if (*abort_flag) {
-          mbar_wait(&bar[Y_Q], 0, abort_flag, nullptr, 0);
-          for (int t = max(0, j - NKS); t < j; ++t) mbar_wait(&bar[Y_KF + t % NKS], (t / NKS) & 1, abort_flag, nullptr, 0);
+          mbar_drain(&bar[Y_Q], 0);
+          for (int t = max(0, j - NKS); t < j; ++t) mbar_drain(&bar[Y_KF + t % NKS], (t / NKS) & 1);
         }
       }
       __syncwarp();
@@ -804,7 +804,7 @@ __global__ void __launch_bounds__(PNT, 1)
             tma_load_4d(smem + L::VH + vs * BN * D * 2 + a2 * BN * 128, &tmv, &bar[Y_VF + vs], 64 * a2, k0, hk, b);
         }
         if (*abort_flag)
-          for (int t = max(0, j - NVS); t < j; ++t) mbar_wait(&bar[Y_VF + t % NVS], (t / NVS) & 1, abort_flag, nullptr, 0);
+          for (int t = max(0, j - NVS); t < j; ++t) mbar_drain(&bar[Y_VF + t % NVS], (t / NVS) & 1);
       }
       __syncwarp();
     } else if (warp == 2) {
@@ -828,7 +828,7 @@ __global__ void __launch_bounds__(PNT, 1)
             bulk_load(stage + BN * 4, fvh + j, 16, &bar[Y_SCF + st]);
           }
           if (*abort_flag)
-            for (int t = max(0, j - NSC); t < j; ++t) mbar_wait(&bar[Y_SCF + t % NSC], (t / NSC) & 1, abort_flag, nullptr, 0);
+            for (int t = max(0, j - NSC); t < j; ++t) mbar_drain(&bar[Y_SCF + t % NSC], (t / NSC) & 1);
         }
       }
       __syncwarp();
@@ -899,7 +899,7 @@ __global__ void __launch_bounds__(PNT, 1)
           if (j + 1 < n) mma_commit(&bar[Y_KE + (j + 1) % NKS]);
         }
         mma_commit(&bar[Y_FIN]);
-        mbar_wait(&bar[Y_FIN], 0, abort_flag, nullptr, 0);
+        mbar_drain(&bar[Y_FIN], 0);
       }
       __syncwarp();
     }

@@ -182,21 +182,22 @@ __global__ void __launch_bounds__(DTHREADS, 2)
       tma_prefetch_desc(&tmv);
       const bool bnsd = p.layout == FA_LAYOUT_BNSD;
       int j = 0;
+      int nk = 0;  // K tiles whose loads were issued (one more than V's when the loop stops between them)
       for (; j < n_tiles; ++j) {
         const int s = j % DNS;
         const int k0 = key0 + j * DBN;
         if (j >= DNS && !mbar_wait(&bar[D_KEMPTY + s], ((j / DNS) - 1) & 1, abort_flag, p.status, 21)) break;
         mbar_arrive_expect_tx(&bar[D_KFULL + s], DBN * D);
         tma_load_4d(smem + L::K + s * DBN * D, &tmk, &bar[D_KFULL + s], 0, bnsd ? k0 : hk, bnsd ? hk : k0, b);
+        nk = j + 1;
         if (j >= DNS && !mbar_wait(&bar[D_VEMPTY + s], ((j / DNS) - 1) & 1, abort_flag, p.status, 22)) break;
         mbar_arrive_expect_tx(&bar[D_VFULL + s], DBN * D);
         tma_load_4d(smem + L::V + s * DBN * D, &tmv, &bar[D_VFULL + s], 0, bnsd ? k0 : hk, bnsd ? hk : k0, b);
       }
       if (*abort_flag) {
-        for (int t = max(0, j - DNS); t < j; ++t) {
-          mbar_wait(&bar[D_KFULL + t % DNS], (t / DNS) & 1, abort_flag, nullptr, 0);
-          mbar_wait(&bar[D_VFULL + t % DNS], (t / DNS) & 1, abort_flag, nullptr, 0);
-        }
+        // let this CTA's issued loads land before it can leave
+        for (int t = max(0, nk - DNS); t < nk; ++t) mbar_drain(&bar[D_KFULL + t % DNS], (t / DNS) & 1);
+        for (int t = max(0, j - DNS); t < j; ++t) mbar_drain(&bar[D_VFULL + t % DNS], (t / DNS) & 1);
       }
     }
     __syncwarp();
@@ -240,7 +241,7 @@ __global__ void __launch_bounds__(DTHREADS, 2)
         }
       }
       mma_commit(&bar[D_FINAL]);
-      mbar_wait(&bar[D_FINAL], 0, abort_flag, nullptr, 0);
+      mbar_drain(&bar[D_FINAL], 0);
     }
     __syncwarp();
   } else if (warp >= 4) {

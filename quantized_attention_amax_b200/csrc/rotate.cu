@@ -333,9 +333,9 @@ __global__ void __launch_bounds__(RTHREADS, 1)
       }
       if (*abort_flag) {
         // let loads already issued land before the CTA can exit
-        if (rload > 0) mbar_wait(&bar[RB_RF], (uint32_t)((rload - 1) & 1), abort_flag, nullptr, 0);
+        if (rload > 0) mbar_drain(&bar[RB_RF], (uint32_t)((rload - 1) & 1));
         for (long long t = (k >= 2 ? k - 2 : 0); t < k; ++t)
-          mbar_wait(&bar[RB_XF + (t & 1)], (uint32_t)((t >> 1) & 1), abort_flag, nullptr, 0);
+          mbar_drain(&bar[RB_XF + (t & 1)], (uint32_t)((t >> 1) & 1));
       }
     }
     __syncwarp();
@@ -375,7 +375,7 @@ __global__ void __launch_bounds__(RTHREADS, 1)
         if (tb) ++tuse1; else ++tuse0;
       }
       mma_commit(&bar[RB_FIN]);
-      mbar_wait(&bar[RB_FIN], 0, abort_flag, nullptr, 0);
+      mbar_drain(&bar[RB_FIN], 0);
     }
     __syncwarp();
   } else {

@@ -102,6 +102,18 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
   }
 }
 
+// Bounded wait that ignores the abort flag: for a CTA draining its own loads and MMAs already in
+// flight (whose phases complete by themselves) before it frees TMEM or leaves.  Gives up after
+// FAQ_WAIT_NS.
+__device__ __forceinline__ bool mbar_drain(uint64_t* bar, uint32_t parity) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  for (;;) {
+    if (mbar_try_wait_sleep(bar, parity, 200000u)) return true;
+    if (globaltimer_ns() - t0 > FAQ_WAIT_NS) return false;
+  }
+}
+
 // ------------------------------------------------------------------ TMA ---
 
 // Untiled bulk copy, global -> this CTA's shared memory, completing on `bar` (complete_tx).
