@@ -138,20 +138,21 @@ def test_no_visible_key_row(orc):
 def test_quantized_operands_dequantize_per_mode(orc):
     """Attention on quantized operands equals attention on their
     dequantization by hand (code * scale from the format tables)."""
-    x = wl.bf16_bits(wl.normal((1, 2, 64, 64), 19))
+    # B = 2 and H = 3, so that a (b, h) scale index taken as (h, b) lands elsewhere
+    x = wl.bf16_bits(wl.normal((2, 3, 64, 64), 19))
     am = orc.calibrate_per_head(x)
     ci, si = orc.quantize_int8_per_head(x, am)
     cf, sf = orc.quantize_fp8_per_token(x)
     cm, em = orc.quantize_mxfp4(x)
     cb, sb = orc.quantize_fp8_block(x, 16)
-    qi = orc.QT("int8_per_head", ci, si, 1, 2, 64, 64)
-    qf = orc.QT("fp8_per_token", cf, sf, 1, 2, 64, 64)
-    qm = orc.QT("mxfp4", cm, em, 1, 2, 64, 64)
-    qb = orc.QT("fp8_block", cb, sb, 1, 2, 64, 64, blk=16)
+    qi = orc.QT("int8_per_head", ci, si, 2, 3, 64, 64)
+    qf = orc.QT("fp8_per_token", cf, sf, 2, 3, 64, 64)
+    qm = orc.QT("mxfp4", cm, em, 2, 3, 64, 64)
+    qb = orc.QT("fp8_block", cb, sb, 2, 3, 64, 64, blk=16)
     by_hand = {
         "i": ci.astype(np.float64) * si[None, :, None, None],
         "f": orc.e4m3_decode(cf) * sf[..., None],
-        "m": orc.e2m1_decode(np.stack([cm & 15, cm >> 4], -1).reshape(1, 2, 64, 64))
+        "m": orc.e2m1_decode(np.stack([cm & 15, cm >> 4], -1).reshape(2, 3, 64, 64))
         * np.ldexp(1.0, np.repeat(em.astype(np.int64) - 127, 32, -1)),
         "b": orc.e4m3_decode(cb) * np.repeat(sb, 16, -1)[..., None],
     }

@@ -7,7 +7,7 @@ coincide."""
 import numpy as np
 
 import workloads as wl
-from test_oracle_quant import bf16_from_f32, bits_of, f32, to_bsnd
+from test_oracle_quant import bf16_from_f32, bits_of, f32, max_walk, to_bsnd
 
 
 # ------------------------------------------------------------ FP8 per head --
@@ -63,18 +63,20 @@ def test_fp8_per_head_grid_round_trip_and_saturation(orc):
 # ----------------------------------------------------------- INT8 per token --
 
 def test_int8_per_token_invariants(orc):
-    x = bits_of(wl.normal_k_outliers((2, 4, 96, 128), "BNSD", 4))
-    codes, sc = orc.quantize_int8_per_token(x)
-    xf = f32(orc, x)
-    assert sc.shape == (2, 4, 96)
-    idx = np.argmax(np.abs(xf), axis=-1)  # the largest |x| of each token codes to +-127
-    top = np.take_along_axis(codes, idx[..., None], -1)[..., 0]
-    assert (np.abs(top.astype(np.int32)) == 127).all()
-    deq = codes.astype(np.float64) * sc[..., None]
-    assert (np.abs(deq - xf) <= sc[..., None] * (0.5 + 127 * 2.0 ** -24)).all()
-    assert codes.min() >= -127  # symmetric: |x| <= amax never reaches -128
-    cb, sb = orc.quantize_int8_per_token(to_bsnd(x), "BSND")
-    assert np.array_equal(cb, to_bsnd(codes)) and np.array_equal(sb, sc)
+    # outlier channels, and a walk that puts each token's largest |x| on a channel from either end
+    for x in (bits_of(wl.normal_k_outliers((2, 4, 96, 128), "BNSD", 4)), max_walk((2, 4, 96, 128), 5)):
+        codes, sc = orc.quantize_int8_per_token(x)
+        xf = f32(orc, x)
+        assert sc.shape == (2, 4, 96)
+        assert np.array_equal(sc, np.abs(xf).max(axis=-1) / np.float32(127))  # s = amax_token / 127
+        idx = np.argmax(np.abs(xf), axis=-1)  # the largest |x| of each token codes to +-127
+        top = np.take_along_axis(codes, idx[..., None], -1)[..., 0]
+        assert (np.abs(top.astype(np.int32)) == 127).all()
+        deq = codes.astype(np.float64) * sc[..., None]
+        assert (np.abs(deq - xf) <= sc[..., None] * (0.5 + 127 * 2.0 ** -24)).all()
+        assert codes.min() >= -127  # symmetric: |x| <= amax never reaches -128
+        cb, sb = orc.quantize_int8_per_token(to_bsnd(x), "BSND")
+        assert np.array_equal(cb, to_bsnd(codes)) and np.array_equal(sb, sc)
 
 
 def test_int8_per_token_equals_per_head_when_every_token_reaches_the_head_max(orc):
@@ -111,12 +113,12 @@ def test_int8_per_token_grid_round_trip_and_zero_token(orc):
 
 
 def test_dequantize_new_modes_by_hand(orc):
-    x = wl.bf16_bits(wl.normal((1, 2, 64, 64), 35))
+    x = wl.bf16_bits(wl.normal((2, 3, 64, 64), 35))  # B = 2, H = 3: (b, h) and (h, b) indices differ
     am = orc.calibrate_per_head(x)
     ch, sh = orc.quantize_fp8_per_head(x, am)
     ct, st = orc.quantize_int8_per_token(x)
-    qh = orc.QT("fp8_per_head", ch, sh, 1, 2, 64, 64)
-    qt = orc.QT("int8_per_token", ct, st, 1, 2, 64, 64)
+    qh = orc.QT("fp8_per_head", ch, sh, 2, 3, 64, 64)
+    qt = orc.QT("int8_per_token", ct, st, 2, 3, 64, 64)
     assert np.array_equal(orc.dequant(qh), orc.e4m3_decode(ch) * sh[None, :, None, None].astype(np.float64))
     assert np.array_equal(orc.dequant(qt), ct.astype(np.float64) * st[..., None])
 

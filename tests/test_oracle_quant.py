@@ -6,6 +6,7 @@ import os
 
 import numpy as np
 import pytest
+import torch
 
 import workloads as wl
 
@@ -24,6 +25,18 @@ def to_bsnd(x):
     return np.ascontiguousarray(x.transpose(0, 2, 1, 3))
 
 
+def max_walk(shape, seed):
+    """bf16 bits of N(0,1) draws clipped to |x| <= 3.9, except that token t (the next-to-last
+    axis) holds +-8 on one channel, taken alternately from both ends of D (0, D-1, 1, D-2,
+    ...): the first and last channels hold some token's largest |x|, and nothing ties with it."""
+    x = wl.normal(shape, seed).float().clamp(-3.9, 3.9)
+    D = shape[-1]
+    t = torch.arange(shape[-2])
+    ch = torch.where(t % 2 == 0, (t // 2) % D, D - 1 - (t // 2) % D)
+    x[..., t, ch] = torch.where(t % 2 == 0, 8.0, -8.0)
+    return wl.bf16_bits(x.to(torch.bfloat16))
+
+
 def bf16_from_f32(a):
     """Exact bf16 bits of float32 values that are bf16-representable."""
     u = np.ascontiguousarray(a, dtype=np.float32).view(np.uint32)
@@ -36,6 +49,14 @@ def bf16_from_f32(a):
 def test_calibrate_running_max(orc):
     a = bits_of(wl.normal((2, 3, 40, 64), 1))
     b = bits_of(wl.normal((2, 3, 40, 64), 2))
+    # each head's largest |x| at an edge: head 0 in the last token of b's last batch entry,
+    # head 1 in the first token of b's first entry, head 2 in the first calibration batch a
+    bf = f32(orc, b).copy()
+    bf[1, 0, 39, 63] = -16.0
+    bf[0, 1, 0, 0] = 16.0
+    af = f32(orc, a).copy()
+    af[0, 2, 39, 5] = 16.0
+    a, b = bf16_from_f32(af), bf16_from_f32(bf)
     am = orc.calibrate_per_head(b, "BNSD", orc.calibrate_per_head(a, "BNSD"))
     both = np.abs(np.concatenate([f32(orc, a), f32(orc, b)], axis=2))
     assert np.array_equal(am, both.max(axis=(0, 2, 3)))
@@ -83,8 +104,10 @@ def test_int8_grid_round_trip_and_out_of_calibration(orc):
 
 # --------------------------------------------------------- FP8 per token --
 
-def test_fp8_per_token_invariants(orc):
-    x = bits_of(wl.normal_k_outliers((2, 4, 96, 128), "BNSD", 4))
+@pytest.mark.parametrize("walk", [False, True])
+def test_fp8_per_token_invariants(orc, walk):
+    # outlier channels, or a walk that puts each token's largest |x| on a channel from either end
+    x = max_walk((2, 4, 96, 128), 5) if walk else bits_of(wl.normal_k_outliers((2, 4, 96, 128), "BNSD", 4))
     codes, sc = orc.quantize_fp8_per_token(x)
     xf = f32(orc, x)
     amax = np.abs(xf).max(axis=-1)
