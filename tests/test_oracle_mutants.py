@@ -26,7 +26,8 @@ import test_oracle_codecs
 import test_oracle_modes_next
 import test_oracle_quant
 
-PIN_MODULES = [test_oracle_codecs, test_oracle_quant, test_oracle_modes_next, test_oracle_attention]
+# cheapest first: the exhaustive codec sweeps take most of the time
+PIN_MODULES = [test_oracle_attention, test_oracle_quant, test_oracle_modes_next, test_oracle_codecs]
 
 # (name, function whose body holds the mistake, original text, planted text)
 MUTANTS = [
@@ -90,6 +91,21 @@ MUTANTS = [
     ("fp8 per-token dequantized with [h, b, s] scales", "case ORC_MODE_FP8_PER_TOKEN:",
      "((const float*)t->scales)[((size_t)b * t->H + h) * t->S + s]",
      "((const float*)t->scales)[((size_t)h * t->B + b) * t->S + s]"),
+    ("fp8 block scales indexed [h, b, g]", "void orc_quantize_fp8_block(",
+     "scales[((size_t)b * H + h) * nblk + g] = sc;", "scales[((size_t)h * B + b) * nblk + g] = sc;"),
+    ("mxfp4 scales indexed [h, b, s]", "void orc_quantize_mxfp4(", "e8m0[(((size_t)b * H + h) * S + s) * G + g]",
+     "e8m0[(((size_t)h * B + b) * S + s) * G + g]"),
+    ("mxfp8 scales indexed [h, b, s]", "void orc_quantize_mxfp8(", "e8m0[(((size_t)b * H + h) * S + s) * G + g]",
+     "e8m0[(((size_t)h * B + b) * S + s) * G + g]"),
+    ("rotation rounded to bf16 through fp32", "void orc_rotate(const", "out[i] = orc_f64_to_bf16(tmp[i]);",
+     "out[i] = orc_f64_to_bf16((double)(float)tmp[i]);"),
+    ("e4m3 exponent bias 8", "uint8_t orc_e4m3_encode(", "((E + 7) << 3)", "((E + 8) << 3)"),
+    ("e8m0 byte e + 128", "void orc_quantize_mxfp4(", "(uint8_t)(e + 127)", "(uint8_t)(e + 128)"),
+    ("zero fp8 scale divides anyway", "void orc_quantize_fp8_per_token(",
+     "(sc > 0.0f) ? orc_e4m3_encode(xf / sc) : (uint8_t)0", "orc_e4m3_encode(xf / sc)"),
+    ("causal mask one key short", "void orc_attention(", "const int last = causal ? i + (Sk - Sq) : Sk - 1;",
+     "const int last = causal ? i + (Sk - Sq) - 1 : Sk - 1;"),
+    ("a row with no visible key divides by zero", "void orc_attention(", "if (nvis <= 0) {", "if (nvis < 0) {"),
 ]
 
 

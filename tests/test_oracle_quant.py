@@ -161,21 +161,21 @@ def test_fp8_zero_token(orc):
 
 def test_mxfp4_invariants(orc):
     assert GOLDEN["mxfp4_block_elems"]["value"] == 32
-    x = bits_of(wl.student_t4((1, 3, 50, 128), 5))
+    x = bits_of(wl.student_t4((2, 3, 50, 128), 5))
     codes, e8 = orc.quantize_mxfp4(x)
-    assert codes.shape == (1, 3, 50, 64) and e8.shape == (1, 3, 50, 4)
+    assert codes.shape == (2, 3, 50, 64) and e8.shape == (2, 3, 50, 4)
     xf = f32(orc, x).astype(np.float64)
-    blocks = xf.reshape(1, 3, 50, 4, 32)
+    blocks = xf.reshape(2, 3, 50, 4, 32)
     amax = np.abs(blocks).max(-1)
     e = e8.astype(np.int64) - 127
     # E8M0 exponent = floor(log2 amax) - emax, emax = 2
     assert np.array_equal(e, np.floor(np.log2(amax)).astype(np.int64) - GOLDEN["e2m1_emax"]["value"])
     lo, hi = codes & 15, codes >> 4
-    nib = np.stack([lo, hi], -1).reshape(1, 3, 50, 128)
+    nib = np.stack([lo, hi], -1).reshape(2, 3, 50, 128)
     deq = orc.e2m1_decode(nib) * np.ldexp(1.0, np.repeat(e, 32, axis=-1))
     # the block maximum codes to magnitude 4 or 6
     bmax_idx = np.argmax(np.abs(blocks), -1)
-    topcode = np.take_along_axis(nib.reshape(1, 3, 50, 4, 32), bmax_idx[..., None], -1)[..., 0] & 7
+    topcode = np.take_along_axis(nib.reshape(2, 3, 50, 4, 32), bmax_idx[..., None], -1)[..., 0] & 7
     assert np.isin(topcode, [6, 7]).all()
     # error bound: half a grid step, or saturation beyond 6
     v = np.abs(xf) / np.ldexp(1.0, np.repeat(e, 32, axis=-1))
@@ -211,18 +211,19 @@ def test_mxfp4_zero_block(orc):
 
 def test_fp8_block_invariants(orc):
     assert GOLDEN["q_block_tokens"]["value"] == 128 and GOLDEN["kv_block_tokens"]["value"] == 256
-    x = bits_of(wl.normal((1, 300, 3, 64), 6))  # BSND, ragged last block
+    x = bits_of(wl.normal((2, 300, 3, 64), 6))  # BSND, ragged last block, B = 2 and H = 3
     for blk in (128, 256):
         codes, sc = orc.quantize_fp8_block(x, blk, "BSND")
         nblk = -(-300 // blk)
-        assert sc.shape == (1, 3, nblk)
+        assert sc.shape == (2, 3, nblk)
         xf = f32(orc, x)  # [B, S, H, D]
-        for h in range(3):
-            for g in range(nblk):
-                blkx = xf[0, g * blk:(g + 1) * blk, h]
-                assert sc[0, h, g] == np.abs(blkx).max() / np.float32(448)
-                i = np.unravel_index(np.argmax(np.abs(blkx)), blkx.shape)
-                assert codes[0, g * blk:(g + 1) * blk, h][i] in (0x7E, 0xFE)
+        for b in range(2):
+            for h in range(3):
+                for g in range(nblk):
+                    blkx = xf[b, g * blk:(g + 1) * blk, h]
+                    assert sc[b, h, g] == np.abs(blkx).max() / np.float32(448)
+                    i = np.unravel_index(np.argmax(np.abs(blkx)), blkx.shape)
+                    assert codes[b, g * blk:(g + 1) * blk, h][i] in (0x7E, 0xFE)
         # a block of exactly one token per block is per-token quantization
     c1, s1 = orc.quantize_fp8_block(x, 1, "BSND")
     c2, s2 = orc.quantize_fp8_per_token(x, "BSND")
@@ -239,6 +240,13 @@ def test_rotate_matches_numpy_matmul(orc):
     assert np.allclose(got, ref, rtol=1e-12, atol=1e-12)
     # and the bf16 output is the nearest bf16 of that sum
     assert np.array_equal(orc.rotate(x, R), orc.f64_to_bf16(got))
+    # rounded once: 1 + 2^-8 + 2^-30 lies just above the midpoint of 1 and 1 + 2^-7 and rounds
+    # up, where a detour through fp32 (1 + 2^-8, a tie) would round to even, 1
+    xo = np.zeros((1, 1, 1, 64), np.float32)
+    xo[0, 0, 0, :3] = [1.0, 2.0 ** -8, 2.0 ** -30]
+    Ro = np.zeros((64, 64), np.float32)
+    Ro[:3, 0] = 1.0
+    assert f32(orc, orc.rotate(bf16_from_f32(xo), bf16_from_f32(Ro)))[0, 0, 0, 0] == 1.0 + 2.0 ** -7
     xb = to_bsnd(x)
     assert np.array_equal(orc.rotate(xb, R, "BSND"), to_bsnd(orc.rotate(x, R)))
 
