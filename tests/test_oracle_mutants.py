@@ -106,6 +106,16 @@ MUTANTS = [
     ("causal mask one key short", "void orc_attention(", "const int last = causal ? i + (Sk - Sq) : Sk - 1;",
      "const int last = causal ? i + (Sk - Sq) - 1 : Sk - 1;"),
     ("a row with no visible key divides by zero", "void orc_attention(", "if (nvis <= 0) {", "if (nvis < 0) {"),
+    ("sampled rows ignored", "void orc_attention(", "const int i = rows ? rows[r] : r;", "const int i = r;"),
+    ("fp8 per-head dequantized with head 0's scale", "case ORC_MODE_FP8_PER_HEAD:", "((const float*)t->scales)[h]",
+     "((const float*)t->scales)[0]"),
+    ("int8 per-head dequantized with head 0's scale", "case ORC_MODE_INT8_PER_HEAD:", "((const float*)t->scales)[h]",
+     "((const float*)t->scales)[0]"),
+    ("mxfp8 dequant exponent bias 128", "case ORC_MODE_MXFP8: {", "- 127;", "- 128;"),
+    ("fp8 block dequantized with the next block's scale", "case ORC_MODE_FP8_BLOCK: {", "nblk + s / t->blk]",
+     "nblk + (s / t->blk + 1) % nblk]"),
+    ("float branch reads the neighbouring element", "case ORC_MODE_FLOAT:", "((const uint16_t*)t->codes)[i]",
+     "((const uint16_t*)t->codes)[i ^ 1]"),
 ]
 
 
