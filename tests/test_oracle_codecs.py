@@ -239,3 +239,33 @@ def test_f64_to_bf16_nearest_by_search(orc):
     pick = np.where(a == grid[i], i, pick)
     expect = bits[pick].astype(np.uint16) | np.where(np.signbit(v), 0x8000, 0).astype(np.uint16)
     assert np.array_equal(got, expect)
+
+
+# ------------------------------------------------------- non-finite values --
+# The method's inputs are finite, but the codecs' edges are part of their definitions:
+# IEEE round-to-nearest carries bf16 past the largest finite value to infinity; E4M3
+# (float8_e4m3fn) has no infinity, saturates finite values at 448 and keeps NaN as
+# S.1111.111; E2M1 has neither infinity nor NaN and saturates at 6; INT8 clamps to
+# [-128, 127] and takes NaN to 0.
+
+def test_bf16_rounds_past_the_largest_finite_value_to_infinity(orc):
+    top = float((np.uint32(0x7F7F) << 16).view(np.float32))  # largest finite bf16, odd mantissa
+    mid = (top + 2.0 ** 128) / 2                              # the tie goes to the even side: infinity
+    got = orc.f64_to_bf16(np.array([top, mid, np.nextafter(mid, 0), 1e39, -1e39, -mid, np.inf, -np.inf]))
+    assert got.tolist() == [0x7F7F, 0x7F80, 0x7F7F, 0x7F80, 0xFF80, 0xFF80, 0x7F80, 0xFF80]
+
+
+def test_e4m3_non_finite(orc):
+    got = orc.e4m3_encode(np.array([np.inf, -np.inf, np.nan, 1e30, -1e30], np.float32))
+    assert got.tolist() == [0x7E, 0xFE, 0x7F, 0x7E, 0xFE]
+    assert np.isnan(orc.e4m3_decode(np.array([0x7F, 0xFF], np.uint8))).all()
+
+
+def test_e2m1_non_finite(orc):
+    got = orc.e2m1_encode(np.array([np.inf, -np.inf, 1e30, -1e30], np.float32))
+    assert got.tolist() == [7, 15, 7, 15]
+
+
+def test_int8_non_finite(orc):
+    got = orc.int8_encode(np.array([np.inf, -np.inf, np.nan], np.float32))
+    assert got.tolist() == [127, -128, 0]

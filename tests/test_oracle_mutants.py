@@ -116,6 +116,19 @@ MUTANTS = [
      "nblk + (s / t->blk + 1) % nblk]"),
     ("float branch reads the neighbouring element", "case ORC_MODE_FLOAT:", "((const uint16_t*)t->codes)[i]",
      "((const uint16_t*)t->codes)[i ^ 1]"),
+    ("bf16 overflow saturates instead of rounding to infinity", "uint16_t orc_f64_to_bf16(", "bits = 0x7F80;",
+     "bits = 0x7F7F;"),
+    ("e4m3 NaN encoded as 448", "uint8_t orc_e4m3_encode(", "if (isnan(v)) return 0x7F;", "if (isnan(v)) return 0x7E;"),
+    ("e2m1 infinity encoded as 0", "uint8_t orc_e2m1_encode(", "if (isnan(a) || isinf(a)) a = 6.0;",
+     "if (isnan(a) || isinf(a)) a = 0.0;"),
+    ("int8 NaN encoded as 127", "int8_t orc_int8_encode(", "if (isnan(v)) return 0;", "if (isnan(v)) return 127;"),
+    ("calibration without the absolute value", "void orc_calibrate_per_head(",
+     "const float a = fabsf(orc_bf16_to_f32(", "const float a = (orc_bf16_to_f32("),
+    ("e4m3 sign dropped", "uint8_t orc_e4m3_encode(", "return (uint8_t)(code | (neg ? 0x80u : 0u));",
+     "return (uint8_t)code;"),
+    ("e2m1 loses the sign of -0", "uint8_t orc_e2m1_encode(", "const int neg = signbit(v) ? 1 : 0;",
+     "const int neg = v < 0.0f ? 1 : 0;"),
+    ("rotation accumulated in fp32", "void orc_rotate_f64(", "double acc = 0.0;", "float acc = 0.0f;"),
 ]
 
 
