@@ -59,6 +59,17 @@ def test_attention_matches_naive_loops(orc, causal, Sq, Sk, Hq, Hkv):
     assert np.allclose(lse, rlse, rtol=1e-12, atol=1e-12)
 
 
+def test_caller_softmax_scale_matches_naive_loops(orc):
+    # a positive scale replaces the default 1/sqrt(D) (FlashAttention's softmax_scale)
+    D = 4
+    q, k, v = rand_bf16((1, 2, 5, D), 4), rand_bf16((1, 1, 9, D), 5), rand_bf16((1, 1, 9, D), 6)
+    for scale in (0.37, 2.0):
+        out, lse = orc.attention(qt_f64_exact(orc, q), qt_f64_exact(orc, k), qt_f64_exact(orc, v), True, scale)
+        ref, rlse = naive(q, k, v, True, scale)
+        assert np.allclose(out, ref, rtol=1e-12, atol=1e-12)
+        assert np.allclose(lse, rlse, rtol=1e-12, atol=1e-12)
+
+
 @pytest.mark.parametrize("causal", [False, True])
 def test_attention_matches_torch_sdpa_fp64(orc, causal):
     B, Hq, Hkv, Sq, Sk, D = 2, 8, 2, 37, 53, 64

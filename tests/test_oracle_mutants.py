@@ -129,6 +129,14 @@ MUTANTS = [
     ("e2m1 loses the sign of -0", "uint8_t orc_e2m1_encode(", "const int neg = signbit(v) ? 1 : 0;",
      "const int neg = v < 0.0f ? 1 : 0;"),
     ("rotation accumulated in fp32", "void orc_rotate_f64(", "double acc = 0.0;", "float acc = 0.0f;"),
+    ("caller's softmax scale ignored", "void orc_attention(", "if (scale <= 0.0) scale = 1.0 / sqrt((double)D);",
+     "scale = 1.0 / sqrt((double)D);"),
+    ("lse written to the mirrored row", "void orc_attention(",
+     "lse[((size_t)b * Hq + h) * nrows + r] = m + log(l);", "lse[((size_t)b * Hq + h) * nrows + (nrows - 1 - r)] = m + log(l);"),
+    ("calibration reads the first batch entry only", "void orc_calibrate_per_head(", "for (int b = 0; b < B; ++b)",
+     "for (int b = 0; b < 1; ++b)"),
+    ("mxfp4 odd elements coded from the even one", "void orc_quantize_mxfp4(",
+     "x[elem_index(layout, H, S, D, b, h, s, d + 1)]", "x[elem_index(layout, H, S, D, b, h, s, d)]"),
 ]
 
 
