@@ -121,8 +121,8 @@ __global__ void __launch_bounds__(DTHREADS, 2)
   float* red = reinterpret_cast<float*>(smem + L::RED);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int split = blockIdx.x;
-  const int bhk = blockIdx.y;
+  const int split = blockIdx.y;
+  const int bhk = blockIdx.x;
   const int b = bhk / p.Hkv, hk = bhk % p.Hkv;
   const int key0 = split * p.chunk;
   const int key1 = min(p.Sk, key0 + p.chunk);
@@ -458,13 +458,11 @@ cudaError_t make_map(CUtensorMap* map, const void* base, int B, int H, int S, in
 template <int D, int G>
 cudaError_t launch_dec(const CUtensorMap& mk, const CUtensorMap& mv, const DecParams& prm, cudaStream_t s) {
   auto kern = decode_kernel<D, G>;
-  static bool attr = false;
-  if (!attr) {
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, DSmem<D>::ALLOC);
-    if (e != cudaSuccess) return e;
-    attr = true;
-  }
-  dim3 grid((unsigned)prm.splits, (unsigned)(prm.B * prm.Hkv));
+  cudaError_t e = set_smem_limit(reinterpret_cast<const void*>(kern), DSmem<D>::ALLOC);
+  if (e != cudaSuccess) return e;
+  // (b, kv head) on x (up to 2^31 - 1), the split on y (at most 256)
+  if ((long long)prm.B * prm.Hkv > 0x7FFFFFFFLL || prm.splits > 65535) return cudaErrorNotSupported;
+  dim3 grid((unsigned)(prm.B * prm.Hkv), (unsigned)prm.splits);
   kern<<<grid, DTHREADS, DSmem<D>::ALLOC, s>>>(mk, mv, prm);
   return cudaGetLastError();
 }

@@ -44,6 +44,7 @@ void* scratch_on_current_device() {
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
 
 }  // namespace
 }  // namespace faq
@@ -59,15 +60,22 @@ extern "C" fa_status fa_attention_decode_noalloc(const fa_qtensor* q, const fa_q
   if (q->layout != k->layout || q->layout != v->layout ||
       (q->layout != FA_LAYOUT_BNSD && q->layout != FA_LAYOUT_BSND))
     return FA_ERR_INVALID_ARG;
-  if (q->B < 1 || k->H < 1 || k->S < 1 || q->H % k->H != 0) return FA_ERR_INVALID_ARG;
+  if (q->B < 0 || k->S < 0 || q->H < 1 || k->H < 1 || q->H % k->H != 0) return FA_ERR_INVALID_ARG;
   if (q->B != k->B || q->B != v->B || k->H != v->H || k->S != v->S) return FA_ERR_INVALID_ARG;
   const int group = q->H / k->H;
   if (!(group == 1 || group == 2 || group == 4 || group == 8 || group == 16)) return FA_ERR_UNSUPPORTED;
   if (num_splits < 0) return FA_ERR_INVALID_ARG;
-  if (!q->codes || !q->scales || !k->codes || !k->scales || !v->codes || !v->scales) return FA_ERR_INVALID_ARG;
-  if (!aligned16(q->codes) || !aligned16(k->codes) || !aligned16(v->codes)) return FA_ERR_INVALID_ARG;
+  // no query rows: nothing to do (as fa_attention_quant)
+  if (q->B == 0) return FA_OK;
+  if (!q->codes || !q->scales || !aligned16(q->codes) || !aligned4(q->scales)) return FA_ERR_INVALID_ARG;
   if (!out || !aligned16(out)) return FA_ERR_INVALID_ARG;
-  if (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)) return FA_ERR_INVALID_ARG;
+  if (lse && !aligned4(lse)) return FA_ERR_INVALID_ARG;
+  cudaStream_t cs = reinterpret_cast<cudaStream_t>(s);
+  // no key: every row's output is 0 and its LSE -inf (as fa_attention_quant)
+  if (k->S == 0) return launch_fill_empty_rows(out, lse, (long long)q->B * q->H, q->D, cs) == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+  if (!k->codes || !k->scales || !v->codes || !v->scales) return FA_ERR_INVALID_ARG;
+  if (!aligned16(k->codes) || !aligned16(v->codes) || !aligned4(k->scales) || !aligned4(v->scales))
+    return FA_ERR_INVALID_ARG;
 
   // Split count: the caller's, else the automatic choice reduced until the
   // partials fit the fixed buffer.
@@ -83,7 +91,7 @@ extern "C" fa_status fa_attention_decode_noalloc(const fa_qtensor* q, const fa_q
   int* status = device_status_ptr();
   if (!scratch || !status) return FA_ERR_CUDA;
   AttnArgs a = {q, k, v, 0, softmax_scale, out, lse, status};
-  const cudaError_t e = launch_attention_decode(a, splits, scratch, reinterpret_cast<cudaStream_t>(s));
+  const cudaError_t e = launch_attention_decode(a, splits, scratch, cs);
   if (e == cudaErrorNotSupported) return FA_ERR_UNSUPPORTED;
   return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }

@@ -4,6 +4,8 @@
 #include <string.h>
 
 #include <mutex>
+#include <set>
+#include <utility>
 
 #include "internal.cuh"
 
@@ -49,6 +51,19 @@ int sm_count() {
     cache[dev] = n > 0 ? n : 148;
   }
   return cache[dev];
+}
+
+cudaError_t set_smem_limit(const void* kernel, int bytes) {
+  static std::mutex mu;
+  static std::set<std::pair<const void*, int>> done;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  std::lock_guard<std::mutex> lock(mu);
+  if (done.count({kernel, dev})) return cudaSuccess;
+  if ((e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes)) != cudaSuccess) return e;
+  done.insert({kernel, dev});
+  return cudaSuccess;
 }
 
 namespace {
@@ -107,7 +122,10 @@ fa_status check_qtensor(const fa_qtensor* t) {
   if (t->B < 0 || t->H < 1 || t->S < 0 || !valid_layout(t->layout)) return FA_ERR_INVALID_ARG;
   if (t->D != 64 && t->D != 128) return FA_ERR_UNSUPPORTED;
   if (t->mode == FA_MODE_FP8_BLOCK && t->block_tokens < 1) return FA_ERR_INVALID_ARG;
-  if ((long long)t->B * t->S > 0 && (!t->codes || !t->scales || !aligned16(t->codes))) return FA_ERR_INVALID_ARG;
+  // codes 16-byte aligned (TMA); scales (fp32, or E8M0 bytes read four at a time) 4-byte aligned
+  if ((long long)t->B * t->S > 0 &&
+      (!t->codes || !t->scales || !aligned16(t->codes) || (reinterpret_cast<uintptr_t>(t->scales) & 3u)))
+    return FA_ERR_INVALID_ARG;
   return FA_OK;
 }
 

@@ -33,6 +33,10 @@ EncodeTiledFn encode_tiled_fn();
 // Number of SMs of the current device (cached).
 int sm_count();
 
+// Raise a kernel's dynamic shared memory limit to `bytes` on the current device.  The attribute
+// belongs to one device, so it is set once per (kernel, device) pair, under a lock.
+cudaError_t set_smem_limit(const void* kernel, int bytes);
+
 // Launchers (quant.cu).
 cudaError_t launch_calibrate(const QuantOperand& op, float* amax, cudaStream_t s);
 cudaError_t launch_quantize_rows(int mode, const QuantOperand* ops, int nops, cudaStream_t s);

@@ -591,12 +591,9 @@ cudaError_t launch_rotate_block_quant(const RotateOperand* ops, int nops, int* s
   prm.items = total;
   if (n == 0) return cudaSuccess;
   if (total > 0x7FFFFFFFLL) return cudaErrorInvalidValue;  // item indices stay below 2^31
-  static bool attr = false;
-  if (!attr) {
-    cudaError_t e = cudaFuncSetAttribute(rotate_block_quant_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         RSmem::ALLOC);
+  {
+    const cudaError_t e = set_smem_limit(reinterpret_cast<const void*>(rotate_block_quant_kernel), RSmem::ALLOC);
     if (e != cudaSuccess) return e;
-    attr = true;
   }
   const long long grid = total < sm_count() ? total : sm_count();
   rotate_block_quant_kernel<<<(unsigned)grid, RTHREADS, RSmem::ALLOC, s>>>(

@@ -161,6 +161,36 @@ def test_attention_validation_before_launch(N):
     qm64, km64 = _q(N, 3, B=2, H=4, S=100, D=64), _q(N, 3, B=2, H=2, S=1000, D=64)
     assert L.fa_attention_workspace_size(by(qm64), by(km64), 0) == 0
     assert L.fa_attention_quant(by(qm64), by(km64), by(km64), 0, 0.0, 0x60000, None, 0, None, 0, None) == 2
+    # scales that are not 4-byte aligned are rejected on the host, for every operand and mode
+    for m in (1, 2, 3, 4, 5, 6, 7):
+        blk = 256 if m == 4 else 0
+        qa = _q(N, m, B=2, H=4, S=100, D=128, blk=blk)
+        ka = _q(N, m, B=2, H=2, S=1000, D=128, blk=blk)
+        kmis = _q(N, m, B=2, H=2, S=1000, D=128, blk=blk, scales=0x30002)
+        qmis = _q(N, m, B=2, H=4, S=100, D=128, blk=blk, scales=0x30001)
+        assert L.fa_attention_quant(by(qa), by(kmis), by(ka), 0, 0.0, 0x60000, None, 0, 0x70000, 1 << 40, None) == 1
+        assert L.fa_attention_quant(by(qa), by(ka), by(kmis), 0, 0.0, 0x60000, None, 0, 0x70000, 1 << 40, None) == 1
+        assert L.fa_attention_quant(by(qmis), by(ka), by(ka), 0, 0.0, 0x60000, None, 0, 0x70000, 1 << 40, None) == 1
+
+
+def test_noalloc_validation_before_launch(N):
+    """The allocation-free decode checks its arguments like fa_attention_quant: misaligned scales
+    are rejected before any launch, and a batch of zero is a successful no-op."""
+    L = N.lib()
+    by = ctypes.byref
+    qd = _q(N, 1, B=2, H=4, S=1, D=128)
+    kd = _q(N, 1, B=2, H=2, S=1000, D=128)
+    for bad in (_q(N, 1, B=2, H=2, S=1000, D=128, scales=0x30002),):
+        assert L.fa_attention_decode_noalloc(by(qd), by(bad), by(kd), 0.0, 0x60000, None, 0, None) == 1
+        assert L.fa_attention_decode_noalloc(by(qd), by(kd), by(bad), 0.0, 0x60000, None, 0, None) == 1
+    qmis = _q(N, 1, B=2, H=4, S=1, D=128, scales=0x30001)
+    assert L.fa_attention_decode_noalloc(by(qmis), by(kd), by(kd), 0.0, 0x60000, None, 0, None) == 1
+    assert L.fa_attention_decode_noalloc(by(qd), by(kd), by(kd), 0.0, 0x60008, None, 0, None) == 1  # out
+    q0, k0 = _q(N, 1, B=0, H=4, S=1, D=128), _q(N, 1, B=0, H=2, S=1000, D=128)
+    assert L.fa_attention_decode_noalloc(by(q0), by(k0), by(k0), 0.0, None, None, 0, None) == 0
+    assert L.fa_attention_decode_noalloc(by(qd), by(kd), by(kd), 0.0, 0x60000, None, -1, None) == 1
+    # partials beyond the fixed buffer: B * Hq * splits * (D + 2) * 4 bytes > 16 MiB
+    assert L.fa_attention_decode_noalloc(by(qd), by(kd), by(kd), 0.0, 0x60000, None, 5000, None) == 7
 
 
 def test_mixed_branch_validation_and_workspace(N):
