@@ -38,10 +38,12 @@ __device__ __forceinline__ void fadd2(float& a0, float& a1, float b0, float b1) 
 
 // 2^x for a pair on the FMA pipe (takes load off the MUFU unit, which runs ex2
 // at a quarter of the FMA rate): x = n + f with n = rint(x), f in [-0.5, 0.5];
-// 2^f from a cubic fitted here for least maximum relative error on that interval
-// (Lawson's reweighted least squares), 7.5e-5 relative error in fp32 -- below
-// half an fp16 ulp, the precision P' is stored in; 2^n enters through the
-// exponent field.  x is clamped at -126: p(f) >= 2^-0.5 has a biased exponent of
+// 2^f from a cubic fitted for least maximum relative error on that interval
+// (Lawson's iteratively reweighted least squares, C. L. Lawson, "Contributions to
+// the theory of linear least maximum approximation", 1961; the fit and its fp32
+// error check are fit_ex2_cubic.py beside this file), 7.5e-5 relative error in
+// fp32 -- below half an fp16 ulp, the precision P' is stored in; 2^n enters
+// through the exponent field.  x is clamped at -126: p(f) >= 2^-0.5 has a biased exponent of
 // at least 126, so n >= -126 never borrows past the exponent field (the result
 // for x <= -126 is a denormal, read as 0 downstream).
 __device__ __forceinline__ void ex2_poly2(float& a, float& b) {

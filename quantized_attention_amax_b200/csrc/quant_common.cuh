@@ -7,7 +7,11 @@ namespace faq {
 
 // x / s rounded to fp32 as IEEE division does, for an FP8 scale s = fl(amax / 448) with
 // s >= kFastDivMin and a bf16 |x| <= amax: q0 = x * r with r the correctly rounded 1 / s, then one
-// FMA for the negated residual q0 * s - x (exact) and one FMA correction q0 - that * r.  Taking the
+// FMA for the negated residual q0 * s - x (exact) and one FMA correction q0 - that * r.  This is
+// the FMA-based quotient correction published by P. Markstein ("Computation of elementary
+// functions on the IBM RISC System/6000 processor", IBM J. Res. Dev. 34(1), 1990; and "IA-64 and
+// Elementary Functions", 2000): given the correctly rounded reciprocal, one residual and one
+// correction step round the quotient as the division would.  Taking the
 // residual negated keeps the sign of a zero x (-0 gives -0 where x - q0 * s would give +0); for a
 // nonzero result the two forms round identically, the sign flips being exact.
 // Its E4M3 codes equal those of IEEE division for every bf16 amax whose scale reaches kFastDivMin
