@@ -447,17 +447,31 @@ def e2e_run(args, w, device, steps):
 
 # --------------------------------------------------------- oracle / CPU ---
 
+def sample_rows(w, n=256, seed=0):
+    """Query rows of the oracle's sample: the first and last rows, the tile boundaries
+    127/128/255/256, and seeded random rows up to n (all rows when Sq <= n)."""
+    import numpy as np
+    if w.Sq <= n:
+        return list(range(w.Sq))
+    fixed = [r for r in (0, 127, 128, 255, 256, w.Sq - 1) if r < w.Sq]
+    rest = [r for r in np.random.default_rng(seed).permutation(w.Sq).tolist() if r not in fixed]
+    return sorted(fixed + rest[:n - len(fixed)])
+
+
 def oracle_sample(w, reps_seconds=None):
     """The oracle on a bounded sample of the workload: quantize one GQA group
-    (its query heads' last 64 rows of batch 0 and the kv head's full K/V)
-    and attention for those 64 query rows per head.  Returns
-    (seconds per sample, FLOPs or bytes per sample, description)."""
+    (batch 0, kv head 0 and its query heads: the whole Q/K/V of the group)
+    and attention for 256 sampled query rows of each of its heads (every row
+    when the sequence is shorter).  Rows are independent, so the sample's
+    time extrapolates to the whole workload by its share of the unmasked
+    (query, key) pairs.  Returns (run_once, FLOPs or bytes per sample,
+    description, full-workload work / sample work)."""
     import numpy as np
     import oracle as orc
     import workloads as wl
 
     G = w.Hq // w.Hkv
-    rows = list(range(max(0, w.Sq - 64), w.Sq))
+    rows = sample_rows(w)
     sub = w.scaled(B=1, Hq=G, Hkv=1)
     inp = wl.make_inputs(sub, calib=(w.mode in STATIC_MODES))
     qb = wl.bf16_bits(inp["q"])
@@ -505,19 +519,22 @@ def oracle_sample(w, reps_seconds=None):
         return time.perf_counter() - t0
 
     diag = w.Sk - w.Sq
-    pairs = sum((min(w.Sk, i + diag + 1) if w.causal else w.Sk) for i in rows) * G
+    pairs = sum((max(0, min(w.Sk, i + diag + 1)) if w.causal else w.Sk) for i in rows) * G
     work = 4.0 * w.D * pairs
+    full = attn_flops(w)
     if w.name == "int8_decode":
         work = 2.0 * w.Sk * w.D  # KV bytes of one kv head
+        full = decode_bytes(w)
     desc = (f"one GQA group (batch 0, kv head 0, its {G} query heads): quantize its Q/K/V "
-            f"({'rotate + ' if Rb is not None else ''}{w.mode}) and attention for query rows "
-            f"{rows[0]}..{rows[-1]} of each head")
-    return run_once, work, desc
+            f"({'rotate + ' if Rb is not None else ''}{w.mode}) and attention for {len(rows)} query rows "
+            f"of each head (rows 0, 127, 128, 255, 256, {w.Sq - 1} and seeded random rows); the rate "
+            f"extrapolates to the whole workload by its unmasked (query, key) pairs")
+    return run_once, work, desc, full / work
 
 
 def cpu_baseline(w, seconds=8.0):
     import oracle as orc
-    run_once, work, desc = oracle_sample(w)
+    run_once, work, desc, scale = oracle_sample(w)
     run_once()  # builds the oracle, warms caches
     ts = []
     t_end = time.perf_counter() + seconds
@@ -527,12 +544,13 @@ def cpu_baseline(w, seconds=8.0):
     unit = "GB/s" if w.name == "int8_decode" else "TFLOP/s"
     val = work / per / (1e9 if unit == "GB/s" else 1e12)
     return {"value": val, "unit": unit, "cores": orc.num_threads(), "kind": "oracle", "sample": desc,
-            "seconds_per_sample": per, "samples": len(ts)}
+            "seconds_per_sample": per, "samples": len(ts),
+            "extrapolated_step_s": per * scale, "extrapolated": True}
 
 
 def reference_arm(args, w):
     import oracle as orc
-    run_once, work, desc = oracle_sample(w)
+    run_once, work, desc, scale = oracle_sample(w)
     for _ in range(max(args.warmup, 0)):
         run_once()
     ts = [run_once() for _ in range(args.steps)]
@@ -544,7 +562,8 @@ def reference_arm(args, w):
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64 (oracle)",
             "data": DATA[w.name], "config": {"workload": f"{w.name}: {DESCR[w.name]}", "sample": desc},
             "cpu_baseline": {"value": val, "unit": unit, "cores": orc.num_threads(), "kind": "oracle",
-                             "sample": desc},
+                             "sample": desc, "extrapolated_step_s": total / args.steps * scale,
+                             "extrapolated": True},
             "e2e": {"value": val, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
