@@ -10,7 +10,9 @@ quantize), then attention on the low-bit operands.  The default workload is
 the FP8 E4M3 per-token LLM prefill (B=2, Hq=32, Hkv=8, S=4096, D=128,
 causal, GQA, BNSD); --workload picks another (int8_tiny, rot_fp8_block,
 mxfp4, int8_decode).  Each step is a CUDA-graph replay timed with CUDA
-events on its stream, with L2 flushed (a 256 MiB write) between steps.
+events on its stream, with L2 flushed between steps (a 256 MiB write, then a
+256 MiB read so that no dirty line of the flush is left for the timed kernels
+to write back).
 Prints one JSON line (rank 0).  Under torchrun every rank runs its own
 independent replica of the workload (weak scaling, no data-path collective);
 time is the max over ranks.
@@ -255,6 +257,23 @@ def make_step(faq, wl, w, device, seed_offset=0):
     return step, attn, quant, st
 
 
+class L2Flush:
+    """Flush L2 between timed steps: write a buffer larger than L2 (126 MB), then read
+    another one, so the next step starts with none of its inputs in L2 and without the
+    write's dirty lines, which the timed kernels would otherwise write back to HBM."""
+
+    def __init__(self, device):
+        import torch
+        self.w = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
+        self.r = torch.ones(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=device)
+        self.sink = torch.empty((), dtype=torch.float32, device=device)
+
+    def __call__(self):
+        import torch
+        self.w.zero_()
+        torch.sum(self.r, dim=0, out=self.sink)
+
+
 def launches_per_step(w):
     """This library's kernels per step: the quantize (or rotate + quantize) launch, then
     the attention call: decode + LSE combine, or for prefill the V' pre-pass and the
@@ -300,7 +319,7 @@ def gpu_run(args, w, rank, world, device):
 
     torch.cuda.set_device(device)
     step, attn, quant, st = make_step(faq, wl, w, device, seed_offset=rank)
-    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
+    flush = L2Flush(device)
     stream = torch.cuda.current_stream()
     for _ in range(max(args.warmup, 3)):
         step()
@@ -320,7 +339,7 @@ def gpu_run(args, w, rank, world, device):
     with torch.cuda.graph(ga):
         attn()
     for _ in range(max(args.warmup, 3)):
-        flush.zero_()
+        flush()
         gq.replay()
         ga.replay()
     torch.cuda.synchronize()
@@ -343,7 +362,7 @@ def gpu_run(args, w, rank, world, device):
     time.sleep(0.25)
     t0 = time.perf_counter()
     for i in range(K):
-        flush.zero_()
+        flush()
         ev[i][0].record(stream)
         gq.replay()
         ev[i][1].record(stream)
@@ -596,11 +615,11 @@ def decode_append_run(w, device, steps):
     torch.cuda.current_stream().wait_stream(s)
     with torch.cuda.graph(g):
         fn()
-    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
+    flush = L2Flush(device)
     stream = torch.cuda.current_stream()
     ms = []
     for i in range(steps + 3):
-        flush.zero_()
+        flush()
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record(stream)
         g.replay()
@@ -738,7 +757,8 @@ def main():
             "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": DTYPE[w.name], "data": DATA[w.name],
             "config": {"workload": f"{w.name}: {DESCR[w.name]}",
-                       "l2": "flushed between steps (256 MiB device write, outside the timed events)",
+                       "l2": "flushed between steps (256 MiB device write, then a 256 MiB read so no dirty "
+                             "line of the flush is left; outside the timed events)",
                        "timing": "CUDA-graph replay per launch, CUDA events on the launch stream",
                        "parallelism": f"replicas x{world} (independent workloads per rank)"},
             "kernels_ms": {"quantize": r["quant_ms"], "attention": r["attn_ms"]},

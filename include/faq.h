@@ -176,6 +176,30 @@ FAQ_API fa_status fa_rotate_quantize(const fa_tensor* q, const fa_tensor* k, con
                              fa_qtensor* v_out, void* rot_q_dbg, void* rot_k_dbg, fa_stream_t s);
 
 /*
+ * fa_rotate_quantize_hadamard -- fa_rotate_quantize for rotations of the
+ * Hadamard-times-signs form, by a fast Walsh-Hadamard transform instead of a
+ * D x D product (the rotation specialization of the same flow).
+ *   Source: MindIE SD "量化", FA量化 / 技术特点: 旋转 (Q and K multiplied by a
+ *   rotation before 块量化), with the rotation R = bf16(H_D diag(sigma) /
+ *   sqrt(D)): H_D the Sylvester Hadamard matrix, entry (i, j) =
+ *   (-1)^popcount(i & j), and sigma a vector of signs.  Every entry of R is
+ *   +-c with c = bf16(1 / sqrt(D)), so x R = c * sigma * FWHT(x) elementwise,
+ *   FWHT(x)_j = sum_d x_d (-1)^popcount(d & j).  The rotated row is evaluated
+ *   in fp32 and rounded once to bf16, then quantized exactly as
+ *   fa_rotate_quantize does (FA_MODE_FP8_BLOCK); the results equal those of
+ *   fa_rotate_quantize given that R up to the order of the fp32 sums.
+ *   sign_bits_q, sign_bits_k: HOST pointers to D / 32 words; bit j % 32 of
+ *   word j / 32 set means sigma_j = -1; NULL means every sigma_j = +1.
+ *   Everything else (q_block, kv_block, outputs, the nullable rot_*_dbg
+ *   outputs, layouts, errors) as fa_rotate_quantize, without R pointers.
+ *   Any block size >= 1 is accepted.
+ */
+FAQ_API fa_status fa_rotate_quantize_hadamard(const fa_tensor* q, const fa_tensor* k, const fa_tensor* v,
+                                              const uint32_t* sign_bits_q, const uint32_t* sign_bits_k,
+                                              int q_block, int kv_block, fa_qtensor* q_out, fa_qtensor* k_out,
+                                              fa_qtensor* v_out, void* rot_q_dbg, void* rot_k_dbg, fa_stream_t s);
+
+/*
  * fa_attention_quant -- flash attention on quantized Q/K/V, bf16 output.
  *   Sources: MindIE SD "量化", FA量化 / FP8 Attention (attention computed
  *   on the low-bit operands, the output dequantized back to the original

@@ -8,9 +8,9 @@ include/faq.h (libfaq.so).  This package is the thin ctypes binding.
 """
 from .api import (LAYOUTS, MODES, FaqError, QTensor, attention, attention_workspace_size, calibrate_per_head,
                   check_device_status, decode_append, dims, empty_qtensor, float_branch, quantize, resolve_config,
-                  rotate_quantize, version)
+                  rotate_quantize, rotate_quantize_hadamard, version)
 
 __all__ = ["LAYOUTS", "MODES", "FaqError", "QTensor", "attention", "attention_workspace_size",
            "calibrate_per_head", "check_device_status", "decode_append", "dims", "empty_qtensor", "float_branch",
            "quantize",
-           "resolve_config", "rotate_quantize", "version"]
+           "resolve_config", "rotate_quantize", "rotate_quantize_hadamard", "version"]

@@ -16,6 +16,7 @@ EXPORTS = (
     "fa_calibrate_per_head",
     "fa_quantize",
     "fa_rotate_quantize",
+    "fa_rotate_quantize_hadamard",
     "fa_attention_quant",
     "fa_attention_workspace_size",
     "fa_attention_workspace_size_qkv",
@@ -65,6 +66,7 @@ def lib() -> ctypes.CDLL:
     L.fa_calibrate_per_head.argtypes = [pT, P, P]
     L.fa_quantize.argtypes = [pT, pT, pT, I, P, P, P, pQ, pQ, pQ, P]
     L.fa_rotate_quantize.argtypes = [pT, pT, pT, P, P, I, I, pQ, pQ, pQ, P, P, P]
+    L.fa_rotate_quantize_hadamard.argtypes = [pT, pT, pT, P, P, I, I, pQ, pQ, pQ, P, P, P]
     L.fa_attention_quant.argtypes = [pQ, pQ, pQ, I, F, P, P, I, P, S, P]
     L.fa_attention_decode_noalloc.argtypes = [pQ, pQ, pQ, F, P, P, I, P]
     L.fa_attention_decode_noalloc.restype = I
@@ -81,6 +83,7 @@ def lib() -> ctypes.CDLL:
     L.fa_status_str.restype = ctypes.c_char_p
     L.fa_version.restype = ctypes.c_char_p
     for name in ("fa_resolve_config", "fa_calibrate_per_head", "fa_quantize", "fa_rotate_quantize",
+                 "fa_rotate_quantize_hadamard",
                  "fa_attention_quant", "fa_check_device_status"):
         getattr(L, name).restype = I
     _lib = L

@@ -194,6 +194,43 @@ def rotate_quantize(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, rot_q: to
     return tuple(outs) + ((dq, dk) if debug else ())
 
 
+def rotate_quantize_hadamard(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, signs_q, signs_k,
+                             layout: str = "BNSD", q_block: int = 128, kv_block: int = 256, debug: bool = False,
+                             out: Optional[Sequence[QTensor]] = None):
+    """Rotate Q and K by R = bf16(H_D diag(signs) / sqrt(D)) with a fast Walsh-Hadamard
+    transform, then FP8 block-quantize Q, K, V (fa_rotate_quantize_hadamard).  signs_q /
+    signs_k: sequences of D values +1 / -1 (or None for all +1).  Returns as rotate_quantize."""
+    ts = [_tensor(x, layout) for x in (q, k, v)]
+    D = ts[0].D
+    blks = (q_block, kv_block, kv_block)
+    outs = list(out) if out is not None else [
+        empty_qtensor(t.B, t.H, t.S, t.D, "fp8_block", layout, blks[i], q.device) for i, t in enumerate(ts)]
+
+    def bits(signs):
+        if signs is None:
+            return None
+        sg = [int(x) for x in signs]
+        if len(sg) != D or any(x not in (1, -1) for x in sg):
+            raise ValueError(f"signs must be {D} values of +1 / -1")
+        words = (ctypes.c_uint32 * (D // 32))()
+        for j, x in enumerate(sg):
+            if x < 0:
+                words[j // 32] |= 1 << (j % 32)
+        return words
+
+    bq, bk = bits(signs_q), bits(signs_k)
+    dq = torch.empty_like(q) if debug else None
+    dk = torch.empty_like(k) if debug else None
+    cq = [o.c() for o in outs]
+    _check(N.lib().fa_rotate_quantize_hadamard(ctypes.byref(ts[0]), ctypes.byref(ts[1]), ctypes.byref(ts[2]),
+                                               bq, bk, q_block, kv_block,
+                                               ctypes.byref(cq[0]), ctypes.byref(cq[1]), ctypes.byref(cq[2]),
+                                               dq.data_ptr() if dq is not None else None,
+                                               dk.data_ptr() if dk is not None else None, _stream()),
+           "fa_rotate_quantize_hadamard")
+    return tuple(outs) + ((dq, dk) if debug else ())
+
+
 def attention_workspace_size(q: QTensor, k: QTensor, num_splits: int = 0, v: Optional[QTensor] = None) -> int:
     cq, ck = q.c(), k.c()
     if v is not None:

@@ -83,7 +83,7 @@ struct P2 {
   const float* ks;
   const float* vs;
   const float* ksp;   // [B, Hkv, ntiles] x 512 B: per-key K scales, zero past Sk (E4M3) / UE8M0 atom (MXFP4)
-  const float4* fvr;  // [B, Hkv, ntiles] V' tile factor records {r_t, 0, 0, 0} (E4M3) / {E_t, 0, 0, 0} (MXFP4)
+  const float4* fvr;  // [B, Hkv, ntiles] V' tile factor records {r_t, log2 r_t, 0, 0} (E4M3) / {E_t, E_t - 127, 0, 0} (MXFP4)
   const uint8_t* qe8; // MXFP4 UE8M0 scales [B, H, S, D / 32]
   const uint8_t* ke8;
   const uint8_t* ve8;
@@ -640,6 +640,11 @@ __global__ void __launch_bounds__(Cfg<NSW>::NT, 1)
 //   QK_A(0) QK_B(0) | PV_A(0) QK_A(1) PV_B(0) QK_B(1) | PV_A(1) QK_A(2) ...
 // so while one warpgroup runs the softmax of tile j, the tensor pipe runs the
 // other tile's P V and next Q K^T.
+// Pairs of exponentials (out of every 8) that the pair kernel computes with the cubic on the
+// FMA pipe instead of the MUFU.
+#ifndef FAQ_PAIR_POLY
+#define FAQ_PAIR_POLY 0
+#endif
 constexpr int PNT = 384;  // warpgroup 0 (loads, MMA, scale ring) + two softmax warpgroups
 constexpr int PR0 = 56;
 constexpr int PRS = 224;
@@ -651,10 +656,13 @@ struct LP {
   static constexpr int NA = RB > 128 ? RB / 128 : 1;     // 128-byte swizzle atoms per row (bf16 at D = 128: 2)
   static constexpr int AB = RB > 128 ? 128 : RB;         // bytes per atom row
   static constexpr int NK = KIND == K_BF16 ? 2 : NKS;    // K stages (bf16 tiles are twice as large)
+  // V' stages: three for the 8-bit kinds, so a V' tile is requested two key-tile steps before its
+  // P V (a 32 KB tile from L2 takes a good part of one step to land); two fit beside bf16 Q / K
+  static constexpr int NV = KIND == K_BF16 ? 2 : 3;
   static constexpr uint32_t Q = 0;                       // 2 x NA x [128][AB]
   static constexpr uint32_t K = Q + 2 * BM * RB;         // NK stages
-  static constexpr uint32_t VH = K + NK * BN * RB;       // NVS stages of fp16 V'
-  static constexpr uint32_t SC = VH + NVS * BN * D * 2;  // NSC stages x ([128] K scales, V' factor record)
+  static constexpr uint32_t VH = K + NK * BN * RB;       // NV stages of fp16 V'
+  static constexpr uint32_t SC = VH + NV * BN * D * 2;   // NSC stages x ([128] K scales, V' factor record)
   static constexpr uint32_t MISC = SC + NSC * 2 * BN * 4;
   static constexpr uint32_t BAR = MISC + 64;
   static constexpr uint32_t TOTAL = BAR + 512;
@@ -667,9 +675,9 @@ enum {
   Y_Q = 0,
   Y_KF = 1,              // [NKS]
   Y_KE = Y_KF + NKS,     // [NKS]
-  Y_VF = Y_KE + NKS,     // [NVS]
-  Y_VE = Y_VF + NVS,     // [NVS]
-  Y_SF = Y_VE + NVS,     // [2] S_A / S_B full
+  Y_VF = Y_KE + NKS,     // [3] (up to three V' stages)
+  Y_VE = Y_VF + 3,       // [3]
+  Y_SF = Y_VE + 3,       // [2] S_A / S_B full
   Y_PF = Y_SF + 2,       // [2] P'_A / P'_B stored
   Y_PVD = Y_PF + 2,      // [2] P V of tile A / B done
   Y_SCF = Y_PVD + 2,     // [NSC]
@@ -687,6 +695,7 @@ __global__ void __launch_bounds__(PNT, 1)
   constexpr bool RING = SC != SC_HEAD;
   using L = LP<KIND, D>;
   constexpr int NKS = L::NK;  // K stages of this kind
+  constexpr int NVS = L::NV;  // V' stages of this kind
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bar = reinterpret_cast<uint64_t*>(smem + L::BAR);
@@ -817,6 +826,7 @@ __global__ void __launch_bounds__(PNT, 1)
         for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
         if (lane == 0) {
           misc[0] = m > 0.0f ? m : 1.0f;  // v_ref: the largest V' factor over this CTA's tiles
+          misc[1] = log2f(misc[0]);
           const float* kph = p.ksp + (long long)bhk * p.ntiles_k * BN;
           int j = 0;
           for (; j < n; ++j) {
@@ -841,32 +851,39 @@ __global__ void __launch_bounds__(PNT, 1)
                                       : KIND == K_BF16 ? make_idesc(kAccF32, kFmtBF16, kFmtBF16, 0, 0, BN, BM)
                                                        : make_idesc(kAccS32, kFmtS8, kFmtS8, 0, 0, BN, BM);
         constexpr uint32_t idesc_pv = make_idesc(kAccF32, kFmtF16, kFmtF16, 0, 1, D, BM);
+        // Descriptors as 32-bit halves: the high half (stride, version, swizzle) is constant per
+        // tile kind, the low half (start address >> 4 | leading offset) is computed once per tile
+        // base, and each MMA adds a compile-time offset (>> 4) to it, which stays inside the 14-bit
+        // address field (shared memory is below 256 KB).  The issuing warp shares its SM
+        // sub-partition with two softmax warps, so each MMA costs it only a few instructions.
+        const uint64_t dq0 = make_sdesc(smem_u32(smem + L::Q), 16, SBO8, SW);
+        const uint64_t dv0 = make_sdesc(smem_u32(smem + L::VH), BN * 128, 1024, kSwz128);
+        const uint32_t qk_hi = (uint32_t)(dq0 >> 32), v_hi = (uint32_t)(dv0 >> 32);
+        const uint32_t q_lo = (uint32_t)dq0, k_lo = (uint32_t)make_sdesc(smem_u32(smem + L::K), 16, SBO8, SW);
+        const uint32_t v_lo = (uint32_t)dv0;
         auto qk = [&](int x, int j) {
-          const uint32_t sQ = smem_u32(smem + L::Q + x * BM * L::RB);
-          const uint32_t sK = smem_u32(smem + L::K + (j % NKS) * BN * L::RB);
+          const uint32_t ql = q_lo + (x ? (uint32_t)((BM * L::RB) >> 4) : 0u);
+          const uint32_t kl = k_lo + (uint32_t)(j % NKS) * (uint32_t)((BN * L::RB) >> 4);
           // one MMA per 32 bytes of the row (K = 32 codes, or K = 16 bf16): atom a = kk * 32 / AB
 #pragma unroll
           for (int kk = 0; kk < L::RB / 32; ++kk) {
-            const uint32_t off = (kk * 32 / L::AB) * BM * L::AB + (kk * 32) % L::AB;
-            const uint64_t da = make_sdesc(sQ + off, 16, SBO8, SW);
-            const uint64_t db = make_sdesc(sK + off, 16, SBO8, SW);
+            const uint32_t off = ((kk * 32 / L::AB) * BM * L::AB + (kk * 32) % L::AB) >> 4;
             if (KIND == K_E4M3)
-              mma_f8f6f4(tbase + x * 128, da, db, idesc_qk, kk > 0);
+              mma_f8f6f4_lh(tbase + x * 128, ql + off, qk_hi, kl + off, qk_hi, idesc_qk, kk > 0);
             else if (KIND == K_BF16)
-              mma_f16(tbase + x * 128, da, db, idesc_qk, kk > 0);
+              mma_f16_lh(tbase + x * 128, ql + off, qk_hi, kl + off, qk_hi, idesc_qk, kk > 0);
             else
-              mma_i8(tbase + x * 128, da, db, idesc_qk, kk > 0);
+              mma_i8_lh(tbase + x * 128, ql + off, qk_hi, kl + off, qk_hi, idesc_qk, kk > 0);
           }
           mma_commit(&bar[Y_SF + x]);
         };
         auto pv = [&](int x, int j) {
           // A = P' in TMEM: key k of the tile sits in column k / 2 of S_x (fp16 pairs)
-          const uint32_t sVh = smem_u32(smem + L::VH + (j % NVS) * BN * D * 2);
+          const uint32_t vl = v_lo + (uint32_t)(j % NVS) * (uint32_t)((BN * D * 2) >> 4);
 #pragma unroll
-          for (int ks = 0; ks < BN / 16; ++ks) {
-            const uint64_t db = make_sdesc(sVh + ks * 16 * 128, BN * 128, 1024, kSwz128);
-            mma_f16_ts(tbase + 256 + x * D, tbase + x * 128 + ks * 8, db, idesc_pv, (j > 0 || ks > 0) ? 1u : 0u);
-          }
+          for (int ks = 0; ks < BN / 16; ++ks)
+            mma_f16_ts_lh(tbase + 256 + x * D, tbase + x * 128 + ks * 8, vl + (uint32_t)((ks * 16 * 128) >> 4), v_hi,
+                          idesc_pv, (j > 0 || ks > 0) ? 1u : 0u);
           mma_commit(&bar[Y_PVD + x]);
         };
         bool ok = mbar_wait(&bar[Y_Q], 0, abort_flag, p.status, 83);
@@ -924,13 +941,17 @@ __global__ void __launch_bounds__(PNT, 1)
     constexpr float kBias = BIASED ? 12582912.0f : 0.0f;
     float vref = RING ? 1.0f : __ldg(p.vs + hk);
     float m_run = -INFINITY, l_run = 0.0f;
+    float lgref = 0.0f;  // log2(v_ref)
     bool ok = true;
     for (int j = 0; j < n && ok; ++j) {
       const int k0 = j * BN;
       const int sst = j % NSC;
       const float* ksc = reinterpret_cast<const float*>(smem + L::SC + sst * 2 * BN * 4);
       if (RING && !warp_wait(&bar[Y_SCF + sst], (j / NSC) & 1, abort_flag, p.status, 90)) { ok = false; break; }
-      if (RING && j == 0) vref = misc[0];
+      if (RING && j == 0) {
+        vref = misc[0];
+        lgref = misc[1];
+      }
       if (j >= nx) {
         // the other tile's key range is longer: release the ring stage and move on
         if (RING) {
@@ -941,7 +962,8 @@ __global__ void __launch_bounds__(PNT, 1)
       }
       float flog = 0.0f, finv = 1.0f, cr = crow;
       if (RING) {
-        flog = fmaxf(__log2f(ksc[BN] / vref), -60.0f);
+        // the V' factor r_t / v_ref as its log2 (the record holds log2 r_t), floored at -60
+        flog = fmaxf(ksc[BN + 1] - lgref, -60.0f);
         finv = ex2(-flog);
       }
       if (SC == SC_TILE) cr *= ksc[0];
@@ -953,79 +975,123 @@ __global__ void __launch_bounds__(PNT, 1)
       }
       if (!warp_wait(&bar[Y_SF + x], j & 1, abort_flag, p.status, 91)) { ok = false; break; }
       tc_fence_after();
-      uint32_t tr[BN];
       float t[BN];
+      // S from TMEM (all four 32-column loads, one wait), the per-key K scale, the masks
+      auto load_s = [&](bool again) {
+        // per-key K scales: two halves of 64 columns, so half of the scales' registers are free
+        // before the second half of S lands; otherwise all four loads and one wait
+        constexpr int NH = SC == SC_COL ? 2 : 1;
 #pragma unroll
-      for (int hh = 0; hh < 2; ++hh) {
+        for (int hh = 0; hh < NH; ++hh) {
+          constexpr int W = BN / NH;
+          uint32_t tr[W];
 #pragma unroll
-        for (int c = 0; c < BN / 64; ++c)
-          tmem_ld32(tS + loff + 64 * hh + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(&tr[64 * hh + 32 * c]));
-        tmem_ld_wait();
-#pragma unroll
-        for (int k = 64 * hh; k < 64 * hh + 64; ++k)
-          t[k] = BIASED ? __uint_as_float(0x4B400000u + tr[k])
-                        : (KIND == K_S8 ? (float)(int)tr[k] : __uint_as_float(tr[k]));
-        if (SC == SC_COL) {
-#pragma unroll
-          for (int k = 64 * hh; k < 64 * hh + 64; k += 2) fmul2(t[k], t[k + 1], ksr[k], ksr[k + 1]);
-        }
-      }
-      const bool need_mask = (k0 + BN > p.Sk) || (p.causal && (k0 + BN - 1 > q0 + diag));
-      if (need_mask) {
-        const int lim = p.causal ? min(p.Sk - 1, row + diag) : p.Sk - 1;
-#pragma unroll
-        for (int k = 0; k < BN; ++k)
-          if (k0 + k > lim) t[k] = -INFINITY;
-      }
-      // row maximum: eight chains of three-input maxima
-      float mx[8];
-#pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        mx[e] = t[e];
-#pragma unroll
-        for (int q = 1; q < BN / 8; q += 2)
-          mx[e] = q + 1 < BN / 8 ? fmax3(mx[e], t[e + 8 * q], t[e + 8 * q + 8]) : fmaxf(mx[e], t[e + 8 * q]);
-      }
-      const float mt = fmax3(fmax3(mx[0], mx[1], mx[2]), fmax3(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7]));
-      const float mts = mt == -INFINITY ? -INFINITY : (mt - kBias) * cr;  // log2 domain
-      // the running max moves only when the tile's max exceeds it by more than 2^8
-      const float m_fin = mts > m_run + 8.0f ? mts : m_run;
-      const float alpha = m_fin != m_run ? ex2(m_run - m_fin) : 1.0f;
-      if (__any_sync(0xffffffffu, m_fin != m_run) && j > 0) {
-        // O is free once P V of tile j-1 has completed
-        if (!warp_wait(&bar[Y_PVD + x], (j - 1) & 1, abort_flag, p.status, 92)) { ok = false; break; }
-        tc_fence_after();
-#pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
-          uint32_t r[32];
-          tmem_ld32(tO + loff + c * 32, r);
+          for (int c = 0; c < W / 32; ++c)
+            tmem_ld32(tS + loff + W * hh + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(&tr[32 * c]));
           tmem_ld_wait();
 #pragma unroll
-          for (int k = 0; k < 32; k += 2) {
-            float a0 = __uint_as_float(r[k]), a1 = __uint_as_float(r[k + 1]);
-            fmul2(a0, a1, alpha, alpha);
-            r[k] = __float_as_uint(a0);
-            r[k + 1] = __float_as_uint(a1);
+          for (int k = 0; k < W; ++k)
+            t[W * hh + k] = BIASED ? __uint_as_float(0x4B400000u + tr[k])
+                                   : (KIND == K_S8 ? (float)(int)tr[k] : __uint_as_float(tr[k]));
+          if (SC == SC_COL) {
+            if (!again) {
+#pragma unroll
+              for (int k = W * hh; k < W * hh + W; k += 2) fmul2(t[k], t[k + 1], ksr[k], ksr[k + 1]);
+            } else {
+              // a second read: the scales again from the ring stage (still held), not kept in registers
+#pragma unroll
+              for (int k = W * hh; k < W * hh + W; k += 4) {
+                const float4 kv = *reinterpret_cast<const float4*>(ksc + k);
+                fmul2(t[k], t[k + 1], kv.x, kv.y);
+                fmul2(t[k + 2], t[k + 3], kv.z, kv.w);
+              }
+            }
           }
-          tmem_st32(tO + loff + c * 32, r);
         }
-        tmem_st_wait();
+        const bool need_mask = (k0 + BN > p.Sk) || (p.causal && (k0 + BN - 1 > q0 + diag));
+        if (need_mask) {
+          const int lim = p.causal ? min(p.Sk - 1, row + diag) : p.Sk - 1;
+#pragma unroll
+          for (int k = 0; k < BN; ++k)
+            if (k0 + k > lim) t[k] = -INFINITY;
+        }
+      };
+      // p' = 2^(t * cr - (bias * cr + m) + log2(r_t / v_ref)) in place, and their sum
+      auto exponentials = [&](float m) -> float {
+        const float nb = (m == -INFINITY ? 0.0f : -(kBias * cr + m)) + flog;
+#pragma unroll
+        for (int k = 0; k < BN; k += 2) {
+          ffma2(t[k], t[k + 1], cr, cr, nb, nb);
+          if (((k >> 1) & 7) < FAQ_PAIR_POLY) {
+            ex2_poly2(t[k], t[k + 1]);  // this share of the pairs on the FMA pipe
+          } else {
+            t[k] = ex2(t[k]);
+            t[k + 1] = ex2(t[k + 1]);
+          }
+        }
+        float ls[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) ls[e] = t[e];
+#pragma unroll
+        for (int k = 8; k < BN; k += 2) fadd2(ls[k & 7], ls[(k & 7) + 1], t[k], t[k + 1]);
+        return ((ls[0] + ls[1]) + (ls[2] + ls[3])) + ((ls[4] + ls[5]) + (ls[6] + ls[7]));
+      };
+      load_s(false);
+      // Speculative exponentials.  After a row's first tile the running max rarely moves, so
+      // the tile is exponentiated against it directly, without its own row maximum.  The sum
+      // tells whether that was safe: below 2^15 every p' stays below 2^15 (fp16 holds it) and
+      // the max would not have moved by more than 2^8 (the lazy rule below).  Otherwise -- and
+      // on a row's first tile -- S is read again (P' has not overwritten it yet), the tile's
+      // maximum taken, O rescaled if the maximum moves, and the exponentials redone.
+      float l_tile = 0.0f;
+      bool exact = __any_sync(0xffffffffu, m_run == -INFINITY);
+      bool failed = false;
+#pragma unroll 1
+      for (int pass = 0; pass < 2; ++pass) {
+        if (exact) {
+          // row maximum: eight chains of three-input maxima
+          float mx[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            mx[e] = t[e];
+#pragma unroll
+            for (int q = 1; q < BN / 8; q += 2)
+              mx[e] = q + 1 < BN / 8 ? fmax3(mx[e], t[e + 8 * q], t[e + 8 * q + 8]) : fmaxf(mx[e], t[e + 8 * q]);
+          }
+          const float mt = fmax3(fmax3(mx[0], mx[1], mx[2]), fmax3(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7]));
+          const float mts = mt == -INFINITY ? -INFINITY : (mt - kBias) * cr;  // log2 domain
+          // the running max moves only when the tile's max exceeds it by more than 2^8
+          const float m_fin = mts > m_run + 8.0f ? mts : m_run;
+          const float alpha = m_fin != m_run ? ex2(m_run - m_fin) : 1.0f;
+          if (__any_sync(0xffffffffu, m_fin != m_run) && j > 0) {
+            // O is free once P V of tile j-1 has completed
+            if (!warp_wait(&bar[Y_PVD + x], (j - 1) & 1, abort_flag, p.status, 92)) { failed = true; break; }
+            tc_fence_after();
+#pragma unroll 1
+            for (int c = 0; c < D / 32; ++c) {
+              uint32_t r[32];
+              tmem_ld32(tO + loff + c * 32, r);
+              tmem_ld_wait();
+#pragma unroll
+              for (int k = 0; k < 32; k += 2) {
+                float a0 = __uint_as_float(r[k]), a1 = __uint_as_float(r[k + 1]);
+                fmul2(a0, a1, alpha, alpha);
+                r[k] = __float_as_uint(a0);
+                r[k + 1] = __float_as_uint(a1);
+              }
+              tmem_st32(tO + loff + c * 32, r);
+            }
+            tmem_st_wait();
+          }
+          l_run *= alpha;
+          m_run = m_fin;
+        }
+        l_tile = exponentials(m_run);
+        if (exact || !__any_sync(0xffffffffu, !(l_tile < 32768.0f))) break;
+        exact = true;
+        load_s(true);
       }
-      l_run *= alpha;
-      m_run = m_fin;
-      // p = 2^(t * cr - (bias * cr + m) + log2(r_t / v_ref))
-      const float nb = (m_run == -INFINITY ? 0.0f : -(kBias * cr + m_run)) + flog;
-#pragma unroll
-      for (int k = 0; k < BN; k += 2) {
-        ffma2(t[k], t[k + 1], cr, cr, nb, nb);
-        t[k] = ex2(t[k]);
-        t[k + 1] = ex2(t[k + 1]);
-      }
-      float ls[8];
-#pragma unroll
-      for (int e = 0; e < 8; ++e) ls[e] = t[e];
-#pragma unroll
-      for (int k = 8; k < BN; k += 2) fadd2(ls[k & 7], ls[(k & 7) + 1], t[k], t[k + 1]);
+      if (failed) { ok = false; break; }
       {
         uint32_t hp[BN / 2];
 #pragma unroll
@@ -1037,7 +1103,7 @@ __global__ void __launch_bounds__(PNT, 1)
         tmem_st32(tS + loff + 32, *reinterpret_cast<uint32_t(*)[32]>(&hp[32]));
       }
       tmem_st_wait();
-      l_run += (((ls[0] + ls[1]) + (ls[2] + ls[3])) + ((ls[4] + ls[5]) + (ls[6] + ls[7]))) * finv;
+      l_run += l_tile * finv;
       tc_fence_before();
       __syncwarp();
       if (lane == 0) {
@@ -1141,7 +1207,7 @@ __global__ void __launch_bounds__(256) vprep_kernel(const uint8_t* __restrict__ 
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, off));
     if (threadIdx.x == 0)
-      fvr[(long long)bh * ntiles + t] = make_float4(MIXED ? ldexpf(1.0f, m - 127) : (float)m, 0.0f, 0.0f, 0.0f);
+      fvr[(long long)bh * ntiles + t] = make_float4(MIXED ? ldexpf(1.0f, m - 127) : (float)m, (float)(m - 127), 0.0f, 0.0f);
     if (MIXED) {
       if (threadIdx.x < BN) ksp[((long long)bh * ntiles + t) * BN + threadIdx.x] = tok0 + (int)threadIdx.x < S ? 1.0f : 0.0f;
     } else if (threadIdx.x < BN) {
@@ -1208,7 +1274,7 @@ __global__ void __launch_bounds__(256) vprep_kernel(const uint8_t* __restrict__ 
     E = max(E, -112);
     const float r = am > 0.0f ? __uint_as_float((uint32_t)(E - 14 + 127) << 23) : 1.0f;
     const float inv = am > 0.0f ? __uint_as_float((uint32_t)(14 - E + 127) << 23) : 1.0f;
-    if (threadIdx.x == 0) fvr[(long long)bh * ntiles + t] = make_float4(r, 0.0f, 0.0f, 0.0f);
+    if (threadIdx.x == 0) fvr[(long long)bh * ntiles + t] = make_float4(r, am > 0.0f ? (float)(E - 14) : 0.0f, 0.0f, 0.0f);
     if (threadIdx.x < BN) ksp[((long long)bh * ntiles + t) * BN + threadIdx.x] = tok0 + (int)threadIdx.x < S ? 1.0f : 0.0f;
     if (!live) return;
     uint4* dst = reinterpret_cast<uint4*>(vh + ((long long)bh * S + tok) * D + (lane & 1) * (D / 2));
@@ -1248,7 +1314,7 @@ __global__ void __launch_bounds__(256) vprep_kernel(const uint8_t* __restrict__ 
     }
     const float r = m > 0.0f ? m : 1.0f;
     f = live ? (v_blk == 0 ? m : __ldg(vsh + tok / v_blk)) / r : 0.0f;
-    if (threadIdx.x == 0) fvr[(long long)bh * ntiles + t] = make_float4(r, 0.0f, 0.0f, 0.0f);
+    if (threadIdx.x == 0) fvr[(long long)bh * ntiles + t] = make_float4(r, log2f(r), 0.0f, 0.0f);
     // the tile's per-key K scales, zero past S, at a 16-byte aligned per-tile slot
     if (threadIdx.x < BN) {
       const int key = tok0 + threadIdx.x;
@@ -1357,12 +1423,7 @@ cudaError_t launch2(const AttnArgs& a, const P2& prm, const Prefill2Ws& w, cudaS
   cudaError_t e;
   if ((e = prepare2<KIND, D, true>(a, prm, w, (int)L::RB, &mq, &mk, &mv, s)) != cudaSuccess) return e;
   auto kern = attn2_kernel<KIND, D, SC, NSW>;
-  static bool attr_set = false;
-  if (!attr_set) {
-    if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::ALLOC)) != cudaSuccess)
-      return e;
-    attr_set = true;
-  }
+  if ((e = set_smem_limit(reinterpret_cast<const void*>(kern), L::ALLOC)) != cudaSuccess) return e;
   const long long grid = (long long)prm.n_qtiles * prm.B * prm.Hq;
   if (grid > 0x7FFFFFFFLL) return cudaErrorInvalidValue;
   kern<<<(unsigned)grid, Cfg<NSW>::NT, L::ALLOC, s>>>(mq, mk, mv, prm);
@@ -1374,12 +1435,7 @@ cudaError_t run_pair(const CUtensorMap& mq, const CUtensorMap& mk, const CUtenso
   using L = LP<KIND, D>;
   cudaError_t e;
   auto kern = attn_pair_kernel<KIND, D, SC>;
-  static bool attr_set = false;
-  if (!attr_set) {
-    if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::ALLOC)) != cudaSuccess)
-      return e;
-    attr_set = true;
-  }
+  if ((e = set_smem_limit(reinterpret_cast<const void*>(kern), L::ALLOC)) != cudaSuccess) return e;
   // GQA groups of even size pair two query heads at one row block (equal key ranges); otherwise
   // a head's row blocks pair up.
   prm.pair_heads = prm.group % 2 == 0;

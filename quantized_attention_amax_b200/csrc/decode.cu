@@ -14,10 +14,13 @@
 //   O^T [D x 16] = V_tile^T . P^T                     kind::i8, A = V codes
 //                                                     (MN-major), B = P (u8)
 //   fold: O_acc = O_acc * 2^(m_prev - m) + O^T (fp32, one thread per dim)
-// Each split writes (O_acc, m, L); attn_combine_kernel merges the splits:
+// Each split writes (O_acc, m, L) and takes a ticket; the last CTA of a (b, kv head) merges
+// the splits in the same launch:
 //   m* = max_c m_c,  O = s_v * sum_c 2^(m_c - m*) O_c / sum_c 2^(m_c - m*) L_c.
 #include <cuda_bf16.h>
 #include <math.h>
+
+#include <atomic>
 
 #include "internal.cuh"
 #include "sm100.cuh"
@@ -39,6 +42,10 @@ struct DecParams {
   const float* vs;
   float* opart;  // [B*Hq][splits][D]
   float* ml;     // [B*Hq][splits][2]  (m in log2 units, L)
+  unsigned long long* tickets;  // [B*Hkv] (epoch << 32 | CTAs done), reset to 0 by the last CTA
+  unsigned int epoch;           // nonzero, new for every call
+  __nv_bfloat16* out;           // [B*Hq][D] (Sq = 1: BNSD and BSND coincide)
+  float* lse;                   // nullable [B*Hq]
   int* status;
   // Fused cache append: Q quantized from bf16 in every CTA, and the new token's K / V rows quantized
   // into the cache at position pos by the CTA whose chunk holds it (before its TMA reads).
@@ -64,7 +71,8 @@ struct DSmem {
   static constexpr uint32_t P = V + DNS * DBN * D;  // 2 x [16][128] u8 (K-major)
   static constexpr uint32_t RED = P + 2 * 2048;     // [2][4 warps][16] floats (tile maxima)
   static constexpr uint32_t LRED = RED + 2 * 4 * 16 * 4;  // [4 warps][16] floats (sums)
-  static constexpr uint32_t BAR = LRED + 4 * 16 * 4;
+  static constexpr uint32_t FLAG = LRED + 4 * 16 * 4;     // the combine's "last CTA" flag
+  static constexpr uint32_t BAR = FLAG + 16;
   static constexpr uint32_t TOTAL = BAR + 512;
   static constexpr uint32_t ALLOC = TOTAL + 1024;
 };
@@ -390,6 +398,56 @@ __global__ void __launch_bounds__(DTHREADS, 2)
         p.ml[row * 2 + 1] = ok ? Lt : 0.0f;
       }
     }
+    // ---- LSE combine, fused: the last CTA of this (b, kv head) to finish merges the splits.
+    // Every CTA fences its partials and takes a ticket; the CTA that takes the last one reads
+    // all of them (no CTA ever waits for another).  A ticket word holds this call's epoch in its
+    // high half, so whatever the workspace held before the first call counts as empty; the
+    // last CTA resets it to 0.
+    __threadfence();
+    asm volatile("bar.sync 1, 128;" ::: "memory");  // the four softmax warps
+    volatile int* last_flag = reinterpret_cast<volatile int*>(smem + L::FLAG);
+    if (i == 0) {
+      unsigned long long* tk = p.tickets + bhk;
+      unsigned long long old = atomicAdd(tk, 0ull);
+      int last = 0;
+      for (int it = 0; it < (1 << 20); ++it) {
+        const unsigned long long nw =
+            (unsigned)(old >> 32) == p.epoch ? old + 1ull : (((unsigned long long)p.epoch << 32) | 1ull);
+        const unsigned long long prev = atomicCAS(tk, old, nw);
+        if (prev == old) {
+          last = (int)(nw & 0xFFFFFFFFull) == p.splits;
+          break;
+        }
+        old = prev;
+        if (it == (1 << 20) - 1 && p.status) atomicCAS(p.status, 0, (35 << 8) | kStatusTimeout);
+      }
+      *last_flag = last;
+    }
+    asm volatile("bar.sync 1, 128;" ::: "memory");
+    if (*last_flag) {
+      __threadfence();
+      const float vsc = p.append ? __fdiv_rn(__ldg(p.amax_v + hk), 127.0f) : __ldg(p.vs + hk);
+      for (int idx = i; idx < G * D; idx += 128) {
+        const int h = idx / D, d = idx - h * D;
+        const long long qrow = (long long)b * p.Hq + hq0 + h;
+        const float* mlr = p.ml + qrow * p.splits * 2;
+        const float* opr = p.opart + qrow * p.splits * D + d;
+        float m = -INFINITY;
+        for (int c = 0; c < p.splits; ++c) m = fmaxf(m, __ldcg(mlr + 2 * c));
+        float Ls = 0.0f, acc = 0.0f;
+        for (int c = 0; c < p.splits; ++c) {
+          const float mc = __ldcg(mlr + 2 * c);
+          if (mc != -INFINITY) {
+            const float wc = ex2f(mc - m);
+            Ls += wc * __ldcg(mlr + 2 * c + 1);
+            acc += wc * __ldcg(opr + (long long)c * D);
+          }
+        }
+        p.out[qrow * D + d] = __float2bfloat16(Ls > 0.0f ? acc * (vsc / Ls) : 0.0f);
+        if (d == 0 && p.lse) p.lse[qrow] = Ls > 0.0f ? (m + __log2f(Ls / 255.0f)) * 0.69314718055994530942f : -INFINITY;
+      }
+      if (i == 0) atomicExch(p.tickets + bhk, 0ull);
+    }
   }
 
   tc_fence_before();
@@ -398,40 +456,6 @@ __global__ void __launch_bounds__(DTHREADS, 2)
     tc_fence_after();
     tmem_dealloc(tbase, 64);
   }
-}
-
-// One warp per (b, query head): merge the splits' (O, m, L).
-__global__ void attn_combine_kernel(const float* __restrict__ opart, const float* __restrict__ ml, int BH, int Hq,
-                                    int Hkv, int splits, int D, const float* vs, __nv_bfloat16* out, float* lse,
-                                    int layout) {
-  const int w = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-  const int lane = threadIdx.x & 31;
-  if (w >= BH) return;
-  const int hq = w % Hq;
-  const int hk = hq / (Hq / Hkv);
-  float m = -INFINITY;
-  for (int c = lane; c < splits; c += 32) m = fmaxf(m, ml[((long long)w * splits + c) * 2]);
-#pragma unroll
-  for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
-  float Lsum = 0.0f;
-  for (int c = lane; c < splits; c += 32) {
-    const float mc = ml[((long long)w * splits + c) * 2];
-    if (mc != -INFINITY) Lsum += ex2f(mc - m) * ml[((long long)w * splits + c) * 2 + 1];
-  }
-#pragma unroll
-  for (int off = 16; off > 0; off >>= 1) Lsum += __shfl_xor_sync(0xffffffffu, Lsum, off);
-  const float scale = Lsum > 0.0f ? __ldg(vs + hk) / Lsum : 0.0f;
-  // BNSD and BSND coincide for Sq = 1: row (b, hq) at (b * Hq + hq) * D.
-  (void)layout;
-  for (int d = lane; d < D; d += 32) {
-    float acc = 0.0f;
-    for (int c = 0; c < splits; ++c) {
-      const float mc = ml[((long long)w * splits + c) * 2];
-      if (mc != -INFINITY) acc += ex2f(mc - m) * opart[((long long)w * splits + c) * D + d];
-    }
-    out[(long long)w * D + d] = __float2bfloat16(acc * scale);
-  }
-  if (lse && lane == 0) lse[w] = Lsum > 0.0f ? (m + __log2f(Lsum / 255.0f)) * 0.69314718055994530942f : -INFINITY;
 }
 
 // Tensor map over int8 codes of S visible tokens stored in a buffer of cap >= S tokens.
@@ -495,8 +519,11 @@ int decode_auto_splits(int B, int Hkv, int Sk) {
   return best;
 }
 
+// Partials [B*Hq][splits][D] and [B*Hq][splits][2] fp32, then one 8-byte ticket per
+// (b, kv head), B * Hq of them at most, 256-byte aligned.
 size_t decode_workspace_bytes(int B, int Hq, int D, int splits) {
-  return (size_t)B * Hq * splits * ((size_t)D + 2) * sizeof(float);
+  const size_t parts = (size_t)B * Hq * splits * ((size_t)D + 2) * sizeof(float);
+  return ((parts + 255) & ~size_t(255)) + (size_t)B * Hq * 8;
 }
 
 namespace {
@@ -505,9 +532,17 @@ namespace {
 // K / V buffers of cap tokens.
 cudaError_t run_decode(DecParams prm, const void* kcodes, const void* vcodes, int D, int kv_len, int cap, int out_layout,
                        void* out, float* lse, cudaStream_t s) {
+  (void)out_layout;  // Sq = 1: row (b, hq) at (b * Hq + hq) * D in either layout
   const int G = prm.group;
   prm.Sk = kv_len;
   prm.chunk = chunk_of(kv_len, prm.splits);
+  prm.out = static_cast<__nv_bfloat16*>(out);
+  prm.lse = lse;
+  // a fresh nonzero epoch per call for the combine tickets
+  static std::atomic<unsigned int> epochs{0};
+  unsigned int ep = epochs.fetch_add(1u) + 1u;
+  if (ep == 0u) ep = epochs.fetch_add(1u) + 1u;
+  prm.epoch = ep;
   CUtensorMap mk, mv;
   cudaError_t e;
   if ((e = make_map(&mk, kcodes, prm.B, prm.Hkv, kv_len, D, prm.layout, cap)) != cudaSuccess) return e;
@@ -524,11 +559,7 @@ cudaError_t run_decode(DecParams prm, const void* kcodes, const void* vcodes, in
   } else {
     return cudaErrorNotSupported;
   }
-  if (e != cudaSuccess) return e;
-  const int BH = prm.B * prm.Hq;
-  attn_combine_kernel<<<(BH * 32 + 255) / 256, 256, 0, s>>>(prm.opart, prm.ml, BH, prm.Hq, prm.Hkv, prm.splits, D,
-                                                            prm.vs, static_cast<__nv_bfloat16*>(out), lse, out_layout);
-  return cudaGetLastError();
+  return e;
 }
 
 DecParams base_params(int B, int Hq, int Hkv, int D, int layout, int splits, float softmax_scale, void* ws,
@@ -540,6 +571,8 @@ DecParams base_params(int B, int Hq, int Hkv, int D, int layout, int splits, flo
   prm.scale_log2 = scale * 1.4426950408889634f;
   prm.opart = static_cast<float*>(ws);
   prm.ml = prm.opart + (size_t)B * Hq * splits * D;
+  const size_t parts = (size_t)B * Hq * splits * ((size_t)D + 2) * sizeof(float);
+  prm.tickets = reinterpret_cast<unsigned long long*>(static_cast<uint8_t*>(ws) + ((parts + 255) & ~size_t(255)));
   prm.status = status;
   return prm;
 }

@@ -259,6 +259,43 @@ fa_status fa_rotate_quantize(const fa_tensor* q, const fa_tensor* k, const fa_te
   return from_cuda(e);
 }
 
+fa_status fa_rotate_quantize_hadamard(const fa_tensor* q, const fa_tensor* k, const fa_tensor* v,
+                                      const uint32_t* sign_bits_q, const uint32_t* sign_bits_k, int q_block,
+                                      int kv_block, fa_qtensor* q_out, fa_qtensor* k_out, fa_qtensor* v_out,
+                                      void* rot_q_dbg, void* rot_k_dbg, fa_stream_t s) {
+  const fa_tensor* in[3] = {q, k, v};
+  fa_qtensor* out[3] = {q_out, k_out, v_out};
+  const uint32_t* sg[3] = {sign_bits_q, sign_bits_k, nullptr};
+  void* dbg[3] = {rot_q_dbg, rot_k_dbg, nullptr};
+  const int blk[3] = {q_block, kv_block, kv_block};
+  HadamardOperand ops[3];
+  int n = 0;
+  for (int i = 0; i < 3; ++i) {
+    if (!in[i]) continue;
+    fa_status st = check_tensor(in[i]);
+    if (st != FA_OK) return st;
+    st = check_out(in[i], out[i], FA_MODE_FP8_BLOCK);
+    if (st != FA_OK) return st;
+    if (blk[i] < 1 || out[i]->block_tokens != blk[i]) return FA_ERR_INVALID_ARG;
+    if (dbg[i] && !aligned16(dbg[i])) return FA_ERR_INVALID_ARG;
+    HadamardOperand& op = ops[n++];
+    op.x = in[i]->data;
+    op.codes = out[i]->codes;
+    op.scales = static_cast<float*>(out[i]->scales);
+    op.dbg = dbg[i];
+    for (int w = 0; w < 4; ++w) op.sign_bits[w] = (sg[i] && w < in[i]->D / 32) ? sg[i][w] : 0u;
+    op.B = in[i]->B; op.H = in[i]->H; op.S = in[i]->S; op.D = in[i]->D; op.layout = in[i]->layout;
+    op.blk = blk[i];
+    op.rotate = i < 2;
+  }
+  if (n == 0) return FA_ERR_INVALID_ARG;
+  for (int i = 1; i < n; ++i)
+    if (ops[i].D != ops[0].D) return FA_ERR_INVALID_ARG;
+  const cudaError_t e = launch_hadamard_block_quant(ops, n, reinterpret_cast<cudaStream_t>(s));
+  if (e == cudaErrorNotSupported) return FA_ERR_UNSUPPORTED;
+  return from_cuda(e);
+}
+
 // Branches in different modes, or any branch not quantized: the bf16 mixed path.
 static bool is_mixed(const fa_qtensor* q, const fa_qtensor* k, const fa_qtensor* v) {
   return q->mode != k->mode || (v && q->mode != v->mode) || q->mode == FA_MODE_FLOAT || k->mode == FA_MODE_FLOAT ||

@@ -53,6 +53,18 @@ struct RotateOperand {
 };
 cudaError_t launch_rotate_block_quant(const RotateOperand* ops, int nops, int* status, cudaStream_t s);
 
+// Launcher (hadamard.cu): rotation R = bf16(H_D diag(sigma) / sqrt(D)) by a fast Walsh-Hadamard
+// transform (rotate = 1) or none (rotate = 0), then FP8 block quantization.
+struct HadamardOperand {
+  const void* x;          // bf16 input [.., D]
+  void* codes;            // e4m3
+  float* scales;          // [B, H, nblk]
+  void* dbg;              // nullable bf16 rotated output
+  uint32_t sign_bits[4];  // bit j set: sigma_j = -1 (D / 32 words used)
+  int B, H, S, D, layout, blk, rotate;
+};
+cudaError_t launch_hadamard_block_quant(const HadamardOperand* ops, int nops, cudaStream_t s);
+
 // Launchers (attn2.cu / decode.cu).
 struct AttnArgs {
   const fa_qtensor* q;

@@ -191,6 +191,31 @@ __device__ __forceinline__ void mma_f16_ts(uint32_t d, uint32_t a_tmem, uint64_t
       "r"(a_tmem), "l"(b), "r"(idesc), "r"(accum)
       : "memory");
 }
+// The same MMAs with each shared-memory descriptor given as its two 32-bit halves (the low half
+// holds the start address and the leading byte offset; the high half is constant for a tile
+// kind), so an issuing thread keeps one 32-bit word per tile and adds offsets to it.
+#define FAQ_MMA_LH(NAME, KIND)                                                                          \
+  __device__ __forceinline__ void NAME(uint32_t d, uint32_t alo, uint32_t ahi, uint32_t blo, uint32_t bhi, \
+                                       uint32_t idesc, uint32_t accum) {                                 \
+    asm volatile(                                                                                        \
+        "{\n\t.reg .pred p;\n\t.reg .b64 da, db;\n\tmov.b64 da, {%1, %2};\n\tmov.b64 db, {%3, %4};\n\t"  \
+        "setp.ne.b32 p, %6, 0;\n\ttcgen05.mma.cta_group::1.kind::" KIND " [%0], da, db, %5, p;\n\t}" ::"r"(d), \
+        "r"(alo), "r"(ahi), "r"(blo), "r"(bhi), "r"(idesc), "r"(accum)                                     \
+        : "memory");                                                                                     \
+  }
+FAQ_MMA_LH(mma_f8f6f4_lh, "f8f6f4")
+FAQ_MMA_LH(mma_i8_lh, "i8")
+FAQ_MMA_LH(mma_f16_lh, "f16")
+#undef FAQ_MMA_LH
+__device__ __forceinline__ void mma_f16_ts_lh(uint32_t d, uint32_t a_tmem, uint32_t blo, uint32_t bhi, uint32_t idesc,
+                                              uint32_t accum) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t.reg .b64 db;\n\tmov.b64 db, {%2, %3};\n\tsetp.ne.b32 p, %5, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], db, %4, p;\n\t}" ::"r"(d),
+      "r"(a_tmem), "r"(blo), "r"(bhi), "r"(idesc), "r"(accum)
+      : "memory");
+}
+
 // Block-scaled FP4 (E2M1 x E2M1, UE8M0 scale per 32 elements along K).
 // Block-scaled E4M3 x E4M3 (one UE8M0 scale per 32 elements of K for A and for B, in TMEM).
 __device__ __forceinline__ void mma_mxf8(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t sfa,

@@ -144,29 +144,42 @@ def test_constant_v(faq, orc):
     assert torch.allclose(o, torch.full_like(o, vq), rtol=0, atol=4e-3 * vq)
 
 
-@pytest.mark.parametrize("name", ["fp8_prefill", "int8_tiny", "mxfp4"])
+def sampled_rows(Sq, seed=0, n=256):
+    """Rows 0, 1, 2, the tile boundaries 127/128/255/256, the last row, and seeded random rows up
+    to n in all (rows are independent, so a sample is exact where taken)."""
+    fixed = [r for r in (0, 1, 2, 127, 128, 255, 256, Sq - 1) if r < Sq]
+    rng = np.random.default_rng(seed)
+    rest = [int(r) for r in rng.permutation(Sq) if int(r) not in fixed]
+    return sorted(fixed + rest[:max(0, n - len(fixed))])
+
+
+# every workload the benchmark reports a prefill number for, in its launch configuration
+@pytest.mark.parametrize("name", ["fp8_prefill", "int8_tiny", "mxfp4", "int8_prefill", "fp8_head_prefill",
+                                  "int8_token_prefill", "mxfp8"])
 def test_full_size_workload(faq, orc, name):
-    """Full-size workload in the benchmark's launch configuration, checked on
-    sampled query rows (rows are independent, so a sample is exact)."""
+    """Full-size workload in the benchmark's launch configuration, checked on 256 sampled query
+    rows per head, element by element against the oracle."""
     w = wl.WORKLOADS[name]
     inp = wl.make_inputs(w)
     bits = {n: wl.bf16_bits(inp[n]) for n in "qkv"}
     amax = {}
-    if w.mode == "int8_per_head":
+    if w.mode in ("int8_per_head", "fp8_per_head"):
         for n in "qkv":
             amax[n] = orc.calibrate_per_head(wl.bf16_bits(inp[n + "_cal"]), w.layout)
     oq = {n: oracle_quantize(orc, w.mode, bits[n], w.layout, 0, amax.get(n)) for n in "qkv"}
-    rng = np.random.default_rng(0)
-    rows = sorted(set([0, 1, 2, 127, 128, 255, 256, w.Sq - 1] + list(rng.choice(w.Sq, min(w.Sq, 120), False))))
-    rows = [r for r in rows if r < w.Sq]
-    ref, _ = orc.attention(oq["q"], oq["k"], oq["v"], w.causal, 0.0, rows)
+    rows = sampled_rows(w.Sq)
+    ref, ref_lse = orc.attention(oq["q"], oq["k"], oq["v"], w.causal, 0.0, rows)
     dev = {n: inp[n].cuda() for n in "qkv"}
-    if w.mode == "int8_per_head":
+    if amax:
         am = [torch.from_numpy(amax[n]).cuda() for n in "qkv"]
         Q, K, V = faq.quantize(dev["q"], dev["k"], dev["v"], w.mode, w.layout, amax=am)
     else:
         Q, K, V = faq.quantize(dev["q"], dev["k"], dev["v"], w.mode, w.layout)
-    out = faq.attention(Q, K, V, causal=w.causal)
+    for n, G in zip("qkv", (Q, K, V)):  # the GPU's codes are the oracle's (so both see the same operands)
+        assert np.array_equal(np_of(G.codes).view(np.uint8), np.ascontiguousarray(oq[n].codes).view(np.uint8)), n
+    out, glse = faq.attention(Q, K, V, causal=w.causal, return_lse=True)
     faq.check_device_status()
     got = to_bnsd(np_of(out.float()), w.layout)[:, :, rows, :]
     assert_attention_close(got, ref, head_vmax(orc, oq["v"], w.Hq), name)
+    gl = np_of(glse)[:, :, rows]
+    assert np.abs(gl - ref_lse).max() < 2e-3 * max(1.0, np.abs(ref_lse).max())

@@ -96,3 +96,24 @@ def test_uniform_and_mixed_paths_side_by_side(faq, orc):
     b = run_mixed(faq, orc, ("fp8_per_token", "fp8_per_token", "float"), "BNSD", 128, 1, 2, 2, 256, 256, True,
                   seed=4)
     assert a[0] < 2e-2 and b[0] < 2e-2
+
+
+def test_full_size_mixed_workload(faq, orc):
+    """The benchmark's mixed-branch workload at full size (Q, K FP8 per token, V left bf16,
+    B=2 Hq=32 Hkv=8 S=4096, causal), checked on 256 sampled query rows per head."""
+    from test_attn_gpu import sampled_rows
+    w = wl.WORKLOADS["mixed_prefill"]
+    inp = wl.make_inputs(w)
+    mq, mk, mv = w.branch_modes
+    bits = {n: wl.bf16_bits(inp[n]) for n in "qkv"}
+    oq = oracle_quantize(orc, mq, bits["q"], w.layout)
+    ok_ = oracle_quantize(orc, mk, bits["k"], w.layout)
+    ov = orc.qt_float(bits["v"], w.layout)
+    rows = sampled_rows(w.Sq)
+    ref, _ = orc.attention(oq, ok_, ov, w.causal, 0.0, rows)
+    Q, K = faq.quantize(inp["q"].cuda(), inp["k"].cuda(), None, mq, w.layout)[:2]
+    V = faq.float_branch(inp["v"].cuda(), w.layout)
+    out = faq.attention(Q, K, V, causal=w.causal)
+    faq.check_device_status()
+    got = to_bnsd(np_of(out.float()), w.layout)[:, :, rows, :]
+    assert_attention_close(got, ref, head_vmax(orc, ov, w.Hq), "mixed_prefill")

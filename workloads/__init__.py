@@ -126,6 +126,12 @@ def normal_k_outliers(shp, layout: str, seed: int, device="cpu") -> torch.Tensor
     return x.to(torch.bfloat16)
 
 
+def rotation_signs(D: int, seed: int) -> list:
+    """The seeded +-1 signs of rotation(D, seed), as a list of D ints."""
+    g = _gen(seed + 11, "cpu")
+    return [int(x) for x in (torch.randint(0, 2, (D,), generator=g) * 2 - 1).tolist()]
+
+
 def rotation(D: int, seed: int, device="cpu") -> torch.Tensor:
     """bf16 [D, D]: Sylvester Hadamard times a seeded diagonal of +-1 signs,
     divided by sqrt(D) (orthogonal before the bf16 rounding)."""
@@ -133,8 +139,7 @@ def rotation(D: int, seed: int, device="cpu") -> torch.Tensor:
     Hm = torch.ones(1, 1, dtype=torch.float64)
     while Hm.shape[0] < D:
         Hm = torch.cat([torch.cat([Hm, Hm], 1), torch.cat([Hm, -Hm], 1)], 0)
-    g = _gen(seed + 11, "cpu")
-    signs = torch.randint(0, 2, (D,), generator=g).to(torch.float64) * 2 - 1
+    signs = torch.tensor(rotation_signs(D, seed), dtype=torch.float64)
     R = Hm * signs[None, :] / (D ** 0.5)
     return R.to(torch.bfloat16).to(device)
 
