@@ -63,13 +63,29 @@ __device__ __forceinline__ uint32_t e2m1x8(const float (&v)[8]) {
   return r;
 }
 
-__device__ __forceinline__ uint32_t s8_of(float x) {
-  int i = __float2int_rn(x);  // round half to even; saturates to the int32 range
-  i = max(-128, min(127, i));
-  return (uint32_t)(i & 0xFF);
-}
+// Int8 codes of four quotients, rounded half to even, on the FMA / ALU pipes (a float-to-integer
+// conversion would run on the quarter-rate XU pipe): adding 1.5 * 2^23 rounds to an integer in
+// the low mantissa bits (exact for |x| < 2^22), whose low byte is the two's-complement code;
+// three byte permutes pack the four codes.  SAT (static scales, which data can exceed): NaN -> 0
+// as a conversion gives, then a clamp to [-128, 127] (before or after rounding gives the same
+// integer, the bounds being integers).  Without SAT (per-token scales) |x / s| <= 127 holds by
+// construction, so no clamp is needed.
+template <bool SAT>
 __device__ __forceinline__ uint32_t s8x4(float a, float b, float c, float d) {
-  return s8_of(a) | (s8_of(b) << 8) | (s8_of(c) << 16) | (s8_of(d) << 24);
+  if (SAT) {
+    a = fminf(fmaxf(a == a ? a : 0.0f, -128.0f), 127.0f);
+    b = fminf(fmaxf(b == b ? b : 0.0f, -128.0f), 127.0f);
+    c = fminf(fmaxf(c == c ? c : 0.0f, -128.0f), 127.0f);
+    d = fminf(fmaxf(d == d ? d : 0.0f, -128.0f), 127.0f);
+  }
+  constexpr float kMagic = 12582912.0f;
+  asm("{\n\t.reg .b64 x, y, m;\n\tmov.b64 x, {%0, %1};\n\tmov.b64 y, {%2, %3};\n\tmov.b64 m, {%4, %4};\n\t"
+      "add.rn.f32x2 x, x, m;\n\tadd.rn.f32x2 y, y, m;\n\tmov.b64 {%0, %1}, x;\n\tmov.b64 {%2, %3}, y;\n\t}"
+      : "+f"(a), "+f"(b), "+f"(c), "+f"(d)
+      : "f"(kMagic));
+  const uint32_t ab = __byte_perm(__float_as_uint(a), __float_as_uint(b), 0x0040);  // low bytes of a, b
+  const uint32_t cd = __byte_perm(__float_as_uint(c), __float_as_uint(d), 0x0040);
+  return __byte_perm(ab, cd, 0x5410);
 }
 
 // Canonical [B, H, S] index of token row r of the data layout.
@@ -213,8 +229,8 @@ __global__ void __launch_bounds__(256) quant_rows_kernel(QuantOperand o0, QuantO
 #pragma unroll
         for (int i = 0; i < 8; ++i) v[i] = sc > 0.0f ? __fdiv_rn(v[i], sc) : 0.0f;
       }
-      w[2 * c] = INT8 ? s8x4(v[0], v[1], v[2], v[3]) : e4m3x4(v[0], v[1], v[2], v[3]);
-      w[2 * c + 1] = INT8 ? s8x4(v[4], v[5], v[6], v[7]) : e4m3x4(v[4], v[5], v[6], v[7]);
+      w[2 * c] = INT8 ? s8x4<PER_HEAD>(v[0], v[1], v[2], v[3]) : e4m3x4(v[0], v[1], v[2], v[3]);
+      w[2 * c + 1] = INT8 ? s8x4<PER_HEAD>(v[4], v[5], v[6], v[7]) : e4m3x4(v[4], v[5], v[6], v[7]);
     }
     if (valid) {
       out[0] = make_uint4(w[0], w[1], w[2], w[3]);
