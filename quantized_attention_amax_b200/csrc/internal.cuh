@@ -19,6 +19,9 @@ struct QuantOperand {
   int B, H, S, D;
   int layout;
   int blk;             // FP8 block: tokens per block
+  // row -> head by multiply-high division (filled by the row quantizer's launcher)
+  uint32_t mS, mH;     // magic multipliers for S and H
+  int lS, lH;          // their shifts
 };
 
 // Per-device status word (timeouts recorded by bounded waits).

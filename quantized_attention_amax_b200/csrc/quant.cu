@@ -88,14 +88,24 @@ __device__ __forceinline__ uint32_t s8x4(float a, float b, float c, float d) {
   return __byte_perm(ab, cd, 0x5410);
 }
 
+// max(|a|, |b|) per half as above, but a NaN in either input gives NaN
+__device__ __forceinline__ uint32_t bf16x2_absmax_nan(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("max.NaN.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+
+// n / d for n < 2^32 by one multiply-high (T. Granlund and P. L. Montgomery, "Division by
+// invariant integers using multiplication", PLDI 1994, unsigned case): m and l from fastdiv_magic.
+__device__ __forceinline__ uint32_t fast_div(uint32_t n, uint32_t m, int l) {
+  return (uint32_t)(((unsigned long long)__umulhi(n, m) + n) >> l);
+}
+
 // Canonical [B, H, S] index of token row r of the data layout.
 __device__ __forceinline__ long long scale_index(long long r, int layout, int H, int S) {
   if (layout == FA_LAYOUT_BNSD) return r;
   const long long h = r % H, bs = r / H;
   return ((bs / S) * H + h) * S + (bs % S);
-}
-__device__ __forceinline__ int head_of(long long r, int layout, int H, int S) {
-  return layout == FA_LAYOUT_BNSD ? (int)((r / S) % H) : (int)(r % H);
 }
 
 // Exponent e of the MX shared scale: floor(log2 amax) - EMAX (2 for E2M1, 8 for E4M3 elements),
@@ -110,8 +120,10 @@ __device__ __forceinline__ int mx_exponent(float amax) {
 // One row = D / 32 lanes; each lane owns 32 consecutive elements (one MX block): four 16-byte
 // loads, so the per-row work (the scale, its reciprocal, the lane shuffles, the addresses) is
 // shared by 32 elements per lane.
+constexpr int kRowThreads = 256;
+
 template <int MODE, int D>
-__global__ void __launch_bounds__(256) quant_rows_kernel(QuantOperand o0, QuantOperand o1, QuantOperand o2) {
+__global__ void __launch_bounds__(kRowThreads) quant_rows_kernel(QuantOperand o0, QuantOperand o1, QuantOperand o2) {
   constexpr int LPR = D / 32;  // lanes per row
   constexpr int RPW = 32 / LPR;  // rows per warp
   const int lane = threadIdx.x & 31;
@@ -202,35 +214,80 @@ __global__ void __launch_bounds__(256) quant_rows_kernel(QuantOperand o0, QuantO
       continue;
     }
     // one scale per row (dynamic modes) or per head (static modes)
-    float sc;
+    float sc = 0.0f, rc = 0.0f;
+    // bounded: every |x| of the warp's rows is within its scale's maximum, so the INT8 quotients
+    // need neither the overflow guard nor the clamp (dynamic scales: by construction)
+    bool bounded = !PER_HEAD;
     if (PER_HEAD) {
-      const int op_layout = which == 0 ? o0.layout : (which == 1 ? o1.layout : o2.layout);
-      const int op_H = which == 0 ? o0.H : (which == 1 ? o1.H : o2.H);
-      const int op_S = which == 0 ? o0.S : (which == 1 ? o1.S : o2.S);
-      const float* op_amax = which == 0 ? o0.amax : (which == 1 ? o1.amax : o2.amax);
-      sc = valid ? __fdiv_rn(__ldg(op_amax + head_of(rr, op_layout, op_H, op_S)), QMAX) : 0.0f;
+      float lim = -1.0f;
+      if (valid) {
+        const int op_layout = which == 0 ? o0.layout : (which == 1 ? o1.layout : o2.layout);
+        const int op_H = which == 0 ? o0.H : (which == 1 ? o1.H : o2.H);
+        // row -> head in 32 bits (rows < 2^32, checked by the launcher)
+        const uint32_t r32 = (uint32_t)rr;
+        const uint32_t mS = which == 0 ? o0.mS : (which == 1 ? o1.mS : o2.mS);
+        const uint32_t mH = which == 0 ? o0.mH : (which == 1 ? o1.mH : o2.mH);
+        const int lS = which == 0 ? o0.lS : (which == 1 ? o1.lS : o2.lS);
+        const int lH = which == 0 ? o0.lH : (which == 1 ? o1.lH : o2.lH);
+        const uint32_t hs = op_layout == FA_LAYOUT_BNSD ? fast_div(r32, mS, lS) : r32;  // row of [B, H] (BNSD)
+        const int h = (int)(hs - fast_div(hs, mH, lH) * (uint32_t)op_H);
+        // the static scale and its reciprocal, recomputed per row (a per-CTA table behind a
+        // barrier measured slower: each CTA handles only a few rows)
+        const float a = __ldg((which == 0 ? o0.amax : (which == 1 ? o1.amax : o2.amax)) + h);
+        sc = __fdiv_rn(a, QMAX);
+        rc = sc >= kFastDivMin ? __frcp_rn(sc) : 0.0f;
+        lim = fabsf(a) < INFINITY ? a : -1.0f;
+      }
+      if (INT8) {
+        // NaN-propagating max |x| of the lane's 32 elements: a NaN fails the comparison
+        uint32_t m2 = 0;
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+          m2 = bf16x2_absmax_nan(bf16x2_absmax_nan(m2, bf16x2_absmax_nan(raw[c].x, raw[c].y)),
+                                 bf16x2_absmax_nan(raw[c].z, raw[c].w));
+        m2 &= 0x7FFF7FFFu;  // the sign bits are the XOR of the inputs' signs
+        const bool in = !valid || (__uint_as_float(m2 << 16) <= lim && __uint_as_float(m2 & 0xFFFF0000u) <= lim);
+        bounded = __all_sync(0xffffffffu, in);
+      }
     } else {
       sc = __fdiv_rn(m, QMAX);
+      rc = sc >= kFastDivMin ? __frcp_rn(sc) : 0.0f;
     }
     // codes, 8 elements at a time straight from the packed row
     uint32_t w[8];
     const bool fast = sc >= kFastDivMin;
-    const float rc = fast ? __frcp_rn(sc) : 0.0f;
+    if (INT8 && bounded) {
 #pragma unroll
-    for (int c = 0; c < 4; ++c) {
-      float v[8];
-      unpack_bf16x8(raw[c], v);
-      if (fast) {
-        // x / s as IEEE division rounds it where that decides the code (quant_common.cuh)
+      for (int c = 0; c < 4; ++c) {
+        float v[8];
+        unpack_bf16x8(raw[c], v);
+        if (fast) {
 #pragma unroll
-        for (int i = 0; i < 8; ++i)
-          v[i] = INT8 ? int8_div(v[i], sc, rc) : (PER_HEAD ? fp8_div_sat(v[i], sc, rc) : fp8_div(v[i], sc, rc));
-      } else {
+          for (int i = 0; i < 8; i += 2) int8_div_bounded_x2(v[i], v[i + 1], sc, rc);
+        } else {
 #pragma unroll
-        for (int i = 0; i < 8; ++i) v[i] = sc > 0.0f ? __fdiv_rn(v[i], sc) : 0.0f;
+          for (int i = 0; i < 8; ++i) v[i] = sc > 0.0f ? __fdiv_rn(v[i], sc) : 0.0f;
+        }
+        w[2 * c] = s8x4<false>(v[0], v[1], v[2], v[3]);
+        w[2 * c + 1] = s8x4<false>(v[4], v[5], v[6], v[7]);
       }
-      w[2 * c] = INT8 ? s8x4<PER_HEAD>(v[0], v[1], v[2], v[3]) : e4m3x4(v[0], v[1], v[2], v[3]);
-      w[2 * c + 1] = INT8 ? s8x4<PER_HEAD>(v[4], v[5], v[6], v[7]) : e4m3x4(v[4], v[5], v[6], v[7]);
+    } else {
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        float v[8];
+        unpack_bf16x8(raw[c], v);
+        if (fast) {
+          // x / s as IEEE division rounds it where that decides the code (quant_common.cuh)
+#pragma unroll
+          for (int i = 0; i < 8; ++i)
+            v[i] = INT8 ? int8_div(v[i], sc, rc) : (PER_HEAD ? fp8_div_sat(v[i], sc, rc) : fp8_div(v[i], sc, rc));
+        } else {
+#pragma unroll
+          for (int i = 0; i < 8; ++i) v[i] = sc > 0.0f ? __fdiv_rn(v[i], sc) : 0.0f;
+        }
+        w[2 * c] = INT8 ? s8x4<true>(v[0], v[1], v[2], v[3]) : e4m3x4(v[0], v[1], v[2], v[3]);
+        w[2 * c + 1] = INT8 ? s8x4<true>(v[4], v[5], v[6], v[7]) : e4m3x4(v[4], v[5], v[6], v[7]);
+      }
     }
     if (valid) {
       out[0] = make_uint4(w[0], w[1], w[2], w[3]);
@@ -338,20 +395,34 @@ __global__ void __launch_bounds__(256) fp8_block_kernel(QuantOperand op) {
   }
 }
 
+// Magic multiplier and shift of fast_div for a divisor d in [1, 2^31): l = ceil(log2 d),
+// m = floor(2^32 (2^l - d) / d) + 1 (below 2^32 for every such d).  d = 0 (an unused operand) -> 1.
+void fastdiv_magic(long long d, uint32_t& m, int& l) {
+  if (d < 1) d = 1;
+  l = 0;
+  while ((1LL << l) < d) ++l;
+  m = (uint32_t)((((1ULL << l) - (unsigned long long)d) << 32) / (unsigned long long)d + 1);
+}
+
 template <int MODE>
-cudaError_t launch_rows_mode(const QuantOperand (&o)[3], int D, cudaStream_t s) {
-  const long long total = o[0].rows + o[1].rows + o[2].rows;
-  if (total == 0) {
-    if (MODE != FA_MODE_INT8_PER_HEAD && MODE != FA_MODE_FP8_PER_HEAD) return cudaSuccess;
+cudaError_t launch_rows_mode(const QuantOperand (&oi)[3], int D, cudaStream_t s) {
+  const long long total = oi[0].rows + oi[1].rows + oi[2].rows;
+  constexpr bool PER_HEAD = MODE == FA_MODE_INT8_PER_HEAD || MODE == FA_MODE_FP8_PER_HEAD;
+  if (total == 0 && !PER_HEAD) return cudaSuccess;
+  QuantOperand o[3] = {oi[0], oi[1], oi[2]};
+  for (int i = 0; i < 3; ++i) {
+    if (PER_HEAD && o[i].rows > 0xFFFFFFFFLL) return cudaErrorInvalidValue;  // heads found in 32 bits
+    fastdiv_magic(o[i].S, o[i].mS, o[i].lS);
+    fastdiv_magic(o[i].H, o[i].mH, o[i].lH);
   }
-  const int rows_per_block = (256 / 32) * (32 / (D / 32));
-  long long want = (total + rows_per_block - 1) / rows_per_block;
+  const int rows_per_block = (kRowThreads / 32) * (32 / (D / 32));
+  const long long want = (total + rows_per_block - 1) / rows_per_block;
   const long long cap = (long long)sm_count() * 8 * 4;  // enough resident warps, grid-stride beyond
-  int grid = (int)(want < 1 ? 1 : (want > cap ? cap : want));
+  const int grid = (int)(want < 1 ? 1 : (want > cap ? cap : want));
   if (D == 128)
-    quant_rows_kernel<MODE, 128><<<grid, 256, 0, s>>>(o[0], o[1], o[2]);
+    quant_rows_kernel<MODE, 128><<<grid, kRowThreads, 0, s>>>(o[0], o[1], o[2]);
   else
-    quant_rows_kernel<MODE, 64><<<grid, 256, 0, s>>>(o[0], o[1], o[2]);
+    quant_rows_kernel<MODE, 64><<<grid, kRowThreads, 0, s>>>(o[0], o[1], o[2]);
   return cudaGetLastError();
 }
 

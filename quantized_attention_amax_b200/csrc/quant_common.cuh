@@ -39,4 +39,25 @@ __device__ __forceinline__ float int8_div(float x, float s, float r) {
   return fabsf(q0) < 0x1p20f ? fmaf(fmaf(-q0, s, x), r, q0) : q0;
 }
 
+// INT8 where |x| <= amax is known (per-token scales, or a per-head row inside its calibrated
+// range): |x / s| <= 127 (1 + 2^-23), so the overflow guard of int8_div is never taken and the
+// correction applies unconditionally.  Same codes as IEEE division on that domain (exhaustive).
+__device__ __forceinline__ float int8_div_bounded(float x, float s, float r) {
+  const float q0 = x * r;
+  return fmaf(fmaf(-q0, s, x), r, q0);
+}
+
+// int8_div_bounded on a pair in packed f32x2 arithmetic: two lanes per instruction, each with the
+// scalar form's three roundings (-q0 * s written as q0 * (-s), an exact sign change).
+__device__ __forceinline__ void int8_div_bounded_x2(float& a, float& b, float s, float r) {
+  asm("{\n\t.reg .b64 x, q, e, ns, rv;\n\t"
+      "mov.b64 x, {%0, %1};\n\tmov.b64 ns, {%2, %2};\n\tmov.b64 rv, {%3, %3};\n\t"
+      "mul.rn.f32x2 q, x, rv;\n\t"
+      "fma.rn.f32x2 e, q, ns, x;\n\t"
+      "fma.rn.f32x2 q, e, rv, q;\n\t"
+      "mov.b64 {%0, %1}, q;\n\t}"
+      : "+f"(a), "+f"(b)
+      : "f"(-s), "f"(r));
+}
+
 }  // namespace faq

@@ -23,7 +23,7 @@ def test_fp8_div_matches_ieee_division_exhaustively(tmp_path):
     r = subprocess.run([exe], capture_output=True, text=True, timeout=300)
     assert r.returncode == 0, r.stderr
     found = re.findall(r"mode (\d) fast rows (\d+) mismatches (\d+)", r.stdout)
-    assert [int(m) for m, _, _ in found] == [0, 1, 2], r.stdout
+    assert [int(m) for m, _, _ in found] == [0, 1, 2, 3, 4], r.stdout
     for _, fast, bad in found:
         assert int(fast) > 26000  # nearly every scale takes the fast path
         assert int(bad) == 0

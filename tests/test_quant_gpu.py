@@ -72,6 +72,47 @@ def test_int8_calibrate_and_quantize_bit_exact(faq, orc, layout, D, S):
         assert np.array_equal(np_of(o.codes), codes)
 
 
+def test_int8_per_head_every_path(faq, orc):
+    """INT8 per head through each branch of the kernel: heads whose rows stay inside amax_h (no
+    clamp), rows past it (saturation), non-finite data (NaN -> 0, +-inf clamped), amax_h = inf
+    and NaN, scales below 2^-90 (IEEE division) and fp32-subnormal scales.  Every head is an
+    exhaustive sweep of the bf16 values its range allows."""
+    bits = np.arange(65536, dtype=np.uint32)
+    f = (bits << 16).view(np.float32)
+    fin = np.isfinite(f)
+    S, D = 300, 128
+    rng = np.random.default_rng(11)
+    # (largest |x| of the data or None for every pattern, amax_h)
+    heads = [(3.0, 3.0), (3.0, 1.0), (None, 448.0), (5.0, np.inf), (5.0, np.nan), (1e-30, 1e-30),
+             (2.0 ** -130, 2.0 ** -130), (65504.0, 65504.0 * 2), (1.0, -1.0)]
+    x = np.empty((1, len(heads), S, D), np.uint16)
+    for h, (lim, _) in enumerate(heads):
+        pool = bits if lim is None else bits[fin & (np.abs(f) <= np.float32(lim))]
+        x[0, h] = np.resize(rng.permutation(pool).astype(np.uint16), S * D).reshape(S, D)
+    am = np.array([a for _, a in heads], np.float32)
+    o, = faq.quantize(bf16_from_bits(x), None, None, "int8_per_head", amax=[torch.from_numpy(am).cuda(), None, None])[:1]
+    torch.cuda.synchronize()
+    codes, scales = orc.quantize_int8_per_head(x, am)
+    assert np.array_equal(np_of(o.scales), scales, equal_nan=True)
+    assert np.array_equal(np_of(o.codes), codes)
+
+
+@pytest.mark.parametrize("mode", ["int8_per_head", "fp8_per_head"])
+def test_per_head_many_heads(faq, orc, mode):
+    """More heads than the kernel's shared-memory scale table holds (the per-row path), in both
+    layouts; half the heads calibrated at half their range."""
+    for layout, D in (("BSND", 64), ("BNSD", 128)):
+        x = rand_bf16(shp(2, 300, 7, D, layout), 77)
+        a = faq.calibrate_per_head(x.cuda(), layout)
+        a[::2] *= 0.5
+        o, = faq.quantize(x.cuda(), None, None, mode, layout, amax=[a, None, None])[:1]
+        torch.cuda.synchronize()
+        fn = orc.quantize_int8_per_head if mode == "int8_per_head" else orc.quantize_fp8_per_head
+        codes, scales = fn(wl.bf16_bits(x), np_of(a), layout)
+        assert np.array_equal(np_of(o.scales), scales)
+        assert np.array_equal(np_of(o.codes), codes)
+
+
 @pytest.mark.parametrize("layout,D,S", CASES)
 def test_fp8_per_head_bit_exact(faq, orc, layout, D, S):
     """FA PerHead with FP8: static scale amax_h / 448 from calibration; data past the
