@@ -177,8 +177,8 @@ FAQ_API fa_status fa_rotate_quantize(const fa_tensor* q, const fa_tensor* k, con
 
 /*
  * fa_rotate_quantize_hadamard -- fa_rotate_quantize for rotations of the
- * Hadamard-times-signs form, by a fast Walsh-Hadamard transform instead of a
- * D x D product (the rotation specialization of the same flow).
+ * Hadamard-times-signs form, given by their signs instead of a D x D matrix
+ * in memory (the rotation specialization of the same flow).
  *   Source: MindIE SD "量化", FA量化 / 技术特点: 旋转 (Q and K multiplied by a
  *   rotation before 块量化), with the rotation R = bf16(H_D diag(sigma) /
  *   sqrt(D)): H_D the Sylvester Hadamard matrix, entry (i, j) =
@@ -186,8 +186,11 @@ FAQ_API fa_status fa_rotate_quantize(const fa_tensor* q, const fa_tensor* k, con
  *   +-c with c = bf16(1 / sqrt(D)), so x R = c * sigma * FWHT(x) elementwise,
  *   FWHT(x)_j = sum_d x_d (-1)^popcount(d & j).  The rotated row is evaluated
  *   in fp32 and rounded once to bf16, then quantized exactly as
- *   fa_rotate_quantize does (FA_MODE_FP8_BLOCK); the results equal those of
- *   fa_rotate_quantize given that R up to the order of the fp32 sums.
+ *   fa_rotate_quantize does (FA_MODE_FP8_BLOCK).  With D = 128 and blocks
+ *   that divide 256 tokens, the rotation runs in fa_rotate_quantize's
+ *   pipeline with R built in shared memory from the signs (results identical
+ *   to fa_rotate_quantize given that R); otherwise a fast Walsh-Hadamard
+ *   transform computes it (results equal up to the order of the fp32 sums).
  *   sign_bits_q, sign_bits_k: HOST pointers to D / 32 words; bit j % 32 of
  *   word j / 32 set means sigma_j = -1; NULL means every sigma_j = +1.
  *   Everything else (q_block, kv_block, outputs, the nullable rot_*_dbg

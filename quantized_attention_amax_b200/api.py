@@ -197,9 +197,10 @@ def rotate_quantize(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, rot_q: to
 def rotate_quantize_hadamard(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, signs_q, signs_k,
                              layout: str = "BNSD", q_block: int = 128, kv_block: int = 256, debug: bool = False,
                              out: Optional[Sequence[QTensor]] = None):
-    """Rotate Q and K by R = bf16(H_D diag(signs) / sqrt(D)) with a fast Walsh-Hadamard
-    transform, then FP8 block-quantize Q, K, V (fa_rotate_quantize_hadamard).  signs_q /
-    signs_k: sequences of D values +1 / -1 (or None for all +1).  Returns as rotate_quantize."""
+    """Rotate Q and K by R = bf16(H_D diag(signs) / sqrt(D)), given by its signs, then FP8
+    block-quantize Q, K, V (fa_rotate_quantize_hadamard: R built on chip for D = 128 with blocks
+    dividing 256, a fast Walsh-Hadamard transform otherwise).  signs_q / signs_k: sequences of D
+    values +1 / -1 (or None for all +1).  Returns as rotate_quantize."""
     ts = [_tensor(x, layout) for x in (q, k, v)]
     D = ts[0].D
     blks = (q_block, kv_block, kv_block)

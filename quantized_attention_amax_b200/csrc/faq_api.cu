@@ -229,7 +229,7 @@ fa_status fa_rotate_quantize(const fa_tensor* q, const fa_tensor* k, const fa_te
   const void* rot[3] = {rot_q, rot_k, nullptr};
   void* dbg[3] = {rot_q_dbg, rot_k_dbg, nullptr};
   const int blk[3] = {q_block, kv_block, kv_block};
-  RotateOperand ops[3];
+  RotateOperand ops[3] = {};
   int n = 0;
   for (int i = 0; i < 3; ++i) {
     if (!in[i]) continue;
@@ -291,6 +291,30 @@ fa_status fa_rotate_quantize_hadamard(const fa_tensor* q, const fa_tensor* k, co
   if (n == 0) return FA_ERR_INVALID_ARG;
   for (int i = 1; i < n; ++i)
     if (ops[i].D != ops[0].D) return FA_ERR_INVALID_ARG;
+  // D = 128 with blocks that divide 256 tokens: the tensor-core rotation pipeline with R generated
+  // in shared memory from the signs (the rotation is HBM-bound there, so a product costs no more
+  // than the transform); otherwise the fast Walsh-Hadamard transform kernel
+  bool pipeline = ops[0].D == 128;
+  for (int i = 0; i < n; ++i) pipeline = pipeline && ops[i].blk <= 256 && 256 % ops[i].blk == 0;
+  if (pipeline) {
+    RotateOperand ro[3] = {};
+    for (int i = 0; i < n; ++i) {
+      const HadamardOperand& h = ops[i];
+      ro[i].x = h.x;
+      ro[i].R = nullptr;
+      ro[i].codes = h.codes;
+      ro[i].scales = h.scales;
+      ro[i].dbg = h.dbg;
+      ro[i].B = h.B; ro[i].H = h.H; ro[i].S = h.S; ro[i].D = h.D; ro[i].layout = h.layout; ro[i].blk = h.blk;
+      ro[i].hadamard = h.rotate;
+      for (int w = 0; w < 4; ++w) ro[i].sign_bits[w] = h.sign_bits[w];
+    }
+    int* status = device_status_ptr();
+    if (!status) return FA_ERR_CUDA;
+    const cudaError_t e = launch_rotate_block_quant(ro, n, status, reinterpret_cast<cudaStream_t>(s));
+    if (e == cudaErrorNotSupported) return FA_ERR_UNSUPPORTED;
+    return from_cuda(e);
+  }
   const cudaError_t e = launch_hadamard_block_quant(ops, n, reinterpret_cast<cudaStream_t>(s));
   if (e == cudaErrorNotSupported) return FA_ERR_UNSUPPORTED;
   return from_cuda(e);

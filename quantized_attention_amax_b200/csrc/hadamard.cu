@@ -9,6 +9,11 @@
 // block scale is amax / 448 over the block's rotated bf16 values, and the codes are the E4M3
 // values of x' / s (rounded as IEEE division rounds it).  V is block-quantized without rotation.
 //
+// This kernel serves D = 64 and block sizes that do not divide 256 tokens; D = 128 with blocks
+// that do goes through the rotation pipeline of rotate.cu with R generated in shared memory from
+// the same signs (the rotation is HBM-bound on the tensor cores, so the product costs nothing
+// there, and that pipeline streams at close to the copy bandwidth).
+//
 // One CTA per quantization block (b, h, blk tokens), 256 threads; each token row is shared by
 // D / 16 lanes (sixteen elements each, one coalesced read of the row), the transform runs in
 // registers with its last log2(D / 16) stages across lanes by shuffles, then the bf16 rounding

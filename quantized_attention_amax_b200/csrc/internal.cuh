@@ -48,11 +48,14 @@ cudaError_t launch_quantize_fp8_block(const QuantOperand* ops, int nops, cudaStr
 // Launchers (rotate.cu).
 struct RotateOperand {
   const void* x;       // bf16 input [.., D]
-  const void* R;       // bf16 [D, D] or nullptr (no rotation)
+  const void* R;       // bf16 [D, D] or nullptr (no rotation, unless hadamard)
   void* codes;         // e4m3
   float* scales;       // [B, H, nblk]
   void* dbg;           // nullable bf16 rotated output
   int B, H, S, D, layout, blk;
+  // R = bf16(H_D diag(sigma) / sqrt(D)) generated in shared memory from the signs (R unused)
+  int hadamard;
+  uint32_t sign_bits[4];  // bit j set: sigma_j = -1
 };
 cudaError_t launch_rotate_block_quant(const RotateOperand* ops, int nops, int* status, cudaStream_t s);
 

@@ -10,7 +10,9 @@
 //               64-element K atoms) into one of two 64 KB input stages; the
 //               items come in operand order (Q, K, V), so the one resident
 //               rotation is loaded when the operand changes, after the MMAs
-//               that read the previous one.
+//               that read the previous one.  A rotation of the Hadamard-
+//               times-signs form is written by this warp from its signs
+//               instead, in the same swizzled layout.
 //   warp 17     tcgen05.mma kind::f16 (bf16 x bf16 -> fp32): X R into one of
 //               two 256-column TMEM buffers, R read as the MN-major B operand
 //               exactly as stored ([D, D] row-major, x' = x R).  V items skip it.
@@ -26,6 +28,7 @@
 // So the loads and MMAs of item k + 1 overlap the epilogue of item k.
 // blk must divide 256.
 #include <cuda_bf16.h>
+#include <math.h>
 #include <string.h>
 
 #include "internal.cuh"
@@ -68,6 +71,9 @@ struct RotOp {
   float* scales;
   __nv_bfloat16* dbg;
   int B, H, S, layout, blk, rotate;
+  int had;               // rotation generated from the signs (Hadamard form) instead of loaded
+  uint32_t sgn[4];       // its signs: bit j set, sigma_j = -1
+  uint32_t cbits;        // bf16 bits of c = bf16(1 / sqrt(D))
   int lblk;              // log2(blk) (blk divides 256, so it is a power of two)
   long long first_item;  // first work item of this operand
   int chunks;            // 256-token chunks per (b, h)
@@ -118,6 +124,33 @@ __device__ __forceinline__ uint32_t e4m3x4(float a, float b, float c, float d) {
   asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(lo) : "f"(b), "f"(a));
   asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(hi) : "f"(d), "f"(c));
   return (uint32_t)lo | ((uint32_t)hi << 16);
+}
+
+// R = bf16(H_D diag(sigma) / sqrt(D)) for D = 128, written by the 32 lanes of one warp straight
+// into the shared-memory layout the TMA copy of a stored R produces: [2 column atoms of 64][128
+// rows d][128 B], 16-byte chunk q of row d at chunk q ^ (d & 7) (the 128-byte swizzle).  Entry
+// (d, j) = +-c, negative when popcount(d & j) + [sigma_j = -1] is odd (the Sylvester Hadamard
+// sign times sigma_j; rounding to bf16 commutes with the sign).
+__device__ __forceinline__ void write_hadamard_rotation(uint8_t* dst, const uint32_t (&sgn)[4], uint32_t cbits,
+                                                        int lane) {
+  // a chunk holds j = j0 .. j0 + 7 with j0 a multiple of 8, so popcount(d & j) = popcount(d & j0) +
+  // popcount(d & t) for t = j - j0: the chunk's eight sign bits are the parity of d & j0 (all
+  // eight), the parities of (d & 7) & t (a pattern per d & 7), and the eight sigma bits
+  const uint32_t c2 = cbits | (cbits << 16);
+  for (int i = lane; i < 2 * 128 * 8; i += 32) {
+    const int nb = i >> 10, d = (i >> 3) & 127, q = i & 7;
+    const int j0 = nb * 64 + q * 8;
+    uint32_t neg = (sgn[j0 >> 5] >> (j0 & 31)) & 0xFFu;
+    if (__popc(d & j0) & 1) neg ^= 0xFFu;
+    const int d7 = d & 7;
+    // bit t: parity of popcount(d7 & t) (the rows of the 8 x 8 Sylvester matrix)
+    const uint32_t pat = ((d7 & 1) ? 0xAAu : 0u) ^ ((d7 & 2) ? 0xCCu : 0u) ^ ((d7 & 4) ? 0xF0u : 0u);
+    neg ^= pat;
+    uint32_t w[4];
+#pragma unroll
+    for (int t = 0; t < 4; ++t) w[t] = c2 | (((neg >> (2 * t)) & 1u) << 15) | (((neg >> (2 * t + 1)) & 1u) << 31);
+    *reinterpret_cast<uint4*>(dst + nb * 16384 + d * 128 + ((q ^ d7) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
+  }
 }
 
 // per half: max(|a|, |b|), its sign the XOR of the inputs' signs (exact; only magnitudes are used)
@@ -303,24 +336,36 @@ __global__ void __launch_bounds__(RTHREADS, 1)
 
   if (warp == WPROD) {
     // ------------------------------------------------------------- producer
-    if (lane == 0) {
-      long long k = 0;
-      int rload = 0, rop = -1;  // rotations loaded so far; the operand whose rotation is resident
-      for (long long g = blockIdx.x; g < prm.items; g += G, ++k) {
-        const int st = (int)(k & 1);
-        if (k >= 2 && !mbar_wait(&bar[RB_XE + st], (uint32_t)(((k >> 1) - 1) & 1), abort_flag, prm.status, 45)) break;
-        const RItem it = decode_item(prm, g);
-        const RotOp& op = prm.op[it.oi];
-        if (op.rotate && it.oi != rop) {
-          // a CTA meets its items in operand order, so each rotation is loaded once; the next
-          // one waits until the MMAs that read the previous one have completed
-          if (rload > 0 && !mbar_wait(&bar[RB_RE], (uint32_t)((rload - 1) & 1), abort_flag, prm.status, 49)) break;
+    // Every lane walks the items (the same sequence); lane 0 issues the barrier operations and
+    // the TMA copies, and the whole warp writes a rotation generated from signs.
+    long long k = 0;
+    int rload = 0, rop = -1;  // rotations loaded so far; the operand whose rotation is resident
+    for (long long g = blockIdx.x; g < prm.items; g += G, ++k) {
+      const int st = (int)(k & 1);
+      bool ok = true;
+      if (lane == 0 && k >= 2) ok = mbar_wait(&bar[RB_XE + st], (uint32_t)(((k >> 1) - 1) & 1), abort_flag, prm.status, 45);
+      if (!__shfl_sync(0xffffffffu, ok, 0)) break;
+      const RItem it = decode_item(prm, g);
+      const RotOp& op = prm.op[it.oi];
+      if (op.rotate && it.oi != rop) {
+        // a CTA meets its items in operand order, so each rotation is loaded once; the next
+        // one waits until the MMAs that read the previous one have completed
+        if (lane == 0 && rload > 0) ok = mbar_wait(&bar[RB_RE], (uint32_t)((rload - 1) & 1), abort_flag, prm.status, 49);
+        if (!__shfl_sync(0xffffffffu, ok, 0)) break;
+        if (op.had) {
+          write_hadamard_rotation(smem + RSmem::R, op.sgn, op.cbits, lane);
+          fence_async_smem();  // the MMA reads it through the async proxy
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&bar[RB_RF]);
+        } else if (lane == 0) {
           mbar_arrive_expect_tx(&bar[RB_RF], 32768);
           for (int nb = 0; nb < 2; ++nb)
             tma_load_4d(smem + RSmem::R + nb * 16384, it.oi == 0 ? &mrq : &mrk, &bar[RB_RF], nb * 64, 0, 0, 0);
-          ++rload;
-          rop = it.oi;
         }
+        ++rload;
+        rop = it.oi;
+      }
+      if (lane == 0) {
         const CUtensorMap* mx = it.oi == 0 ? &mq : (it.oi == 1 ? &mk : &mv);
         const bool bnsd = op.layout == FA_LAYOUT_BNSD;
         mbar_arrive_expect_tx(&bar[RB_XF + st], it.ntile * 2 * 16384);
@@ -331,12 +376,13 @@ __global__ void __launch_bounds__(RTHREADS, 1)
                         bnsd ? t : it.h, bnsd ? it.h : t, it.b);
           }
       }
-      if (*abort_flag) {
-        // let loads already issued land before the CTA can exit
-        if (rload > 0) mbar_drain(&bar[RB_RF], (uint32_t)((rload - 1) & 1));
-        for (long long t = (k >= 2 ? k - 2 : 0); t < k; ++t)
-          mbar_drain(&bar[RB_XF + (t & 1)], (uint32_t)((t >> 1) & 1));
-      }
+      __syncwarp();
+    }
+    if (lane == 0 && *abort_flag) {
+      // let loads already issued land before the CTA can exit
+      if (rload > 0) mbar_drain(&bar[RB_RF], (uint32_t)((rload - 1) & 1));
+      for (long long t = (k >= 2 ? k - 2 : 0); t < k; ++t)
+        mbar_drain(&bar[RB_XF + (t & 1)], (uint32_t)((t >> 1) & 1));
     }
     __syncwarp();
   } else if (warp == WMMA) {
@@ -568,7 +614,16 @@ cudaError_t launch_rotate_block_quant(const RotateOperand* ops, int nops, int* s
     r.scales = o.scales;
     r.dbg = static_cast<__nv_bfloat16*>(o.dbg);
     r.B = o.B; r.H = o.H; r.S = o.S; r.layout = o.layout; r.blk = o.blk;
-    r.rotate = o.R != nullptr;
+    r.rotate = o.R != nullptr || o.hadamard;
+    r.had = o.hadamard;
+    for (int w = 0; w < 4; ++w) r.sgn[w] = o.hadamard ? o.sign_bits[w] : 0u;
+    {
+      // c = bf16(1 / sqrt(D)), round to nearest even
+      const float c32 = 1.0f / sqrtf((float)o.D);
+      uint32_t bits;
+      memcpy(&bits, &c32, 4);
+      r.cbits = ((bits + 0x7FFFu + ((bits >> 16) & 1u)) >> 16) & 0xFFFFu;
+    }
     r.chunks = (o.S + CH - 1) / CH;
     r.lblk = 0;
     while ((1 << r.lblk) < o.blk) ++r.lblk;
@@ -580,7 +635,7 @@ cudaError_t launch_rotate_block_quant(const RotateOperand* ops, int nops, int* s
     if (e != cudaSuccess) return e;
     e = make_code_map(&cmaps[n], o.codes, o.B, o.H, o.S, o.layout);
     if (e != cudaSuccess) return e;
-    if (r.rotate) {
+    if (r.rotate && !r.had) {
       // Q and K each bring their own rotation; slot by operand position.
       e = make_rot_map(&rmaps[n < 2 ? n : 1], o.R);
       if (e != cudaSuccess) return e;
