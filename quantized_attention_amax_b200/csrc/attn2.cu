@@ -132,6 +132,12 @@ enum {
 };
 static_assert(X_COUNT * 8 + 8 <= 512, "barrier block overflows its region");
 
+// Pairs of exponentials (out of every 4) that the one-tile kernel computes with the cubic on the
+// FMA pipe instead of the MUFU.
+#ifndef FAQ_MX_POLY
+#define FAQ_MX_POLY 1
+#endif
+
 template <int R>
 __device__ __forceinline__ void setmaxnreg_inc() { asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(R)); }
 template <int R>
@@ -481,8 +487,8 @@ __global__ void __launch_bounds__(Cfg<NSW>::NT, 1)
 #pragma unroll
       for (int k = 0; k < HN; k += 2) {
         ffma2(t[k], t[k + 1], cr, cr, nb, nb);
-        if (k & 2) {
-          ex2_poly2(t[k], t[k + 1]);  // every other pair on the FMA pipe
+        if (((k >> 1) & 3) < FAQ_MX_POLY) {
+          ex2_poly2(t[k], t[k + 1]);  // this share of the pairs on the FMA pipe
         } else {
           t[k] = ex2(t[k]);
           t[k + 1] = ex2(t[k + 1]);
@@ -1396,7 +1402,7 @@ Prefill2Ws carve_ws(void* ws, int B, int Hkv, int Sk, int D) {
 }
 
 #ifndef FAQ_ATTN_NSW
-#define FAQ_ATTN_NSW 4
+#define FAQ_ATTN_NSW 2
 #endif
 
 // Tensor maps over the Q and K codes and V', then the V pre-pass.
