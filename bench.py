@@ -194,6 +194,9 @@ class ClockSampler:
 
 # ------------------------------------------------------------- GPU arm ---
 
+ROTATION = "matrix"  # rotating workloads: fa_rotate_quantize with R, or fa_rotate_quantize_hadamard
+
+
 def make_step(faq, wl, w, device, seed_offset=0):
     """Allocate inputs on the device and return (step_fn, attn_fn, quant_fn, state)."""
     import torch
@@ -228,6 +231,14 @@ def make_step(faq, wl, w, device, seed_offset=0):
 
         def quant():
             faq.quantize(q, k, None, mq, w.layout, out=QK)
+    elif w.rotate and ROTATION == "hadamard":
+        # the same rotation given by its signs (R = bf16(H diag(signs) / sqrt(D)))
+        sg = wl.rotation_signs(w.D, w2.seed)
+        QKV = list(faq.rotate_quantize_hadamard(q, k, v, sg, sg, w.layout, w.q_block, w.kv_block))
+        st["QKV"] = QKV
+
+        def quant():
+            faq.rotate_quantize_hadamard(q, k, v, sg, sg, w.layout, w.q_block, w.kv_block, out=QKV)
     elif w.rotate:
         QKV = list(faq.rotate_quantize(q, k, v, inp["R"], inp["R"], w.layout, w.q_block, w.kv_block))
         st["QKV"] = QKV
@@ -396,6 +407,7 @@ def e2e_run(args, w, device, steps):
     host = {n: inp[n].pin_memory() for n in ("q", "k", "v")}
     dev = [{n: torch.empty_like(host[n], device=device) for n in host} for _ in range(2)]
     R = inp["R"].to(device) if inp.get("R") is not None else None
+    signs = wl.rotation_signs(w.D, w.seed) if w.rotate else None
     amax = None
     if w.mode in STATIC_MODES:
         amax = [faq.calibrate_per_head(inp[n + "_cal"].to(device), w.layout) for n in "qkv"]
@@ -430,6 +442,9 @@ def e2e_run(args, w, device, steps):
             if decode:
                 Q = faq.quantize(d["q"], None, None, w.mode, w.layout, amax=[amax[0], None, None])[0]
                 K, V = cache[1], cache[2]
+            elif w.rotate and ROTATION == "hadamard":
+                Q, K, V = faq.rotate_quantize_hadamard(d["q"], d["k"], d["v"], signs, signs, w.layout, w.q_block,
+                                                       w.kv_block)
             elif w.rotate:
                 Q, K, V = faq.rotate_quantize(d["q"], d["k"], d["v"], R, R, w.layout, w.q_block, w.kv_block)
             elif amax is not None:
@@ -682,7 +697,11 @@ def main():
     ap.add_argument("--no-supplemental", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--rotation", default="matrix", choices=["matrix", "hadamard"],
+                    help="rotating workloads: R from memory, or the same R given by its signs")
     args = ap.parse_args()
+    global ROTATION
+    ROTATION = args.rotation
 
     import workloads as wl
     w = wl.WORKLOADS[args.workload]
@@ -760,7 +779,10 @@ def main():
                        "l2": "flushed between steps (256 MiB device write, then a 256 MiB read so no dirty "
                              "line of the flush is left; outside the timed events)",
                        "timing": "CUDA-graph replay per launch, CUDA events on the launch stream",
-                       "parallelism": f"replicas x{world} (independent workloads per rank)"},
+                       "parallelism": f"replicas x{world} (independent workloads per rank)",
+                       **({"rotation": "R from memory (fa_rotate_quantize)" if ROTATION == "matrix" else
+                           "R = bf16(H diag(signs) / sqrt(D)) from its signs (fa_rotate_quantize_hadamard)"}
+                          if w.rotate else {})},
             "kernels_ms": {"quantize": r["quant_ms"], "attention": r["attn_ms"]},
             "quantize_roofline": {"bound": "hbm", "achieved": quant_bytes(w) / (r["quant_ms"] * 1e-3) / 1e9,
                                   "peak": pk["hbm_gbs"], "unit": "GB/s",
