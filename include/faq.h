@@ -59,7 +59,8 @@ typedef enum {
   FA_ERR_CONFIG_CONFLICT = 4, /* qconfig and details both given             */
   FA_ERR_CUDA = 5,            /* a CUDA runtime call or launch failed       */
   FA_ERR_TIMEOUT = 6,         /* a kernel's bounded wait ran out            */
-  FA_ERR_WORKSPACE = 7        /* workspace missing or too small             */
+  FA_ERR_WORKSPACE = 7,       /* workspace missing or too small             */
+  FA_ERR_BOUNDS = 8           /* FA_DEBUG_BOUNDS build: an index check failed */
 } fa_status;
 
 typedef enum { FA_LAYOUT_BNSD = 0, FA_LAYOUT_BSND = 1 } fa_layout;
@@ -330,7 +331,10 @@ FAQ_API size_t fa_attention_workspace_size_qkv(const fa_qtensor* q, const fa_qte
 
 /* Synchronise `s`, read and clear this device's status word.  Returns
  * FA_ERR_TIMEOUT if a kernel's bounded wait ran out since the last check,
- * FA_ERR_CUDA if the stream reports an error, FA_OK otherwise. */
+ * FA_ERR_BOUNDS if (in a library built with FA_DEBUG_BOUNDS) an index check
+ * failed -- the access was skipped, so the outputs are not valid --,
+ * FA_ERR_CUDA if the stream reports an error, FA_OK otherwise.  The first
+ * event since the last check is the one reported. */
 FAQ_API fa_status fa_check_device_status(fa_stream_t s);
 
 /* Static text for a status code. */

@@ -8,7 +8,9 @@ from __future__ import annotations
 import ctypes
 import os
 
-LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libfaq.so")
+# FAQ_LIB=bounds selects the bounds-checked build (libfaq_bounds.so, see build.py)
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)),
+                        "libfaq_bounds.so" if os.environ.get("FAQ_LIB") == "bounds" else "libfaq.so")
 
 # Every entry point include/faq.h declares.
 EXPORTS = (
@@ -30,7 +32,7 @@ EXPORTS = (
 
 STATUS = {
     0: "FA_OK", 1: "FA_ERR_INVALID_ARG", 2: "FA_ERR_UNSUPPORTED", 3: "FA_ERR_NO_CALIBRATION",
-    4: "FA_ERR_CONFIG_CONFLICT", 5: "FA_ERR_CUDA", 6: "FA_ERR_TIMEOUT", 7: "FA_ERR_WORKSPACE",
+    4: "FA_ERR_CONFIG_CONFLICT", 5: "FA_ERR_CUDA", 6: "FA_ERR_TIMEOUT", 7: "FA_ERR_WORKSPACE", 8: "FA_ERR_BOUNDS",
 }
 
 

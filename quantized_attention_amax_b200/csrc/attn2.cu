@@ -588,9 +588,11 @@ __global__ void __launch_bounds__(Cfg<NSW>::NT, 1)
       const float vmul = MX ? exp2f(vref - 127.0f) : vref;
       const float ofac = l_tot > 0.0f ? vmul / l_tot : 0.0f;
       __nv_bfloat16* orow = nullptr;
+      bool out_ok = row_ok;
       if (row_ok) {
         const long long ridx = p.layout == FA_LAYOUT_BNSD ? ((long long)qbh * p.Sq + row)
                                                           : (((long long)b * p.Sq + row) * p.Hq + hq);
+        out_ok = in_bounds(ridx >= 0 && ridx < (long long)p.B * p.Hq * p.Sq, 121);
         orow = p.out + ridx * D + h * DC;
       }
       constexpr int OW = DC >= 32 ? 32 : 16;  // O columns per TMEM load
@@ -607,7 +609,7 @@ __global__ void __launch_bounds__(Cfg<NSW>::NT, 1)
 #pragma unroll
           for (int k = 0; k < OW; ++k) r[k] = 0u;
         }
-        if (row_ok) {
+        if (out_ok) {
 #pragma unroll
           for (int k = 0; k < OW; k += 8) {
             uint32_t o[4];
@@ -621,7 +623,7 @@ __global__ void __launch_bounds__(Cfg<NSW>::NT, 1)
           }
         }
       }
-      if (h == 0 && row_ok && p.lse)
+      if (h == 0 && out_ok && p.lse && in_bounds((long long)qbh * p.Sq + row < (long long)p.B * p.Hq * p.Sq, 122))
         p.lse[(long long)qbh * p.Sq + row] =
             l_tot > 0.0f ? (m_run + __log2f(l_tot)) * 0.69314718055994530942f : -INFINITY;
     }
@@ -1125,9 +1127,11 @@ __global__ void __launch_bounds__(PNT, 1)
     if (q0 < p.Sq) {
       const float ofac = l_run > 0.0f ? vref / l_run : 0.0f;
       __nv_bfloat16* orow = nullptr;
+      bool out_ok = row_ok;
       if (row_ok) {
         const long long ridx = p.layout == FA_LAYOUT_BNSD ? ((long long)qbh * p.Sq + row)
                                                           : (((long long)b * p.Sq + row) * p.Hq + hq);
+        out_ok = in_bounds(ridx >= 0 && ridx < (long long)p.B * p.Hq * p.Sq, 123);
         orow = p.out + ridx * D;
       }
 #pragma unroll
@@ -1140,7 +1144,7 @@ __global__ void __launch_bounds__(PNT, 1)
 #pragma unroll
           for (int k = 0; k < 32; ++k) r[k] = 0u;
         }
-        if (row_ok) {
+        if (out_ok) {
 #pragma unroll
           for (int k = 0; k < 32; k += 8) {
             uint32_t o[4];
@@ -1154,7 +1158,7 @@ __global__ void __launch_bounds__(PNT, 1)
           }
         }
       }
-      if (row_ok && p.lse)
+      if (out_ok && p.lse && in_bounds((long long)qbh * p.Sq + row < (long long)p.B * p.Hq * p.Sq, 124))
         p.lse[(long long)qbh * p.Sq + row] =
             l_run > 0.0f ? (m_run + __log2f(l_run)) * 0.69314718055994530942f : -INFINITY;
     }
@@ -1185,6 +1189,8 @@ __global__ void __launch_bounds__(256) vprep_kernel(const uint8_t* __restrict__ 
                                                     float* __restrict__ ksp, const uint8_t* __restrict__ ve8,
                                                     const uint8_t* __restrict__ ke8) {
   const int t = blockIdx.x, bh = blockIdx.y;
+  // the tile's records and V' rows: tile t of ntiles, (b, h) row bh of the launch's B * H
+  if (!in_bounds(t < ntiles && (long long)t * BN < (long long)S + BN, 125)) return;
   const int b = bh / H, h = bh % H;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int tok0 = t * BN;
@@ -1626,6 +1632,7 @@ size_t prefill2_workspace_bytes(int B, int Hkv, int Sk, int D) {
 }
 
 cudaError_t launch_attention_prefill2(const AttnArgs& a, void* ws, cudaStream_t s) {
+  if (const cudaError_t be = bounds_attach(); be != cudaSuccess) return be;
   const fa_qtensor* q = a.q;
   const fa_qtensor* k = a.k;
   P2 prm = {};
@@ -1684,6 +1691,7 @@ size_t mixed_workspace_bytes(const fa_qtensor* q, const fa_qtensor* k) {
 }
 
 cudaError_t launch_attention_mixed(const AttnArgs& a, void* ws, cudaStream_t s) {
+  if (const cudaError_t be = bounds_attach(); be != cudaSuccess) return be;
   const fa_qtensor* q = a.q;
   const fa_qtensor* k = a.k;
   const int D = q->D;
@@ -1735,6 +1743,7 @@ cudaError_t launch_attention_mixed(const AttnArgs& a, void* ws, cudaStream_t s) 
 }
 
 cudaError_t launch_fill_empty_rows(void* out, float* lse, long long rows, int D, cudaStream_t s) {
+  if (const cudaError_t be = bounds_attach(); be != cudaSuccess) return be;
   const long long n = rows * D;
   int grid = (int)((n + 255) / 256);
   if (grid > 4096) grid = 4096;

@@ -391,6 +391,7 @@ __global__ void __launch_bounds__(DTHREADS, 2)
 #pragma unroll
     for (int h = 0; h < G; ++h) {
       const long long row = ((long long)b * p.Hq + hq0 + h) * p.splits + split;
+      if (!in_bounds(row >= 0 && row < (long long)p.B * p.Hq * p.splits, 131)) continue;
       if (i < D) p.opart[row * D + i] = ok ? Oacc[h] : 0.0f;
       if (i == 0) {
         const float Lt = lred[h] + lred[16 + h] + lred[32 + h] + lred[48 + h];
@@ -430,6 +431,7 @@ __global__ void __launch_bounds__(DTHREADS, 2)
       for (int idx = i; idx < G * D; idx += 128) {
         const int h = idx / D, d = idx - h * D;
         const long long qrow = (long long)b * p.Hq + hq0 + h;
+        if (!in_bounds(qrow >= 0 && qrow < (long long)p.B * p.Hq, 132)) continue;
         const float* mlr = p.ml + qrow * p.splits * 2;
         const float* opr = p.opart + qrow * p.splits * D + d;
         float m = -INFINITY;
@@ -532,6 +534,7 @@ namespace {
 // K / V buffers of cap tokens.
 cudaError_t run_decode(DecParams prm, const void* kcodes, const void* vcodes, int D, int kv_len, int cap, int out_layout,
                        void* out, float* lse, cudaStream_t s) {
+  if (const cudaError_t be = bounds_attach(); be != cudaSuccess) return be;
   (void)out_layout;  // Sq = 1: row (b, hq) at (b * Hq + hq) * D in either layout
   const int G = prm.group;
   prm.Sk = kv_len;

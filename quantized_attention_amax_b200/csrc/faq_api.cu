@@ -8,6 +8,7 @@
 #include <utility>
 
 #include "internal.cuh"
+#include "sm100.cuh"
 
 namespace faq {
 
@@ -159,6 +160,7 @@ const char* fa_status_str(fa_status st) {
     case FA_ERR_CUDA: return "CUDA error";
     case FA_ERR_TIMEOUT: return "kernel wait timed out";
     case FA_ERR_WORKSPACE: return "workspace missing or too small";
+    case FA_ERR_BOUNDS: return "index check failed (bounds-checked build)";
   }
   return "unknown status";
 }
@@ -474,7 +476,7 @@ fa_status fa_check_device_status(fa_stream_t s) {
   if (v != 0) {
     const int zero = 0;
     if (cudaMemcpy(p, &zero, sizeof zero, cudaMemcpyHostToDevice) != cudaSuccess) return FA_ERR_CUDA;
-    return FA_ERR_TIMEOUT;
+    return (v & 0xFF) == kStatusBounds ? FA_ERR_BOUNDS : FA_ERR_TIMEOUT;
   }
   return FA_OK;
 }

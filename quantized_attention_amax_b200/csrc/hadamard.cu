@@ -25,6 +25,7 @@
 
 #include "internal.cuh"
 #include "quant_common.cuh"
+#include "sm100.cuh"
 
 namespace faq {
 namespace {
@@ -233,7 +234,7 @@ __global__ void __launch_bounds__(HT) hadamard_block_quant_kernel(const __grid_c
     uint32_t pr[8];
     m2 = habsmax(m2, lane_rotated<D>(o, ra, rb, sub, p.c, pr));
     const int r = st * C::RPC + rsub;
-    if (o.dbg && r < rows) {
+    if (o.dbg && r < rows && in_bounds(row_off(o, b, h, s0 + r, D) < (long long)o.B * o.H * o.S * D, 151)) {
       uint4* dd = reinterpret_cast<uint4*>(o.dbg + row_off(o, b, h, s0 + r, D)) + 2 * sub;
       dd[0] = make_uint4(pr[0], pr[1], pr[2], pr[3]);
       dd[1] = make_uint4(pr[4], pr[5], pr[6], pr[7]);
@@ -255,7 +256,7 @@ __global__ void __launch_bounds__(HT) hadamard_block_quant_kernel(const __grid_c
 #pragma unroll
   for (int w = 0; w < HT / 32; ++w) m = fmaxf(m, wmax[w]);
   const float sc = __fdiv_rn(m, 448.0f);
-  if (tid == 0) o.scales[bh * o.nblk + g] = sc;
+  if (tid == 0 && in_bounds(bh * o.nblk + g < (long long)o.B * o.H * o.nblk, 152)) o.scales[bh * o.nblk + g] = sc;
   // pass 2: codes, one coalesced 16-byte store per lane and row
   for (int st = 0; st < nsteps; ++st) {
     uint32_t pr[8];
@@ -272,7 +273,8 @@ __global__ void __launch_bounds__(HT) hadamard_block_quant_kernel(const __grid_c
       lane_rotated<D>(o, ra, rb, sub, p.c, pr);
     }
     const int r = st * C::RPC + rsub;
-    if (r < rows) reinterpret_cast<uint4*>(o.codes + row_off(o, b, h, s0 + r, D))[sub] = lane_codes(pr, sc);
+    if (r < rows && in_bounds(row_off(o, b, h, s0 + r, D) < (long long)o.B * o.H * o.S * D, 153))
+      reinterpret_cast<uint4*>(o.codes + row_off(o, b, h, s0 + r, D))[sub] = lane_codes(pr, sc);
   }
 }
 
@@ -290,6 +292,7 @@ cudaError_t launch_had(const HadParams& prm, long long ctas, cudaStream_t s) {
 }  // namespace
 
 cudaError_t launch_hadamard_block_quant(const HadamardOperand* ops, int nops, cudaStream_t s) {
+  if (const cudaError_t be = bounds_attach(); be != cudaSuccess) return be;
   HadParams prm = {};
   long long ctas = 0;
   int D = 0;

@@ -24,8 +24,29 @@ struct QuantOperand {
   int lS, lH;          // their shifts
 };
 
-// Per-device status word (timeouts recorded by bounded waits).
+// Per-device status word (timeouts recorded by bounded waits; failed index checks in
+// FA_DEBUG_BOUNDS builds).
 int* device_status_ptr();
+
+// FA_DEBUG_BOUNDS builds: point this translation unit's index checks at the device status word
+// (once per device); a no-op otherwise.  Each launcher calls it before its launches.
+#ifdef FA_DEBUG_BOUNDS
+inline cudaError_t bounds_attach_impl(const void* symbol) {
+  static int done[64] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess || dev < 0 || dev >= 64) return e;
+  if (done[dev]) return cudaSuccess;
+  int* p = device_status_ptr();
+  if (!p) return cudaErrorUnknown;
+  if ((e = cudaMemcpyToSymbol(symbol, &p, sizeof p)) != cudaSuccess) return e;
+  done[dev] = 1;
+  return cudaSuccess;
+}
+#define bounds_attach() bounds_attach_impl(reinterpret_cast<const void*>(&g_bounds_status))
+#else
+#define bounds_attach() cudaSuccess
+#endif
 
 // Driver entry point for tensor-map encoding (resolved once).
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,

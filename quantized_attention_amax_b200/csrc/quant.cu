@@ -159,8 +159,10 @@ __global__ void __launch_bounds__(kRowThreads) quant_rows_kernel(QuantOperand o0
     void* const op_scales = which == 0 ? o0.scales : (which == 1 ? o1.scales : o2.scales);
     uint4 raw[4];
     const uint4* src = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(op_x) + rr * D) + gl * 4;
+    const long long op_rows = which == 0 ? o0.rows : (which == 1 ? o1.rows : o2.rows);
+    const bool ld_ok = valid && in_bounds(rr * D + (gl + 1) * 32 <= op_rows * D, 101);
 #pragma unroll
-    for (int c = 0; c < 4; ++c) raw[c] = valid ? __ldg(src + c) : make_uint4(0, 0, 0, 0);
+    for (int c = 0; c < 4; ++c) raw[c] = ld_ok ? __ldg(src + c) : make_uint4(0, 0, 0, 0);
     // max |x| over the lane's 32 elements on the packed bf16 pairs (exact, no unpacking)
     float m = 0.0f;
     if (!PER_HEAD) {
@@ -191,8 +193,10 @@ __global__ void __launch_bounds__(kRowThreads) quant_rows_kernel(QuantOperand o0
             w[2 * c + 1] = e4m3x4(f[4] * inv, f[5] * inv, f[6] * inv, f[7] * inv);
           }
           uint4* dst = reinterpret_cast<uint4*>(static_cast<uint8_t*>(op_codes) + rr * D + gl * 32);
-          dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
-          dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
+          if (in_bounds(rr * D + (gl + 1) * 32 <= op_rows * D, 102)) {
+            dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
+            dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
+          }
         } else {
           uint32_t w[4];
 #pragma unroll
@@ -203,13 +207,15 @@ __global__ void __launch_bounds__(kRowThreads) quant_rows_kernel(QuantOperand o0
             for (int k = 0; k < 8; ++k) v8[k] *= inv;
             w[i] = e2m1x8(v8);
           }
-          *reinterpret_cast<uint4*>(static_cast<uint8_t*>(op_codes) + rr * (D / 2) + gl * 16) =
-              make_uint4(w[0], w[1], w[2], w[3]);
+          if (in_bounds(rr * (D / 2) + (gl + 1) * 16 <= op_rows * (D / 2), 103))
+            *reinterpret_cast<uint4*>(static_cast<uint8_t*>(op_codes) + rr * (D / 2) + gl * 16) =
+                make_uint4(w[0], w[1], w[2], w[3]);
         }
         const int op_layout = which == 0 ? o0.layout : (which == 1 ? o1.layout : o2.layout);
         const int op_H = which == 0 ? o0.H : (which == 1 ? o1.H : o2.H);
         const int op_S = which == 0 ? o0.S : (which == 1 ? o1.S : o2.S);
-        static_cast<uint8_t*>(op_scales)[scale_index(rr, op_layout, op_H, op_S) * (D / 32) + gl] = (uint8_t)(e + 127);
+        const long long si = scale_index(rr, op_layout, op_H, op_S) * (D / 32) + gl;
+        if (in_bounds(si >= 0 && si < op_rows * (D / 32), 104)) static_cast<uint8_t*>(op_scales)[si] = (uint8_t)(e + 127);
       }
       continue;
     }
@@ -233,7 +239,7 @@ __global__ void __launch_bounds__(kRowThreads) quant_rows_kernel(QuantOperand o0
         const int h = (int)(hs - fast_div(hs, mH, lH) * (uint32_t)op_H);
         // the static scale and its reciprocal, recomputed per row (a per-CTA table behind a
         // barrier measured slower: each CTA handles only a few rows)
-        const float a = __ldg((which == 0 ? o0.amax : (which == 1 ? o1.amax : o2.amax)) + h);
+        const float a = in_bounds(h >= 0 && h < op_H, 107) ? __ldg((which == 0 ? o0.amax : (which == 1 ? o1.amax : o2.amax)) + h) : 0.0f;
         sc = __fdiv_rn(a, QMAX);
         rc = sc >= kFastDivMin ? __frcp_rn(sc) : 0.0f;
         lim = fabsf(a) < INFINITY ? a : -1.0f;
@@ -293,13 +299,16 @@ __global__ void __launch_bounds__(kRowThreads) quant_rows_kernel(QuantOperand o0
       out[0] = make_uint4(w[0], w[1], w[2], w[3]);
       out[1] = make_uint4(w[4], w[5], w[6], w[7]);
       uint4* dst = reinterpret_cast<uint4*>(static_cast<uint8_t*>(op_codes) + rr * D + gl * 32);
-      dst[0] = out[0];
-      dst[1] = out[1];
+      if (in_bounds(rr * D + (gl + 1) * 32 <= op_rows * D, 105)) {
+        dst[0] = out[0];
+        dst[1] = out[1];
+      }
       if (!PER_HEAD && gl == 0) {
         const int op_layout = which == 0 ? o0.layout : (which == 1 ? o1.layout : o2.layout);
         const int op_H = which == 0 ? o0.H : (which == 1 ? o1.H : o2.H);
         const int op_S = which == 0 ? o0.S : (which == 1 ? o1.S : o2.S);
-        static_cast<float*>(op_scales)[scale_index(rr, op_layout, op_H, op_S)] = sc;
+        const long long si = scale_index(rr, op_layout, op_H, op_S);
+        if (in_bounds(si >= 0 && si < op_rows, 106)) static_cast<float*>(op_scales)[si] = sc;
       }
     }
   }
@@ -322,6 +331,8 @@ __global__ void __launch_bounds__(256) calibrate_kernel(const __nv_bfloat16* __r
                                                        : x + (long long)b * S * H * D + (long long)h * D;
     for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < nvec;
          i += (long long)gridDim.x * blockDim.x) {
+      const long long off = (xb - x) + (i >> VSH) * rstride + (i & (VPR - 1)) * 8;
+      if (!in_bounds(off >= 0 && off + 8 <= (long long)B * H * S * D, 108)) continue;
       const uint4 u = __ldg(reinterpret_cast<const uint4*>(xb + (i >> VSH) * rstride) + (i & (VPR - 1)));
       float f[8];
       unpack_bf16x8(u, f);
@@ -355,6 +366,8 @@ __global__ void __launch_bounds__(256) fp8_block_kernel(QuantOperand op) {
   };
   float m = 0.0f;
   for (int i = threadIdx.x; i < nvec; i += blockDim.x) {
+    const long long nrows = (long long)op.B * op.H * op.S;
+    if (!in_bounds(row_of(s0 + i / vpr) < nrows, 109)) continue;
     const uint4 u = __ldg(reinterpret_cast<const uint4*>(x + row_of(s0 + i / vpr) * op.D) + (i % vpr));
     float f[8];
     unpack_bf16x8(u, f);
@@ -372,13 +385,15 @@ __global__ void __launch_bounds__(256) fp8_block_kernel(QuantOperand op) {
     for (int w = 0; w < (int)(blockDim.x >> 5); ++w) bm = fmaxf(bm, wm[w]);
     s_sc = __fdiv_rn(bm, 448.0f);
     const int nblk = (op.S + op.blk - 1) / op.blk;
-    static_cast<float*>(op.scales)[((long long)b * op.H + h) * nblk + g] = s_sc;
+    if (in_bounds(((long long)b * op.H + h) * nblk + g < (long long)op.B * op.H * nblk, 110))
+      static_cast<float*>(op.scales)[((long long)b * op.H + h) * nblk + g] = s_sc;
   }
   __syncthreads();
   const float sc = s_sc;
   const float rc = sc >= kFastDivMin ? __frcp_rn(sc) : 0.0f;
   for (int i = threadIdx.x; i < nvec; i += blockDim.x) {
     const long long row = row_of(s0 + i / vpr);
+    if (!in_bounds(row < (long long)op.B * op.H * op.S, 111)) continue;
     const uint4 u = __ldg(reinterpret_cast<const uint4*>(x + row * op.D) + (i % vpr));
     float f[8];
     unpack_bf16x8(u, f);
@@ -406,6 +421,7 @@ void fastdiv_magic(long long d, uint32_t& m, int& l) {
 
 template <int MODE>
 cudaError_t launch_rows_mode(const QuantOperand (&oi)[3], int D, cudaStream_t s) {
+  if (const cudaError_t be = bounds_attach(); be != cudaSuccess) return be;
   const long long total = oi[0].rows + oi[1].rows + oi[2].rows;
   constexpr bool PER_HEAD = MODE == FA_MODE_INT8_PER_HEAD || MODE == FA_MODE_FP8_PER_HEAD;
   if (total == 0 && !PER_HEAD) return cudaSuccess;
@@ -429,6 +445,7 @@ cudaError_t launch_rows_mode(const QuantOperand (&oi)[3], int D, cudaStream_t s)
 }  // namespace
 
 cudaError_t launch_calibrate(const QuantOperand& op, float* amax, cudaStream_t s) {
+  if (const cudaError_t be = bounds_attach(); be != cudaSuccess) return be;
   const long long nvec = (long long)op.B * op.S * (op.D / 8);
   if (nvec == 0) return cudaSuccess;
   if (op.H > 65535) return cudaErrorInvalidValue;
@@ -467,6 +484,7 @@ cudaError_t launch_quantize_rows(int mode, const QuantOperand* ops, int nops, cu
 }
 
 cudaError_t launch_quantize_fp8_block(const QuantOperand* ops, int nops, cudaStream_t s) {
+  if (const cudaError_t be = bounds_attach(); be != cudaSuccess) return be;
   for (int i = 0; i < nops; ++i) {
     const QuantOperand& op = ops[i];
     if (op.rows == 0) continue;

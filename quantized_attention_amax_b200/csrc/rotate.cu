@@ -267,7 +267,8 @@ __device__ __forceinline__ void stage_codes(const RotOp& op, const RItem& it, co
   const float sc = __fdiv_rn(m, 448.0f);
   if (part == 0 && (r_in & (op.blk - 1)) == 0) {
     const int nblk = (op.S + op.blk - 1) >> op.lblk;
-    op.scales[((long long)it.b * op.H + it.h) * nblk + (t >> op.lblk)] = sc;
+    const long long si = ((long long)it.b * op.H + it.h) * nblk + (t >> op.lblk);
+    if (in_bounds(si >= 0 && si < (long long)op.B * op.H * nblk, 141)) op.scales[si] = sc;
   }
   if (sc >= kFastDivMin) {
     const float rc = __frcp_rn(sc);
@@ -502,7 +503,7 @@ __global__ void __launch_bounds__(RTHREADS, 1)
         am = fmaxf(__uint_as_float(m2 << 16), __uint_as_float(m2 & 0xFFFF0000u));
       }
       const long long ridx = bnsd ? (((long long)it.b * op.H + it.h) * op.S + t) : (((long long)it.b * op.S + t) * op.H + it.h);
-      if (live && op.dbg) {
+      if (live && op.dbg && in_bounds(ridx >= 0 && ridx < (long long)op.B * op.H * op.S, 142)) {
         uint4* d = reinterpret_cast<uint4*>(op.dbg + ridx * 128 + part * CW);
 #pragma unroll
         for (int q = 0; q < CW / 8; ++q) d[q] = make_uint4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
@@ -596,6 +597,7 @@ cudaError_t make_rot_map(CUtensorMap* map, const void* R) {
 }  // namespace
 
 cudaError_t launch_rotate_block_quant(const RotateOperand* ops, int nops, int* status, cudaStream_t s) {
+  if (const cudaError_t be = bounds_attach(); be != cudaSuccess) return be;
   RotParams prm = {};
   prm.status = status;
   CUtensorMap maps[3], rmaps[2], cmaps[3];

@@ -24,7 +24,23 @@ namespace faq {
 enum : int {
   kStatusOk = 0,
   kStatusTimeout = 1,
+  kStatusBounds = 2,  // FA_DEBUG_BOUNDS builds: an index check failed (the access was skipped)
 };
+
+// FA_DEBUG_BOUNDS builds check the index of each computed global access against the extent the
+// kernel's arguments give that buffer before making it: a failed check records the site and
+// kStatusBounds in the device status word and skips the access, so it never faults.  The status
+// word's device address reaches each translation unit's kernels through a file-local symbol that
+// bounds_attach() sets once per device.  Ordinary builds compile every check to true.
+#ifdef FA_DEBUG_BOUNDS
+static __device__ int* g_bounds_status;
+__device__ __forceinline__ bool in_bounds(bool ok, int where) {
+  if (!ok && g_bounds_status) atomicCAS(g_bounds_status, 0, (where << 8) | kStatusBounds);
+  return ok;
+}
+#else
+__device__ __forceinline__ constexpr bool in_bounds(bool, int) { return true; }
+#endif
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));

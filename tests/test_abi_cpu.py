@@ -42,9 +42,20 @@ def test_library_exports_every_declared_symbol(N):
 
 def test_status_strings(N):
     L = N.lib()
-    for code in range(8):
+    for code in range(9):
         assert L.fa_status_str(code)
+    assert L.fa_status_str(8) != L.fa_status_str(99)  # FA_ERR_BOUNDS has its own text
     assert b"x" in L.fa_version() or L.fa_version()
+
+
+def test_bounds_checked_build_exports_the_same_boundary():
+    """The FA_DEBUG_BOUNDS build (index checks that set the status word instead of faulting)
+    compiles from the same sources and exports the same symbols."""
+    from quantized_attention_amax_b200 import build
+    path = build.build(bounds=True)
+    out = subprocess.run(["nm", "-D", "--defined-only", path], capture_output=True, text=True).stdout
+    exported = set(re.findall(r"\bT (fa_\w+)", out))
+    assert set(declared_symbols()) <= exported
 
 
 def test_resolve_config_rules():
