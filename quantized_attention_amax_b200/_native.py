@@ -8,9 +8,12 @@ from __future__ import annotations
 import ctypes
 import os
 
-# FAQ_LIB=bounds selects the bounds-checked build (libfaq_bounds.so, see build.py)
-LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)),
-                        "libfaq_bounds.so" if os.environ.get("FAQ_LIB") == "bounds" else "libfaq.so")
+# FAQ_LIB=bounds selects the bounds-checked build (libfaq_bounds.so, see build.py); an absolute
+# path selects another build of the same library
+_sel = os.environ.get("FAQ_LIB", "")
+LIB_PATH = (_sel if os.path.isabs(_sel) else
+            os.path.join(os.path.dirname(os.path.abspath(__file__)),
+                         "libfaq_bounds.so" if _sel == "bounds" else "libfaq.so"))
 
 # Every entry point include/faq.h declares.
 EXPORTS = (
