@@ -118,6 +118,38 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
   }
 }
 
+// Non-blocking probe of the phase with the given parity.
+__device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// The same bounded wait as mbar_wait, polling with test_wait instead of suspending: the thread
+// sees the phase complete within a few cycles, at the price of issue slots while it waits.
+__device__ __forceinline__ bool mbar_wait_spin(uint64_t* bar, uint32_t parity, volatile int* abort, int* status,
+                                               int where) {
+  if (mbar_test_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  for (uint32_t it = 1;; ++it) {
+    if (mbar_test_wait(bar, parity)) return true;
+    if ((it & 255u) == 0) {
+      if (*abort) return false;
+      if (globaltimer_ns() - t0 > FAQ_WAIT_NS) {
+        *abort = 1;
+        if (status) atomicCAS(status, 0, (where << 8) | kStatusTimeout);
+        return false;
+      }
+    }
+  }
+}
+
 // Bounded wait that ignores the abort flag: for a CTA draining its own loads and MMAs already in
 // flight (whose phases complete by themselves) before it frees TMEM or leaves.  Gives up after
 // FAQ_WAIT_NS.
