@@ -287,8 +287,11 @@ class L2Flush:
 
 def launches_per_step(w):
     """This library's kernels per step: the quantize (or rotate + quantize) launch, then
-    the attention call: decode + LSE combine, or for prefill the V' pre-pass and the
-    attention kernel (mixed branches: one bf16 dequantize launch per quantized Q / K first)."""
+    the attention call: the split-KV decode kernel (its last CTA per head combines the
+    partials), or for prefill the V' pre-pass and the attention kernel (mixed branches: one
+    bf16 dequantize launch per quantized Q / K first)."""
+    if w.name == "int8_decode":
+        return 1 + 1
     if w.branch_modes is not None:
         return 1 + sum(m != "float" for m in w.branch_modes[:2]) + 2
     return 1 + 2
@@ -297,11 +300,11 @@ def launches_per_step(w):
 def attention_kernels(w):
     """(label, source file) of the attention call's kernels for this workload."""
     if w.name == "int8_decode":
-        return "decode_kernel + attn_combine_kernel", "decode.cu"
+        return "decode_kernel with the LSE combine fused (one fa_attention_quant call)", "decode.cu"
     if w.branch_modes is not None:
         return "deq_bf16_kernel x2 + vprep_kernel + attn_pair_kernel<bf16> (one fa_attention_quant call)", "attn2.cu"
     if w.mode in ("mxfp4", "mxfp8"):
-        return "vprep_kernel + attn2_kernel (one fa_attention_quant call)", "attn2.cu"
+        return "vprep_kernel + attn_pair_kernel<MX, 112-key tiles> (one fa_attention_quant call)", "attn2.cu"
     return "vprep_kernel + attn_pair_kernel (one fa_attention_quant call)", "attn2.cu"
 
 

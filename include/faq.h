@@ -313,9 +313,9 @@ FAQ_API size_t fa_decode_append_workspace_size(const fa_tensor* q, const fa_qten
 
 /* Workspace bytes fa_attention_quant needs for these operands and split
  * count: decode B*Hq*splits*(D+2)*4; prefill (every mode, the MX modes with
- * D == 128 only) B*Hkv*Sk*D*2 + B*Hkv*ceil(Sk/128)*16 +
- * B*Hkv*ceil(Sk/128)*512, each part rounded up to 256.  Returns 0 on
- * invalid arguments. */
+ * D == 128 only) B*Hkv*Sk*D*2 + B*Hkv*T*16 + B*Hkv*T*512, each part rounded
+ * up to 256, with T the number of key tiles: ceil(Sk/112) for the MX modes
+ * (MXFP4, MXFP8), ceil(Sk/128) otherwise.  Returns 0 on invalid arguments. */
 FAQ_API size_t fa_attention_workspace_size(const fa_qtensor* q, const fa_qtensor* k, int num_splits);
 
 /* The same for any three branches: equal to fa_attention_workspace_size when

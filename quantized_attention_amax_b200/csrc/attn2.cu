@@ -4,36 +4,17 @@
 //
 // Two kernels per call:
 //   vprep: V codes -> V' = fp16(code * s_v / r_t) once per call, r_t = the
-//     largest V scale of 128-key tile t (INT8: V' = fp16(code), exact; MXFP4:
-//     V' = fp16(e2m1 * 2^(e - E_t)) with E_t the tile's largest block exponent),
+//     largest V scale of key tile t (INT8: V' = fp16(code), exact; MX:
+//     V' = fp16(code * 2^(e - E_t)) with E_t the tile's largest block exponent),
 //     into a caller workspace, with r_t beside it.  Every query tile reads the
 //     same V tiles, so the conversion is done once instead of once per query
 //     tile.  The same pass lays out each K tile's scales for the attention:
-//     128 per-key floats (E4M3) or the tile's UE8M0 scale-factor atom (MXFP4).
-//   attn2: one CTA owns one 128-row query tile of one head and streams its
-//     visible 128-key tiles.  S is double-buffered in TMEM, so Q K^T of tile
-//     j+1 runs on the tensor pipe while the softmax of tile j runs on the SM
-//     cores:
-//   warpgroup 0 (setmaxnreg shrinks it):
-//     warp 0   Q once, then per tile the K codes (3-stage ring), by TMA.
-//     warp 3   per tile the V' tile (2-stage ring), by TMA.
-//     warp 2   per tile the K scales (or atom) and the V' factor record into a
-//              4-stage shared ring by bulk copies; MXFP4: Q's scale atom.
-//     warp 1   MMA issuer (one thread): S_b = Q K^T (kind::f8f6f4 / kind::i8 /
-//              kind::mxf4 with the 32-element block scales copied into TMEM
-//              beside the accumulators) into TMEM buffer b = j % 2, and
-//              O += P' V' (kind::f16, A = P' read from TMEM where the softmax
-//              stored it over S_b).  QK(j+2) is issued right after PV(j); the
-//              tensor pipe runs them in order, so P'_b is consumed before S_b
-//              is rewritten.
-//   NSW softmax warpgroups (setmaxnreg grows them): one thread per (query row,
-//     128 / NSW keys of the tile): S from TMEM, per-key K scale, mask, the
-//     tile's row maximum combined across the groups through shared memory,
-//     online max in the exp2 domain (O rescaled in TMEM only when the max grows
-//     by more than 2^8), p = exp2(t * c - m), and P' = fp16(p * r_t / v_ref)
-//     (the factor enters the exponent; the row sum takes p itself) stored over
-//     the group's own S columns (tcgen05.st).
-// TMEM: S_0/P'_0, S_1/P'_1, O, and for MXFP4 the Q and K scale factors.
+//     128 per-key floats (E4M3, INT8 per token) or the tile's UE8M0
+//     scale-factor atom (MX).
+//   attn_pair: one CTA owns two 128-row query tiles that read the same K / V'
+//     tiles (the layout and schedule are described above the kernel).  Key
+//     tiles hold 128 keys, or 112 for the MX kinds, whose block-scale factors
+//     need TMEM columns beside the two S tiles and two O accumulators.
 // Every wait is bounded.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
@@ -49,20 +30,7 @@ using namespace attn;
 
 constexpr int BM = 128;
 constexpr int BN = 128;
-// NSW softmax warpgroups share each S tile, NSW * 128 + 128 threads.
-template <int NSW>
-struct Cfg {
-  static constexpr int NT = 128 * (NSW + 1);
-  static constexpr int HN = BN / NSW;  // keys per softmax thread and tile
-  // setmaxnreg split of the launch's registers (65536 / NT, rounded down to 8, per thread):
-  // warpgroup 0 shrinks to R0, the softmax warpgroups grow to RS; 128 * R0 + NSW * 128 * RS
-  // stays within NT * (launch registers).
-  static constexpr int R0 = NSW == 2 ? 88 : 56;
-  static constexpr int RS = NSW == 2 ? 208 : 104;
-  static_assert(128 * R0 + NSW * 128 * RS <= NT * ((65536 / NT) & ~7), "register split exceeds the launch");
-};
 constexpr int NKS = 3;      // K code stages
-constexpr int NVS = 2;      // V' stages
 constexpr int NSC = 4;      // scale ring stages
 
 // per half: max(|a|, |b|), its sign the XOR of the inputs' signs (only magnitudes are used)
@@ -102,554 +70,18 @@ struct P2 {
   int pair_heads;  // two-tile kernel: 1 = the two tiles are query heads 2h, 2h+1 at one row block, 0 = row blocks 2t, 2t+1 of one head
 };
 
-template <int KIND, int D>
-struct L2 {
-  static constexpr uint32_t RB = KIND == K_MXF4 ? D / 2 : D;  // code bytes per token row (E2M1: two per byte)
-  static constexpr uint32_t Q = 0;                     // [128][RB]
-  static constexpr uint32_t K = Q + BM * RB;           // NKS stages
-  static constexpr uint32_t VH = K + NKS * BN * RB;    // NVS stages of fp16 V'
-  static constexpr uint32_t SC = VH + NVS * BN * D * 2;  // NSC stages x ([128] k scale, V' factor log2, its inverse)
-  static constexpr uint32_t XM = SC + NSC * 2 * BN * 4;  // 2 stages x 4 key groups x [128] tile row max
-  static constexpr uint32_t XL = XM + 2 * 4 * BM * 4;    // 4 key groups x [128] row sum
-  static constexpr uint32_t MISC = XL + 4 * BM * 4;
-  static constexpr uint32_t SFA = MISC + 64;           // MXFP4: Q scale-factor atom (512 B)
-  static constexpr uint32_t BAR = SFA + 512;
-  static constexpr uint32_t TOTAL = BAR + 512;
-  static constexpr uint32_t ALLOC = TOTAL + 1024;
-  static_assert(ALLOC <= 227 * 1024, "shared memory per CTA");
-};
-
-// mbarrier slots, laid out from the ring depths
-enum {
-  X_Q = 0,
-  X_KF = 1,              // [NKS] K stage full
-  X_KE = X_KF + NKS,     // [NKS] K stage empty
-  X_VF = X_KE + NKS,     // [NVS] V' stage full
-  X_VE = X_VF + NVS,     // [NVS] V' stage empty
-  X_SF = X_VE + NVS,     // [2] S buffer full
-  X_PF = X_SF + 2,       // [2] P' buffer full
-  X_PVD = X_PF + 2,      // P V done
-  X_SCF = X_PVD + 1,     // [NSC] scale ring stage full
-  X_SCE = X_SCF + NSC,   // [NSC] scale ring stage empty
-  X_MX = X_SCE + NSC,    // [2] row-max exchange
-  X_LX = X_MX + 2,       // row-sum exchange
-  X_FIN = X_LX + 1,
-  X_COUNT = X_FIN + 1
-};
-static_assert(X_COUNT * 8 + 8 <= 512, "barrier block overflows its region");
-
-// Pairs of exponentials (out of every 4) that the one-tile kernel computes with the cubic on the
-// FMA pipe instead of the MUFU.
-#ifndef FAQ_MX_POLY
-#define FAQ_MX_POLY 1
-#endif
-
 template <int R>
 __device__ __forceinline__ void setmaxnreg_inc() { asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(R)); }
 template <int R>
 __device__ __forceinline__ void setmaxnreg_dec() { asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(R)); }
 
-template <int KIND, int D, int SC, int NSW>
-__global__ void __launch_bounds__(Cfg<NSW>::NT, 1)
-    attn2_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
-                 const __grid_constant__ CUtensorMap tmv, const P2 p) {
-  static_assert(KIND == K_E4M3 || SC == SC_HEAD, "INT8 and MXFP4 operands take no per-key scale path");
-  constexpr bool MX = KIND == K_MXF4 || KIND == K_MXF8;  // block-scaled QK^T (UE8M0 factors in TMEM)
-  constexpr bool RING = MX || SC != SC_HEAD;  // per-tile records (and K scales / atoms) through the scale ring
-  using L = L2<KIND, D>;
-  constexpr uint32_t RB = L::RB;
-  constexpr int HN = Cfg<NSW>::HN;
-  constexpr int NSWW = 4 * NSW;   // softmax warps
-  constexpr int DC = D / NSW;     // O columns per softmax thread
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* bar = reinterpret_cast<uint64_t*>(smem + L::BAR);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar + X_COUNT);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(bar + X_COUNT + 1);
-  float* misc = reinterpret_cast<float*>(smem + L::MISC);  // [0] = v_ref (MXFP4: E_ref)
-
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-
-  // ---- work item: (b, query head, query tile); causal runs the longest tiles first
-  int b, hq, q0;
-  {
-    const int per_t = p.B * p.Hq;
-    const int widx = blockIdx.x;
-    const int qt = p.causal ? (p.n_qtiles - 1 - widx / per_t) : (widx / per_t);
-    const int r = widx % per_t;
-    b = r / p.Hq;
-    hq = r % p.Hq;
-    q0 = qt * BM;
-  }
-  const int hk = hq / p.group;
-  const int diag = p.Sk - p.Sq;
-  int kv_end = 0;
-  if (q0 < p.Sq) kv_end = p.causal ? min(p.Sk, max(0, min(q0 + BM, p.Sq) - 1 + diag + 1)) : p.Sk;
-  const int n = (kv_end + BN - 1) / BN;
-  const int bhk = b * p.Hkv + hk;
-
-  if (tid == 0) {
-    mbar_init(&bar[X_Q], MX ? 2 : 1);  // MXFP4: the Q codes and the Q scale-factor atom
-    for (int i = 0; i < NKS; ++i) {
-      mbar_init(&bar[X_KF + i], 1);
-      mbar_init(&bar[X_KE + i], 1);
-    }
-    for (int i = 0; i < NVS; ++i) {
-      mbar_init(&bar[X_VF + i], 1);
-      mbar_init(&bar[X_VE + i], 1);
-    }
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(&bar[X_SF + i], 1);
-      mbar_init(&bar[X_PF + i], NSWW);
-      mbar_init(&bar[X_MX + i], NSWW);
-    }
-    for (int i = 0; i < NSC; ++i) {
-      mbar_init(&bar[X_SCF + i], 1);
-      mbar_init(&bar[X_SCE + i], NSWW);  // the softmax warps
-    }
-    mbar_init(&bar[X_PVD], 1);
-    mbar_init(&bar[X_LX], NSWW);
-    mbar_init(&bar[X_FIN], 1);
-    *abort_flag = 0;
-    fence_barrier_init();
-  }
-  if (warp == 1) {
-    tmem_alloc(tmem_slot, 512);
-    tmem_relinquish();
-  }
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tbase = *tmem_slot;
-  const uint32_t tO = tbase + 256;
-  const uint32_t tSFA = tbase + 384;  // MXFP4 scale factors: Q, then K for S buffers 0 and 1
-  const uint32_t tSFB[2] = {tbase + 392, tbase + 400};
-
-  if (warp < 4) {
-    setmaxnreg_dec<Cfg<NSW>::R0>();
-    const bool bnsd = p.layout == FA_LAYOUT_BNSD;
-    if (warp == 0) {
-      // ------------------------------------------------------ Q and K loads
-      if (lane == 0 && n > 0) {
-        tma_prefetch_desc(&tmq);
-        tma_prefetch_desc(&tmk);
-        mbar_arrive_expect_tx(&bar[X_Q], BM * RB);
-        tma_load_4d(smem + L::Q, &tmq, &bar[X_Q], 0, bnsd ? q0 : hq, bnsd ? hq : q0, b);
-        int j = 0;
-        for (; j < n; ++j) {
-          const int k0 = j * BN, ks = j % NKS;
-          if (j >= NKS && !mbar_wait(&bar[X_KE + ks], ((j / NKS) - 1) & 1, abort_flag, p.status, 61)) break;
-          mbar_arrive_expect_tx(&bar[X_KF + ks], BN * RB);
-          tma_load_4d(smem + L::K + ks * BN * RB, &tmk, &bar[X_KF + ks], 0, bnsd ? k0 : hk, bnsd ? hk : k0, b);
-        }
-        if (*abort_flag) {
-          // let issued loads land before the CTA can exit
-          mbar_drain(&bar[X_Q], 0);
-          for (int t = max(0, j - NKS); t < j; ++t) mbar_drain(&bar[X_KF + t % NKS], (t / NKS) & 1);
-        }
-      }
-      __syncwarp();
-    } else if (warp == 3) {
-      // --------------------------------------------------------- V' loads
-      if (lane == 0 && n > 0) {
-        tma_prefetch_desc(&tmv);
-        int j = 0;
-        for (; j < n; ++j) {
-          const int k0 = j * BN, vs = j % NVS;
-          if (j >= NVS && !mbar_wait(&bar[X_VE + vs], ((j / NVS) - 1) & 1, abort_flag, p.status, 62)) break;
-          // V' [b][hk][token][D] fp16: one 64-column box per 128-byte swizzle atom
-          mbar_arrive_expect_tx(&bar[X_VF + vs], BN * D * 2);
-#pragma unroll
-          for (int a2 = 0; a2 < D / 64; ++a2)
-            tma_load_4d(smem + L::VH + vs * BN * D * 2 + a2 * BN * 128, &tmv, &bar[X_VF + vs], 64 * a2, k0, hk, b);
-        }
-        if (*abort_flag)
-          for (int t = max(0, j - NVS); t < j; ++t) mbar_drain(&bar[X_VF + t % NVS], (t / NVS) & 1);
-      }
-      __syncwarp();
-    } else if (warp == 2) {
-      // ------------------------------------------------------- scale ring
-      // Per tile, the pre-pass's 128 per-key K scales (MXFP4: the K scale-factor atom) and
-      // the V' factor record land in a ring stage by two bulk copies (512 + 16 bytes) that
-      // complete on the stage's barrier.
-      if (MX && n > 0) {
-        // Q's scale-factor atom, published with the Q codes' barrier
-        write_sf_atom(smem + L::SFA, p.qe8, (long long)(b * p.Hq + hq) * p.Sq + q0, p.Sq - q0, lane);
-        fence_async_smem();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&bar[X_Q]);
-      }
-      if (RING && n > 0) {
-        const float4* fvh = p.fvr + (long long)bhk * p.ntiles_k;
-        float m = 0.0f;
-        for (int t = lane; t < n; t += 32) m = fmaxf(m, __ldg(&fvh[t].x));
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
-        if (lane == 0) {
-          // v_ref: the largest V' factor over this CTA's visible tiles (MXFP4: the largest E_t)
-          misc[0] = MX ? m : (m > 0.0f ? m : 1.0f);
-          const float* kph = p.ksp + (long long)bhk * p.ntiles_k * BN;
-          int j = 0;
-          for (; j < n; ++j) {
-            const int st = j % NSC;
-            if (j >= NSC && !mbar_wait(&bar[X_SCE + st], ((j / NSC) - 1) & 1, abort_flag, p.status, 60)) break;
-            uint8_t* stage = smem + L::SC + st * 2 * BN * 4;
-            mbar_arrive_expect_tx(&bar[X_SCF + st], BN * 4 + 16);
-            bulk_load(stage, kph + (long long)j * BN, BN * 4, &bar[X_SCF + st]);
-            bulk_load(stage + BN * 4, fvh + j, 16, &bar[X_SCF + st]);
-          }
-          if (*abort_flag)
-            for (int t = max(0, j - NSC); t < j; ++t) mbar_drain(&bar[X_SCF + t % NSC], (t / NSC) & 1);
-        }
-      }
-      __syncwarp();
-    } else if (warp == 1) {
-      // ---------------------------------------------------------- MMA issuer
-      if (lane == 0 && n > 0) {
-        constexpr uint32_t SW = RB == 128 ? kSwz128 : kSwz64;
-        constexpr uint32_t SBO8 = RB == 128 ? 1024 : 512;
-        constexpr uint32_t idesc_qk = KIND == K_E4M3 ? make_idesc(kAccF32, kFmtE4M3, kFmtE4M3, 0, 0, BN, BM)
-                                                     : make_idesc(kAccS32, kFmtS8, kFmtS8, 0, 0, BN, BM);
-        static_assert(!MX || D == 128, "MX paths: head_dim 128");
-        constexpr uint32_t idesc_pv = make_idesc(kAccF32, kFmtF16, kFmtF16, 0, 1, D, BM);
-        const uint32_t sQ = smem_u32(smem + L::Q);
-        auto qk = [&](int j) {
-          const uint32_t sK = smem_u32(smem + L::K + (j % NKS) * BN * RB);
-          // MXFP4: the tile's K scale factors into TMEM, ordered before the MMAs that read them
-          if (MX) sf_to_tmem(tSFB[j & 1], smem_u32(smem + L::SC + (j % NSC) * 2 * BN * 4));
-#pragma unroll
-          for (int kk = 0; kk < (int)RB / 32; ++kk) {
-            const uint64_t da = make_sdesc(sQ + kk * 32, 16, SBO8, SW);
-            const uint64_t db = make_sdesc(sK + kk * 32, 16, SBO8, SW);
-            if (KIND == K_E4M3)
-              mma_f8f6f4(tbase + (j & 1) * 128, da, db, idesc_qk, kk > 0);
-            else if (KIND == K_S8)
-              mma_i8(tbase + (j & 1) * 128, da, db, idesc_qk, kk > 0);
-            else if (KIND == K_MXF4)  // 64 E2M1 per MMA: scale bytes 2kk and 2kk + 1 of each row
-              mma_mxf4(tbase + (j & 1) * 128, da, db, make_idesc_bs(kFmtE2M1x, kFmtE2M1x, BN, BM, 2 * kk, 2 * kk),
-                       tSFA, tSFB[j & 1], kk > 0);
-            else  // 32 E4M3 per MMA: scale byte kk of each row
-              mma_mxf8(tbase + (j & 1) * 128, da, db, make_idesc_bs(kFmtE4M3, kFmtE4M3, BN, BM, kk, kk), tSFA,
-                       tSFB[j & 1], kk > 0);
-          }
-          mma_commit(&bar[X_SF + (j & 1)]);
-          mma_commit(&bar[X_KE + j % NKS]);
-        };
-        auto pv = [&](int j) {
-          // A = P' in TMEM: key group g's HN keys sit (as fp16 pairs) in columns
-          // [g * HN, g * HN + HN / 2) of the S buffer; 16 keys (8 columns) per MMA.
-          const uint32_t sVh = smem_u32(smem + L::VH + (j % NVS) * BN * D * 2);
-          const uint32_t tP = tbase + (j & 1) * 128;
-#pragma unroll
-          for (int ks = 0; ks < BN / 16; ++ks) {
-            const uint64_t db = make_sdesc(sVh + ks * 16 * 128, BN * 128, 1024, kSwz128);
-            const int g = ks * 16 / HN;
-            mma_f16_ts(tO, tP + g * HN + ((ks * 16 - g * HN) >> 1), db, idesc_pv, (j > 0 || ks > 0) ? 1u : 0u);
-          }
-          mma_commit(&bar[X_PVD]);
-          mma_commit(&bar[X_VE + j % NVS]);
-        };
-        // MXFP4: QK(j) also needs the tile's scale-factor atom in its scale ring stage
-        auto sf_ready = [&](int j) {
-          return !MX || mbar_wait(&bar[X_SCF + j % NSC], (j / NSC) & 1, abort_flag, p.status, 68);
-        };
-        bool ok = mbar_wait(&bar[X_Q], 0, abort_flag, p.status, 63);
-        if (MX && ok) {
-          tc_fence_after();
-          sf_to_tmem(tSFA, smem_u32(smem + L::SFA));
-        }
-        for (int j = 0; ok && j < 2 && j < n; ++j) {
-          ok = mbar_wait(&bar[X_KF + j], 0, abort_flag, p.status, 64) && sf_ready(j);
-          if (ok) {
-            tc_fence_after();
-            qk(j);
-          }
-        }
-        for (int j = 0; ok && j < n; ++j) {
-          ok = mbar_wait(&bar[X_PF + (j & 1)], (j >> 1) & 1, abort_flag, p.status, 65);
-          if (ok) ok = mbar_wait(&bar[X_VF + j % NVS], (j / NVS) & 1, abort_flag, p.status, 66);
-          if (!ok) break;
-          tc_fence_after();
-          pv(j);
-          if (j + 2 < n) {
-            ok = mbar_wait(&bar[X_KF + (j + 2) % NKS], ((j + 2) / NKS) & 1, abort_flag, p.status, 67) && sf_ready(j + 2);
-            if (!ok) break;
-            tc_fence_after();
-            qk(j + 2);
-          }
-        }
-        mma_commit(&bar[X_FIN]);
-        mbar_drain(&bar[X_FIN], 0);
-      }
-      __syncwarp();
-    }
-  } else {
-    setmaxnreg_inc<Cfg<NSW>::RS>();
-    // ------------------------------------------------------------- softmax
-    const int h = (warp - 4) >> 2;  // key group: columns [h * HN, h * HN + HN) of each S tile
-    const int i = tid - 128 - h * 128;
-    const uint32_t loff = (uint32_t)((warp & 3) * 32) << 16;
-    const int cb = h * HN;
-    const int row = q0 + i;
-    const bool row_ok = row < p.Sq;
-    const int qbh = b * p.Hq + hq;
-    float* xm = reinterpret_cast<float*>(smem + L::XM);
-    float* xl = reinterpret_cast<float*>(smem + L::XL);
-    // MXFP4: the block scales are applied inside the MMA, so only the softmax scale
-    const float sq = MX ? 1.0f : (row_ok ? scale_at(p.qs, p.q_blk, p.q_nblk, qbh, hq, row) : 0.0f);
-    float crow = sq * p.scale_log2;
-    if (!RING) crow *= __ldg(p.ks + hk);
-    // S8 accumulators arrive biased: t = float(0x4B400000 + acc) = 1.5 * 2^23 + acc (exact, |acc| < 2^22)
-    constexpr float kBias = KIND == K_S8 ? 12582912.0f : 0.0f;
-    float vref = RING ? 1.0f : __ldg(p.vs + hk);
-    float m_run = -INFINITY, l_run = 0.0f;
-    bool ok = true;
-    for (int j = 0; j < n && ok; ++j) {
-      const int k0 = j * BN, st = j & 1;
-      const uint32_t tS = tbase + st * 128 + cb;
-      const int sst = j % NSC;
-      const float* ksc = reinterpret_cast<const float*>(smem + L::SC + sst * 2 * BN * 4);
-      if (RING && !warp_wait(&bar[X_SCF + sst], (j / NSC) & 1, abort_flag, p.status, 70)) { ok = false; break; }
-      if (RING && j == 0) vref = misc[0];
-      // this tile's K scales and V' factor, loaded while S is still being computed
-      float4 kk4[HN / 4];
-      if (SC == SC_COL) {
-#pragma unroll
-        for (int k = 0; k < HN; k += 4) kk4[k / 4] = *reinterpret_cast<const float4*>(ksc + cb + k);
-      }
-      float flog = 0.0f, finv = 1.0f, ktile = 1.0f;
-      if (RING) {
-        // V' factor r_t / v_ref enters the exponent as its log2, floored at -60 (a tile that
-        // small adds nothing visible to O); the row sum divides it back out.  MXFP4: the
-        // factor is 2^(E_t - E_ref), its log2 an exact integer.
-        flog = fmaxf(MX ? ksc[BN] - vref : __log2f(ksc[BN] / vref), -60.0f);
-        finv = ex2(-flog);
-      }
-      if (SC == SC_TILE) ktile = ksc[0];
-      if (!warp_wait(&bar[X_SF + st], (j >> 1) & 1, abort_flag, p.status, 71)) { ok = false; break; }
-      tc_fence_after();
-      uint32_t tr[HN];
-#pragma unroll
-      for (int c = 0; c < HN / 32; ++c) tmem_ld32(tS + loff + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(&tr[32 * c]));
-      tmem_ld_wait();
-      float t[HN];
-#pragma unroll
-      for (int k = 0; k < HN; ++k) t[k] = KIND == K_S8 ? __uint_as_float(0x4B400000u + tr[k]) : __uint_as_float(tr[k]);
-      // per-key K scale; a tile-constant K scale folds into the row constant
-      float cr = crow;
-      if (SC == SC_COL) {
-#pragma unroll
-        for (int k = 0; k < HN; k += 4) {
-          fmul2(t[k], t[k + 1], kk4[k / 4].x, kk4[k / 4].y);
-          fmul2(t[k + 2], t[k + 3], kk4[k / 4].z, kk4[k / 4].w);
-        }
-      } else if (SC == SC_TILE) {
-        cr *= ktile;
-      }
-      // masks: keys past the sequence, and causal
-      const int kc0 = k0 + cb;
-      const bool need_mask = (kc0 + HN > p.Sk) || (p.causal && (kc0 + HN - 1 > q0 + diag));
-      if (need_mask) {
-        const int lim = p.causal ? min(p.Sk - 1, row + diag) : p.Sk - 1;
-#pragma unroll
-        for (int k = 0; k < HN; ++k)
-          if (kc0 + k > lim) t[k] = -INFINITY;
-      }
-      // eight max chains over HN / 8 keys each, three-input max
-      constexpr int PER = HN / 8;
-      float mx[8];
-#pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        mx[e] = t[e];
-#pragma unroll
-        for (int q = 1; q < PER; q += 2) mx[e] = q + 1 < PER ? fmax3(mx[e], t[e + 8 * q], t[e + 8 * q + 8]) : fmaxf(mx[e], t[e + 8 * q]);
-      }
-      const float mt = fmax3(fmax3(mx[0], mx[1], mx[2]), fmax3(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7]));
-      const float mts = mt == -INFINITY ? -INFINITY : (mt - kBias) * cr;  // this group's tile max, log2 domain
-      // publish this group's maximum; the others' are read once they are needed
-      xm[(st * 4 + h) * BM + i] = mts;
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bar[X_MX + st]);
-      auto others_max = [&]() {
-        float m = -INFINITY;
-#pragma unroll
-        for (int g = 0; g < NSW; ++g)
-          if (g != h) m = fmaxf(m, xm[(st * 4 + g) * BM + i]);
-        return m;
-      };
-      // The running max moves only when a tile's max exceeds it by more than 2^8, so the
-      // exponentials normally use m_run before the partner's half is known.  A warp where
-      // this half alone forces a move (always on a row's first visible tile) takes both
-      // halves' maxima first.
-      float m_use = m_run;
-      bool have_part = false;
-      if (__any_sync(0xffffffffu, mts > m_run + 8.0f)) {
-        if (!warp_wait(&bar[X_MX + st], (j >> 1) & 1, abort_flag, p.status, 75)) { ok = false; break; }
-        have_part = true;
-        const float m_new = fmaxf(m_run, fmaxf(mts, others_max()));
-        if (m_new > m_run + 8.0f) m_use = m_new;
-      }
-      // exp2 argument: t * cr - (bias * cr + m) + log2(r_t / v_ref)   (bias 0 for E4M3; factor 1 for INT8)
-      const float nb = (m_use == -INFINITY ? 0.0f : -(kBias * cr + m_use)) + flog;
-#pragma unroll
-      for (int k = 0; k < HN; k += 2) {
-        ffma2(t[k], t[k + 1], cr, cr, nb, nb);
-        if (((k >> 1) & 3) < FAQ_MX_POLY) {
-          ex2_poly2(t[k], t[k + 1]);  // this share of the pairs on the FMA pipe
-        } else {
-          t[k] = ex2(t[k]);
-          t[k + 1] = ex2(t[k + 1]);
-        }
-      }
-      if (!have_part && !warp_wait(&bar[X_MX + st], (j >> 1) & 1, abort_flag, p.status, 75)) { ok = false; break; }
-      // the decision every group takes from the same numbers
-      const float m_new = fmaxf(m_run, fmaxf(mts, others_max()));
-      const float m_fin = m_new > m_run + 8.0f ? m_new : m_run;
-      if (__any_sync(0xffffffffu, m_fin != m_use)) {
-        // another group moved the max: rescale this group's p (each <= 2^8 here)
-        const float c = m_fin != m_use ? ex2(m_use - m_fin) : 1.0f;
-#pragma unroll
-        for (int k = 0; k < HN; k += 2) fmul2(t[k], t[k + 1], c, c);
-      }
-      const float alpha = m_fin != m_run ? ex2(m_run - m_fin) : 1.0f;
-      if (__any_sync(0xffffffffu, m_fin != m_run) && j > 0) {
-        // O is free once P V of tile j-1 has completed; each group rescales its own DC O columns.
-        if (!warp_wait(&bar[X_PVD], (j - 1) & 1, abort_flag, p.status, 72)) { ok = false; break; }
-        tc_fence_after();
-        if (DC >= 32) {
-#pragma unroll
-          for (int c = 0; c < DC / 32; ++c) {
-            uint32_t r[32];
-            tmem_ld32(tO + loff + h * DC + c * 32, r);
-            tmem_ld_wait();
-#pragma unroll
-            for (int k = 0; k < 32; k += 2) {
-              float a0 = __uint_as_float(r[k]), a1 = __uint_as_float(r[k + 1]);
-              fmul2(a0, a1, alpha, alpha);
-              r[k] = __float_as_uint(a0);
-              r[k + 1] = __float_as_uint(a1);
-            }
-            tmem_st32(tO + loff + h * DC + c * 32, r);
-          }
-        } else {
-          uint32_t r[16];
-          tmem_ld16(tO + loff + h * DC, r);
-          tmem_ld_wait();
-#pragma unroll
-          for (int k = 0; k < 16; k += 2) {
-            float a0 = __uint_as_float(r[k]), a1 = __uint_as_float(r[k + 1]);
-            fmul2(a0, a1, alpha, alpha);
-            r[k] = __float_as_uint(a0);
-            r[k + 1] = __float_as_uint(a1);
-          }
-          tmem_st16(tO + loff + h * DC, r);
-        }
-        tmem_st_wait();
-      }
-      l_run *= alpha;
-      m_run = m_fin;
-      float ls[8];
-#pragma unroll
-      for (int e = 0; e < 8; ++e) ls[e] = t[e];
-#pragma unroll
-      for (int k = 8; k < HN; k += 2) fadd2(ls[k & 7], ls[(k & 7) + 1], t[k], t[k + 1]);
-      // P' = fp16(p) over this group's first HN / 2 S columns
-      {
-        uint32_t hp[HN / 2];
-#pragma unroll
-        for (int e = 0; e < HN / 2; ++e) {
-          const __half2 hv = __floats2half2_rn(t[2 * e], t[2 * e + 1]);
-          hp[e] = *reinterpret_cast<const uint32_t*>(&hv);
-        }
-        if constexpr (HN == 64)
-          tmem_st32(tS + loff, *reinterpret_cast<uint32_t(*)[32]>(&hp[0]));
-        else
-          tmem_st16(tS + loff, *reinterpret_cast<uint32_t(*)[16]>(&hp[0]));
-      }
-      tmem_st_wait();
-      l_run += (((ls[0] + ls[1]) + (ls[2] + ls[3])) + ((ls[4] + ls[5]) + (ls[6] + ls[7]))) * finv;
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) {
-        mbar_arrive(&bar[X_PF + st]);
-        if (RING) mbar_arrive(&bar[X_SCE + sst]);
-      }
-    }
-    // ---------------------------------------------------------- epilogue
-    if (ok && n > 0) {
-      ok = warp_wait(&bar[X_PVD], (n - 1) & 1, abort_flag, p.status, 73);
-      tc_fence_after();
-    }
-    // row sum = the groups' partial sums (added in one order by every group)
-    xl[h * BM + i] = l_run;
-    __syncwarp();
-    if (lane == 0) mbar_arrive(&bar[X_LX]);
-    const bool lx = warp_wait(&bar[X_LX], 0, abort_flag, p.status, 76);
-    float l_tot = 0.0f;
-    if (lx) {
-#pragma unroll
-      for (int g = 0; g < NSW; ++g) l_tot += xl[g * BM + i];
-    }
-    if (q0 < p.Sq) {
-      // MXFP4: V' was divided by 2^(E_ref - 127)
-      const float vmul = MX ? exp2f(vref - 127.0f) : vref;
-      const float ofac = l_tot > 0.0f ? vmul / l_tot : 0.0f;
-      __nv_bfloat16* orow = nullptr;
-      bool out_ok = row_ok;
-      if (row_ok) {
-        const long long ridx = p.layout == FA_LAYOUT_BNSD ? ((long long)qbh * p.Sq + row)
-                                                          : (((long long)b * p.Sq + row) * p.Hq + hq);
-        out_ok = in_bounds(ridx >= 0 && ridx < (long long)p.B * p.Hq * p.Sq, 121);
-        orow = p.out + ridx * D + h * DC;
-      }
-      constexpr int OW = DC >= 32 ? 32 : 16;  // O columns per TMEM load
-#pragma unroll
-      for (int c = 0; c < DC / OW; ++c) {
-        uint32_t r[OW];
-        if (ok && n > 0) {
-          if constexpr (OW == 32)
-            tmem_ld32(tO + loff + h * DC + c * 32, r);
-          else
-            tmem_ld16(tO + loff + h * DC, r);
-          tmem_ld_wait();
-        } else {
-#pragma unroll
-          for (int k = 0; k < OW; ++k) r[k] = 0u;
-        }
-        if (out_ok) {
-#pragma unroll
-          for (int k = 0; k < OW; k += 8) {
-            uint32_t o[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const __nv_bfloat162 v2 = __floats2bfloat162_rn(__uint_as_float(r[k + 2 * e]) * ofac,
-                                                              __uint_as_float(r[k + 2 * e + 1]) * ofac);
-              o[e] = *reinterpret_cast<const uint32_t*>(&v2);
-            }
-            *reinterpret_cast<uint4*>(orow + c * OW + k) = make_uint4(o[0], o[1], o[2], o[3]);
-          }
-        }
-      }
-      if (h == 0 && out_ok && p.lse && in_bounds((long long)qbh * p.Sq + row < (long long)p.B * p.Hq * p.Sq, 122))
-        p.lse[(long long)qbh * p.Sq + row] =
-            l_tot > 0.0f ? (m_run + __log2f(l_tot)) * 0.69314718055994530942f : -INFINITY;
-    }
-  }
-
-  tc_fence_before();
-  __syncthreads();
-  if (warp == 1) {
-    tc_fence_after();
-    tmem_dealloc(tbase, 512);
-  }
-}
-
-
-// ---- two query tiles per CTA (E4M3 / INT8) ------------------------------
+// ---- two query tiles per CTA (E4M3 / INT8 / MX / bf16) ------------------
 // One CTA owns two 128-row query tiles A and B that read the same K / V' tiles
 // (query heads 2h, 2h+1 of one kv head, or row blocks 2t, 2t+1 of one head),
 // with one S and one O accumulator each in TMEM (S_A, S_B, O_A, O_B = 512
-// columns for D = 128).  Each tile has its own softmax warpgroup, one thread
-// per query row holding the row's 128 scores, so the row maximum needs no
+// columns for D = 128; the MX kinds' 112-key S tiles leave room for the Q and
+// K block-scale factors).  Each tile has its own softmax warpgroup, one thread
+// per query row holding the row's scores, so the row maximum needs no
 // exchange between threads.  The MMA thread alternates the tiles:
 //   QK_A(0) QK_B(0) | PV_A(0) QK_A(1) PV_B(0) QK_B(1) | PV_A(1) QK_A(2) ...
 // so while one warpgroup runs the softmax of tile j, the tensor pipe runs the
@@ -658,6 +90,12 @@ __global__ void __launch_bounds__(Cfg<NSW>::NT, 1)
 // FMA pipe instead of the MUFU.
 #ifndef FAQ_PAIR_POLY
 #define FAQ_PAIR_POLY 0
+#endif
+// The same for the MX kinds (their 112-key tiles leave the MUFU the larger share of the step):
+// 0 / 1 / 2 / 3 of every 8 pairs measured at mxfp4 259 / 259 / 261 / 255 us, mxfp8 275 / 267 / 269 /
+// 265 us.
+#ifndef FAQ_PAIR_POLY_MX
+#define FAQ_PAIR_POLY_MX 3
 #endif
 // Waits of the per-tile chain that poll (test_wait) instead of suspending: bit 0 the MMA
 // thread's wait for P', bit 1 the softmax's wait for S, bit 2 the MMA thread's K / V' waits.
@@ -673,7 +111,11 @@ static_assert(128 * PR0 + 256 * PRS <= PNT * ((65536 / PNT) & ~7), "register spl
 
 template <int KIND, int D>
 struct LP {
-  static constexpr int RB = KIND == K_BF16 ? 2 * D : D;  // Q / K bytes per token row
+  // MX kinds: block-scaled Q K^T with the scale factors in TMEM.  Their 16 factor columns leave
+  // no room beside two 128-key S tiles and two O accumulators, so their key tiles hold 112 keys.
+  static constexpr bool MX = KIND == K_MXF4 || KIND == K_MXF8;
+  static constexpr int TN = MX ? 112 : BN;               // keys per tile
+  static constexpr int RB = KIND == K_BF16 ? 2 * D : KIND == K_MXF4 ? D / 2 : D;  // Q / K bytes per token row
   static constexpr int NA = RB > 128 ? RB / 128 : 1;     // 128-byte swizzle atoms per row (bf16 at D = 128: 2)
   static constexpr int AB = RB > 128 ? 128 : RB;         // bytes per atom row
   static constexpr int NK = KIND == K_BF16 ? 2 : NKS;    // K stages (bf16 tiles are twice as large)
@@ -682,14 +124,25 @@ struct LP {
   static constexpr int NV = KIND == K_BF16 ? 2 : 3;
   static constexpr uint32_t Q = 0;                       // 2 x NA x [128][AB]
   static constexpr uint32_t K = Q + 2 * BM * RB;         // NK stages
-  static constexpr uint32_t VH = K + NK * BN * RB;       // NV stages of fp16 V'
-  static constexpr uint32_t SC = VH + NV * BN * D * 2;   // NSC stages x ([128] K scales, V' factor record)
+  static constexpr uint32_t VH = K + NK * TN * RB;       // NV stages of fp16 V'
+  static constexpr uint32_t SC = VH + NV * TN * D * 2;   // NSC stages x ([128] K scales or atom, V' factor record)
   static constexpr uint32_t MISC = SC + NSC * 2 * BN * 4;
-  static constexpr uint32_t BAR = MISC + 64;
+  static constexpr uint32_t SFA = MISC + 64;             // MX: the two Q tiles' scale-factor atoms
+  static constexpr uint32_t BAR = SFA + (MX ? 2 * 512 : 0);
   static constexpr uint32_t TOTAL = BAR + 512;
   static constexpr uint32_t ALLOC = TOTAL + 1024;
   static_assert(ALLOC <= 227 * 1024, "shared memory per CTA");
   static_assert(VH % 1024 == 0, "V' stages need 1024-byte alignment for the 128-byte swizzle");
+  static_assert((TN * RB) % 1024 == 0 && (TN * D * 2) % 1024 == 0, "stage sizes keep the swizzle alignment");
+  // TMEM columns.  E4M3 / INT8 / bf16: S_A, S_B at 0, 128; O_A, O_B at 256, 256 + D.  MX (D = 128):
+  // O_A, O_B at 0, 128; S_A at 256 and S_B at 384 (112 columns each); the Q tiles' factors at 368
+  // and 376 and the K tiles' (two slots) at 496 and 504, every block 8-column aligned.
+  static constexpr uint32_t TS0 = MX ? 256 : 0;
+  static constexpr uint32_t TO0 = MX ? 0 : 256;
+  static constexpr uint32_t TO1 = MX ? 128 : 256 + D;
+  static constexpr uint32_t TSFQ = 368;
+  static constexpr uint32_t TSFK = 496;
+  static_assert(!MX || D == 128, "MX paths: head_dim 128");
 };
 
 enum {
@@ -712,9 +165,13 @@ template <int KIND, int D, int SC>
 __global__ void __launch_bounds__(PNT, 1)
     attn_pair_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
                      const __grid_constant__ CUtensorMap tmv, const P2 p) {
-  static_assert(KIND == K_E4M3 || KIND == K_BF16 || (KIND == K_S8 && SC != SC_TILE), "E4M3, INT8 or bf16 operands");
-  constexpr bool RING = SC != SC_HEAD;
+  static_assert(KIND == K_E4M3 || KIND == K_BF16 || (KIND == K_S8 && SC != SC_TILE) ||
+                    ((KIND == K_MXF4 || KIND == K_MXF8) && SC == SC_HEAD),
+                "E4M3, INT8, MX or bf16 operands");
   using L = LP<KIND, D>;
+  constexpr bool MX = L::MX;
+  constexpr int TN = L::TN;
+  constexpr bool RING = MX || SC != SC_HEAD;  // per-tile records (and K scales / atoms) through the scale ring
   constexpr int NKS = L::NK;  // K stages of this kind
   constexpr int NVS = L::NV;  // V' stages of this kind
   extern __shared__ uint8_t smem_raw[];
@@ -752,13 +209,13 @@ __global__ void __launch_bounds__(PNT, 1)
   for (int x = 0; x < 2; ++x) {
     int kv_end = 0;
     if (q0t[x] < p.Sq) kv_end = p.causal ? min(p.Sk, max(0, min(q0t[x] + BM, p.Sq) - 1 + diag + 1)) : p.Sk;
-    nt[x] = (kv_end + BN - 1) / BN;
+    nt[x] = (kv_end + TN - 1) / TN;
   }
   const int n = max(nt[0], nt[1]);
   const int bhk = b * p.Hkv + hk;
 
   if (tid == 0) {
-    mbar_init(&bar[Y_Q], 1);
+    mbar_init(&bar[Y_Q], MX ? 2 : 1);  // MX: the Q codes and the Q tiles' scale-factor atoms
     for (int i = 0; i < NKS; ++i) {
       mbar_init(&bar[Y_KF + i], 1);
       mbar_init(&bar[Y_KE + i], 1);
@@ -786,7 +243,7 @@ __global__ void __launch_bounds__(PNT, 1)
   }
   __syncthreads();
   tc_fence_after();
-  const uint32_t tbase = *tmem_slot;  // S_A, S_B at columns 0, 128; O_A, O_B at 256, 256 + D
+  const uint32_t tbase = *tmem_slot;  // columns as in LP
 
   if (warp < 4) {
     setmaxnreg_dec<PR0>();
@@ -806,12 +263,12 @@ __global__ void __launch_bounds__(PNT, 1)
                           bnsd ? q0t[x] : hqt[x], bnsd ? hqt[x] : q0t[x], b);
         int j = 0;
         for (; j < n; ++j) {
-          const int k0 = j * BN, ks = j % NKS;
+          const int k0 = j * TN, ks = j % NKS;
           if (j >= NKS && !mbar_wait(&bar[Y_KE + ks], ((j / NKS) - 1) & 1, abort_flag, p.status, 81)) break;
-          mbar_arrive_expect_tx(&bar[Y_KF + ks], BN * L::RB);
+          mbar_arrive_expect_tx(&bar[Y_KF + ks], TN * L::RB);
 #pragma unroll
           for (int a = 0; a < L::NA; ++a)
-            tma_load_4d(smem + L::K + ks * BN * L::RB + a * BN * L::AB, &tmk, &bar[Y_KF + ks], a * L::AB,
+            tma_load_4d(smem + L::K + ks * TN * L::RB + a * TN * L::AB, &tmk, &bar[Y_KF + ks], a * L::AB,
                         bnsd ? k0 : hk, bnsd ? hk : k0, b);
         }
         if (*abort_flag) {
@@ -826,12 +283,12 @@ __global__ void __launch_bounds__(PNT, 1)
         tma_prefetch_desc(&tmv);
         int j = 0;
         for (; j < n; ++j) {
-          const int k0 = j * BN, vs = j % NVS;
+          const int k0 = j * TN, vs = j % NVS;
           if (j >= NVS && !mbar_wait(&bar[Y_VE + vs], ((j / NVS) - 1) & 1, abort_flag, p.status, 82)) break;
-          mbar_arrive_expect_tx(&bar[Y_VF + vs], BN * D * 2);
+          mbar_arrive_expect_tx(&bar[Y_VF + vs], TN * D * 2);
 #pragma unroll
           for (int a2 = 0; a2 < D / 64; ++a2)
-            tma_load_4d(smem + L::VH + vs * BN * D * 2 + a2 * BN * 128, &tmv, &bar[Y_VF + vs], 64 * a2, k0, hk, b);
+            tma_load_4d(smem + L::VH + vs * TN * D * 2 + a2 * TN * 128, &tmv, &bar[Y_VF + vs], 64 * a2, k0, hk, b);
         }
         if (*abort_flag)
           for (int t = max(0, j - NVS); t < j; ++t) mbar_drain(&bar[Y_VF + t % NVS], (t / NVS) & 1);
@@ -839,6 +296,16 @@ __global__ void __launch_bounds__(PNT, 1)
       __syncwarp();
     } else if (warp == 2) {
       // ------------------------------------------------------- scale ring
+      if (MX && n > 0) {
+        // the Q tiles' scale-factor atoms, published with the Q codes' barrier (rows past Sq: 0)
+#pragma unroll
+        for (int x = 0; x < 2; ++x)
+          write_sf_atom(smem + L::SFA + x * 512, p.qe8, (long long)(b * p.Hq + hqt[x]) * p.Sq + q0t[x], p.Sq - q0t[x],
+                        lane);
+        fence_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bar[Y_Q]);
+      }
       if (RING && n > 0) {
         const float4* fvh = p.fvr + (long long)bhk * p.ntiles_k;
         float m = 0.0f;
@@ -846,8 +313,10 @@ __global__ void __launch_bounds__(PNT, 1)
 #pragma unroll
         for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
         if (lane == 0) {
-          misc[0] = m > 0.0f ? m : 1.0f;  // v_ref: the largest V' factor over this CTA's tiles
-          misc[1] = log2f(misc[0]);
+          // v_ref: the largest V' factor over this CTA's tiles, and its log2.  MX: the records hold
+          // {E_t, E_t - 127}, so v_ref = 2^(E_ref - 127) with E_ref the largest E_t.
+          misc[0] = MX ? exp2f(m - 127.0f) : (m > 0.0f ? m : 1.0f);
+          misc[1] = MX ? m - 127.0f : log2f(misc[0]);
           const float* kph = p.ksp + (long long)bhk * p.ntiles_k * BN;
           int j = 0;
           for (; j < n; ++j) {
@@ -868,9 +337,9 @@ __global__ void __launch_bounds__(PNT, 1)
       if (lane == 0 && n > 0) {
         constexpr uint32_t SW = L::AB == 128 ? kSwz128 : kSwz64;
         constexpr uint32_t SBO8 = L::AB == 128 ? 1024 : 512;
-        constexpr uint32_t idesc_qk = KIND == K_E4M3   ? make_idesc(kAccF32, kFmtE4M3, kFmtE4M3, 0, 0, BN, BM)
-                                      : KIND == K_BF16 ? make_idesc(kAccF32, kFmtBF16, kFmtBF16, 0, 0, BN, BM)
-                                                       : make_idesc(kAccS32, kFmtS8, kFmtS8, 0, 0, BN, BM);
+        constexpr uint32_t idesc_qk = KIND == K_E4M3   ? make_idesc(kAccF32, kFmtE4M3, kFmtE4M3, 0, 0, TN, BM)
+                                      : KIND == K_BF16 ? make_idesc(kAccF32, kFmtBF16, kFmtBF16, 0, 0, TN, BM)
+                                                       : make_idesc(kAccS32, kFmtS8, kFmtS8, 0, 0, TN, BM);
         constexpr uint32_t idesc_pv = make_idesc(kAccF32, kFmtF16, kFmtF16, 0, 1, D, BM);
         // Descriptors as 32-bit halves: the high half (stride, version, swizzle) is constant per
         // tile kind, the low half (start address >> 4 | leading offset) is computed once per tile
@@ -878,37 +347,64 @@ __global__ void __launch_bounds__(PNT, 1)
         // address field (shared memory is below 256 KB).  The issuing warp shares its SM
         // sub-partition with two softmax warps, so each MMA costs it only a few instructions.
         const uint64_t dq0 = make_sdesc(smem_u32(smem + L::Q), 16, SBO8, SW);
-        const uint64_t dv0 = make_sdesc(smem_u32(smem + L::VH), BN * 128, 1024, kSwz128);
+        const uint64_t dv0 = make_sdesc(smem_u32(smem + L::VH), TN * 128, 1024, kSwz128);
         const uint32_t qk_hi = (uint32_t)(dq0 >> 32), v_hi = (uint32_t)(dv0 >> 32);
         const uint32_t q_lo = (uint32_t)dq0, k_lo = (uint32_t)make_sdesc(smem_u32(smem + L::K), 16, SBO8, SW);
         const uint32_t v_lo = (uint32_t)dv0;
         auto qk = [&](int x, int j) {
           const uint32_t ql = q_lo + (x ? (uint32_t)((BM * L::RB) >> 4) : 0u);
-          const uint32_t kl = k_lo + (uint32_t)(j % NKS) * (uint32_t)((BN * L::RB) >> 4);
-          // one MMA per 32 bytes of the row (K = 32 codes, or K = 16 bf16): atom a = kk * 32 / AB
+          const uint32_t kl = k_lo + (uint32_t)(j % NKS) * (uint32_t)((TN * L::RB) >> 4);
+          // one MMA per 32 bytes of the row (K = 32 codes, 64 E2M1, or 16 bf16): atom a = kk * 32 / AB
 #pragma unroll
           for (int kk = 0; kk < L::RB / 32; ++kk) {
             const uint32_t off = ((kk * 32 / L::AB) * BM * L::AB + (kk * 32) % L::AB) >> 4;
-            if (KIND == K_E4M3)
+            if constexpr (MX) {
+              // block scales from TMEM: this tile's Q factors, the K tile's (slot j % 2); the
+              // factor id picks the row's scale bytes for this MMA's K range
+              const uint64_t da = ((uint64_t)qk_hi << 32) | (ql + off), db = ((uint64_t)qk_hi << 32) | (kl + off);
+              const uint32_t sfa = tbase + L::TSFQ + 8 * x, sfb = tbase + L::TSFK + 8 * (j & 1);
+              if (KIND == K_MXF4)
+                mma_mxf4(tbase + L::TS0 + x * 128, da, db,
+                         make_idesc_bs(kFmtE2M1x, kFmtE2M1x, TN, BM, 2 * kk, 2 * kk), sfa, sfb, kk > 0);
+              else
+                mma_mxf8(tbase + L::TS0 + x * 128, da, db, make_idesc_bs(kFmtE4M3, kFmtE4M3, TN, BM, kk, kk), sfa,
+                         sfb, kk > 0);
+            } else if (KIND == K_E4M3) {
               mma_f8f6f4_lh(tbase + x * 128, ql + off, qk_hi, kl + off, qk_hi, idesc_qk, kk > 0);
-            else if (KIND == K_BF16)
+            } else if (KIND == K_BF16) {
               mma_f16_lh(tbase + x * 128, ql + off, qk_hi, kl + off, qk_hi, idesc_qk, kk > 0);
-            else
+            } else {
               mma_i8_lh(tbase + x * 128, ql + off, qk_hi, kl + off, qk_hi, idesc_qk, kk > 0);
+            }
           }
           mma_commit(&bar[Y_SF + x]);
         };
         auto pv = [&](int x, int j) {
           // A = P' in TMEM: key k of the tile sits in column k / 2 of S_x (fp16 pairs)
-          const uint32_t vl = v_lo + (uint32_t)(j % NVS) * (uint32_t)((BN * D * 2) >> 4);
+          const uint32_t vl = v_lo + (uint32_t)(j % NVS) * (uint32_t)((TN * D * 2) >> 4);
 #pragma unroll
-          for (int ks = 0; ks < BN / 16; ++ks)
-            mma_f16_ts_lh(tbase + 256 + x * D, tbase + x * 128 + ks * 8, vl + (uint32_t)((ks * 16 * 128) >> 4), v_hi,
-                          idesc_pv, (j > 0 || ks > 0) ? 1u : 0u);
+          for (int ks = 0; ks < TN / 16; ++ks)
+            mma_f16_ts_lh(tbase + L::TO0 + x * (L::TO1 - L::TO0), tbase + L::TS0 + x * 128 + ks * 8,
+                          vl + (uint32_t)((ks * 16 * 128) >> 4), v_hi, idesc_pv, (j > 0 || ks > 0) ? 1u : 0u);
           mma_commit(&bar[Y_PVD + x]);
         };
+        // MX: K tile j's scale-factor atom (in its scale ring stage) into TMEM slot j % 2, ordered
+        // before the MMAs that read it
+        auto k_factors = [&](int j) {
+          if constexpr (MX) {
+            if (!mbar_wait(&bar[Y_SCF + j % NSC], (j / NSC) & 1, abort_flag, p.status, 88)) return false;
+            tc_fence_after();
+            sf_to_tmem(tbase + L::TSFK + 8 * (j & 1), smem_u32(smem + L::SC + (j % NSC) * 2 * BN * 4));
+          }
+          return true;
+        };
         bool ok = mbar_wait(&bar[Y_Q], 0, abort_flag, p.status, 83);
-        if (ok) ok = mbar_wait(&bar[Y_KF], 0, abort_flag, p.status, 84);
+        if (MX && ok) {
+          tc_fence_after();
+          sf_to_tmem(tbase + L::TSFQ, smem_u32(smem + L::SFA));
+          sf_to_tmem(tbase + L::TSFQ + 8, smem_u32(smem + L::SFA + 512));
+        }
+        if (ok) ok = mbar_wait(&bar[Y_KF], 0, abort_flag, p.status, 84) && k_factors(0);
         if (ok) {
           tc_fence_after();
           if (nt[0] > 0) qk(0, 0);
@@ -930,7 +426,8 @@ __global__ void __launch_bounds__(PNT, 1)
             if (j + 1 < nt[x]) {
               if (!k_ready)
                 ok = k_ready = chain_wait<(FAQ_PAIR_SPIN & 4) != 0>(&bar[Y_KF + (j + 1) % NKS], ((j + 1) / NKS) & 1,
-                                                                    abort_flag, p.status, 87);
+                                                                    abort_flag, p.status, 87) &&
+                               k_factors(j + 1);
               if (!ok) break;
               tc_fence_after();
               qk(x, j + 1);
@@ -955,9 +452,10 @@ __global__ void __launch_bounds__(PNT, 1)
     const int row = q0 + i;
     const bool row_ok = row < p.Sq;
     const int qbh = b * p.Hq + hq;
-    const uint32_t tS = tbase + x * 128;
-    const uint32_t tO = tbase + 256 + x * D;
-    const float sq = row_ok ? scale_at(p.qs, p.q_blk, p.q_nblk, qbh, hq, row) : 0.0f;
+    const uint32_t tS = tbase + L::TS0 + x * 128;
+    const uint32_t tO = tbase + L::TO0 + x * (L::TO1 - L::TO0);
+    // MX: the block scales are applied inside the MMA, so only the softmax scale
+    const float sq = row_ok ? (MX ? 1.0f : scale_at(p.qs, p.q_blk, p.q_nblk, qbh, hq, row)) : 0.0f;
     float crow = sq * p.scale_log2;
     if (!RING) crow *= __ldg(p.ks + hk);
     // S8 accumulators with one K scale per head arrive biased (t = 1.5 * 2^23 + acc, exact for
@@ -969,7 +467,7 @@ __global__ void __launch_bounds__(PNT, 1)
     float lgref = 0.0f;  // log2(v_ref)
     bool ok = true;
     for (int j = 0; j < n && ok; ++j) {
-      const int k0 = j * BN;
+      const int k0 = j * TN;
       const int sst = j % NSC;
       const float* ksc = reinterpret_cast<const float*>(smem + L::SC + sst * 2 * BN * 4);
       if (RING && !warp_wait(&bar[Y_SCF + sst], (j / NSC) & 1, abort_flag, p.status, 90)) { ok = false; break; }
@@ -1003,7 +501,7 @@ __global__ void __launch_bounds__(PNT, 1)
         break;
       }
       tc_fence_after();
-      float t[BN];
+      float t[TN];
       // S from TMEM (all four 32-column loads, one wait), the per-key K scale, the masks
       auto load_s = [&](bool again) {
         // per-key K scales: two halves of 64 columns, so half of the scales' registers are free
@@ -1011,11 +509,14 @@ __global__ void __launch_bounds__(PNT, 1)
         constexpr int NH = SC == SC_COL ? 2 : 1;
 #pragma unroll
         for (int hh = 0; hh < NH; ++hh) {
-          constexpr int W = BN / NH;
+          constexpr int W = TN / NH;
+          static_assert(W % 16 == 0, "S loads of 32 and 16 columns");
           uint32_t tr[W];
 #pragma unroll
           for (int c = 0; c < W / 32; ++c)
             tmem_ld32(tS + loff + W * hh + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(&tr[32 * c]));
+          if constexpr (W % 32 != 0)  // 112-key tiles: the last 16 columns
+            tmem_ld16(tS + loff + W * hh + W / 32 * 32, *reinterpret_cast<uint32_t(*)[16]>(&tr[W / 32 * 32]));
           tmem_ld_wait();
 #pragma unroll
           for (int k = 0; k < W; ++k)
@@ -1036,11 +537,11 @@ __global__ void __launch_bounds__(PNT, 1)
             }
           }
         }
-        const bool need_mask = (k0 + BN > p.Sk) || (p.causal && (k0 + BN - 1 > q0 + diag));
+        const bool need_mask = (k0 + TN > p.Sk) || (p.causal && (k0 + TN - 1 > q0 + diag));
         if (need_mask) {
           const int lim = p.causal ? min(p.Sk - 1, row + diag) : p.Sk - 1;
 #pragma unroll
-          for (int k = 0; k < BN; ++k)
+          for (int k = 0; k < TN; ++k)
             if (k0 + k > lim) t[k] = -INFINITY;
         }
       };
@@ -1048,9 +549,9 @@ __global__ void __launch_bounds__(PNT, 1)
       auto exponentials = [&](float m) -> float {
         const float nb = (m == -INFINITY ? 0.0f : -(kBias * cr + m)) + flog;
 #pragma unroll
-        for (int k = 0; k < BN; k += 2) {
+        for (int k = 0; k < TN; k += 2) {
           ffma2(t[k], t[k + 1], cr, cr, nb, nb);
-          if (((k >> 1) & 7) < FAQ_PAIR_POLY) {
+          if (((k >> 1) & 7) < (MX ? FAQ_PAIR_POLY_MX : FAQ_PAIR_POLY)) {
             ex2_poly2(t[k], t[k + 1]);  // this share of the pairs on the FMA pipe
           } else {
             t[k] = ex2(t[k]);
@@ -1061,7 +562,7 @@ __global__ void __launch_bounds__(PNT, 1)
 #pragma unroll
         for (int e = 0; e < 8; ++e) ls[e] = t[e];
 #pragma unroll
-        for (int k = 8; k < BN; k += 2) fadd2(ls[k & 7], ls[(k & 7) + 1], t[k], t[k + 1]);
+        for (int k = 8; k < TN; k += 2) fadd2(ls[k & 7], ls[(k & 7) + 1], t[k], t[k + 1]);
         return ((ls[0] + ls[1]) + (ls[2] + ls[3])) + ((ls[4] + ls[5]) + (ls[6] + ls[7]));
       };
       load_s(false);
@@ -1083,8 +584,8 @@ __global__ void __launch_bounds__(PNT, 1)
           for (int e = 0; e < 8; ++e) {
             mx[e] = t[e];
 #pragma unroll
-            for (int q = 1; q < BN / 8; q += 2)
-              mx[e] = q + 1 < BN / 8 ? fmax3(mx[e], t[e + 8 * q], t[e + 8 * q + 8]) : fmaxf(mx[e], t[e + 8 * q]);
+            for (int q = 1; q < TN / 8; q += 2)
+              mx[e] = q + 1 < TN / 8 ? fmax3(mx[e], t[e + 8 * q], t[e + 8 * q + 8]) : fmaxf(mx[e], t[e + 8 * q]);
           }
           const float mt = fmax3(fmax3(mx[0], mx[1], mx[2]), fmax3(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7]));
           const float mts = mt == -INFINITY ? -INFINITY : (mt - kBias) * cr;  // log2 domain
@@ -1121,14 +622,20 @@ __global__ void __launch_bounds__(PNT, 1)
       }
       if (failed) { ok = false; break; }
       {
-        uint32_t hp[BN / 2];
+        uint32_t hp[TN / 2];
 #pragma unroll
-        for (int e = 0; e < BN / 2; ++e) {
+        for (int e = 0; e < TN / 2; ++e) {
           const __half2 hv = __floats2half2_rn(t[2 * e], t[2 * e + 1]);
           hp[e] = *reinterpret_cast<const uint32_t*>(&hv);
         }
         tmem_st32(tS + loff, *reinterpret_cast<uint32_t(*)[32]>(&hp[0]));
-        tmem_st32(tS + loff + 32, *reinterpret_cast<uint32_t(*)[32]>(&hp[32]));
+        if constexpr (TN == 128) {
+          tmem_st32(tS + loff + 32, *reinterpret_cast<uint32_t(*)[32]>(&hp[32]));
+        } else {  // 112 keys: 56 columns
+          static_assert(TN == 112, "P' stores of 32 + 16 + 8 columns");
+          tmem_st16(tS + loff + 32, *reinterpret_cast<uint32_t(*)[16]>(&hp[32]));
+          tmem_st8(tS + loff + 48, *reinterpret_cast<uint32_t(*)[8]>(&hp[48]));
+        }
       }
       tmem_st_wait();
       l_run += l_tile * finv;
@@ -1201,21 +708,26 @@ __global__ void __launch_bounds__(PNT, 1)
 // V pre-pass: V' fp16 tiles + per-tile factor records (+ the K tile's per-key scales).  MIXED:
 // records are linear factors for every kind (the bf16 pair kernel's scale ring) and the per-key K
 // scales are 1 (Q and K arrive dequantized).
-template <int KIND, int D, bool VSC, bool MIXED = false>
+// TN: keys per tile (112 for the MX pair kernel; 128 otherwise).
+template <int KIND, int D, bool VSC, bool MIXED = false, int TN = BN>
 __global__ void __launch_bounds__(256) vprep_kernel(const uint8_t* __restrict__ codes, const float* __restrict__ vs,
                                                     int v_blk, int v_nblk, int H, int S, int layout,
                                                     __half* __restrict__ vh, float4* __restrict__ fvr, int ntiles,
                                                     const float* __restrict__ ks, int k_blk, int k_nblk,
                                                     float* __restrict__ ksp, const uint8_t* __restrict__ ve8,
                                                     const uint8_t* __restrict__ ke8) {
+  static_assert(TN == BN || KIND == K_MXF4 || KIND == K_MXF8, "112-key tiles: MX kinds only");
+  static_assert(TN <= BN && TN % 16 == 0, "a tile fits the CTA's 128 token slots");
   const int t = blockIdx.x, bh = blockIdx.y;
   // the tile's records and V' rows: tile t of ntiles, (b, h) row bh of the launch's B * H
-  if (!in_bounds(t < ntiles && (long long)t * BN < (long long)S + BN, 125)) return;
+  if (!in_bounds(t < ntiles && (long long)t * TN < (long long)S + TN, 125)) return;
   const int b = bh / H, h = bh % H;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int tok0 = t * BN;
-  const int tok = tok0 + warp * 16 + (lane >> 1);
-  const bool live = tok < S;  // rows past S stay unwritten: the attention's TMA box reads them as zero
+  const int tok0 = t * TN;
+  const int slot = warp * 16 + (lane >> 1);  // token slot of this thread within the tile
+  const int tok = tok0 + slot;
+  // rows past S stay unwritten: the attention's TMA box reads them as zero
+  const bool live = tok < S && slot < TN;
   const long long src_row = layout == FA_LAYOUT_BNSD ? ((long long)bh * S + tok) : (((long long)b * S + tok) * H + h);
   if constexpr (KIND == K_MXF4 || KIND == K_MXF8) {
     static_assert(D == 128, "MX paths: head_dim 128");
@@ -1231,7 +743,7 @@ __global__ void __launch_bounds__(256) vprep_kernel(const uint8_t* __restrict__ 
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
       const int tt = tok0 + lane * 4 + q;
-      if (tt < S) {
+      if (tt < S && lane * 4 + q < TN) {
         const uint32_t w = __ldg(ve4 + tt);
         m = max(m, (int)max(max(w & 0xFFu, (w >> 8) & 0xFFu), max((w >> 16) & 0xFFu, w >> 24)));
       }
@@ -1244,8 +756,11 @@ __global__ void __launch_bounds__(256) vprep_kernel(const uint8_t* __restrict__ 
       if (threadIdx.x < BN) ksp[((long long)bh * ntiles + t) * BN + threadIdx.x] = tok0 + (int)threadIdx.x < S ? 1.0f : 0.0f;
     } else if (threadIdx.x < BN) {
       // the K tile's scale-factor atom: token row r at byte (r % 32) * 16 + (r / 32) * 4, zero past S
+      // (and, for 112-key tiles, in the atom's last 16 rows)
       const int key = tok0 + threadIdx.x;
-      const uint32_t w = key < S ? __ldg(reinterpret_cast<const uint32_t*>(ke8) + (long long)bh * S + key) : 0u;
+      const uint32_t w = (key < S && (int)threadIdx.x < TN)
+                             ? __ldg(reinterpret_cast<const uint32_t*>(ke8) + (long long)bh * S + key)
+                             : 0u;
       reinterpret_cast<uint32_t*>(ksp + ((long long)bh * ntiles + t) * BN)[(threadIdx.x & 31) * 4 + (threadIdx.x >> 5)] = w;
     }
     if (!live) return;
@@ -1392,13 +907,13 @@ __global__ void __launch_bounds__(256) vprep_kernel(const uint8_t* __restrict__ 
   }
 }
 
-// Tensor map over V' [B][H][S][D] fp16: 64-column x 128-token boxes, 128-byte swizzle.
-cudaError_t make_vh_map(CUtensorMap* map, const void* base, int B, int H, int S, int D) {
+// Tensor map over V' [B][H][S][D] fp16: 64-column x `rows`-token boxes, 128-byte swizzle.
+cudaError_t make_vh_map(CUtensorMap* map, const void* base, int B, int H, int S, int D, int rows) {
   EncodeTiledFn enc = encode_tiled_fn();
   if (!enc) return cudaErrorNotSupported;
   const cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)S, (cuuint64_t)H, (cuuint64_t)B};
   const cuuint64_t strides[3] = {(cuuint64_t)D * 2, (cuuint64_t)S * D * 2, (cuuint64_t)H * S * D * 2};
-  const cuuint32_t box[4] = {64, (cuuint32_t)BN, 1, 1};
+  const cuuint32_t box[4] = {64, (cuuint32_t)rows, 1, 1};
   const cuuint32_t es[4] = {1, 1, 1, 1};
   const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 4, const_cast<void*>(base), dims, strides, box, es,
                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -1414,9 +929,10 @@ struct Prefill2Ws {
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
-// Workspace: V' fp16 [B, Hkv, Sk, D] | V' factor records [B, Hkv, ntiles] | K scales [B, Hkv, ntiles * 128].
-Prefill2Ws carve_ws(void* ws, int B, int Hkv, int Sk, int D) {
-  const size_t ntiles = ((size_t)Sk + BN - 1) / BN;
+// Workspace: V' fp16 [B, Hkv, Sk, D] | V' factor records [B, Hkv, ntiles] | K scales [B, Hkv, ntiles * 128],
+// ntiles = the key tiles of `tn` keys.
+Prefill2Ws carve_ws(void* ws, int B, int Hkv, int Sk, int D, int tn = BN) {
+  const size_t ntiles = ((size_t)Sk + tn - 1) / tn;
   uint8_t* base = static_cast<uint8_t*>(ws);
   Prefill2Ws w;
   w.vh = reinterpret_cast<__half*>(base);
@@ -1427,38 +943,18 @@ Prefill2Ws carve_ws(void* ws, int B, int Hkv, int Sk, int D) {
   return w;
 }
 
-#ifndef FAQ_ATTN_NSW
-#define FAQ_ATTN_NSW 2
-#endif
-
-// Tensor maps over the Q and K codes and V', then the V pre-pass.
-template <int KIND, int D, bool VSC>
+template <int KIND, int D, bool VSC, int TN = BN>
 cudaError_t prepare2(const AttnArgs& a, const P2& prm, const Prefill2Ws& w, int RB, CUtensorMap* mq, CUtensorMap* mk,
                      CUtensorMap* mv, cudaStream_t s) {
   cudaError_t e;
   if ((e = make_code_map(mq, a.q->codes, a.q->B, a.q->H, a.q->S, RB, a.q->layout, BM)) != cudaSuccess) return e;
-  if ((e = make_code_map(mk, a.k->codes, a.k->B, a.k->H, a.k->S, RB, a.k->layout, BN)) != cudaSuccess) return e;
-  if ((e = make_vh_map(mv, w.vh, a.v->B, a.v->H, a.v->S, D)) != cudaSuccess) return e;
+  if ((e = make_code_map(mk, a.k->codes, a.k->B, a.k->H, a.k->S, RB, a.k->layout, TN)) != cudaSuccess) return e;
+  if ((e = make_vh_map(mv, w.vh, a.v->B, a.v->H, a.v->S, D, TN)) != cudaSuccess) return e;
   const dim3 pgrid((unsigned)prm.ntiles_k, (unsigned)(a.v->B * a.v->H));
   if (pgrid.y > 65535u) return cudaErrorInvalidValue;
-  vprep_kernel<KIND, D, VSC><<<pgrid, 256, 0, s>>>(static_cast<const uint8_t*>(a.v->codes), prm.vs, prm.v_blk,
+  vprep_kernel<KIND, D, VSC, false, TN><<<pgrid, 256, 0, s>>>(static_cast<const uint8_t*>(a.v->codes), prm.vs, prm.v_blk,
                                                prm.v_nblk, a.v->H, a.v->S, a.v->layout, w.vh, w.fvr, prm.ntiles_k,
                                                prm.ks, prm.k_blk, prm.k_nblk, w.ksp, prm.ve8, prm.ke8);
-  return cudaGetLastError();
-}
-
-template <int KIND, int D, int SC>
-cudaError_t launch2(const AttnArgs& a, const P2& prm, const Prefill2Ws& w, cudaStream_t s) {
-  constexpr int NSW = FAQ_ATTN_NSW;
-  using L = L2<KIND, D>;
-  CUtensorMap mq, mk, mv;
-  cudaError_t e;
-  if ((e = prepare2<KIND, D, true>(a, prm, w, (int)L::RB, &mq, &mk, &mv, s)) != cudaSuccess) return e;
-  auto kern = attn2_kernel<KIND, D, SC, NSW>;
-  if ((e = set_smem_limit(reinterpret_cast<const void*>(kern), L::ALLOC)) != cudaSuccess) return e;
-  const long long grid = (long long)prm.n_qtiles * prm.B * prm.Hq;
-  if (grid > 0x7FFFFFFFLL) return cudaErrorInvalidValue;
-  kern<<<(unsigned)grid, Cfg<NSW>::NT, L::ALLOC, s>>>(mq, mk, mv, prm);
   return cudaGetLastError();
 }
 
@@ -1480,9 +976,11 @@ cudaError_t run_pair(const CUtensorMap& mq, const CUtensorMap& mk, const CUtenso
 
 template <int KIND, int D, int SC>
 cudaError_t launch_pair(const AttnArgs& a, P2 prm, const Prefill2Ws& w, cudaStream_t s) {
+  using L = LP<KIND, D>;
   CUtensorMap mq, mk, mv;
   cudaError_t e;
-  if ((e = prepare2<KIND, D, SC != SC_HEAD>(a, prm, w, D, &mq, &mk, &mv, s)) != cudaSuccess) return e;
+  if ((e = prepare2<KIND, D, L::MX || SC != SC_HEAD, L::TN>(a, prm, w, L::RB, &mq, &mk, &mv, s)) != cudaSuccess)
+    return e;
   return run_pair<KIND, D, SC>(mq, mk, mv, prm, s);
 }
 
@@ -1644,9 +1142,15 @@ void scale_desc2(const fa_qtensor* t, int& blk, int& nblk) {
 
 }  // namespace
 
+// Keys per tile of the prefill kernel for Q's mode: 112 for the MX modes, 128 otherwise.
+int prefill_tile_keys(int q_mode) {
+  const bool mx = q_mode == FA_MODE_MXFP4_PER_BLOCK || q_mode == FA_MODE_MXFP8_PER_BLOCK;
+  return mx ? LP<K_MXF4, 128>::TN : BN;
+}
+
 // Prefill attention for E4M3, INT8 and MXFP4 operands.
-size_t prefill2_workspace_bytes(int B, int Hkv, int Sk, int D) {
-  const size_t ntiles = ((size_t)Sk + BN - 1) / BN;
+size_t prefill2_workspace_bytes(int B, int Hkv, int Sk, int D, int tile_keys) {
+  const size_t ntiles = ((size_t)Sk + tile_keys - 1) / tile_keys;
   return align256((size_t)B * Hkv * Sk * D * 2) + align256((size_t)B * Hkv * ntiles * 16) +
          align256((size_t)B * Hkv * ntiles * BN * 4);
 }
@@ -1670,8 +1174,9 @@ cudaError_t launch_attention_prefill2(const AttnArgs& a, void* ws, cudaStream_t 
   prm.lse = a.lse;
   prm.status = a.status;
   prm.n_qtiles = (q->S + BM - 1) / BM;
-  prm.ntiles_k = (k->S + BN - 1) / BN;
-  const Prefill2Ws w = carve_ws(ws, k->B, k->H, k->S, q->D);
+  const int tn = prefill_tile_keys(q->mode);
+  prm.ntiles_k = (k->S + tn - 1) / tn;
+  const Prefill2Ws w = carve_ws(ws, k->B, k->H, k->S, q->D, tn);
   prm.fvr = w.fvr;
   prm.ksp = w.ksp;
   int sc = SC_HEAD;
@@ -1694,8 +1199,8 @@ cudaError_t launch_attention_prefill2(const AttnArgs& a, void* ws, cudaStream_t 
       prm.qe8 = static_cast<const uint8_t*>(q->scales);
       prm.ke8 = static_cast<const uint8_t*>(k->scales);
       prm.ve8 = static_cast<const uint8_t*>(a.v->scales);
-      return q->mode == FA_MODE_MXFP4_PER_BLOCK ? launch2<K_MXF4, 128, SC_HEAD>(a, prm, w, s)
-                                                 : launch2<K_MXF8, 128, SC_HEAD>(a, prm, w, s);
+      return q->mode == FA_MODE_MXFP4_PER_BLOCK ? launch_pair<K_MXF4, 128, SC_HEAD>(a, prm, w, s)
+                                                 : launch_pair<K_MXF8, 128, SC_HEAD>(a, prm, w, s);
     default:
       return cudaErrorNotSupported;
   }
@@ -1753,7 +1258,7 @@ cudaError_t launch_attention_mixed(const AttnArgs& a, void* ws, cudaStream_t s) 
   const int rb = 2 * D, ab = rb > 128 ? 128 : rb;
   if ((e = make_code_map(&mq, qb, q->B, q->H, q->S, rb, q->layout, BM, ab)) != cudaSuccess) return e;
   if ((e = make_code_map(&mk, kb, k->B, k->H, k->S, rb, k->layout, BN, ab)) != cudaSuccess) return e;
-  if ((e = make_vh_map(&mv, w.vh, a.v->B, a.v->H, a.v->S, D)) != cudaSuccess) return e;
+  if ((e = make_vh_map(&mv, w.vh, a.v->B, a.v->H, a.v->S, D, BN)) != cudaSuccess) return e;
   if (D == 128) {
     if ((e = vprep_mixed<128>(a, prm, w, s)) != cudaSuccess) return e;
     return run_pair<K_BF16, 128, SC_TILE>(mq, mk, mv, prm, s);

@@ -351,7 +351,7 @@ static size_t attention_ws(const fa_qtensor* q, const fa_qtensor* k, const fa_qt
   }
   if (q->mode == FA_MODE_MXFP4_PER_BLOCK || q->mode == FA_MODE_MXFP8_PER_BLOCK) {
     if (k->B < 0 || k->S < 0 || q->D != 128) return 0;
-    return prefill2_workspace_bytes(k->B, k->H, k->S, q->D);
+    return prefill2_workspace_bytes(k->B, k->H, k->S, q->D, prefill_tile_keys(q->mode));
   }
   return 0;
 }
@@ -394,7 +394,7 @@ fa_status fa_attention_quant(const fa_qtensor* q, const fa_qtensor* k, const fa_
   if (k->S > 0) {
     const size_t need = mixed    ? mixed_workspace_bytes(q, k)
                         : decode ? decode_workspace_bytes(q->B, q->H, q->D, splits)
-                                 : prefill2_workspace_bytes(k->B, k->H, k->S, q->D);
+                                 : prefill2_workspace_bytes(k->B, k->H, k->S, q->D, prefill_tile_keys(q->mode));
     if (!workspace || ws_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255u)) return FA_ERR_WORKSPACE;
   }
   cudaStream_t cs = reinterpret_cast<cudaStream_t>(s);

@@ -103,8 +103,10 @@ struct AttnArgs {
   float* lse;
   int* status;
 };
-// Prefill (E4M3, INT8, MXFP4): V' pre-pass + attention; `ws` holds prefill2_workspace_bytes().
-size_t prefill2_workspace_bytes(int B, int Hkv, int Sk, int D);
+// Prefill (E4M3, INT8, MXFP4): V' pre-pass + attention; `ws` holds prefill2_workspace_bytes(), sized for
+// key tiles of `tile_keys` keys (prefill_tile_keys(Q's mode): 112 for the MX modes, 128 otherwise).
+size_t prefill2_workspace_bytes(int B, int Hkv, int Sk, int D, int tile_keys = 128);
+int prefill_tile_keys(int q_mode);
 cudaError_t launch_attention_prefill2(const AttnArgs& a, void* ws, cudaStream_t s);
 // Mixed branches (modes differ, or a branch is not quantized): bf16 Q / K pair kernel;
 // `ws` holds mixed_workspace_bytes(q, k).

@@ -160,14 +160,21 @@ def test_attention_validation_before_launch(N):
                                 None) == 7
     assert L.fa_attention_quant(by(qp), by(kd), by(kd), 0, 0.0, 0x60000, None, 0, 0x70010, need_p,
                                 None) == 7  # workspace not 256-byte aligned
-    # the FA PerHead FP8 / PerToken INT8 / PerBlock MXFP8 modes use the same prefill workspace
-    for m in (5, 6, 7):
+    # the FA PerHead FP8 / PerToken INT8 modes use the same prefill workspace
+    for m in (5, 6):
         assert L.fa_attention_workspace_size(by(_q(N, m, B=2, H=4, S=100, D=128)), by(_q(N, m, B=2, H=2, S=1000, D=128)),
                                              0) == need_p
-    # MXFP4 prefill: the same parts (its K scales are the tile's scale-factor atom); head_dim 128 only
+    # MXFP4 / MXFP8 prefill: the same parts over 112-key tiles (their K scales are the tile's
+    # scale-factor atom); head_dim 128 only
+    ntiles_mx = (1000 + 111) // 112
+    parts_mx = (2 * 2 * 1000 * 128 * 2, 2 * 2 * ntiles_mx * 16, 2 * 2 * ntiles_mx * 128 * 4)
+    need_mx = sum(((x + 255) // 256) * 256 for x in parts_mx)
+    assert need_mx > need_p
+    assert L.fa_attention_workspace_size(by(_q(N, 7, B=2, H=4, S=100, D=128)), by(_q(N, 7, B=2, H=2, S=1000, D=128)),
+                                         0) == need_mx
     qm = _q(N, 3, B=2, H=4, S=100, D=128)
     km = _q(N, 3, B=2, H=2, S=1000, D=128)
-    assert L.fa_attention_workspace_size(by(qm), by(km), 0) == need_p
+    assert L.fa_attention_workspace_size(by(qm), by(km), 0) == need_mx
     assert L.fa_attention_quant(by(qm), by(km), by(km), 0, 0.0, 0x60000, None, 0, None, 0, None) == 7
     qm64, km64 = _q(N, 3, B=2, H=4, S=100, D=64), _q(N, 3, B=2, H=2, S=1000, D=64)
     assert L.fa_attention_workspace_size(by(qm64), by(km64), 0) == 0
