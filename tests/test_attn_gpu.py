@@ -87,6 +87,11 @@ CASES = [
     ("mxfp8", "BNSD", 128, 1, 2, 2, 300, 300, False),
     ("mxfp8", "BSND", 128, 2, 4, 2, 257, 257, True),
     ("mxfp8", "BNSD", 128, 1, 2, 1, 100, 300, True),
+    # MX key tiles hold 112 keys: Sk an exact multiple of 112, Sk below one tile, and a causal
+    # run over more tiles than the K, V' and scale rings have stages (each ring wraps)
+    ("mxfp4", "BNSD", 128, 1, 2, 2, 224, 224, False),
+    ("mxfp8", "BSND", 128, 1, 2, 1, 50, 50, True),
+    ("mxfp4", "BNSD", 128, 1, 4, 2, 700, 700, True),
 ]
 
 
