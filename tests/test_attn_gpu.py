@@ -92,6 +92,11 @@ CASES = [
     ("mxfp4", "BNSD", 128, 1, 2, 2, 224, 224, False),
     ("mxfp8", "BSND", 128, 1, 2, 1, 50, 50, True),
     ("mxfp4", "BNSD", 128, 1, 4, 2, 700, 700, True),
+    # one query row (the second query tile of the pair is empty), one key, and an odd GQA group
+    # (query row blocks paired instead of heads)
+    ("mxfp4", "BNSD", 128, 2, 2, 2, 1, 300, False),
+    ("mxfp8", "BNSD", 128, 1, 2, 2, 130, 1, False),
+    ("mxfp4", "BSND", 128, 1, 3, 1, 260, 260, True),
 ]
 
 
