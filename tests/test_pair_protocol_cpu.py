@@ -20,25 +20,7 @@ key-tile counts per query tile:
 import random
 
 import pytest
-
-
-class Bar:
-    """An mbarrier: `need` arrivals complete a phase; `count` phases have completed."""
-
-    def __init__(self, name, need):
-        self.name, self.need, self.arr, self.count = name, need, 0, 0
-
-    def arrive(self):
-        self.arr += 1
-        assert self.arr <= self.need, f"{self.name}: more arrivals than the phase needs"
-        if self.arr == self.need:
-            self.arr, self.count = 0, self.count + 1
-
-    def done(self, k):
-        # a parity wait for phase k sees the phase bit only: it is right only while the barrier
-        # is at phase k (not yet complete) or k + 1 (complete)
-        assert self.count in (k, k + 1), f"{self.name}: waiter for phase {k} found {self.count} completed"
-        return self.count == k + 1
+from _protocol import Bar, run, wait
 
 
 class Model:
@@ -74,8 +56,7 @@ class Model:
 
     # --------------------------------------------------------------- helpers
     def wait(self, bar, k):
-        while not bar.done(k):
-            yield False
+        return wait(bar, k)
 
     def pending(self, kind, pred):
         return any(op[0] == kind and pred(op) for op in self.pipe)
@@ -249,34 +230,12 @@ class Model:
             assert self.pv_done[x] == nx, "epilogue read O before the last P·V"
 
     # ------------------------------------------------------------------ run
-    def run(self, max_steps=200000):
-        finite = {"k": self.k_loader(), "v": self.v_loader(), "ring": self.ring_loader(), "mma": self.mma()}
+    def run(self):
+        roles = {"k": self.k_loader(), "v": self.v_loader(), "ring": self.ring_loader(), "mma": self.mma()}
         for x in (0, 1):
             for w in range(4):
-                finite[f"s{x}{w}"] = self.softmax(x, w)
-        daemons = [self.engine(), self.tensor_pipe()]
-        live = dict(finite)
-        idle_polls = 0
-        for _ in range(max_steps):
-            if not live:
-                break
-            actors = list(live.items()) + [(None, d) for d in daemons]
-            self.rnd.shuffle(actors)
-            if idle_polls:  # after a poll without progress, poll every role
-                chosen = actors
-            else:
-                chosen = actors[: self.rnd.randint(1, len(actors))]
-            progressed = False
-            for name, gen in chosen:
-                try:
-                    progressed |= bool(next(gen))
-                except StopIteration:
-                    live.pop(name, None)
-                    progressed = True
-            idle_polls = 0 if progressed else idle_polls + 1
-            # two full polls of every role without progress: every role waits for another
-            assert idle_polls < 3, f"deadlock: {sorted(live)} wait; pipe {self.pipe[:4]}"
-        assert not live, f"did not finish: {sorted(live)}"
+                roles[f"s{x}{w}"] = self.softmax(x, w)
+        run(roles, [self.engine(), self.tensor_pipe()], self.rnd)
         assert not self.pipe and not self.inflight
 
 
